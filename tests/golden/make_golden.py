@@ -1,0 +1,44 @@
+"""Writes tests/golden/exact_tiny.json: exact rational outputs of the KATA
+causal forward on tiny integer inputs, computed by oracle/exact.py (Python
+Fractions; no floating point).  The pages print no worked example, so these
+fixtures pin the definition (gist.science summary of "Kernelized Linear
+Attention: Breaking the Capacity Wall with Symmetric Cones", Technical summary
+2.1 and 2.2) by exact arithmetic instead.
+
+Run from the repository root:  python tests/golden/make_golden.py
+"""
+import json
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+sys.path.insert(0, ROOT)
+
+from oracle.exact import forward_exact  # noqa: E402
+
+CASES = [
+    # name, q, k, v (one head; T x d lists of small integers)
+    ("T4_d2", [[1, 0], [1, 1], [0, 2], [-1, 1]], [[1, 1], [2, -1], [0, 1], [1, 3]],
+     [[1, -2], [3, 0], [-1, 1], [2, 2]]),
+    ("T5_d3_zero_query", [[1, 2, 0], [0, 0, 0], [1, -1, 1], [2, 0, -1], [0, 1, 1]],
+     [[1, 0, 1], [0, 1, 0], [1, 1, -1], [-2, 1, 0], [1, -1, 2]],
+     [[1], [-1], [2], [0], [3]]),
+    ("T3_d1", [[2], [-1], [3]], [[1], [-2], [1]], [[4, -1], [0, 2], [1, 1]]),
+]
+
+
+def main():
+    out = []
+    for name, q, k, v in CASES:
+        y = forward_exact(q, k, v)
+        out.append({"name": name, "q": q, "k": k, "v": v,
+                    "y": [[f"{x.numerator}/{x.denominator}" for x in row] for row in y]})
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "exact_tiny.json")
+    with open(path, "w") as f:
+        json.dump({"source": "oracle/exact.py (Fractions) via tests/golden/make_golden.py",
+                   "cases": out}, f, indent=1)
+    print("wrote", path)
+
+
+if __name__ == "__main__":
+    main()
