@@ -1,0 +1,145 @@
+/*
+ * kata.h — C ABI of the KATA causal forward on NVIDIA B200 (sm_100a).
+ *
+ * KATA ("Kernelized Linear Attention: Breaking the Capacity Wall with
+ * Symmetric Cones") with the rank-one PSD feature phi(x) = vec(x x^T):
+ * every attention weight is <q q^T, k k^T> = (q.k)^2 >= 0, and dividing by the
+ * running sum of weights makes each output a convex combination of the values
+ * seen so far.  Per head, for t = 0 .. T-1:
+ *
+ *     y_t = sum_{s<=t} (q_t.k_s)^2 v_s / sum_{s<=t} (q_t.k_s)^2     (y_t = 0 if 0)
+ *
+ * Sources (page title and section):
+ *   - gist.science summary of the paper, Technical summary 2.2 "PSD cone
+ *     (rank one)": psi(u) = u u^T squares the raw inner product.
+ *   - same, 2.1 "output gating": the normalised denominator is a convex,
+ *     parameter-free gate between the previous readout and the current value
+ *     (so the current token is included, s <= t).
+ *   - same, 2.3 "hardware-aligned implementation": chunked parallelism,
+ *     tensor cores inside a chunk, an associative scan (parallel prefix sum)
+ *     of chunk states across chunks, depth O(log N_C).
+ *   - arXiv abstract of the paper: "exact O(T) chunked-state form",
+ *     "constant-time recurrent inference".
+ *
+ * Readings where the pages are silent: no scale constant; no epsilon in the
+ * denominator; a zero denominator gives y = 0; the state and normaliser are
+ * kept in fp32; the output has the input's dtype.
+ *
+ * General contract of every entry point
+ *   - All tensor pointers are DEVICE pointers, owned by the caller, 16-byte
+ *     aligned, dense row-major with the layout stated per argument.  The
+ *     library allocates nothing and keeps no state between calls.
+ *   - Work is enqueued on `stream` (NULL = legacy default stream) and the call
+ *     returns without synchronising.  Errors found on the host (bad sizes,
+ *     null or misaligned pointers, short workspace) return before anything is
+ *     launched; a launch failure returns KATA_ERR_CUDA.  Errors raised while
+ *     kernels run are recorded in a device status word that
+ *     kata_get_device_status() reads.
+ *   - Outputs must not alias inputs.
+ *   - Supported head sizes: dk = dv in {16, 32, 64}; others return
+ *     KATA_ERR_UNSUPPORTED.  T >= 1 (any value; the ragged tail is exact).
+ *   - Calls on different streams may run concurrently if their buffers are
+ *     disjoint.
+ */
+#ifndef KATA_H_
+#define KATA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *kata_stream_t;
+
+typedef enum {
+    KATA_OK = 0,
+    KATA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, non-positive size, bad chunk size */
+    KATA_ERR_UNSUPPORTED = 2, /* a head size or dtype the kernels do not cover */
+    KATA_ERR_WORKSPACE = 3,   /* workspace null or smaller than the size query returned */
+    KATA_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
+    KATA_ERR_TIMEOUT = 5      /* a bounded on-device wait gave up (device status only) */
+} kata_status;
+
+typedef enum {
+    KATA_F32 = 0, /* float32 q, k, v and out */
+    KATA_BF16 = 1 /* bfloat16 q, k, v and out; fp32 accumulation */
+} kata_dtype;
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int kata_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kata_status_string(kata_status status);
+
+/*
+ * Bytes of device workspace kata_chunked_forward needs for this problem.
+ * Returns 0 for arguments the forward would reject.  The value depends only
+ * on the arguments and may be 0 for short sequences (no state needs storing).
+ */
+size_t kata_chunked_forward_workspace_bytes(int B, int H, int T, int dk, int dv, int C,
+                                            kata_dtype dtype);
+
+/*
+ * Causal KATA forward in the exact chunked-state form
+ * (gist.science summary 2.3 and the arXiv abstract, "exact O(T)
+ * chunked-state form"; the associative scan of chunk states of summary 2.3).
+ *
+ *   q, k   [B, H, T, dk]  dtype      queries, keys
+ *   v      [B, H, T, dv]  dtype      values
+ *   out    [B, H, T, dv]  dtype      y_t as defined above
+ *   C      chunk size, one of 16, 32, 64, 128, 256.  The result does not
+ *          depend on C (the form is exact); states are stored only at
+ *          segment boundaries that are multiples of C, and everything inside
+ *          a segment is computed in its causal quadratic form.
+ *   state_out  nullable, [B, H, dk*dk, dv] fp32: S_T = sum_{s<T} phi(k_s) v_s^T,
+ *          row index i*dk + j (symmetric in i, j), ready for kata_decode_step.
+ *   z_out  nullable, [B, H, dk, dk] fp32: Z_T = sum_{s<T} k_s k_s^T.
+ *          state_out and z_out must be both NULL or both non-NULL.
+ *   workspace, workspace_bytes: device scratch of at least
+ *          kata_chunked_forward_workspace_bytes(...) bytes (may be NULL when
+ *          that is 0).  Its contents on entry do not matter.
+ *
+ * dtype KATA_BF16 runs the tensor-core (tcgen05) path where the head size
+ * has one, KATA_F32 runs fp32 CUDA-core arithmetic end to end.
+ */
+kata_status kata_chunked_forward(const void *q, const void *k, const void *v, void *out, int B,
+                                 int H, int T, int dk, int dv, int C, kata_dtype dtype,
+                                 float *state_out, float *z_out, void *workspace,
+                                 size_t workspace_bytes, kata_stream_t stream);
+
+/*
+ * One recurrent decode step for every head, in place
+ * (arXiv abstract, "constant-time recurrent inference"; gist.science summary
+ * 1: a fixed-size state replaces the key-value cache):
+ *
+ *     S <- S + phi(k) v^T,   Z <- Z + k k^T,   y = phi(q)^T S / (q^T Z q)
+ *
+ * The readout includes the current token, so a forward over T tokens
+ * followed by a decode step on token T gives row T of a forward over T + 1
+ * tokens.
+ *
+ *   q, k   [B, H, dk]  dtype;  v, out  [B, H, dv]  dtype
+ *   state  [B, H, dk*dk, dv] fp32, read and updated in place
+ *   z      [B, H, dk, dk] fp32, read and updated in place
+ *
+ * The state must be symmetric in (i, j), as every state the forward writes
+ * is; the update keeps it symmetric.
+ */
+kata_status kata_decode_step(const void *q, const void *k, const void *v, void *out,
+                             float *state, float *z, int B, int H, int dk, int dv,
+                             kata_dtype dtype, kata_stream_t stream);
+
+/*
+ * Synchronises `stream`, returns and clears the device status word that
+ * kernels set when an on-device check fails (KATA_OK if none did), or
+ * KATA_ERR_CUDA if the synchronisation itself reports an error.
+ */
+kata_status kata_get_device_status(kata_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KATA_H_ */

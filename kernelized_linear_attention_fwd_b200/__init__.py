@@ -1,0 +1,16 @@
+"""KATA kernelized linear attention (rank-one PSD features), causal forward and
+recurrent decode on NVIDIA B200 (sm_100a).
+
+The compute path is libkata.so (hand-written CUDA kernels behind the C ABI in
+include/kata.h); ``binding`` marshals torch CUDA tensors into it.
+"""
+from .binding import (  # noqa: F401
+    KataError,
+    kata_chunked_forward,
+    kata_chunked_forward_workspace_bytes,
+    kata_decode_step,
+    kata_get_device_status,
+    kata_status_string,
+    kata_version,
+    load_library,
+)

@@ -1,0 +1,181 @@
+"""Python binding of libkata (the C ABI in include/kata.h).
+
+Argument marshalling only: every step of the forward and the decode runs in
+the library's CUDA kernels.  Tensors are torch CUDA tensors (torch supplies
+device memory and streams); the functions carry the C names and raise
+``KataError`` on any status other than KATA_OK.  There is no fallback: if
+libkata.so is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkata.so")
+
+KATA_OK = 0
+KATA_ERR_INVALID_ARG = 1
+KATA_ERR_UNSUPPORTED = 2
+KATA_ERR_WORKSPACE = 3
+KATA_ERR_CUDA = 4
+KATA_ERR_TIMEOUT = 5
+
+KATA_F32 = 0
+KATA_BF16 = 1
+
+# Every symbol include/kata.h declares.
+EXPORTS = (
+    "kata_version",
+    "kata_status_string",
+    "kata_chunked_forward_workspace_bytes",
+    "kata_chunked_forward",
+    "kata_decode_step",
+    "kata_get_device_status",
+)
+
+
+class KataError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {kata_status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads libkata.so once and declares the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"libkata.so not found at {path}; build it with "
+            "`python kernelized_linear_attention_fwd_b200/csrc/build.py`")
+    lib = ctypes.CDLL(path)
+    vp, sz, i32, fp = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p
+    lib.kata_version.restype = i32
+    lib.kata_version.argtypes = []
+    lib.kata_status_string.restype = ctypes.c_char_p
+    lib.kata_status_string.argtypes = [i32]
+    lib.kata_chunked_forward_workspace_bytes.restype = sz
+    lib.kata_chunked_forward_workspace_bytes.argtypes = [i32] * 7
+    lib.kata_chunked_forward.restype = i32
+    lib.kata_chunked_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                         fp, fp, vp, sz, vp]
+    lib.kata_decode_step.restype = i32
+    lib.kata_decode_step.argtypes = [vp, vp, vp, vp, fp, fp, i32, i32, i32, i32, i32, vp]
+    lib.kata_get_device_status.restype = i32
+    lib.kata_get_device_status.argtypes = [vp]
+    _lib = lib
+    return lib
+
+
+def kata_version() -> int:
+    return load_library().kata_version()
+
+
+def kata_status_string(status: int) -> str:
+    return load_library().kata_status_string(int(status)).decode()
+
+
+def _dtype_code(t):
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return KATA_BF16
+    if t.dtype == torch.float32:
+        return KATA_F32
+    raise KataError(KATA_ERR_UNSUPPORTED, f"dtype {t.dtype}")
+
+
+def _stream_handle(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t, name, shape, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} must be contiguous")
+    if tuple(t.shape) != tuple(shape):
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} has shape {tuple(t.shape)}, want {shape}")
+    if dtype is not None and t.dtype != dtype:
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} has dtype {t.dtype}, want {dtype}")
+
+
+def kata_chunked_forward_workspace_bytes(B, H, T, dk, dv, C, dtype_code) -> int:
+    return int(load_library().kata_chunked_forward_workspace_bytes(B, H, T, dk, dv, C,
+                                                                   dtype_code))
+
+
+def kata_chunked_forward(q, k, v, C=64, out=None, state_out=None, z_out=None, workspace=None,
+                         stream=None):
+    """out[B,H,T,dv] = causal KATA forward of q, k [B,H,T,dk] and v [B,H,T,dv].
+
+    Optionally writes the final state S [B,H,dk*dk,dv] and Z [B,H,dk,dk] (fp32).
+    `workspace` is a uint8 CUDA tensor of at least
+    kata_chunked_forward_workspace_bytes(...) bytes; allocated here if None.
+    """
+    import torch
+
+    lib = load_library()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", (B, H, T, dk))
+    _check(k, "k", (B, H, T, dk), q.dtype)
+    _check(v, "v", (B, H, T, dv), q.dtype)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", (B, H, T, dv), q.dtype)
+    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32)
+    _check(z_out, "z_out", (B, H, dk, dk), torch.float32)
+    need = lib.kata_chunked_forward_workspace_bytes(B, H, T, dk, dv, C, code)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.kata_chunked_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv, int(C),
+                                  code, _ptr(state_out), _ptr(z_out), _ptr(workspace), ws_bytes,
+                                  _stream_handle(stream))
+    if st != KATA_OK:
+        raise KataError(st, "kata_chunked_forward")
+    return out
+
+
+def kata_decode_step(q, k, v, state, z, out=None, stream=None):
+    """One recurrent step, in place on (state, z); q, k [B,H,dk], v [B,H,dv]."""
+    import torch
+
+    lib = load_library()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", (B, H, dk))
+    _check(k, "k", (B, H, dk), q.dtype)
+    _check(v, "v", (B, H, dv), q.dtype)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", (B, H, dv), q.dtype)
+    _check(state, "state", (B, H, dk * dk, dv), torch.float32)
+    _check(z, "z", (B, H, dk, dk), torch.float32)
+    st = lib.kata_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state), _ptr(z), B, H,
+                              dk, dv, code, _stream_handle(stream))
+    if st != KATA_OK:
+        raise KataError(st, "kata_decode_step")
+    return out
+
+
+def kata_get_device_status(stream=None) -> int:
+    return int(load_library().kata_get_device_status(_stream_handle(stream)))

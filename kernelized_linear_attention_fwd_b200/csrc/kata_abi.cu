@@ -1,0 +1,170 @@
+// C ABI of libkata: argument checks, the forward plan, and kernel dispatch.
+// Declarations and the contract of every entry point: include/kata.h.
+#include <stdint.h>
+
+#include "kata_internal.cuh"
+
+namespace kata {
+
+namespace {
+
+__device__ int g_device_status = 0;
+
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_chunk(int C) {
+    return C == 16 || C == 32 || C == 64 || C == 128 || C == 256;
+}
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+// Segment length: states are stored every L tokens.  Inside a segment the
+// exact causal quadratic form is used, so L trades state traffic (~1/L)
+// against quadratic work (~L); L is a multiple of C and of 128.
+int segment_length(int dk, int C) {
+    const int target = dk >= 64 ? 1024 : (dk >= 32 ? 512 : 256);
+    return target > C ? target : C;
+}
+
+}  // namespace
+
+int *device_status_ptr() {
+    static int *ptrs[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int *>(p);
+    }
+    return ptrs[dev];
+}
+
+kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype, Plan &p) {
+    if (B < 1 || H < 1 || T < 1 || dk < 1 || dv < 1) return KATA_ERR_INVALID_ARG;
+    if (!valid_chunk(C)) return KATA_ERR_INVALID_ARG;
+    if (dtype != KATA_F32 && dtype != KATA_BF16) return KATA_ERR_UNSUPPORTED;
+    if (dk != dv || (dk != 16 && dk != 32 && dk != 64)) return KATA_ERR_UNSUPPORTED;
+    const long long BH = (long long)B * H;
+    if (BH * (long long)T > (1LL << 40)) return KATA_ERR_UNSUPPORTED;
+    p.B = B;
+    p.H = H;
+    p.T = T;
+    p.dk = dk;
+    p.dv = dv;
+    p.C = C;
+    p.dtype = dtype;
+    p.BH = BH;
+    p.R = packed_rows(dk);
+    p.L = segment_length(dk, C);
+    p.n_seg = (T + p.L - 1) / p.L;
+    p.path = Path::kSimt;
+    const size_t E = (size_t)p.R * (dv + 1);
+    const size_t seg_bytes = (size_t)BH * p.n_seg * E * sizeof(float);
+    const size_t total_bytes = p.n_seg > 1 ? (size_t)BH * E * sizeof(float) : 0;
+    p.ws_seg_state = 0;
+    p.ws_total = align_up(seg_bytes);
+    p.ws_extra = p.ws_total + align_up(total_bytes);
+    p.ws_bytes = p.ws_extra;
+    return KATA_OK;
+}
+
+}  // namespace kata
+
+using kata::Plan;
+using kata::aligned16;
+using kata::overlaps;
+
+extern "C" {
+
+int kata_version(void) { return 100; }
+
+const char *kata_status_string(kata_status s) {
+    switch (s) {
+        case KATA_OK: return "KATA_OK";
+        case KATA_ERR_INVALID_ARG: return "KATA_ERR_INVALID_ARG";
+        case KATA_ERR_UNSUPPORTED: return "KATA_ERR_UNSUPPORTED";
+        case KATA_ERR_WORKSPACE: return "KATA_ERR_WORKSPACE";
+        case KATA_ERR_CUDA: return "KATA_ERR_CUDA";
+        case KATA_ERR_TIMEOUT: return "KATA_ERR_TIMEOUT";
+    }
+    return "KATA_ERR_UNKNOWN";
+}
+
+size_t kata_chunked_forward_workspace_bytes(int B, int H, int T, int dk, int dv, int C,
+                                            kata_dtype dtype) {
+    Plan p;
+    if (kata::make_plan(B, H, T, dk, dv, C, dtype, p) != KATA_OK) return 0;
+    return p.ws_bytes;
+}
+
+kata_status kata_chunked_forward(const void *q, const void *k, const void *v, void *out, int B,
+                                 int H, int T, int dk, int dv, int C, kata_dtype dtype,
+                                 float *state_out, float *z_out, void *workspace,
+                                 size_t workspace_bytes, kata_stream_t stream) {
+    Plan p;
+    const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p);
+    if (ps != KATA_OK) return ps;
+    if (!q || !k || !v || !out) return KATA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return KATA_ERR_INVALID_ARG;
+    if ((state_out == nullptr) != (z_out == nullptr)) return KATA_ERR_INVALID_ARG;
+    if (state_out && (!aligned16(state_out) || !aligned16(z_out))) return KATA_ERR_INVALID_ARG;
+    const size_t es = dtype == KATA_BF16 ? 2 : 4;
+    const size_t nq = (size_t)p.BH * T * dk * es, nv = (size_t)p.BH * T * dv * es;
+    if (overlaps(out, nv, q, nq) || overlaps(out, nv, k, nq) || overlaps(out, nv, v, nv))
+        return KATA_ERR_INVALID_ARG;
+    if (p.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < p.ws_bytes) return KATA_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_WORKSPACE;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e =
+        kata::launch_simt_forward(p, q, k, v, out, state_out, z_out, workspace, st);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+}
+
+kata_status kata_decode_step(const void *q, const void *k, const void *v, void *out,
+                             float *state, float *z, int B, int H, int dk, int dv,
+                             kata_dtype dtype, kata_stream_t stream) {
+    if (B < 1 || H < 1 || dk < 1 || dv < 1) return KATA_ERR_INVALID_ARG;
+    if (dtype != KATA_F32 && dtype != KATA_BF16) return KATA_ERR_UNSUPPORTED;
+    if (dk != dv || (dk != 16 && dk != 32 && dk != 64)) return KATA_ERR_UNSUPPORTED;
+    if ((long long)B * H > 0x7fffffffLL) return KATA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !out || !state || !z) return KATA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state) ||
+        !aligned16(z))
+        return KATA_ERR_INVALID_ARG;
+    const size_t es = dtype == KATA_BF16 ? 2 : 4;
+    const size_t BH = (size_t)B * H;
+    const size_t ns = BH * dk * dk * dv * 4, nz = BH * dk * dk * 4, no = BH * dv * es;
+    if (overlaps(state, ns, z, nz) || overlaps(out, no, state, ns) || overlaps(out, no, z, nz))
+        return KATA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = kata::launch_decode(B, H, dk, dv, dtype, q, k, v, out, state, z, st);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+}
+
+kata_status kata_get_device_status(kata_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return KATA_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpyFromSymbol(&word, kata::g_device_status, sizeof(int)) != cudaSuccess)
+        return KATA_ERR_CUDA;
+    if (word != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(kata::g_device_status, &zero, sizeof(int)) != cudaSuccess)
+            return KATA_ERR_CUDA;
+    }
+    return static_cast<kata_status>(word);
+}
+
+}  // extern "C"

@@ -1,0 +1,92 @@
+// Internal declarations shared by the CUDA translation units of libkata.
+// Not part of the public ABI (that is include/kata.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kata.h"
+
+namespace kata {
+
+// ---------------------------------------------------------------------------
+// Packed symmetric feature rows.
+//
+// phi(x) = vec(x x^T) has dk^2 entries but only dk(dk+1)/2 distinct ones:
+// (q.k)^2 = sum_i q_i^2 k_i^2 + 2 sum_{i<j} q_i q_j k_i k_j.  The state is kept
+// on the half triangle i <= j (row r enumerates (i, j) with i outer), storing
+// the plain sums sum_s k_si k_sj v_s; the weight c_ij (1 on the diagonal, 2
+// off it) is applied on the query side at readout.
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr int packed_rows(int d) { return d * (d + 1) / 2; }
+
+__host__ __device__ inline int packed_row_start(int d, int i) { return i * d - (i * (i - 1)) / 2; }
+
+__host__ __device__ inline void packed_row_ij(int d, int r, int &i, int &j) {
+    int a = 0;
+    while (r >= d - a) {
+        r -= d - a;
+        ++a;
+    }
+    i = a;
+    j = a + r;
+}
+
+// ---------------------------------------------------------------------------
+// Forward plan: segment length, number of segments, workspace layout.
+// ---------------------------------------------------------------------------
+enum class Path : int { kSimt = 0, kTensorCore = 1 };
+
+struct Plan {
+    int B, H, T, dk, dv, C;
+    kata_dtype dtype;
+    long long BH;
+    int L;      // segment length (tokens), a multiple of C and of 128
+    int n_seg;  // ceil(T / L)
+    int R;      // packed feature rows
+    Path path;
+    // workspace (bytes from the base, all 256-byte aligned)
+    size_t ws_seg_state;  // fp32 per-segment states, exclusive prefix after the scan
+    size_t ws_total;      // fp32 total state (packed), when needed
+    size_t ws_extra;      // path-specific
+    size_t ws_bytes;
+};
+
+// Fills `p`; returns KATA_OK or the error the forward must return.
+kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype, Plan &p);
+
+// Device address of the status word that kernels set when an on-device check
+// fails (one per device; resolved on first use with that device current).
+int *device_status_ptr();
+
+// Kernel timing (include/kata_profile.h): no-ops unless profiling is enabled.
+int prof_begin(const char *name, cudaStream_t st);
+void prof_end(int ev, cudaStream_t st);
+
+struct ProfScope {
+    int ev;
+    cudaStream_t st;
+    ProfScope(const char *name, cudaStream_t s) : ev(prof_begin(name, s)), st(s) {}
+    ~ProfScope() { prof_end(ev, st); }
+};
+
+// Element loads as fp32.
+__device__ __forceinline__ float load_f32(const float *p, long long i) { return p[i]; }
+__device__ __forceinline__ float load_f32(const __nv_bfloat16 *p, long long i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void store_out(float *p, long long i, float x) { p[i] = x; }
+__device__ __forceinline__ void store_out(__nv_bfloat16 *p, long long i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+// Launchers (return cudaSuccess or the launch error).
+cudaError_t launch_simt_forward(const Plan &p, const void *q, const void *k, const void *v,
+                                void *out, float *state_out, float *z_out, void *ws,
+                                cudaStream_t st);
+cudaError_t launch_decode(int B, int H, int dk, int dv, kata_dtype dtype, const void *q,
+                          const void *k, const void *v, void *out, float *state, float *z,
+                          cudaStream_t st);
+
+}  // namespace kata

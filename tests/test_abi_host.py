@@ -1,0 +1,136 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+Every call here carries arguments the library must reject before it launches
+anything (sizes, null or misaligned pointers, short workspace), so nothing
+reaches a device.  Also checks that libkata.so exports every function the
+public header declares, and the workspace-size query.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from kernelized_linear_attention_fwd_b200 import binding
+from kernelized_linear_attention_fwd_b200.csrc import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kata.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return binding.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kata_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_expected_entry_points():
+    names = declared_functions()
+    for n in ("kata_chunked_forward", "kata_decode_step", "kata_chunked_forward_workspace_bytes",
+              "kata_get_device_status", "kata_status_string", "kata_version"):
+        assert n in names
+    assert set(names) == set(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert getattr(lib, name) is not None
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "KATA_OK"), (1, "KATA_ERR_INVALID_ARG"), (2, "KATA_ERR_UNSUPPORTED"),
+                       (3, "KATA_ERR_WORKSPACE"), (4, "KATA_ERR_CUDA"), (5, "KATA_ERR_TIMEOUT")]:
+        assert binding.kata_status_string(code) == name
+    assert binding.kata_status_string(99) == "KATA_ERR_UNKNOWN"
+    assert binding.kata_version() >= 100
+
+
+def test_workspace_query(lib):
+    W = lib.kata_chunked_forward_workspace_bytes
+    # rejected arguments -> 0
+    assert W(0, 1, 16, 64, 64, 64, 1) == 0
+    assert W(1, 1, 16, 48, 48, 64, 1) == 0   # unsupported head size
+    assert W(1, 1, 16, 64, 32, 64, 1) == 0   # dk != dv
+    assert W(1, 1, 16, 64, 64, 48, 1) == 0   # bad chunk
+    assert W(1, 1, 16, 64, 64, 64, 7) == 0   # bad dtype
+    # positive, monotone in T and in heads
+    a = W(1, 8, 131072, 64, 64, 64, 1)
+    b = W(1, 8, 65536, 64, 64, 64, 1)
+    c = W(2, 8, 131072, 64, 64, 64, 1)
+    assert a > b > 0 and c >= 2 * a - 512
+    assert W(1, 1, 256, 16, 16, 64, 0) > 0
+
+
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced: every call below fails first
+
+
+def _fwd(lib, q=FAKE, k=FAKE + 0x10000000, v=FAKE + 0x20000000, out=FAKE + 0x30000000, B=1, H=1,
+         T=64, dk=16, dv=16, C=64, dt=0, so=None, zo=None, ws=None, wsb=0):
+    vp = ctypes.c_void_p
+    return lib.kata_chunked_forward(vp(q) if q else None, vp(k) if k else None,
+                                    vp(v) if v else None, vp(out) if out else None, B, H, T, dk,
+                                    dv, C, dt, vp(so) if so else None, vp(zo) if zo else None,
+                                    vp(ws) if ws else None, wsb, None)
+
+
+def test_forward_rejects_bad_arguments(lib):
+    E = binding
+    assert _fwd(lib, q=0) == E.KATA_ERR_INVALID_ARG
+    assert _fwd(lib, out=0) == E.KATA_ERR_INVALID_ARG
+    assert _fwd(lib, q=FAKE + 2) == E.KATA_ERR_INVALID_ARG            # misaligned
+    assert _fwd(lib, B=0) == E.KATA_ERR_INVALID_ARG
+    assert _fwd(lib, T=0) == E.KATA_ERR_INVALID_ARG
+    assert _fwd(lib, T=-5) == E.KATA_ERR_INVALID_ARG
+    assert _fwd(lib, C=48) == E.KATA_ERR_INVALID_ARG
+    assert _fwd(lib, C=512) == E.KATA_ERR_INVALID_ARG
+    assert _fwd(lib, dk=128, dv=128) == E.KATA_ERR_UNSUPPORTED
+    assert _fwd(lib, dk=16, dv=32) == E.KATA_ERR_UNSUPPORTED
+    assert _fwd(lib, dt=3) == E.KATA_ERR_UNSUPPORTED
+    # state_out without z_out
+    assert _fwd(lib, so=FAKE + 0x40000000) == E.KATA_ERR_INVALID_ARG
+    # out aliasing an input
+    assert _fwd(lib, out=FAKE + 0x10000000) == E.KATA_ERR_INVALID_ARG
+    # missing / short / misaligned workspace for a problem that needs one
+    need = lib.kata_chunked_forward_workspace_bytes(1, 1, 4096, 16, 16, 64, 0)
+    assert need > 0
+    assert _fwd(lib, T=4096, ws=None, wsb=0) == E.KATA_ERR_WORKSPACE
+    assert _fwd(lib, T=4096, ws=FAKE + 0x50000000, wsb=need - 1) == E.KATA_ERR_WORKSPACE
+    assert _fwd(lib, T=4096, ws=FAKE + 0x50000010, wsb=need) == E.KATA_ERR_WORKSPACE
+
+
+def test_decode_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    E = binding
+
+    def dec(q=FAKE, k=FAKE + 0x100, v=FAKE + 0x200, out=FAKE + 0x300, S=FAKE + 0x10000,
+            Z=FAKE + 0x10000000, B=1, H=1, dk=16, dv=16, dt=0):
+        return lib.kata_decode_step(vp(q) if q else None, vp(k) if k else None,
+                                    vp(v) if v else None, vp(out) if out else None,
+                                    vp(S) if S else None, vp(Z) if Z else None, B, H, dk, dv, dt,
+                                    None)
+
+    assert dec(q=0) == E.KATA_ERR_INVALID_ARG
+    assert dec(S=0) == E.KATA_ERR_INVALID_ARG
+    assert dec(B=0) == E.KATA_ERR_INVALID_ARG
+    assert dec(dk=48, dv=48) == E.KATA_ERR_UNSUPPORTED
+    assert dec(dt=9) == E.KATA_ERR_UNSUPPORTED
+    assert dec(S=FAKE + 0x10008) == E.KATA_ERR_INVALID_ARG                 # misaligned
+    assert dec(Z=FAKE + 0x10000 + 4096) == E.KATA_ERR_INVALID_ARG          # Z inside S
+    assert dec(out=FAKE + 0x10000) == E.KATA_ERR_INVALID_ARG               # out inside S
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    saved = binding._lib
+    try:
+        binding._lib = None
+        with pytest.raises(RuntimeError):
+            binding.load_library(str(tmp_path / "missing.so"))
+    finally:
+        binding._lib = saved

@@ -1,0 +1,234 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Inputs are the seeded generator's bits (kernelized_linear_attention_fwd_b200
+/inputs.py); the oracle widens exactly those bits to fp64.  The metric and
+tolerances are in tests/gpu_util.py (row-normwise relative error, 1e-4 for
+fp32 inputs, 2e-2 for bf16 inputs).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+from kernelized_linear_attention_fwd_b200 import inputs
+from tests.gpu_util import TOL, from_device, row_err, sample_rows, to_device
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # collected on CPU machines, run only with a GPU
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+import kernelized_linear_attention_fwd_b200 as K  # noqa: E402
+from kernelized_linear_attention_fwd_b200.csrc import build as kbuild  # noqa: E402
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    kbuild.build()
+    K.load_library()
+    yield
+    assert K.kata_get_device_status() == 0
+
+
+def seg_len(d, C):
+    target = 1024 if d >= 64 else (512 if d >= 32 else 256)
+    return max(target, C)
+
+
+def run_forward(q, k, v, dtype, C, want_state=False):
+    qd, kd, vd = to_device(q, dtype), to_device(k, dtype), to_device(v, dtype)
+    B, H, T, dk = q.shape
+    so = zo = None
+    if want_state:
+        so = torch.empty((B, H, dk * dk, dk), dtype=torch.float32, device="cuda")
+        zo = torch.empty((B, H, dk, dk), dtype=torch.float32, device="cuda")
+    out = K.kata_chunked_forward(qd, kd, vd, C=C, state_out=so, z_out=zo)
+    torch.cuda.synchronize()
+    return out, so, zo
+
+
+def full_check(oracle_mod, q, k, v, dtype, C, tol=None):
+    out, _, _ = run_forward(q, k, v, dtype, C)
+    yref = oracle_mod.forward(inputs.widen(q, dtype), inputs.widen(k, dtype),
+                              inputs.widen(v, dtype))
+    err = row_err(from_device(out), yref)
+    assert err <= (tol or TOL[dtype]), f"row-normwise error {err:.3e} (C={C})"
+    return err
+
+
+# ---------------------------------------------------------------------------
+# The named workloads
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("C", [16, 32, 64, 128, 256])
+def test_tiny_f32_full(oracle_mod, C):
+    w = inputs.WORKLOADS["tiny_B1H1_T256_d16_f32"]
+    q, k, v = inputs.make_workload(w)
+    full_check(oracle_mod, q, k, v, "f32", C)
+
+
+def test_small_bf16_full(oracle_mod):
+    w = inputs.WORKLOADS["small_B2H4_T4096_d32_bf16"]
+    q, k, v = inputs.make_workload(w)
+    full_check(oracle_mod, q, k, v, "bf16", w.C)
+
+
+def _sampled_check(oracle_mod, q, k, v, dtype, Cs, n_uniform=512):
+    B, H, T, d = q.shape
+    q64, k64, v64 = (inputs.widen(x, dtype).reshape(B * H, T, -1) for x in (q, k, v))
+    rows = sample_rows(T, min(Cs), seg_len(d, max(Cs)), n_uniform=n_uniform)
+    bh = np.repeat(np.arange(B * H), len(rows))
+    tt = np.tile(rows, B * H)
+    yref = oracle_mod.forward_rows(q64, k64, v64, bh, tt)
+    errs = {}
+    for C in Cs:
+        out, _, _ = run_forward(q, k, v, dtype, C)
+        y = from_device(out).reshape(B * H, T, -1)[bh, tt]
+        errs[C] = row_err(y, yref)
+        assert errs[C] <= TOL[dtype], f"C={C}: row-normwise error {errs[C]:.3e}"
+    return errs
+
+
+def test_lm340m_layer_sampled(oracle_mod):
+    w = inputs.WORKLOADS["lm340m_B4H16_T16384_d64_bf16"]
+    q, k, v = inputs.make_workload(w)
+    _sampled_check(oracle_mod, q, k, v, "bf16", [w.C], n_uniform=128)
+
+
+@pytest.mark.parametrize("T", [8192, 32768, 131072])
+def test_long_context_sampled(oracle_mod, T):
+    w = inputs.WORKLOADS["long_B1H8_T131072_d64_bf16"]
+    q, k, v = inputs.make_workload(w, T=T)
+    Cs = list(w.chunk_sweep) if T == w.T else [w.C]
+    _sampled_check(oracle_mod, q, k, v, "bf16", Cs, n_uniform=512 if T == w.T else 256)
+
+
+# ---------------------------------------------------------------------------
+# Edge cases
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [16, 32, 64])
+@pytest.mark.parametrize("T", [1, 2, 63, 257, 1000, 2049])
+def test_ragged_lengths_all_head_sizes(oracle_mod, dtype, d, T):
+    q, k, v = inputs.make_qkv(1, 2, T, d, d, dtype, seed=T + d)
+    full_check(oracle_mod, q, k, v, dtype, 64)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_multi_segment_f32_and_bf16(oracle_mod, dtype):
+    # several segments, ragged tail, every chunk size
+    q, k, v = inputs.make_qkv(1, 2, 3 * 1024 + 77, 64, 64, dtype, seed=11)
+    for C in (16, 64, 256):
+        full_check(oracle_mod, q, k, v, dtype, C)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_zero_denominator_rows(oracle_mod, dtype):
+    q, k, v = inputs.make_qkv(1, 2, 1500, 32, 32, dtype, seed=3)
+    zero = inputs.f32_to_bf16_bits(np.zeros(1, np.float32))[0] if dtype == "bf16" else 0.0
+    for t in (0, 5, 511, 512, 1499):
+        q[0, 0, t] = zero
+    q[0, 1, 700] = zero
+    out, _, _ = run_forward(q, k, v, dtype, 64)
+    y = from_device(out)
+    for (h, t) in [(0, 0), (0, 5), (0, 511), (0, 512), (0, 1499), (1, 700)]:
+        assert np.all(y[0, h, t] == 0.0), (h, t)
+    yref = oracle_mod.forward(inputs.widen(q, dtype), inputs.widen(k, dtype),
+                              inputs.widen(v, dtype))
+    assert row_err(y, yref) <= TOL[dtype]
+
+
+def test_convex_combination_invariant():
+    """Every output coordinate lies within [min, max] of the prefix values
+    (gist.science summary 2.1, convex output gate), up to bf16 rounding."""
+    q, k, v = inputs.make_qkv(2, 2, 4096, 64, 64, "bf16", seed=21)
+    out, _, _ = run_forward(q, k, v, "bf16", 64)
+    y = from_device(out)
+    vv = inputs.widen(v, "bf16")
+    lo = np.minimum.accumulate(vv, axis=2)
+    hi = np.maximum.accumulate(vv, axis=2)
+    slack = 1e-2 * np.maximum(np.abs(lo), np.abs(hi)) + 1e-3
+    assert np.all(y >= lo - slack) and np.all(y <= hi + slack)
+
+
+# ---------------------------------------------------------------------------
+# State export and decode
+# ---------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d,T", [(16, 300), (32, 1500), (64, 2500)])
+def test_state_export(oracle_mod, dtype, d, T):
+    q, k, v = inputs.make_qkv(1, 3, T, d, d, dtype, seed=d)
+    out, so, zo = run_forward(q, k, v, dtype, 64, want_state=True)
+    S, Z = oracle_mod.state(inputs.widen(k, dtype), inputs.widen(v, dtype))
+    Sg, Zg = from_device(so), from_device(zo)
+    tol = 1e-5 if dtype == "f32" else 2e-3
+    assert np.abs(Sg - S).max() <= tol * np.abs(S).max()
+    assert np.abs(Zg - Z).max() <= tol * np.abs(Z).max()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [16, 32, 64])
+def test_forward_then_decode_steps(oracle_mod, dtype, d):
+    """forward(T) + n decode steps == rows T..T+n-1 of forward(T + n)."""
+    T, n = 1100, 6
+    q, k, v = inputs.make_qkv(2, 2, T + n, d, d, dtype, seed=100 + d)
+    _, so, zo = run_forward(q[:, :, :T], k[:, :, :T], v[:, :, :T], dtype, 64, want_state=True)
+    ys = []
+    for s in range(n):
+        qs = to_device(np.ascontiguousarray(q[:, :, T + s]), dtype)
+        ks = to_device(np.ascontiguousarray(k[:, :, T + s]), dtype)
+        vs = to_device(np.ascontiguousarray(v[:, :, T + s]), dtype)
+        ys.append(from_device(K.kata_decode_step(qs, ks, vs, so, zo)))
+    torch.cuda.synchronize()
+    yd = np.stack(ys, axis=2)
+    q64, k64, v64 = (inputs.widen(x, dtype) for x in (q, k, v))
+    yref = oracle_mod.forward(q64, k64, v64)[:, :, T:]
+    assert row_err(yd, yref) <= TOL[dtype]
+
+
+def test_recall_decode_workload(oracle_mod):
+    """Prefill of 64 x 16 heads over 32768 tokens, then 1024 decode steps whose
+    queries repeat the keys of 4096 marked pairs (recall-shaped workload).
+    Checked against the oracle: 16 seeded heads at every decode step, plus 64
+    seeded prefill rows of each of those heads."""
+    w = inputs.WORKLOADS["recall_decode_B64H16_T32768_d64_bf16"]
+    B, H, T, d, n = w.B, w.H, w.T, w.d, w.decode_steps
+    q, k, v = inputs.make_qkv_device(B, H, T, d, d, seed=w.seed)
+    so = torch.empty((B, H, d * d, d), dtype=torch.float32, device="cuda")
+    zo = torch.empty((B, H, d, d), dtype=torch.float32, device="cuda")
+    out = K.kata_chunked_forward(q, k, v, C=w.C, state_out=so, z_out=zo)
+    pair_pos, pick = inputs.recall_decode_plan(w)
+    # fresh unit keys and N(0, 1) values for the decode tokens
+    _, k_dec, v_dec = inputs.make_qkv_device(B, H, n, d, d, seed=w.seed + 1)
+    pos_t = torch.from_numpy(pair_pos[pick]).cuda()  # [n, B, H]
+    ys = torch.empty((n, B, H, d), dtype=torch.bfloat16, device="cuda")
+    q_dec = torch.empty((n, B, H, d), dtype=torch.bfloat16, device="cuda")
+    bidx = torch.arange(B, device="cuda")[:, None].expand(B, H)
+    hidx = torch.arange(H, device="cuda")[None, :].expand(B, H)
+    for s in range(n):
+        q_dec[s] = k[bidx, hidx, pos_t[s]]
+        K.kata_decode_step(q_dec[s], k_dec[:, :, s].contiguous(), v_dec[:, :, s].contiguous(),
+                           so, zo, out=ys[s])
+    torch.cuda.synchronize()
+    assert K.kata_get_device_status() == 0
+
+    g = np.random.default_rng(5)
+    heads = g.choice(B * H, size=16, replace=False)
+    tq, tk, tv = (x.view(B * H, T, d) for x in (q, k, v))
+    for hh in heads:
+        b, h = divmod(int(hh), H)
+        qa = np.concatenate([from_device(tq[hh]), from_device(q_dec[:, b, h])])
+        ka = np.concatenate([from_device(tk[hh]), from_device(k_dec[b, h])])
+        va = np.concatenate([from_device(tv[hh]), from_device(v_dec[b, h])])
+        rows = np.concatenate([np.arange(T, T + n), g.integers(0, T, size=64)])
+        yref = oracle_mod.forward_rows(qa[None], ka[None], va[None], np.zeros_like(rows), rows)
+        ydec = from_device(ys[:, b, h])
+        ypre = from_device(out[b, h])[rows[n:]]
+        assert row_err(ydec, yref[:n]) <= TOL["bf16"], f"decode head {hh}"
+        assert row_err(ypre, yref[n:]) <= TOL["bf16"], f"prefill head {hh}"
