@@ -110,6 +110,40 @@ kata_status kata_chunked_forward(const void *q, const void *k, const void *v, vo
                                  size_t workspace_bytes, kata_stream_t stream);
 
 /*
+ * kata_chunked_forward without a caller-provided workspace, for callers that
+ * cannot allocate device memory themselves: code running inside a host
+ * framework that owns all device memory through its own pool, or a
+ * latency-critical loop whose memory is fixed before it starts.
+ * The paper has no counterpart; this is a deployment convenience.
+ *
+ * The scratch lives in a statically sized device array inside libkata of
+ * KATA_NOALLOC_SCRATCH_BYTES bytes.  Every GPU that loads the library keeps
+ * that array for the life of the process.  The call allocates nothing and
+ * frees nothing.  Arguments, layouts and results are those of
+ * kata_chunked_forward (same kernels).
+ *
+ *   - A problem fits when kata_chunked_forward_workspace_bytes(...) <=
+ *     KATA_NOALLOC_SCRATCH_BYTES; larger ones return KATA_ERR_WORKSPACE before
+ *     anything is launched.
+ *   - The scratch of the CURRENT device is used: make the device that owns
+ *     the tensors current before the call.
+ *   - The first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress) and caches it.  Make that first call before
+ *     any stream capture on that device.
+ *   - All calls on a device share the one array, and the array keeps what the
+ *     last call wrote.  Every scratch element a call reads was first written
+ *     by that same call, so nothing needs clearing between calls.  Calls
+ *     that can overlap on the GPU (different streams, or several host
+ *     threads) race on the array: serialise them.
+ */
+#define KATA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+kata_status kata_chunked_forward_noalloc(const void *q, const void *k, const void *v, void *out,
+                                         int B, int H, int T, int dk, int dv, int C,
+                                         kata_dtype dtype, float *state_out, float *z_out,
+                                         kata_stream_t stream);
+
+/*
  * One recurrent decode step for every head, in place
  * (arXiv abstract, "constant-time recurrent inference"; gist.science summary
  * 1: a fixed-size state replaces the key-value cache):

@@ -7,6 +7,7 @@ include/kata.h); ``binding`` marshals torch CUDA tensors into it.
 from .binding import (  # noqa: F401
     KataError,
     kata_chunked_forward,
+    kata_chunked_forward_noalloc,
     kata_chunked_forward_workspace_bytes,
     kata_decode_step,
     kata_get_device_status,

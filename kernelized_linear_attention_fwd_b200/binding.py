@@ -30,6 +30,7 @@ EXPORTS = (
     "kata_status_string",
     "kata_chunked_forward_workspace_bytes",
     "kata_chunked_forward",
+    "kata_chunked_forward_noalloc",
     "kata_decode_step",
     "kata_get_device_status",
 )
@@ -64,6 +65,9 @@ def load_library(path: str = LIB_PATH):
     lib.kata_chunked_forward.restype = i32
     lib.kata_chunked_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                          fp, fp, vp, sz, vp]
+    lib.kata_chunked_forward_noalloc.restype = i32
+    lib.kata_chunked_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                                 i32, fp, fp, vp]
     lib.kata_decode_step.restype = i32
     lib.kata_decode_step.argtypes = [vp, vp, vp, vp, fp, fp, i32, i32, i32, i32, i32, vp]
     lib.kata_get_device_status.restype = i32
@@ -151,6 +155,39 @@ def kata_chunked_forward(q, k, v, C=64, out=None, state_out=None, z_out=None, wo
                                   _stream_handle(stream))
     if st != KATA_OK:
         raise KataError(st, "kata_chunked_forward")
+    return out
+
+
+# Bytes of the library's static scratch used by kata_chunked_forward_noalloc.
+KATA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def kata_chunked_forward_noalloc(q, k, v, C=64, out=None, state_out=None, z_out=None,
+                                 stream=None):
+    """kata_chunked_forward with the library's static device scratch instead of
+    a workspace: for callers that cannot allocate device memory.  `out`
+    (and the optional state buffers) must be passed in by such callers; when
+    `out` is None it is allocated here for convenience.  Problems needing more
+    than KATA_NOALLOC_SCRATCH_BYTES of scratch raise KATA_ERR_WORKSPACE."""
+    import torch
+
+    lib = load_library()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", (B, H, T, dk))
+    _check(k, "k", (B, H, T, dk), q.dtype)
+    _check(v, "v", (B, H, T, dv), q.dtype)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", (B, H, T, dv), q.dtype)
+    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32)
+    _check(z_out, "z_out", (B, H, dk, dk), torch.float32)
+    st = lib.kata_chunked_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv,
+                                          int(C), code, _ptr(state_out), _ptr(z_out),
+                                          _stream_handle(stream))
+    if st != KATA_OK:
+        raise KataError(st, "kata_chunked_forward_noalloc")
     return out
 
 
