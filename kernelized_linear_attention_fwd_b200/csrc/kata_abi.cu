@@ -66,7 +66,11 @@ kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dty
     p.R = packed_rows(dk);
     p.L = segment_length(dk, C);
     p.n_seg = (T + p.L - 1) / p.L;
-    p.path = Path::kSimt;
+    p.path = (dtype == KATA_BF16 && dk == 64) ? Path::kTensorCore : Path::kSimt;
+    if (p.path == Path::kTensorCore) {
+        tc::plan_tc_workspace(p);
+        return KATA_OK;
+    }
     const size_t E = (size_t)p.R * (dv + 1);
     const size_t seg_bytes = (size_t)BH * p.n_seg * E * sizeof(float);
     const size_t total_bytes = p.n_seg > 1 ? (size_t)BH * E * sizeof(float) : 0;
@@ -128,7 +132,9 @@ kata_status kata_chunked_forward(const void *q, const void *k, const void *v, vo
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e =
-        kata::launch_simt_forward(p, q, k, v, out, state_out, z_out, workspace, st);
+        p.path == kata::Path::kTensorCore
+            ? kata::tc::launch_tc_forward(p, q, k, v, out, state_out, z_out, workspace, st)
+            : kata::launch_simt_forward(p, q, k, v, out, state_out, z_out, workspace, st);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
 }
 

@@ -85,6 +85,14 @@ __device__ __forceinline__ void store_out(__nv_bfloat16 *p, long long i, float x
 cudaError_t launch_simt_forward(const Plan &p, const void *q, const void *k, const void *v,
                                 void *out, float *state_out, float *z_out, void *ws,
                                 cudaStream_t st);
+namespace tc {
+// Tensor-core path (bf16, d = dv = 64): workspace layout and launcher.
+void plan_tc_workspace(Plan &p);
+cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v,
+                              void *out, float *state_out, float *z_out, void *ws,
+                              cudaStream_t st);
+}  // namespace tc
+
 cudaError_t launch_decode(int B, int H, int dk, int dv, kata_dtype dtype, const void *q,
                           const void *k, const void *v, void *out, float *state, float *z,
                           cudaStream_t st);

@@ -1,0 +1,630 @@
+// KATA causal forward, tensor-core path (bf16 q, k, v, d = dv = 64, sm_100a).
+//
+// Exact chunked-state form (gist.science summary of "Kernelized Linear
+// Attention: Breaking the Capacity Wall with Symmetric Cones", Technical
+// summary 2.3: tensor cores inside a chunk, associative scan of chunk states
+// across chunks; arXiv abstract: "exact O(T) chunked-state form").  States are
+// stored every L tokens (a segment); inside a segment the causal quadratic
+// form is used, which equals the chunk-by-chunk propagation exactly.
+//
+//   tc_state_build   per segment: dS = sum phi(k) v^T on the half-strip rows
+//                    (tc_layout.cuh) and dZ = sum k k^T, fp32
+//   tc_seg_scan      exclusive prefix over segments (associative scan) into a
+//                    bf16 copy for the readout, plus the fp32 total
+//   tc_read          per 256 queries: phi(Q) S_prev and q^T Z_prev q on tcgen05
+//                    (phi(Q) generated from registers into tensor memory), the
+//                    intra-segment squared-score term on tcgen05, the division
+//   tc_state_expand  fp32 total -> dense [64*64, 64] state and [64, 64] Z
+#include <cuda_bf16.h>
+
+#include "kata_internal.cuh"
+#include "sm100.cuh"
+#include "tc_layout.cuh"
+#include "tmap.cuh"
+
+namespace kata {
+namespace tc {
+namespace {
+
+using namespace kata::sm100;
+
+constexpr long long kF32PerSeg = (long long)kF32Rows * kD;    // 167,936 floats
+constexpr long long kBf16PerSeg = (long long)kBf16Rows * kD;  // 172,032 bf16
+
+// ---------------------------------------------------------------------------
+// State builder (fp32 CUDA cores, half-strip row order).
+// grid.x = row-block (82 of 32 rows) + 82 * (segment + n_build * bh);
+// block 256 = 32 rows x 8 groups of 8 value columns.
+// Rows 0..2559: dS[r][e] = sum_s k_si k_sj v_se; rows 2560..2623: Z[i][e] =
+// sum_s k_si k_se.
+// ---------------------------------------------------------------------------
+constexpr int kBuildTok = 64;
+
+__global__ void __launch_bounds__(256)
+tc_state_build_simt(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
+                    float *__restrict__ seg_state, int T, int L, int n_seg, int n_build) {
+    constexpr int NRB = (kF32Rows + 31) / 32;
+    __shared__ float sk[kBuildTok][kD + 1];
+    __shared__ float sv[kBuildTok][kD];
+    const int tid = threadIdx.x, lr = tid & 31, eg = tid >> 5;
+    long long blk = blockIdx.x;
+    const int rb = (int)(blk % NRB);
+    blk /= NRB;
+    const int g = (int)(blk % n_build);
+    const long long bh = blk / n_build;
+    const int r = rb * 32 + lr;
+    const bool live = r < kF32Rows;
+    int i = 0, j = 0;
+    const bool zrow = r >= kStateRows;
+    if (live && !zrow) {
+        i = hs_i(r / 16);
+        j = hs_jb(r / 16) + r % 16;
+    } else if (live) {
+        i = r - kStateRows;
+    }
+    float acc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+    const int s0 = g * L, s1 = min(T, s0 + L);
+    for (int t0 = s0; t0 < s1; t0 += kBuildTok) {
+        __syncthreads();
+        for (int x = tid; x < kBuildTok * kD; x += 256) {
+            const int s = x / kD, c = x % kD, ts = t0 + s;
+            const bool in = ts < s1;
+            sk[s][c] = in ? __bfloat162float(k[(bh * T + ts) * kD + c]) : 0.f;
+            sv[s][c] = in ? __bfloat162float(v[(bh * T + ts) * kD + c]) : 0.f;
+        }
+        __syncthreads();
+        const int n = min(kBuildTok, s1 - t0);
+        if (zrow) {
+            for (int s = 0; s < n; ++s) {
+                const float a = sk[s][i];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc[u] = fmaf(a, sk[s][eg * 8 + u], acc[u]);
+            }
+        } else {
+            for (int s = 0; s < n; ++s) {
+                const float f = sk[s][i] * sk[s][j];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) acc[u] = fmaf(f, sv[s][eg * 8 + u], acc[u]);
+            }
+        }
+    }
+    if (live) {
+        float *dst = seg_state + (bh * n_seg + g) * kF32PerSeg + (long long)r * kD + eg * 8;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) dst[u] = acc[u];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Exclusive prefix over segments -> bf16 copy (+ Z split into hi and lo), and
+// the fp32 total.  Same scheme as seg_scan: 32-segment x 32-element tiles
+// through shared memory, Kogge-Stone shuffle scan down each element column.
+// grid.x = element-tile + n_et * bh; block (32, 8)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ prefix,
+            float *__restrict__ total, int n_seg, int n_valid) {
+    __shared__ float tile[32][33];
+    const int lane = threadIdx.x, w = threadIdx.y;
+    constexpr long long E = kF32PerSeg;
+    constexpr long long n_et = E / 32;
+    const long long et = blockIdx.x % n_et;
+    const long long bh = blockIdx.x / n_et;
+    const long long e_base = et * 32;
+    const float *base = seg_state + bh * (long long)n_seg * E;
+    __nv_bfloat16 *pbase = prefix + bh * (long long)n_seg * kBf16PerSeg;
+    float carry[4] = {0.f, 0.f, 0.f, 0.f};
+    const bool z_tile = e_base >= (long long)kStateRows * kD;
+
+    for (int g0 = 0; g0 < n_seg; g0 += 32) {
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            const int gs = w + 8 * rr, g = g0 + gs;
+            tile[gs][lane] = g < n_valid ? base[(long long)g * E + e_base + lane] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+            const int c = w + 8 * cc;
+            const float x = tile[lane][c];
+            float inc = x;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, inc, off);
+                if (lane >= off) inc += y;
+            }
+            tile[lane][c] = carry[cc] + (inc - x);
+            carry[cc] += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+            const int gs = w + 8 * rr, g = g0 + gs;
+            if (g < 1 || g >= n_seg) continue;  // segment 0 has an empty prefix
+            const float p = tile[gs][lane];
+            __nv_bfloat16 *dst = pbase + (long long)g * kBf16PerSeg;
+            if (!z_tile) {
+                dst[e_base + lane] = __float2bfloat16_rn(p);
+            } else {
+                const long long z = e_base + lane - (long long)kStateRows * kD;
+                const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
+                dst[(long long)kZHiRow0 * kD + z] = hi;
+                dst[(long long)kZLoRow0 * kD + z] = lo;
+            }
+        }
+        __syncthreads();
+    }
+    if (total != nullptr && lane == 0) {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) total[bh * E + e_base + w + 8 * cc] = carry[cc];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// fp32 total (half-strip layout) -> dense state [64*64][64] and Z [64][64].
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__restrict__ state_out,
+                float *__restrict__ z_out, long long BH) {
+    const long long per = (long long)kD * kD * kD + kD * kD;
+    const long long idx = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (idx >= per * BH) return;
+    const long long bh = idx / per;
+    long long x = idx % per;
+    const float *src = total + bh * stride_bh;
+    if (x < (long long)kD * kD * kD) {
+        const int row = (int)(x / kD), e = (int)(x % kD);
+        int i = row / kD, j = row % kD;
+        if (i > j) { const int t = i; i = j; j = t; }
+        const int h = hs_index(i, j);
+        state_out[bh * kD * kD * kD + x] = src[((long long)h * 16 + (j - hs_jb(h))) * kD + e];
+    } else {
+        x -= (long long)kD * kD * kD;
+        z_out[bh * kD * kD + x] = src[(long long)kZRow0 * kD + x];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Readout kernel.
+// ---------------------------------------------------------------------------
+constexpr int kQT = 128;                 // query tile (MMA M)
+constexpr int kTiles = 2;                // query tiles per CTA
+constexpr int kCtaQ = kQT * kTiles;      // 256 queries per CTA
+constexpr int kKB = 128;                 // key block
+constexpr int kRing = 4;                 // inter-term pipeline depth
+constexpr int kInterStages = kHalfStrips / 2;  // 80 stages of 2 half-strips
+constexpr int kGenWarps = 8;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kReadThreads = 320;
+
+// shared memory (from a 1024-byte aligned base)
+constexpr int kSmQ = 0;                          // 2 x [128 x 64] bf16, K-major, swizzled
+constexpr int kSmZ = kSmQ + kTiles * 16384;      // Z hi [64 x 64], Z lo [64 x 64]
+constexpr int kSmS = kSmZ + 16384;               // ring of [32 x 64] state tiles
+constexpr int kSmK = kSmS + kRing * 4096;        // 2 x [128 x 64] keys
+constexpr int kSmV = kSmK + 2 * 16384;           // 2 x [128 x 64] values
+constexpr int kSmBytes = kSmV + 2 * 16384;
+constexpr int kSmAlloc = kSmBytes + 1024;
+
+// tensor memory columns (512 allocated)
+constexpr uint32_t kTmO = 0;     // O[g]: 64 columns at 64 g
+constexpr uint32_t kTmS = 128;   // scores S[g]: 128 columns at 128 + 128 g (U[g] first)
+constexpr uint32_t kTmA = 384;   // phi(Q) stages / P[g]: 64 columns at 384 + 64 g
+
+struct ReadBars {
+    uint64_t q, u, o;
+    uint64_t bfull[kRing], bempty[kRing], afull[kRing], aempty[kRing];
+    uint64_t kvfull[2], kvempty[2];
+    uint64_t sfull[kTiles], pfull[kTiles];
+};
+
+__device__ __forceinline__ uint32_t dup_lo(uint32_t x) { return __byte_perm(x, 0, 0x1010); }
+__device__ __forceinline__ uint32_t dup_hi(uint32_t x) { return __byte_perm(x, 0, 0x3232); }
+
+// phi(q) weights for the 16 rows of half-strip H: c_ij q_i q_j with c = 2 for
+// j > i, 1 for j = i, 0 for j < i (mirrored entries), packed two rows per
+// 32-bit word (tensor-memory A layout: row pair (2p, 2p+1) in column p).
+template <int H>
+__device__ __forceinline__ void gen_halfstrip(const uint32_t (&q2)[32], uint32_t *out) {
+    constexpr int i = hs_i(H);
+    constexpr int jb = hs_jb(H);
+    const uint32_t qi = (i & 1) ? dup_hi(q2[i / 2]) : dup_lo(q2[i / 2]);
+    const uint32_t qi2 = mul_bf16x2(qi, 0x40004000u);  // 2 q_i, exact
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+        const int j0 = jb + 2 * p, j1 = j0 + 1;
+        if (j1 < i) {
+            out[p] = 0u;
+        } else if (j0 > i) {
+            out[p] = mul_bf16x2(qi2, q2[j0 / 2]);
+        } else if (j0 == i) {
+            out[p] = mul_bf16x2(__byte_perm(qi, qi2, 0x7610), q2[j0 / 2]);  // (1, 2)
+        } else {  // j1 == i
+            out[p] = mul_bf16x2(qi & 0xFFFF0000u, q2[j0 / 2]);  // (0, 1)
+        }
+    }
+}
+
+template <int ST>
+__device__ __forceinline__ void gen_stage(const uint32_t (&q2)[32], uint32_t *a) {
+    gen_halfstrip<2 * ST>(q2, a);
+    gen_halfstrip<2 * ST + 1>(q2, a + 8);
+}
+
+template <int ST>
+struct GenLoop {
+    __device__ __forceinline__ static bool run(const uint32_t (&q2)[32], ReadBars &bars,
+                                               uint32_t ta_base, volatile int *abort) {
+        constexpr int stage = ST % kRing;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[stage], ((ST / kRing) & 1) ^ 1, abort)))
+            return false;
+        tc_fence_after();
+        uint32_t a[16];
+        gen_stage<ST>(q2, a);
+        tmem_st16(ta_base + 16 * stage, a);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars.afull[stage]);
+        return GenLoop<ST + 1>::run(q2, bars, ta_base, abort);
+    }
+};
+template <>
+struct GenLoop<kInterStages> {
+    __device__ __forceinline__ static bool run(const uint32_t (&)[32], ReadBars &, uint32_t,
+                                               volatile int *) {
+        return true;
+    }
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    const uint32_t s = smem_u32(p);
+    return p + ((1024u - (s & 1023u)) & 1023u);
+}
+
+__device__ __forceinline__ void set_timeout_status(int *status) {
+    atomicCAS(status, 0, (int)KATA_ERR_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(kReadThreads, 1)
+tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
+        __nv_bfloat16 *__restrict__ out, int T, int L, int n_seg, int n_ct, int *status) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ ReadBars bars;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+
+    uint8_t *sm = align1024(smem_raw);
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int bh = blockIdx.x / n_ct;
+    const int t0 = (blockIdx.x % n_ct) * kCtaQ;
+    const int g = t0 / L;
+    const int seg0 = g * L;
+    const bool inter = g > 0;
+    const int n_kb = (t0 + kCtaQ - seg0) / kKB;
+    const int sidx = bh * n_seg + g;
+
+    if (tid == 0) {
+        abort_flag = 0;
+        mbar_init(&bars.q, 1);
+        mbar_init(&bars.u, 1);
+        mbar_init(&bars.o, 1);
+        for (int s = 0; s < kRing; ++s) {
+            mbar_init(&bars.bfull[s], 1);
+            mbar_init(&bars.bempty[s], 1);
+            mbar_init(&bars.afull[s], kGenWarps * 32);
+            mbar_init(&bars.aempty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bars.kvfull[s], 1);
+            mbar_init(&bars.kvempty[s], 1);
+        }
+        for (int s = 0; s < kTiles; ++s) {
+            mbar_init(&bars.sfull[s], 1);
+            mbar_init(&bars.pfull[s], 4 * 32);
+        }
+        fence_mbarrier_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(&tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tmem_base;
+    volatile int *abort = &abort_flag;
+
+    if (warp == kTmaWarp) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_s);
+            mbar_arrive_expect_tx(&bars.q, kTiles * 16384 + (inter ? 16384 : 0));
+            for (int tl = 0; tl < kTiles; ++tl)
+                tma_load_3d(sm + kSmQ + tl * 16384, &tm_q, &bars.q, 0, t0 + tl * kQT, bh);
+            if (inter) {
+                for (int zz = 0; zz < 4; ++zz)  // Z hi rows 2560..2623, Z lo rows 2624..2687
+                    tma_load_3d(sm + kSmZ + zz * 4096, &tm_s, &bars.q, 0, kZHiRow0 + 32 * zz,
+                                sidx);
+            }
+            int issued_b = 0, issued_kv = 0;
+            bool ok = true;
+            if (inter) {
+                for (int st = 0; st < kInterStages && ok; ++st) {
+                    const int s = st % kRing;
+                    ok = mbar_wait(&bars.bempty[s], ((st / kRing) & 1) ^ 1, abort);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&bars.bfull[s], 4096);
+                    tma_load_3d(sm + kSmS + s * 4096, &tm_s, &bars.bfull[s], 0, 32 * st, sidx);
+                    ++issued_b;
+                }
+            }
+            for (int kb = 0; kb < n_kb && ok; ++kb) {
+                const int s = kb & 1;
+                ok = mbar_wait(&bars.kvempty[s], ((kb >> 1) & 1) ^ 1, abort);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&bars.kvfull[s], 32768);
+                tma_load_3d(sm + kSmK + s * 16384, &tm_k, &bars.kvfull[s], 0, seg0 + kb * kKB, bh);
+                tma_load_3d(sm + kSmV + s * 16384, &tm_v, &bars.kvfull[s], 0, seg0 + kb * kKB, bh);
+                ++issued_kv;
+            }
+            // drain: every load issued must have landed before the CTA exits
+            mbar_wait(&bars.q, 0, abort);
+            for (int st = (issued_b > kRing ? issued_b - kRing : 0); st < issued_b; ++st)
+                mbar_wait(&bars.bfull[st % kRing], (st / kRing) & 1, abort);
+            for (int kb = (issued_kv > 2 ? issued_kv - 2 : 0); kb < issued_kv; ++kb)
+                mbar_wait(&bars.kvfull[kb & 1], (kb >> 1) & 1, abort);
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            const uint32_t id_qk = idesc_bf16(kQT, kKB, 0, 0);
+            const uint32_t id_n64 = idesc_bf16(kQT, 64, 0, 1);
+            const uint32_t sQ = smem_u32(sm + kSmQ), sZ = smem_u32(sm + kSmZ);
+            const uint32_t sS = smem_u32(sm + kSmS), sK = smem_u32(sm + kSmK),
+                           sV = smem_u32(sm + kSmV);
+            bool ok = mbar_wait(&bars.q, 0, abort);
+            bool acc_o[kTiles] = {false, false};
+            if (ok) tc_fence_after();
+            if (ok && inter) {
+                for (int tl = 0; tl < kTiles; ++tl) {
+                    const uint32_t dU = tm + kTmS + 128 * tl;
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ss(dU, desc_sw128(sQ + tl * 16384 + 32 * ks, 16, 1024),
+                               desc_sw128(sZ + 2048 * ks, 8192, 1024), id_n64, ks > 0);
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ss(dU, desc_sw128(sQ + tl * 16384 + 32 * ks, 16, 1024),
+                               desc_sw128(sZ + 8192 + 2048 * ks, 8192, 1024), id_n64, 1);
+                }
+                mma_commit(&bars.u);
+                for (int st = 0; st < kInterStages && ok; ++st) {
+                    const int s = st % kRing;
+                    const uint32_t ph = (st / kRing) & 1;
+                    ok = mbar_wait(&bars.bfull[s], ph, abort) && mbar_wait(&bars.afull[s], ph, abort);
+                    if (!ok) break;
+                    tc_fence_after();
+                    for (int tl = 0; tl < kTiles; ++tl)
+                        for (int ks = 0; ks < 2; ++ks)
+                            mma_ts(tm + kTmO + 64 * tl, tm + kTmA + 64 * tl + 16 * s + 8 * ks,
+                                   desc_sw128(sS + s * 4096 + 2048 * ks, 8192, 1024), id_n64,
+                                   (st | ks) > 0);
+                    mma_commit(&bars.bempty[s]);
+                    mma_commit(&bars.aempty[s]);
+                }
+                acc_o[0] = acc_o[1] = true;
+            }
+            for (int kb = 0; kb < n_kb && ok; ++kb) {
+                const int s = kb & 1;
+                ok = mbar_wait(&bars.kvfull[s], (kb >> 1) & 1, abort);
+                if (!ok) break;
+                tc_fence_after();
+                const int kbs = seg0 + kb * kKB;
+                for (int tl = 0; tl < kTiles; ++tl) {
+                    if (kbs >= t0 + tl * kQT + kQT) continue;  // block entirely after the tile
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ss(tm + kTmS + 128 * tl, desc_sw128(sQ + tl * 16384 + 32 * ks, 16, 1024),
+                               desc_sw128(sK + s * 16384 + 32 * ks, 16, 1024), id_qk, ks > 0);
+                    mma_commit(&bars.sfull[tl]);
+                }
+                for (int tl = 0; tl < kTiles && ok; ++tl) {
+                    if (kbs >= t0 + tl * kQT + kQT) continue;
+                    ok = mbar_wait(&bars.pfull[tl], kb & 1, abort);
+                    if (!ok) break;
+                    tc_fence_after();
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_ts(tm + kTmO + 64 * tl, tm + kTmA + 64 * tl + 8 * ks,
+                               desc_sw128(sV + s * 16384 + 2048 * ks, 8192, 1024), id_n64,
+                               (acc_o[tl] || ks > 0) ? 1u : 0u);
+                    acc_o[tl] = true;
+                }
+                mma_commit(&bars.kvempty[s]);
+            }
+            mma_commit(&bars.o);
+            mbar_wait(&bars.o, 0, abort);  // drain before the CTA may free tensor memory
+        }
+    } else {
+        // ------------------------------------------------------------ generation / softmax
+        const int tl = warp / 4, qd = warp % 4;
+        const int row = 32 * qd + lane;
+        const int tq = t0 + tl * kQT + row;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars.q, 0, abort));
+        uint32_t q2[32];
+        {
+            const uint8_t *qrow = sm + kSmQ + tl * 16384 + row * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(qrow + ((c ^ (row & 7)) * 16));
+                q2[4 * c + 0] = x.x;
+                q2[4 * c + 1] = x.y;
+                q2[4 * c + 2] = x.z;
+                q2[4 * c + 3] = x.w;
+            }
+        }
+        float den_inter = 0.f;
+        if (ok && inter) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars.u, 0, abort));
+            if (ok) {
+                tc_fence_after();
+                uint32_t u[32];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    tmem_ld32(tm + kTmS + 128 * tl + lane_base + 32 * half, u);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) {
+                        const uint32_t w = q2[16 * half + x];
+                        den_inter = fmaf(__uint_as_float(w << 16), __uint_as_float(u[2 * x]), den_inter);
+                        den_inter = fmaf(__uint_as_float(w & 0xFFFF0000u),
+                                         __uint_as_float(u[2 * x + 1]), den_inter);
+                    }
+                }
+                ok = GenLoop<0>::run(q2, bars, tm + kTmA + 64 * tl + lane_base, abort);
+            }
+        }
+        float l = 0.f;
+        const uint32_t tS = tm + kTmS + 128 * tl + lane_base;
+        const uint32_t tP = tm + kTmA + 64 * tl + lane_base;
+        for (int kb = 0; kb < n_kb && ok; ++kb) {
+            const int kbs = seg0 + kb * kKB;
+            if (kbs >= t0 + tl * kQT + kQT) continue;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfull[tl], kb & 1, abort));
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32], p[16];
+                tmem_ld32(tS + 32 * c, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    const int key = kbs + 32 * c + 2 * x;
+                    const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
+                    const float w0 = key <= tq ? s0 * s0 : 0.f;
+                    const float w1 = key + 1 <= tq ? s1 * s1 : 0.f;
+                    l += w0 + w1;
+                    p[x] = pack_bf16x2(w0, w1);
+                }
+                tmem_st16(tP + 16 * c, p);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars.pfull[tl]);
+        }
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.o, 0, abort));
+        if (ok) {
+            tc_fence_after();
+            const float den = l + den_inter;
+            const float inv = den == 0.f ? 0.f : 1.f / den;
+            uint32_t o[32];
+            uint4 *dst = reinterpret_cast<uint4 *>(out + ((long long)bh * T + tq) * kD);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                tmem_ld32(tm + kTmO + 64 * tl + lane_base + 32 * half, o);
+                tmem_ld_wait();
+                if (tq < T) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
+                        v.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
+                        v.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
+                        v.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
+                        dst[4 * half + c] = v;
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) tmem_dealloc(tm, 512);
+    if (tid == 0 && abort_flag) set_timeout_status(status);
+}
+
+bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const void *prefix,
+               CUtensorMap *mq, CUtensorMap *mk, CUtensorMap *mv, CUtensorMap *ms) {
+    const uint64_t dqkv[3] = {(uint64_t)kD, (uint64_t)p.T, (uint64_t)p.BH};
+    const uint64_t sqkv[2] = {(uint64_t)kD * 2, (uint64_t)p.T * kD * 2};
+    const uint32_t bqkv[3] = {64, 128, 1};
+    const uint64_t ds[3] = {(uint64_t)kD, (uint64_t)kBf16Rows, (uint64_t)(p.BH * p.n_seg)};
+    const uint64_t ss[2] = {(uint64_t)kD * 2, (uint64_t)kBf16Rows * kD * 2};
+    const uint32_t bs[3] = {64, 32, 1};
+    return make_tmap_bf16(mq, q, 3, dqkv, sqkv, bqkv) && make_tmap_bf16(mk, k, 3, dqkv, sqkv, bqkv) &&
+           make_tmap_bf16(mv, v, 3, dqkv, sqkv, bqkv) &&
+           make_tmap_bf16(ms, prefix ? prefix : q, 3, ds, ss, bs);
+}
+
+}  // namespace
+
+// Workspace of the tensor-core path (bytes; 256-aligned parts):
+//   fp32 segment states  BH * n_seg * 2624 * 64 * 4
+//   fp32 total           BH * 2624 * 64 * 4
+//   bf16 prefixes        BH * n_seg * 2688 * 64 * 2
+void plan_tc_workspace(Plan &p) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t seg = (size_t)p.BH * p.n_seg * kF32PerSeg * 4;
+    const size_t tot = (size_t)p.BH * kF32PerSeg * 4;
+    const size_t pre = (size_t)p.BH * p.n_seg * kBf16PerSeg * 2;
+    p.ws_seg_state = 0;
+    p.ws_total = up(seg);
+    p.ws_extra = p.ws_total + up(tot);
+    p.ws_bytes = p.ws_extra + up(pre);
+}
+
+cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
+                              float *state_out, float *z_out, void *ws, cudaStream_t st) {
+    char *w = static_cast<char *>(ws);
+    float *seg = reinterpret_cast<float *>(w + p.ws_seg_state);
+    float *total = reinterpret_cast<float *>(w + p.ws_total);
+    __nv_bfloat16 *prefix = reinterpret_cast<__nv_bfloat16 *>(w + p.ws_extra);
+    const bool want_state = state_out != nullptr;
+    const int n_build = want_state ? p.n_seg : p.n_seg - 1;
+    const long long BH = p.BH;
+    int *status = device_status_ptr();
+    if (!status) return cudaErrorUnknown;
+
+    if (n_build > 0) {
+        ProfScope ps("tc_state_build_simt", st);
+        const long long grid = (long long)((kF32Rows + 31) / 32) * n_build * BH;
+        tc_state_build_simt<<<(unsigned)grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), seg, p.T,
+            p.L, p.n_seg, n_build);
+    }
+    if (p.n_seg > 1) {
+        ProfScope ps("tc_seg_scan", st);
+        const long long grid = (kF32PerSeg / 32) * BH;
+        tc_seg_scan<<<(unsigned)grid, dim3(32, 8), 0, st>>>(seg, prefix, want_state ? total : nullptr,
+                                                            p.n_seg, n_build);
+    }
+    {
+        CUtensorMap mq, mk, mv, ms;
+        if (!make_maps(p, q, k, v, prefix, &mq, &mk, &mv, &ms)) return cudaErrorInvalidValue;
+        cudaError_t e = cudaFuncSetAttribute(tc_read, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmAlloc);
+        if (e != cudaSuccess) return e;
+        const int n_ct = (p.T + kCtaQ - 1) / kCtaQ;
+        ProfScope ps("tc_read", st);
+        tc_read<<<(unsigned)(n_ct * BH), kReadThreads, kSmAlloc, st>>>(
+            mq, mk, mv, ms, static_cast<__nv_bfloat16 *>(out), p.T, p.L, p.n_seg, n_ct, status);
+    }
+    if (want_state) {
+        const float *src = p.n_seg > 1 ? total : seg;
+        const long long stride = p.n_seg > 1 ? kF32PerSeg : kF32PerSeg * p.n_seg;
+        const long long n = ((long long)kD * kD * kD + kD * kD) * BH;
+        ProfScope ps("tc_state_expand", st);
+        tc_state_expand<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, stride, state_out, z_out, BH);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace tc
+}  // namespace kata
