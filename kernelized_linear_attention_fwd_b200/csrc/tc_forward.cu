@@ -7,8 +7,9 @@
 // stored every L tokens (a segment); inside a segment the causal quadratic
 // form is used, which equals the chunk-by-chunk propagation exactly.
 //
-//   tc_state_build   per segment: dS = sum phi(k) v^T on the half-strip rows
-//                    (tc_layout.cuh) and dZ = sum k k^T, fp32
+//   k_transpose      keys transposed per head (tokens contiguous)
+//   tc_build         per segment on tcgen05: dS = sum phi(k) v^T on the
+//                    half-strip rows (tc_layout.cuh) and dZ = sum k k^T, fp32
 //   tc_seg_scan      exclusive prefix over segments (associative scan) into a
 //                    bf16 copy for the readout, plus the fp32 total
 //   tc_read          per 256 queries: phi(Q) S_prev and q^T Z_prev q on tcgen05
@@ -30,72 +31,6 @@ using namespace kata::sm100;
 
 constexpr long long kF32PerSeg = (long long)kF32Rows * kD;    // 167,936 floats
 constexpr long long kBf16PerSeg = (long long)kBf16Rows * kD;  // 172,032 bf16
-
-// ---------------------------------------------------------------------------
-// State builder (fp32 CUDA cores, half-strip row order).
-// grid.x = row-block (82 of 32 rows) + 82 * (segment + n_build * bh);
-// block 256 = 32 rows x 8 groups of 8 value columns.
-// Rows 0..2559: dS[r][e] = sum_s k_si k_sj v_se; rows 2560..2623: Z[i][e] =
-// sum_s k_si k_se.
-// ---------------------------------------------------------------------------
-constexpr int kBuildTok = 64;
-
-__global__ void __launch_bounds__(256)
-tc_state_build_simt(const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
-                    float *__restrict__ seg_state, int T, int L, int n_seg, int n_build) {
-    constexpr int NRB = (kF32Rows + 31) / 32;
-    __shared__ float sk[kBuildTok][kD + 1];
-    __shared__ float sv[kBuildTok][kD];
-    const int tid = threadIdx.x, lr = tid & 31, eg = tid >> 5;
-    long long blk = blockIdx.x;
-    const int rb = (int)(blk % NRB);
-    blk /= NRB;
-    const int g = (int)(blk % n_build);
-    const long long bh = blk / n_build;
-    const int r = rb * 32 + lr;
-    const bool live = r < kF32Rows;
-    int i = 0, j = 0;
-    const bool zrow = r >= kStateRows;
-    if (live && !zrow) {
-        i = hs_i(r / 16);
-        j = hs_jb(r / 16) + r % 16;
-    } else if (live) {
-        i = r - kStateRows;
-    }
-    float acc[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) acc[u] = 0.f;
-    const int s0 = g * L, s1 = min(T, s0 + L);
-    for (int t0 = s0; t0 < s1; t0 += kBuildTok) {
-        __syncthreads();
-        for (int x = tid; x < kBuildTok * kD; x += 256) {
-            const int s = x / kD, c = x % kD, ts = t0 + s;
-            const bool in = ts < s1;
-            sk[s][c] = in ? __bfloat162float(k[(bh * T + ts) * kD + c]) : 0.f;
-            sv[s][c] = in ? __bfloat162float(v[(bh * T + ts) * kD + c]) : 0.f;
-        }
-        __syncthreads();
-        const int n = min(kBuildTok, s1 - t0);
-        if (zrow) {
-            for (int s = 0; s < n; ++s) {
-                const float a = sk[s][i];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) acc[u] = fmaf(a, sk[s][eg * 8 + u], acc[u]);
-            }
-        } else {
-            for (int s = 0; s < n; ++s) {
-                const float f = sk[s][i] * sk[s][j];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) acc[u] = fmaf(f, sv[s][eg * 8 + u], acc[u]);
-            }
-        }
-    }
-    if (live) {
-        float *dst = seg_state + (bh * n_seg + g) * kF32PerSeg + (long long)r * kD + eg * 8;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) dst[u] = acc[u];
-    }
-}
 
 // ---------------------------------------------------------------------------
 // Exclusive prefix over segments -> bf16 copy (+ Z split into hi and lo), and
@@ -287,6 +222,248 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 
 __device__ __forceinline__ void set_timeout_status(int *status) {
     atomicCAS(status, 0, (int)KATA_ERR_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------
+// Keys transposed per head: kt[bh][d][t] (tokens contiguous), zero-padded to
+// T_pad (a multiple of 64), so the state builder can read, for a feature
+// index, 16 consecutive tokens as one 32-byte run.
+// grid.x = token-tile (T_pad / 64) + n_tt * bh; block 256.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+k_transpose(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ kt, int T, int T_pad) {
+    __shared__ uint16_t tile[64][66];
+    const int n_tt = T_pad / 64;
+    const long long bh = blockIdx.x / n_tt;
+    const int t0 = (blockIdx.x % n_tt) * 64;
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(k);
+    for (int x = threadIdx.x; x < 64 * 32; x += 256) {
+        const int s = x / 32, c2 = x % 32, t = t0 + s;
+        const uint32_t w = t < T ? src[((bh * T + t) * kD) / 2 + c2] : 0u;
+        tile[s][2 * c2] = static_cast<uint16_t>(w & 0xFFFFu);
+        tile[s][2 * c2 + 1] = static_cast<uint16_t>(w >> 16);
+    }
+    __syncthreads();
+    uint32_t *dst = reinterpret_cast<uint32_t *>(kt);
+    for (int x = threadIdx.x; x < 64 * 32; x += 256) {
+        const int d = x / 32, s2 = x % 32;
+        const uint32_t w = static_cast<uint32_t>(tile[2 * s2][d]) |
+                           (static_cast<uint32_t>(tile[2 * s2 + 1][d]) << 16);
+        dst[((bh * kD + d) * T_pad + t0) / 2 + s2] = w;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// State builder on tcgen05.
+//
+// Per (head, segment) 5 CTAs; CTA c accumulates the 4 tiles of 128 state rows
+// (half-strips h = 32 c + 8 m + s, m = tile, s = 16-lane slot) over the
+// segment's tokens:  D[m] += A[m] . V  with  A[m][(i, j)][token] = k_i k_j,
+// generated from the transposed keys into tensor memory by the thread that
+// owns the row's lane, and V (tokens x 64) the MN-major B operand in shared
+// memory.  CTA 0 adds a fifth tile, Z = K^T K (A rows k_i for lanes 0..63, B
+// the key tile itself).  Each thread reads its own key column k_j once per 16
+// tokens and the broadcast column k_i once per tile.
+// Two generation warpgroups take alternate 16-token steps.
+// ---------------------------------------------------------------------------
+constexpr int kBCtas = 5;
+constexpr int kBTiles = 4;
+constexpr int kBRing = 4;                 // A stages, one 16-token step each
+constexpr int kBTok = 64;                 // tokens per TMA tile
+constexpr int kBTileRing = 4;
+constexpr int kBStageBytes = 3 * 8192;    // K^T, V, K tiles
+constexpr int kBSmAlloc = kBTileRing * kBStageBytes + 1024 + 16384;  // padded: one CTA per SM
+constexpr int kBTmaWarp = 8;
+constexpr int kBMmaWarp = 9;
+constexpr int kBuildThreads = 320;
+constexpr uint32_t kBTmA = 320;           // A[stage][m] at 320 + 40 stage + 8 m
+
+struct BuildBars {
+    uint64_t tfull[kBTileRing], tempty[kBTileRing];
+    uint64_t afull[kBRing], aempty[kBRing];
+    uint64_t done;
+};
+
+__global__ void __launch_bounds__(kBuildThreads, 1)
+tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_v,
+         const __grid_constant__ CUtensorMap tm_k, float *__restrict__ seg_state, int T, int L,
+         int n_seg, int n_build, int *status) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ BuildBars bars;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+
+    uint8_t *sm = align1024(smem_raw);
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int c = blockIdx.x % kBCtas;
+    const int rest = blockIdx.x / kBCtas;
+    const int g = rest % n_build;
+    const int bh = rest / n_build;
+    const bool zc = c == 0;
+    const int nm = kBTiles + (zc ? 1 : 0);
+    const int s0 = g * L;
+    const int ntok = min(L, T - s0);
+    const int n_tt = (ntok + kBTok - 1) / kBTok;
+    const int n_ks = 4 * n_tt;
+
+    if (tid == 0) {
+        abort_flag = 0;
+        for (int x = 0; x < kBTileRing; ++x) {
+            mbar_init(&bars.tfull[x], 1);
+            mbar_init(&bars.tempty[x], 1);
+        }
+        for (int x = 0; x < kBRing; ++x) {
+            mbar_init(&bars.afull[x], 128);
+            mbar_init(&bars.aempty[x], 1);
+        }
+        mbar_init(&bars.done, 1);
+        fence_mbarrier_init();
+    }
+    if (warp == kBMmaWarp) {
+        tmem_alloc(&tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = tmem_base;
+    volatile int *abort = &abort_flag;
+
+    if (warp == kBTmaWarp) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_kt);
+            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_k);
+            int issued = 0;
+            for (int t = 0; t < n_tt; ++t) {
+                const int b = t % kBTileRing;
+                if (!mbar_wait(&bars.tempty[b], ((t / kBTileRing) & 1) ^ 1, abort)) break;
+                uint8_t *st = sm + b * kBStageBytes;
+                mbar_arrive_expect_tx(&bars.tfull[b], zc ? 3 * 8192 : 2 * 8192);
+                tma_load_3d(st, &tm_kt, &bars.tfull[b], s0 + kBTok * t, 0, bh);
+                tma_load_3d(st + 8192, &tm_v, &bars.tfull[b], 0, s0 + kBTok * t, bh);
+                if (zc) tma_load_3d(st + 16384, &tm_k, &bars.tfull[b], 0, s0 + kBTok * t, bh);
+                ++issued;
+            }
+            for (int t = (issued > kBTileRing ? issued - kBTileRing : 0); t < issued; ++t)
+                mbar_wait(&bars.tfull[t % kBTileRing], (t / kBTileRing) & 1, abort);
+        }
+    } else if (warp == kBMmaWarp) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(128, 64, 0, 1);
+            const uint32_t sbase = smem_u32(sm);
+            bool ok = true;
+            for (int step = 0; step < n_ks && ok; ++step) {
+                const int t = step / 4, kk = step % 4, b = t % kBTileRing, a = step % kBRing;
+                if (kk == 0) ok = mbar_wait(&bars.tfull[b], (t / kBTileRing) & 1, abort);
+                ok = ok && mbar_wait(&bars.afull[a], (step / kBRing) & 1, abort);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t stb = sbase + b * kBStageBytes;
+                for (int m = 0; m < nm; ++m) {
+                    const uint32_t bsrc = stb + (m == kBTiles ? 16384 : 8192) + 2048 * kk;
+                    mma_ts(tm + 64 * m, tm + kBTmA + 40 * a + 8 * m, desc_sw128(bsrc, 8192, 1024),
+                           idesc, step > 0 ? 1u : 0u);
+                }
+                mma_commit(&bars.aempty[a]);
+                if (kk == 3) mma_commit(&bars.tempty[b]);
+            }
+            mma_commit(&bars.done);
+            mbar_wait(&bars.done, 0, abort);
+        }
+    } else {
+        const int wg = warp / 4, qd = warp % 4;
+        const int row = 32 * qd + lane;          // lane within the 128-row tile
+        const int slot = row / 16, jj = row % 16;
+        const int j = hs_jb(32 * c + slot) + jj;
+        int im[kBTiles];
+#pragma unroll
+        for (int m = 0; m < kBTiles; ++m) im[m] = hs_i(32 * c + 8 * m + slot);
+        const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+        bool ok = true;
+        for (int step = wg; step < n_ks && ok; step += 2) {
+            const int t = step / 4, kk = step % 4, b = t % kBTileRing, a = step % kBRing;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars.tfull[b], (t / kBTileRing) & 1, abort) &&
+                                             mbar_wait(&bars.aempty[a], ((step / kBRing) & 1) ^ 1, abort));
+            if (!ok) break;
+            tc_fence_after();
+            const uint8_t *kt = sm + b * kBStageBytes;  // row d: 64 tokens, swizzled
+            const int c0 = 2 * kk, c1 = 2 * kk + 1;
+            uint32_t own[8];
+            {
+                const uint8_t *r = kt + j * 128;
+                const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (j & 7)) * 16));
+                const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (j & 7)) * 16));
+                own[0] = x0.x; own[1] = x0.y; own[2] = x0.z; own[3] = x0.w;
+                own[4] = x1.x; own[5] = x1.y; own[6] = x1.z; own[7] = x1.w;
+            }
+            const uint32_t ta = tm + kBTmA + 40 * a + lane_base;
+#pragma unroll
+            for (int m = 0; m < kBTiles; ++m) {
+                const int i = im[m];
+                const uint8_t *r = kt + i * 128;
+                const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (i & 7)) * 16));
+                const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (i & 7)) * 16));
+                uint32_t p[8];
+                p[0] = mul_bf16x2(own[0], x0.x); p[1] = mul_bf16x2(own[1], x0.y);
+                p[2] = mul_bf16x2(own[2], x0.z); p[3] = mul_bf16x2(own[3], x0.w);
+                p[4] = mul_bf16x2(own[4], x1.x); p[5] = mul_bf16x2(own[5], x1.y);
+                p[6] = mul_bf16x2(own[6], x1.z); p[7] = mul_bf16x2(own[7], x1.w);
+                tmem_st8(ta + 8 * m, p);
+            }
+            if (zc) {
+                // Z tile: lane i < 64 holds k_i over the tokens, lanes 64.. hold zero
+                uint32_t p[8];
+                if (row < kD) {
+                    const uint8_t *r = kt + row * 128;
+                    const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (row & 7)) * 16));
+                    const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (row & 7)) * 16));
+                    p[0] = x0.x; p[1] = x0.y; p[2] = x0.z; p[3] = x0.w;
+                    p[4] = x1.x; p[5] = x1.y; p[6] = x1.z; p[7] = x1.w;
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) p[x] = 0u;
+                }
+                tmem_st8(ta + 8 * kBTiles, p);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars.afull[a]);
+        }
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.done, 0, abort));
+        if (ok) {
+            tc_fence_after();
+            float *base = seg_state + ((long long)bh * n_seg + g) * kF32PerSeg;
+            // warpgroup 0 stores tiles 0, 1 (and Z), warpgroup 1 tiles 2, 3
+            for (int m = 2 * wg; m < 2 * wg + 2 + ((wg == 0 && zc) ? 1 : 0); ++m) {
+                const int mm = (m == 2 && wg == 0) ? kBTiles : m;
+                uint32_t o[32];
+                float *dst;
+                if (mm == kBTiles)
+                    dst = base + (long long)(kZRow0 + row) * kD;
+                else
+                    dst = base + ((long long)16 * (32 * c + 8 * mm + slot) + jj) * kD;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    tmem_ld32(tm + 64 * mm + lane_base + 32 * half, o);
+                    tmem_ld_wait();
+                    if (mm != kBTiles || row < kD) {
+                        float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * half);
+#pragma unroll
+                        for (int x = 0; x < 8; ++x)
+                            d4[x] = make_float4(__uint_as_float(o[4 * x]), __uint_as_float(o[4 * x + 1]),
+                                                __uint_as_float(o[4 * x + 2]),
+                                                __uint_as_float(o[4 * x + 3]));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kBMmaWarp) tmem_dealloc(tm, 512);
+    if (tid == 0 && abort_flag) set_timeout_status(status);
 }
 
 __global__ void __launch_bounds__(kReadThreads, 1)
@@ -569,15 +746,19 @@ bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const
 //   fp32 segment states  BH * n_seg * 2624 * 64 * 4
 //   fp32 total           BH * 2624 * 64 * 4
 //   bf16 prefixes        BH * n_seg * 2688 * 64 * 2
+//   transposed keys      BH * 64 * T_pad * 2      (T_pad = T rounded up to 64)
 void plan_tc_workspace(Plan &p) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     const size_t seg = (size_t)p.BH * p.n_seg * kF32PerSeg * 4;
     const size_t tot = (size_t)p.BH * kF32PerSeg * 4;
     const size_t pre = (size_t)p.BH * p.n_seg * kBf16PerSeg * 2;
+    const size_t T_pad = (size_t)(p.T + 63) / 64 * 64;
+    const size_t kt = (size_t)p.BH * kD * T_pad * 2;
     p.ws_seg_state = 0;
     p.ws_total = up(seg);
     p.ws_extra = p.ws_total + up(tot);
-    p.ws_bytes = p.ws_extra + up(pre);
+    p.ws_aux = p.ws_extra + up(pre);
+    p.ws_bytes = p.ws_aux + up(kt);
 }
 
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
@@ -586,18 +767,36 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
     float *seg = reinterpret_cast<float *>(w + p.ws_seg_state);
     float *total = reinterpret_cast<float *>(w + p.ws_total);
     __nv_bfloat16 *prefix = reinterpret_cast<__nv_bfloat16 *>(w + p.ws_extra);
+    __nv_bfloat16 *kt = reinterpret_cast<__nv_bfloat16 *>(w + p.ws_aux);
     const bool want_state = state_out != nullptr;
     const int n_build = want_state ? p.n_seg : p.n_seg - 1;
     const long long BH = p.BH;
+    const int T_pad = (p.T + 63) / 64 * 64;
     int *status = device_status_ptr();
     if (!status) return cudaErrorUnknown;
 
     if (n_build > 0) {
-        ProfScope ps("tc_state_build_simt", st);
-        const long long grid = (long long)((kF32Rows + 31) / 32) * n_build * BH;
-        tc_state_build_simt<<<(unsigned)grid, 256, 0, st>>>(
-            static_cast<const __nv_bfloat16 *>(k), static_cast<const __nv_bfloat16 *>(v), seg, p.T,
-            p.L, p.n_seg, n_build);
+        {
+            ProfScope ps("tc_k_transpose", st);
+            k_transpose<<<(unsigned)((T_pad / 64) * BH), 256, 0, st>>>(
+                static_cast<const __nv_bfloat16 *>(k), kt, p.T, T_pad);
+        }
+        CUtensorMap mkt, mvb, mkb;
+        const uint64_t dkt[3] = {(uint64_t)T_pad, (uint64_t)kD, (uint64_t)BH};
+        const uint64_t skt[2] = {(uint64_t)T_pad * 2, (uint64_t)kD * T_pad * 2};
+        const uint32_t bkt[3] = {64, 64, 1};
+        const uint64_t dqkv[3] = {(uint64_t)kD, (uint64_t)p.T, (uint64_t)BH};
+        const uint64_t sqkv[2] = {(uint64_t)kD * 2, (uint64_t)p.T * kD * 2};
+        const uint32_t b64[3] = {64, 64, 1};
+        if (!make_tmap_bf16(&mkt, kt, 3, dkt, skt, bkt) || !make_tmap_bf16(&mvb, v, 3, dqkv, sqkv, b64) ||
+            !make_tmap_bf16(&mkb, k, 3, dqkv, sqkv, b64))
+            return cudaErrorInvalidValue;
+        cudaError_t e = cudaFuncSetAttribute(tc_build, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kBSmAlloc);
+        if (e != cudaSuccess) return e;
+        ProfScope ps("tc_build", st);
+        tc_build<<<(unsigned)(kBCtas * n_build * BH), kBuildThreads, kBSmAlloc, st>>>(
+            mkt, mvb, mkb, seg, p.T, p.L, p.n_seg, n_build, status);
     }
     if (p.n_seg > 1) {
         ProfScope ps("tc_seg_scan", st);
