@@ -21,17 +21,12 @@
 namespace kata {
 namespace sm100 {
 
-// Upper bound of any on-device wait before the kernel gives up (ns).
-constexpr uint64_t kWaitTimeoutNs = 4000000000ull;
+// Upper bound of any on-device wait before the kernel gives up, in SM clock
+// cycles (2^33 cycles: about 4.4 s at 1.965 GHz, longer at lower clocks).
+constexpr long long kWaitTimeoutCycles = 1ll << 33;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
 }
 
 // ---------------------------------------------------------------------------
@@ -72,18 +67,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for phase `parity` of `bar` to complete.  Gives up after
-// kWaitTimeoutNs, or as soon as *abort is set by another thread; on a time-out
-// it sets *abort itself.  Returns true when the phase completed.
+// Waits for phase `parity` of `bar` to complete.  Spins on try_wait; every
+// 1024 unsuccessful tries it checks *abort (set by another thread that gave
+// up) and the cycle budget kWaitTimeoutCycles, after which it sets *abort
+// itself.  Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    for (;;) {
+    const long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (globaltimer() - t0 > kWaitTimeoutNs) {
-            *abort = 1;
-            return false;
+        if ((it & 1023u) == 0) {
+            if (*abort) return false;
+            if (clock64() - t0 > kWaitTimeoutCycles) {
+                *abort = 1;
+                return false;
+            }
         }
     }
 }
@@ -216,6 +214,19 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
         "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
 

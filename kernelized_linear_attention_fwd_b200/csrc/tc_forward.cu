@@ -124,35 +124,46 @@ tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__r
 
 // ---------------------------------------------------------------------------
 // Readout kernel.
+//
+// A CTA owns 256 queries (two 128-query tiles) of one segment.  Roles:
+//   warps 0-3 / 4-7  phi(Q) generation, then squared-score masking and the
+//                    epilogue, for tile 0 / tile 1 (thread = query row)
+//   warp 8           TMA producer (Q, Z prefix, state-prefix stages, K/V blocks)
+//   warps 9, 10      MMA issuers.  In the inter phase they take alternate
+//                    stages (so one issuer's wait overlaps the other's queued
+//                    MMAs); in the intra phase issuer t serves query tile t.
+// Accumulators are zeroed by tcgen05.st before the first MMA, and every MMA
+// accumulates, so the order in which the two issuers' MMAs run is free.
 // ---------------------------------------------------------------------------
 constexpr int kQT = 128;                 // query tile (MMA M)
 constexpr int kTiles = 2;                // query tiles per CTA
 constexpr int kCtaQ = kQT * kTiles;      // 256 queries per CTA
 constexpr int kKB = 128;                 // key block
-constexpr int kRing = 4;                 // inter-term pipeline depth
-constexpr int kInterStages = kHalfStrips / 2;  // 80 stages of 2 half-strips
-constexpr int kGenWarps = 8;
+constexpr int kRHs = 4;                  // half-strips per inter stage (64 state rows)
+constexpr int kRStages = kHalfStrips / kRHs;  // 40
+constexpr int kRRing = 4;                // inter ring depth
 constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kReadThreads = 320;
+constexpr int kIssuer0 = 9;
+constexpr int kReadThreads = 352;
 
 // shared memory (from a 1024-byte aligned base)
 constexpr int kSmQ = 0;                          // 2 x [128 x 64] bf16, K-major, swizzled
 constexpr int kSmZ = kSmQ + kTiles * 16384;      // Z hi [64 x 64], Z lo [64 x 64]
-constexpr int kSmS = kSmZ + 16384;               // ring of [32 x 64] state tiles
-constexpr int kSmK = kSmS + kRing * 4096;        // 2 x [128 x 64] keys
+constexpr int kSmS = kSmZ + 16384;               // ring of [64 x 64] state-prefix tiles
+constexpr int kSmK = kSmS + kRRing * 8192;       // 2 x [128 x 64] keys
 constexpr int kSmV = kSmK + 2 * 16384;           // 2 x [128 x 64] values
 constexpr int kSmBytes = kSmV + 2 * 16384;
 constexpr int kSmAlloc = kSmBytes + 1024;
 
 // tensor memory columns (512 allocated)
-constexpr uint32_t kTmO = 0;     // O[g]: 64 columns at 64 g
-constexpr uint32_t kTmS = 128;   // scores S[g]: 128 columns at 128 + 128 g (U[g] first)
-constexpr uint32_t kTmA = 384;   // phi(Q) stages / P[g]: 64 columns at 384 + 64 g
+constexpr uint32_t kTmO = 0;     // O[t]: 64 columns at 64 t
+constexpr uint32_t kTmA = 128;   // inter stages: 64 columns at 128 + 64 s (tile t at + 32 t)
+constexpr uint32_t kTmS = 128;   // intra scores S[t]: 128 columns at 128 + 128 t (after the inter phase)
+constexpr uint32_t kTmP = 384;   // U[t] (first) and P[t]: 64 columns at 384 + 64 t
 
 struct ReadBars {
-    uint64_t q, u, o;
-    uint64_t bfull[kRing], bempty[kRing], afull[kRing], aempty[kRing];
+    uint64_t q, u, interdone, o;
+    uint64_t bfull[kRRing], bempty[kRRing], afull[kRRing], aempty[kRRing];
     uint64_t kvfull[2], kvempty[2];
     uint64_t sfull[kTiles], pfull[kTiles];
 };
@@ -185,30 +196,27 @@ __device__ __forceinline__ void gen_halfstrip(const uint32_t (&q2)[32], uint32_t
 }
 
 template <int ST>
-__device__ __forceinline__ void gen_stage(const uint32_t (&q2)[32], uint32_t *a) {
-    gen_halfstrip<2 * ST>(q2, a);
-    gen_halfstrip<2 * ST + 1>(q2, a + 8);
-}
-
-template <int ST>
 struct GenLoop {
     __device__ __forceinline__ static bool run(const uint32_t (&q2)[32], ReadBars &bars,
-                                               uint32_t ta_base, volatile int *abort) {
-        constexpr int stage = ST % kRing;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[stage], ((ST / kRing) & 1) ^ 1, abort)))
+                                               uint32_t ta_tile, volatile int *abort) {
+        constexpr int s = ST % kRRing;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[s], ((ST / kRRing) & 1) ^ 1, abort)))
             return false;
         tc_fence_after();
-        uint32_t a[16];
-        gen_stage<ST>(q2, a);
-        tmem_st16(ta_base + 16 * stage, a);
+        uint32_t a[32];
+        gen_halfstrip<kRHs * ST + 0>(q2, a);
+        gen_halfstrip<kRHs * ST + 1>(q2, a + 8);
+        gen_halfstrip<kRHs * ST + 2>(q2, a + 16);
+        gen_halfstrip<kRHs * ST + 3>(q2, a + 24);
+        tmem_st32(ta_tile + 64 * s, a);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars.afull[stage]);
-        return GenLoop<ST + 1>::run(q2, bars, ta_base, abort);
+        mbar_arrive(&bars.afull[s]);
+        return GenLoop<ST + 1>::run(q2, bars, ta_tile, abort);
     }
 };
 template <>
-struct GenLoop<kInterStages> {
+struct GenLoop<kRStages> {
     __device__ __forceinline__ static bool run(const uint32_t (&)[32], ReadBars &, uint32_t,
                                                volatile int *) {
         return true;
@@ -224,6 +232,9 @@ __device__ __forceinline__ void set_timeout_status(int *status) {
     atomicCAS(status, 0, (int)KATA_ERR_TIMEOUT);
 }
 
+// Start address of a descriptor advanced by `bytes` (16-byte units in the low bits).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 // ---------------------------------------------------------------------------
 // Keys transposed per head: kt[bh][d][t] (tokens contiguous), zero-padded to
 // T_pad (a multiple of 64), so the state builder can read, for a feature
@@ -232,24 +243,33 @@ __device__ __forceinline__ void set_timeout_status(int *status) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 k_transpose(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ kt, int T, int T_pad) {
-    __shared__ uint16_t tile[64][66];
+    __shared__ uint16_t tile[64][72];  // [token][d], rows padded to 144 B
     const int n_tt = T_pad / 64;
     const long long bh = blockIdx.x / n_tt;
     const int t0 = (blockIdx.x % n_tt) * 64;
-    const uint32_t *src = reinterpret_cast<const uint32_t *>(k);
-    for (int x = threadIdx.x; x < 64 * 32; x += 256) {
-        const int s = x / 32, c2 = x % 32, t = t0 + s;
-        const uint32_t w = t < T ? src[((bh * T + t) * kD) / 2 + c2] : 0u;
-        tile[s][2 * c2] = static_cast<uint16_t>(w & 0xFFFFu);
-        tile[s][2 * c2 + 1] = static_cast<uint16_t>(w >> 16);
+    const uint4 *src = reinterpret_cast<const uint4 *>(k);
+    uint4 in[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {  // 64 tokens x 8 chunks of 8 values
+        const int x = threadIdx.x + 256 * r, s = x / 8, c8 = x % 8, t = t0 + s;
+        in[r] = t < T ? src[((bh * T + t) * kD) / 8 + c8] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int x = threadIdx.x + 256 * r, s = x / 8, c8 = x % 8;
+        *reinterpret_cast<uint4 *>(&tile[s][8 * c8]) = in[r];
     }
     __syncthreads();
-    uint32_t *dst = reinterpret_cast<uint32_t *>(kt);
-    for (int x = threadIdx.x; x < 64 * 32; x += 256) {
-        const int d = x / 32, s2 = x % 32;
-        const uint32_t w = static_cast<uint32_t>(tile[2 * s2][d]) |
-                           (static_cast<uint32_t>(tile[2 * s2 + 1][d]) << 16);
-        dst[((bh * kD + d) * T_pad + t0) / 2 + s2] = w;
+    uint4 *dst = reinterpret_cast<uint4 *>(kt);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {  // 64 features x 8 runs of 8 tokens
+        const int x = threadIdx.x + 256 * r, d = x / 8, s8 = x % 8;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            w[e] = static_cast<uint32_t>(tile[8 * s8 + 2 * e][d]) |
+                   (static_cast<uint32_t>(tile[8 * s8 + 2 * e + 1][d]) << 16);
+        dst[((bh * kD + d) * T_pad + t0) / 8 + s8] = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -264,23 +284,26 @@ k_transpose(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ kt,
 // memory.  CTA 0 adds a fifth tile, Z = K^T K (A rows k_i for lanes 0..63, B
 // the key tile itself).  Each thread reads its own key column k_j once per 16
 // tokens and the broadcast column k_i once per tile.
-// Two generation warpgroups take alternate 16-token steps.
+// Roles: warps 0-3 / 4-7 generate the first / second 16-token step of every
+// 32-token stage; warp 8 is the TMA producer; warps 9 and 10 issue the MMAs of
+// alternate stages.  Accumulators are zeroed by tcgen05.st first and every
+// MMA accumulates.
 // ---------------------------------------------------------------------------
 constexpr int kBCtas = 5;
 constexpr int kBTiles = 4;
-constexpr int kBRing = 4;                 // A stages, one 16-token step each
-constexpr int kBTok = 64;                 // tokens per TMA tile
+constexpr int kBTok = 64;                 // tokens per TMA tile (2 stages)
 constexpr int kBTileRing = 4;
 constexpr int kBStageBytes = 3 * 8192;    // K^T, V, K tiles
 constexpr int kBSmAlloc = kBTileRing * kBStageBytes + 1024 + 16384;  // padded: one CTA per SM
 constexpr int kBTmaWarp = 8;
-constexpr int kBMmaWarp = 9;
-constexpr int kBuildThreads = 320;
-constexpr uint32_t kBTmA = 320;           // A[stage][m] at 320 + 40 stage + 8 m
+constexpr int kBIssuer0 = 9;
+constexpr int kBuildThreads = 352;
+constexpr uint32_t kBTmZ = 256;           // Z accumulator (CTA 0)
+constexpr uint32_t kBTmA = 320;           // A ring: slot s at 320 + 80 s, step kk at + 40 kk
 
 struct BuildBars {
     uint64_t tfull[kBTileRing], tempty[kBTileRing];
-    uint64_t afull[kBRing], aempty[kBRing];
+    uint64_t afull[2], aempty[2];
     uint64_t done;
 };
 
@@ -300,26 +323,25 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
     const int g = rest % n_build;
     const int bh = rest / n_build;
     const bool zc = c == 0;
-    const int nm = kBTiles + (zc ? 1 : 0);
     const int s0 = g * L;
     const int ntok = min(L, T - s0);
     const int n_tt = (ntok + kBTok - 1) / kBTok;
-    const int n_ks = 4 * n_tt;
+    const int n_st = 2 * n_tt;               // 32-token stages
 
     if (tid == 0) {
         abort_flag = 0;
         for (int x = 0; x < kBTileRing; ++x) {
             mbar_init(&bars.tfull[x], 1);
-            mbar_init(&bars.tempty[x], 1);
+            mbar_init(&bars.tempty[x], 2);
         }
-        for (int x = 0; x < kBRing; ++x) {
-            mbar_init(&bars.afull[x], 128);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bars.afull[x], 256);
             mbar_init(&bars.aempty[x], 1);
         }
-        mbar_init(&bars.done, 1);
+        mbar_init(&bars.done, 2);
         fence_mbarrier_init();
     }
-    if (warp == kBMmaWarp) {
+    if (warp == kBIssuer0) {
         tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
@@ -348,25 +370,30 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             for (int t = (issued > kBTileRing ? issued - kBTileRing : 0); t < issued; ++t)
                 mbar_wait(&bars.tfull[t % kBTileRing], (t / kBTileRing) & 1, abort);
         }
-    } else if (warp == kBMmaWarp) {
+    } else if (warp == kBIssuer0 || warp == kBIssuer0 + 1) {
         if (lane == 0) {
+            const int me = warp - kBIssuer0;
             const uint32_t idesc = idesc_bf16(128, 64, 0, 1);
-            const uint32_t sbase = smem_u32(sm);
+            const uint64_t d0 = desc_sw128(smem_u32(sm), 8192, 1024);
             bool ok = true;
-            for (int step = 0; step < n_ks && ok; ++step) {
-                const int t = step / 4, kk = step % 4, b = t % kBTileRing, a = step % kBRing;
-                if (kk == 0) ok = mbar_wait(&bars.tfull[b], (t / kBTileRing) & 1, abort);
-                ok = ok && mbar_wait(&bars.afull[a], (step / kBRing) & 1, abort);
+            for (int st = me; st < n_st && ok; st += 2) {
+                const int t = st / 2, half = st % 2, b = t % kBTileRing;
+                ok = mbar_wait(&bars.tfull[b], (t / kBTileRing) & 1, abort) &&
+                     mbar_wait(&bars.afull[me], (st / 2) & 1, abort);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t stb = sbase + b * kBStageBytes;
-                for (int m = 0; m < nm; ++m) {
-                    const uint32_t bsrc = stb + (m == kBTiles ? 16384 : 8192) + 2048 * kk;
-                    mma_ts(tm + 64 * m, tm + kBTmA + 40 * a + 8 * m, desc_sw128(bsrc, 8192, 1024),
-                           idesc, step > 0 ? 1u : 0u);
+                const uint64_t dv = desc_add(d0, b * kBStageBytes + 8192 + 4096 * half);
+                const uint64_t dk = desc_add(d0, b * kBStageBytes + 16384 + 4096 * half);
+                const uint32_t ta = tm + kBTmA + 80 * me;
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+#pragma unroll
+                    for (int m = 0; m < kBTiles; ++m)
+                        mma_ts(tm + 64 * m, ta + 40 * kk + 8 * m, desc_add(dv, 2048 * kk), idesc, 1);
+                    if (zc) mma_ts(tm + kBTmZ, ta + 40 * kk + 32, desc_add(dk, 2048 * kk), idesc, 1);
                 }
-                mma_commit(&bars.aempty[a]);
-                if (kk == 3) mma_commit(&bars.tempty[b]);
+                mma_commit(&bars.aempty[me]);
+                mma_commit(&bars.tempty[b]);
             }
             mma_commit(&bars.done);
             mbar_wait(&bars.done, 0, abort);
@@ -380,15 +407,22 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
 #pragma unroll
         for (int m = 0; m < kBTiles; ++m) im[m] = hs_i(32 * c + 8 * m + slot);
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+        {   // zero the accumulators (warpgroup 0: columns 0..159, warpgroup 1: 160..319)
+            uint32_t z[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) z[x] = 0u;
+#pragma unroll
+            for (int x = 0; x < 5; ++x) tmem_st32(tm + 160 * wg + 32 * x + lane_base, z);
+        }
         bool ok = true;
-        for (int step = wg; step < n_ks && ok; step += 2) {
-            const int t = step / 4, kk = step % 4, b = t % kBTileRing, a = step % kBRing;
+        for (int st = 0; st < n_st && ok; ++st) {
+            const int t = st / 2, half = st % 2, b = t % kBTileRing, a = st % 2;
             ok = __all_sync(0xffffffffu, mbar_wait(&bars.tfull[b], (t / kBTileRing) & 1, abort) &&
-                                             mbar_wait(&bars.aempty[a], ((step / kBRing) & 1) ^ 1, abort));
+                                             mbar_wait(&bars.aempty[a], ((st / 2) & 1) ^ 1, abort));
             if (!ok) break;
             tc_fence_after();
             const uint8_t *kt = sm + b * kBStageBytes;  // row d: 64 tokens, swizzled
-            const int c0 = 2 * kk, c1 = 2 * kk + 1;
+            const int c0 = 4 * half + 2 * wg, c1 = c0 + 1;  // this warpgroup's 16 tokens
             uint32_t own[8];
             {
                 const uint8_t *r = kt + j * 128;
@@ -397,34 +431,34 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
                 own[0] = x0.x; own[1] = x0.y; own[2] = x0.z; own[3] = x0.w;
                 own[4] = x1.x; own[5] = x1.y; own[6] = x1.z; own[7] = x1.w;
             }
-            const uint32_t ta = tm + kBTmA + 40 * a + lane_base;
+            const uint32_t ta = tm + kBTmA + 80 * a + 40 * wg + lane_base;
+            uint32_t p[32];
 #pragma unroll
             for (int m = 0; m < kBTiles; ++m) {
                 const int i = im[m];
                 const uint8_t *r = kt + i * 128;
                 const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (i & 7)) * 16));
                 const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (i & 7)) * 16));
-                uint32_t p[8];
-                p[0] = mul_bf16x2(own[0], x0.x); p[1] = mul_bf16x2(own[1], x0.y);
-                p[2] = mul_bf16x2(own[2], x0.z); p[3] = mul_bf16x2(own[3], x0.w);
-                p[4] = mul_bf16x2(own[4], x1.x); p[5] = mul_bf16x2(own[5], x1.y);
-                p[6] = mul_bf16x2(own[6], x1.z); p[7] = mul_bf16x2(own[7], x1.w);
-                tmem_st8(ta + 8 * m, p);
+                p[8 * m + 0] = mul_bf16x2(own[0], x0.x); p[8 * m + 1] = mul_bf16x2(own[1], x0.y);
+                p[8 * m + 2] = mul_bf16x2(own[2], x0.z); p[8 * m + 3] = mul_bf16x2(own[3], x0.w);
+                p[8 * m + 4] = mul_bf16x2(own[4], x1.x); p[8 * m + 5] = mul_bf16x2(own[5], x1.y);
+                p[8 * m + 6] = mul_bf16x2(own[6], x1.z); p[8 * m + 7] = mul_bf16x2(own[7], x1.w);
             }
+            tmem_st32(ta, p);
             if (zc) {
                 // Z tile: lane i < 64 holds k_i over the tokens, lanes 64.. hold zero
-                uint32_t p[8];
+                uint32_t zz[8];
                 if (row < kD) {
                     const uint8_t *r = kt + row * 128;
                     const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (row & 7)) * 16));
                     const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (row & 7)) * 16));
-                    p[0] = x0.x; p[1] = x0.y; p[2] = x0.z; p[3] = x0.w;
-                    p[4] = x1.x; p[5] = x1.y; p[6] = x1.z; p[7] = x1.w;
+                    zz[0] = x0.x; zz[1] = x0.y; zz[2] = x0.z; zz[3] = x0.w;
+                    zz[4] = x1.x; zz[5] = x1.y; zz[6] = x1.z; zz[7] = x1.w;
                 } else {
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) p[x] = 0u;
+                    for (int x = 0; x < 8; ++x) zz[x] = 0u;
                 }
-                tmem_st8(ta + 8 * kBTiles, p);
+                tmem_st8(ta + 32, zz);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -444,11 +478,11 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
                 else
                     dst = base + ((long long)16 * (32 * c + 8 * mm + slot) + jj) * kD;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tm + 64 * mm + lane_base + 32 * half, o);
+                for (int hh = 0; hh < 2; ++hh) {
+                    tmem_ld32(tm + 64 * mm + lane_base + 32 * hh, o);
                     tmem_ld_wait();
                     if (mm != kBTiles || row < kD) {
-                        float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * half);
+                        float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * hh);
 #pragma unroll
                         for (int x = 0; x < 8; ++x)
                             d4[x] = make_float4(__uint_as_float(o[4 * x]), __uint_as_float(o[4 * x + 1]),
@@ -462,7 +496,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
 
     tc_fence_before();
     __syncthreads();
-    if (warp == kBMmaWarp) tmem_dealloc(tm, 512);
+    if (warp == kBIssuer0) tmem_dealloc(tm, 512);
     if (tid == 0 && abort_flag) set_timeout_status(status);
 }
 
@@ -489,24 +523,25 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         abort_flag = 0;
         mbar_init(&bars.q, 1);
         mbar_init(&bars.u, 1);
-        mbar_init(&bars.o, 1);
-        for (int s = 0; s < kRing; ++s) {
+        mbar_init(&bars.interdone, 2);
+        mbar_init(&bars.o, 2);
+        for (int s = 0; s < kRRing; ++s) {
             mbar_init(&bars.bfull[s], 1);
             mbar_init(&bars.bempty[s], 1);
-            mbar_init(&bars.afull[s], kGenWarps * 32);
+            mbar_init(&bars.afull[s], 8 * 32);
             mbar_init(&bars.aempty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bars.kvfull[s], 1);
-            mbar_init(&bars.kvempty[s], 1);
+            mbar_init(&bars.kvempty[s], 2);
         }
-        for (int s = 0; s < kTiles; ++s) {
-            mbar_init(&bars.sfull[s], 1);
-            mbar_init(&bars.pfull[s], 4 * 32);
+        for (int t = 0; t < kTiles; ++t) {
+            mbar_init(&bars.sfull[t], 1);
+            mbar_init(&bars.pfull[t], 4 * 32);
         }
         fence_mbarrier_init();
     }
-    if (warp == kMmaWarp) {
+    if (warp == kIssuer0) {
         tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
     }
@@ -524,24 +559,21 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_s);
             mbar_arrive_expect_tx(&bars.q, kTiles * 16384 + (inter ? 16384 : 0));
-            for (int tl = 0; tl < kTiles; ++tl)
-                tma_load_3d(sm + kSmQ + tl * 16384, &tm_q, &bars.q, 0, t0 + tl * kQT, bh);
-            if (inter) {
+            for (int t = 0; t < kTiles; ++t)
+                tma_load_3d(sm + kSmQ + t * 16384, &tm_q, &bars.q, 0, t0 + t * kQT, bh);
+            if (inter)
                 for (int zz = 0; zz < 4; ++zz)  // Z hi rows 2560..2623, Z lo rows 2624..2687
-                    tma_load_3d(sm + kSmZ + zz * 4096, &tm_s, &bars.q, 0, kZHiRow0 + 32 * zz,
-                                sidx);
-            }
+                    tma_load_3d(sm + kSmZ + zz * 4096, &tm_s, &bars.q, 0, kZHiRow0 + 32 * zz, sidx);
             int issued_b = 0, issued_kv = 0;
             bool ok = true;
-            if (inter) {
-                for (int st = 0; st < kInterStages && ok; ++st) {
-                    const int s = st % kRing;
-                    ok = mbar_wait(&bars.bempty[s], ((st / kRing) & 1) ^ 1, abort);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&bars.bfull[s], 4096);
-                    tma_load_3d(sm + kSmS + s * 4096, &tm_s, &bars.bfull[s], 0, 32 * st, sidx);
-                    ++issued_b;
-                }
+            for (int st = 0; inter && st < kRStages && ok; ++st) {
+                const int s = st % kRRing;
+                ok = mbar_wait(&bars.bempty[s], ((st / kRRing) & 1) ^ 1, abort);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&bars.bfull[s], 8192);
+                tma_load_3d(sm + kSmS + s * 8192, &tm_s, &bars.bfull[s], 0, 64 * st, sidx);
+                tma_load_3d(sm + kSmS + s * 8192 + 4096, &tm_s, &bars.bfull[s], 0, 64 * st + 32, sidx);
+                ++issued_b;
             }
             for (int kb = 0; kb < n_kb && ok; ++kb) {
                 const int s = kb & 1;
@@ -554,72 +586,83 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             }
             // drain: every load issued must have landed before the CTA exits
             mbar_wait(&bars.q, 0, abort);
-            for (int st = (issued_b > kRing ? issued_b - kRing : 0); st < issued_b; ++st)
-                mbar_wait(&bars.bfull[st % kRing], (st / kRing) & 1, abort);
+            for (int st = (issued_b > kRRing ? issued_b - kRRing : 0); st < issued_b; ++st)
+                mbar_wait(&bars.bfull[st % kRRing], (st / kRRing) & 1, abort);
             for (int kb = (issued_kv > 2 ? issued_kv - 2 : 0); kb < issued_kv; ++kb)
                 mbar_wait(&bars.kvfull[kb & 1], (kb >> 1) & 1, abort);
         }
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ MMA issue
+    } else if (warp == kIssuer0 || warp == kIssuer0 + 1) {
+        // ------------------------------------------------------------ MMA issuers
         if (lane == 0) {
+            const int me = warp - kIssuer0;
             const uint32_t id_qk = idesc_bf16(kQT, kKB, 0, 0);
             const uint32_t id_n64 = idesc_bf16(kQT, 64, 0, 1);
-            const uint32_t sQ = smem_u32(sm + kSmQ), sZ = smem_u32(sm + kSmZ);
-            const uint32_t sS = smem_u32(sm + kSmS), sK = smem_u32(sm + kSmK),
-                           sV = smem_u32(sm + kSmV);
+            const uint64_t dQ0 = desc_sw128(smem_u32(sm + kSmQ), 16, 1024);
+            const uint64_t dZ = desc_sw128(smem_u32(sm + kSmZ), 8192, 1024);
+            const uint64_t dS = desc_sw128(smem_u32(sm + kSmS), 8192, 1024);
+            const uint64_t dK = desc_sw128(smem_u32(sm + kSmK), 16, 1024);
+            const uint64_t dV = desc_sw128(smem_u32(sm + kSmV), 8192, 1024);
             bool ok = mbar_wait(&bars.q, 0, abort);
-            bool acc_o[kTiles] = {false, false};
             if (ok) tc_fence_after();
             if (ok && inter) {
-                for (int tl = 0; tl < kTiles; ++tl) {
-                    const uint32_t dU = tm + kTmS + 128 * tl;
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_ss(dU, desc_sw128(sQ + tl * 16384 + 32 * ks, 16, 1024),
-                               desc_sw128(sZ + 2048 * ks, 8192, 1024), id_n64, ks > 0);
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_ss(dU, desc_sw128(sQ + tl * 16384 + 32 * ks, 16, 1024),
-                               desc_sw128(sZ + 8192 + 2048 * ks, 8192, 1024), id_n64, 1);
+                if (me == 0) {
+                    for (int t = 0; t < kTiles; ++t) {
+                        const uint32_t dU = tm + kTmP + 64 * t;
+                        const uint64_t dq = desc_add(dQ0, t * 16384);
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_ss(dU, desc_add(dq, 32 * ks), desc_add(dZ, 2048 * ks), id_n64, ks > 0);
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_ss(dU, desc_add(dq, 32 * ks), desc_add(dZ, 8192 + 2048 * ks), id_n64, 1);
+                    }
+                    mma_commit(&bars.u);
                 }
-                mma_commit(&bars.u);
-                for (int st = 0; st < kInterStages && ok; ++st) {
-                    const int s = st % kRing;
-                    const uint32_t ph = (st / kRing) & 1;
+                for (int st = me; st < kRStages && ok; st += 2) {
+                    const int s = st % kRRing;
+                    const uint32_t ph = (st / kRRing) & 1;
                     ok = mbar_wait(&bars.bfull[s], ph, abort) && mbar_wait(&bars.afull[s], ph, abort);
                     if (!ok) break;
                     tc_fence_after();
-                    for (int tl = 0; tl < kTiles; ++tl)
-                        for (int ks = 0; ks < 2; ++ks)
-                            mma_ts(tm + kTmO + 64 * tl, tm + kTmA + 64 * tl + 16 * s + 8 * ks,
-                                   desc_sw128(sS + s * 4096 + 2048 * ks, 8192, 1024), id_n64,
-                                   (st | ks) > 0);
+                    const uint32_t ta = tm + kTmA + 64 * s;
+                    const uint64_t db = desc_add(dS, 8192 * s);
+#pragma unroll
+                    for (int ks = 0; ks < kRHs; ++ks) {
+                        mma_ts(tm + kTmO, ta + 8 * ks, desc_add(db, 2048 * ks), id_n64, 1);
+                        mma_ts(tm + kTmO + 64, ta + 32 + 8 * ks, desc_add(db, 2048 * ks), id_n64, 1);
+                    }
                     mma_commit(&bars.bempty[s]);
                     mma_commit(&bars.aempty[s]);
                 }
-                acc_o[0] = acc_o[1] = true;
+                mma_commit(&bars.interdone);
+                // scores reuse the inter stage columns: every inter MMA must be done
+                ok = ok && mbar_wait(&bars.interdone, 0, abort);
+                if (ok) tc_fence_after();
             }
+            // intra phase: issuer `me` serves query tile `me`
+            const int t = me;
+            const uint64_t dq = desc_add(dQ0, t * 16384);
             for (int kb = 0; kb < n_kb && ok; ++kb) {
                 const int s = kb & 1;
                 ok = mbar_wait(&bars.kvfull[s], (kb >> 1) & 1, abort);
                 if (!ok) break;
                 tc_fence_after();
                 const int kbs = seg0 + kb * kKB;
-                for (int tl = 0; tl < kTiles; ++tl) {
-                    if (kbs >= t0 + tl * kQT + kQT) continue;  // block entirely after the tile
+                if (kbs < t0 + t * kQT + kQT) {  // block not entirely after the tile
+                    const uint64_t dk = desc_add(dK, 16384 * s);
+#pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        mma_ss(tm + kTmS + 128 * tl, desc_sw128(sQ + tl * 16384 + 32 * ks, 16, 1024),
-                               desc_sw128(sK + s * 16384 + 32 * ks, 16, 1024), id_qk, ks > 0);
-                    mma_commit(&bars.sfull[tl]);
-                }
-                for (int tl = 0; tl < kTiles && ok; ++tl) {
-                    if (kbs >= t0 + tl * kQT + kQT) continue;
-                    ok = mbar_wait(&bars.pfull[tl], kb & 1, abort);
+                        mma_ss(tm + kTmS + 128 * t, desc_add(dq, 32 * ks), desc_add(dk, 32 * ks), id_qk,
+                               ks > 0);
+                    mma_commit(&bars.sfull[t]);
+                    ok = mbar_wait(&bars.pfull[t], kb & 1, abort);
                     if (!ok) break;
                     tc_fence_after();
+                    const uint64_t dv = desc_add(dV, 16384 * s);
+#pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        mma_ts(tm + kTmO + 64 * tl, tm + kTmA + 64 * tl + 8 * ks,
-                               desc_sw128(sV + s * 16384 + 2048 * ks, 8192, 1024), id_n64,
-                               (acc_o[tl] || ks > 0) ? 1u : 0u);
-                    acc_o[tl] = true;
+                        mma_ts(tm + kTmO + 64 * t, tm + kTmP + 64 * t + 8 * ks, desc_add(dv, 2048 * ks),
+                               id_n64, 1);
                 }
                 mma_commit(&bars.kvempty[s]);
             }
@@ -627,15 +670,23 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             mbar_wait(&bars.o, 0, abort);  // drain before the CTA may free tensor memory
         }
     } else {
-        // ------------------------------------------------------------ generation / softmax
-        const int tl = warp / 4, qd = warp % 4;
+        // ------------------------------------------------------------ generation / scores / epilogue
+        const int t = warp / 4, qd = warp % 4;
         const int row = 32 * qd + lane;
-        const int tq = t0 + tl * kQT + row;
+        const int tq = t0 + t * kQT + row;
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+        // zero this thread's accumulator row; every MMA accumulates
+        {
+            uint32_t z[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) z[x] = 0u;
+            tmem_st32(tm + kTmO + 64 * t + lane_base, z);
+            tmem_st32(tm + kTmO + 64 * t + 32 + lane_base, z);
+        }
         bool ok = __all_sync(0xffffffffu, mbar_wait(&bars.q, 0, abort));
         uint32_t q2[32];
         {
-            const uint8_t *qrow = sm + kSmQ + tl * 16384 + row * 128;
+            const uint8_t *qrow = sm + kSmQ + t * 16384 + row * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 const uint4 x = *reinterpret_cast<const uint4 *>(qrow + ((c ^ (row & 7)) * 16));
@@ -653,26 +704,29 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                 uint32_t u[32];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tm + kTmS + 128 * tl + lane_base + 32 * half, u);
+                    tmem_ld32(tm + kTmP + 64 * t + lane_base + 32 * half, u);
                     tmem_ld_wait();
 #pragma unroll
                     for (int x = 0; x < 16; ++x) {
                         const uint32_t w = q2[16 * half + x];
                         den_inter = fmaf(__uint_as_float(w << 16), __uint_as_float(u[2 * x]), den_inter);
-                        den_inter = fmaf(__uint_as_float(w & 0xFFFF0000u),
-                                         __uint_as_float(u[2 * x + 1]), den_inter);
+                        den_inter = fmaf(__uint_as_float(w & 0xFFFF0000u), __uint_as_float(u[2 * x + 1]),
+                                         den_inter);
                     }
                 }
-                ok = GenLoop<0>::run(q2, bars, tm + kTmA + 64 * tl + lane_base, abort);
+                ok = GenLoop<0>::run(q2, bars, tm + kTmA + 32 * t + lane_base, abort);
             }
+        } else {
+            tmem_st_wait();  // the zeroed accumulator is ordered before the first P hand-off
+            tc_fence_before();
         }
         float l = 0.f;
-        const uint32_t tS = tm + kTmS + 128 * tl + lane_base;
-        const uint32_t tP = tm + kTmA + 64 * tl + lane_base;
+        const uint32_t tS = tm + kTmS + 128 * t + lane_base;
+        const uint32_t tP = tm + kTmP + 64 * t + lane_base;
         for (int kb = 0; kb < n_kb && ok; ++kb) {
             const int kbs = seg0 + kb * kKB;
-            if (kbs >= t0 + tl * kQT + kQT) continue;
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfull[tl], kb & 1, abort));
+            if (kbs >= t0 + t * kQT + kQT) continue;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfull[t], kb & 1, abort));
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -693,7 +747,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&bars.pfull[tl]);
+            mbar_arrive(&bars.pfull[t]);
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.o, 0, abort));
         if (ok) {
@@ -704,7 +758,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             uint4 *dst = reinterpret_cast<uint4 *>(out + ((long long)bh * T + tq) * kD);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                tmem_ld32(tm + kTmO + 64 * tl + lane_base + 32 * half, o);
+                tmem_ld32(tm + kTmO + 64 * t + lane_base + 32 * half, o);
                 tmem_ld_wait();
                 if (tq < T) {
 #pragma unroll
@@ -723,7 +777,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
 
     tc_fence_before();
     __syncthreads();
-    if (warp == kMmaWarp) tmem_dealloc(tm, 512);
+    if (warp == kIssuer0) tmem_dealloc(tm, 512);
     if (tid == 0 && abort_flag) set_timeout_status(status);
 }
 
