@@ -33,69 +33,94 @@ constexpr long long kF32PerSeg = (long long)kF32Rows * kD;    // 167,936 floats
 constexpr long long kBf16PerSeg = (long long)kBf16Rows * kD;  // 172,032 bf16
 
 // ---------------------------------------------------------------------------
-// Exclusive prefix over segments -> bf16 copy (+ Z split into hi and lo), and
-// the fp32 total.  Same scheme as seg_scan: 32-segment x 32-element tiles
-// through shared memory, Kogge-Stone shuffle scan down each element column.
-// grid.x = element-tile + n_et * bh; block (32, 8)
+// Exclusive prefix over segments (the associative scan across chunk states)
+// -> bf16 copy for the readout (Z split into hi and lo parts), and the fp32
+// total.  Reduce-then-scan per block of 128 consecutive elements of one head
+// (32 lanes x float4): warp w takes a run of kScanRun consecutive segments,
+// holds them in registers and forms their running sums; the 8 run totals are
+// scanned across warps in shared memory in log2(8) = 3 steps; each warp adds
+// its offset and writes its run.  Every global access is a coalesced 16-byte
+// (fp32) or 8-byte (bf16) vector per lane.
+// grid.x = element-block + n_eb * bh; block 256.
 // ---------------------------------------------------------------------------
+constexpr int kScanWarps = 8;
+constexpr int kScanRun = 16;
+
+__device__ __forceinline__ float4 f4add(float4 a, float4 b) {
+    return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
 __global__ void __launch_bounds__(256)
 tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ prefix,
             float *__restrict__ total, int n_seg, int n_valid) {
-    __shared__ float tile[32][33];
-    const int lane = threadIdx.x, w = threadIdx.y;
+    __shared__ float4 part[2][kScanWarps][32];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     constexpr long long E = kF32PerSeg;
-    constexpr long long n_et = E / 32;
-    const long long et = blockIdx.x % n_et;
-    const long long bh = blockIdx.x / n_et;
-    const long long e_base = et * 32;
-    const float *base = seg_state + bh * (long long)n_seg * E;
+    constexpr long long n_eb = E / 128;
+    const long long eb = blockIdx.x % n_eb;
+    const long long bh = blockIdx.x / n_eb;
+    const long long e0 = eb * 128 + 4 * lane;
+    const float *base = seg_state + bh * (long long)n_seg * E + e0;
     __nv_bfloat16 *pbase = prefix + bh * (long long)n_seg * kBf16PerSeg;
-    float carry[4] = {0.f, 0.f, 0.f, 0.f};
-    const bool z_tile = e_base >= (long long)kStateRows * kD;
+    const bool z_part = e0 >= (long long)kStateRows * kD;
+    const long long z = e0 - (long long)kStateRows * kD;
+    float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
 
-    for (int g0 = 0; g0 < n_seg; g0 += 32) {
+    for (int g0 = 0; g0 < n_seg; g0 += kScanWarps * kScanRun) {
+        const int gw = g0 + w * kScanRun;
+        float4 v[kScanRun];
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-            const int gs = w + 8 * rr, g = g0 + gs;
-            tile[gs][lane] = g < n_valid ? base[(long long)g * E + e_base + lane] : 0.f;
+        for (int i = 0; i < kScanRun; ++i)
+            v[i] = gw + i < n_valid ? *reinterpret_cast<const float4 *>(base + (long long)(gw + i) * E)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < kScanRun; ++i) {  // exclusive running sum within the run
+            const float4 x = v[i];
+            v[i] = run;
+            run = f4add(run, x);
         }
+        // inclusive Kogge-Stone scan of the 8 run totals across warps
+        int buf = 0;
+        part[0][w][lane] = run;
         __syncthreads();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            const int c = w + 8 * cc;
-            const float x = tile[lane][c];
-            float inc = x;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, inc, off);
-                if (lane >= off) inc += y;
-            }
-            tile[lane][c] = carry[cc] + (inc - x);
-            carry[cc] += __shfl_sync(0xffffffffu, inc, 31);
+        for (int off = 1; off < kScanWarps; off <<= 1) {
+            float4 x = part[buf][w][lane];
+            if (w >= off) x = f4add(x, part[buf][w - off][lane]);
+            part[buf ^ 1][w][lane] = x;
+            buf ^= 1;
+            __syncthreads();
         }
-        __syncthreads();
+        const float4 incl = part[buf][w][lane];
+        const float4 all = part[buf][kScanWarps - 1][lane];
+        const float4 off = f4add(carry, make_float4(incl.x - run.x, incl.y - run.y, incl.z - run.z,
+                                                    incl.w - run.w));
+        carry = f4add(carry, all);
+        __syncthreads();  // part is rewritten by the next pass
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr) {
-            const int gs = w + 8 * rr, g = g0 + gs;
+        for (int i = 0; i < kScanRun; ++i) {
+            const int g = gw + i;
             if (g < 1 || g >= n_seg) continue;  // segment 0 has an empty prefix
-            const float p = tile[gs][lane];
+            const float4 p = f4add(v[i], off);
             __nv_bfloat16 *dst = pbase + (long long)g * kBf16PerSeg;
-            if (!z_tile) {
-                dst[e_base + lane] = __float2bfloat16_rn(p);
+            if (!z_part) {
+                uint2 o;
+                o.x = pack_bf16x2(p.x, p.y);
+                o.y = pack_bf16x2(p.z, p.w);
+                *reinterpret_cast<uint2 *>(dst + e0) = o;
             } else {
-                const long long z = e_base + lane - (long long)kStateRows * kD;
-                const __nv_bfloat16 hi = __float2bfloat16_rn(p);
-                const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
-                dst[(long long)kZHiRow0 * kD + z] = hi;
-                dst[(long long)kZLoRow0 * kD + z] = lo;
+                const uint32_t h01 = pack_bf16x2(p.x, p.y), h23 = pack_bf16x2(p.z, p.w);
+                const float r0 = p.x - __uint_as_float(h01 << 16), r1 = p.y - __uint_as_float(h01 & 0xFFFF0000u);
+                const float r2 = p.z - __uint_as_float(h23 << 16), r3 = p.w - __uint_as_float(h23 & 0xFFFF0000u);
+                *reinterpret_cast<uint2 *>(dst + (long long)kZHiRow0 * kD + z) = make_uint2(h01, h23);
+                *reinterpret_cast<uint2 *>(dst + (long long)kZLoRow0 * kD + z) =
+                    make_uint2(pack_bf16x2(r0, r1), pack_bf16x2(r2, r3));
             }
         }
-        __syncthreads();
     }
-    if (total != nullptr && lane == 0) {
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) total[bh * E + e_base + w + 8 * cc] = carry[cc];
-    }
+    if (total != nullptr && w == 0)
+        *reinterpret_cast<float4 *>(total + bh * E + e0) = carry;
 }
 
 // ---------------------------------------------------------------------------
@@ -243,33 +268,33 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { retur
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 k_transpose(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ kt, int T, int T_pad) {
-    __shared__ uint16_t tile[64][72];  // [token][d], rows padded to 144 B
+    // [token][feature] tile in 32-bit words, even tokens in rows 0..31 and odd
+    // tokens in rows 32..63; rows of 33 words keep both the row-wise writes
+    // and the column-wise reads free of bank conflicts.
+    __shared__ uint32_t tile[64][33];
     const int n_tt = T_pad / 64;
     const long long bh = blockIdx.x / n_tt;
     const int t0 = (blockIdx.x % n_tt) * 64;
-    const uint4 *src = reinterpret_cast<const uint4 *>(k);
-    uint4 in[2];
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(k);
+    uint32_t in[8];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {  // 64 tokens x 8 chunks of 8 values
-        const int x = threadIdx.x + 256 * r, s = x / 8, c8 = x % 8, t = t0 + s;
-        in[r] = t < T ? src[((bh * T + t) * kD) / 8 + c8] : make_uint4(0u, 0u, 0u, 0u);
+    for (int r = 0; r < 8; ++r) {  // 64 tokens x 32 words
+        const int x = threadIdx.x + 256 * r, s = x / 32, w = x % 32, t = t0 + s;
+        in[r] = t < T ? src[((bh * T + t) * kD) / 2 + w] : 0u;
     }
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int x = threadIdx.x + 256 * r, s = x / 8, c8 = x % 8;
-        *reinterpret_cast<uint4 *>(&tile[s][8 * c8]) = in[r];
+    for (int r = 0; r < 8; ++r) {
+        const int x = threadIdx.x + 256 * r, s = x / 32;
+        tile[(s & 1) * 32 + s / 2][x % 32] = in[r];
     }
     __syncthreads();
-    uint4 *dst = reinterpret_cast<uint4 *>(kt);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(kt);
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {  // 64 features x 8 runs of 8 tokens
-        const int x = threadIdx.x + 256 * r, d = x / 8, s8 = x % 8;
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            w[e] = static_cast<uint32_t>(tile[8 * s8 + 2 * e][d]) |
-                   (static_cast<uint32_t>(tile[8 * s8 + 2 * e + 1][d]) << 16);
-        dst[((bh * kD + d) * T_pad + t0) / 8 + s8] = make_uint4(w[0], w[1], w[2], w[3]);
+    for (int r = 0; r < 8; ++r) {  // 64 features x 32 token pairs
+        const int x = threadIdx.x + 256 * r, d = x / 32, s2 = x % 32;
+        const uint32_t a = tile[s2][d / 2], b2 = tile[32 + s2][d / 2];
+        const uint32_t w = (d & 1) ? ((a >> 16) | (b2 & 0xFFFF0000u)) : ((a & 0xFFFFu) | (b2 << 16));
+        dst[((bh * kD + d) * T_pad + t0) / 2 + s2] = w;
     }
 }
 
@@ -466,30 +491,39 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.done, 0, abort));
         if (ok) {
+            // Tile m holds 128 consecutive state rows in lane order (half-strips
+            // 32 c + 8 m .. + 7): stage each warp's 32 rows in shared memory
+            // (rows of 68 floats: conflict-free) and write them back two rows
+            // (512 contiguous bytes) per store instruction.  The rings are idle
+            // once `done` has completed, so their space is reused.
             tc_fence_after();
             float *base = seg_state + ((long long)bh * n_seg + g) * kF32PerSeg;
+            float *stage = reinterpret_cast<float *>(sm) + warp * (32 * 68);
             // warpgroup 0 stores tiles 0, 1 (and Z), warpgroup 1 tiles 2, 3
             for (int m = 2 * wg; m < 2 * wg + 2 + ((wg == 0 && zc) ? 1 : 0); ++m) {
                 const int mm = (m == 2 && wg == 0) ? kBTiles : m;
-                uint32_t o[32];
-                float *dst;
-                if (mm == kBTiles)
-                    dst = base + (long long)(kZRow0 + row) * kD;
-                else
-                    dst = base + ((long long)16 * (32 * c + 8 * mm + slot) + jj) * kD;
+                if (mm == kBTiles && qd >= 2) continue;  // Z has 64 rows (warps 0, 1)
+                float *dst = mm == kBTiles ? base + (long long)(kZRow0 + 32 * qd) * kD
+                                           : base + ((long long)16 * (32 * c + 8 * mm) + 32 * qd) * kD;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t o[32];
                     tmem_ld32(tm + 64 * mm + lane_base + 32 * hh, o);
                     tmem_ld_wait();
-                    if (mm != kBTiles || row < kD) {
-                        float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * hh);
 #pragma unroll
-                        for (int x = 0; x < 8; ++x)
-                            d4[x] = make_float4(__uint_as_float(o[4 * x]), __uint_as_float(o[4 * x + 1]),
-                                                __uint_as_float(o[4 * x + 2]),
-                                                __uint_as_float(o[4 * x + 3]));
-                    }
+                    for (int x = 0; x < 8; ++x)
+                        *reinterpret_cast<float4 *>(stage + lane * 68 + 32 * hh + 4 * x) =
+                            make_float4(__uint_as_float(o[4 * x]), __uint_as_float(o[4 * x + 1]),
+                                        __uint_as_float(o[4 * x + 2]), __uint_as_float(o[4 * x + 3]));
                 }
+                __syncwarp();
+#pragma unroll
+                for (int it = 0; it < 16; ++it) {
+                    const int r = 2 * it + lane / 16, ch = lane % 16;
+                    *reinterpret_cast<float4 *>(dst + r * kD + 4 * ch) =
+                        *reinterpret_cast<const float4 *>(stage + r * 68 + 4 * ch);
+                }
+                __syncwarp();
             }
         }
     }
@@ -854,9 +888,9 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
     }
     if (p.n_seg > 1) {
         ProfScope ps("tc_seg_scan", st);
-        const long long grid = (kF32PerSeg / 32) * BH;
-        tc_seg_scan<<<(unsigned)grid, dim3(32, 8), 0, st>>>(seg, prefix, want_state ? total : nullptr,
-                                                            p.n_seg, n_build);
+        const long long grid = (kF32PerSeg / 128) * BH;
+        tc_seg_scan<<<(unsigned)grid, 256, 0, st>>>(seg, prefix, want_state ? total : nullptr,
+                                                     p.n_seg, n_build);
     }
     {
         CUtensorMap mq, mk, mv, ms;
