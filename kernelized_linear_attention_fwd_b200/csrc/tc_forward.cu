@@ -29,7 +29,6 @@ namespace {
 
 using namespace kata::sm100;
 
-constexpr long long kF32PerSeg = (long long)kF32Rows * kD;    // 167,936 floats
 constexpr long long kBf16PerSeg = (long long)kBf16Rows * kD;  // 172,032 bf16
 
 // ---------------------------------------------------------------------------
@@ -57,13 +56,17 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     constexpr long long E = kF32PerSeg;
     constexpr long long n_eb = E / 128;
-    const long long eb = blockIdx.x % n_eb;
+    constexpr long long n_zb = kStateRows / 128;  // packed-z blocks (scattered writes): run them first
+    const long long eb = (blockIdx.x % n_eb + (n_eb - n_zb)) % n_eb;
     const long long bh = blockIdx.x / n_eb;
     const long long e0 = eb * 128 + 4 * lane;
     const float *base = seg_state + bh * (long long)n_seg * E + e0;
     __nv_bfloat16 *pbase = prefix + bh * (long long)n_seg * kBf16PerSeg;
-    const bool z_part = e0 >= (long long)kStateRows * kD;
-    const long long z = e0 - (long long)kStateRows * kD;
+    // packed z: the thread's 4 rows lie in one half-strip (row i, columns j0..j0+3)
+    const bool z_part = e0 >= kZPacked0;
+    const int zr = (int)(e0 - kZPacked0);
+    const int zi = z_part ? hs_i(zr / 16) : 0;
+    const int zj = z_part ? hs_jb(zr / 16) + zr % 16 : 0;
     float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
 
     for (int g0 = 0; g0 < n_seg; g0 += kScanWarps * kScanRun) {
@@ -110,12 +113,19 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
                 o.y = pack_bf16x2(p.z, p.w);
                 *reinterpret_cast<uint2 *>(dst + e0) = o;
             } else {
-                const uint32_t h01 = pack_bf16x2(p.x, p.y), h23 = pack_bf16x2(p.z, p.w);
-                const float r0 = p.x - __uint_as_float(h01 << 16), r1 = p.y - __uint_as_float(h01 & 0xFFFF0000u);
-                const float r2 = p.z - __uint_as_float(h23 << 16), r3 = p.w - __uint_as_float(h23 & 0xFFFF0000u);
-                *reinterpret_cast<uint2 *>(dst + (long long)kZHiRow0 * kD + z) = make_uint2(h01, h23);
-                *reinterpret_cast<uint2 *>(dst + (long long)kZLoRow0 * kD + z) =
-                    make_uint2(pack_bf16x2(r0, r1), pack_bf16x2(r2, r3));
+                // dense Z[i][j] and Z[j][i] as hi + lo bf16 (the mirrored entries of the
+                // diagonal half-strips carry identical values and write the same bits)
+                const float pv[4] = {p.x, p.y, p.z, p.w};
+                __nv_bfloat16 *zh = dst + (long long)kZHiRow0 * kD, *zl = dst + (long long)kZLoRow0 * kD;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(pv[x]);
+                    const __nv_bfloat16 lo = __float2bfloat16_rn(pv[x] - __bfloat162float(hi));
+                    zh[zi * kD + zj + x] = hi;
+                    zl[zi * kD + zj + x] = lo;
+                    zh[(zj + x) * kD + zi] = hi;
+                    zl[(zj + x) * kD + zi] = lo;
+                }
             }
         }
     }
@@ -143,7 +153,10 @@ tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__r
         state_out[bh * kD * kD * kD + x] = src[((long long)h * 16 + (j - hs_jb(h))) * kD + e];
     } else {
         x -= (long long)kD * kD * kD;
-        z_out[bh * kD * kD + x] = src[(long long)kZRow0 * kD + x];
+        int i = (int)(x / kD), j = (int)(x % kD);
+        if (i > j) { const int t = i; i = j; j = t; }
+        const int h = hs_index(i, j);
+        z_out[bh * kD * kD + x] = src[kZPacked0 + (long long)h * 16 + (j - hs_jb(h))];
     }
 }
 
@@ -164,9 +177,11 @@ constexpr int kQT = 128;                 // query tile (MMA M)
 constexpr int kTiles = 2;                // query tiles per CTA
 constexpr int kCtaQ = kQT * kTiles;      // 256 queries per CTA
 constexpr int kKB = 128;                 // key block
-constexpr int kRHs = 4;                  // half-strips per inter stage (64 state rows)
-constexpr int kRStages = kHalfStrips / kRHs;  // 40
-constexpr int kRRing = 4;                // inter ring depth
+constexpr int kRHs = 8;                  // half-strips per inter stage (128 state rows)
+constexpr int kRStages = kHalfStrips / kRHs;  // 20
+constexpr int kRRing = 2;                // inter A ring depth (tensor memory)
+constexpr int kRBRing = 4;               // inter B ring depth (state-prefix tiles, shared memory)
+constexpr int kRStageBytes = kRHs * 16 * 128;   // bf16 state-prefix rows per stage
 constexpr int kTmaWarp = 8;
 constexpr int kIssuer0 = 9;
 constexpr int kReadThreads = 352;
@@ -174,21 +189,21 @@ constexpr int kReadThreads = 352;
 // shared memory (from a 1024-byte aligned base)
 constexpr int kSmQ = 0;                          // 2 x [128 x 64] bf16, K-major, swizzled
 constexpr int kSmZ = kSmQ + kTiles * 16384;      // Z hi [64 x 64], Z lo [64 x 64]
-constexpr int kSmS = kSmZ + 16384;               // ring of [64 x 64] state-prefix tiles
-constexpr int kSmK = kSmS + kRRing * 8192;       // 2 x [128 x 64] keys
+constexpr int kSmS = kSmZ + 16384;               // ring of [128 x 64] state-prefix tiles
+constexpr int kSmK = kSmS + kRBRing * kRStageBytes;  // 2 x [128 x 64] keys
 constexpr int kSmV = kSmK + 2 * 16384;           // 2 x [128 x 64] values
 constexpr int kSmBytes = kSmV + 2 * 16384;
 constexpr int kSmAlloc = kSmBytes + 1024;
 
 // tensor memory columns (512 allocated)
 constexpr uint32_t kTmO = 0;     // O[t]: 64 columns at 64 t
-constexpr uint32_t kTmA = 128;   // inter stages: 64 columns at 128 + 64 s (tile t at + 32 t)
+constexpr uint32_t kTmA = 128;   // inter stages: 128 columns at 128 + 128 s (tile t at + 64 t)
 constexpr uint32_t kTmS = 128;   // intra scores S[t]: 128 columns at 128 + 128 t (after the inter phase)
 constexpr uint32_t kTmP = 384;   // U[t] (first) and P[t]: 64 columns at 384 + 64 t
 
 struct ReadBars {
     uint64_t q, u, interdone, o;
-    uint64_t bfull[kRRing], bempty[kRRing], afull[kRRing], aempty[kRRing];
+    uint64_t bfull[kRBRing], bempty[kRBRing], afull[kRRing], aempty[kRRing];
     uint64_t kvfull[2], kvempty[2];
     uint64_t sfull[kTiles], pfull[kTiles];
 };
@@ -233,7 +248,12 @@ struct GenLoop {
         gen_halfstrip<kRHs * ST + 1>(q2, a + 8);
         gen_halfstrip<kRHs * ST + 2>(q2, a + 16);
         gen_halfstrip<kRHs * ST + 3>(q2, a + 24);
-        tmem_st32(ta_tile + 64 * s, a);
+        tmem_st32(ta_tile + 128 * s, a);
+        gen_halfstrip<kRHs * ST + 4>(q2, a);
+        gen_halfstrip<kRHs * ST + 5>(q2, a + 8);
+        gen_halfstrip<kRHs * ST + 6>(q2, a + 16);
+        gen_halfstrip<kRHs * ST + 7>(q2, a + 24);
+        tmem_st32(ta_tile + 128 * s + 32, a);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars.afull[s]);
@@ -299,43 +319,47 @@ k_transpose(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ kt,
 }
 
 // ---------------------------------------------------------------------------
-// State builder on tcgen05.
+// State builder on tcgen05 (persistent: one CTA per SM loops over work items).
 //
-// Per (head, segment) 5 CTAs; CTA c accumulates the 4 tiles of 128 state rows
-// (half-strips h = 32 c + 8 m + s, m = tile, s = 16-lane slot) over the
-// segment's tokens:  D[m] += A[m] . V  with  A[m][(i, j)][token] = k_i k_j,
-// generated from the transposed keys into tensor memory by the thread that
-// owns the row's lane, and V (tokens x 64) the MN-major B operand in shared
-// memory.  CTA 0 adds a fifth tile, Z = K^T K (A rows k_i for lanes 0..63, B
-// the key tile itself).  Each thread reads its own key column k_j once per 16
-// tokens and the broadcast column k_i once per tile.
+// Work item = (head, segment, c), c = 0..4; item c accumulates the 4 tiles of
+// 128 state rows (half-strips h = 32 c + 8 m + s, m = tile, s = 16-lane slot)
+// over the segment's tokens:  D[m] += A[m] . [V | 1]  with
+// A[m][(i, j)][token] = k_i k_j generated from the transposed keys into tensor
+// memory by the thread owning the row's lane, and the MN-major B operand
+// [V | 1] = the value tile (64 columns) followed by a constant block whose
+// first column is one, so column 64 of D accumulates the packed normaliser
+// z = sum k_i k_j (N = 80; an N = 64 MMA costs the same issue time).
 // Roles: warps 0-3 / 4-7 generate the first / second 16-token step of every
-// 32-token stage; warp 8 is the TMA producer; warps 9 and 10 issue the MMAs of
-// alternate stages.  Accumulators are zeroed by tcgen05.st first and every
-// MMA accumulates.
+// 32-token stage and run the epilogue; warp 8 is the TMA producer; warps 9
+// and 10 issue the MMAs of alternate stages.  Barrier phases run on across
+// items, so the next item's tiles load while the current one is written back.
+// Accumulators are zeroed by tcgen05.st and every MMA accumulates.
 // ---------------------------------------------------------------------------
 constexpr int kBCtas = 5;
 constexpr int kBTiles = 4;
+constexpr int kBN = 80;                   // MMA N: 64 values, the ones column, 15 zero columns
 constexpr int kBTok = 64;                 // tokens per TMA tile (2 stages)
-constexpr int kBTileRing = 4;
-constexpr int kBStageBytes = 3 * 8192;    // K^T, V, K tiles
-constexpr int kBSmAlloc = kBTileRing * kBStageBytes + 1024 + 16384;  // padded: one CTA per SM
+constexpr int kBTileRing = 6;
+constexpr int kBTileBytes = 2 * 8192;     // K^T tile, V tile
+constexpr int kBOnes = kBTileRing * kBTileBytes;   // ones block [64 x 64] bf16, swizzled
+constexpr int kBStage = kBOnes + 8192;             // epilogue staging, 8 warps x 32 rows x 68 floats
+constexpr int kBSmAlloc = kBStage + 8 * 32 * 68 * 4 + 1024;
+constexpr int kBARing = 3;                // A stages in tensor memory
 constexpr int kBTmaWarp = 8;
 constexpr int kBIssuer0 = 9;
 constexpr int kBuildThreads = 352;
-constexpr uint32_t kBTmZ = 256;           // Z accumulator (CTA 0)
-constexpr uint32_t kBTmA = 320;           // A ring: slot s at 320 + 80 s, step kk at + 40 kk
+constexpr uint32_t kBTmA = kBTiles * kBN; // 320: A slot s at 320 + 64 s, step kk at + 32 kk
 
 struct BuildBars {
     uint64_t tfull[kBTileRing], tempty[kBTileRing];
-    uint64_t afull[2], aempty[2];
+    uint64_t afull[kBARing], aempty[kBARing];
     uint64_t done;
 };
 
 __global__ void __launch_bounds__(kBuildThreads, 1)
 tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_v,
-         const __grid_constant__ CUtensorMap tm_k, float *__restrict__ seg_state, int T, int L,
-         int n_seg, int n_build, int *status) {
+         float *__restrict__ seg_state, int T, int L, int n_seg, int n_build, int n_items,
+         int *status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ BuildBars bars;
     __shared__ uint32_t tmem_base;
@@ -343,15 +367,6 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
 
     uint8_t *sm = align1024(smem_raw);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int c = blockIdx.x % kBCtas;
-    const int rest = blockIdx.x / kBCtas;
-    const int g = rest % n_build;
-    const int bh = rest / n_build;
-    const bool zc = c == 0;
-    const int s0 = g * L;
-    const int ntok = min(L, T - s0);
-    const int n_tt = (ntok + kBTok - 1) / kBTok;
-    const int n_st = 2 * n_tt;               // 32-token stages
 
     if (tid == 0) {
         abort_flag = 0;
@@ -359,13 +374,19 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             mbar_init(&bars.tfull[x], 1);
             mbar_init(&bars.tempty[x], 2);
         }
-        for (int x = 0; x < 2; ++x) {
+        for (int x = 0; x < kBARing; ++x) {
             mbar_init(&bars.afull[x], 256);
             mbar_init(&bars.aempty[x], 1);
         }
         mbar_init(&bars.done, 2);
         fence_mbarrier_init();
     }
+    // constant ones block: logical column 0 of each of the 64 rows is 1.0
+    for (int x = tid; x < 8192 / 4; x += kBuildThreads) {
+        const int r = x / 32, w = x % 32;  // 32-bit word w of row r
+        reinterpret_cast<uint32_t *>(sm + kBOnes)[x] = (w == 4 * (r & 7)) ? 0x3F80u : 0u;
+    }
+    fence_proxy_async_smem();
     if (warp == kBIssuer0) {
         tmem_alloc(&tmem_base, 512);
         tmem_relinquish();
@@ -376,139 +397,146 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
     const uint32_t tm = tmem_base;
     volatile int *abort = &abort_flag;
 
+    // item -> (c, g, bh, token range)
+    auto item_geom = [&](int item, int &c, int &g, int &bh, int &s0, int &n_tt) {
+        c = item % kBCtas;
+        const int rest = item / kBCtas;
+        g = rest % n_build;
+        bh = rest / n_build;
+        s0 = g * L;
+        n_tt = (min(L, T - s0) + kBTok - 1) / kBTok;
+    };
+
     if (warp == kBTmaWarp) {
         if (lane == 0) {
             tma_prefetch_desc(&tm_kt);
             tma_prefetch_desc(&tm_v);
-            tma_prefetch_desc(&tm_k);
-            int issued = 0;
-            for (int t = 0; t < n_tt; ++t) {
-                const int b = t % kBTileRing;
-                if (!mbar_wait(&bars.tempty[b], ((t / kBTileRing) & 1) ^ 1, abort)) break;
-                uint8_t *st = sm + b * kBStageBytes;
-                mbar_arrive_expect_tx(&bars.tfull[b], zc ? 3 * 8192 : 2 * 8192);
-                tma_load_3d(st, &tm_kt, &bars.tfull[b], s0 + kBTok * t, 0, bh);
-                tma_load_3d(st + 8192, &tm_v, &bars.tfull[b], 0, s0 + kBTok * t, bh);
-                if (zc) tma_load_3d(st + 16384, &tm_k, &bars.tfull[b], 0, s0 + kBTok * t, bh);
-                ++issued;
+            int tt = 0;  // global tile counter
+            bool ok = true;
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+                int c, g, bh, s0, n_tt;
+                item_geom(item, c, g, bh, s0, n_tt);
+                for (int t = 0; t < n_tt; ++t, ++tt) {
+                    const int b = tt % kBTileRing;
+                    ok = mbar_wait(&bars.tempty[b], ((tt / kBTileRing) & 1) ^ 1, abort);
+                    if (!ok) break;
+                    uint8_t *st = sm + b * kBTileBytes;
+                    mbar_arrive_expect_tx(&bars.tfull[b], kBTileBytes);
+                    tma_load_3d(st, &tm_kt, &bars.tfull[b], s0 + kBTok * t, 0, bh);
+                    tma_load_3d(st + 8192, &tm_v, &bars.tfull[b], 0, s0 + kBTok * t, bh);
+                }
             }
-            for (int t = (issued > kBTileRing ? issued - kBTileRing : 0); t < issued; ++t)
+            for (int t = (tt > kBTileRing ? tt - kBTileRing : 0); t < tt; ++t)
                 mbar_wait(&bars.tfull[t % kBTileRing], (t / kBTileRing) & 1, abort);
         }
     } else if (warp == kBIssuer0 || warp == kBIssuer0 + 1) {
         if (lane == 0) {
             const int me = warp - kBIssuer0;
-            const uint32_t idesc = idesc_bf16(128, 64, 0, 1);
-            const uint64_t d0 = desc_sw128(smem_u32(sm), 8192, 1024);
+            const uint32_t idesc = idesc_bf16(128, kBN, 0, 1);
+            const uint32_t sbase = smem_u32(sm);
+            int tt = 0, j = 0;  // global tile counter, local item counter
             bool ok = true;
-            for (int st = me; st < n_st && ok; st += 2) {
-                const int t = st / 2, half = st % 2, b = t % kBTileRing;
-                ok = mbar_wait(&bars.tfull[b], (t / kBTileRing) & 1, abort) &&
-                     mbar_wait(&bars.afull[me], (st / 2) & 1, abort);
-                if (!ok) break;
-                tc_fence_after();
-                const uint64_t dv = desc_add(d0, b * kBStageBytes + 8192 + 4096 * half);
-                const uint64_t dk = desc_add(d0, b * kBStageBytes + 16384 + 4096 * half);
-                const uint32_t ta = tm + kBTmA + 80 * me;
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
+                int c, g, bh, s0, n_tt;
+                item_geom(item, c, g, bh, s0, n_tt);
+                for (int t = 0; t < n_tt && ok; ++t, ++tt) {
+                    const int G = 2 * tt + me;  // global stage: this issuer takes one half of each tile
+                    const int b = tt % kBTileRing, a = G % kBARing;
+                    ok = mbar_wait(&bars.tfull[b], (tt / kBTileRing) & 1, abort) &&
+                         mbar_wait(&bars.afull[a], (G / kBARing) & 1, abort);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t vaddr = sbase + b * kBTileBytes + 8192 + 4096 * me;
+                    const uint32_t oaddr = sbase + kBOnes + 4096 * me;
+                    const uint64_t dv = desc_sw128(vaddr, oaddr - vaddr, 1024);
+                    const uint32_t ta = tm + kBTmA + 64 * a;
 #pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
+                    for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
-                    for (int m = 0; m < kBTiles; ++m)
-                        mma_ts(tm + 64 * m, ta + 40 * kk + 8 * m, desc_add(dv, 2048 * kk), idesc, 1);
-                    if (zc) mma_ts(tm + kBTmZ, ta + 40 * kk + 32, desc_add(dk, 2048 * kk), idesc, 1);
+                        for (int m = 0; m < kBTiles; ++m)
+                            mma_ts(tm + kBN * m, ta + 32 * kk + 8 * m, desc_add(dv, 2048 * kk), idesc, 1);
+                    mma_commit(&bars.aempty[a]);
+                    mma_commit(&bars.tempty[b]);
                 }
-                mma_commit(&bars.aempty[me]);
-                mma_commit(&bars.tempty[b]);
+                mma_commit(&bars.done);  // this item's accumulation complete (with the other issuer)
             }
-            mma_commit(&bars.done);
-            mbar_wait(&bars.done, 0, abort);
+            mbar_wait(&bars.done, (j - 1) & 1, abort);  // drain before the CTA may free tensor memory
         }
     } else {
         const int wg = warp / 4, qd = warp % 4;
         const int row = 32 * qd + lane;          // lane within the 128-row tile
         const int slot = row / 16, jj = row % 16;
-        const int j = hs_jb(32 * c + slot) + jj;
-        int im[kBTiles];
-#pragma unroll
-        for (int m = 0; m < kBTiles; ++m) im[m] = hs_i(32 * c + 8 * m + slot);
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
-        {   // zero the accumulators (warpgroup 0: columns 0..159, warpgroup 1: 160..319)
-            uint32_t z[32];
-#pragma unroll
-            for (int x = 0; x < 32; ++x) z[x] = 0u;
-#pragma unroll
-            for (int x = 0; x < 5; ++x) tmem_st32(tm + 160 * wg + 32 * x + lane_base, z);
-        }
+        float *stage = reinterpret_cast<float *>(sm + kBStage) + warp * (32 * 68);
+        int tt = 0, j = 0;
         bool ok = true;
-        for (int st = 0; st < n_st && ok; ++st) {
-            const int t = st / 2, half = st % 2, b = t % kBTileRing, a = st % 2;
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars.tfull[b], (t / kBTileRing) & 1, abort) &&
-                                             mbar_wait(&bars.aempty[a], ((st / 2) & 1) ^ 1, abort));
-            if (!ok) break;
-            tc_fence_after();
-            const uint8_t *kt = sm + b * kBStageBytes;  // row d: 64 tokens, swizzled
-            const int c0 = 4 * half + 2 * wg, c1 = c0 + 1;  // this warpgroup's 16 tokens
-            uint32_t own[8];
-            {
-                const uint8_t *r = kt + j * 128;
-                const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (j & 7)) * 16));
-                const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (j & 7)) * 16));
-                own[0] = x0.x; own[1] = x0.y; own[2] = x0.z; own[3] = x0.w;
-                own[4] = x1.x; own[5] = x1.y; own[6] = x1.z; own[7] = x1.w;
-            }
-            const uint32_t ta = tm + kBTmA + 80 * a + 40 * wg + lane_base;
-            uint32_t p[32];
+        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
+            int c, g, bh, s0, n_tt;
+            item_geom(item, c, g, bh, s0, n_tt);
+            const int jcol = hs_jb(32 * c + slot) + jj;
+            int im[kBTiles];
 #pragma unroll
-            for (int m = 0; m < kBTiles; ++m) {
-                const int i = im[m];
-                const uint8_t *r = kt + i * 128;
-                const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (i & 7)) * 16));
-                const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (i & 7)) * 16));
-                p[8 * m + 0] = mul_bf16x2(own[0], x0.x); p[8 * m + 1] = mul_bf16x2(own[1], x0.y);
-                p[8 * m + 2] = mul_bf16x2(own[2], x0.z); p[8 * m + 3] = mul_bf16x2(own[3], x0.w);
-                p[8 * m + 4] = mul_bf16x2(own[4], x1.x); p[8 * m + 5] = mul_bf16x2(own[5], x1.y);
-                p[8 * m + 6] = mul_bf16x2(own[6], x1.z); p[8 * m + 7] = mul_bf16x2(own[7], x1.w);
-            }
-            tmem_st32(ta, p);
-            if (zc) {
-                // Z tile: lane i < 64 holds k_i over the tokens, lanes 64.. hold zero
-                uint32_t zz[8];
-                if (row < kD) {
-                    const uint8_t *r = kt + row * 128;
-                    const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (row & 7)) * 16));
-                    const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (row & 7)) * 16));
-                    zz[0] = x0.x; zz[1] = x0.y; zz[2] = x0.z; zz[3] = x0.w;
-                    zz[4] = x1.x; zz[5] = x1.y; zz[6] = x1.z; zz[7] = x1.w;
-                } else {
+            for (int m = 0; m < kBTiles; ++m) im[m] = hs_i(32 * c + 8 * m + slot);
+            {   // zero the accumulators (warpgroup 0: tiles 0, 1; warpgroup 1: tiles 2, 3)
+                uint32_t z[32];
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) zz[x] = 0u;
+                for (int x = 0; x < 32; ++x) z[x] = 0u;
+#pragma unroll
+                for (int x = 0; x < 5; ++x) tmem_st32(tm + 2 * kBN * wg + 32 * x + lane_base, z);
+            }
+            for (int t = 0; t < n_tt && ok; ++t, ++tt) {
+                const int b = tt % kBTileRing;
+                for (int half = 0; half < 2 && ok; ++half) {
+                    const int G = 2 * tt + half, a = G % kBARing;
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(&bars.tfull[b], (tt / kBTileRing) & 1, abort) &&
+                                        mbar_wait(&bars.aempty[a], ((G / kBARing) & 1) ^ 1, abort));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint8_t *kt = sm + b * kBTileBytes;  // row d: 64 tokens, swizzled
+                    const int c0 = 4 * half + 2 * wg, c1 = c0 + 1;  // this warpgroup's 16 tokens
+                    uint32_t own[8];
+                    {
+                        const uint8_t *r = kt + jcol * 128;
+                        const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (jcol & 7)) * 16));
+                        const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (jcol & 7)) * 16));
+                        own[0] = x0.x; own[1] = x0.y; own[2] = x0.z; own[3] = x0.w;
+                        own[4] = x1.x; own[5] = x1.y; own[6] = x1.z; own[7] = x1.w;
+                    }
+                    uint32_t p[32];
+#pragma unroll
+                    for (int m = 0; m < kBTiles; ++m) {
+                        const int i = im[m];
+                        const uint8_t *r = kt + i * 128;
+                        const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (i & 7)) * 16));
+                        const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (i & 7)) * 16));
+                        p[8 * m + 0] = mul_bf16x2(own[0], x0.x); p[8 * m + 1] = mul_bf16x2(own[1], x0.y);
+                        p[8 * m + 2] = mul_bf16x2(own[2], x0.z); p[8 * m + 3] = mul_bf16x2(own[3], x0.w);
+                        p[8 * m + 4] = mul_bf16x2(own[4], x1.x); p[8 * m + 5] = mul_bf16x2(own[5], x1.y);
+                        p[8 * m + 6] = mul_bf16x2(own[6], x1.z); p[8 * m + 7] = mul_bf16x2(own[7], x1.w);
+                    }
+                    tmem_st32(tm + kBTmA + 64 * a + 32 * wg + lane_base, p);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(&bars.afull[a]);
                 }
-                tmem_st8(ta + 32, zz);
             }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bars.afull[a]);
-        }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.done, 0, abort));
-        if (ok) {
-            // Tile m holds 128 consecutive state rows in lane order (half-strips
-            // 32 c + 8 m .. + 7): stage each warp's 32 rows in shared memory
-            // (rows of 68 floats: conflict-free) and write them back two rows
-            // (512 contiguous bytes) per store instruction.  The rings are idle
-            // once `done` has completed, so their space is reused.
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.done, j & 1, abort));
+            if (!ok) break;
+            // Epilogue.  Tile m holds 128 consecutive state rows in lane order
+            // (half-strips 32 c + 8 m .. + 7) and their packed z in column 64:
+            // stage each warp's 32 rows in shared memory (rows of 68 floats,
+            // conflict-free) and write them back two rows (512 contiguous bytes)
+            // per store.  Warpgroup 0 writes tiles 0, 1, warpgroup 1 tiles 2, 3.
             tc_fence_after();
             float *base = seg_state + ((long long)bh * n_seg + g) * kF32PerSeg;
-            float *stage = reinterpret_cast<float *>(sm) + warp * (32 * 68);
-            // warpgroup 0 stores tiles 0, 1 (and Z), warpgroup 1 tiles 2, 3
-            for (int m = 2 * wg; m < 2 * wg + 2 + ((wg == 0 && zc) ? 1 : 0); ++m) {
-                const int mm = (m == 2 && wg == 0) ? kBTiles : m;
-                if (mm == kBTiles && qd >= 2) continue;  // Z has 64 rows (warps 0, 1)
-                float *dst = mm == kBTiles ? base + (long long)(kZRow0 + 32 * qd) * kD
-                                           : base + ((long long)16 * (32 * c + 8 * mm) + 32 * qd) * kD;
+#pragma unroll 1
+            for (int m = 2 * wg; m < 2 * wg + 2; ++m) {
+                const long long row0 = (long long)16 * (32 * c + 8 * m) + 32 * qd;
+                uint32_t o[32];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t o[32];
-                    tmem_ld32(tm + 64 * mm + lane_base + 32 * hh, o);
+                    tmem_ld32(tm + kBN * m + lane_base + 32 * hh, o);
                     tmem_ld_wait();
 #pragma unroll
                     for (int x = 0; x < 8; ++x)
@@ -516,7 +544,11 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
                             make_float4(__uint_as_float(o[4 * x]), __uint_as_float(o[4 * x + 1]),
                                         __uint_as_float(o[4 * x + 2]), __uint_as_float(o[4 * x + 3]));
                 }
+                tmem_ld8(tm + kBN * m + 64 + lane_base, o);
+                tmem_ld_wait();
+                base[kZPacked0 + row0 + lane] = __uint_as_float(o[0]);
                 __syncwarp();
+                float *dst = base + row0 * kD;
 #pragma unroll
                 for (int it = 0; it < 16; ++it) {
                     const int r = 2 * it + lane / 16, ch = lane % 16;
@@ -525,6 +557,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
                 }
                 __syncwarp();
             }
+            tc_fence_before();  // accumulator reads ordered before the next item's zeroing
         }
     }
 
@@ -559,9 +592,11 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         mbar_init(&bars.u, 1);
         mbar_init(&bars.interdone, 2);
         mbar_init(&bars.o, 2);
-        for (int s = 0; s < kRRing; ++s) {
+        for (int s = 0; s < kRBRing; ++s) {
             mbar_init(&bars.bfull[s], 1);
             mbar_init(&bars.bempty[s], 1);
+        }
+        for (int s = 0; s < kRRing; ++s) {
             mbar_init(&bars.afull[s], 8 * 32);
             mbar_init(&bars.aempty[s], 1);
         }
@@ -601,12 +636,13 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             int issued_b = 0, issued_kv = 0;
             bool ok = true;
             for (int st = 0; inter && st < kRStages && ok; ++st) {
-                const int s = st % kRRing;
-                ok = mbar_wait(&bars.bempty[s], ((st / kRRing) & 1) ^ 1, abort);
+                const int s = st % kRBRing;
+                ok = mbar_wait(&bars.bempty[s], ((st / kRBRing) & 1) ^ 1, abort);
                 if (!ok) break;
-                mbar_arrive_expect_tx(&bars.bfull[s], 8192);
-                tma_load_3d(sm + kSmS + s * 8192, &tm_s, &bars.bfull[s], 0, 64 * st, sidx);
-                tma_load_3d(sm + kSmS + s * 8192 + 4096, &tm_s, &bars.bfull[s], 0, 64 * st + 32, sidx);
+                mbar_arrive_expect_tx(&bars.bfull[s], kRStageBytes);
+                for (int bx = 0; bx < kRStageBytes / 4096; ++bx)
+                    tma_load_3d(sm + kSmS + s * kRStageBytes + 4096 * bx, &tm_s, &bars.bfull[s], 0,
+                                16 * kRHs * st + 32 * bx, sidx);
                 ++issued_b;
             }
             for (int kb = 0; kb < n_kb && ok; ++kb) {
@@ -620,8 +656,8 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             }
             // drain: every load issued must have landed before the CTA exits
             mbar_wait(&bars.q, 0, abort);
-            for (int st = (issued_b > kRRing ? issued_b - kRRing : 0); st < issued_b; ++st)
-                mbar_wait(&bars.bfull[st % kRRing], (st / kRRing) & 1, abort);
+            for (int st = (issued_b > kRBRing ? issued_b - kRBRing : 0); st < issued_b; ++st)
+                mbar_wait(&bars.bfull[st % kRBRing], (st / kRBRing) & 1, abort);
             for (int kb = (issued_kv > 2 ? issued_kv - 2 : 0); kb < issued_kv; ++kb)
                 mbar_wait(&bars.kvfull[kb & 1], (kb >> 1) & 1, abort);
         }
@@ -653,19 +689,19 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     mma_commit(&bars.u);
                 }
                 for (int st = me; st < kRStages && ok; st += 2) {
-                    const int s = st % kRRing;
-                    const uint32_t ph = (st / kRRing) & 1;
-                    ok = mbar_wait(&bars.bfull[s], ph, abort) && mbar_wait(&bars.afull[s], ph, abort);
+                    const int s = st % kRRing, sb = st % kRBRing;
+                    ok = mbar_wait(&bars.bfull[sb], (st / kRBRing) & 1, abort) &&
+                         mbar_wait(&bars.afull[s], (st / kRRing) & 1, abort);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t ta = tm + kTmA + 64 * s;
-                    const uint64_t db = desc_add(dS, 8192 * s);
+                    const uint32_t ta = tm + kTmA + 128 * s;
+                    const uint64_t db = desc_add(dS, kRStageBytes * sb);
 #pragma unroll
                     for (int ks = 0; ks < kRHs; ++ks) {
                         mma_ts(tm + kTmO, ta + 8 * ks, desc_add(db, 2048 * ks), id_n64, 1);
-                        mma_ts(tm + kTmO + 64, ta + 32 + 8 * ks, desc_add(db, 2048 * ks), id_n64, 1);
+                        mma_ts(tm + kTmO + 64, ta + 64 + 8 * ks, desc_add(db, 2048 * ks), id_n64, 1);
                     }
-                    mma_commit(&bars.bempty[s]);
+                    mma_commit(&bars.bempty[sb]);
                     mma_commit(&bars.aempty[s]);
                 }
                 mma_commit(&bars.interdone);
@@ -748,7 +784,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                                          den_inter);
                     }
                 }
-                ok = GenLoop<0>::run(q2, bars, tm + kTmA + 32 * t + lane_base, abort);
+                ok = GenLoop<0>::run(q2, bars, tm + kTmA + 64 * t + lane_base, abort);
             }
         } else {
             tmem_st_wait();  // the zeroed accumulator is ordered before the first P hand-off
@@ -830,6 +866,19 @@ bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const
 
 }  // namespace
 
+// Streaming multiprocessors of the current device (persistent grids).
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 // Workspace of the tensor-core path (bytes; 256-aligned parts):
 //   fp32 segment states  BH * n_seg * 2624 * 64 * 4
 //   fp32 total           BH * 2624 * 64 * 4
@@ -869,22 +918,23 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
             k_transpose<<<(unsigned)((T_pad / 64) * BH), 256, 0, st>>>(
                 static_cast<const __nv_bfloat16 *>(k), kt, p.T, T_pad);
         }
-        CUtensorMap mkt, mvb, mkb;
+        CUtensorMap mkt, mvb;
         const uint64_t dkt[3] = {(uint64_t)T_pad, (uint64_t)kD, (uint64_t)BH};
         const uint64_t skt[2] = {(uint64_t)T_pad * 2, (uint64_t)kD * T_pad * 2};
         const uint32_t bkt[3] = {64, 64, 1};
         const uint64_t dqkv[3] = {(uint64_t)kD, (uint64_t)p.T, (uint64_t)BH};
         const uint64_t sqkv[2] = {(uint64_t)kD * 2, (uint64_t)p.T * kD * 2};
         const uint32_t b64[3] = {64, 64, 1};
-        if (!make_tmap_bf16(&mkt, kt, 3, dkt, skt, bkt) || !make_tmap_bf16(&mvb, v, 3, dqkv, sqkv, b64) ||
-            !make_tmap_bf16(&mkb, k, 3, dqkv, sqkv, b64))
+        if (!make_tmap_bf16(&mkt, kt, 3, dkt, skt, bkt) || !make_tmap_bf16(&mvb, v, 3, dqkv, sqkv, b64))
             return cudaErrorInvalidValue;
         cudaError_t e = cudaFuncSetAttribute(tc_build, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kBSmAlloc);
         if (e != cudaSuccess) return e;
+        const long long n_items = (long long)kBCtas * n_build * BH;
+        const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
         ProfScope ps("tc_build", st);
-        tc_build<<<(unsigned)(kBCtas * n_build * BH), kBuildThreads, kBSmAlloc, st>>>(
-            mkt, mvb, mkb, seg, p.T, p.L, p.n_seg, n_build, status);
+        tc_build<<<(unsigned)grid, kBuildThreads, kBSmAlloc, st>>>(mkt, mvb, seg, p.T, p.L, p.n_seg,
+                                                                    n_build, (int)n_items, status);
     }
     if (p.n_seg > 1) {
         ProfScope ps("tc_seg_scan", st);

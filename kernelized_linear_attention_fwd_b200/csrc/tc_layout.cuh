@@ -17,8 +17,9 @@
 // r = 16 h + (j - jb).
 //
 // Per (head, segment) the fp32 state is 2560 rows x 64 (the half-strips) then
-// 64 x 64 dense Z = sum k k^T; the bf16 prefix copy read by the readout is the
-// 2560 rows, then Z split into hi and lo bf16 parts (64 rows each).
+// the packed normaliser z[r] = sum k_i k_j for the same 2560 rows; the bf16
+// prefix copy read by the readout is the 2560 rows, then the dense
+// Z = sum k k^T split into hi and lo bf16 parts (64 rows each).
 #pragma once
 
 namespace kata {
@@ -27,8 +28,8 @@ namespace tc {
 constexpr int kD = 64;
 constexpr int kHalfStrips = 160;
 constexpr int kStateRows = 16 * kHalfStrips;        // 2560
-constexpr int kZRow0 = kStateRows;                  // fp32 Z rows start
-constexpr int kF32Rows = kStateRows + kD;           // 2624 rows of 64 floats
+constexpr long long kZPacked0 = (long long)kStateRows * kD;     // fp32 packed z offset
+constexpr long long kF32PerSeg = kZPacked0 + kStateRows;        // 166,400 floats
 constexpr int kBf16Rows = kStateRows + 2 * kD;      // 2688 rows of 64 bf16
 constexpr int kZHiRow0 = kStateRows;                // bf16 Z hi rows
 constexpr int kZLoRow0 = kStateRows + kD;           // bf16 Z lo rows
