@@ -72,6 +72,34 @@ def load_peaks():
 
 
 # ---------------------------------------------------------------------------
+# Multi-rank plumbing (weak scaling over independent heads)
+# ---------------------------------------------------------------------------
+
+
+def rank_seed(base_seed, rank):
+    """Each rank draws its own batch of independent heads."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(value, world, device="cuda"):
+    """Max of a per-rank float over all ranks (the slowest rank sets the job
+    time); identity for one rank.  Same collective on every rank."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, tokens_per_rank, ms_max):
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank / (ms_max / 1e3)
+
+
+# ---------------------------------------------------------------------------
 # Algorithmic work per unit (per token-head, canonical dense d^2 state form)
 # ---------------------------------------------------------------------------
 
@@ -257,8 +285,8 @@ def run_ours(args, rank, world):
     B, H, T, d = w.B, w.H, w.T, w.d
     BH = B * H
     # each rank: its own batch of independent heads (seed offset by rank)
-    qh, kh, vh = inputs.make_qkv(B, H, T, d, d, w.dtype, seed=w.seed + 1000 * rank, qk=w.qk)
-    q1h, k1h, v1h = inputs.make_qkv(B, H, 1, d, d, w.dtype, seed=w.seed + 1000 * rank, qk=w.qk,
+    qh, kh, vh = inputs.make_qkv(B, H, T, d, d, w.dtype, seed=rank_seed(w.seed, rank), qk=w.qk)
+    q1h, k1h, v1h = inputs.make_qkv(B, H, 1, d, d, w.dtype, seed=rank_seed(w.seed, rank), qk=w.qk,
                                     tag=1)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
@@ -317,11 +345,7 @@ def run_ours(args, rank, world):
     step_ms = [a.elapsed_time(b) for a, b in ev]
     prof = profile_read()
     ms_local = sum(step_ms) / len(step_ms)
-    ms_max = ms_local
-    if world > 1:
-        t = torch.tensor([ms_local], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms_local, world)
     status = K.kata_get_device_status()
 
     # end-to-end through the public API with host buffers
@@ -354,15 +378,11 @@ def run_ours(args, rank, world):
             e2e_step()
             eve[i][1].record(stream)
         torch.cuda.synchronize()
-        e2e_ms = sum(a.elapsed_time(b) for a, b in eve) / args.steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in eve) / args.steps, world)
         es = 2 if w.dtype == "bf16" else 4
         h2d = 3 * BH * T * d * es + 3 * BH * d * es
         d2h = BH * T * d * es + BH * d * es
-        e2e = {"value": world * B * T / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": job_throughput(world, B * T, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     # decode bandwidth on the 64 x 16-head decode workload
@@ -391,11 +411,7 @@ def run_ours(args, rank, world):
             evd[i][1].record(stream)
         torch.cuda.synchronize()
         dms = sorted(a.elapsed_time(b) for a, b in evd)
-        dmean = sum(dms) / nd
-        if world > 1:
-            t = torch.tensor([dmean], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            dmean = float(t.item())
+        dmean = max_over_ranks(sum(dms) / nd, world)
         es = 2 if w.dtype == "bf16" else 4
         dbytes = Bd * Hd * ((d * d * d + d * d) * 4 * 2 + 4 * d * es)
         peaks, src = load_peaks()
@@ -451,7 +467,7 @@ def run_ours(args, rank, world):
              "note": "whole step (all kernels), canonical dense d^2 flops of the chunked form"}
     line = {
         "metric": METRIC,
-        "value": tokens / (ms_max / 1e3),
+        "value": job_throughput(world, B * T, ms_max),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
