@@ -22,8 +22,8 @@ namespace kata {
 namespace sm100 {
 
 // Upper bound of any on-device wait before the kernel gives up, in SM clock
-// cycles (2^33 cycles: about 4.4 s at 1.965 GHz, longer at lower clocks).
-constexpr long long kWaitTimeoutCycles = 1ll << 33;
+// cycles (2^31 cycles: about 1.1 s at 1.965 GHz, longer at lower clocks).
+constexpr long long kWaitTimeoutCycles = 1ll << 31;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -83,6 +83,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
                 return false;
             }
         }
+    }
+}
+
+// Waits for an asynchronous copy or MMA that was already issued (so it
+// completes by itself): spins on try_wait, ignoring *abort, for at most
+// kWaitTimeoutCycles.  Used before a CTA exits, so that no copy lands in, and
+// no MMA reads, memory the CTA has given up.
+__device__ __forceinline__ bool mbar_wait_issued(uint64_t *bar, uint32_t parity) {
+    const long long t0 = clock64();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 1023u) == 1023u && clock64() - t0 > kWaitTimeoutCycles) return false;
     }
 }
 

@@ -161,25 +161,33 @@ tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__r
 }
 
 // ---------------------------------------------------------------------------
-// Readout kernel.
+// Readout kernel (persistent: one CTA per SM walks a contiguous range of work
+// items, so consecutive items of a segment reuse its state prefix and keys
+// from L2).
 //
-// A CTA owns 256 queries (two 128-query tiles) of one segment.  Roles:
+// Work item = 256 queries (two 128-query tiles) of one segment.  Roles:
 //   warps 0-3 / 4-7  phi(Q) generation, then squared-score masking and the
 //                    epilogue, for tile 0 / tile 1 (thread = query row)
-//   warp 8           TMA producer (Q, Z prefix, state-prefix stages, K/V blocks)
+//   warp 8           TMA producer (Q and the Z prefix into a double-buffered
+//                    item slot, state-prefix stages, K/V blocks)
 //   warps 9, 10      MMA issuers.  In the inter phase they take alternate
 //                    stages (so one issuer's wait overlaps the other's queued
-//                    MMAs); in the intra phase issuer t serves query tile t.
-// Accumulators are zeroed by tcgen05.st before the first MMA, and every MMA
-// accumulates, so the order in which the two issuers' MMAs run is free.
+//                    MMAs); in the intra phase issuer t serves query tile t,
+//                    running the scores of key block b + 1 while the
+//                    generation warps square and mask block b.
+// Every barrier phase runs on across items.  Accumulators are zeroed by
+// tcgen05.st (at the start, then by each epilogue right after it reads them)
+// and every MMA accumulates, so the order in which the two issuers' MMAs run
+// is free.
 // ---------------------------------------------------------------------------
 constexpr int kQT = 128;                 // query tile (MMA M)
-constexpr int kTiles = 2;                // query tiles per CTA
-constexpr int kCtaQ = kQT * kTiles;      // 256 queries per CTA
-constexpr int kKB = 128;                 // key block
+constexpr int kTiles = 2;                // query tiles per item
+constexpr int kCtaQ = kQT * kTiles;      // 256 queries per item
+constexpr int kKB = 128;                 // key/value block loaded by TMA
+constexpr int kSB = 64;                  // score block (MMA N of Q K^T)
 constexpr int kRHs = 8;                  // half-strips per inter stage (128 state rows)
 constexpr int kRStages = kHalfStrips / kRHs;  // 20
-constexpr int kRRing = 2;                // inter A ring depth (tensor memory)
+constexpr int kRRing = 3;                // inter A ring depth (tensor memory)
 constexpr int kRBRing = 4;               // inter B ring depth (state-prefix tiles, shared memory)
 constexpr int kRStageBytes = kRHs * 16 * 128;   // bf16 state-prefix rows per stage
 constexpr int kTmaWarp = 8;
@@ -187,9 +195,9 @@ constexpr int kIssuer0 = 9;
 constexpr int kReadThreads = 352;
 
 // shared memory (from a 1024-byte aligned base)
-constexpr int kSmQ = 0;                          // 2 x [128 x 64] bf16, K-major, swizzled
-constexpr int kSmZ = kSmQ + kTiles * 16384;      // Z hi [64 x 64], Z lo [64 x 64]
-constexpr int kSmS = kSmZ + 16384;               // ring of [128 x 64] state-prefix tiles
+constexpr int kItemBytes = kTiles * 16384 + 16384;  // Q tiles [128 x 64] x 2, Z hi / lo [64 x 64]
+constexpr int kSmItem = 0;                       // 2 item slots (double buffer)
+constexpr int kSmS = kSmItem + 2 * kItemBytes;   // ring of [128 x 64] state-prefix tiles
 constexpr int kSmK = kSmS + kRBRing * kRStageBytes;  // 2 x [128 x 64] keys
 constexpr int kSmV = kSmK + 2 * 16384;           // 2 x [128 x 64] values
 constexpr int kSmBytes = kSmV + 2 * 16384;
@@ -197,16 +205,45 @@ constexpr int kSmAlloc = kSmBytes + 1024;
 
 // tensor memory columns (512 allocated)
 constexpr uint32_t kTmO = 0;     // O[t]: 64 columns at 64 t
-constexpr uint32_t kTmA = 128;   // inter stages: 128 columns at 128 + 128 s (tile t at + 64 t)
-constexpr uint32_t kTmS = 128;   // intra scores S[t]: 128 columns at 128 + 128 t (after the inter phase)
-constexpr uint32_t kTmP = 384;   // U[t] (first) and P[t]: 64 columns at 384 + 64 t
+constexpr uint32_t kTmA = 128;   // inter A slot s: 128 columns at 128 + 128 s (tile t at + 64 t)
+constexpr uint32_t kTmU = 384;   // U[t] = Q Z (before slot 2 is first written): 64 columns at 384 + 64 t
+constexpr uint32_t kTmS = 128;   // intra scores S[t][x]: 64 columns at 128 + 128 t + 64 x
+constexpr uint32_t kTmP = 384;   // intra weights P[t][x] (bf16 pairs): 32 columns at 384 + 64 t + 32 x
 
 struct ReadBars {
-    uint64_t q, u, interdone, o;
+    uint64_t qfull[2], qempty[2], u, interdone, done, genin;
     uint64_t bfull[kRBRing], bempty[kRBRing], afull[kRRing], aempty[kRRing];
     uint64_t kvfull[2], kvempty[2];
-    uint64_t sfull[kTiles], pfull[kTiles];
+    uint64_t sfull[kTiles][2], pfull[kTiles][2], pempty[kTiles][2];
+    uint64_t drain[2];
 };
+
+// One work item of the readout.
+struct ReadItem {
+    int bh, t0, seg0, sidx, n_kv;
+    bool inter;
+};
+
+__device__ __forceinline__ ReadItem read_item(int i, int n_ct, int T, int L, int n_seg) {
+    ReadItem it;
+    it.bh = i / n_ct;
+    it.t0 = (i % n_ct) * kCtaQ;
+    const int g = it.t0 / L;
+    it.seg0 = g * L;
+    it.sidx = it.bh * n_seg + g;
+    it.inter = g > 0;
+    const int tend = min(it.t0 + kCtaQ, T);
+    it.n_kv = (tend - it.seg0 + kKB - 1) / kKB;
+    return it;
+}
+
+// 64-key score blocks of tile t: keys seg0 .. min(end of tile, T) - 1; none
+// when the tile starts at or after T.
+__device__ __forceinline__ int read_tile_blocks(const ReadItem &it, int t, int T) {
+    const int q0 = it.t0 + kQT * t;
+    if (q0 >= T) return 0;
+    return (min(q0 + kQT, T) - it.seg0 + kSB - 1) / kSB;
+}
 
 __device__ __forceinline__ uint32_t dup_lo(uint32_t x) { return __byte_perm(x, 0, 0x1010); }
 __device__ __forceinline__ uint32_t dup_hi(uint32_t x) { return __byte_perm(x, 0, 0x3232); }
@@ -235,12 +272,15 @@ __device__ __forceinline__ void gen_halfstrip(const uint32_t (&q2)[32], uint32_t
     }
 }
 
+// Generates the 20 inter stages of one item into the A ring.  `g0` is the
+// number of stages generated before this item (ring slot and phase).
 template <int ST>
 struct GenLoop {
     __device__ __forceinline__ static bool run(const uint32_t (&q2)[32], ReadBars &bars,
-                                               uint32_t ta_tile, volatile int *abort) {
-        constexpr int s = ST % kRRing;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[s], ((ST / kRRing) & 1) ^ 1, abort)))
+                                               uint32_t ta_tile, int g0, volatile int *abort) {
+        const int G = g0 + ST;
+        const int s = G % kRRing;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[s], ((G / kRRing) & 1) ^ 1, abort)))
             return false;
         tc_fence_after();
         uint32_t a[32];
@@ -257,12 +297,12 @@ struct GenLoop {
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars.afull[s]);
-        return GenLoop<ST + 1>::run(q2, bars, ta_tile, abort);
+        return GenLoop<ST + 1>::run(q2, bars, ta_tile, g0, abort);
     }
 };
 template <>
 struct GenLoop<kRStages> {
-    __device__ __forceinline__ static bool run(const uint32_t (&)[32], ReadBars &, uint32_t,
+    __device__ __forceinline__ static bool run(const uint32_t (&)[32], ReadBars &, uint32_t, int,
                                                volatile int *) {
         return true;
     }
@@ -570,7 +610,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
 __global__ void __launch_bounds__(kReadThreads, 1)
 tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
-        __nv_bfloat16 *__restrict__ out, int T, int L, int n_seg, int n_ct, int *status) {
+        __nv_bfloat16 *__restrict__ out, int T, int L, int n_seg, int n_ct, int n_items, int *status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ ReadBars bars;
     __shared__ uint32_t tmem_base;
@@ -578,20 +618,22 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
 
     uint8_t *sm = align1024(smem_raw);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int bh = blockIdx.x / n_ct;
-    const int t0 = (blockIdx.x % n_ct) * kCtaQ;
-    const int g = t0 / L;
-    const int seg0 = g * L;
-    const bool inter = g > 0;
-    const int n_kb = (t0 + kCtaQ - seg0) / kKB;
-    const int sidx = bh * n_seg + g;
+    const int i_begin = (int)((long long)blockIdx.x * n_items / gridDim.x);
+    const int i_end = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x);
 
     if (tid == 0) {
         abort_flag = 0;
-        mbar_init(&bars.q, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars.qfull[b], 1);
+            mbar_init(&bars.qempty[b], 2 + 8);  // both issuers' commits + one arrival per generation warp
+            mbar_init(&bars.kvfull[b], 1);
+            mbar_init(&bars.kvempty[b], 2);
+            mbar_init(&bars.drain[b], 1);
+        }
         mbar_init(&bars.u, 1);
         mbar_init(&bars.interdone, 2);
-        mbar_init(&bars.o, 2);
+        mbar_init(&bars.done, 2);
+        mbar_init(&bars.genin, 8);
         for (int s = 0; s < kRBRing; ++s) {
             mbar_init(&bars.bfull[s], 1);
             mbar_init(&bars.bempty[s], 1);
@@ -600,14 +642,12 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             mbar_init(&bars.afull[s], 8 * 32);
             mbar_init(&bars.aempty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars.kvfull[s], 1);
-            mbar_init(&bars.kvempty[s], 2);
-        }
-        for (int t = 0; t < kTiles; ++t) {
-            mbar_init(&bars.sfull[t], 1);
-            mbar_init(&bars.pfull[t], 4 * 32);
-        }
+        for (int t = 0; t < kTiles; ++t)
+            for (int x = 0; x < 2; ++x) {
+                mbar_init(&bars.sfull[t][x], 1);
+                mbar_init(&bars.pfull[t][x], 4 * 32);
+                mbar_init(&bars.pempty[t][x], 1);
+            }
         fence_mbarrier_init();
     }
     if (warp == kIssuer0) {
@@ -627,154 +667,224 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_s);
-            mbar_arrive_expect_tx(&bars.q, kTiles * 16384 + (inter ? 16384 : 0));
-            for (int t = 0; t < kTiles; ++t)
-                tma_load_3d(sm + kSmQ + t * 16384, &tm_q, &bars.q, 0, t0 + t * kQT, bh);
-            if (inter)
-                for (int zz = 0; zz < 4; ++zz)  // Z hi rows 2560..2623, Z lo rows 2624..2687
-                    tma_load_3d(sm + kSmZ + zz * 4096, &tm_s, &bars.q, 0, kZHiRow0 + 32 * zz, sidx);
-            int issued_b = 0, issued_kv = 0;
+            int n_q = 0, n_bs = 0, n_kv = 0;  // loads issued into each ring
             bool ok = true;
-            for (int st = 0; inter && st < kRStages && ok; ++st) {
-                const int s = st % kRBRing;
-                ok = mbar_wait(&bars.bempty[s], ((st / kRBRing) & 1) ^ 1, abort);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&bars.bfull[s], kRStageBytes);
-                for (int bx = 0; bx < kRStageBytes / 4096; ++bx)
-                    tma_load_3d(sm + kSmS + s * kRStageBytes + 4096 * bx, &tm_s, &bars.bfull[s], 0,
-                                16 * kRHs * st + 32 * bx, sidx);
-                ++issued_b;
+            for (int i = i_begin; i < i_end && ok; ++i) {
+                const ReadItem it = read_item(i, n_ct, T, L, n_seg);
+                {
+                    const int qb = n_q & 1;
+                    uint8_t *slot = sm + kSmItem + qb * kItemBytes;
+                    ok = mbar_wait(&bars.qempty[qb], ((n_q >> 1) & 1) ^ 1, abort);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&bars.qfull[qb], kTiles * 16384 + (it.inter ? 16384 : 0));
+                    for (int t = 0; t < kTiles; ++t)
+                        tma_load_3d(slot + t * 16384, &tm_q, &bars.qfull[qb], 0, it.t0 + t * kQT, it.bh);
+                    if (it.inter)
+                        for (int zz = 0; zz < 4; ++zz)  // Z hi rows 2560..2623, Z lo rows 2624..2687
+                            tma_load_3d(slot + kTiles * 16384 + zz * 4096, &tm_s, &bars.qfull[qb], 0,
+                                        kZHiRow0 + 32 * zz, it.sidx);
+                    ++n_q;
+                }
+                for (int st = 0; it.inter && st < kRStages && ok; ++st) {
+                    const int s = n_bs % kRBRing;
+                    ok = mbar_wait(&bars.bempty[s], ((n_bs / kRBRing) & 1) ^ 1, abort);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&bars.bfull[s], kRStageBytes);
+                    for (int bx = 0; bx < kRStageBytes / 4096; ++bx)
+                        tma_load_3d(sm + kSmS + s * kRStageBytes + 4096 * bx, &tm_s, &bars.bfull[s], 0,
+                                    16 * kRHs * st + 32 * bx, it.sidx);
+                    ++n_bs;
+                }
+                for (int kb = 0; kb < it.n_kv && ok; ++kb) {
+                    const int s = n_kv & 1;
+                    ok = mbar_wait(&bars.kvempty[s], ((n_kv >> 1) & 1) ^ 1, abort);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&bars.kvfull[s], 32768);
+                    tma_load_3d(sm + kSmK + s * 16384, &tm_k, &bars.kvfull[s], 0, it.seg0 + kb * kKB, it.bh);
+                    tma_load_3d(sm + kSmV + s * 16384, &tm_v, &bars.kvfull[s], 0, it.seg0 + kb * kKB, it.bh);
+                    ++n_kv;
+                }
             }
-            for (int kb = 0; kb < n_kb && ok; ++kb) {
-                const int s = kb & 1;
-                ok = mbar_wait(&bars.kvempty[s], ((kb >> 1) & 1) ^ 1, abort);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&bars.kvfull[s], 32768);
-                tma_load_3d(sm + kSmK + s * 16384, &tm_k, &bars.kvfull[s], 0, seg0 + kb * kKB, bh);
-                tma_load_3d(sm + kSmV + s * 16384, &tm_v, &bars.kvfull[s], 0, seg0 + kb * kKB, bh);
-                ++issued_kv;
-            }
-            // drain: every load issued must have landed before the CTA exits
-            mbar_wait(&bars.q, 0, abort);
-            for (int st = (issued_b > kRBRing ? issued_b - kRBRing : 0); st < issued_b; ++st)
-                mbar_wait(&bars.bfull[st % kRBRing], (st / kRBRing) & 1, abort);
-            for (int kb = (issued_kv > 2 ? issued_kv - 2 : 0); kb < issued_kv; ++kb)
-                mbar_wait(&bars.kvfull[kb & 1], (kb >> 1) & 1, abort);
+            // every load issued must have landed before the CTA exits
+            for (int x = (n_q > 2 ? n_q - 2 : 0); x < n_q; ++x)
+                mbar_wait_issued(&bars.qfull[x & 1], (x >> 1) & 1);
+            for (int x = (n_bs > kRBRing ? n_bs - kRBRing : 0); x < n_bs; ++x)
+                mbar_wait_issued(&bars.bfull[x % kRBRing], (x / kRBRing) & 1);
+            for (int x = (n_kv > 2 ? n_kv - 2 : 0); x < n_kv; ++x)
+                mbar_wait_issued(&bars.kvfull[x & 1], (x >> 1) & 1);
         }
     } else if (warp == kIssuer0 || warp == kIssuer0 + 1) {
         // ------------------------------------------------------------ MMA issuers
         if (lane == 0) {
-            const int me = warp - kIssuer0;
-            const uint32_t id_qk = idesc_bf16(kQT, kKB, 0, 0);
-            const uint32_t id_n64 = idesc_bf16(kQT, 64, 0, 1);
-            const uint64_t dQ0 = desc_sw128(smem_u32(sm + kSmQ), 16, 1024);
-            const uint64_t dZ = desc_sw128(smem_u32(sm + kSmZ), 8192, 1024);
+            const int me = warp - kIssuer0, t = me;
+            const uint32_t id_n64 = idesc_bf16(kQT, 64, 0, 1);  // B MN-major, N = 64
+            const uint32_t id_qk = idesc_bf16(kQT, kSB, 0, 0);  // B = keys, K-major
             const uint64_t dS = desc_sw128(smem_u32(sm + kSmS), 8192, 1024);
             const uint64_t dK = desc_sw128(smem_u32(sm + kSmK), 16, 1024);
             const uint64_t dV = desc_sw128(smem_u32(sm + kSmV), 8192, 1024);
-            bool ok = mbar_wait(&bars.q, 0, abort);
-            if (ok) tc_fence_after();
-            if (ok && inter) {
-                if (me == 0) {
-                    for (int t = 0; t < kTiles; ++t) {
-                        const uint32_t dU = tm + kTmP + 64 * t;
-                        const uint64_t dq = desc_add(dQ0, t * 16384);
+            const uint32_t tS = tm + kTmS + 128 * t, tP = tm + kTmP + 64 * t, tO = tm + kTmO + 64 * t;
+            int n_inter = 0, g_kv = 0, g_b = 0, j = 0;
+            bool ok = true;
+            // weights of score block bb (global index g_b + bb) times its values
+            auto pv = [&](int bb) -> bool {
+                const int n = g_b + bb, x = n & 1;
+                if (!mbar_wait(&bars.pfull[t][x], (n >> 1) & 1, abort)) return false;
+                tc_fence_after();
+                const int G = g_kv + bb / 2;
+                const uint64_t dv = desc_add(dV, 16384 * (G & 1) + 8192 * (bb & 1));
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            mma_ss(dU, desc_add(dq, 32 * ks), desc_add(dZ, 2048 * ks), id_n64, ks > 0);
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            mma_ss(dU, desc_add(dq, 32 * ks), desc_add(dZ, 8192 + 2048 * ks), id_n64, 1);
-                    }
-                    mma_commit(&bars.u);
-                }
-                for (int st = me; st < kRStages && ok; st += 2) {
-                    const int s = st % kRRing, sb = st % kRBRing;
-                    ok = mbar_wait(&bars.bfull[sb], (st / kRBRing) & 1, abort) &&
-                         mbar_wait(&bars.afull[s], (st / kRRing) & 1, abort);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t ta = tm + kTmA + 128 * s;
-                    const uint64_t db = desc_add(dS, kRStageBytes * sb);
-#pragma unroll
-                    for (int ks = 0; ks < kRHs; ++ks) {
-                        mma_ts(tm + kTmO, ta + 8 * ks, desc_add(db, 2048 * ks), id_n64, 1);
-                        mma_ts(tm + kTmO + 64, ta + 64 + 8 * ks, desc_add(db, 2048 * ks), id_n64, 1);
-                    }
-                    mma_commit(&bars.bempty[sb]);
-                    mma_commit(&bars.aempty[s]);
-                }
-                mma_commit(&bars.interdone);
-                // scores reuse the inter stage columns: every inter MMA must be done
-                ok = ok && mbar_wait(&bars.interdone, 0, abort);
-                if (ok) tc_fence_after();
-            }
-            // intra phase: issuer `me` serves query tile `me`
-            const int t = me;
-            const uint64_t dq = desc_add(dQ0, t * 16384);
-            for (int kb = 0; kb < n_kb && ok; ++kb) {
-                const int s = kb & 1;
-                ok = mbar_wait(&bars.kvfull[s], (kb >> 1) & 1, abort);
+                for (int ks = 0; ks < kSB / 16; ++ks)
+                    mma_ts(tO, tP + 32 * x + 8 * ks, desc_add(dv, 2048 * ks), id_n64, 1);
+                mma_commit(&bars.pempty[t][x]);
+                return true;
+            };
+            for (int i = i_begin; i < i_end && ok; ++i, ++j) {
+                const ReadItem it = read_item(i, n_ct, T, L, n_seg);
+                const int qb = j & 1;
+                const uint32_t slot = smem_u32(sm + kSmItem + qb * kItemBytes);
+                ok = mbar_wait(&bars.qfull[qb], (j >> 1) & 1, abort);
                 if (!ok) break;
                 tc_fence_after();
-                const int kbs = seg0 + kb * kKB;
-                if (kbs < t0 + t * kQT + kQT) {  // block not entirely after the tile
-                    const uint64_t dk = desc_add(dK, 16384 * s);
+                if (it.inter) {
+                    if (me == 0) {
+                        // U = Q (Z hi + Z lo) into columns that held the previous item's weights
+                        if (j > 0) {
+                            ok = mbar_wait(&bars.done, (j - 1) & 1, abort);
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
+                        const uint64_t dZ = desc_sw128(slot + kTiles * 16384, 8192, 1024);
+                        for (int u = 0; u < kTiles; ++u) {
+                            const uint64_t dq = desc_sw128(slot + u * 16384, 16, 1024);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_ss(tm + kTmS + 128 * t, desc_add(dq, 32 * ks), desc_add(dk, 32 * ks), id_qk,
-                               ks > 0);
-                    mma_commit(&bars.sfull[t]);
-                    ok = mbar_wait(&bars.pfull[t], kb & 1, abort);
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_ss(tm + kTmU + 64 * u, desc_add(dq, 32 * ks), desc_add(dZ, 2048 * ks),
+                                       id_n64, ks > 0);
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_ss(tm + kTmU + 64 * u, desc_add(dq, 32 * ks),
+                                       desc_add(dZ, 8192 + 2048 * ks), id_n64, 1);
+                        }
+                        mma_commit(&bars.u);
+                    }
+                    for (int st = me; st < kRStages && ok; st += 2) {
+                        const int G = n_inter * kRStages + st;
+                        const int s = G % kRRing, sb = G % kRBRing;
+                        ok = mbar_wait(&bars.bfull[sb], (G / kRBRing) & 1, abort) &&
+                             mbar_wait(&bars.afull[s], (G / kRRing) & 1, abort);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t ta = tm + kTmA + 128 * s;
+                        const uint64_t db = desc_add(dS, kRStageBytes * sb);
+#pragma unroll
+                        for (int ks = 0; ks < kRHs; ++ks) {
+                            mma_ts(tm + kTmO, ta + 8 * ks, desc_add(db, 2048 * ks), id_n64, 1);
+                            mma_ts(tm + kTmO + 64, ta + 64 + 8 * ks, desc_add(db, 2048 * ks), id_n64, 1);
+                        }
+                        mma_commit(&bars.bempty[sb]);
+                        mma_commit(&bars.aempty[s]);
+                    }
+                    if (!ok) break;
+                    mma_commit(&bars.interdone);
+                    // the scores reuse the A ring's columns: every inter MMA must be done
+                    ok = mbar_wait(&bars.interdone, n_inter & 1, abort);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint64_t dv = desc_add(dV, 16384 * s);
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_ts(tm + kTmO + 64 * t, tm + kTmP + 64 * t + 8 * ks, desc_add(dv, 2048 * ks),
-                               id_n64, 1);
+                    ++n_inter;
                 }
-                mma_commit(&bars.kvempty[s]);
+                // intra phase: scores of block b are issued before the weights of block b - 1
+                const int n_b = read_tile_blocks(it, t, T);
+                const uint64_t dQt = desc_sw128(slot + t * 16384, 16, 1024);
+                for (int b = 0; b < n_b && ok; ++b) {
+                    const int n = g_b + b, x = n & 1;
+                    const int G = g_kv + b / 2;
+                    if ((b & 1) == 0) {
+                        ok = mbar_wait(&bars.kvfull[G & 1], (G >> 1) & 1, abort);
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+                    const uint64_t dk = desc_add(dK, 16384 * (G & 1) + 8192 * (b & 1));
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ss(tS + 64 * x, desc_add(dQt, 32 * ks), desc_add(dk, 32 * ks), id_qk, ks > 0);
+                    mma_commit(&bars.sfull[t][x]);
+                    if (b > 0) {
+                        ok = pv(b - 1);
+                        if (ok && ((b - 1) & 1)) mma_commit(&bars.kvempty[(g_kv + (b - 1) / 2) & 1]);
+                    }
+                }
+                if (ok && n_b > 0) {
+                    ok = pv(n_b - 1);
+                    if (ok) mma_commit(&bars.kvempty[(g_kv + (n_b - 1) / 2) & 1]);
+                }
+                // key/value blocks this tile does not need: release them once loaded
+                for (int kb = (n_b + 1) / 2; kb < it.n_kv && ok; ++kb) {
+                    const int G = g_kv + kb;
+                    ok = mbar_wait(&bars.kvfull[G & 1], (G >> 1) & 1, abort);
+                    if (ok) mma_commit(&bars.kvempty[G & 1]);
+                }
+                if (!ok) break;
+                g_kv += it.n_kv;
+                g_b += n_b;
+                // every generation warp has entered this item, so `done` cannot run a phase ahead of it
+                ok = mbar_wait(&bars.genin, j & 1, abort);
+                if (!ok) break;
+                mma_commit(&bars.done);
+                mma_commit(&bars.qempty[qb]);
             }
-            mma_commit(&bars.o);
-            mbar_wait(&bars.o, 0, abort);  // drain before the CTA may free tensor memory
+            // no MMA of this CTA may still read or write tensor memory when it is freed
+            mma_commit(&bars.drain[me]);
+            mbar_wait_issued(&bars.drain[me], 0);
         }
     } else {
         // ------------------------------------------------------------ generation / scores / epilogue
         const int t = warp / 4, qd = warp % 4;
         const int row = 32 * qd + lane;
-        const int tq = t0 + t * kQT + row;
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+        const uint32_t tO = tm + kTmO + 64 * t + lane_base;
+        const uint32_t tS = tm + kTmS + 128 * t + lane_base;
+        const uint32_t tP = tm + kTmP + 64 * t + lane_base;
+        const uint32_t tU = tm + kTmU + 64 * t + lane_base;
+        const uint32_t tA = tm + kTmA + 64 * t + lane_base;
+        uint32_t zero[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) zero[x] = 0u;
         // zero this thread's accumulator row; every MMA accumulates
-        {
-            uint32_t z[32];
+        tmem_st32(tO, zero);
+        tmem_st32(tO + 32, zero);
+        tmem_st_wait();
+        int n_inter = 0, g_b = 0, j = 0;
+        bool ok = true;
+        for (int i = i_begin; i < i_end && ok; ++i, ++j) {
+            const ReadItem it = read_item(i, n_ct, T, L, n_seg);
+            const int qb = j & 1;
+            if (lane == 0) mbar_arrive(&bars.genin);
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars.qfull[qb], (j >> 1) & 1, abort));
+            if (!ok) break;
+            uint32_t q2[32];
+            {
+                const uint8_t *qrow = sm + kSmItem + qb * kItemBytes + t * 16384 + row * 128;
 #pragma unroll
-            for (int x = 0; x < 32; ++x) z[x] = 0u;
-            tmem_st32(tm + kTmO + 64 * t + lane_base, z);
-            tmem_st32(tm + kTmO + 64 * t + 32 + lane_base, z);
-        }
-        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars.q, 0, abort));
-        uint32_t q2[32];
-        {
-            const uint8_t *qrow = sm + kSmQ + t * 16384 + row * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 x = *reinterpret_cast<const uint4 *>(qrow + ((c ^ (row & 7)) * 16));
-                q2[4 * c + 0] = x.x;
-                q2[4 * c + 1] = x.y;
-                q2[4 * c + 2] = x.z;
-                q2[4 * c + 3] = x.w;
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 x = *reinterpret_cast<const uint4 *>(qrow + ((c ^ (row & 7)) * 16));
+                    q2[4 * c + 0] = x.x;
+                    q2[4 * c + 1] = x.y;
+                    q2[4 * c + 2] = x.z;
+                    q2[4 * c + 3] = x.w;
+                }
             }
-        }
-        float den_inter = 0.f;
-        if (ok && inter) {
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars.u, 0, abort));
-            if (ok) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.qempty[qb]);
+            const int tq0 = it.t0 + kQT * t, tq = tq0 + row;
+            float den_inter = 0.f;
+            if (it.inter) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars.u, n_inter & 1, abort));
+                if (!ok) break;
                 tc_fence_after();
                 uint32_t u[32];
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tm + kTmP + 64 * t + lane_base + 32 * half, u);
+                    tmem_ld32(tU + 32 * half, u);
                     tmem_ld_wait();
 #pragma unroll
                     for (int x = 0; x < 16; ++x) {
@@ -784,65 +894,80 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                                          den_inter);
                     }
                 }
-                ok = GenLoop<0>::run(q2, bars, tm + kTmA + 64 * t + lane_base, abort);
+                ok = GenLoop<0>::run(q2, bars, tA, n_inter * kRStages, abort);
+                if (!ok) break;
+                ++n_inter;
             }
-        } else {
-            tmem_st_wait();  // the zeroed accumulator is ordered before the first P hand-off
-            tc_fence_before();
-        }
-        float l = 0.f;
-        const uint32_t tS = tm + kTmS + 128 * t + lane_base;
-        const uint32_t tP = tm + kTmP + 64 * t + lane_base;
-        for (int kb = 0; kb < n_kb && ok; ++kb) {
-            const int kbs = seg0 + kb * kKB;
-            if (kbs >= t0 + t * kQT + kQT) continue;
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfull[t], kb & 1, abort));
-            if (!ok) break;
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t r[32], p[16];
-                tmem_ld32(tS + 32 * c, r);
+            float l = 0.f;
+            const int n_b = read_tile_blocks(it, t, T);
+            for (int b = 0; b < n_b && ok; ++b) {
+                const int n = g_b + b, x = n & 1;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfull[t][x], (n >> 1) & 1, abort));
+                if (!ok) break;
+                tc_fence_after();
+                uint32_t r[64], p[32];
+                tmem_ld32(tS + 64 * x, r);
+                tmem_ld32(tS + 64 * x + 32, r + 32);
                 tmem_ld_wait();
+                const int kbs = it.seg0 + kSB * b;
+                if (kbs + kSB - 1 <= tq0) {  // every key of the block precedes every query of the tile
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    const int key = kbs + 32 * c + 2 * x;
-                    const float s0 = __uint_as_float(r[2 * x]), s1 = __uint_as_float(r[2 * x + 1]);
-                    const float w0 = key <= tq ? s0 * s0 : 0.f;
-                    const float w1 = key + 1 <= tq ? s1 * s1 : 0.f;
-                    l += w0 + w1;
-                    p[x] = pack_bf16x2(w0, w1);
-                }
-                tmem_st16(tP + 16 * c, p);
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&bars.pfull[t]);
-        }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.o, 0, abort));
-        if (ok) {
-            tc_fence_after();
-            const float den = l + den_inter;
-            const float inv = den == 0.f ? 0.f : 1.f / den;
-            uint32_t o[32];
-            uint4 *dst = reinterpret_cast<uint4 *>(out + ((long long)bh * T + tq) * kD);
+                    for (int y = 0; y < 32; ++y) {
+                        const float s0 = __uint_as_float(r[2 * y]), s1 = __uint_as_float(r[2 * y + 1]);
+                        const float w0 = s0 * s0, w1 = s1 * s1;
+                        l += w0 + w1;
+                        p[y] = pack_bf16x2(w0, w1);
+                    }
+                } else {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                tmem_ld32(tm + kTmO + 64 * t + lane_base + 32 * half, o);
-                tmem_ld_wait();
-                if (tq < T) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
-                        v.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
-                        v.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
-                        v.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
-                        dst[4 * half + c] = v;
+                    for (int y = 0; y < 32; ++y) {
+                        const int key = kbs + 2 * y;
+                        const float s0 = __uint_as_float(r[2 * y]), s1 = __uint_as_float(r[2 * y + 1]);
+                        const float w0 = key <= tq ? s0 * s0 : 0.f;
+                        const float w1 = key + 1 <= tq ? s1 * s1 : 0.f;
+                        l += w0 + w1;
+                        p[y] = pack_bf16x2(w0, w1);
                     }
                 }
+                // the weights of block n - 2 (same buffer) must have been consumed
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars.pempty[t][x], ((n >> 1) & 1) ^ 1, abort));
+                if (!ok) break;
+                tc_fence_after();
+                tmem_st32(tP + 32 * x, p);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&bars.pfull[t][x]);
+            }
+            if (!ok) break;
+            g_b += n_b;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars.done, j & 1, abort));
+            if (!ok) break;
+            tc_fence_after();
+            tmem_st_wait();
+            uint32_t o[64];
+            tmem_ld32(tO, o);
+            tmem_ld32(tO + 32, o + 32);
+            tmem_ld_wait();
+            // zero the accumulator for the next item (ordered before its first MMA by the
+            // tcgen05.st wait that precedes every hand-off to the issuers)
+            tmem_st32(tO, zero);
+            tmem_st32(tO + 32, zero);
+            const float den = l + den_inter;
+            const float inv = den == 0.f ? 0.f : 1.f / den;
+            if (tq < T) {
+                uint4 *dst = reinterpret_cast<uint4 *>(out + ((long long)it.bh * T + tq) * kD);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
+                    v.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
+                    v.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
+                    v.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
+                    dst[c] = v;
+                }
             }
         }
+        tmem_st_wait();
     }
 
     tc_fence_before();
@@ -949,9 +1074,13 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
                                              kSmAlloc);
         if (e != cudaSuccess) return e;
         const int n_ct = (p.T + kCtaQ - 1) / kCtaQ;
+        const long long n_items = (long long)n_ct * BH;
+        if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;
+        const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
         ProfScope ps("tc_read", st);
-        tc_read<<<(unsigned)(n_ct * BH), kReadThreads, kSmAlloc, st>>>(
-            mq, mk, mv, ms, static_cast<__nv_bfloat16 *>(out), p.T, p.L, p.n_seg, n_ct, status);
+        tc_read<<<(unsigned)grid, kReadThreads, kSmAlloc, st>>>(
+            mq, mk, mv, ms, static_cast<__nv_bfloat16 *>(out), p.T, p.L, p.n_seg, n_ct, (int)n_items,
+            status);
     }
     if (want_state) {
         const float *src = p.n_seg > 1 ? total : seg;

@@ -126,6 +126,26 @@ def test_multi_segment_f32_and_bf16(oracle_mod, dtype):
         full_check(oracle_mod, q, k, v, dtype, C)
 
 
+@pytest.mark.parametrize("T", [600, 2500, 1024 + 128])
+def test_many_heads_every_cta_walks_several_items(oracle_mod, T):
+    # More 256-query work items than streaming multiprocessors, so each
+    # persistent readout CTA runs several items back to back (barrier phases
+    # and accumulator zeroing carried across items), with ragged tails, an
+    # empty second query tile (T = 1152) and single-segment heads (T = 600).
+    B, H = 2, 80
+    q, k, v = inputs.make_qkv(B, H, T, 64, 64, "bf16", seed=T)
+    out, _, _ = run_forward(q, k, v, "bf16", 64)
+    rows = np.unique(np.concatenate([np.arange(0, T, 7), [T - 1]]))
+    BH = B * H
+    bh = np.repeat(np.arange(BH), len(rows))
+    tt = np.tile(rows, BH)
+    q64, k64, v64 = (inputs.widen(x, "bf16").reshape(BH, T, -1) for x in (q, k, v))
+    yref = oracle_mod.forward_rows(q64, k64, v64, bh, tt)
+    y = from_device(out).reshape(BH, T, -1)[bh, tt]
+    err = row_err(y, yref)
+    assert err <= TOL["bf16"], f"row-normwise error {err:.3e}"
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_zero_denominator_rows(oracle_mod, dtype):
     q, k, v = inputs.make_qkv(1, 2, 1500, 32, 32, dtype, seed=3)
