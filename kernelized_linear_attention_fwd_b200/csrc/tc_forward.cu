@@ -29,7 +29,7 @@ namespace {
 
 using namespace kata::sm100;
 
-constexpr long long kBf16PerSeg = (long long)kBf16Rows * kD;  // 172,032 bf16
+constexpr long long kBf16PerSeg = (long long)kBf16Rows * kD;  // 147,456 bf16
 
 // ---------------------------------------------------------------------------
 // Exclusive prefix over segments (the associative scan across chunk states)
@@ -62,11 +62,16 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
     const long long e0 = eb * 128 + 4 * lane;
     const float *base = seg_state + bh * (long long)n_seg * E + e0;
     __nv_bfloat16 *pbase = prefix + bh * (long long)n_seg * kBf16PerSeg;
-    // packed z: the thread's 4 rows lie in one half-strip (row i, columns j0..j0+3)
+    // packed z: the thread's 4 rows and their pairs (i, j); padding rows have i > j
     const bool z_part = e0 >= kZPacked0;
-    const int zr = (int)(e0 - kZPacked0);
-    const int zi = z_part ? hs_i(zr / 16) : 0;
-    const int zj = z_part ? hs_jb(zr / 16) + zr % 16 : 0;
+    const int zr = z_part ? (int)(e0 - kZPacked0) : 0;
+    int zi[4], zj[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+        const PairIJ pij = row_ij(zr + x);
+        zi[x] = pij.i;
+        zj[x] = pij.j;
+    }
     float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
 
     for (int g0 = 0; g0 < n_seg; g0 += kScanWarps * kScanRun) {
@@ -113,18 +118,18 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
                 o.y = pack_bf16x2(p.z, p.w);
                 *reinterpret_cast<uint2 *>(dst + e0) = o;
             } else {
-                // dense Z[i][j] and Z[j][i] as hi + lo bf16 (the mirrored entries of the
-                // diagonal half-strips carry identical values and write the same bits)
+                // dense Z[i][j] and Z[j][i] as hi + lo bf16
                 const float pv[4] = {p.x, p.y, p.z, p.w};
                 __nv_bfloat16 *zh = dst + (long long)kZHiRow0 * kD, *zl = dst + (long long)kZLoRow0 * kD;
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
+                    if (zi[x] > zj[x]) continue;
                     const __nv_bfloat16 hi = __float2bfloat16_rn(pv[x]);
                     const __nv_bfloat16 lo = __float2bfloat16_rn(pv[x] - __bfloat162float(hi));
-                    zh[zi * kD + zj + x] = hi;
-                    zl[zi * kD + zj + x] = lo;
-                    zh[(zj + x) * kD + zi] = hi;
-                    zl[(zj + x) * kD + zi] = lo;
+                    zh[zi[x] * kD + zj[x]] = hi;
+                    zl[zi[x] * kD + zj[x]] = lo;
+                    zh[zj[x] * kD + zi[x]] = hi;
+                    zl[zj[x] * kD + zi[x]] = lo;
                 }
             }
         }
@@ -134,7 +139,7 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
 }
 
 // ---------------------------------------------------------------------------
-// fp32 total (half-strip layout) -> dense state [64*64][64] and Z [64][64].
+// fp32 total (packed rows) -> dense state [64*64][64] and Z [64][64].
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__restrict__ state_out,
@@ -149,14 +154,12 @@ tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__r
         const int row = (int)(x / kD), e = (int)(x % kD);
         int i = row / kD, j = row % kD;
         if (i > j) { const int t = i; i = j; j = t; }
-        const int h = hs_index(i, j);
-        state_out[bh * kD * kD * kD + x] = src[((long long)h * 16 + (j - hs_jb(h))) * kD + e];
+        state_out[bh * kD * kD * kD + x] = src[(long long)row_index(i, j) * kD + e];
     } else {
         x -= (long long)kD * kD * kD;
         int i = (int)(x / kD), j = (int)(x % kD);
         if (i > j) { const int t = i; i = j; j = t; }
-        const int h = hs_index(i, j);
-        z_out[bh * kD * kD + x] = src[kZPacked0 + (long long)h * 16 + (j - hs_jb(h))];
+        z_out[bh * kD * kD + x] = src[kZPacked0 + row_index(i, j)];
     }
 }
 
@@ -185,11 +188,11 @@ constexpr int kTiles = 2;                // query tiles per item
 constexpr int kCtaQ = kQT * kTiles;      // 256 queries per item
 constexpr int kKB = 128;                 // key/value block loaded by TMA
 constexpr int kSB = 64;                  // score block (MMA N of Q K^T)
-constexpr int kRHs = 8;                  // half-strips per inter stage (128 state rows)
-constexpr int kRStages = kHalfStrips / kRHs;  // 20
+constexpr int kRKs = 8;                  // 16-row K-steps per inter stage (128 state rows)
+constexpr int kRStages = kStateRows / (16 * kRKs);  // 17
 constexpr int kRRing = 3;                // inter A ring depth (tensor memory)
 constexpr int kRBRing = 4;               // inter B ring depth (state-prefix tiles, shared memory)
-constexpr int kRStageBytes = kRHs * 16 * 128;   // bf16 state-prefix rows per stage
+constexpr int kRStageBytes = kRKs * 16 * 128;   // bf16 state-prefix rows per stage
 constexpr int kTmaWarp = 8;
 constexpr int kIssuer0 = 9;
 constexpr int kReadThreads = 352;
@@ -245,65 +248,103 @@ __device__ __forceinline__ int read_tile_blocks(const ReadItem &it, int t, int T
     return (min(q0 + kQT, T) - it.seg0 + kSB - 1) / kSB;
 }
 
-__device__ __forceinline__ uint32_t dup_lo(uint32_t x) { return __byte_perm(x, 0, 0x1010); }
-__device__ __forceinline__ uint32_t dup_hi(uint32_t x) { return __byte_perm(x, 0, 0x3232); }
+// q_x duplicated into both halves of a bf16 pair.
+template <int X>
+__device__ __forceinline__ uint32_t dup_q(const uint32_t (&q2)[32]) {
+    return __byte_perm(q2[X / 2], 0, (X & 1) ? 0x3232 : 0x1010);
+}
 
-// phi(q) weights for the 16 rows of half-strip H: c_ij q_i q_j with c = 2 for
-// j > i, 1 for j = i, 0 for j < i (mirrored entries), packed two rows per
-// 32-bit word (tensor-memory A layout: row pair (2p, 2p+1) in column p).
-template <int H>
-__device__ __forceinline__ void gen_halfstrip(const uint32_t (&q2)[32], uint32_t *out) {
-    constexpr int i = hs_i(H);
-    constexpr int jb = hs_jb(H);
-    const uint32_t qi = (i & 1) ? dup_hi(q2[i / 2]) : dup_lo(q2[i / 2]);
-    const uint32_t qi2 = mul_bf16x2(qi, 0x40004000u);  // 2 q_i, exact
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-        const int j0 = jb + 2 * p, j1 = j0 + 1;
-        if (j1 < i) {
-            out[p] = 0u;
-        } else if (j0 > i) {
-            out[p] = mul_bf16x2(qi2, q2[j0 / 2]);
-        } else if (j0 == i) {
-            out[p] = mul_bf16x2(__byte_perm(qi, qi2, 0x7610), q2[j0 / 2]);  // (1, 2)
-        } else {  // j1 == i
-            out[p] = mul_bf16x2(qi & 0xFFFF0000u, q2[j0 / 2]);  // (0, 1)
-        }
+__host__ __device__ constexpr uint32_t bf16_small(int c) { return c == 2 ? 0x4000u : c == 1 ? 0x3F80u : 0u; }
+__host__ __device__ constexpr int pair_weight(PairIJ p) { return p.i < p.j ? 2 : p.i == p.j ? 1 : 0; }
+
+// Word of phi(q) holding state rows R and R + 1 (tensor-memory A layout: row
+// pair (2p, 2p+1) in column p): c_ij q_i q_j for both rows, c = 2 for i < j,
+// 1 for i = j, 0 for padding rows.  The layout makes the word q_i (q_j,
+// q_j+1) or (q_i, q_i+1) q_j, one bf16x2 product; a common factor 2 is put on
+// the duplicated operand (exact), other weights multiply the product (exact).
+template <int R>
+__device__ __forceinline__ uint32_t gen_word(const uint32_t (&q2)[32]) {
+    constexpr PairIJ a = row_ij(R), b = row_ij(R + 1);
+    constexpr int c0 = pair_weight(a), c1 = pair_weight(b);
+    static_assert((a.i == b.i && b.j == a.j + 1 && a.j % 2 == 0) ||
+                      (a.j == b.j && b.i == a.i + 1 && a.i % 2 == 0),
+                  "state rows of one word must share i or j");
+    constexpr bool share_i = a.i == b.i;
+    if constexpr (c0 == 0 && c1 == 0) {
+        return 0u;
+    } else {
+        uint32_t dup = share_i ? dup_q<a.i>(q2) : dup_q<a.j>(q2);
+        const uint32_t pr = share_i ? q2[a.j / 2] : q2[a.i / 2];
+        if constexpr (c0 == 2 && c1 == 2) dup = mul_bf16x2(dup, 0x40004000u);
+        uint32_t w = mul_bf16x2(dup, pr);
+        if constexpr (!(c0 == 2 && c1 == 2) && !(c0 == 1 && c1 == 1))
+            w = mul_bf16x2(w, bf16_small(c0) | (bf16_small(c1) << 16));
+        return w;
     }
 }
 
-// Generates the 20 inter stages of one item into the A ring.  `g0` is the
-// number of stages generated before this item (ring slot and phase).
+// The 8 words of K-step K (state rows 16 K .. 16 K + 15).
+template <int K>
+__device__ __forceinline__ void gen_kstep(const uint32_t (&q2)[32], uint32_t *out) {
+    out[0] = gen_word<16 * K + 0>(q2);
+    out[1] = gen_word<16 * K + 2>(q2);
+    out[2] = gen_word<16 * K + 4>(q2);
+    out[3] = gen_word<16 * K + 6>(q2);
+    out[4] = gen_word<16 * K + 8>(q2);
+    out[5] = gen_word<16 * K + 10>(q2);
+    out[6] = gen_word<16 * K + 12>(q2);
+    out[7] = gen_word<16 * K + 14>(q2);
+}
+
+// First half (K-steps 0-3) of inter stage ST.
+template <int ST>
+__device__ __forceinline__ void gen_stage_lo(const uint32_t (&q2)[32], uint32_t (&x)[32]) {
+    gen_kstep<kRKs * ST + 0>(q2, x);
+    gen_kstep<kRKs * ST + 1>(q2, x + 8);
+    gen_kstep<kRKs * ST + 2>(q2, x + 16);
+    gen_kstep<kRKs * ST + 3>(q2, x + 24);
+}
+
+// Generates the inter stages of one item into the A ring, software-pipelined:
+// the first half of stage ST (`x`) was generated before its slot frees up;
+// while the tensor-memory stores of stage ST are in flight, the first half of
+// stage ST + 1 is generated.  `g0` is the number of stages generated before
+// this item (ring slot and phase).
 template <int ST>
 struct GenLoop {
     __device__ __forceinline__ static bool run(const uint32_t (&q2)[32], ReadBars &bars,
-                                               uint32_t ta_tile, int g0, volatile int *abort) {
+                                               uint32_t ta_tile, int g0, volatile int *abort,
+                                               const uint32_t (&x)[32]) {
         const int G = g0 + ST;
         const int s = G % kRRing;
         if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[s], ((G / kRRing) & 1) ^ 1, abort)))
             return false;
         tc_fence_after();
-        uint32_t a[32];
-        gen_halfstrip<kRHs * ST + 0>(q2, a);
-        gen_halfstrip<kRHs * ST + 1>(q2, a + 8);
-        gen_halfstrip<kRHs * ST + 2>(q2, a + 16);
-        gen_halfstrip<kRHs * ST + 3>(q2, a + 24);
-        tmem_st32(ta_tile + 128 * s, a);
-        gen_halfstrip<kRHs * ST + 4>(q2, a);
-        gen_halfstrip<kRHs * ST + 5>(q2, a + 8);
-        gen_halfstrip<kRHs * ST + 6>(q2, a + 16);
-        gen_halfstrip<kRHs * ST + 7>(q2, a + 24);
-        tmem_st32(ta_tile + 128 * s + 32, a);
+        tmem_st32(ta_tile + 128 * s, x);
+        {
+            uint32_t y[16];
+            gen_kstep<kRKs * ST + 4>(q2, y);
+            gen_kstep<kRKs * ST + 5>(q2, y + 8);
+            tmem_st16(ta_tile + 128 * s + 32, y);
+        }
+        {
+            uint32_t y[16];
+            gen_kstep<kRKs * ST + 6>(q2, y);
+            gen_kstep<kRKs * ST + 7>(q2, y + 8);
+            tmem_st16(ta_tile + 128 * s + 48, y);
+        }
+        uint32_t xn[32];
+        if constexpr (ST + 1 < kRStages) gen_stage_lo<ST + 1>(q2, xn);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars.afull[s]);
-        return GenLoop<ST + 1>::run(q2, bars, ta_tile, g0, abort);
+        return GenLoop<ST + 1>::run(q2, bars, ta_tile, g0, abort, xn);
     }
 };
 template <>
 struct GenLoop<kRStages> {
     __device__ __forceinline__ static bool run(const uint32_t (&)[32], ReadBars &, uint32_t, int,
-                                               volatile int *) {
+                                               volatile int *, const uint32_t (&)[32]) {
         return true;
     }
 };
@@ -361,45 +402,136 @@ k_transpose(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ kt,
 // ---------------------------------------------------------------------------
 // State builder on tcgen05 (persistent: one CTA per SM loops over work items).
 //
-// Work item = (head, segment, c), c = 0..4; item c accumulates the 4 tiles of
-// 128 state rows (half-strips h = 32 c + 8 m + s, m = tile, s = 16-lane slot)
-// over the segment's tokens:  D[m] += A[m] . [V | 1]  with
+// Work item = (head, segment, c), c = 0..4; item c accumulates its state
+// tiles (4 tiles for c < 4, the single tile 16 for c = 4; rows as laid out in
+// tc_layout.cuh) over the segment's tokens:  D[m] += A[m] . [V | 1]  with
 // A[m][(i, j)][token] = k_i k_j generated from the transposed keys into tensor
 // memory by the thread owning the row's lane, and the MN-major B operand
 // [V | 1] = the value tile (64 columns) followed by a constant block whose
 // first column is one, so column 64 of D accumulates the packed normaliser
 // z = sum k_i k_j (N = 80; an N = 64 MMA costs the same issue time).
 // Roles: warps 0-3 / 4-7 generate the first / second 16-token step of every
-// 32-token stage and run the epilogue; warp 8 is the TMA producer; warps 9
-// and 10 issue the MMAs of alternate stages.  Barrier phases run on across
-// items, so the next item's tiles load while the current one is written back.
+// 32-token stage (software-pipelined: the next stage's products are formed
+// while this stage's tensor-memory stores are in flight) and drain the
+// accumulators into swizzled shared memory; warp 8 is the TMA producer;
+// warps 9 and 10 issue the MMAs of alternate stages; warp 11 writes the
+// drained tiles back with TMA stores, so the next item's MMAs start as soon as
+// the accumulators are read.  Barrier phases run on across items.
 // Accumulators are zeroed by tcgen05.st and every MMA accumulates.
 // ---------------------------------------------------------------------------
-constexpr int kBCtas = 5;
-constexpr int kBTiles = 4;
+constexpr int kBTiles = 4;                // accumulator tiles (the most an item uses)
 constexpr int kBN = 80;                   // MMA N: 64 values, the ones column, 15 zero columns
 constexpr int kBTok = 64;                 // tokens per TMA tile (2 stages)
-constexpr int kBTileRing = 6;
+constexpr int kBTileRing = 5;
 constexpr int kBTileBytes = 2 * 8192;     // K^T tile, V tile
 constexpr int kBOnes = kBTileRing * kBTileBytes;   // ones block [64 x 64] bf16, swizzled
-constexpr int kBStage = kBOnes + 8192;             // epilogue staging, 8 warps x 32 rows x 68 floats
-constexpr int kBSmAlloc = kBStage + 8 * 32 * 68 * 4 + 1024;
+constexpr int kBStage = kBOnes + 8192;             // staging: tile m, half h at + (2 m + h) * 16 KB
+constexpr int kBStageBox = 16384;                  // [128 rows x 32 fp32], 128-byte swizzle
+constexpr int kBSmAlloc = kBStage + 2 * kBTiles * kBStageBox + 1024;
 constexpr int kBARing = 3;                // A stages in tensor memory
 constexpr int kBTmaWarp = 8;
 constexpr int kBIssuer0 = 9;
-constexpr int kBuildThreads = 352;
+constexpr int kBStoreWarp = 11;
+constexpr int kBuildThreads = 384;
 constexpr uint32_t kBTmA = kBTiles * kBN; // 320: A slot s at 320 + 64 s, step kk at + 32 kk
 
 struct BuildBars {
     uint64_t tfull[kBTileRing], tempty[kBTileRing];
     uint64_t afull[kBARing], aempty[kBARing];
-    uint64_t done;
+    uint64_t done, staged, sfree;
+    uint64_t drain[2];
 };
+
+// Products k_i k_j of one 16-token step (this warpgroup's half of a 32-token
+// stage) for the thread's NT rows: p[8 m + w] holds tokens 2 w, 2 w + 1.
+template <int NT>
+__device__ __forceinline__ void build_products(const uint8_t *kt, int half, int wg, int jcol,
+                                               const int (&im)[kBTiles], uint32_t (&p)[8 * NT]) {
+    const int c0 = 4 * half + 2 * wg, c1 = c0 + 1;  // 16-byte chunks of this warpgroup's 16 tokens
+    uint32_t own[8];
+    {
+        const uint8_t *r = kt + jcol * 128;
+        const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (jcol & 7)) * 16));
+        const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (jcol & 7)) * 16));
+        own[0] = x0.x; own[1] = x0.y; own[2] = x0.z; own[3] = x0.w;
+        own[4] = x1.x; own[5] = x1.y; own[6] = x1.z; own[7] = x1.w;
+    }
+#pragma unroll
+    for (int m = 0; m < NT; ++m) {
+        const int i = im[m];
+        const uint8_t *r = kt + i * 128;
+        const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (i & 7)) * 16));
+        const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (i & 7)) * 16));
+        p[8 * m + 0] = mul_bf16x2(own[0], x0.x); p[8 * m + 1] = mul_bf16x2(own[1], x0.y);
+        p[8 * m + 2] = mul_bf16x2(own[2], x0.z); p[8 * m + 3] = mul_bf16x2(own[3], x0.w);
+        p[8 * m + 4] = mul_bf16x2(own[4], x1.x); p[8 * m + 5] = mul_bf16x2(own[5], x1.y);
+        p[8 * m + 6] = mul_bf16x2(own[6], x1.z); p[8 * m + 7] = mul_bf16x2(own[7], x1.w);
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ void build_store(uint32_t taddr, const uint32_t (&p)[8 * NT]) {
+    if constexpr (NT == 4) tmem_st32(taddr, p);
+    else tmem_st8(taddr, p);
+}
+
+// Generation side of one item: 2 stages per 64-token tile.  `tt` is the
+// CTA's running tile counter (ring slot and phase), advanced past the item.
+template <int NT>
+__device__ __forceinline__ bool build_item_gen(BuildBars &bars, const uint8_t *sm, uint32_t ta, int wg,
+                                               int jcol, const int (&im)[kBTiles], int &tt, int n_tt,
+                                               volatile int *abort) {
+    uint32_t pa[8 * NT], pb[8 * NT];
+    {
+        const int b = tt % kBTileRing;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.tfull[b], (tt / kBTileRing) & 1, abort))) return false;
+        build_products<NT>(sm + b * kBTileBytes, 0, wg, jcol, im, pa);
+    }
+    for (int t = 0; t < n_tt; ++t, ++tt) {
+        const int b = tt % kBTileRing;
+        int G = 2 * tt, a = G % kBARing;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((G / kBARing) & 1) ^ 1, abort)))
+            return false;
+        tc_fence_after();
+        build_store<NT>(ta + 64 * a, pa);
+        build_products<NT>(sm + b * kBTileBytes, 1, wg, jcol, im, pb);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars.afull[a]);
+
+        G = 2 * tt + 1;
+        a = G % kBARing;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((G / kBARing) & 1) ^ 1, abort)))
+            return false;
+        tc_fence_after();
+        build_store<NT>(ta + 64 * a, pb);
+        if (t + 1 < n_tt) {
+            const int bn = (tt + 1) % kBTileRing;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars.tfull[bn], ((tt + 1) / kBTileRing) & 1, abort)))
+                return false;
+            build_products<NT>(sm + bn * kBTileBytes, 0, wg, jcol, im, pa);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars.afull[a]);
+    }
+    return true;
+}
+
+__device__ __forceinline__ void build_item_geom(int item, int n_build, int T, int L, int &c, int &g, int &bh,
+                                                int &s0, int &n_tt) {
+    c = item % kBuildItems;
+    const int rest = item / kBuildItems;
+    g = rest % n_build;
+    bh = rest / n_build;
+    s0 = g * L;
+    n_tt = (min(L, T - s0) + kBTok - 1) / kBTok;
+}
 
 __global__ void __launch_bounds__(kBuildThreads, 1)
 tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_v,
-         float *__restrict__ seg_state, int T, int L, int n_seg, int n_build, int n_items,
-         int *status) {
+         const __grid_constant__ CUtensorMap tm_st, float *__restrict__ seg_state, int T, int L,
+         int n_seg, int n_build, int n_items, int *status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ BuildBars bars;
     __shared__ uint32_t tmem_base;
@@ -419,6 +551,10 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             mbar_init(&bars.aempty[x], 1);
         }
         mbar_init(&bars.done, 2);
+        mbar_init(&bars.staged, 256);
+        mbar_init(&bars.sfree, 1);
+        mbar_init(&bars.drain[0], 1);
+        mbar_init(&bars.drain[1], 1);
         fence_mbarrier_init();
     }
     // constant ones block: logical column 0 of each of the 64 rows is 1.0
@@ -437,17 +573,8 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
     const uint32_t tm = tmem_base;
     volatile int *abort = &abort_flag;
 
-    // item -> (c, g, bh, token range)
-    auto item_geom = [&](int item, int &c, int &g, int &bh, int &s0, int &n_tt) {
-        c = item % kBCtas;
-        const int rest = item / kBCtas;
-        g = rest % n_build;
-        bh = rest / n_build;
-        s0 = g * L;
-        n_tt = (min(L, T - s0) + kBTok - 1) / kBTok;
-    };
-
     if (warp == kBTmaWarp) {
+        // ------------------------------------------------------------ producer
         if (lane == 0) {
             tma_prefetch_desc(&tm_kt);
             tma_prefetch_desc(&tm_v);
@@ -455,7 +582,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 int c, g, bh, s0, n_tt;
-                item_geom(item, c, g, bh, s0, n_tt);
+                build_item_geom(item, n_build, T, L, c, g, bh, s0, n_tt);
                 for (int t = 0; t < n_tt; ++t, ++tt) {
                     const int b = tt % kBTileRing;
                     ok = mbar_wait(&bars.tempty[b], ((tt / kBTileRing) & 1) ^ 1, abort);
@@ -467,18 +594,20 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
                 }
             }
             for (int t = (tt > kBTileRing ? tt - kBTileRing : 0); t < tt; ++t)
-                mbar_wait(&bars.tfull[t % kBTileRing], (t / kBTileRing) & 1, abort);
+                mbar_wait_issued(&bars.tfull[t % kBTileRing], (t / kBTileRing) & 1);
         }
     } else if (warp == kBIssuer0 || warp == kBIssuer0 + 1) {
+        // ------------------------------------------------------------ MMA issuers
         if (lane == 0) {
             const int me = warp - kBIssuer0;
             const uint32_t idesc = idesc_bf16(128, kBN, 0, 1);
             const uint32_t sbase = smem_u32(sm);
-            int tt = 0, j = 0;  // global tile counter, local item counter
+            int tt = 0;  // global tile counter
             bool ok = true;
-            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 int c, g, bh, s0, n_tt;
-                item_geom(item, c, g, bh, s0, n_tt);
+                build_item_geom(item, n_build, T, L, c, g, bh, s0, n_tt);
+                const int nt = build_item_tiles(c);
                 for (int t = 0; t < n_tt && ok; ++t, ++tt) {
                     const int G = 2 * tt + me;  // global stage: this issuer takes one half of each tile
                     const int b = tt % kBTileRing, a = G % kBARing;
@@ -494,111 +623,100 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
                     for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
                         for (int m = 0; m < kBTiles; ++m)
-                            mma_ts(tm + kBN * m, ta + 32 * kk + 8 * m, desc_add(dv, 2048 * kk), idesc, 1);
+                            if (m < nt)
+                                mma_ts(tm + kBN * m, ta + 32 * kk + 8 * m, desc_add(dv, 2048 * kk), idesc, 1);
                     mma_commit(&bars.aempty[a]);
                     mma_commit(&bars.tempty[b]);
                 }
-                mma_commit(&bars.done);  // this item's accumulation complete (with the other issuer)
+                if (ok) mma_commit(&bars.done);  // this item's accumulation complete (with the other issuer)
             }
-            mbar_wait(&bars.done, (j - 1) & 1, abort);  // drain before the CTA may free tensor memory
+            // no MMA of this CTA may still read or write tensor memory when it is freed
+            mma_commit(&bars.drain[me]);
+            mbar_wait_issued(&bars.drain[me], 0);
+        }
+    } else if (warp == kBStoreWarp) {
+        // ------------------------------------------------------------ write-back of drained tiles
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_st);
+            int j = 0;
+            for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
+                int c, g, bh, s0, n_tt;
+                build_item_geom(item, n_build, T, L, c, g, bh, s0, n_tt);
+                if (!mbar_wait(&bars.staged, j & 1, abort)) break;
+                for (int m = 0; m < build_item_tiles(c); ++m)
+                    for (int h = 0; h < 2; ++h)
+                        tma_store_3d(&tm_st, sm + kBStage + (2 * m + h) * kBStageBox, 32 * h,
+                                     128 * build_item_tile(c, m), bh * n_seg + g);
+                bulk_commit_group();
+                bulk_wait_read_all();
+                mbar_arrive(&bars.sfree);
+            }
+            bulk_wait_all();
         }
     } else {
+        // ------------------------------------------------------------ generation / drain
         const int wg = warp / 4, qd = warp % 4;
         const int row = 32 * qd + lane;          // lane within the 128-row tile
-        const int slot = row / 16, jj = row % 16;
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
-        float *stage = reinterpret_cast<float *>(sm + kBStage) + warp * (32 * 68);
+        uint32_t zero[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) zero[x] = 0u;
+        // zero this warpgroup's accumulators (tiles 2 wg, 2 wg + 1; 80 columns each)
+        auto zero_acc = [&]() {
+#pragma unroll
+            for (int m = 2 * wg; m < 2 * wg + 2; ++m) {
+                tmem_st32(tm + kBN * m + lane_base, zero);
+                tmem_st32(tm + kBN * m + 32 + lane_base, zero);
+                tmem_st16(tm + kBN * m + 64 + lane_base, zero);
+            }
+        };
+        zero_acc();
         int tt = 0, j = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
             int c, g, bh, s0, n_tt;
-            item_geom(item, c, g, bh, s0, n_tt);
-            const int jcol = hs_jb(32 * c + slot) + jj;
-            int im[kBTiles];
+            build_item_geom(item, n_build, T, L, c, g, bh, s0, n_tt);
+            const int nt = build_item_tiles(c);
+            int im[kBTiles], jcol = 0;
 #pragma unroll
-            for (int m = 0; m < kBTiles; ++m) im[m] = hs_i(32 * c + 8 * m + slot);
-            {   // zero the accumulators (warpgroup 0: tiles 0, 1; warpgroup 1: tiles 2, 3)
-                uint32_t z[32];
-#pragma unroll
-                for (int x = 0; x < 32; ++x) z[x] = 0u;
-#pragma unroll
-                for (int x = 0; x < 5; ++x) tmem_st32(tm + 2 * kBN * wg + 32 * x + lane_base, z);
+            for (int m = 0; m < kBTiles; ++m) {
+                const PairIJ pij = row_ij(128 * build_item_tile(c, m < nt ? m : 0) + row);
+                im[m] = pij.i;
+                jcol = pij.j;  // the same for every tile of the item
             }
-            for (int t = 0; t < n_tt && ok; ++t, ++tt) {
-                const int b = tt % kBTileRing;
-                for (int half = 0; half < 2 && ok; ++half) {
-                    const int G = 2 * tt + half, a = G % kBARing;
-                    ok = __all_sync(0xffffffffu,
-                                    mbar_wait(&bars.tfull[b], (tt / kBTileRing) & 1, abort) &&
-                                        mbar_wait(&bars.aempty[a], ((G / kBARing) & 1) ^ 1, abort));
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint8_t *kt = sm + b * kBTileBytes;  // row d: 64 tokens, swizzled
-                    const int c0 = 4 * half + 2 * wg, c1 = c0 + 1;  // this warpgroup's 16 tokens
-                    uint32_t own[8];
-                    {
-                        const uint8_t *r = kt + jcol * 128;
-                        const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (jcol & 7)) * 16));
-                        const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (jcol & 7)) * 16));
-                        own[0] = x0.x; own[1] = x0.y; own[2] = x0.z; own[3] = x0.w;
-                        own[4] = x1.x; own[5] = x1.y; own[6] = x1.z; own[7] = x1.w;
-                    }
-                    uint32_t p[32];
-#pragma unroll
-                    for (int m = 0; m < kBTiles; ++m) {
-                        const int i = im[m];
-                        const uint8_t *r = kt + i * 128;
-                        const uint4 x0 = *reinterpret_cast<const uint4 *>(r + ((c0 ^ (i & 7)) * 16));
-                        const uint4 x1 = *reinterpret_cast<const uint4 *>(r + ((c1 ^ (i & 7)) * 16));
-                        p[8 * m + 0] = mul_bf16x2(own[0], x0.x); p[8 * m + 1] = mul_bf16x2(own[1], x0.y);
-                        p[8 * m + 2] = mul_bf16x2(own[2], x0.z); p[8 * m + 3] = mul_bf16x2(own[3], x0.w);
-                        p[8 * m + 4] = mul_bf16x2(own[4], x1.x); p[8 * m + 5] = mul_bf16x2(own[5], x1.y);
-                        p[8 * m + 6] = mul_bf16x2(own[6], x1.z); p[8 * m + 7] = mul_bf16x2(own[7], x1.w);
-                    }
-                    tmem_st32(tm + kBTmA + 64 * a + 32 * wg + lane_base, p);
-                    tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(&bars.afull[a]);
-                }
-            }
+            const uint32_t ta = tm + kBTmA + 32 * wg + lane_base;
+            ok = nt == kBTiles ? build_item_gen<kBTiles>(bars, sm, ta, wg, jcol, im, tt, n_tt, abort)
+                               : build_item_gen<1>(bars, sm, ta, wg, jcol, im, tt, n_tt, abort);
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.done, j & 1, abort));
+            if (ok && j > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfree, (j - 1) & 1, abort));
             if (!ok) break;
-            // Epilogue.  Tile m holds 128 consecutive state rows in lane order
-            // (half-strips 32 c + 8 m .. + 7) and their packed z in column 64:
-            // stage each warp's 32 rows in shared memory (rows of 68 floats,
-            // conflict-free) and write them back two rows (512 contiguous bytes)
-            // per store.  Warpgroup 0 writes tiles 0, 1, warpgroup 1 tiles 2, 3.
+            // Drain: tile m's 128 rows go to shared memory as two [128 x 32] fp32
+            // boxes in the 128-byte swizzle of the store's tensor map (16-byte
+            // chunk c of row r at chunk c ^ (r % 8): conflict-free), its packed z
+            // (column 64) straight to global memory.
             tc_fence_after();
-            float *base = seg_state + ((long long)bh * n_seg + g) * kF32PerSeg;
-#pragma unroll 1
-            for (int m = 2 * wg; m < 2 * wg + 2; ++m) {
-                const long long row0 = (long long)16 * (32 * c + 8 * m) + 32 * qd;
+            float *zbase = seg_state + ((long long)bh * n_seg + g) * kF32PerSeg + kZPacked0;
+            for (int m = 2 * wg; m < 2 * wg + 2 && m < nt; ++m) {
                 uint32_t o[32];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    tmem_ld32(tm + kBN * m + lane_base + 32 * hh, o);
+                for (int h = 0; h < 2; ++h) {
+                    tmem_ld32(tm + kBN * m + 32 * h + lane_base, o);
                     tmem_ld_wait();
+                    uint8_t *box = sm + kBStage + (2 * m + h) * kBStageBox + row * 128;
 #pragma unroll
                     for (int x = 0; x < 8; ++x)
-                        *reinterpret_cast<float4 *>(stage + lane * 68 + 32 * hh + 4 * x) =
-                            make_float4(__uint_as_float(o[4 * x]), __uint_as_float(o[4 * x + 1]),
-                                        __uint_as_float(o[4 * x + 2]), __uint_as_float(o[4 * x + 3]));
+                        *reinterpret_cast<uint4 *>(box + ((x ^ (row & 7)) * 16)) =
+                            make_uint4(o[4 * x], o[4 * x + 1], o[4 * x + 2], o[4 * x + 3]);
                 }
                 tmem_ld8(tm + kBN * m + 64 + lane_base, o);
                 tmem_ld_wait();
-                base[kZPacked0 + row0 + lane] = __uint_as_float(o[0]);
-                __syncwarp();
-                float *dst = base + row0 * kD;
-#pragma unroll
-                for (int it = 0; it < 16; ++it) {
-                    const int r = 2 * it + lane / 16, ch = lane % 16;
-                    *reinterpret_cast<float4 *>(dst + r * kD + 4 * ch) =
-                        *reinterpret_cast<const float4 *>(stage + r * 68 + 4 * ch);
-                }
-                __syncwarp();
+                zbase[128 * build_item_tile(c, m) + row] = __uint_as_float(o[0]);
             }
-            tc_fence_before();  // accumulator reads ordered before the next item's zeroing
+            fence_proxy_async_smem();
+            mbar_arrive(&bars.staged);
+            zero_acc();  // ordered before the next item's first MMA by the hand-off's tcgen05.st wait
         }
+        tmem_st_wait();
     }
 
     tc_fence_before();
@@ -692,7 +810,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     mbar_arrive_expect_tx(&bars.bfull[s], kRStageBytes);
                     for (int bx = 0; bx < kRStageBytes / 4096; ++bx)
                         tma_load_3d(sm + kSmS + s * kRStageBytes + 4096 * bx, &tm_s, &bars.bfull[s], 0,
-                                    16 * kRHs * st + 32 * bx, it.sidx);
+                                    16 * kRKs * st + 32 * bx, it.sidx);
                     ++n_bs;
                 }
                 for (int kb = 0; kb < it.n_kv && ok; ++kb) {
@@ -777,7 +895,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                         const uint32_t ta = tm + kTmA + 128 * s;
                         const uint64_t db = desc_add(dS, kRStageBytes * sb);
 #pragma unroll
-                        for (int ks = 0; ks < kRHs; ++ks) {
+                        for (int ks = 0; ks < kRKs; ++ks) {
                             mma_ts(tm + kTmO, ta + 8 * ks, desc_add(db, 2048 * ks), id_n64, 1);
                             mma_ts(tm + kTmO + 64, ta + 64 + 8 * ks, desc_add(db, 2048 * ks), id_n64, 1);
                         }
@@ -894,7 +1012,9 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                                          den_inter);
                     }
                 }
-                ok = GenLoop<0>::run(q2, bars, tA, n_inter * kRStages, abort);
+                uint32_t x0[32];
+                gen_stage_lo<0>(q2, x0);
+                ok = GenLoop<0>::run(q2, bars, tA, n_inter * kRStages, abort, x0);
                 if (!ok) break;
                 ++n_inter;
             }
@@ -1005,9 +1125,9 @@ int num_sms() {
 }
 
 // Workspace of the tensor-core path (bytes; 256-aligned parts):
-//   fp32 segment states  BH * n_seg * 2624 * 64 * 4
-//   fp32 total           BH * 2624 * 64 * 4
-//   bf16 prefixes        BH * n_seg * 2688 * 64 * 2
+//   fp32 segment states  BH * n_seg * 2176 * 65 * 4   (state rows, then packed z)
+//   fp32 total           BH * 2176 * 65 * 4
+//   bf16 prefixes        BH * n_seg * 2304 * 64 * 2
 //   transposed keys      BH * 64 * T_pad * 2      (T_pad = T rounded up to 64)
 void plan_tc_workspace(Plan &p) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
@@ -1043,22 +1163,26 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
             k_transpose<<<(unsigned)((T_pad / 64) * BH), 256, 0, st>>>(
                 static_cast<const __nv_bfloat16 *>(k), kt, p.T, T_pad);
         }
-        CUtensorMap mkt, mvb;
+        CUtensorMap mkt, mvb, mst;
         const uint64_t dkt[3] = {(uint64_t)T_pad, (uint64_t)kD, (uint64_t)BH};
         const uint64_t skt[2] = {(uint64_t)T_pad * 2, (uint64_t)kD * T_pad * 2};
         const uint32_t bkt[3] = {64, 64, 1};
         const uint64_t dqkv[3] = {(uint64_t)kD, (uint64_t)p.T, (uint64_t)BH};
         const uint64_t sqkv[2] = {(uint64_t)kD * 2, (uint64_t)p.T * kD * 2};
         const uint32_t b64[3] = {64, 64, 1};
-        if (!make_tmap_bf16(&mkt, kt, 3, dkt, skt, bkt) || !make_tmap_bf16(&mvb, v, 3, dqkv, sqkv, b64))
+        const uint64_t dst[3] = {(uint64_t)kD, (uint64_t)kStateRows, (uint64_t)(BH * p.n_seg)};
+        const uint64_t sst[2] = {(uint64_t)kD * 4, (uint64_t)kF32PerSeg * 4};
+        const uint32_t bst[3] = {32, 128, 1};
+        if (!make_tmap_bf16(&mkt, kt, 3, dkt, skt, bkt) || !make_tmap_bf16(&mvb, v, 3, dqkv, sqkv, b64) ||
+            !make_tmap(&mst, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, seg, 3, dst, sst, bst))
             return cudaErrorInvalidValue;
         cudaError_t e = cudaFuncSetAttribute(tc_build, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kBSmAlloc);
         if (e != cudaSuccess) return e;
-        const long long n_items = (long long)kBCtas * n_build * BH;
+        const long long n_items = (long long)kBuildItems * n_build * BH;
         const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
         ProfScope ps("tc_build", st);
-        tc_build<<<(unsigned)grid, kBuildThreads, kBSmAlloc, st>>>(mkt, mvb, seg, p.T, p.L, p.n_seg,
+        tc_build<<<(unsigned)grid, kBuildThreads, kBSmAlloc, st>>>(mkt, mvb, mst, seg, p.T, p.L, p.n_seg,
                                                                     n_build, (int)n_items, status);
     }
     if (p.n_seg > 1) {

@@ -1,53 +1,104 @@
 // Layout of the tensor-core path's per-segment state (d = dv = 64).
 //
-// The packed feature rows are grouped in 16-row "half-strips": half-strip h
-// holds the rows (i, j) for one i and j = jb .. jb + 15 (jb a multiple of 16).
-// Only half-strips that contain some j >= i are kept: for jb = 16 b, i runs
-// over 0 .. 16 b + 15, giving 16 + 32 + 48 + 64 = 160 half-strips = 2560 rows
-// (the 2080 rows of the exact half triangle plus the 480 mirrored entries of
-// the 16 diagonal blocks, which the readout weights by zero).
+// The state is indexed by the packed symmetric feature rows (i, j), i <= j:
+// phi(q) . S = sum_{i<=j} c_ij q_i q_j S_(i,j) with c_ij = 2 for i < j and 1
+// for i = j, so 64 * 65 / 2 = 2080 rows carry the whole state.  They are laid
+// out in 17 tiles of 128 rows (2176 rows; the 96 extra rows have i > j, are
+// weighted by zero in the readout and never exported).  The order serves both
+// tensor-core kernels:
 //
-// The order of the half-strips follows the state builder's work split: 5
-// CTAs per (head, segment), each with 4 accumulator tiles of 128 rows; tile
-// lanes come in 8 slots of 16 lanes, and a slot keeps the same jb in all 4
-// tiles of its CTA, so each builder thread reads its own key column once per
-// token block.  With global slot gs = 8 c + s (CTA c, slot s) the slots of
-// class b (jb = 16 b) are gs = 4 b (b + 1) / 2 .. ; slot u of class b covers
-// i = 4 u + m in tile m.  Half-strip index: h = 32 c + 8 m + s, state row
-// r = 16 h + (j - jb).
+//   tiles 0-11   off-diagonal blocks (i / 16 < j / 16) in 16-row groups of one
+//                i and 16 consecutive j (a "half-strip").  Tile 4 c + m, lane
+//                16 s + jj: global slot gs = 8 c + s selects the j block bj
+//                (gs 0-3: bj = 1, 4-11: bj = 2, 12-23: bj = 3), i = 4 (gs -
+//                first slot of bj) + m, j = 16 bj + jj.
+//   tiles 12-16  the four diagonal 16 x 16 triangles, as column groups: group
+//                (b, q, j) holds the rows (16 b + 4 q + m, j), m = 0..3, for
+//                j = 16 b + 4 q .. 16 b + 15 (rows with i > j are the padding).
+//                The groups run in the order of the runs (b, q) = (r % 4,
+//                r / 4), r = 0..15, columns ascending; the first 128 groups
+//                fill tiles 12-15 (lane = group, tile 12 + m = row m), the
+//                last 32 fill tile 16 (lane 4 g + m).
 //
-// Per (head, segment) the fp32 state is 2560 rows x 64 (the half-strips) then
-// the packed normaliser z[r] = sum k_i k_j for the same 2560 rows; the bf16
-// prefix copy read by the readout is the 2560 rows, then the dense
-// Z = sum k k^T split into hi and lo bf16 parts (64 rows each).
+// State builder: a work item is 4 tiles (tiles 4 c .. 4 c + 3, c = 0..3) or
+// the single tile 16 (c = 4); a builder thread owns the same lane in each of
+// its item's tiles, and within items 0-3 that lane's j is the same in all 4
+// tiles, so the thread reads its key column k_j once per token block.
+// Readout: two consecutive rows (one 32-bit word of the bf16 A operand) are
+// always (i, j), (i, j + 1) with j even or (i, j), (i + 1, j) with i even, so
+// every word of phi(q) is one bf16x2 product of register pairs.
+//
+// Per (head, segment) the fp32 state is the 2176 rows x 64 values, then the
+// packed normaliser z[r] = sum k_i k_j of the same rows; the bf16 prefix copy
+// read by the readout is the 2176 rows, then the dense Z = sum k k^T split
+// into hi and lo bf16 parts (64 rows each).
 #pragma once
+
+#if defined(__CUDACC__)
+#define KATA_HD __host__ __device__
+#else
+#define KATA_HD
+#endif
 
 namespace kata {
 namespace tc {
 
 constexpr int kD = 64;
-constexpr int kHalfStrips = 160;
-constexpr int kStateRows = 16 * kHalfStrips;        // 2560
+constexpr int kStateTiles = 17;
+constexpr int kStateRows = 128 * kStateTiles;       // 2176
+constexpr int kPairRows = kD * (kD + 1) / 2;        // 2080 rows with i <= j
 constexpr long long kZPacked0 = (long long)kStateRows * kD;     // fp32 packed z offset
-constexpr long long kF32PerSeg = kZPacked0 + kStateRows;        // 166,400 floats
-constexpr int kBf16Rows = kStateRows + 2 * kD;      // 2688 rows of 64 bf16
+constexpr long long kF32PerSeg = kZPacked0 + kStateRows;        // 141,440 floats
+constexpr int kBf16Rows = kStateRows + 2 * kD;      // 2304 rows of 64 bf16
 constexpr int kZHiRow0 = kStateRows;                // bf16 Z hi rows
 constexpr int kZLoRow0 = kStateRows + kD;           // bf16 Z lo rows
+constexpr int kBuildItems = 5;                      // builder items per (head, segment)
 
-__host__ __device__ constexpr int hs_class(int gs) { return gs < 4 ? 0 : gs < 12 ? 1 : gs < 24 ? 2 : 3; }
-__host__ __device__ constexpr int hs_class_start(int b) { return b == 0 ? 0 : b == 1 ? 4 : b == 2 ? 12 : 24; }
+// Tiles of builder item c, and the state tile holding its tile m.
+KATA_HD constexpr int build_item_tiles(int c) { return c < 4 ? 4 : 1; }
+KATA_HD constexpr int build_item_tile(int c, int m) { return c < 4 ? 4 * c + m : 16; }
 
-// i and jb of half-strip h.
-__host__ __device__ constexpr int hs_i(int h) {
-    return 4 * ((8 * (h / 32) + h % 8) - hs_class_start(hs_class(8 * (h / 32) + h % 8))) +
-           (h / 8) % 4;
+struct PairIJ {
+    int i, j;
+};
+
+KATA_HD constexpr int od_class(int gs) { return gs < 4 ? 1 : gs < 12 ? 2 : 3; }
+KATA_HD constexpr int od_first_slot(int bj) { return bj == 1 ? 0 : bj == 2 ? 4 : 12; }
+KATA_HD constexpr int run_groups(int run) { return 16 - 4 * (run >> 2); }
+
+// (i, j) of state row r (0 <= r < kStateRows); i > j marks a padding row.
+KATA_HD constexpr PairIJ row_ij(int r) {
+    const int tile = r / 128, lane = r % 128;
+    if (tile < 12) {
+        const int c = tile / 4, m = tile % 4, s = lane / 16, jj = lane % 16;
+        const int gs = 8 * c + s, bj = od_class(gs);
+        return PairIJ{4 * (gs - od_first_slot(bj)) + m, 16 * bj + jj};
+    }
+    const bool first = tile < 16;
+    int g = first ? lane : lane / 4;
+    const int m = first ? tile - 12 : lane % 4;
+    int run = first ? 0 : 10;
+    while (g >= run_groups(run)) {
+        g -= run_groups(run);
+        ++run;
+    }
+    const int b = run & 3, q = run >> 2;
+    return PairIJ{16 * b + 4 * q + m, 16 * b + 4 * q + g};
 }
-__host__ __device__ constexpr int hs_jb(int h) { return 16 * hs_class(8 * (h / 32) + h % 8); }
 
-// Half-strip holding row (i, j) for i <= j (requires i <= 16 (j / 16) + 15).
-__host__ __device__ constexpr int hs_index(int i, int j) {
-    return 32 * ((hs_class_start(j / 16) + i / 4) / 8) + 8 * (i % 4) +
-           (hs_class_start(j / 16) + i / 4) % 8;
+// State row of the pair (i, j), i <= j.
+KATA_HD constexpr int row_index(int i, int j) {
+    if (i / 16 < j / 16) {
+        const int bj = j / 16, jj = j % 16, gs = od_first_slot(bj) + i / 4, m = i % 4;
+        return 128 * (4 * (gs / 8) + m) + 16 * (gs % 8) + jj;
+    }
+    const int b = i / 16, q = (i % 16) / 4, m = i % 4;
+    const int run = 4 * q + b;
+    const bool first = run < 10;
+    int off = 0;
+    for (int r = first ? 0 : 10; r < run; ++r) off += run_groups(r);
+    const int g = off + (j - (16 * b + 4 * q));
+    return first ? 128 * (12 + m) + g : 128 * 16 + 4 * g + m;
 }
 
 }  // namespace tc

@@ -26,13 +26,14 @@ inline EncodeTiledFn encode_tiled_fn() {
     return fn;
 }
 
-// bf16 tensor of `rank` dims; dims[0] is the contiguous one.  strides_bytes
-// holds the byte strides of dims 1..rank-1 (multiples of 16).  Box dims[0] *
-// 2 bytes must be <= 128 for the 128-byte swizzle.  Out-of-bounds elements
-// read as zero.  Returns false if the driver rejects the map.
-inline bool make_tmap_bf16(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
-                           const uint64_t *strides_bytes, const uint32_t *box,
-                           CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+// Tensor of `rank` dims and element type `dtype`; dims[0] is the contiguous
+// one.  strides_bytes holds the byte strides of dims 1..rank-1 (multiples of
+// 16).  With the 128-byte swizzle, box dims[0] times the element size must be
+// <= 128 bytes.  Out-of-bounds elements read as zero and are not written by
+// stores.  Returns false if the driver rejects the map.
+inline bool make_tmap(CUtensorMap *map, CUtensorMapDataType dtype, const void *base, int rank,
+                      const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+                      CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return false;
     cuuint64_t gdim[5], gstride[4];
@@ -43,10 +44,16 @@ inline bool make_tmap_bf16(CUtensorMap *map, const void *base, int rank, const u
         estride[i] = 1;
     }
     for (int i = 0; i + 1 < rank; ++i) gstride[i] = strides_bytes[i];
-    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base),
-                          gdim, gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUresult r = fn(map, dtype, rank, const_cast<void *>(base), gdim, gstride, bdim, estride,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+inline bool make_tmap_bf16(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+                           const uint64_t *strides_bytes, const uint32_t *box,
+                           CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+    return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box, swizzle);
 }
 
 }  // namespace kata
