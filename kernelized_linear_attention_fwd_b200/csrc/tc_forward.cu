@@ -175,9 +175,13 @@ tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__r
 //                    item slot, state-prefix stages, K/V blocks)
 //   warps 9, 10      MMA issuers.  In the inter phase they take alternate
 //                    stages (so one issuer's wait overlaps the other's queued
-//                    MMAs); in the intra phase issuer t serves query tile t,
-//                    running the scores of key block b + 1 while the
-//                    generation warps square and mask block b.
+//                    MMAs).  In the intra phase warp 9 issues the scores
+//                    Q K^T of both tiles and warp 10 the weights times
+//                    values P V, so the scores of key block b + 1 run while
+//                    block b is squared, and neither issuer waits right
+//                    behind its own just-committed MMAs.
+//   warp 11          writes the finished output tiles (staged by the
+//                    epilogue in the item's Q slot) back with TMA stores.
 // Every barrier phase runs on across items.  Accumulators are zeroed by
 // tcgen05.st (at the start, then by each epilogue right after it reads them)
 // and every MMA accumulates, so the order in which the two issuers' MMAs run
@@ -195,7 +199,8 @@ constexpr int kRBRing = 4;               // inter B ring depth (state-prefix til
 constexpr int kRStageBytes = kRKs * 16 * 128;   // bf16 state-prefix rows per stage
 constexpr int kTmaWarp = 8;
 constexpr int kIssuer0 = 9;
-constexpr int kReadThreads = 352;
+constexpr int kStoreWarp = 11;
+constexpr int kReadThreads = 384;
 
 // shared memory (from a 1024-byte aligned base)
 constexpr int kItemBytes = kTiles * 16384 + 16384;  // Q tiles [128 x 64] x 2, Z hi / lo [64 x 64]
@@ -214,7 +219,7 @@ constexpr uint32_t kTmS = 128;   // intra scores S[t][x]: 64 columns at 128 + 12
 constexpr uint32_t kTmP = 384;   // intra weights P[t][x] (bf16 pairs): 32 columns at 384 + 64 t + 32 x
 
 struct ReadBars {
-    uint64_t qfull[2], qempty[2], u, interdone, done, genin;
+    uint64_t qfull[2], qempty[2], u, interdone, done, genin, ostaged;
     uint64_t bfull[kRBRing], bempty[kRBRing], afull[kRRing], aempty[kRRing];
     uint64_t kvfull[2], kvempty[2];
     uint64_t sfull[kTiles][2], pfull[kTiles][2], pempty[kTiles][2];
@@ -728,7 +733,8 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
 __global__ void __launch_bounds__(kReadThreads, 1)
 tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
-        __nv_bfloat16 *__restrict__ out, int T, int L, int n_seg, int n_ct, int n_items, int *status) {
+        const __grid_constant__ CUtensorMap tm_o, int T, int L, int n_seg, int n_ct, int n_items,
+        int *status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ ReadBars bars;
     __shared__ uint32_t tmem_base;
@@ -743,7 +749,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         abort_flag = 0;
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars.qfull[b], 1);
-            mbar_init(&bars.qempty[b], 2 + 8);  // both issuers' commits + one arrival per generation warp
+            mbar_init(&bars.qempty[b], 3);  // both issuers' commits + the output store's read
             mbar_init(&bars.kvfull[b], 1);
             mbar_init(&bars.kvempty[b], 2);
             mbar_init(&bars.drain[b], 1);
@@ -752,6 +758,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         mbar_init(&bars.interdone, 2);
         mbar_init(&bars.done, 2);
         mbar_init(&bars.genin, 8);
+        mbar_init(&bars.ostaged, 8);
         for (int s = 0; s < kRBRing; ++s) {
             mbar_init(&bars.bfull[s], 1);
             mbar_init(&bars.bempty[s], 1);
@@ -834,28 +841,14 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
     } else if (warp == kIssuer0 || warp == kIssuer0 + 1) {
         // ------------------------------------------------------------ MMA issuers
         if (lane == 0) {
-            const int me = warp - kIssuer0, t = me;
+            const int me = warp - kIssuer0;
             const uint32_t id_n64 = idesc_bf16(kQT, 64, 0, 1);  // B MN-major, N = 64
             const uint32_t id_qk = idesc_bf16(kQT, kSB, 0, 0);  // B = keys, K-major
             const uint64_t dS = desc_sw128(smem_u32(sm + kSmS), 8192, 1024);
             const uint64_t dK = desc_sw128(smem_u32(sm + kSmK), 16, 1024);
             const uint64_t dV = desc_sw128(smem_u32(sm + kSmV), 8192, 1024);
-            const uint32_t tS = tm + kTmS + 128 * t, tP = tm + kTmP + 64 * t, tO = tm + kTmO + 64 * t;
-            int n_inter = 0, g_kv = 0, g_b = 0, j = 0;
+            int n_inter = 0, g_kv = 0, g_b0 = 0, g_b1 = 0, j = 0;
             bool ok = true;
-            // weights of score block bb (global index g_b + bb) times its values
-            auto pv = [&](int bb) -> bool {
-                const int n = g_b + bb, x = n & 1;
-                if (!mbar_wait(&bars.pfull[t][x], (n >> 1) & 1, abort)) return false;
-                tc_fence_after();
-                const int G = g_kv + bb / 2;
-                const uint64_t dv = desc_add(dV, 16384 * (G & 1) + 8192 * (bb & 1));
-#pragma unroll
-                for (int ks = 0; ks < kSB / 16; ++ks)
-                    mma_ts(tO, tP + 32 * x + 8 * ks, desc_add(dv, 2048 * ks), id_n64, 1);
-                mma_commit(&bars.pempty[t][x]);
-                return true;
-            };
             for (int i = i_begin; i < i_end && ok; ++i, ++j) {
                 const ReadItem it = read_item(i, n_ct, T, L, n_seg);
                 const int qb = j & 1;
@@ -910,40 +903,66 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     tc_fence_after();
                     ++n_inter;
                 }
-                // intra phase: scores of block b are issued before the weights of block b - 1
-                const int n_b = read_tile_blocks(it, t, T);
-                const uint64_t dQt = desc_sw128(slot + t * 16384, 16, 1024);
-                for (int b = 0; b < n_b && ok; ++b) {
-                    const int n = g_b + b, x = n & 1;
+                // intra phase over 64-key blocks b (block b uses K/V block b / 2, half b % 2)
+                const int nb[kTiles] = {read_tile_blocks(it, 0, T), read_tile_blocks(it, 1, T)};
+                const int gb[kTiles] = {g_b0, g_b1};
+                const int nbm = max(nb[0], nb[1]);
+                for (int b = 0; b < nbm && ok; ++b) {
                     const int G = g_kv + b / 2;
-                    if ((b & 1) == 0) {
-                        ok = mbar_wait(&bars.kvfull[G & 1], (G >> 1) & 1, abort);
+                    if ((b & 1) == 0) ok = mbar_wait(&bars.kvfull[G & 1], (G >> 1) & 1, abort);
+                    if (me == 0) {
+                        // scores Q K^T into S[t][n % 2] (n = the tile's running block count),
+                        // once the squaring warps have read block n - 2 from that buffer,
+                        // which may belong to the previous item
+#pragma unroll
+                        for (int t = 0; t < kTiles; ++t)
+                            if (ok && gb[t] + b >= 2 && b < nb[t]) {
+                                const int n = gb[t] + b - 2;
+                                ok = mbar_wait(&bars.pfull[t][n & 1], (n >> 1) & 1, abort);
+                            }
                         if (!ok) break;
                         tc_fence_after();
-                    }
-                    const uint64_t dk = desc_add(dK, 16384 * (G & 1) + 8192 * (b & 1));
+                        const uint64_t dk = desc_add(dK, 16384 * (G & 1) + 8192 * (b & 1));
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_ss(tS + 64 * x, desc_add(dQt, 32 * ks), desc_add(dk, 32 * ks), id_qk, ks > 0);
-                    mma_commit(&bars.sfull[t][x]);
-                    if (b > 0) {
-                        ok = pv(b - 1);
-                        if (ok && ((b - 1) & 1)) mma_commit(&bars.kvempty[(g_kv + (b - 1) / 2) & 1]);
+                        for (int t = 0; t < kTiles; ++t) {
+                            if (b >= nb[t]) continue;
+                            const int n = gb[t] + b, x = n & 1;
+                            const uint64_t dQt = desc_sw128(slot + t * 16384, 16, 1024);
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_ss(tm + kTmS + 128 * t + 64 * x, desc_add(dQt, 32 * ks), desc_add(dk, 32 * ks),
+                                       id_qk, ks > 0);
+                            mma_commit(&bars.sfull[t][x]);
+                        }
+                    } else {
+                        // weights P (from tensor memory) times values into O[t]
+#pragma unroll
+                        for (int t = 0; t < kTiles; ++t)
+                            if (ok && b < nb[t]) {
+                                const int n = gb[t] + b;
+                                ok = mbar_wait(&bars.pfull[t][n & 1], (n >> 1) & 1, abort);
+                            }
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t dv = desc_add(dV, 16384 * (G & 1) + 8192 * (b & 1));
+#pragma unroll
+                        for (int t = 0; t < kTiles; ++t) {
+                            if (b >= nb[t]) continue;
+                            const int n = gb[t] + b, x = n & 1;
+#pragma unroll
+                            for (int ks = 0; ks < kSB / 16; ++ks)
+                                mma_ts(tm + kTmO + 64 * t, tm + kTmP + 64 * t + 32 * x + 8 * ks,
+                                       desc_add(dv, 2048 * ks), id_n64, 1);
+                            mma_commit(&bars.pempty[t][x]);
+                        }
                     }
-                }
-                if (ok && n_b > 0) {
-                    ok = pv(n_b - 1);
-                    if (ok) mma_commit(&bars.kvempty[(g_kv + (n_b - 1) / 2) & 1]);
-                }
-                // key/value blocks this tile does not need: release them once loaded
-                for (int kb = (n_b + 1) / 2; kb < it.n_kv && ok; ++kb) {
-                    const int G = g_kv + kb;
-                    ok = mbar_wait(&bars.kvfull[G & 1], (G >> 1) & 1, abort);
-                    if (ok) mma_commit(&bars.kvempty[G & 1]);
+                    // this issuer is done with K/V block b / 2
+                    if ((b & 1) || b == nbm - 1) mma_commit(&bars.kvempty[G & 1]);
                 }
                 if (!ok) break;
                 g_kv += it.n_kv;
-                g_b += n_b;
+                g_b0 += nb[0];
+                g_b1 += nb[1];
                 // every generation warp has entered this item, so `done` cannot run a phase ahead of it
                 ok = mbar_wait(&bars.genin, j & 1, abort);
                 if (!ok) break;
@@ -953,6 +972,24 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             // no MMA of this CTA may still read or write tensor memory when it is freed
             mma_commit(&bars.drain[me]);
             mbar_wait_issued(&bars.drain[me], 0);
+        }
+    } else if (warp == kStoreWarp) {
+        // ------------------------------------------------------------ output write-back
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_o);
+            int j = 0;
+            for (int i = i_begin; i < i_end; ++i, ++j) {
+                const ReadItem it = read_item(i, n_ct, T, L, n_seg);
+                const int qb = j & 1;
+                if (!mbar_wait(&bars.ostaged, j & 1, abort)) break;
+                for (int t = 0; t < kTiles; ++t)
+                    if (it.t0 + kQT * t < T)
+                        tma_store_3d(&tm_o, sm + kSmItem + qb * kItemBytes + t * 16384, 0, it.t0 + kQT * t, it.bh);
+                bulk_commit_group();
+                bulk_wait_read_all();
+                mbar_arrive(&bars.qempty[qb]);  // the slot may be refilled
+            }
+            bulk_wait_all();
         }
     } else {
         // ------------------------------------------------------------ generation / scores / epilogue
@@ -991,8 +1028,6 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     q2[4 * c + 3] = x.w;
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.qempty[qb]);
             const int tq0 = it.t0 + kQT * t, tq = tq0 + row;
             float den_inter = 0.f;
             if (it.inter) {
@@ -1030,24 +1065,32 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                 tmem_ld32(tS + 64 * x + 32, r + 32);
                 tmem_ld_wait();
                 const int kbs = it.seg0 + kSB * b;
+                // weights w = s^2 (packed fp32 pairs), four partial row sums
+                uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
                 if (kbs + kSB - 1 <= tq0) {  // every key of the block precedes every query of the tile
 #pragma unroll
                     for (int y = 0; y < 32; ++y) {
-                        const float s0 = __uint_as_float(r[2 * y]), s1 = __uint_as_float(r[2 * y + 1]);
-                        const float w0 = s0 * s0, w1 = s1 * s1;
-                        l += w0 + w1;
-                        p[y] = pack_bf16x2(w0, w1);
+                        const uint64_t s2 = f32x2_pack(r[2 * y], r[2 * y + 1]);
+                        const uint64_t w2 = f32x2_mul(s2, s2);
+                        acc[y & 3] = f32x2_add(acc[y & 3], w2);
+                        p[y] = f32x2_to_bf16x2(w2);
                     }
                 } else {
+                    const int lim = tq - kbs;  // keys kbs + c with c <= lim are visible
 #pragma unroll
                     for (int y = 0; y < 32; ++y) {
-                        const int key = kbs + 2 * y;
-                        const float s0 = __uint_as_float(r[2 * y]), s1 = __uint_as_float(r[2 * y + 1]);
-                        const float w0 = key <= tq ? s0 * s0 : 0.f;
-                        const float w1 = key + 1 <= tq ? s1 * s1 : 0.f;
-                        l += w0 + w1;
-                        p[y] = pack_bf16x2(w0, w1);
+                        const uint32_t m0 = 2 * y <= lim ? r[2 * y] : 0u;
+                        const uint32_t m1 = 2 * y + 1 <= lim ? r[2 * y + 1] : 0u;
+                        const uint64_t s2 = f32x2_pack(m0, m1);
+                        const uint64_t w2 = f32x2_mul(s2, s2);
+                        acc[y & 3] = f32x2_add(acc[y & 3], w2);
+                        p[y] = f32x2_to_bf16x2(w2);
                     }
+                }
+                {
+                    const uint64_t a01 = f32x2_add(acc[0], acc[1]), a23 = f32x2_add(acc[2], acc[3]);
+                    const uint64_t a = f32x2_add(a01, a23);
+                    l += f32x2_lo(a) + f32x2_hi(a);
                 }
                 // the weights of block n - 2 (same buffer) must have been consumed
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars.pempty[t][x], ((n >> 1) & 1) ^ 1, abort));
@@ -1074,17 +1117,23 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             tmem_st32(tO + 32, zero);
             const float den = l + den_inter;
             const float inv = den == 0.f ? 0.f : 1.f / den;
-            if (tq < T) {
-                uint4 *dst = reinterpret_cast<uint4 *>(out + ((long long)it.bh * T + tq) * kD);
+            // the output row replaces this thread's own query row in the item slot (same
+            // swizzled layout); warp 11 stores both tiles with TMA once all rows are in
+            {
+                uint8_t *orow = sm + kSmItem + qb * kItemBytes + t * 16384 + row * 128;
+                const uint64_t inv2 = f32x2_pack(__float_as_uint(inv), __float_as_uint(inv));
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint4 v;
-                    v.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
-                    v.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
-                    v.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
-                    v.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
-                    dst[c] = v;
+                    v.x = f32x2_to_bf16x2(f32x2_mul(f32x2_pack(o[8 * c + 0], o[8 * c + 1]), inv2));
+                    v.y = f32x2_to_bf16x2(f32x2_mul(f32x2_pack(o[8 * c + 2], o[8 * c + 3]), inv2));
+                    v.z = f32x2_to_bf16x2(f32x2_mul(f32x2_pack(o[8 * c + 4], o[8 * c + 5]), inv2));
+                    v.w = f32x2_to_bf16x2(f32x2_mul(f32x2_pack(o[8 * c + 6], o[8 * c + 7]), inv2));
+                    *reinterpret_cast<uint4 *>(orow + ((c ^ (row & 7)) * 16)) = v;
                 }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars.ostaged);
             }
         }
         tmem_st_wait();
@@ -1096,8 +1145,8 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
     if (tid == 0 && abort_flag) set_timeout_status(status);
 }
 
-bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const void *prefix,
-               CUtensorMap *mq, CUtensorMap *mk, CUtensorMap *mv, CUtensorMap *ms) {
+bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const void *prefix, void *out,
+               CUtensorMap *mq, CUtensorMap *mk, CUtensorMap *mv, CUtensorMap *ms, CUtensorMap *mo) {
     const uint64_t dqkv[3] = {(uint64_t)kD, (uint64_t)p.T, (uint64_t)p.BH};
     const uint64_t sqkv[2] = {(uint64_t)kD * 2, (uint64_t)p.T * kD * 2};
     const uint32_t bqkv[3] = {64, 128, 1};
@@ -1106,7 +1155,7 @@ bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const
     const uint32_t bs[3] = {64, 32, 1};
     return make_tmap_bf16(mq, q, 3, dqkv, sqkv, bqkv) && make_tmap_bf16(mk, k, 3, dqkv, sqkv, bqkv) &&
            make_tmap_bf16(mv, v, 3, dqkv, sqkv, bqkv) &&
-           make_tmap_bf16(ms, prefix ? prefix : q, 3, ds, ss, bs);
+           make_tmap_bf16(ms, prefix ? prefix : q, 3, ds, ss, bs) && make_tmap_bf16(mo, out, 3, dqkv, sqkv, bqkv);
 }
 
 }  // namespace
@@ -1192,8 +1241,8 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
                                                      p.n_seg, n_build);
     }
     {
-        CUtensorMap mq, mk, mv, ms;
-        if (!make_maps(p, q, k, v, prefix, &mq, &mk, &mv, &ms)) return cudaErrorInvalidValue;
+        CUtensorMap mq, mk, mv, ms, mo;
+        if (!make_maps(p, q, k, v, prefix, out, &mq, &mk, &mv, &ms, &mo)) return cudaErrorInvalidValue;
         cudaError_t e = cudaFuncSetAttribute(tc_read, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kSmAlloc);
         if (e != cudaSuccess) return e;
@@ -1203,8 +1252,7 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
         const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
         ProfScope ps("tc_read", st);
         tc_read<<<(unsigned)grid, kReadThreads, kSmAlloc, st>>>(
-            mq, mk, mv, ms, static_cast<__nv_bfloat16 *>(out), p.T, p.L, p.n_seg, n_ct, (int)n_items,
-            status);
+            mq, mk, mv, ms, mo, p.T, p.L, p.n_seg, n_ct, (int)n_items, status);
     }
     if (want_state) {
         const float *src = p.n_seg > 1 ? total : seg;
