@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override the workload's T (smaller cases of the same workload for profiling)")
     return ap.parse_args()
 
 
@@ -282,7 +284,7 @@ def run_ours(args, rank, world):
     dev = torch.cuda.current_device()
     w = inputs.WORKLOADS[args.workload]
     C = args.chunk
-    B, H, T, d = w.B, w.H, w.T, w.d
+    B, H, T, d = w.B, w.H, (args.seq_len or w.T), w.d
     BH = B * H
     # each rank: its own batch of independent heads (seed offset by rank)
     qh, kh, vh = inputs.make_qkv(B, H, T, d, d, w.dtype, seed=rank_seed(w.seed, rank), qk=w.qk)
