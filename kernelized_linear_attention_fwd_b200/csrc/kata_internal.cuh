@@ -92,6 +92,8 @@ void plan_tc_workspace(Plan &p);
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v,
                               void *out, float *state_out, float *z_out, void *ws,
                               cudaStream_t st);
+// Streaming multiprocessors of the current device (cached).
+int num_sms();
 }  // namespace tc
 
 cudaError_t launch_decode(int B, int H, int dk, int dv, kata_dtype dtype, const void *q,
