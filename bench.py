@@ -17,8 +17,10 @@ Printed (rank 0): one JSON line.  Besides the contract keys it carries the
 roofline of the dominant kernel (timed live with CUDA events recorded by the
 library around each launch), the CPU baseline (the fp64 oracle on a bounded
 sample, host cores), the end-to-end number through the public API with host
-buffers, the SM clocks sampled during the timed region, and the decode-step
-bandwidth on the 64 x 16-head decode workload.
+buffers, the SM clocks sampled during the timed region, the decode-step
+bandwidth on the 64 x 16-head decode workload, and the quadratic
+(flash-attention-style) form timed on the same inputs beside a library causal
+flash-attention forward of the same shape (context only).
 
 --impl reference times the fp64 CPU oracle (the only other implementation of
 this path) on a bounded sample per step, on rank 0 only.
@@ -59,6 +61,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-quadratic", action="store_true")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override the workload's T (smaller cases of the same workload for profiling)")
     return ap.parse_args()
@@ -425,6 +428,13 @@ def run_ours(args, rank, world):
                   "peak_source": src}
         del Sd, Zd
 
+    # the quadratic (flash-attention-style) form of the same forward
+    quad = None
+    if not args.no_quadratic:
+        quad = measure_quadratic(K, q, k, v, out, stream, flush, world, rank, ms_max, n=3)
+        if K.kata_get_device_status() != 0:
+            raise RuntimeError("device status set by the quadratic form")
+
     if rank != 0:
         return None
 
@@ -493,10 +503,93 @@ def run_ours(args, rank, world):
         "kernels_ms_per_step": {n: t / args.steps for n, (c, t) in prof.items()},
         "clocks": clk,
         "decode": decode,
+        "quadratic_form": quad,
         "device_status": status,
         "forward_canonical": canon,
     }
     return line
+
+
+def quadratic_flops(BH, T, d, dv):
+    """Algorithmic flops of the causal quadratic form: 2 d (score) + 2 dv
+    (weighted values) per (query, key) pair with key <= query."""
+    return BH * T * (T + 1) // 2 * 2 * (d + dv)
+
+
+def time_launches(fn, stream, flush, n, warm=2):
+    """Mean device ms of fn() over n launches (CUDA events on `stream`, L2
+    flushed before each, outside the events)."""
+    import torch
+
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    for a, b in ev:
+        flush()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev) / n
+
+
+def library_flash_attention(q, k, v, stream, flush, n):
+    """Context only: a library causal flash-attention forward (softmax
+    attention) of the same shape on this GPU, the pages' point of comparison.
+    FlashAttention-2 (flash_attn) if it runs here, else torch's SDPA with its
+    flash backend.  Returns (backend, mean ms) or (None, reason)."""
+    import torch
+
+    errs = []
+    try:
+        from flash_attn import flash_attn_func
+
+        qt, kt, vt = (x.transpose(1, 2).contiguous() for x in (q, k, v))  # [B, T, H, d]
+        ms = time_launches(lambda: flash_attn_func(qt, kt, vt, causal=True), stream, flush, n)
+        del qt, kt, vt
+        return "flash_attn " + __import__("flash_attn").__version__, ms
+    except Exception as e:  # not built for this GPU, or not installed
+        errs.append(f"flash_attn: {type(e).__name__}: {str(e)[:120]}")
+    try:
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        from torch.nn.functional import scaled_dot_product_attention as sdpa
+
+        def run():
+            with sdpa_kernel(SDPBackend.FLASH_ATTENTION):
+                sdpa(q, k, v, is_causal=True)
+
+        return "torch sdpa (flash backend)", time_launches(run, stream, flush, n)
+    except Exception as e:
+        errs.append(f"torch sdpa: {type(e).__name__}: {str(e)[:120]}")
+    return None, "; ".join(errs)
+
+
+def measure_quadratic(K, q, k, v, out, stream, flush, world, rank, chunked_ms, n):
+    """The quadratic (flash-attention-style) form on the step's own inputs."""
+    B, H, T, d = q.shape
+    BH = B * H
+    ms = max_over_ranks(time_launches(lambda: K.kata_quadratic_forward(q, k, v, out=out,
+                                                                       stream=stream),
+                                      stream, flush, n), world)
+    peaks, src = load_peaks()
+    fl = quadratic_flops(BH, T, d, d)
+    tf = fl / (ms / 1e3) / 1e12
+    res = {"ms": ms, "tokens_per_s": world * B * T / (ms / 1e3),
+           "flop_per_launch": fl, "achieved_tflops": tf, "peak_tflops": peaks["bf16_tflops"],
+           "frac": tf / peaks["bf16_tflops"], "peak_source": f"{src} (burst)",
+           "flop_note": "causal pairs x 2(d + dv); masked halves of diagonal blocks not counted"}
+    if rank == 0:
+        backend, fa = library_flash_attention(q, k, v, stream, flush, n)
+        if backend is None:
+            res["library_flash_attention"] = {"unavailable": fa}
+        else:
+            res["library_flash_attention"] = {
+                "backend": backend, "ms": fa, "achieved_tflops": fl / (fa / 1e3) / 1e12,
+                "quadratic_speedup": fa / ms, "chunked_step_speedup": fa / chunked_ms,
+                "note": "context only: softmax attention of the same B, H, T, d, causal"}
+    return res
 
 
 # ---------------------------------------------------------------------------

@@ -144,6 +144,30 @@ kata_status kata_chunked_forward_noalloc(const void *q, const void *k, const voi
                                          kata_stream_t stream);
 
 /*
+ * Causal KATA forward in its quadratic form: the flash-attention-style
+ * operating point (gist.science summary 2.3, "two operating points", the
+ * O(T^2) forward that never forms the state; arXiv abstract,
+ * "flash-attention-style forward").
+ *
+ * Same y_t as kata_chunked_forward, computed from the T x T causal weights
+ * (q_t.k_s)^2 in tiles that never leave the chip; no state is formed, so
+ * nothing is exported and no workspace is needed.  Work grows as T^2: the
+ * chunked form is the one to use for long sequences, this one for short
+ * ones and as an independent check of the chunked form.
+ *
+ *   q, k   [B, H, T, dk]  dtype      queries, keys
+ *   v      [B, H, T, dv]  dtype      values
+ *   out    [B, H, T, dv]  dtype      y_t as defined at the top of this file
+ *
+ * dtype KATA_BF16 with dk = 64 runs the tensor-core (tcgen05) path; other
+ * cases run fp32 CUDA-core arithmetic.  Errors as in the general contract;
+ * B * H * ceil(T / 256) must stay below 2^31 (else KATA_ERR_UNSUPPORTED).
+ */
+kata_status kata_quadratic_forward(const void *q, const void *k, const void *v, void *out, int B,
+                                   int H, int T, int dk, int dv, kata_dtype dtype,
+                                   kata_stream_t stream);
+
+/*
  * One recurrent decode step for every head, in place
  * (arXiv abstract, "constant-time recurrent inference"; gist.science summary
  * 1: a fixed-size state replaces the key-value cache):

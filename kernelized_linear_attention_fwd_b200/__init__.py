@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     kata_chunked_forward_workspace_bytes,
     kata_decode_step,
     kata_get_device_status,
+    kata_quadratic_forward,
     kata_status_string,
     kata_version,
     load_library,

@@ -31,6 +31,7 @@ EXPORTS = (
     "kata_chunked_forward_workspace_bytes",
     "kata_chunked_forward",
     "kata_chunked_forward_noalloc",
+    "kata_quadratic_forward",
     "kata_decode_step",
     "kata_get_device_status",
 )
@@ -68,6 +69,8 @@ def load_library(path: str = LIB_PATH):
     lib.kata_chunked_forward_noalloc.restype = i32
     lib.kata_chunked_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                  i32, fp, fp, vp]
+    lib.kata_quadratic_forward.restype = i32
+    lib.kata_quadratic_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
     lib.kata_decode_step.restype = i32
     lib.kata_decode_step.argtypes = [vp, vp, vp, vp, fp, fp, i32, i32, i32, i32, i32, vp]
     lib.kata_get_device_status.restype = i32
@@ -188,6 +191,28 @@ def kata_chunked_forward_noalloc(q, k, v, C=64, out=None, state_out=None, z_out=
                                           _stream_handle(stream))
     if st != KATA_OK:
         raise KataError(st, "kata_chunked_forward_noalloc")
+    return out
+
+
+def kata_quadratic_forward(q, k, v, out=None, stream=None):
+    """out[B,H,T,dv] = causal KATA forward of q, k [B,H,T,dk] and v [B,H,T,dv] in
+    the quadratic (flash-attention-style) form: no state, no workspace."""
+    import torch
+
+    lib = load_library()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", (B, H, T, dk))
+    _check(k, "k", (B, H, T, dk), q.dtype)
+    _check(v, "v", (B, H, T, dv), q.dtype)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", (B, H, T, dv), q.dtype)
+    st = lib.kata_quadratic_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv, code,
+                                    _stream_handle(stream))
+    if st != KATA_OK:
+        raise KataError(st, "kata_quadratic_forward")
     return out
 
 

@@ -81,6 +81,42 @@ kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dty
     return KATA_OK;
 }
 
+// The quadratic form is the chunked plan with one segment spanning the whole
+// sequence: no state is built, scanned or stored, so no workspace is used.
+kata_status make_quadratic_plan(int B, int H, int T, int dk, int dv, kata_dtype dtype, Plan &p) {
+    const kata_status s = make_plan(B, H, T, dk, dv, 256, dtype, p);
+    if (s != KATA_OK) return s;
+    p.L = T;
+    p.n_seg = 1;
+    p.ws_seg_state = p.ws_total = p.ws_extra = p.ws_aux = p.ws_bytes = 0;
+    return KATA_OK;
+}
+
+namespace {
+
+// Checks shared by both forward entry points: q, k, v, out present, 16-byte
+// aligned, and out disjoint from the inputs.
+kata_status check_forward_io(const Plan &p, const void *q, const void *k, const void *v,
+                             const void *out) {
+    if (!q || !k || !v || !out) return KATA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return KATA_ERR_INVALID_ARG;
+    const size_t es = p.dtype == KATA_BF16 ? 2 : 4;
+    const size_t nq = (size_t)p.BH * p.T * p.dk * es, nv = (size_t)p.BH * p.T * p.dv * es;
+    if (overlaps(out, nv, q, nq) || overlaps(out, nv, k, nq) || overlaps(out, nv, v, nv))
+        return KATA_ERR_INVALID_ARG;
+    return KATA_OK;
+}
+
+cudaError_t launch_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
+                           float *state_out, float *z_out, void *ws, cudaStream_t st) {
+    return p.path == Path::kTensorCore
+               ? tc::launch_tc_forward(p, q, k, v, out, state_out, z_out, ws, st)
+               : launch_simt_forward(p, q, k, v, out, state_out, z_out, ws, st);
+}
+
+}  // namespace
+
 }  // namespace kata
 
 using kata::Plan;
@@ -117,24 +153,30 @@ kata_status kata_chunked_forward(const void *q, const void *k, const void *v, vo
     Plan p;
     const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p);
     if (ps != KATA_OK) return ps;
-    if (!q || !k || !v || !out) return KATA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-        return KATA_ERR_INVALID_ARG;
+    const kata_status io = kata::check_forward_io(p, q, k, v, out);
+    if (io != KATA_OK) return io;
     if ((state_out == nullptr) != (z_out == nullptr)) return KATA_ERR_INVALID_ARG;
     if (state_out && (!aligned16(state_out) || !aligned16(z_out))) return KATA_ERR_INVALID_ARG;
-    const size_t es = dtype == KATA_BF16 ? 2 : 4;
-    const size_t nq = (size_t)p.BH * T * dk * es, nv = (size_t)p.BH * T * dv * es;
-    if (overlaps(out, nv, q, nq) || overlaps(out, nv, k, nq) || overlaps(out, nv, v, nv))
-        return KATA_ERR_INVALID_ARG;
     if (p.ws_bytes > 0) {
         if (!workspace || workspace_bytes < p.ws_bytes) return KATA_ERR_WORKSPACE;
         if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_WORKSPACE;
     }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const cudaError_t e =
-        p.path == kata::Path::kTensorCore
-            ? kata::tc::launch_tc_forward(p, q, k, v, out, state_out, z_out, workspace, st)
-            : kata::launch_simt_forward(p, q, k, v, out, state_out, z_out, workspace, st);
+    const cudaError_t e = kata::launch_forward(p, q, k, v, out, state_out, z_out, workspace, st);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+}
+
+kata_status kata_quadratic_forward(const void *q, const void *k, const void *v, void *out, int B,
+                                   int H, int T, int dk, int dv, kata_dtype dtype,
+                                   kata_stream_t stream) {
+    Plan p;
+    const kata_status ps = kata::make_quadratic_plan(B, H, T, dk, dv, dtype, p);
+    if (ps != KATA_OK) return ps;
+    const kata_status io = kata::check_forward_io(p, q, k, v, out);
+    if (io != KATA_OK) return io;
+    if (p.BH * ((T + 255LL) / 256) >= 0x7fffffffLL) return KATA_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = kata::launch_forward(p, q, k, v, out, nullptr, nullptr, nullptr, st);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
 }
 

@@ -42,7 +42,7 @@ struct Plan {
     int B, H, T, dk, dv, C;
     kata_dtype dtype;
     long long BH;
-    int L;      // segment length (tokens), a multiple of C and of 128
+    int L;      // segment length (tokens), a multiple of C and of 128; T in the quadratic plan
     int n_seg;  // ceil(T / L)
     int R;      // packed feature rows
     Path path;
@@ -56,6 +56,8 @@ struct Plan {
 
 // Fills `p`; returns KATA_OK or the error the forward must return.
 kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype, Plan &p);
+// The plan of the quadratic form: one segment of T tokens, no workspace.
+kata_status make_quadratic_plan(int B, int H, int T, int dk, int dv, kata_dtype dtype, Plan &p);
 
 // Device address of the status word that kernels set when an on-device check
 // fails (one per device; resolved on first use with that device current).

@@ -180,9 +180,19 @@ seg_read(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__rest
 
     const int tid = threadIdx.x;
     const int tq = tid >> 4, te = tid & 15;
+    // One segment (the quadratic form): the latest query tiles, whose work is
+    // largest, are scheduled first, across all heads.
     const int n_qt = (T + kTok - 1) / kTok;
-    const long long bh = blockIdx.x / n_qt;
-    const int t0 = (int)(blockIdx.x % n_qt) * kTok;
+    long long bh;
+    int t0;
+    if (n_seg == 1) {
+        const long long BH = gridDim.x / n_qt;
+        bh = blockIdx.x % BH;
+        t0 = (n_qt - 1 - (int)(blockIdx.x / BH)) * kTok;
+    } else {
+        bh = blockIdx.x / n_qt;
+        t0 = (int)(blockIdx.x % n_qt) * kTok;
+    }
     const int g = t0 / L;
     const int seg0 = g * L;
 
@@ -328,8 +338,10 @@ cudaError_t run(const Plan &p, const TIn *q, const TIn *k, const TIn *v, TIn *ou
     constexpr int R = packed_rows(DK);
     constexpr long long E = (long long)R * (DV + 1);
     const long long BH = p.BH;
-    float *seg = reinterpret_cast<float *>(static_cast<char *>(ws) + p.ws_seg_state);
-    float *total = reinterpret_cast<float *>(static_cast<char *>(ws) + p.ws_total);
+    // no workspace (the quadratic plan): no state is built, scanned or read
+    char *w = static_cast<char *>(ws);
+    float *seg = w ? reinterpret_cast<float *>(w + p.ws_seg_state) : nullptr;
+    float *total = w ? reinterpret_cast<float *>(w + p.ws_total) : nullptr;
     const bool want_state = state_out != nullptr;
     const int n_build = want_state ? p.n_seg : p.n_seg - 1;
 

@@ -245,6 +245,36 @@ __device__ __forceinline__ ReadItem read_item(int i, int n_ct, int T, int L, int
     return it;
 }
 
+// Work items a CTA walks.  Several segments: a contiguous range of the natural
+// order (head-major), so the items of a segment reuse its state prefix and keys
+// from L2.  One segment (the quadratic form): the costliest items (latest
+// queries) first, dealt round-robin to the CTAs, which balances work that grows
+// with the query position.
+struct ReadSched {
+    int first, end, stride, n_ct, BH;
+    bool longest_first;
+    __device__ __forceinline__ int item(int x) const {  // natural item index of position x
+        return longest_first ? (x % BH) * n_ct + (n_ct - 1 - x / BH) : x;
+    }
+};
+
+__device__ __forceinline__ ReadSched read_sched(int n_items, int n_ct, int n_seg) {
+    ReadSched s;
+    s.n_ct = n_ct;
+    s.BH = n_items / n_ct;
+    s.longest_first = n_seg == 1;
+    if (s.longest_first) {
+        s.first = blockIdx.x;
+        s.end = n_items;
+        s.stride = gridDim.x;
+    } else {
+        s.first = (int)((long long)blockIdx.x * n_items / gridDim.x);
+        s.end = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x);
+        s.stride = 1;
+    }
+    return s;
+}
+
 // 64-key score blocks of tile t: keys seg0 .. min(end of tile, T) - 1; none
 // when the tile starts at or after T.
 __device__ __forceinline__ int read_tile_blocks(const ReadItem &it, int t, int T) {
@@ -742,8 +772,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
 
     uint8_t *sm = align1024(smem_raw);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int i_begin = (int)((long long)blockIdx.x * n_items / gridDim.x);
-    const int i_end = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x);
+    const ReadSched sched = read_sched(n_items, n_ct, n_seg);
 
     if (tid == 0) {
         abort_flag = 0;
@@ -794,8 +823,8 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             tma_prefetch_desc(&tm_s);
             int n_q = 0, n_bs = 0, n_kv = 0;  // loads issued into each ring
             bool ok = true;
-            for (int i = i_begin; i < i_end && ok; ++i) {
-                const ReadItem it = read_item(i, n_ct, T, L, n_seg);
+            for (int x = sched.first; x < sched.end && ok; x += sched.stride) {
+                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg);
                 {
                     const int qb = n_q & 1;
                     uint8_t *slot = sm + kSmItem + qb * kItemBytes;
@@ -849,8 +878,8 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             const uint64_t dV = desc_sw128(smem_u32(sm + kSmV), 8192, 1024);
             int n_inter = 0, g_kv = 0, g_b0 = 0, g_b1 = 0, j = 0;
             bool ok = true;
-            for (int i = i_begin; i < i_end && ok; ++i, ++j) {
-                const ReadItem it = read_item(i, n_ct, T, L, n_seg);
+            for (int x = sched.first; x < sched.end && ok; x += sched.stride, ++j) {
+                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg);
                 const int qb = j & 1;
                 const uint32_t slot = smem_u32(sm + kSmItem + qb * kItemBytes);
                 ok = mbar_wait(&bars.qfull[qb], (j >> 1) & 1, abort);
@@ -978,8 +1007,8 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         if (lane == 0) {
             tma_prefetch_desc(&tm_o);
             int j = 0;
-            for (int i = i_begin; i < i_end; ++i, ++j) {
-                const ReadItem it = read_item(i, n_ct, T, L, n_seg);
+            for (int x = sched.first; x < sched.end; x += sched.stride, ++j) {
+                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg);
                 const int qb = j & 1;
                 if (!mbar_wait(&bars.ostaged, j & 1, abort)) break;
                 for (int t = 0; t < kTiles; ++t)
@@ -1010,8 +1039,8 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         tmem_st_wait();
         int n_inter = 0, g_b = 0, j = 0;
         bool ok = true;
-        for (int i = i_begin; i < i_end && ok; ++i, ++j) {
-            const ReadItem it = read_item(i, n_ct, T, L, n_seg);
+        for (int x = sched.first; x < sched.end && ok; x += sched.stride, ++j) {
+            const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg);
             const int qb = j & 1;
             if (lane == 0) mbar_arrive(&bars.genin);
             ok = __all_sync(0xffffffffu, mbar_wait(&bars.qfull[qb], (j >> 1) & 1, abort));
@@ -1194,11 +1223,12 @@ void plan_tc_workspace(Plan &p) {
 
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
                               float *state_out, float *z_out, void *ws, cudaStream_t st) {
+    // no workspace (the quadratic plan): no state is built, scanned or read
     char *w = static_cast<char *>(ws);
-    float *seg = reinterpret_cast<float *>(w + p.ws_seg_state);
-    float *total = reinterpret_cast<float *>(w + p.ws_total);
-    __nv_bfloat16 *prefix = reinterpret_cast<__nv_bfloat16 *>(w + p.ws_extra);
-    __nv_bfloat16 *kt = reinterpret_cast<__nv_bfloat16 *>(w + p.ws_aux);
+    float *seg = w ? reinterpret_cast<float *>(w + p.ws_seg_state) : nullptr;
+    float *total = w ? reinterpret_cast<float *>(w + p.ws_total) : nullptr;
+    __nv_bfloat16 *prefix = w ? reinterpret_cast<__nv_bfloat16 *>(w + p.ws_extra) : nullptr;
+    __nv_bfloat16 *kt = w ? reinterpret_cast<__nv_bfloat16 *>(w + p.ws_aux) : nullptr;
     const bool want_state = state_out != nullptr;
     const int n_build = want_state ? p.n_seg : p.n_seg - 1;
     const long long BH = p.BH;
@@ -1248,7 +1278,7 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
         if (e != cudaSuccess) return e;
         const int n_ct = (p.T + kCtaQ - 1) / kCtaQ;
         const long long n_items = (long long)n_ct * BH;
-        if (n_items > 0x7fffffffLL) return cudaErrorInvalidValue;
+        if (n_items >= 0x7fffffffLL - 4096) return cudaErrorInvalidValue;
         const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
         ProfScope ps("tc_read", st);
         tc_read<<<(unsigned)grid, kReadThreads, kSmAlloc, st>>>(

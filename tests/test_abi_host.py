@@ -105,6 +105,27 @@ def test_forward_rejects_bad_arguments(lib):
     assert _fwd(lib, T=4096, ws=FAKE + 0x50000010, wsb=need) == E.KATA_ERR_WORKSPACE
 
 
+def test_quadratic_forward_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    E = binding
+
+    def quad(q=FAKE, k=FAKE + 0x10000000, v=FAKE + 0x20000000, out=FAKE + 0x30000000, B=1, H=1,
+             T=64, dk=16, dv=16, dt=0):
+        return lib.kata_quadratic_forward(vp(q) if q else None, vp(k) if k else None,
+                                          vp(v) if v else None, vp(out) if out else None, B, H,
+                                          T, dk, dv, dt, None)
+
+    assert quad(q=0) == E.KATA_ERR_INVALID_ARG
+    assert quad(v=0) == E.KATA_ERR_INVALID_ARG
+    assert quad(k=FAKE + 0x10000008) == E.KATA_ERR_INVALID_ARG         # misaligned
+    assert quad(H=0) == E.KATA_ERR_INVALID_ARG
+    assert quad(T=0) == E.KATA_ERR_INVALID_ARG
+    assert quad(dk=48, dv=48) == E.KATA_ERR_UNSUPPORTED
+    assert quad(dk=64, dv=32) == E.KATA_ERR_UNSUPPORTED
+    assert quad(dt=2) == E.KATA_ERR_UNSUPPORTED
+    assert quad(out=FAKE + 0x20000000 + 256) == E.KATA_ERR_INVALID_ARG  # out inside v
+
+
 def test_decode_rejects_bad_arguments(lib):
     vp = ctypes.c_void_p
     E = binding

@@ -5,7 +5,7 @@ issuers (alternate inter stages; scores Q K^T by issuer 0, weights times values
 by issuer 1), the output-store warp and the squaring warps -- with the same
 ring sizes, barrier counts and phase arithmetic as the kernel, run over
 sequences of work items (ragged tails, empty second tiles, single-segment
-heads, several items per CTA).  TMA loads and MMA commits complete
+heads, several items per CTA, and the quadratic form's longest-first order).  TMA loads and MMA commits complete
 asynchronously at random later times (one issuer's commits in order), and the
 roles interleave at random.  Checked: no deadlock, and every wait observes
 exactly the phase it intends (a barrier never runs two phases past a waiter,
@@ -235,8 +235,32 @@ def run_cases(prm, seeds, planted=False):
                          1000 * seed + c, prm, planted)
 
 
+QUADRATIC_CASES = [  # T, heads, CTAs (one segment: L = T)
+    (2300, 2, 4), (600, 160, 3), (130, 5, 1), (5000, 3, 5), (1152, 80, 7), (257, 1, 1),
+]
+
+
+def quadratic_items(n_ct, BH, grid, c):
+    """Items CTA c walks in the quadratic form: latest query tiles first, across
+    heads, dealt round-robin to the CTAs."""
+    return [(x % BH) * n_ct + (n_ct - 1 - x // BH) for x in range(c, n_ct * BH, grid)]
+
+
 def test_readout_protocol_is_deadlock_free_and_phase_exact():
     run_cases(KERNEL, seeds=range(2))
+
+
+def test_quadratic_schedule_is_deadlock_free_and_phase_exact():
+    cq = KERNEL['kQT'] * KERNEL['kTiles']
+    for T, BH, grid in QUADRATIC_CASES:
+        n_ct = (T + cq - 1) // cq
+        g = min(grid, n_ct * BH)
+        walked = []
+        for c in range(g):
+            items = quadratic_items(n_ct, BH, g, c)
+            walked += items
+            simulate(T, T, BH, items, 7 * T + c, KERNEL)
+        assert sorted(walked) == list(range(n_ct * BH))  # every item exactly once
 
 
 def test_model_catches_a_score_buffer_reused_across_items():
