@@ -110,6 +110,65 @@ kata_status kata_chunked_forward(const void *q, const void *k, const void *v, vo
                                  size_t workspace_bytes, kata_stream_t stream);
 
 /*
+ * The state after T tokens, without the outputs: S_T = sum_{s<T} phi(k_s) v_s^T
+ * and Z_T = sum_{s<T} k_s k_s^T, from the chunk states and their scan
+ * (gist.science summary 2.3; arXiv abstract, "exact O(T) chunked-state form"
+ * and "constant-time recurrent inference": the state a prefill hands to the
+ * recurrent decode).  It is also the first step of the sequence-sharded
+ * forward: each block of a long sequence computes its own total, and a later
+ * block starts from the sum of the earlier blocks' totals
+ * (kata_chunked_forward_from_state), the chunk scan taken one level up.
+ *
+ *   k      [B, H, T, dk]  dtype;  v  [B, H, T, dv]  dtype
+ *   state_out  [B, H, dk*dk, dv] fp32, required (layout as kata_chunked_forward)
+ *   z_out      [B, H, dk, dk] fp32, required
+ *   workspace  as kata_chunked_forward, of at least
+ *              kata_chunked_forward_workspace_bytes(...) bytes
+ *
+ * The outputs must not overlap k, v or each other.
+ */
+kata_status kata_chunked_state(const void *k, const void *v, int B, int H, int T, int dk, int dv,
+                               int C, kata_dtype dtype, float *state_out, float *z_out,
+                               void *workspace, size_t workspace_bytes, kata_stream_t stream);
+
+/*
+ * kata_chunked_forward continuing from a given state: tokens 0 .. T-1 of the
+ * call are preceded by a history whose state is S_0 = sum_m state_in[m],
+ * Z_0 = sum_m z_in[m] (m = 0 .. n_in-1), so
+ *
+ *   y_t = (phi(q_t)^T S_0 + sum_{s<=t} (q_t.k_s)^2 v_s)
+ *         / (q_t^T Z_0 q_t + sum_{s<=t} (q_t.k_s)^2)                (0 if 0)
+ *
+ * (the same chunked-state form with the initial state as the prefix of the
+ * first chunk: gist.science summary 2.3; arXiv abstract).  Uses: a long
+ * prompt processed in pieces, and the sequence-sharded forward, where block
+ * r passes the all-gathered totals of all blocks with n_in = r.
+ *
+ *   q, k, v, out, B .. dtype, workspace: as kata_chunked_forward (same size
+ *          query, same workspace).
+ *   state_in   n_in fp32 states [B, H, dk*dk, dv] (symmetric in (i, j), as
+ *              every state this library writes); state m starts at
+ *              state_in + m * s_stride (floats; a multiple of 4 when n_in > 1).
+ *   z_in       n_in fp32 [B, H, dk, dk]; z m starts at z_in + m * z_stride.
+ *              Separately stacked inputs take s_stride = B*H*dk*dk*dv and
+ *              z_stride = B*H*dk*dk; one gathered buffer of [S | Z] blocks
+ *              takes the block size for both.
+ *   n_in       number of inputs to sum, >= 0; 0 behaves as kata_chunked_forward
+ *              (state_in and z_in may then be NULL).
+ *   state_out, z_out  nullable (both or neither): S_0 + S_T and Z_0 + Z_T,
+ *              the state after the call's last token.  With n_in = 1 they may
+ *              be state_in and z_in themselves (updated in place); otherwise
+ *              they must not overlap the inputs.
+ */
+kata_status kata_chunked_forward_from_state(const void *q, const void *k, const void *v, void *out,
+                                            int B, int H, int T, int dk, int dv, int C,
+                                            kata_dtype dtype, const float *state_in,
+                                            const float *z_in, int n_in, size_t s_stride,
+                                            size_t z_stride, float *state_out, float *z_out,
+                                            void *workspace, size_t workspace_bytes,
+                                            kata_stream_t stream);
+
+/*
  * kata_chunked_forward without a caller-provided workspace, for callers that
  * cannot allocate device memory themselves: code running inside a host
  * framework that owns all device memory through its own pool, or a

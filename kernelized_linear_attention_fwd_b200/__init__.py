@@ -7,8 +7,10 @@ include/kata.h); ``binding`` marshals torch CUDA tensors into it.
 from .binding import (  # noqa: F401
     KataError,
     kata_chunked_forward,
+    kata_chunked_forward_from_state,
     kata_chunked_forward_noalloc,
     kata_chunked_forward_workspace_bytes,
+    kata_chunked_state,
     kata_decode_step,
     kata_get_device_status,
     kata_quadratic_forward,

@@ -30,6 +30,8 @@ EXPORTS = (
     "kata_status_string",
     "kata_chunked_forward_workspace_bytes",
     "kata_chunked_forward",
+    "kata_chunked_state",
+    "kata_chunked_forward_from_state",
     "kata_chunked_forward_noalloc",
     "kata_quadratic_forward",
     "kata_decode_step",
@@ -66,6 +68,11 @@ def load_library(path: str = LIB_PATH):
     lib.kata_chunked_forward.restype = i32
     lib.kata_chunked_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
                                          fp, fp, vp, sz, vp]
+    lib.kata_chunked_state.restype = i32
+    lib.kata_chunked_state.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, fp, fp, vp, sz, vp]
+    lib.kata_chunked_forward_from_state.restype = i32
+    lib.kata_chunked_forward_from_state.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                                    i32, fp, fp, i32, sz, sz, fp, fp, vp, sz, vp]
     lib.kata_chunked_forward_noalloc.restype = i32
     lib.kata_chunked_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                  i32, fp, fp, vp]
@@ -158,6 +165,96 @@ def kata_chunked_forward(q, k, v, C=64, out=None, state_out=None, z_out=None, wo
                                   _stream_handle(stream))
     if st != KATA_OK:
         raise KataError(st, "kata_chunked_forward")
+    return out
+
+
+def _workspace(lib, workspace, B, H, T, dk, dv, C, code, device):
+    import torch
+
+    need = lib.kata_chunked_forward_workspace_bytes(B, H, T, dk, dv, C, code)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return workspace, nbytes
+
+
+def kata_chunked_state(k, v, C=64, state_out=None, z_out=None, workspace=None, stream=None):
+    """(S [B,H,dk*dk,dv], Z [B,H,dk,dk]) fp32: the state after the T tokens of
+    k, v [B,H,T,*], without the outputs.  Allocated here when not given."""
+    import torch
+
+    lib = load_library()
+    B, H, T, dk = k.shape
+    dv = v.shape[-1]
+    _check(k, "k", (B, H, T, dk))
+    _check(v, "v", (B, H, T, dv), k.dtype)
+    code = _dtype_code(k)
+    if state_out is None:
+        state_out = torch.empty((B, H, dk * dk, dv), dtype=torch.float32, device=k.device)
+    if z_out is None:
+        z_out = torch.empty((B, H, dk, dk), dtype=torch.float32, device=k.device)
+    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32)
+    _check(z_out, "z_out", (B, H, dk, dk), torch.float32)
+    workspace, nbytes = _workspace(lib, workspace, B, H, T, dk, dv, C, code, k.device)
+    st = lib.kata_chunked_state(_ptr(k), _ptr(v), B, H, T, dk, dv, int(C), code, _ptr(state_out),
+                                _ptr(z_out), _ptr(workspace), nbytes, _stream_handle(stream))
+    if st != KATA_OK:
+        raise KataError(st, "kata_chunked_state")
+    return state_out, z_out
+
+
+def _stacked(t, name, inner, n_name):
+    """(n, stride in elements) of a stack of states: t is [n, *inner] whose
+    blocks t[m] are each contiguous (any stride between blocks), or one state
+    [*inner] (n = 1)."""
+    import torch
+
+    if t is None:
+        return 0, 0
+    if not t.is_cuda or t.dtype != torch.float32:
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} must be a CUDA float32 tensor")
+    if tuple(t.shape) == tuple(inner):
+        t = t.unsqueeze(0)
+    if t.dim() != len(inner) + 1 or tuple(t.shape[1:]) != tuple(inner):
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} has shape {tuple(t.shape)}, want "
+                                              f"[{n_name}, {', '.join(map(str, inner))}]")
+    if t.shape[0] > 0 and not t[0].is_contiguous():
+        raise KataError(KATA_ERR_INVALID_ARG, f"each state of {name} must be contiguous")
+    return t.shape[0], t.stride(0)
+
+
+def kata_chunked_forward_from_state(q, k, v, state_in, z_in, C=64, out=None, state_out=None,
+                                    z_out=None, workspace=None, stream=None):
+    """out[B,H,T,dv]: the chunked forward of q, k, v continuing from the state
+    sum_m state_in[m], sum_m z_in[m].  state_in is [n, B, H, dk*dk, dv] (or one
+    [B, H, dk*dk, dv] state), z_in [n, B, H, dk, dk]; each state contiguous,
+    any stride between them.  state_out / z_out (optional) receive the state
+    after the last token; they may be state_in / z_in themselves for one input."""
+    import torch
+
+    lib = load_library()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    _check(q, "q", (B, H, T, dk))
+    _check(k, "k", (B, H, T, dk), q.dtype)
+    _check(v, "v", (B, H, T, dv), q.dtype)
+    code = _dtype_code(q)
+    n_s, s_stride = _stacked(state_in, "state_in", (B, H, dk * dk, dv), "n")
+    n_z, z_stride = _stacked(z_in, "z_in", (B, H, dk, dk), "n")
+    if n_s != n_z:
+        raise KataError(KATA_ERR_INVALID_ARG, f"state_in holds {n_s} states, z_in {n_z}")
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", (B, H, T, dv), q.dtype)
+    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32)
+    _check(z_out, "z_out", (B, H, dk, dk), torch.float32)
+    workspace, nbytes = _workspace(lib, workspace, B, H, T, dk, dv, C, code, q.device)
+    st = lib.kata_chunked_forward_from_state(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv, int(C), code,
+        _ptr(state_in) if n_s else None, _ptr(z_in) if n_z else None, n_s, s_stride, z_stride,
+        _ptr(state_out), _ptr(z_out), _ptr(workspace), nbytes, _stream_handle(stream))
+    if st != KATA_OK:
+        raise KataError(st, "kata_chunked_forward_from_state")
     return out
 
 

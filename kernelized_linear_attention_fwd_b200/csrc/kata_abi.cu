@@ -73,7 +73,7 @@ kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dty
     }
     const size_t E = (size_t)p.R * (dv + 1);
     const size_t seg_bytes = (size_t)BH * p.n_seg * E * sizeof(float);
-    const size_t total_bytes = p.n_seg > 1 ? (size_t)BH * E * sizeof(float) : 0;
+    const size_t total_bytes = (size_t)BH * E * sizeof(float);  // also for one segment + initial state
     p.ws_seg_state = 0;
     p.ws_total = align_up(seg_bytes);
     p.ws_extra = p.ws_total + align_up(total_bytes);
@@ -109,10 +109,38 @@ kata_status check_forward_io(const Plan &p, const void *q, const void *k, const 
 }
 
 cudaError_t launch_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
-                           float *state_out, float *z_out, void *ws, cudaStream_t st) {
+                           float *state_out, float *z_out, const InitState &init, void *ws,
+                           cudaStream_t st) {
     return p.path == Path::kTensorCore
-               ? tc::launch_tc_forward(p, q, k, v, out, state_out, z_out, ws, st)
-               : launch_simt_forward(p, q, k, v, out, state_out, z_out, ws, st);
+               ? tc::launch_tc_forward(p, q, k, v, out, state_out, z_out, init, ws, st)
+               : launch_simt_forward(p, q, k, v, out, state_out, z_out, init, ws, st);
+}
+
+// Workspace present, large enough and 256-byte aligned when the plan needs one.
+kata_status check_workspace(const Plan &p, const void *workspace, size_t workspace_bytes) {
+    if (p.ws_bytes == 0) return KATA_OK;
+    if (!workspace || workspace_bytes < p.ws_bytes) return KATA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_WORKSPACE;
+    return KATA_OK;
+}
+
+// state_out and z_out: both or neither, 16-byte aligned, disjoint from each
+// other and from the inputs.
+kata_status check_state_out(const Plan &p, const float *state_out, const float *z_out,
+                            const void *q, const void *k, const void *v, bool required) {
+    if ((state_out == nullptr) != (z_out == nullptr)) return KATA_ERR_INVALID_ARG;
+    if (!state_out) return required ? KATA_ERR_INVALID_ARG : KATA_OK;
+    if (!aligned16(state_out) || !aligned16(z_out)) return KATA_ERR_INVALID_ARG;
+    const size_t es = p.dtype == KATA_BF16 ? 2 : 4;
+    const size_t ns = (size_t)p.BH * p.dk * p.dk * p.dv * 4, nz = (size_t)p.BH * p.dk * p.dk * 4;
+    const size_t nq = (size_t)p.BH * p.T * p.dk * es, nv = (size_t)p.BH * p.T * p.dv * es;
+    if (overlaps(state_out, ns, z_out, nz)) return KATA_ERR_INVALID_ARG;
+    for (const float *o : {state_out, z_out}) {
+        const size_t n = o == state_out ? ns : nz;
+        if ((q && overlaps(o, n, q, nq)) || overlaps(o, n, k, nq) || overlaps(o, n, v, nv))
+            return KATA_ERR_INVALID_ARG;
+    }
+    return KATA_OK;
 }
 
 }  // namespace
@@ -155,14 +183,77 @@ kata_status kata_chunked_forward(const void *q, const void *k, const void *v, vo
     if (ps != KATA_OK) return ps;
     const kata_status io = kata::check_forward_io(p, q, k, v, out);
     if (io != KATA_OK) return io;
-    if ((state_out == nullptr) != (z_out == nullptr)) return KATA_ERR_INVALID_ARG;
-    if (state_out && (!aligned16(state_out) || !aligned16(z_out))) return KATA_ERR_INVALID_ARG;
-    if (p.ws_bytes > 0) {
-        if (!workspace || workspace_bytes < p.ws_bytes) return KATA_ERR_WORKSPACE;
-        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KATA_ERR_WORKSPACE;
-    }
+    const kata_status so = kata::check_state_out(p, state_out, z_out, q, k, v, false);
+    if (so != KATA_OK) return so;
+    const kata_status ws = kata::check_workspace(p, workspace, workspace_bytes);
+    if (ws != KATA_OK) return ws;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const cudaError_t e = kata::launch_forward(p, q, k, v, out, state_out, z_out, workspace, st);
+    const cudaError_t e =
+        kata::launch_forward(p, q, k, v, out, state_out, z_out, kata::InitState{}, workspace, st);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+}
+
+kata_status kata_chunked_state(const void *k, const void *v, int B, int H, int T, int dk, int dv,
+                               int C, kata_dtype dtype, float *state_out, float *z_out,
+                               void *workspace, size_t workspace_bytes, kata_stream_t stream) {
+    Plan p;
+    const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p);
+    if (ps != KATA_OK) return ps;
+    if (!k || !v || !aligned16(k) || !aligned16(v)) return KATA_ERR_INVALID_ARG;
+    const kata_status so = kata::check_state_out(p, state_out, z_out, nullptr, k, v, true);
+    if (so != KATA_OK) return so;
+    const kata_status ws = kata::check_workspace(p, workspace, workspace_bytes);
+    if (ws != KATA_OK) return ws;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = kata::launch_forward(p, nullptr, k, v, nullptr, state_out, z_out,
+                                               kata::InitState{}, workspace, st);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+}
+
+kata_status kata_chunked_forward_from_state(const void *q, const void *k, const void *v, void *out,
+                                            int B, int H, int T, int dk, int dv, int C,
+                                            kata_dtype dtype, const float *state_in,
+                                            const float *z_in, int n_in, size_t s_stride,
+                                            size_t z_stride, float *state_out, float *z_out,
+                                            void *workspace, size_t workspace_bytes,
+                                            kata_stream_t stream) {
+    Plan p;
+    const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p);
+    if (ps != KATA_OK) return ps;
+    const kata_status io = kata::check_forward_io(p, q, k, v, out);
+    if (io != KATA_OK) return io;
+    const kata_status so = kata::check_state_out(p, state_out, z_out, q, k, v, false);
+    if (so != KATA_OK) return so;
+    if (n_in < 0) return KATA_ERR_INVALID_ARG;
+    kata::InitState init;
+    if (n_in > 0) {
+        if (!state_in || !z_in || !aligned16(state_in) || !aligned16(z_in))
+            return KATA_ERR_INVALID_ARG;
+        if (n_in > 1 && s_stride % 4 != 0) return KATA_ERR_INVALID_ARG;  // 16-byte rows
+        const size_t ns = (size_t)p.BH * dk * dk * dv * 4, nz = (size_t)p.BH * dk * dk * 4;
+        const size_t span_s = (size_t)(n_in - 1) * s_stride * 4 + ns;
+        const size_t span_z = (size_t)(n_in - 1) * z_stride * 4 + nz;
+        const size_t no = (size_t)p.BH * T * dv * (dtype == KATA_BF16 ? 2 : 4);
+        if (overlaps(out, no, state_in, span_s) || overlaps(out, no, z_in, span_z))
+            return KATA_ERR_INVALID_ARG;
+        // every input is read before the state is written: state_out may be state_in
+        // itself (one input, updated in place) but must not overlap the inputs otherwise
+        const bool in_place = n_in == 1 && state_out == state_in && z_out == z_in;
+        if (state_out && !in_place &&
+            (overlaps(state_out, ns, state_in, span_s) || overlaps(state_out, ns, z_in, span_z) ||
+             overlaps(z_out, nz, state_in, span_s) || overlaps(z_out, nz, z_in, span_z)))
+            return KATA_ERR_INVALID_ARG;
+        init.s = state_in;
+        init.z = z_in;
+        init.n = n_in;
+        init.s_stride = (long long)s_stride;
+        init.z_stride = (long long)z_stride;
+    }
+    const kata_status ws = kata::check_workspace(p, workspace, workspace_bytes);
+    if (ws != KATA_OK) return ws;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e =
+        kata::launch_forward(p, q, k, v, out, state_out, z_out, init, workspace, st);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
 }
 
@@ -176,7 +267,8 @@ kata_status kata_quadratic_forward(const void *q, const void *k, const void *v, 
     if (io != KATA_OK) return io;
     if (p.BH * ((T + 255LL) / 256) >= 0x7fffffffLL) return KATA_ERR_UNSUPPORTED;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const cudaError_t e = kata::launch_forward(p, q, k, v, out, nullptr, nullptr, nullptr, st);
+    const cudaError_t e =
+        kata::launch_forward(p, q, k, v, out, nullptr, nullptr, kata::InitState{}, nullptr, st);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
 }
 

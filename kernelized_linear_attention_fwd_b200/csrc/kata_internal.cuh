@@ -84,16 +84,27 @@ __device__ __forceinline__ void store_out(__nv_bfloat16 *p, long long i, float x
     p[i] = __float2bfloat16_rn(x);
 }
 
-// Launchers (return cudaSuccess or the launch error).
+// Initial state of a forward: the sum of n dense states, S [B, H, dk*dk, dv]
+// and Z [B, H, dk, dk] fp32; input m starts s_stride (z_stride) floats after
+// input m - 1.  n = 0: the forward starts from the empty state.
+struct InitState {
+    const float *s = nullptr;
+    const float *z = nullptr;
+    int n = 0;
+    long long s_stride = 0, z_stride = 0;
+};
+
+// Launchers (return cudaSuccess or the launch error).  out == nullptr skips
+// the readout (state only: state_out and z_out are then required).
 cudaError_t launch_simt_forward(const Plan &p, const void *q, const void *k, const void *v,
-                                void *out, float *state_out, float *z_out, void *ws,
-                                cudaStream_t st);
+                                void *out, float *state_out, float *z_out, const InitState &init,
+                                void *ws, cudaStream_t st);
 namespace tc {
 // Tensor-core path (bf16, d = dv = 64): workspace layout and launcher.
 void plan_tc_workspace(Plan &p);
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v,
-                              void *out, float *state_out, float *z_out, void *ws,
-                              cudaStream_t st);
+                              void *out, float *state_out, float *z_out, const InitState &init,
+                              void *ws, cudaStream_t st);
 // Streaming multiprocessors of the current device (cached).
 int num_sms();
 }  // namespace tc

@@ -90,12 +90,15 @@ seg_state_build(const TIn *__restrict__ k, const TIn *__restrict__ v, float *__r
 // of 32 segments x 32 elements are staged through shared memory (coalesced
 // loads and stores along elements), each warp then scans element columns
 // across 32 segments with a Kogge-Stone shuffle scan (5 steps) and carries
-// the column total into the next tile.
+// the column total into the next tile.  An initial state (the sum of n_in
+// dense states) seeds the carries, so every prefix, segment 0's included,
+// and the total contain it.
 // grid.x = element-tile + n_et * bh; block (32, 8)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 seg_scan(float *__restrict__ seg_state, float *__restrict__ total, long long E, int n_seg,
-         int n_valid) {
+         int n_valid, int dk, int dv, const float *__restrict__ init_s,
+         const float *__restrict__ init_z, int n_in, long long s_stride, long long z_stride) {
     __shared__ float tile[32][33];
     const int lane = threadIdx.x, w = threadIdx.y;
     const long long n_et = (E + 31) / 32;
@@ -104,6 +107,18 @@ seg_scan(float *__restrict__ seg_state, float *__restrict__ total, long long E, 
     const long long e_base = et * 32;
     float *base = seg_state + bh * (long long)n_seg * E;
     float carry[4] = {0.f, 0.f, 0.f, 0.f};
+    const long long R = E / (dv + 1);
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {  // packed element e = row (i, j): dense row i * dk + j
+        const long long e = e_base + threadIdx.y + 8 * cc;
+        if (e >= E) continue;
+        const bool z_part = e >= R * dv;
+        int i, j;
+        packed_row_ij(dk, (int)(z_part ? e - R * dv : e / dv), i, j);
+        for (int n = 0; n < n_in; ++n)
+            carry[cc] += z_part ? init_z[n * z_stride + (bh * dk + i) * dk + j]
+                                : init_s[n * s_stride + ((bh * dk + i) * dk + j) * dv + e % dv];
+    }
 
     for (int g0 = 0; g0 < n_seg; g0 += 32) {
         // load 32 segments x 32 elements
@@ -165,7 +180,8 @@ struct ReadSmem {
 template <int DK, int DV, typename TIn>
 __global__ void __launch_bounds__(256)
 seg_read(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
-         TIn *__restrict__ out, const float *__restrict__ seg_state, int T, int L, int n_seg) {
+         TIn *__restrict__ out, const float *__restrict__ seg_state, int T, int L, int n_seg,
+         bool has_init) {
     constexpr int R = packed_rows(DK);
     constexpr long long E = (long long)R * (DV + 1);
     constexpr int TE = DV / 16;
@@ -215,7 +231,8 @@ seg_read(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__rest
     __syncthreads();
 
     // inter-segment term: phi(q)^T S_prev and q^T Z_prev q, from the packed prefix
-    if (g > 0) {
+    // (segment 0 has one when the forward starts from a given state)
+    if (g > 0 || has_init) {
         const float *Sg = seg_state + (bh * n_seg + g) * E;
         for (int r0 = 0; r0 < R; r0 += kRowB) {
             for (int x = tid; x < kRowB * DV; x += 256) {
@@ -334,7 +351,7 @@ state_expand(const float *__restrict__ total, long long stride_bh, float *__rest
 
 template <int DK, int DV, typename TIn>
 cudaError_t run(const Plan &p, const TIn *q, const TIn *k, const TIn *v, TIn *out,
-                float *state_out, float *z_out, void *ws, cudaStream_t st) {
+                float *state_out, float *z_out, const InitState &init, void *ws, cudaStream_t st) {
     constexpr int R = packed_rows(DK);
     constexpr long long E = (long long)R * (DV + 1);
     const long long BH = p.BH;
@@ -342,8 +359,13 @@ cudaError_t run(const Plan &p, const TIn *q, const TIn *k, const TIn *v, TIn *ou
     char *w = static_cast<char *>(ws);
     float *seg = w ? reinterpret_cast<float *>(w + p.ws_seg_state) : nullptr;
     float *total = w ? reinterpret_cast<float *>(w + p.ws_total) : nullptr;
+    const bool readout = out != nullptr;
     const bool want_state = state_out != nullptr;
+    const bool has_init = init.n > 0;
+    // the last segment's increment is needed only for the total
     const int n_build = want_state ? p.n_seg : p.n_seg - 1;
+    const bool scan = p.n_seg > 1 || has_init;
+    if ((has_init || n_build > 0 || want_state) && !w) return cudaErrorInvalidValue;
 
     if (n_build > 0) {
         const long long grid = (long long)((R + 31) / 32) * n_build * BH;
@@ -351,13 +373,14 @@ cudaError_t run(const Plan &p, const TIn *q, const TIn *k, const TIn *v, TIn *ou
         seg_state_build<DK, DV, TIn><<<(unsigned)grid, 256, 0, st>>>(k, v, seg, p.T, p.L, p.n_seg,
                                                                      n_build);
     }
-    if (p.n_seg > 1) {
+    if (scan) {
         const long long grid = ((E + 31) / 32) * BH;
         ProfScope ps("seg_scan", st);
         seg_scan<<<(unsigned)grid, dim3(32, 8), 0, st>>>(seg, want_state ? total : nullptr, E,
-                                                         p.n_seg, n_build);
+                                                         p.n_seg, n_build, DK, DV, init.s, init.z,
+                                                         init.n, init.s_stride, init.z_stride);
     }
-    {
+    if (readout) {
         using SM = ReadSmem<DK, DV>;
         cudaError_t e = cudaFuncSetAttribute(seg_read<DK, DV, TIn>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -366,11 +389,11 @@ cudaError_t run(const Plan &p, const TIn *q, const TIn *k, const TIn *v, TIn *ou
         const long long grid = (long long)((p.T + kTok - 1) / kTok) * BH;
         ProfScope ps("simt_seg_read", st);
         seg_read<DK, DV, TIn><<<(unsigned)grid, 256, SM::kBytes, st>>>(q, k, v, out, seg, p.T,
-                                                                        p.L, p.n_seg);
+                                                                        p.L, p.n_seg, has_init);
     }
     if (want_state) {
-        const float *src = p.n_seg > 1 ? total : seg;
-        const long long stride = p.n_seg > 1 ? E : E * p.n_seg;
+        const float *src = scan ? total : seg;
+        const long long stride = scan ? E : E * p.n_seg;
         const long long n = ((long long)DK * DK * DV + DK * DK) * BH;
         ProfScope ps("state_expand", st);
         state_expand<DK, DV><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, stride, state_out,
@@ -381,15 +404,15 @@ cudaError_t run(const Plan &p, const TIn *q, const TIn *k, const TIn *v, TIn *ou
 
 template <typename TIn>
 cudaError_t dispatch(const Plan &p, const void *q, const void *k, const void *v, void *out,
-                     float *so, float *zo, void *ws, cudaStream_t st) {
+                     float *so, float *zo, const InitState &init, void *ws, cudaStream_t st) {
     const TIn *Q = static_cast<const TIn *>(q);
     const TIn *K = static_cast<const TIn *>(k);
     const TIn *V = static_cast<const TIn *>(v);
     TIn *O = static_cast<TIn *>(out);
     switch (p.dk) {
-        case 16: return run<16, 16, TIn>(p, Q, K, V, O, so, zo, ws, st);
-        case 32: return run<32, 32, TIn>(p, Q, K, V, O, so, zo, ws, st);
-        case 64: return run<64, 64, TIn>(p, Q, K, V, O, so, zo, ws, st);
+        case 16: return run<16, 16, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
+        case 32: return run<32, 32, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
+        case 64: return run<64, 64, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -397,11 +420,11 @@ cudaError_t dispatch(const Plan &p, const void *q, const void *k, const void *v,
 }  // namespace
 
 cudaError_t launch_simt_forward(const Plan &p, const void *q, const void *k, const void *v,
-                                void *out, float *state_out, float *z_out, void *ws,
-                                cudaStream_t st) {
+                                void *out, float *state_out, float *z_out, const InitState &init,
+                                void *ws, cudaStream_t st) {
     if (p.dtype == KATA_BF16)
-        return dispatch<__nv_bfloat16>(p, q, k, v, out, state_out, z_out, ws, st);
-    return dispatch<float>(p, q, k, v, out, state_out, z_out, ws, st);
+        return dispatch<__nv_bfloat16>(p, q, k, v, out, state_out, z_out, init, ws, st);
+    return dispatch<float>(p, q, k, v, out, state_out, z_out, init, ws, st);
 }
 
 }  // namespace kata

@@ -34,7 +34,10 @@ constexpr long long kBf16PerSeg = (long long)kBf16Rows * kD;  // 147,456 bf16
 // ---------------------------------------------------------------------------
 // Exclusive prefix over segments (the associative scan across chunk states)
 // -> bf16 copy for the readout (Z split into hi and lo parts), and the fp32
-// total.  Reduce-then-scan per block of 128 consecutive elements of one head
+// total.  An initial state (the sum of n_in dense states) seeds the running
+// sum, so every prefix and the total include it and segment 0 gets a prefix
+// too; prefix == nullptr computes the total only.
+// Reduce-then-scan per block of 128 consecutive elements of one head
 // (32 lanes x float4): warp w takes a run of kScanRun consecutive segments,
 // holds them in registers and forms their running sums; the 8 run totals are
 // scanned across warps in shared memory in log2(8) = 3 steps; each warp adds
@@ -51,7 +54,8 @@ __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
 
 __global__ void __launch_bounds__(256)
 tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ prefix,
-            float *__restrict__ total, int n_seg, int n_valid) {
+            float *__restrict__ total, int n_seg, int n_valid, const float *__restrict__ init_s,
+            const float *__restrict__ init_z, int n_in, long long s_stride, long long z_stride) {
     __shared__ float4 part[2][kScanWarps][32];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     constexpr long long E = kF32PerSeg;
@@ -72,7 +76,24 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
         zi[x] = pij.i;
         zj[x] = pij.j;
     }
+    // the initial state of these 4 packed elements: dense rows i * 64 + j
     float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int n = 0; n < n_in; ++n) {
+        if (!z_part) {
+            const PairIJ pij = row_ij((int)(e0 / kD));
+            if (pij.i <= pij.j)
+                carry = f4add(carry, *reinterpret_cast<const float4 *>(
+                                         init_s + n * s_stride +
+                                         ((bh * kD + pij.i) * kD + pij.j) * kD + e0 % kD));
+        } else {
+            const float *zn = init_z + n * z_stride + bh * kD * kD;
+            float zv[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) zv[x] = zi[x] <= zj[x] ? zn[zi[x] * kD + zj[x]] : 0.f;
+            carry = f4add(carry, make_float4(zv[0], zv[1], zv[2], zv[3]));
+        }
+    }
+    const int g_first = n_in > 0 ? 0 : 1;  // without one, segment 0 has an empty prefix
 
     for (int g0 = 0; g0 < n_seg; g0 += kScanWarps * kScanRun) {
         const int gw = g0 + w * kScanRun;
@@ -109,7 +130,7 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
 #pragma unroll
         for (int i = 0; i < kScanRun; ++i) {
             const int g = gw + i;
-            if (g < 1 || g >= n_seg) continue;  // segment 0 has an empty prefix
+            if (prefix == nullptr || g < g_first || g >= n_seg) continue;
             const float4 p = f4add(v[i], off);
             __nv_bfloat16 *dst = pbase + (long long)g * kBf16PerSeg;
             if (!z_part) {
@@ -232,14 +253,15 @@ struct ReadItem {
     bool inter;
 };
 
-__device__ __forceinline__ ReadItem read_item(int i, int n_ct, int T, int L, int n_seg) {
+// has_init: the forward starts from a given state, so segment 0 has a prefix too.
+__device__ __forceinline__ ReadItem read_item(int i, int n_ct, int T, int L, int n_seg, bool has_init) {
     ReadItem it;
     it.bh = i / n_ct;
     it.t0 = (i % n_ct) * kCtaQ;
     const int g = it.t0 / L;
     it.seg0 = g * L;
     it.sidx = it.bh * n_seg + g;
-    it.inter = g > 0;
+    it.inter = g > 0 || has_init;
     const int tend = min(it.t0 + kCtaQ, T);
     it.n_kv = (tend - it.seg0 + kKB - 1) / kKB;
     return it;
@@ -764,7 +786,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
 tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
         const __grid_constant__ CUtensorMap tm_o, int T, int L, int n_seg, int n_ct, int n_items,
-        int *status) {
+        bool has_init, int *status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ ReadBars bars;
     __shared__ uint32_t tmem_base;
@@ -824,7 +846,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             int n_q = 0, n_bs = 0, n_kv = 0;  // loads issued into each ring
             bool ok = true;
             for (int x = sched.first; x < sched.end && ok; x += sched.stride) {
-                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg);
+                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg, has_init);
                 {
                     const int qb = n_q & 1;
                     uint8_t *slot = sm + kSmItem + qb * kItemBytes;
@@ -879,7 +901,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             int n_inter = 0, g_kv = 0, g_b0 = 0, g_b1 = 0, j = 0;
             bool ok = true;
             for (int x = sched.first; x < sched.end && ok; x += sched.stride, ++j) {
-                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg);
+                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg, has_init);
                 const int qb = j & 1;
                 const uint32_t slot = smem_u32(sm + kSmItem + qb * kItemBytes);
                 ok = mbar_wait(&bars.qfull[qb], (j >> 1) & 1, abort);
@@ -1008,7 +1030,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             tma_prefetch_desc(&tm_o);
             int j = 0;
             for (int x = sched.first; x < sched.end; x += sched.stride, ++j) {
-                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg);
+                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg, has_init);
                 const int qb = j & 1;
                 if (!mbar_wait(&bars.ostaged, j & 1, abort)) break;
                 for (int t = 0; t < kTiles; ++t)
@@ -1040,7 +1062,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         int n_inter = 0, g_b = 0, j = 0;
         bool ok = true;
         for (int x = sched.first; x < sched.end && ok; x += sched.stride, ++j) {
-            const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg);
+            const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg, has_init);
             const int qb = j & 1;
             if (lane == 0) mbar_arrive(&bars.genin);
             ok = __all_sync(0xffffffffu, mbar_wait(&bars.qfull[qb], (j >> 1) & 1, abort));
@@ -1222,19 +1244,25 @@ void plan_tc_workspace(Plan &p) {
 }
 
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
-                              float *state_out, float *z_out, void *ws, cudaStream_t st) {
+                              float *state_out, float *z_out, const InitState &init, void *ws,
+                              cudaStream_t st) {
     // no workspace (the quadratic plan): no state is built, scanned or read
     char *w = static_cast<char *>(ws);
     float *seg = w ? reinterpret_cast<float *>(w + p.ws_seg_state) : nullptr;
     float *total = w ? reinterpret_cast<float *>(w + p.ws_total) : nullptr;
     __nv_bfloat16 *prefix = w ? reinterpret_cast<__nv_bfloat16 *>(w + p.ws_extra) : nullptr;
     __nv_bfloat16 *kt = w ? reinterpret_cast<__nv_bfloat16 *>(w + p.ws_aux) : nullptr;
+    const bool readout = out != nullptr;
     const bool want_state = state_out != nullptr;
+    const bool has_init = init.n > 0;
+    // the last segment's increment is needed only for the total
     const int n_build = want_state ? p.n_seg : p.n_seg - 1;
+    const bool scan = p.n_seg > 1 || has_init;
     const long long BH = p.BH;
     const int T_pad = (p.T + 63) / 64 * 64;
     int *status = device_status_ptr();
     if (!status) return cudaErrorUnknown;
+    if ((has_init || n_build > 0 || want_state) && !w) return cudaErrorInvalidValue;
 
     if (n_build > 0) {
         {
@@ -1264,13 +1292,15 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
         tc_build<<<(unsigned)grid, kBuildThreads, kBSmAlloc, st>>>(mkt, mvb, mst, seg, p.T, p.L, p.n_seg,
                                                                     n_build, (int)n_items, status);
     }
-    if (p.n_seg > 1) {
+    if (scan) {
         ProfScope ps("tc_seg_scan", st);
         const long long grid = (kF32PerSeg / 128) * BH;
-        tc_seg_scan<<<(unsigned)grid, 256, 0, st>>>(seg, prefix, want_state ? total : nullptr,
-                                                     p.n_seg, n_build);
+        tc_seg_scan<<<(unsigned)grid, 256, 0, st>>>(seg, readout ? prefix : nullptr,
+                                                     want_state ? total : nullptr, p.n_seg, n_build,
+                                                     init.s, init.z, init.n, init.s_stride,
+                                                     init.z_stride);
     }
-    {
+    if (readout) {
         CUtensorMap mq, mk, mv, ms, mo;
         if (!make_maps(p, q, k, v, prefix, out, &mq, &mk, &mv, &ms, &mo)) return cudaErrorInvalidValue;
         cudaError_t e = cudaFuncSetAttribute(tc_read, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1282,11 +1312,11 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
         const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
         ProfScope ps("tc_read", st);
         tc_read<<<(unsigned)grid, kReadThreads, kSmAlloc, st>>>(
-            mq, mk, mv, ms, mo, p.T, p.L, p.n_seg, n_ct, (int)n_items, status);
+            mq, mk, mv, ms, mo, p.T, p.L, p.n_seg, n_ct, (int)n_items, has_init, status);
     }
     if (want_state) {
-        const float *src = p.n_seg > 1 ? total : seg;
-        const long long stride = p.n_seg > 1 ? kF32PerSeg : kF32PerSeg * p.n_seg;
+        const float *src = scan ? total : seg;
+        const long long stride = scan ? kF32PerSeg : kF32PerSeg * p.n_seg;
         const long long n = ((long long)kD * kD * kD + kD * kD) * BH;
         ProfScope ps("tc_state_expand", st);
         tc_state_expand<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, stride, state_out, z_out, BH);

@@ -13,6 +13,14 @@ from kernelized_linear_attention_fwd_b200 import inputs
 # (zero denominator) must be exactly zero.
 TOL = {"f32": 1e-4, "bf16": 2e-2}
 
+# Bound of an exported state entry: |S - S_ref| <= u * B (+1e-6), with
+# B = sum_s |k_si k_sj v_se| the state of |k|, |v| (for Z, v = 1).  bf16: the
+# tensor-core path rounds each product k_si k_sj to bf16 (unit roundoff 2^-9)
+# before the fp32 accumulation, so 2^-9 B plus the fp32 accumulation stays
+# within 2^-8 B; fp32 rounds only in fp32 (2^-16 B covers T <= 2^16 tokens of
+# random-walk accumulation error).
+STATE_BOUND = {"f32": 2.0 ** -16, "bf16": 2.0 ** -8}
+
 
 def to_device(a: np.ndarray, dtype: str):
     import torch

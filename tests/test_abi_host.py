@@ -20,6 +20,13 @@ HEADER = os.path.join(ROOT, "include", "kata.h")
 
 @pytest.fixture(scope="module")
 def lib():
+    # The calls below pass fake device addresses that only the host-side checks
+    # may see; on a machine with a GPU a check that failed to reject one would
+    # launch a kernel on them, so these tests run only where no GPU is visible.
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("host-side ABI checks use fake device pointers: run without a GPU")
     kbuild.build()
     return binding.load_library()
 
@@ -124,6 +131,55 @@ def test_quadratic_forward_rejects_bad_arguments(lib):
     assert quad(dk=64, dv=32) == E.KATA_ERR_UNSUPPORTED
     assert quad(dt=2) == E.KATA_ERR_UNSUPPORTED
     assert quad(out=FAKE + 0x20000000 + 256) == E.KATA_ERR_INVALID_ARG  # out inside v
+
+
+def test_state_only_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    E = binding
+    need = lib.kata_chunked_forward_workspace_bytes(1, 1, 4096, 16, 16, 64, 0)
+
+    def cs(k=FAKE, v=FAKE + 0x10000000, so=FAKE + 0x40000000, zo=FAKE + 0x48000000, T=4096,
+           dk=16, C=64, ws=FAKE + 0x50000000, wsb=None):
+        return lib.kata_chunked_state(vp(k) if k else None, vp(v) if v else None, 1, 1, T, dk, dk,
+                                      C, 0, vp(so) if so else None, vp(zo) if zo else None,
+                                      vp(ws) if ws else None, need if wsb is None else wsb, None)
+
+    assert cs(k=0) == E.KATA_ERR_INVALID_ARG
+    assert cs(so=0, zo=0) == E.KATA_ERR_INVALID_ARG              # the state is the output
+    assert cs(zo=0) == E.KATA_ERR_INVALID_ARG
+    assert cs(so=FAKE + 0x40000004) == E.KATA_ERR_INVALID_ARG    # misaligned
+    assert cs(so=FAKE + 0x10000000) == E.KATA_ERR_INVALID_ARG    # state_out over v
+    assert cs(zo=FAKE + 0x40000000 + 4096) == E.KATA_ERR_INVALID_ARG  # z_out inside state_out
+    assert cs(C=40) == E.KATA_ERR_INVALID_ARG
+    assert cs(dk=48) == E.KATA_ERR_UNSUPPORTED
+    assert cs(ws=0, wsb=0) == E.KATA_ERR_WORKSPACE
+    assert cs(wsb=need - 1) == E.KATA_ERR_WORKSPACE
+
+
+def test_forward_from_state_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    E = binding
+    need = lib.kata_chunked_forward_workspace_bytes(1, 1, 64, 16, 16, 64, 0)
+    S0, Z0 = FAKE + 0x60000000, FAKE + 0x68000000
+
+    def ffs(q=FAKE, out=FAKE + 0x30000000, si=S0, zi=Z0, n=1, ss=0, zs=0, so=None, zo=None):
+        return lib.kata_chunked_forward_from_state(
+            vp(q) if q else None, vp(FAKE + 0x10000000), vp(FAKE + 0x20000000),
+            vp(out) if out else None, 1, 1, 64, 16, 16, 64, 0, vp(si) if si else None,
+            vp(zi) if zi else None, n, ss, zs, vp(so) if so else None, vp(zo) if zo else None,
+            vp(FAKE + 0x50000000), need, None)
+
+    assert ffs(q=0) == E.KATA_ERR_INVALID_ARG
+    assert ffs(n=-1) == E.KATA_ERR_INVALID_ARG
+    assert ffs(si=0) == E.KATA_ERR_INVALID_ARG                   # n_in = 1 needs both inputs
+    assert ffs(zi=0) == E.KATA_ERR_INVALID_ARG
+    assert ffs(si=S0 + 8) == E.KATA_ERR_INVALID_ARG              # misaligned
+    assert ffs(n=3, ss=16 * 16 * 16 + 2, zs=256) == E.KATA_ERR_INVALID_ARG  # rows off 16 bytes
+    assert ffs(out=S0) == E.KATA_ERR_INVALID_ARG                 # out over an input state
+    # state_out overlapping the inputs, unless it is the one input itself
+    assert ffs(n=2, ss=4096, zs=256, so=S0 + 4 * 4096, zo=Z0 + 0x100000) == E.KATA_ERR_INVALID_ARG
+    assert ffs(so=S0 + 256, zo=Z0 + 256) == E.KATA_ERR_INVALID_ARG
+    assert ffs(so=S0, zo=0) == E.KATA_ERR_INVALID_ARG            # both or neither
 
 
 def test_decode_rejects_bad_arguments(lib):

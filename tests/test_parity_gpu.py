@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 
 from kernelized_linear_attention_fwd_b200 import inputs
-from tests.gpu_util import TOL, from_device, row_err, sample_rows, to_device
+from tests.gpu_util import STATE_BOUND, TOL, from_device, row_err, sample_rows, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -180,14 +180,9 @@ def test_convex_combination_invariant():
 # ---------------------------------------------------------------------------
 
 
-# Elementwise error bound of an exported state entry, relative to
-# B = sum_s |k_si k_sj v_se| (the state of |k| and |v|; for Z, v = 1):  the
-# bf16 tensor-core path rounds each product k_si k_sj to bf16 (unit roundoff
-# 2^-9) before the fp32 accumulation, so |S - S_ref| <= 2^-9 B + (fp32
-# accumulation) <= 2^-8 B;
-# the fp32 path rounds only in fp32 (2^-16 B covers T <= 2^8 * 2^8 tokens of
-# random-walk accumulation error).
-STATE_BOUND = {"f32": 2.0 ** -16, "bf16": 2.0 ** -8}
+# STATE_BOUND (tests/gpu_util.py): elementwise error bound of an exported
+# state entry, relative to B = sum_s |k_si k_sj v_se| (the state of |k| and
+# |v|; for Z, v = 1).
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])

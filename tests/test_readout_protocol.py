@@ -5,7 +5,9 @@ issuers (alternate inter stages; scores Q K^T by issuer 0, weights times values
 by issuer 1), the output-store warp and the squaring warps -- with the same
 ring sizes, barrier counts and phase arithmetic as the kernel, run over
 sequences of work items (ragged tails, empty second tiles, single-segment
-heads, several items per CTA, and the quadratic form's longest-first order).  TMA loads and MMA commits complete
+heads, several items per CTA, the quadratic form's longest-first order, and
+first-segment items with an inter phase when the forward starts from a given
+state).  TMA loads and MMA commits complete
 asynchronously at random later times (one issuer's commits in order), and the
 roles interleave at random.  Checked: no deadlock, and every wait observes
 exactly the phase it intends (a barrier never runs two phases past a waiter,
@@ -44,7 +46,7 @@ class Bar:
         return (self.phase & 1) != parity
 
 
-def simulate(T, L, BH, items, seed, prm, planted=False):
+def simulate(T, L, BH, items, seed, prm, planted=False, init=False):
     kQT, kTiles, kSB, kKB = prm['kQT'], prm['kTiles'], prm['kSB'], prm['kKB']
     kKVRing, kRStages, kRRing, kRBRing, kSlots = (prm['kKVRing'], prm['kRStages'], prm['kRRing'],
                                                   prm['kRBRing'], prm['kItemSlots'])
@@ -69,7 +71,7 @@ def simulate(T, L, BH, items, seed, prm, planted=False):
     def item(i):
         t0 = (i % n_ct) * kCtaQ
         seg0 = (t0 // L) * L
-        return dict(t0=t0, seg0=seg0, inter=seg0 > 0,
+        return dict(t0=t0, seg0=seg0, inter=seg0 > 0 or init,
                     n_kv=(min(t0 + kCtaQ, T) - seg0 + kKB - 1) // kKB)
 
     def blocks(it, t):
@@ -248,6 +250,21 @@ def quadratic_items(n_ct, BH, grid, c):
 
 def test_readout_protocol_is_deadlock_free_and_phase_exact():
     run_cases(KERNEL, seeds=range(2))
+
+
+def test_initial_state_gives_every_item_an_inter_phase():
+    # a forward from a given state: first-segment items read a prefix too
+    cq = KERNEL['kQT'] * KERNEL['kTiles']
+    for T, L, BH, grid in CASES[:4]:
+        n_items = (T + cq - 1) // cq * BH
+        g = min(grid, n_items)
+        for c in range(g):
+            items = list(range(c * n_items // g, (c + 1) * n_items // g))
+            simulate(T, L, BH, items, 11 * T + c, KERNEL, init=True)
+        if T <= L:  # one segment: the longest-first order
+            n_ct = (T + cq - 1) // cq
+            for c in range(g):
+                simulate(T, T, BH, quadratic_items(n_ct, BH, g, c), 13 * T + c, KERNEL, init=True)
 
 
 def test_quadratic_schedule_is_deadlock_free_and_phase_exact():
