@@ -426,7 +426,19 @@ def run_ours(args, rank, world):
                   "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
                   "frac": gbs / peaks["hbm_gbs"], "frac_of_8tbs_spec": gbs / SPEC_HBM_GBS,
                   "peak_source": src}
+        # the same steps on the packed layout (rows i <= j: half the bytes)
+        Sp, Zp = K.kata_state_pack(Sd, Zd, stream=stream)
         del Sd, Zd
+        pms = max_over_ranks(time_launches(
+            lambda: K.kata_decode_step_packed(qd_, kd_, vd_, Sp, Zp, out=od, stream=stream),
+            stream, lambda: None, nd, warm=5), world)
+        R = d * (d + 1) // 2
+        pbytes = Bd * Hd * ((R * d + R) * 4 * 2 + 4 * d * es)
+        pgbs = pbytes / (pms / 1e3) / 1e9
+        decode["packed"] = {"ms_per_step": pms, "tokens_per_s": world * Bd / (pms / 1e3),
+                            "bytes_per_step": pbytes, "achieved_gbs": pgbs,
+                            "frac": pgbs / peaks["hbm_gbs"], "speedup_vs_dense": dmean / pms}
+        del Sp, Zp
 
     # the quadratic (flash-attention-style) form of the same forward
     quad = None
@@ -434,6 +446,12 @@ def run_ours(args, rank, world):
         quad = measure_quadratic(K, q, k, v, out, stream, flush, world, rank, ms_max, n=3)
         if K.kata_get_device_status() != 0:
             raise RuntimeError("device status set by the quadratic form")
+
+    # one rank's compute of the sequence-sharded forward, on this GPU
+    seq_split = None
+    if not args.no_quadratic and w.dtype == "bf16":
+        fwd_ms = sum(t for n, (c, t) in prof.items() if "decode" not in n) / args.steps
+        seq_split = measure_sequence_split(K, q, k, v, C, stream, flush, fwd_ms)
 
     if rank != 0:
         return None
@@ -504,6 +522,7 @@ def run_ours(args, rank, world):
         "clocks": clk,
         "decode": decode,
         "quadratic_form": quad,
+        "sequence_split": seq_split,
         "device_status": status,
         "forward_canonical": canon,
     }
@@ -589,6 +608,49 @@ def measure_quadratic(K, q, k, v, out, stream, flush, world, rank, chunked_ms, n
                 "backend": backend, "ms": fa, "achieved_tflops": fl / (fa / 1e3) / 1e12,
                 "quadratic_speedup": fa / ms, "chunked_step_speedup": fa / chunked_ms,
                 "note": "context only: softmax attention of the same B, H, T, d, causal"}
+    return res
+
+
+def measure_sequence_split(K, q, k, v, C, stream, flush, chunked_ms, splits=(2, 8)):
+    """Per-rank compute of the sequence-sharded forward, on this one GPU: the
+    block of one of N ranks (T / N tokens of every head) through
+    kata_chunked_state and kata_chunked_forward_from_state with N - 1 gathered
+    totals as inputs (the last rank's work).  The all-gather itself is not
+    run (it needs N GPUs)."""
+    import torch
+
+    from kernelized_linear_attention_fwd_b200 import sharded
+
+    B, H, T, d = q.shape
+    res = {}
+    for N in splits:
+        if T % N:
+            continue
+        Tb = T // N
+        bq, bk, bv = (x[:, :, :Tb].contiguous() for x in (q, k, v))
+        flat = sharded.block_state(bk, bv, C)
+        gathered = flat.repeat(N, 1)  # stands in for the N gathered totals
+        out = torch.empty_like(bq)
+        ws = torch.empty(max(K.kata_chunked_forward_workspace_bytes(B, H, Tb, d, d, C, 1), 256),
+                         dtype=torch.uint8, device=q.device)
+        ns, nz = sharded.state_numel(B, H, d, d)
+        S = flat[:ns].view(B, H, d * d, d)
+        Z = flat[ns:].view(B, H, d, d)
+        s_in, z_in = sharded.gathered_views(gathered, N - 1, B, H, d, d)
+
+        def rank_work():
+            K.kata_chunked_state(bk, bv, C=C, state_out=S, z_out=Z, workspace=ws, stream=stream)
+            K.kata_chunked_forward_from_state(bq, bk, bv, s_in, z_in, C=C, out=out, workspace=ws,
+                                              stream=stream)
+
+        ms = time_launches(rank_work, stream, flush, 5)
+        res[f"N{N}"] = {"tokens_per_rank": B * Tb, "per_rank_ms": ms,
+                        "ideal_ms": chunked_ms / N, "compute_efficiency": chunked_ms / N / ms,
+                        "projected_tokens_per_s": B * T / (ms / 1e3)}
+        del bq, bk, bv, flat, gathered, out, ws
+    res["note"] = ("one GPU: one rank's compute (state pass + forward from N-1 gathered totals) "
+                   "against the single-GPU forward's kernel time / N; the all-gather of the "
+                   "totals (1 MiB + 16 KiB per head) is not included")
     return res
 
 

@@ -249,6 +249,32 @@ kata_status kata_decode_step(const void *q, const void *k, const void *v, void *
                              kata_dtype dtype, kata_stream_t stream);
 
 /*
+ * Packed state layout for decode.  The state is symmetric in (i, j), so the
+ * rows i <= j hold all of it: R = dk(dk+1)/2 rows, i outer, row
+ * r(i, j) = i*dk - i(i-1)/2 + (j - i), each the plain sum over tokens of
+ * k_i k_j v (state) or k_i k_j (normaliser); the readout weighs row (i, j) by
+ * 2 q_i q_j off the diagonal and q_i^2 on it, which gives the same
+ * phi(q)^T S = sum_{i,j} q_i q_j S_ij (gist.science summary 2.2: the weight
+ * is the squared inner product, symmetric in the feature indices).  Half the
+ * bytes of the dense layout, so the HBM-bound decode step moves half the data.
+ *
+ *   state_p  [B, H, R, dv] fp32      z_p  [B, H, R] fp32
+ *
+ * kata_state_pack converts a dense state (as the forward exports it) into
+ * this layout, reading the rows i <= j; kata_state_unpack writes both (i, j)
+ * and (j, i) of the dense layout from row r(i, j).  Sources and destinations
+ * must not overlap.  kata_decode_step_packed is kata_decode_step on this
+ * layout: same arguments, same results up to fp32 summation order.
+ */
+kata_status kata_state_pack(const float *state, const float *z, float *state_p, float *z_p, int B,
+                            int H, int dk, int dv, kata_stream_t stream);
+kata_status kata_state_unpack(const float *state_p, const float *z_p, float *state, float *z,
+                              int B, int H, int dk, int dv, kata_stream_t stream);
+kata_status kata_decode_step_packed(const void *q, const void *k, const void *v, void *out,
+                                    float *state_p, float *z_p, int B, int H, int dk, int dv,
+                                    kata_dtype dtype, kata_stream_t stream);
+
+/*
  * Synchronises `stream`, returns and clears the device status word that
  * kernels set when an on-device check fails (KATA_OK if none did), or
  * KATA_ERR_CUDA if the synchronisation itself reports an error.

@@ -12,8 +12,11 @@ from .binding import (  # noqa: F401
     kata_chunked_forward_workspace_bytes,
     kata_chunked_state,
     kata_decode_step,
+    kata_decode_step_packed,
     kata_get_device_status,
     kata_quadratic_forward,
+    kata_state_pack,
+    kata_state_unpack,
     kata_status_string,
     kata_version,
     load_library,

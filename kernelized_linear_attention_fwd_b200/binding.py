@@ -35,6 +35,9 @@ EXPORTS = (
     "kata_chunked_forward_noalloc",
     "kata_quadratic_forward",
     "kata_decode_step",
+    "kata_decode_step_packed",
+    "kata_state_pack",
+    "kata_state_unpack",
     "kata_get_device_status",
 )
 
@@ -80,6 +83,11 @@ def load_library(path: str = LIB_PATH):
     lib.kata_quadratic_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
     lib.kata_decode_step.restype = i32
     lib.kata_decode_step.argtypes = [vp, vp, vp, vp, fp, fp, i32, i32, i32, i32, i32, vp]
+    lib.kata_decode_step_packed.restype = i32
+    lib.kata_decode_step_packed.argtypes = [vp, vp, vp, vp, fp, fp, i32, i32, i32, i32, i32, vp]
+    for name in ("kata_state_pack", "kata_state_unpack"):
+        getattr(lib, name).restype = i32
+        getattr(lib, name).argtypes = [fp, fp, fp, fp, i32, i32, i32, i32, vp]
     lib.kata_get_device_status.restype = i32
     lib.kata_get_device_status.argtypes = [vp]
     _lib = lib
@@ -334,6 +342,83 @@ def kata_decode_step(q, k, v, state, z, out=None, stream=None):
     if st != KATA_OK:
         raise KataError(st, "kata_decode_step")
     return out
+
+
+def packed_rows(d: int) -> int:
+    """Rows of the packed state layout: the pairs i <= j."""
+    return d * (d + 1) // 2
+
+
+def kata_decode_step_packed(q, k, v, state_p, z_p, out=None, stream=None):
+    """kata_decode_step on the packed layout: state_p [B,H,R,dv], z_p [B,H,R],
+    R = dk(dk+1)/2, updated in place."""
+    import torch
+
+    lib = load_library()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    R = packed_rows(dk)
+    _check(q, "q", (B, H, dk))
+    _check(k, "k", (B, H, dk), q.dtype)
+    _check(v, "v", (B, H, dv), q.dtype)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", (B, H, dv), q.dtype)
+    _check(state_p, "state_p", (B, H, R, dv), torch.float32)
+    _check(z_p, "z_p", (B, H, R), torch.float32)
+    st = lib.kata_decode_step_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state_p),
+                                     _ptr(z_p), B, H, dk, dv, code, _stream_handle(stream))
+    if st != KATA_OK:
+        raise KataError(st, "kata_decode_step_packed")
+    return out
+
+
+def kata_state_pack(state, z, state_p=None, z_p=None, stream=None):
+    """Dense (state [B,H,dk*dk,dv], z [B,H,dk,dk]) -> packed (state_p, z_p)."""
+    import torch
+
+    lib = load_library()
+    B, H, dd, dv = state.shape
+    dk = z.shape[-1]
+    R = packed_rows(dk)
+    _check(state, "state", (B, H, dk * dk, dv), torch.float32)
+    _check(z, "z", (B, H, dk, dk), torch.float32)
+    if state_p is None:
+        state_p = torch.empty((B, H, R, dv), dtype=torch.float32, device=state.device)
+    if z_p is None:
+        z_p = torch.empty((B, H, R), dtype=torch.float32, device=state.device)
+    _check(state_p, "state_p", (B, H, R, dv), torch.float32)
+    _check(z_p, "z_p", (B, H, R), torch.float32)
+    st = lib.kata_state_pack(_ptr(state), _ptr(z), _ptr(state_p), _ptr(z_p), B, H, dk, dv,
+                             _stream_handle(stream))
+    if st != KATA_OK:
+        raise KataError(st, "kata_state_pack")
+    return state_p, z_p
+
+
+def kata_state_unpack(state_p, z_p, state=None, z=None, stream=None):
+    """Packed (state_p [B,H,R,dv], z_p [B,H,R]) -> dense (state, z)."""
+    import torch
+
+    lib = load_library()
+    B, H, R, dv = state_p.shape
+    dk = next(d for d in (16, 32, 64) if packed_rows(d) == R) if R in (136, 528, 2080) else 0
+    if dk == 0:
+        raise KataError(KATA_ERR_UNSUPPORTED, f"no supported head size has {R} packed rows")
+    _check(state_p, "state_p", (B, H, R, dv), torch.float32)
+    _check(z_p, "z_p", (B, H, R), torch.float32)
+    if state is None:
+        state = torch.empty((B, H, dk * dk, dv), dtype=torch.float32, device=state_p.device)
+    if z is None:
+        z = torch.empty((B, H, dk, dk), dtype=torch.float32, device=state_p.device)
+    _check(state, "state", (B, H, dk * dk, dv), torch.float32)
+    _check(z, "z", (B, H, dk, dk), torch.float32)
+    st = lib.kata_state_unpack(_ptr(state_p), _ptr(z_p), _ptr(state), _ptr(z), B, H, dk, dv,
+                               _stream_handle(stream))
+    if st != KATA_OK:
+        raise KataError(st, "kata_state_unpack")
+    return state, z
 
 
 def kata_get_device_status(stream=None) -> int:

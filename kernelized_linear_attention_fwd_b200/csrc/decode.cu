@@ -13,6 +13,12 @@
 // With few heads, each head is split over a thread-block cluster of P CTAs
 // (so the whole GPU streams the state) and the P partial readouts are summed
 // through distributed shared memory: no global scratch, no atomics.
+//
+// Two state layouts: dense (d^2 rows i * d + j, the layout the forward
+// exports) and packed (the d(d+1)/2 rows i <= j, i outer, weighted c_ij = 2
+// off the diagonal and 1 on it at readout), which holds the same information
+// in half the bytes, so the step moves half the data.  Pack and unpack
+// kernels convert between them.
 #include <cooperative_groups.h>
 
 #include "kata_internal.cuh"
@@ -28,25 +34,40 @@ constexpr int kMaxParts = 8;  // portable cluster size
 template <int DV>
 constexpr int rows_per_pass() { return kThreads / (DV / 4); }
 
-// Largest split of a head's DK * DK rows into P parts (a power of two, at most
-// kMaxParts) that still gives every CTA whole passes.
-template <int DK, int DV>
+template <int DK, bool PACKED>
+constexpr int state_rows() { return PACKED ? DK * (DK + 1) / 2 : DK * DK; }
+
+// Largest split of a head's rows into P parts (a power of two, at most
+// kMaxParts) that still gives every CTA at least one full pass.
+template <int DK, int DV, bool PACKED>
 constexpr int max_parts() {
     int p = 1;
-    while (2 * p <= kMaxParts && (DK * DK) / (2 * p) >= rows_per_pass<DV>()) p *= 2;
+    while (2 * p <= kMaxParts && state_rows<DK, PACKED>() / (2 * p) >= rows_per_pass<DV>()) p *= 2;
     return p;
 }
 
-template <int DK, int DV, int P, typename TIn>
+// (i, j), i <= j, of packed row r: the largest i with start(i) <= r, start(i) =
+// i d - i (i - 1) / 2; the square-root estimate is corrected to the exact i.
+template <int DK>
+__device__ __forceinline__ void packed_ij(int r, int &i, int &j) {
+    constexpr float b = 2.f * DK + 1.f;
+    int a = (int)((b - sqrtf(b * b - 8.f * (float)r)) * 0.5f);
+    a = a < 0 ? 0 : (a > DK - 1 ? DK - 1 : a);
+    while (a > 0 && a * DK - a * (a - 1) / 2 > r) --a;
+    while (a < DK - 1 && (a + 1) * DK - (a + 1) * a / 2 <= r) ++a;
+    i = a;
+    j = a + (r - (a * DK - a * (a - 1) / 2));
+}
+
+template <int DK, int DV, int P, bool PACKED, typename TIn>
 __global__ void __launch_bounds__(kThreads)
 decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
                    TIn *__restrict__ out, float *__restrict__ S, float *__restrict__ Z) {
-    constexpr int ROWS = DK * DK;
-    constexpr int PROWS = ROWS / P;          // rows of this CTA's slice
+    constexpr int ROWS = state_rows<DK, PACKED>();
     constexpr int V4 = DV / 4;               // float4 slots per state row
     constexpr int RPI = kThreads / V4;       // rows covered per pass
-    constexpr int UNR = (PROWS / RPI) < kUnroll ? (PROWS / RPI) : kUnroll;
-    static_assert(PROWS % (RPI * UNR) == 0, "rows must tile the passes");
+    constexpr int UNR = (ROWS / P / RPI) < kUnroll ? (ROWS / P / RPI) : kUnroll;
+    static_assert(UNR >= 1, "every CTA covers at least one pass");
     __shared__ float sq[DK], sk[DK], sv[DV];
     __shared__ float red[RPI][DV + 1];
     __shared__ float redz[kThreads / 32];
@@ -55,7 +76,8 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
     const int tid = threadIdx.x;
     const long long bh = blockIdx.x / P;
     const int part = blockIdx.x % P;         // = the block's rank in its cluster
-    const int row_base = part * PROWS;
+    const int row_base = part * ROWS / P;    // this CTA's slice [row_base, row_end)
+    const int row_end = (part + 1) * ROWS / P;
     if (tid < DK) {
         sq[tid] = load_f32(q, bh * DK + tid);
         sk[tid] = load_f32(k, bh * DK + tid);
@@ -68,15 +90,24 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
     float4 *Sh = reinterpret_cast<float4 *>(S + bh * (long long)ROWS * DV);
     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 
-    for (int row0 = row_base + rg; row0 < row_base + PROWS; row0 += RPI * UNR) {
+    for (int row0 = row_base + rg; row0 < row_end; row0 += RPI * UNR) {
         float4 s[UNR];
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) s[u] = Sh[(long long)(row0 + u * RPI) * V4 + c4];
+        for (int u = 0; u < UNR; ++u)
+            if (row0 + u * RPI < row_end) s[u] = Sh[(long long)(row0 + u * RPI) * V4 + c4];
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            const int row = row0 + u * RPI, i = row / DK, j = row % DK;
+            const int row = row0 + u * RPI;
+            if (row >= row_end) continue;
+            int i, j;
+            if constexpr (PACKED) {
+                packed_ij<DK>(row, i, j);
+            } else {
+                i = row / DK;
+                j = row % DK;
+            }
             const float f = sk[i] * sk[j];
-            const float w = sq[i] * sq[j];
+            const float w = (PACKED && i != j ? 2.f : 1.f) * (sq[i] * sq[j]);
             s[u].x = fmaf(f, vv.x, s[u].x);
             s[u].y = fmaf(f, vv.y, s[u].y);
             s[u].z = fmaf(f, vv.z, s[u].z);
@@ -87,17 +118,24 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
             a3 = fmaf(w, s[u].w, a3);
         }
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) Sh[(long long)(row0 + u * RPI) * V4 + c4] = s[u];
+        for (int u = 0; u < UNR; ++u)
+            if (row0 + u * RPI < row_end) Sh[(long long)(row0 + u * RPI) * V4 + c4] = s[u];
     }
 
     // normaliser: Z += k k^T, den = q^T Z q (this CTA's slice of the d^2 entries)
     float dz = 0.f;
     float *Zh = Z + bh * (long long)ROWS;
-    for (int x = row_base + tid; x < row_base + PROWS; x += kThreads) {
-        const int i = x / DK, j = x % DK;
+    for (int x = row_base + tid; x < row_end; x += kThreads) {
+        int i, j;
+        if constexpr (PACKED) {
+            packed_ij<DK>(x, i, j);
+        } else {
+            i = x / DK;
+            j = x % DK;
+        }
         const float z = Zh[x] + sk[i] * sk[j];
         Zh[x] = z;
-        dz = fmaf(sq[i] * sq[j], z, dz);
+        dz = fmaf((PACKED && i != j ? 2.f : 1.f) * (sq[i] * sq[j]), z, dz);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) dz += __shfl_xor_sync(0xffffffffu, dz, off);
@@ -136,10 +174,10 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
     }
 }
 
-template <int DK, int DV, int P, typename TIn>
+template <int DK, int DV, int P, bool PACKED, typename TIn>
 cudaError_t launch_parts(int BH, const void *q, const void *k, const void *v, void *out, float *S,
                          float *Z, cudaStream_t st) {
-    auto kern = decode_step_kernel<DK, DV, P, TIn>;
+    auto kern = decode_step_kernel<DK, DV, P, PACKED, TIn>;
     const TIn *qq = static_cast<const TIn *>(q), *kk = static_cast<const TIn *>(k),
               *vv = static_cast<const TIn *>(v);
     TIn *oo = static_cast<TIn *>(out);
@@ -163,42 +201,122 @@ cudaError_t launch_parts(int BH, const void *q, const void *k, const void *v, vo
     }
 }
 
-template <int DK, int DV, typename TIn>
+template <int DK, int DV, bool PACKED, typename TIn>
 cudaError_t run(int BH, const void *q, const void *k, const void *v, void *out, float *S,
                 float *Z, cudaStream_t st) {
     // split heads over clusters while a CTA per head would leave SMs idle
+    constexpr int MP = max_parts<DK, DV, PACKED>();
     int parts = 1;
     const int sms = tc::num_sms();
-    while (parts < max_parts<DK, DV>() && (long long)BH * parts < sms) parts *= 2;
-    ProfScope ps("decode_step", st);
+    while (parts < MP && (long long)BH * parts < sms) parts *= 2;
+    ProfScope ps(PACKED ? "decode_step_packed" : "decode_step", st);
     switch (parts) {
-        case 1: return launch_parts<DK, DV, 1, TIn>(BH, q, k, v, out, S, Z, st);
-        case 2: return launch_parts<DK, DV, (max_parts<DK, DV>() >= 2 ? 2 : 1), TIn>(BH, q, k, v, out, S, Z, st);
-        case 4: return launch_parts<DK, DV, (max_parts<DK, DV>() >= 4 ? 4 : 1), TIn>(BH, q, k, v, out, S, Z, st);
-        default: return launch_parts<DK, DV, (max_parts<DK, DV>() >= 8 ? 8 : 1), TIn>(BH, q, k, v, out, S, Z, st);
+        case 1: return launch_parts<DK, DV, 1, PACKED, TIn>(BH, q, k, v, out, S, Z, st);
+        case 2: return launch_parts<DK, DV, (MP >= 2 ? 2 : 1), PACKED, TIn>(BH, q, k, v, out, S, Z, st);
+        case 4: return launch_parts<DK, DV, (MP >= 4 ? 4 : 1), PACKED, TIn>(BH, q, k, v, out, S, Z, st);
+        default: return launch_parts<DK, DV, (MP >= 8 ? 8 : 1), PACKED, TIn>(BH, q, k, v, out, S, Z, st);
     }
 }
 
-template <typename TIn>
+template <bool PACKED, typename TIn>
 cudaError_t dispatch(int BH, int dk, const void *q, const void *k, const void *v, void *out,
                      float *S, float *Z, cudaStream_t st) {
     switch (dk) {
-        case 16: return run<16, 16, TIn>(BH, q, k, v, out, S, Z, st);
-        case 32: return run<32, 32, TIn>(BH, q, k, v, out, S, Z, st);
-        case 64: return run<64, 64, TIn>(BH, q, k, v, out, S, Z, st);
+        case 16: return run<16, 16, PACKED, TIn>(BH, q, k, v, out, S, Z, st);
+        case 32: return run<32, 32, PACKED, TIn>(BH, q, k, v, out, S, Z, st);
+        case 64: return run<64, 64, PACKED, TIn>(BH, q, k, v, out, S, Z, st);
         default: return cudaErrorInvalidValue;
     }
+}
+
+// Dense [BH, d*d, dv] + [BH, d*d]  ->  packed [BH, R, dv] + [BH, R]: row r = (i, j),
+// i <= j, takes dense row i * d + j.  One thread per packed float4 / z entry.
+template <int DK, int DV>
+__global__ void __launch_bounds__(256)
+state_pack(const float *__restrict__ S, const float *__restrict__ Z, float *__restrict__ Sp,
+           float *__restrict__ Zp, long long BH) {
+    constexpr int R = DK * (DK + 1) / 2, V4 = DV / 4;
+    constexpr long long per = (long long)R * V4 + R;
+    const long long idx = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (idx >= per * BH) return;
+    const long long bh = idx / per;
+    const long long x = idx % per;
+    int i, j;
+    if (x < (long long)R * V4) {
+        const int r = (int)(x / V4), c = (int)(x % V4);
+        packed_ij<DK>(r, i, j);
+        reinterpret_cast<float4 *>(Sp)[(bh * R + r) * V4 + c] =
+            reinterpret_cast<const float4 *>(S)[(bh * DK * DK + i * DK + j) * V4 + c];
+    } else {
+        const int r = (int)(x - (long long)R * V4);
+        packed_ij<DK>(r, i, j);
+        Zp[bh * R + r] = Z[bh * DK * DK + i * DK + j];
+    }
+}
+
+// Packed -> dense: dense row a * d + b (either order) takes packed row
+// (min(a, b), max(a, b)), so the result is symmetric.  One thread per dense
+// float4 / z entry.
+template <int DK, int DV>
+__global__ void __launch_bounds__(256)
+state_unpack(const float *__restrict__ Sp, const float *__restrict__ Zp, float *__restrict__ S,
+             float *__restrict__ Z, long long BH) {
+    constexpr int R = DK * (DK + 1) / 2, V4 = DV / 4;
+    constexpr long long per = (long long)DK * DK * V4 + DK * DK;
+    const long long idx = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (idx >= per * BH) return;
+    const long long bh = idx / per;
+    const long long x = idx % per;
+    const bool z_part = x >= (long long)DK * DK * V4;
+    const int dr = z_part ? (int)(x - (long long)DK * DK * V4) : (int)(x / V4);
+    const int a = dr / DK, b = dr % DK;
+    const int i = a < b ? a : b, j = a < b ? b : a;
+    const int r = i * DK - i * (i - 1) / 2 + (j - i);
+    if (z_part)
+        Z[bh * DK * DK + dr] = Zp[bh * R + r];
+    else
+        reinterpret_cast<float4 *>(S)[(bh * DK * DK + dr) * V4 + x % V4] =
+            reinterpret_cast<const float4 *>(Sp)[(bh * R + r) * V4 + x % V4];
+}
+
+template <int DK, int DV>
+cudaError_t convert(bool pack, long long BH, const float *src_s, const float *src_z, float *dst_s,
+                    float *dst_z, cudaStream_t st) {
+    constexpr long long R = DK * (DK + 1) / 2;
+    const long long per = pack ? R * (DV / 4) + R : (long long)DK * DK * (DV / 4) + DK * DK;
+    const unsigned grid = (unsigned)((per * BH + 255) / 256);
+    ProfScope ps(pack ? "state_pack" : "state_unpack", st);
+    if (pack)
+        state_pack<DK, DV><<<grid, 256, 0, st>>>(src_s, src_z, dst_s, dst_z, BH);
+    else
+        state_unpack<DK, DV><<<grid, 256, 0, st>>>(src_s, src_z, dst_s, dst_z, BH);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_decode(int B, int H, int dk, int dv, kata_dtype dtype, const void *q,
                           const void *k, const void *v, void *out, float *state, float *z,
-                          cudaStream_t st) {
+                          bool packed, cudaStream_t st) {
     (void)dv;
     const int BH = B * H;
-    if (dtype == KATA_BF16) return dispatch<__nv_bfloat16>(BH, dk, q, k, v, out, state, z, st);
-    return dispatch<float>(BH, dk, q, k, v, out, state, z, st);
+    if (packed)
+        return dtype == KATA_BF16
+                   ? dispatch<true, __nv_bfloat16>(BH, dk, q, k, v, out, state, z, st)
+                   : dispatch<true, float>(BH, dk, q, k, v, out, state, z, st);
+    return dtype == KATA_BF16 ? dispatch<false, __nv_bfloat16>(BH, dk, q, k, v, out, state, z, st)
+                              : dispatch<false, float>(BH, dk, q, k, v, out, state, z, st);
+}
+
+cudaError_t launch_state_convert(bool pack, int B, int H, int dk, const float *src_s,
+                                 const float *src_z, float *dst_s, float *dst_z, cudaStream_t st) {
+    const long long BH = (long long)B * H;
+    switch (dk) {
+        case 16: return convert<16, 16>(pack, BH, src_s, src_z, dst_s, dst_z, st);
+        case 32: return convert<32, 32>(pack, BH, src_s, src_z, dst_s, dst_z, st);
+        case 64: return convert<64, 64>(pack, BH, src_s, src_z, dst_s, dst_z, st);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace kata

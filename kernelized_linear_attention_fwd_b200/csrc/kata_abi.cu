@@ -143,6 +143,51 @@ kata_status check_state_out(const Plan &p, const float *state_out, const float *
     return KATA_OK;
 }
 
+// The decode step on either state layout.
+kata_status decode_step(const void *q, const void *k, const void *v, void *out, float *state,
+                        float *z, int B, int H, int dk, int dv, kata_dtype dtype, bool packed,
+                        kata_stream_t stream) {
+    if (B < 1 || H < 1 || dk < 1 || dv < 1) return KATA_ERR_INVALID_ARG;
+    if (dtype != KATA_F32 && dtype != KATA_BF16) return KATA_ERR_UNSUPPORTED;
+    if (dk != dv || (dk != 16 && dk != 32 && dk != 64)) return KATA_ERR_UNSUPPORTED;
+    if ((long long)B * H > 0x7fffffffLL / 8) return KATA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !out || !state || !z) return KATA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state) ||
+        !aligned16(z))
+        return KATA_ERR_INVALID_ARG;
+    const size_t es = dtype == KATA_BF16 ? 2 : 4;
+    const size_t BH = (size_t)B * H;
+    const size_t rows = packed ? (size_t)packed_rows(dk) : (size_t)dk * dk;
+    const size_t ns = BH * rows * dv * 4, nz = BH * rows * 4, no = BH * dv * es;
+    if (overlaps(state, ns, z, nz) || overlaps(out, no, state, ns) || overlaps(out, no, z, nz))
+        return KATA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = launch_decode(B, H, dk, dv, dtype, q, k, v, out, state, z, packed, st);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+}
+
+kata_status state_convert(bool pack, const float *src_s, const float *src_z, float *dst_s,
+                          float *dst_z, int B, int H, int dk, int dv, kata_stream_t stream) {
+    if (B < 1 || H < 1 || dk < 1 || dv < 1) return KATA_ERR_INVALID_ARG;
+    if (dk != dv || (dk != 16 && dk != 32 && dk != 64)) return KATA_ERR_UNSUPPORTED;
+    if (!src_s || !src_z || !dst_s || !dst_z) return KATA_ERR_INVALID_ARG;
+    if (!aligned16(src_s) || !aligned16(src_z) || !aligned16(dst_s) || !aligned16(dst_z))
+        return KATA_ERR_INVALID_ARG;
+    const size_t BH = (size_t)B * H;
+    const size_t dense_s = BH * dk * dk * dv * 4, dense_z = BH * dk * dk * 4;
+    const size_t pk_s = BH * packed_rows(dk) * dv * 4, pk_z = BH * packed_rows(dk) * 4;
+    const size_t ss = pack ? dense_s : pk_s, sz = pack ? dense_z : pk_z;
+    const size_t ds = pack ? pk_s : dense_s, dz = pack ? pk_z : dense_z;
+    for (const void *d : {static_cast<const void *>(dst_s), static_cast<const void *>(dst_z)}) {
+        const size_t n = d == dst_s ? ds : dz;
+        if (overlaps(d, n, src_s, ss) || overlaps(d, n, src_z, sz)) return KATA_ERR_INVALID_ARG;
+    }
+    if (overlaps(dst_s, ds, dst_z, dz)) return KATA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = launch_state_convert(pack, B, H, dk, src_s, src_z, dst_s, dst_z, st);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+}
+
 }  // namespace
 
 }  // namespace kata
@@ -275,22 +320,23 @@ kata_status kata_quadratic_forward(const void *q, const void *k, const void *v, 
 kata_status kata_decode_step(const void *q, const void *k, const void *v, void *out,
                              float *state, float *z, int B, int H, int dk, int dv,
                              kata_dtype dtype, kata_stream_t stream) {
-    if (B < 1 || H < 1 || dk < 1 || dv < 1) return KATA_ERR_INVALID_ARG;
-    if (dtype != KATA_F32 && dtype != KATA_BF16) return KATA_ERR_UNSUPPORTED;
-    if (dk != dv || (dk != 16 && dk != 32 && dk != 64)) return KATA_ERR_UNSUPPORTED;
-    if ((long long)B * H > 0x7fffffffLL) return KATA_ERR_UNSUPPORTED;
-    if (!q || !k || !v || !out || !state || !z) return KATA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(state) ||
-        !aligned16(z))
-        return KATA_ERR_INVALID_ARG;
-    const size_t es = dtype == KATA_BF16 ? 2 : 4;
-    const size_t BH = (size_t)B * H;
-    const size_t ns = BH * dk * dk * dv * 4, nz = BH * dk * dk * 4, no = BH * dv * es;
-    if (overlaps(state, ns, z, nz) || overlaps(out, no, state, ns) || overlaps(out, no, z, nz))
-        return KATA_ERR_INVALID_ARG;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const cudaError_t e = kata::launch_decode(B, H, dk, dv, dtype, q, k, v, out, state, z, st);
-    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+    return kata::decode_step(q, k, v, out, state, z, B, H, dk, dv, dtype, false, stream);
+}
+
+kata_status kata_decode_step_packed(const void *q, const void *k, const void *v, void *out,
+                                    float *state_p, float *z_p, int B, int H, int dk, int dv,
+                                    kata_dtype dtype, kata_stream_t stream) {
+    return kata::decode_step(q, k, v, out, state_p, z_p, B, H, dk, dv, dtype, true, stream);
+}
+
+kata_status kata_state_pack(const float *state, const float *z, float *state_p, float *z_p, int B,
+                            int H, int dk, int dv, kata_stream_t stream) {
+    return kata::state_convert(true, state, z, state_p, z_p, B, H, dk, dv, stream);
+}
+
+kata_status kata_state_unpack(const float *state_p, const float *z_p, float *state, float *z,
+                              int B, int H, int dk, int dv, kata_stream_t stream) {
+    return kata::state_convert(false, state_p, z_p, state, z, B, H, dk, dv, stream);
 }
 
 kata_status kata_get_device_status(kata_stream_t stream) {

@@ -109,8 +109,12 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
 int num_sms();
 }  // namespace tc
 
+// Decode step on the dense (d^2 rows) or packed (d(d+1)/2 rows) state layout.
 cudaError_t launch_decode(int B, int H, int dk, int dv, kata_dtype dtype, const void *q,
                           const void *k, const void *v, void *out, float *state, float *z,
-                          cudaStream_t st);
+                          bool packed, cudaStream_t st);
+// Dense <-> packed state conversion (pack: dense -> packed).
+cudaError_t launch_state_convert(bool pack, int B, int H, int dk, const float *src_s,
+                                 const float *src_z, float *dst_s, float *dst_z, cudaStream_t st);
 
 }  // namespace kata

@@ -203,6 +203,36 @@ def test_decode_rejects_bad_arguments(lib):
     assert dec(out=FAKE + 0x10000) == E.KATA_ERR_INVALID_ARG               # out inside S
 
 
+def test_packed_layout_calls_reject_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    E = binding
+    S, Z, Sp, Zp = FAKE + 0x10000, FAKE + 0x10000000, FAKE + 0x20000000, FAKE + 0x30000000
+
+    def dec(q=FAKE, S=Sp, Z=Zp, dk=16, dv=16, dt=0, out=FAKE + 0x300):
+        return lib.kata_decode_step_packed(vp(q) if q else None, vp(FAKE + 0x100),
+                                           vp(FAKE + 0x200), vp(out), vp(S) if S else None,
+                                           vp(Z) if Z else None, 1, 1, dk, dv, dt, None)
+
+    def conv(fn, a=S, b=Z, c=Sp, d=Zp, dk=16):
+        return fn(vp(a) if a else None, vp(b) if b else None, vp(c) if c else None,
+                  vp(d) if d else None, 1, 1, dk, dk, None)
+
+    assert dec(q=0) == E.KATA_ERR_INVALID_ARG
+    assert dec(S=0) == E.KATA_ERR_INVALID_ARG
+    assert dec(dk=48, dv=48) == E.KATA_ERR_UNSUPPORTED
+    assert dec(dt=4) == E.KATA_ERR_UNSUPPORTED
+    # packed z right after the packed state: 136 rows x 16 x 4 B; one byte less overlaps
+    assert dec(Z=Sp + 136 * 16 * 4 - 16) == E.KATA_ERR_INVALID_ARG
+    assert dec(out=Sp + 64) == E.KATA_ERR_INVALID_ARG
+    for fn in (lib.kata_state_pack, lib.kata_state_unpack):
+        assert conv(fn, a=0) == E.KATA_ERR_INVALID_ARG
+        assert conv(fn, d=0) == E.KATA_ERR_INVALID_ARG
+        assert conv(fn, c=Sp + 4) == E.KATA_ERR_INVALID_ARG         # misaligned
+        assert conv(fn, dk=24) == E.KATA_ERR_UNSUPPORTED
+        assert conv(fn, c=S + 64) == E.KATA_ERR_INVALID_ARG          # destination over source
+        assert conv(fn, d=Sp + 16) == E.KATA_ERR_INVALID_ARG         # destinations overlap
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     saved = binding._lib
     try:
