@@ -61,7 +61,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-quadratic", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the sub-measures beside the step (quadratic form, other workloads, sequence split)")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override the workload's T (smaller cases of the same workload for profiling)")
     return ap.parse_args()
@@ -442,16 +443,30 @@ def run_ours(args, rank, world):
 
     # the quadratic (flash-attention-style) form of the same forward
     quad = None
-    if not args.no_quadratic:
+    if not args.no_extras:
         quad = measure_quadratic(K, q, k, v, out, stream, flush, world, rank, ms_max, n=3)
         if K.kata_get_device_status() != 0:
             raise RuntimeError("device status set by the quadratic form")
 
+    # the chunked forward on the other forward workloads
+    others = None
+    if not args.no_extras and w.name == WORKLOAD:
+        others = measure_other_configs(K, inputs, stream, flush)
+
     # one rank's compute of the sequence-sharded forward, on this GPU
     seq_split = None
-    if not args.no_quadratic and w.dtype == "bf16":
+    if not args.no_extras and w.dtype == "bf16":
         fwd_ms = sum(t for n, (c, t) in prof.items() if "decode" not in n) / args.steps
-        seq_split = measure_sequence_split(K, q, k, v, C, stream, flush, fwd_ms)
+        def kernel_times(fn, n):  # per-kernel device ms per call, from the library's events
+            lib.kata_profile_enable(1)
+            for _ in range(n):
+                flush()
+                fn()
+            torch.cuda.synchronize()
+            lib.kata_profile_enable(0)
+            return {name: round(t / n, 4) for name, (c, t) in profile_read().items()}
+
+        seq_split = measure_sequence_split(K, q, k, v, C, stream, flush, fwd_ms, kernel_times)
 
     if rank != 0:
         return None
@@ -523,6 +538,7 @@ def run_ours(args, rank, world):
         "decode": decode,
         "quadratic_form": quad,
         "sequence_split": seq_split,
+        "other_workloads": others,
         "device_status": status,
         "forward_canonical": canon,
     }
@@ -611,7 +627,8 @@ def measure_quadratic(K, q, k, v, out, stream, flush, world, rank, chunked_ms, n
     return res
 
 
-def measure_sequence_split(K, q, k, v, C, stream, flush, chunked_ms, splits=(2, 8)):
+def measure_sequence_split(K, q, k, v, C, stream, flush, chunked_ms, kernel_times,
+                           splits=(2, 8)):
     """Per-rank compute of the sequence-sharded forward, on this one GPU: the
     block of one of N ranks (T / N tokens of every head) through
     kata_chunked_state and kata_chunked_forward_from_state with N - 1 gathered
@@ -638,19 +655,59 @@ def measure_sequence_split(K, q, k, v, C, stream, flush, chunked_ms, splits=(2, 
         Z = flat[ns:].view(B, H, d, d)
         s_in, z_in = sharded.gathered_views(gathered, N - 1, B, H, d, d)
 
-        def rank_work():
-            K.kata_chunked_state(bk, bv, C=C, state_out=S, z_out=Z, workspace=ws, stream=stream)
-            K.kata_chunked_forward_from_state(bq, bk, bv, s_in, z_in, C=C, out=out, workspace=ws,
-                                              stream=stream)
+        def rank_work():  # on the current stream (the capture stream while capturing)
+            K.kata_chunked_state(bk, bv, C=C, state_out=S, z_out=Z, workspace=ws)
+            K.kata_chunked_forward_from_state(bq, bk, bv, s_in, z_in, C=C, out=out, workspace=ws)
 
-        ms = time_launches(rank_work, stream, flush, 5)
-        res[f"N{N}"] = {"tokens_per_rank": B * Tb, "per_rank_ms": ms,
-                        "ideal_ms": chunked_ms / N, "compute_efficiency": chunked_ms / N / ms,
-                        "projected_tokens_per_s": B * T / (ms / 1e3)}
+        eager = time_launches(rank_work, stream, flush, 5)
+        # the same calls replayed from a CUDA graph: at a few hundred microseconds of
+        # GPU work per rank the host cannot issue them as fast as the GPU runs them
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                rank_work()
+            ms = time_launches(graph.replay, stream, flush, 10)
+            del graph
+        except Exception as e:  # report the eager time only
+            ms, res[f"N{N}_graph_error"] = None, f"{type(e).__name__}: {str(e)[:100]}"
+        best = ms if ms is not None else eager
+        res[f"N{N}"] = {"tokens_per_rank": B * Tb, "per_rank_ms": ms, "per_rank_ms_eager": eager,
+                        "ideal_ms": chunked_ms / N, "compute_efficiency": chunked_ms / N / best,
+                        "projected_tokens_per_s": B * T / (best / 1e3),
+                        "kernels_ms": kernel_times(rank_work, 3)}
         del bq, bk, bv, flat, gathered, out, ws
-    res["note"] = ("one GPU: one rank's compute (state pass + forward from N-1 gathered totals) "
-                   "against the single-GPU forward's kernel time / N; the all-gather of the "
-                   "totals (1 MiB + 16 KiB per head) is not included")
+    res["note"] = ("one GPU: one rank's compute (state pass + forward from N-1 gathered totals, "
+                   "replayed from a CUDA graph) against the single-GPU forward's kernel time / N; "
+                   "the all-gather of the totals (1 MiB + 16 KiB per head) is not included")
+    return res
+
+
+def measure_other_configs(K, inputs, stream, flush, names=("lm340m_B4H16_T16384_d64_bf16",
+                                                            "small_B2H4_T4096_d32_bf16")):
+    """The chunked forward (with state export) on the other forward workloads,
+    inputs generated on the device, L2 flushed before each launch."""
+    import torch
+
+    peaks, _ = load_peaks()
+    res = {}
+    for name in names:
+        w = inputs.WORKLOADS[name]
+        q, k, v = inputs.make_qkv_device(w.B, w.H, w.T, w.d, w.d, seed=w.seed)
+        so = torch.empty((w.B, w.H, w.d * w.d, w.d), dtype=torch.float32, device=q.device)
+        zo = torch.empty((w.B, w.H, w.d, w.d), dtype=torch.float32, device=q.device)
+        out = torch.empty_like(v)
+        ws = torch.empty(max(K.kata_chunked_forward_workspace_bytes(w.B, w.H, w.T, w.d, w.d, w.C,
+                                                                    1), 256),
+                         dtype=torch.uint8, device=q.device)
+        ms = time_launches(lambda: K.kata_chunked_forward(q, k, v, C=w.C, out=out, state_out=so,
+                                                          z_out=zo, workspace=ws),
+                           stream, flush, 10, warm=3)
+        canon = w.B * w.H * w.T * alg_flops_per_token_head("forward", w.d, w.d, w.C)
+        res[name] = {"ms": ms, "tokens_per_s": w.B * w.T / (ms / 1e3),
+                     "canonical_tflops": canon / (ms / 1e3) / 1e12,
+                     "frac_of_measured_peak": canon / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                     "path": "tensor cores" if w.d == 64 else "fp32 CUDA cores"}
+        del q, k, v, so, zo, out, ws
     return res
 
 

@@ -59,8 +59,13 @@ __device__ __forceinline__ void packed_ij(int r, int &i, int &j) {
     j = a + (r - (a * DK - a * (a - 1) / 2));
 }
 
+// CTAs per SM the register budget must allow (loads in flight per SM): 4 fit
+// the dense single-CTA kernel without spills, 3 the others.
+template <int P, bool PACKED>
+constexpr int min_ctas_per_sm() { return !PACKED && P == 1 ? 4 : 3; }
+
 template <int DK, int DV, int P, bool PACKED, typename TIn>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, min_ctas_per_sm<P, PACKED>())
 decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
                    TIn *__restrict__ out, float *__restrict__ S, float *__restrict__ Z) {
     constexpr int ROWS = state_rows<DK, PACKED>();
@@ -72,6 +77,8 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
     __shared__ float red[RPI][DV + 1];
     __shared__ float redz[kThreads / 32];
     __shared__ float part_num[DV], part_den;
+    // packed layout: (i, j) of each row of this CTA's slice, i | j << 8
+    __shared__ uint16_t sij[PACKED ? (ROWS + P - 1) / P + 1 : 1];
 
     const int tid = threadIdx.x;
     const long long bh = blockIdx.x / P;
@@ -83,6 +90,13 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
         sk[tid] = load_f32(k, bh * DK + tid);
     }
     if (tid < DV) sv[tid] = load_f32(v, bh * DV + tid);
+    if constexpr (PACKED) {
+        for (int r = row_base + tid; r < row_end; r += kThreads) {
+            int i, j;
+            packed_ij<DK>(r, i, j);
+            sij[r - row_base] = (uint16_t)(i | (j << 8));
+        }
+    }
     __syncthreads();
 
     const int c4 = tid % V4, rg = tid / V4;
@@ -101,7 +115,9 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
             if (row >= row_end) continue;
             int i, j;
             if constexpr (PACKED) {
-                packed_ij<DK>(row, i, j);
+                const int ij = sij[row - row_base];
+                i = ij & 255;
+                j = ij >> 8;
             } else {
                 i = row / DK;
                 j = row % DK;
@@ -128,7 +144,9 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
     for (int x = row_base + tid; x < row_end; x += kThreads) {
         int i, j;
         if constexpr (PACKED) {
-            packed_ij<DK>(x, i, j);
+            const int ij = sij[x - row_base];
+            i = ij & 255;
+            j = ij >> 8;
         } else {
             i = x / DK;
             j = x % DK;

@@ -74,6 +74,21 @@ struct ProfScope {
     ~ProfScope() { prof_end(ev, st); }
 };
 
+// Opt-in dynamic shared memory of a kernel, set once per device: the
+// attribute lasts for the life of the context, and setting it on every launch
+// costs host time that small launches cannot hide.
+template <auto Kernel>
+cudaError_t smem_opt_in_once(int bytes) {
+    static int set_bytes[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && set_bytes[dev] == bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) set_bytes[dev] = bytes;
+    return e;
+}
+
 // Element loads as fp32.
 __device__ __forceinline__ float load_f32(const float *p, long long i) { return p[i]; }
 __device__ __forceinline__ float load_f32(const __nv_bfloat16 *p, long long i) {

@@ -382,9 +382,7 @@ cudaError_t run(const Plan &p, const TIn *q, const TIn *k, const TIn *v, TIn *ou
     }
     if (readout) {
         using SM = ReadSmem<DK, DV>;
-        cudaError_t e = cudaFuncSetAttribute(seg_read<DK, DV, TIn>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SM::kBytes);
+        cudaError_t e = smem_opt_in_once<seg_read<DK, DV, TIn>>((int)SM::kBytes);
         if (e != cudaSuccess) return e;
         const long long grid = (long long)((p.T + kTok - 1) / kTok) * BH;
         ProfScope ps("simt_seg_read", st);

@@ -38,21 +38,24 @@ constexpr long long kBf16PerSeg = (long long)kBf16Rows * kD;  // 147,456 bf16
 // sum, so every prefix and the total include it and segment 0 gets a prefix
 // too; prefix == nullptr computes the total only.
 // Reduce-then-scan per block of 128 consecutive elements of one head
-// (32 lanes x float4): warp w takes a run of kScanRun consecutive segments,
+// (32 lanes x float4): warp w takes a run of RUN consecutive segments,
 // holds them in registers and forms their running sums; the 8 run totals are
 // scanned across warps in shared memory in log2(8) = 3 steps; each warp adds
 // its offset and writes its run.  Every global access is a coalesced 16-byte
-// (fp32) or 8-byte (bf16) vector per lane.
+// (fp32) or 8-byte (bf16) vector per lane.  RUN is the smallest of 2, 4, 8,
+// 16 whose pass covers every segment (at most 16): with few segments a short
+// run keeps the registers, and so the blocks resident per SM, that the
+// latency of these short blocks needs.
 // grid.x = element-block + n_eb * bh; block 256.
 // ---------------------------------------------------------------------------
 constexpr int kScanWarps = 8;
-constexpr int kScanRun = 16;
 
 __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
     return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
 
-__global__ void __launch_bounds__(256)
+template <int RUN>
+__global__ void __launch_bounds__(256, RUN == 2 ? 5 : RUN == 4 ? 4 : 2)  // blocks per SM without spills
 tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ prefix,
             float *__restrict__ total, int n_seg, int n_valid, const float *__restrict__ init_s,
             const float *__restrict__ init_z, int n_in, long long s_stride, long long z_stride) {
@@ -65,7 +68,7 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
     const long long bh = blockIdx.x / n_eb;
     const long long e0 = eb * 128 + 4 * lane;
     const float *base = seg_state + bh * (long long)n_seg * E + e0;
-    __nv_bfloat16 *pbase = prefix + bh * (long long)n_seg * kBf16PerSeg;
+    __nv_bfloat16 *pbase = prefix ? prefix + bh * (long long)n_seg * kBf16PerSeg : nullptr;
     // packed z: the thread's 4 rows and their pairs (i, j); padding rows have i > j
     const bool z_part = e0 >= kZPacked0;
     const int zr = z_part ? (int)(e0 - kZPacked0) : 0;
@@ -95,16 +98,16 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
     }
     const int g_first = n_in > 0 ? 0 : 1;  // without one, segment 0 has an empty prefix
 
-    for (int g0 = 0; g0 < n_seg; g0 += kScanWarps * kScanRun) {
-        const int gw = g0 + w * kScanRun;
-        float4 v[kScanRun];
+    for (int g0 = 0; g0 < n_seg; g0 += kScanWarps * RUN) {
+        const int gw = g0 + w * RUN;
+        float4 v[RUN];
 #pragma unroll
-        for (int i = 0; i < kScanRun; ++i)
+        for (int i = 0; i < RUN; ++i)
             v[i] = gw + i < n_valid ? *reinterpret_cast<const float4 *>(base + (long long)(gw + i) * E)
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
         float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < kScanRun; ++i) {  // exclusive running sum within the run
+        for (int i = 0; i < RUN; ++i) {  // exclusive running sum within the run
             const float4 x = v[i];
             v[i] = run;
             run = f4add(run, x);
@@ -128,7 +131,7 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
         carry = f4add(carry, all);
         __syncthreads();  // part is rewritten by the next pass
 #pragma unroll
-        for (int i = 0; i < kScanRun; ++i) {
+        for (int i = 0; i < RUN; ++i) {
             const int g = gw + i;
             if (prefix == nullptr || g < g_first || g >= n_seg) continue;
             const float4 p = f4add(v[i], off);
@@ -1283,8 +1286,7 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
         if (!make_tmap_bf16(&mkt, kt, 3, dkt, skt, bkt) || !make_tmap_bf16(&mvb, v, 3, dqkv, sqkv, b64) ||
             !make_tmap(&mst, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, seg, 3, dst, sst, bst))
             return cudaErrorInvalidValue;
-        cudaError_t e = cudaFuncSetAttribute(tc_build, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kBSmAlloc);
+        cudaError_t e = smem_opt_in_once<tc_build>(kBSmAlloc);
         if (e != cudaSuccess) return e;
         const long long n_items = (long long)kBuildItems * n_build * BH;
         const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
@@ -1295,16 +1297,18 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
     if (scan) {
         ProfScope ps("tc_seg_scan", st);
         const long long grid = (kF32PerSeg / 128) * BH;
-        tc_seg_scan<<<(unsigned)grid, 256, 0, st>>>(seg, readout ? prefix : nullptr,
-                                                     want_state ? total : nullptr, p.n_seg, n_build,
-                                                     init.s, init.z, init.n, init.s_stride,
-                                                     init.z_stride);
+        auto kern = p.n_seg <= 2 * kScanWarps ? tc_seg_scan<2>
+                    : p.n_seg <= 4 * kScanWarps ? tc_seg_scan<4>
+                    : p.n_seg <= 8 * kScanWarps ? tc_seg_scan<8>
+                                                : tc_seg_scan<16>;
+        kern<<<(unsigned)grid, 256, 0, st>>>(seg, readout ? prefix : nullptr,
+                                             want_state ? total : nullptr, p.n_seg, n_build, init.s,
+                                             init.z, init.n, init.s_stride, init.z_stride);
     }
     if (readout) {
         CUtensorMap mq, mk, mv, ms, mo;
         if (!make_maps(p, q, k, v, prefix, out, &mq, &mk, &mv, &ms, &mo)) return cudaErrorInvalidValue;
-        cudaError_t e = cudaFuncSetAttribute(tc_read, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmAlloc);
+        cudaError_t e = smem_opt_in_once<tc_read>(kSmAlloc);
         if (e != cudaSuccess) return e;
         const int n_ct = (p.T + kCtaQ - 1) / kCtaQ;
         const long long n_items = (long long)n_ct * BH;
