@@ -105,6 +105,20 @@ def test_long_context_sampled(oracle_mod, T):
     _sampled_check(oracle_mod, q, k, v, "bf16", Cs, n_uniform=512 if T == w.T else 256)
 
 
+def test_maximum_length_sampled(oracle_mod):
+    # 2^20 tokens per head: 1024 segments, so the scan makes 8 passes of 128
+    T = 1 << 20
+    q, k, v = inputs.make_qkv(1, 2, T, 64, 64, "bf16", seed=17)
+    out, _, _ = run_forward(q, k, v, "bf16", 64)
+    rows = sample_rows(T, 64, 1024, n_uniform=48, n_bound=16)
+    bh = np.repeat(np.arange(2), len(rows))
+    tt = np.tile(rows, 2)
+    q64, k64, v64 = (inputs.widen(x, "bf16").reshape(2, T, -1) for x in (q, k, v))
+    yref = oracle_mod.forward_rows(q64, k64, v64, bh, tt)
+    err = row_err(from_device(out).reshape(2, T, -1)[bh, tt], yref)
+    assert err <= TOL["bf16"], f"row-normwise error {err:.3e}"
+
+
 # ---------------------------------------------------------------------------
 # Edge cases
 # ---------------------------------------------------------------------------

@@ -100,6 +100,13 @@ def test_long_context_sampled(oracle_mod):
     sampled_check(oracle_mod, q, k, v, "bf16", sample_rows(w.T, 64, w.T, n_uniform=64, n_bound=16))
 
 
+def test_maximum_length_single_head(oracle_mod):
+    # 2^20 keys for the last queries of one head: 4096 work items, one segment
+    T = 1 << 20
+    q, k, v = inputs.make_qkv(1, 1, T, 64, 64, "bf16", seed=23)
+    sampled_check(oracle_mod, q, k, v, "bf16", sample_rows(T, 64, T, n_uniform=48, n_bound=16))
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_zero_denominator_rows(oracle_mod, dtype):
     for d in (32, 64):
