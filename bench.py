@@ -657,7 +657,8 @@ def measure_sequence_split(K, q, k, v, C, stream, flush, chunked_ms, kernel_time
 
         def rank_work():  # on the current stream (the capture stream while capturing)
             K.kata_chunked_state(bk, bv, C=C, state_out=S, z_out=Z, workspace=ws)
-            K.kata_chunked_forward_from_state(bq, bk, bv, s_in, z_in, C=C, out=out, workspace=ws)
+            K.kata_chunked_forward_from_state(bq, bk, bv, s_in, z_in, C=C, out=out, workspace=ws,
+                                              reuse_segment_states=True)
 
         eager = time_launches(rank_work, stream, flush, 5)
         # the same calls replayed from a CUDA graph: at a few hundred microseconds of
@@ -676,8 +677,8 @@ def measure_sequence_split(K, q, k, v, C, stream, flush, chunked_ms, kernel_time
                         "projected_tokens_per_s": B * T / (best / 1e3),
                         "kernels_ms": kernel_times(rank_work, 3)}
         del bq, bk, bv, flat, gathered, out, ws
-    res["note"] = ("one GPU: one rank's compute (state pass + forward from N-1 gathered totals, "
-                   "replayed from a CUDA graph) against the single-GPU forward's kernel time / N; "
+    res["note"] = ("one GPU: one rank's compute (state pass + forward from N-1 gathered totals "
+                   "reusing the state pass's segment states, replayed from a CUDA graph) against the single-GPU forward's kernel time / N; "
                    "the all-gather of the totals (1 MiB + 16 KiB per head) is not included")
     return res
 

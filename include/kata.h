@@ -159,14 +159,25 @@ kata_status kata_chunked_state(const void *k, const void *v, int B, int H, int T
  *              the state after the call's last token.  With n_in = 1 they may
  *              be state_in and z_in themselves (updated in place); otherwise
  *              they must not overlap the inputs.
+ *   flags      0, or KATA_REUSE_SEGMENT_STATES: the workspace holds what
+ *              kata_chunked_state last wrote into it for the same k, v, B, H,
+ *              T, dk, dv, C and dtype, and nothing has written it since (the
+ *              sequence-sharded forward: the state pass before the all-gather,
+ *              this call after it).  The tensor-core path then skips building
+ *              the per-segment states again; the fp32 path rebuilds them.
+ *              The result is the same either way; a workspace that does not
+ *              hold those states gives wrong outputs, never a fault.  Other
+ *              bits: KATA_ERR_INVALID_ARG.
  */
+#define KATA_REUSE_SEGMENT_STATES 1u
+
 kata_status kata_chunked_forward_from_state(const void *q, const void *k, const void *v, void *out,
                                             int B, int H, int T, int dk, int dv, int C,
                                             kata_dtype dtype, const float *state_in,
                                             const float *z_in, int n_in, size_t s_stride,
                                             size_t z_stride, float *state_out, float *z_out,
                                             void *workspace, size_t workspace_bytes,
-                                            kata_stream_t stream);
+                                            unsigned flags, kata_stream_t stream);
 
 /*
  * kata_chunked_forward without a caller-provided workspace, for callers that

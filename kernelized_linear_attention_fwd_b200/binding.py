@@ -75,7 +75,8 @@ def load_library(path: str = LIB_PATH):
     lib.kata_chunked_state.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, fp, fp, vp, sz, vp]
     lib.kata_chunked_forward_from_state.restype = i32
     lib.kata_chunked_forward_from_state.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
-                                                    i32, fp, fp, i32, sz, sz, fp, fp, vp, sz, vp]
+                                                    i32, fp, fp, i32, sz, sz, fp, fp, vp, sz,
+                                                    ctypes.c_uint, vp]
     lib.kata_chunked_forward_noalloc.restype = i32
     lib.kata_chunked_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                  i32, fp, fp, vp]
@@ -231,13 +232,19 @@ def _stacked(t, name, inner, n_name):
     return t.shape[0], t.stride(0)
 
 
+KATA_REUSE_SEGMENT_STATES = 1
+
+
 def kata_chunked_forward_from_state(q, k, v, state_in, z_in, C=64, out=None, state_out=None,
-                                    z_out=None, workspace=None, stream=None):
+                                    z_out=None, workspace=None, stream=None,
+                                    reuse_segment_states=False):
     """out[B,H,T,dv]: the chunked forward of q, k, v continuing from the state
     sum_m state_in[m], sum_m z_in[m].  state_in is [n, B, H, dk*dk, dv] (or one
     [B, H, dk*dk, dv] state), z_in [n, B, H, dk, dk]; each state contiguous,
     any stride between them.  state_out / z_out (optional) receive the state
-    after the last token; they may be state_in / z_in themselves for one input."""
+    after the last token; they may be state_in / z_in themselves for one input.
+    reuse_segment_states: `workspace` holds what kata_chunked_state last wrote
+    into it for the same k, v and sizes (KATA_REUSE_SEGMENT_STATES)."""
     import torch
 
     lib = load_library()
@@ -256,11 +263,14 @@ def kata_chunked_forward_from_state(q, k, v, state_in, z_in, C=64, out=None, sta
     _check(out, "out", (B, H, T, dv), q.dtype)
     _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32)
     _check(z_out, "z_out", (B, H, dk, dk), torch.float32)
+    if reuse_segment_states and workspace is None:
+        raise KataError(KATA_ERR_WORKSPACE, "reusing segment states needs the state call's workspace")
     workspace, nbytes = _workspace(lib, workspace, B, H, T, dk, dv, C, code, q.device)
     st = lib.kata_chunked_forward_from_state(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv, int(C), code,
         _ptr(state_in) if n_s else None, _ptr(z_in) if n_z else None, n_s, s_stride, z_stride,
-        _ptr(state_out), _ptr(z_out), _ptr(workspace), nbytes, _stream_handle(stream))
+        _ptr(state_out), _ptr(z_out), _ptr(workspace), nbytes,
+        KATA_REUSE_SEGMENT_STATES if reuse_segment_states else 0, _stream_handle(stream))
     if st != KATA_OK:
         raise KataError(st, "kata_chunked_forward_from_state")
     return out

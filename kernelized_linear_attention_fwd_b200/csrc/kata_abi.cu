@@ -108,11 +108,15 @@ kata_status check_forward_io(const Plan &p, const void *q, const void *k, const 
     return KATA_OK;
 }
 
+// reuse_seg: the workspace holds the segment states a state-only launch wrote
+// for the same inputs and sizes.  The tensor-core path then skips building
+// them; the fp32 path's state-only scan leaves prefixes, not the states, in
+// place, so it rebuilds them (same result).
 cudaError_t launch_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
                            float *state_out, float *z_out, const InitState &init, void *ws,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool reuse_seg = false) {
     return p.path == Path::kTensorCore
-               ? tc::launch_tc_forward(p, q, k, v, out, state_out, z_out, init, ws, st)
+               ? tc::launch_tc_forward(p, q, k, v, out, state_out, z_out, init, ws, st, reuse_seg)
                : launch_simt_forward(p, q, k, v, out, state_out, z_out, init, ws, st);
 }
 
@@ -261,8 +265,9 @@ kata_status kata_chunked_forward_from_state(const void *q, const void *k, const 
                                             const float *z_in, int n_in, size_t s_stride,
                                             size_t z_stride, float *state_out, float *z_out,
                                             void *workspace, size_t workspace_bytes,
-                                            kata_stream_t stream) {
+                                            unsigned flags, kata_stream_t stream) {
     Plan p;
+    if (flags & ~KATA_REUSE_SEGMENT_STATES) return KATA_ERR_INVALID_ARG;
     const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p);
     if (ps != KATA_OK) return ps;
     const kata_status io = kata::check_forward_io(p, q, k, v, out);
@@ -297,8 +302,8 @@ kata_status kata_chunked_forward_from_state(const void *q, const void *k, const 
     const kata_status ws = kata::check_workspace(p, workspace, workspace_bytes);
     if (ws != KATA_OK) return ws;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const cudaError_t e =
-        kata::launch_forward(p, q, k, v, out, state_out, z_out, init, workspace, st);
+    const cudaError_t e = kata::launch_forward(p, q, k, v, out, state_out, z_out, init, workspace,
+                                               st, (flags & KATA_REUSE_SEGMENT_STATES) != 0);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
 }
 

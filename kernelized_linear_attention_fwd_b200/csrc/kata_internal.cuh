@@ -116,10 +116,12 @@ cudaError_t launch_simt_forward(const Plan &p, const void *q, const void *k, con
                                 void *ws, cudaStream_t st);
 namespace tc {
 // Tensor-core path (bf16, d = dv = 64): workspace layout and launcher.
+// reuse_seg: the workspace already holds every segment's state, written by a
+// state-only launch for the same keys, values and sizes; skip building them.
 void plan_tc_workspace(Plan &p);
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v,
                               void *out, float *state_out, float *z_out, const InitState &init,
-                              void *ws, cudaStream_t st);
+                              void *ws, cudaStream_t st, bool reuse_seg = false);
 // Streaming multiprocessors of the current device (cached).
 int num_sms();
 }  // namespace tc

@@ -1248,7 +1248,7 @@ void plan_tc_workspace(Plan &p) {
 
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
                               float *state_out, float *z_out, const InitState &init, void *ws,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool reuse_seg) {
     // no workspace (the quadratic plan): no state is built, scanned or read
     char *w = static_cast<char *>(ws);
     float *seg = w ? reinterpret_cast<float *>(w + p.ws_seg_state) : nullptr;
@@ -1258,14 +1258,16 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
     const bool readout = out != nullptr;
     const bool want_state = state_out != nullptr;
     const bool has_init = init.n > 0;
-    // the last segment's increment is needed only for the total
-    const int n_build = want_state ? p.n_seg : p.n_seg - 1;
+    // the last segment's increment is needed only for the total; with reuse_seg
+    // every segment's increment is in the workspace already
+    const int n_build = reuse_seg ? 0 : want_state ? p.n_seg : p.n_seg - 1;
+    const int n_valid = reuse_seg ? p.n_seg : n_build;
     const bool scan = p.n_seg > 1 || has_init;
     const long long BH = p.BH;
     const int T_pad = (p.T + 63) / 64 * 64;
     int *status = device_status_ptr();
     if (!status) return cudaErrorUnknown;
-    if ((has_init || n_build > 0 || want_state) && !w) return cudaErrorInvalidValue;
+    if ((has_init || n_build > 0 || want_state || reuse_seg) && !w) return cudaErrorInvalidValue;
 
     if (n_build > 0) {
         {
@@ -1302,7 +1304,7 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
                     : p.n_seg <= 8 * kScanWarps ? tc_seg_scan<8>
                                                 : tc_seg_scan<16>;
         kern<<<(unsigned)grid, 256, 0, st>>>(seg, readout ? prefix : nullptr,
-                                             want_state ? total : nullptr, p.n_seg, n_build, init.s,
+                                             want_state ? total : nullptr, p.n_seg, n_valid, init.s,
                                              init.z, init.n, init.s_stride, init.z_stride);
     }
     if (readout) {

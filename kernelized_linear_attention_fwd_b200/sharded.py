@@ -12,7 +12,9 @@ scan).  The same scan one level up shards a sequence over ranks:
    NVLink, 8 MiB + 128 KiB per rank for 8 heads of d = 64);
 3. rank r runs kata_chunked_forward_from_state on its block with the first r
    gathered totals as inputs: the library sums them while it scans its own
-   segments, so the exclusive prefix over ranks costs no extra pass.
+   segments, so the exclusive prefix over ranks costs no extra pass.  The
+   block's per-segment states, built in step 1, stay in the workspace and
+   are reused (KATA_REUSE_SEGMENT_STATES) instead of being built again.
 
 Rank r's optional state output is the state after its block's last token
 (the last rank's is the whole sequence's).  Every step runs in libkata's
@@ -24,17 +26,28 @@ from . import binding
 
 
 class LibkataOps:
-    """The two library calls a block needs (the default; tests of the
-    multi-rank orchestration substitute their own)."""
+    """The library calls a block needs (the default; tests of the multi-rank
+    orchestration substitute their own)."""
 
     @staticmethod
-    def chunked_state(k, v, C, state_out, z_out):
-        binding.kata_chunked_state(k, v, C=C, state_out=state_out, z_out=z_out)
+    def workspace(k, v, C):
+        import torch
+
+        B, H, T, dk = k.shape
+        code = binding.KATA_BF16 if k.dtype == torch.bfloat16 else binding.KATA_F32
+        n = binding.kata_chunked_forward_workspace_bytes(B, H, T, dk, v.shape[-1], C, code)
+        return torch.empty(max(n, 256), dtype=torch.uint8, device=k.device)
 
     @staticmethod
-    def forward_from_state(q, k, v, state_in, z_in, C, out, state_out, z_out):
+    def chunked_state(k, v, C, state_out, z_out, workspace):
+        binding.kata_chunked_state(k, v, C=C, state_out=state_out, z_out=z_out,
+                                   workspace=workspace)
+
+    @staticmethod
+    def forward_from_state(q, k, v, state_in, z_in, C, out, state_out, z_out, workspace, reuse):
         binding.kata_chunked_forward_from_state(q, k, v, state_in, z_in, C=C, out=out,
-                                                state_out=state_out, z_out=z_out)
+                                                state_out=state_out, z_out=z_out,
+                                                workspace=workspace, reuse_segment_states=reuse)
 
 
 def state_numel(B, H, dk, dv):
@@ -42,15 +55,20 @@ def state_numel(B, H, dk, dv):
     return B * H * dk * dk * dv, B * H * dk * dk
 
 
-def block_state(k, v, C=64, ops=LibkataOps):
-    """This block's total state as one flat fp32 buffer [S | Z]."""
+def block_state(k, v, C=64, ops=LibkataOps, workspace=None):
+    """This block's total state as one flat fp32 buffer [S | Z].  `workspace`
+    (from ops.workspace) then holds the block's per-segment states for
+    block_forward(..., reuse=True)."""
     import torch
 
     B, H, _, dk = k.shape
     dv = v.shape[-1]
     ns, nz = state_numel(B, H, dk, dv)
     flat = torch.empty(ns + nz, dtype=torch.float32, device=k.device)
-    ops.chunked_state(k, v, C, flat[:ns].view(B, H, dk * dk, dv), flat[ns:].view(B, H, dk, dk))
+    if workspace is None:
+        workspace = ops.workspace(k, v, C)
+    ops.chunked_state(k, v, C, flat[:ns].view(B, H, dk * dk, dv), flat[ns:].view(B, H, dk, dk),
+                      workspace)
     return flat
 
 
@@ -67,17 +85,20 @@ def gathered_views(gathered, n, B, H, dk, dv):
 
 
 def block_forward(q, k, v, gathered, rank, C=64, out=None, state_out=None, z_out=None,
-                  ops=LibkataOps):
+                  ops=LibkataOps, workspace=None, reuse=False):
     """Outputs of block `rank`, starting from the sum of the totals of blocks
-    0 .. rank-1 (rows of `gathered`)."""
+    0 .. rank-1 (rows of `gathered`).  reuse: `workspace` is the one
+    block_state filled for these k, v, untouched since."""
     import torch
 
     B, H, T, dk = q.shape
     dv = v.shape[-1]
     if out is None:
         out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    if workspace is None:
+        workspace, reuse = ops.workspace(k, v, C), False
     s_in, z_in = gathered_views(gathered, rank, B, H, dk, dv)
-    ops.forward_from_state(q, k, v, s_in, z_in, C, out, state_out, z_out)
+    ops.forward_from_state(q, k, v, s_in, z_in, C, out, state_out, z_out, workspace, reuse)
     return out
 
 
@@ -91,8 +112,9 @@ def sequence_sharded_forward(q, k, v, C=64, group=None, out=None, state_out=None
 
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
-    flat = block_state(k, v, C, ops)
+    ws = ops.workspace(k, v, C)
+    flat = block_state(k, v, C, ops, ws)
     gathered = torch.empty(world * flat.numel(), dtype=flat.dtype, device=flat.device)
     dist.all_gather_into_tensor(gathered, flat, group=group)
     return block_forward(q, k, v, gathered.view(world, flat.numel()), rank, C, out, state_out,
-                         z_out, ops)
+                         z_out, ops, ws, reuse=True)

@@ -162,12 +162,13 @@ def test_forward_from_state_rejects_bad_arguments(lib):
     need = lib.kata_chunked_forward_workspace_bytes(1, 1, 64, 16, 16, 64, 0)
     S0, Z0 = FAKE + 0x60000000, FAKE + 0x68000000
 
-    def ffs(q=FAKE, out=FAKE + 0x30000000, si=S0, zi=Z0, n=1, ss=0, zs=0, so=None, zo=None):
+    def ffs(q=FAKE, out=FAKE + 0x30000000, si=S0, zi=Z0, n=1, ss=0, zs=0, so=None, zo=None,
+            flags=0):
         return lib.kata_chunked_forward_from_state(
             vp(q) if q else None, vp(FAKE + 0x10000000), vp(FAKE + 0x20000000),
             vp(out) if out else None, 1, 1, 64, 16, 16, 64, 0, vp(si) if si else None,
             vp(zi) if zi else None, n, ss, zs, vp(so) if so else None, vp(zo) if zo else None,
-            vp(FAKE + 0x50000000), need, None)
+            vp(FAKE + 0x50000000), need, flags, None)
 
     assert ffs(q=0) == E.KATA_ERR_INVALID_ARG
     assert ffs(n=-1) == E.KATA_ERR_INVALID_ARG
@@ -180,6 +181,8 @@ def test_forward_from_state_rejects_bad_arguments(lib):
     assert ffs(n=2, ss=4096, zs=256, so=S0 + 4 * 4096, zo=Z0 + 0x100000) == E.KATA_ERR_INVALID_ARG
     assert ffs(so=S0 + 256, zo=Z0 + 256) == E.KATA_ERR_INVALID_ARG
     assert ffs(so=S0, zo=0) == E.KATA_ERR_INVALID_ARG            # both or neither
+    assert ffs(flags=2) == E.KATA_ERR_INVALID_ARG                # unknown flag bits
+    assert ffs(q=0, flags=1) == E.KATA_ERR_INVALID_ARG
 
 
 def test_decode_rejects_bad_arguments(lib):

@@ -142,17 +142,20 @@ def test_pieces_in_place(oracle_mod, dtype, d):
     check_state(oracle_mod, S, Z, k64, v64, dtype)
 
 
-def emulated_sharded(q, k, v, bounds, dtype, C=64):
-    """The sequence-sharded forward with its ranks run one after another."""
+def emulated_sharded(q, k, v, bounds, dtype, C=64, reuse=True):
+    """The sequence-sharded forward with its ranks run one after another, each
+    keeping its own workspace from the state pass to the forward."""
     blocks = [[dev(x[:, :, a:b], dtype) for x in (q, k, v)] for a, b in zip(bounds, bounds[1:])]
-    flats = [sharded.block_state(bk, bv, C) for _, bk, bv in blocks]
+    wss = [sharded.LibkataOps.workspace(bk, bv, C) for _, bk, bv in blocks]
+    flats = [sharded.block_state(bk, bv, C, workspace=ws) for (_, bk, bv), ws in zip(blocks, wss)]
     gathered = torch.stack(flats)  # the all-gather's [world, |S| + |Z|] layout
     B, H, _, d = q.shape
     outs, states = [], []
     for r, (bq, bk, bv) in enumerate(blocks):
         so = torch.empty((B, H, d * d, d), dtype=torch.float32, device="cuda")
         zo = torch.empty((B, H, d, d), dtype=torch.float32, device="cuda")
-        outs.append(sharded.block_forward(bq, bk, bv, gathered, r, C, state_out=so, z_out=zo))
+        outs.append(sharded.block_forward(bq, bk, bv, gathered, r, C, state_out=so, z_out=zo,
+                                          workspace=wss[r], reuse=reuse))
         states.append((so, zo))
     torch.cuda.synchronize()
     return np.concatenate([from_device(o) for o in outs], axis=2), states
@@ -171,6 +174,20 @@ def test_sequence_sharded_ranks_emulated(oracle_mod, dtype, d, bounds):
     for r, (so, zo) in enumerate(states):  # each rank's state: after its block
         n = bounds[r + 1]
         check_state(oracle_mod, so, zo, k64[:, :, :n], v64[:, :, :n], dtype)
+
+
+@pytest.mark.parametrize("dtype,d", [("f32", 32), ("bf16", 64)])
+def test_reused_segment_states_match_rebuilt(oracle_mod, dtype, d):
+    # the forward after the state pass, with and without the reuse flag
+    bounds = (0, 1500, 3600)
+    q, k, v = inputs.make_qkv(1, 2, bounds[-1], d, d, dtype, seed=77 + d)
+    y1, s1 = emulated_sharded(q, k, v, bounds, dtype, reuse=True)
+    y0, s0 = emulated_sharded(q, k, v, bounds, dtype, reuse=False)
+    q64, k64, v64 = (inputs.widen(x, dtype) for x in (q, k, v))
+    yref = oracle_mod.forward(q64, k64, v64)
+    assert row_err(y1, yref) <= TOL[dtype] and row_err(y0, yref) <= TOL[dtype]
+    assert row_err(y1, y0) <= (1e-6 if dtype == "f32" else 2.0 ** -7)
+    check_state(oracle_mod, *s1[-1], k64, v64, dtype)
 
 
 def test_sequence_sharded_long_context(oracle_mod):

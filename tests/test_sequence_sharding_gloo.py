@@ -34,10 +34,17 @@ def _free_port():
 
 class OracleOps:
     """fp64 oracle stand-ins for kata_chunked_state and
-    kata_chunked_forward_from_state, on CPU tensors."""
+    kata_chunked_forward_from_state, on CPU tensors.  The workspace records the
+    keys the state call saw, so a forward told to reuse it checks that it got
+    the workspace of its own block's state call."""
 
     @staticmethod
-    def chunked_state(k, v, C, state_out, z_out):
+    def workspace(k, v, C):
+        return {"keys": None}
+
+    @staticmethod
+    def chunked_state(k, v, C, state_out, z_out, workspace):
+        workspace["keys"] = k
         from oracle import oracle
 
         S, Z = oracle.state(k.double().numpy(), v.double().numpy())
@@ -45,8 +52,10 @@ class OracleOps:
         z_out.copy_(torch.from_numpy(Z))
 
     @staticmethod
-    def forward_from_state(q, k, v, state_in, z_in, C, out, state_out, z_out):
+    def forward_from_state(q, k, v, state_in, z_in, C, out, state_out, z_out, workspace, reuse):
         from oracle import oracle
+
+        assert not reuse or workspace["keys"] is k  # reused only for the same block
 
         B, H, T, dk = q.shape
         dv = v.shape[-1]
