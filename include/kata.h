@@ -180,6 +180,36 @@ kata_status kata_chunked_forward_from_state(const void *q, const void *k, const 
                                             unsigned flags, kata_stream_t stream);
 
 /*
+ * kata_chunked_forward on q, k, v and out in HOST memory (pin it, e.g. with
+ * cudaHostAlloc, for the copies to overlap; pageable memory works but
+ * serialises them).  A deployment convenience, not a step of the method:
+ * the heads are independent, so they run in groups of heads_per_group
+ * (<= 0: the library picks about 8 groups), and while one group computes on
+ * `stream` the next group's inputs are copied to the device and the previous
+ * group's outputs back to the host, on two streams of the call's own.
+ *
+ *   q, k, v, out   host, [B, H, T, dk|dv] as kata_chunked_forward
+ *   state_out, z_out  nullable DEVICE pointers, as kata_chunked_forward
+ *   device_buffer  device scratch of at least
+ *                  kata_chunked_forward_host_buffer_bytes(...) bytes,
+ *                  256-byte aligned: two groups' staged q, k, v and out, and
+ *                  one group's forward workspace
+ *
+ * Work is ordered after what is already queued on `stream`, and `stream`
+ * completes only after every copy of the call (out holds the result once
+ * `stream` has been synchronised).  The call creates two streams and a few
+ * events and releases them when their work is done.  Same results as
+ * kata_chunked_forward on device copies of the inputs.
+ */
+size_t kata_chunked_forward_host_buffer_bytes(int B, int H, int T, int dk, int dv, int C,
+                                              kata_dtype dtype, int heads_per_group);
+kata_status kata_chunked_forward_host(const void *q, const void *k, const void *v, void *out,
+                                      int B, int H, int T, int dk, int dv, int C,
+                                      kata_dtype dtype, float *state_out, float *z_out,
+                                      void *device_buffer, size_t device_buffer_bytes,
+                                      int heads_per_group, kata_stream_t stream);
+
+/*
  * kata_chunked_forward without a caller-provided workspace, for callers that
  * cannot allocate device memory themselves: code running inside a host
  * framework that owns all device memory through its own pool, or a

@@ -8,6 +8,8 @@ from .binding import (  # noqa: F401
     KataError,
     kata_chunked_forward,
     kata_chunked_forward_from_state,
+    kata_chunked_forward_host,
+    kata_chunked_forward_host_buffer_bytes,
     kata_chunked_forward_noalloc,
     kata_chunked_forward_workspace_bytes,
     kata_chunked_state,

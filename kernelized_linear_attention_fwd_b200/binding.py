@@ -33,6 +33,8 @@ EXPORTS = (
     "kata_chunked_state",
     "kata_chunked_forward_from_state",
     "kata_chunked_forward_noalloc",
+    "kata_chunked_forward_host_buffer_bytes",
+    "kata_chunked_forward_host",
     "kata_quadratic_forward",
     "kata_decode_step",
     "kata_decode_step_packed",
@@ -77,6 +79,11 @@ def load_library(path: str = LIB_PATH):
     lib.kata_chunked_forward_from_state.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                     i32, fp, fp, i32, sz, sz, fp, fp, vp, sz,
                                                     ctypes.c_uint, vp]
+    lib.kata_chunked_forward_host_buffer_bytes.restype = sz
+    lib.kata_chunked_forward_host_buffer_bytes.argtypes = [i32] * 8
+    lib.kata_chunked_forward_host.restype = i32
+    lib.kata_chunked_forward_host.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                              fp, fp, vp, sz, i32, vp]
     lib.kata_chunked_forward_noalloc.restype = i32
     lib.kata_chunked_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                  i32, fp, fp, vp]
@@ -273,6 +280,55 @@ def kata_chunked_forward_from_state(q, k, v, state_in, z_in, C=64, out=None, sta
         KATA_REUSE_SEGMENT_STATES if reuse_segment_states else 0, _stream_handle(stream))
     if st != KATA_OK:
         raise KataError(st, "kata_chunked_forward_from_state")
+    return out
+
+
+def _check_host(t, name, shape, dtype=None):
+    if t.is_cuda:
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} must be contiguous")
+    if tuple(t.shape) != tuple(shape):
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} has shape {tuple(t.shape)}, want {shape}")
+    if dtype is not None and t.dtype != dtype:
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} has dtype {t.dtype}, want {dtype}")
+
+
+def kata_chunked_forward_host_buffer_bytes(B, H, T, dk, dv, C, dtype_code, heads_per_group=0):
+    return int(load_library().kata_chunked_forward_host_buffer_bytes(
+        B, H, T, dk, dv, C, dtype_code, heads_per_group))
+
+
+def kata_chunked_forward_host(q, k, v, out, C=64, state_out=None, z_out=None,
+                              device_buffer=None, heads_per_group=0, stream=None):
+    """The chunked forward on host tensors q, k [B,H,T,dk], v, out [B,H,T,dv]
+    (pinned for the copies to overlap with the compute), heads in groups.
+    state_out / z_out are CUDA tensors; device_buffer a uint8 CUDA tensor of at
+    least kata_chunked_forward_host_buffer_bytes(...) bytes (allocated here if
+    None).  `out` holds the result once `stream` is synchronised."""
+    import torch
+
+    lib = load_library()
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    _check_host(q, "q", (B, H, T, dk))
+    _check_host(k, "k", (B, H, T, dk), q.dtype)
+    _check_host(v, "v", (B, H, T, dv), q.dtype)
+    _check_host(out, "out", (B, H, T, dv), q.dtype)
+    code = _dtype_code(q)
+    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32)
+    _check(z_out, "z_out", (B, H, dk, dk), torch.float32)
+    need = kata_chunked_forward_host_buffer_bytes(B, H, T, dk, dv, int(C), code,
+                                                  int(heads_per_group))
+    if device_buffer is None:
+        device_buffer = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+    nbytes = device_buffer.numel() * device_buffer.element_size()
+    st = lib.kata_chunked_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv,
+                                       int(C), code, _ptr(state_out), _ptr(z_out),
+                                       _ptr(device_buffer), nbytes, int(heads_per_group),
+                                       _stream_handle(stream))
+    if st != KATA_OK:
+        raise KataError(st, "kata_chunked_forward_host")
     return out
 
 

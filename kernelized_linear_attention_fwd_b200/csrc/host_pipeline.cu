@@ -1,0 +1,156 @@
+// kata_chunked_forward_host: the chunked forward on q, k, v and out held in
+// pinned host memory.  The heads are independent, so they are processed in
+// groups, and three streams overlap the transfers with the compute: while
+// group g runs on the caller's stream, group g+1's inputs cross PCIe to the
+// device on a copy stream and group g-1's outputs cross back on another.
+// Each group runs through kata_chunked_forward itself (same kernels, same
+// checks).  Two device slots, each holding one group's q, k, v and out,
+// alternate between groups; events order the reuse of a slot after the copy
+// that last read it.  Streams and events are created per call and released
+// when their work completes.
+#include <stdint.h>
+
+#include "kata_internal.cuh"
+
+namespace kata {
+namespace {
+
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct HostPlan {
+    long long BH;
+    int G;                 // heads per group
+    int n_groups;
+    size_t q_head, v_head;  // bytes of one head's q (= k) and v (= out) rows
+    size_t slot_bytes;     // q, k, v, out of G heads
+    size_t ws_offset, ws_bytes;
+    size_t total;
+};
+
+constexpr int kSlots = 2;
+
+kata_status host_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype,
+                      int heads_per_group, HostPlan &hp) {
+    Plan p;
+    const kata_status ps = make_plan(B, H, T, dk, dv, C, dtype, p);
+    if (ps != KATA_OK) return ps;
+    hp.BH = p.BH;
+    long long G = heads_per_group > 0 ? heads_per_group : (p.BH + 7) / 8;  // about 8 groups
+    if (G > p.BH) G = p.BH;
+    if (G > 0x7fffffffLL) return KATA_ERR_UNSUPPORTED;
+    hp.G = (int)G;
+    hp.n_groups = (int)((p.BH + G - 1) / G);
+    const size_t es = dtype == KATA_BF16 ? 2 : 4;
+    hp.q_head = (size_t)T * dk * es;
+    hp.v_head = (size_t)T * dv * es;
+    hp.slot_bytes = 2 * up256(G * hp.q_head) + 2 * up256(G * hp.v_head);
+    Plan pg;
+    if (make_plan(1, hp.G, T, dk, dv, C, dtype, pg) != KATA_OK) return KATA_ERR_UNSUPPORTED;
+    hp.ws_offset = kSlots * hp.slot_bytes;
+    hp.ws_bytes = pg.ws_bytes;
+    hp.total = hp.ws_offset + up256(hp.ws_bytes);
+    return KATA_OK;
+}
+
+}  // namespace
+}  // namespace kata
+
+extern "C" {
+
+size_t kata_chunked_forward_host_buffer_bytes(int B, int H, int T, int dk, int dv, int C,
+                                              kata_dtype dtype, int heads_per_group) {
+    kata::HostPlan hp;
+    if (kata::host_plan(B, H, T, dk, dv, C, dtype, heads_per_group, hp) != KATA_OK) return 0;
+    return hp.total;
+}
+
+kata_status kata_chunked_forward_host(const void *q, const void *k, const void *v, void *out,
+                                      int B, int H, int T, int dk, int dv, int C,
+                                      kata_dtype dtype, float *state_out, float *z_out,
+                                      void *device_buffer, size_t device_buffer_bytes,
+                                      int heads_per_group, kata_stream_t stream) {
+    kata::HostPlan hp;
+    const kata_status ps = kata::host_plan(B, H, T, dk, dv, C, dtype, heads_per_group, hp);
+    if (ps != KATA_OK) return ps;
+    if (!q || !k || !v || !out) return KATA_ERR_INVALID_ARG;
+    if ((state_out == nullptr) != (z_out == nullptr)) return KATA_ERR_INVALID_ARG;
+    if (!device_buffer || device_buffer_bytes < hp.total ||
+        (reinterpret_cast<uintptr_t>(device_buffer) & 255u) != 0)
+        return KATA_ERR_WORKSPACE;
+
+    cudaStream_t user = reinterpret_cast<cudaStream_t>(stream);
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t e_start = nullptr, e_in[kata::kSlots] = {}, e_comp[kata::kSlots] = {},
+                e_out[kata::kSlots] = {};
+    bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&e_start, cudaEventDisableTiming) == cudaSuccess;
+    for (int s = 0; s < kata::kSlots && ok; ++s)
+        ok = cudaEventCreateWithFlags(&e_in[s], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&e_comp[s], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&e_out[s], cudaEventDisableTiming) == cudaSuccess;
+    // the copies start after the work already queued on the caller's stream
+    ok = ok && cudaEventRecord(e_start, user) == cudaSuccess &&
+         cudaStreamWaitEvent(s_in, e_start, 0) == cudaSuccess &&
+         cudaStreamWaitEvent(s_out, e_start, 0) == cudaSuccess;
+
+    kata_status status = ok ? KATA_OK : KATA_ERR_CUDA;
+    const char *qh = static_cast<const char *>(q), *kh = static_cast<const char *>(k),
+               *vh = static_cast<const char *>(v);
+    char *oh = static_cast<char *>(out);
+    char *dev = static_cast<char *>(device_buffer);
+    const size_t es_q = hp.q_head, es_v = hp.v_head;
+    for (int g = 0; g < hp.n_groups && status == KATA_OK; ++g) {
+        const int s = g % kata::kSlots;
+        const long long h0 = (long long)g * hp.G;
+        const int gh = (int)(hp.BH - h0 < hp.G ? hp.BH - h0 : hp.G);
+        char *slot = dev + s * hp.slot_bytes;
+        char *dq = slot, *dk_ = dq + kata::up256(hp.G * es_q), *dv_ = dk_ + kata::up256(hp.G * es_q),
+             *dout = dv_ + kata::up256(hp.G * es_v);
+        // inputs: once the compute of the group that last used this slot is done
+        ok = cudaStreamWaitEvent(s_in, e_comp[s], 0) == cudaSuccess &&
+             cudaMemcpyAsync(dq, qh + h0 * es_q, gh * es_q, cudaMemcpyHostToDevice, s_in) ==
+                 cudaSuccess &&
+             cudaMemcpyAsync(dk_, kh + h0 * es_q, gh * es_q, cudaMemcpyHostToDevice, s_in) ==
+                 cudaSuccess &&
+             cudaMemcpyAsync(dv_, vh + h0 * es_v, gh * es_v, cudaMemcpyHostToDevice, s_in) ==
+                 cudaSuccess &&
+             cudaEventRecord(e_in[s], s_in) == cudaSuccess;
+        // compute: once the inputs are in and the slot's previous output has left
+        ok = ok && cudaStreamWaitEvent(user, e_in[s], 0) == cudaSuccess &&
+             cudaStreamWaitEvent(user, e_out[s], 0) == cudaSuccess;
+        if (!ok) {
+            status = KATA_ERR_CUDA;
+            break;
+        }
+        const long long so = h0 * (long long)dk * dk * dv, zo = h0 * (long long)dk * dk;
+        status = kata_chunked_forward(dq, dk_, dv_, dout, 1, gh, T, dk, dv, C, dtype,
+                                      state_out ? state_out + so : nullptr,
+                                      z_out ? z_out + zo : nullptr, dev + hp.ws_offset,
+                                      hp.ws_bytes, stream);
+        if (status != KATA_OK) break;
+        // output: once computed
+        ok = cudaEventRecord(e_comp[s], user) == cudaSuccess &&
+             cudaStreamWaitEvent(s_out, e_comp[s], 0) == cudaSuccess &&
+             cudaMemcpyAsync(oh + h0 * es_v, dout, gh * es_v, cudaMemcpyDeviceToHost, s_out) ==
+                 cudaSuccess &&
+             cudaEventRecord(e_out[s], s_out) == cudaSuccess;
+        if (!ok) status = KATA_ERR_CUDA;
+    }
+    // the caller's stream completes after every copy this call queued
+    for (int s = 0; s < kata::kSlots; ++s) {
+        if (e_out[s]) cudaStreamWaitEvent(user, e_out[s], 0);
+        if (e_in[s]) cudaStreamWaitEvent(user, e_in[s], 0);
+    }
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+    if (e_start) cudaEventDestroy(e_start);
+    for (int s = 0; s < kata::kSlots; ++s) {
+        if (e_in[s]) cudaEventDestroy(e_in[s]);
+        if (e_comp[s]) cudaEventDestroy(e_comp[s]);
+        if (e_out[s]) cudaEventDestroy(e_out[s]);
+    }
+    return status;
+}
+
+}  // extern "C"

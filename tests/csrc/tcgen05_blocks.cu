@@ -6,6 +6,10 @@
 //   blocks_mma_ts    D = A B with A written to tensor memory by tcgen05.st
 //                    (row m in lane m, K pairs packed per 32-bit column) and
 //                    B MN-major [K x 64] through TMA
+//   blocks_wait_timeout  the bounded-wait failure path: two warps wait on
+//                    mbarriers that nothing completes; the first wait gives up
+//                    after the library's cycle budget and raises the CTA's
+//                    abort flag, the other sees the flag and leaves too
 // Every wait is bounded; a time-out sets *status and the kernel returns.
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -184,6 +188,31 @@ __global__ void k_mma_ts(const __nv_bfloat16 *A, int KK, const __grid_constant__
     if (warp == 0) tmem_dealloc(tD, 256);
 }
 
+// Lane 0 of warps 0 and 1 each wait on a barrier whose phase never completes
+// (nothing arrives).  out[w] = 1 if warp w's wait returned true, out[2 + w] =
+// the cycles it waited; *status = 5 (the library's time-out code) when the
+// abort flag was raised.
+__global__ void k_wait_timeout(long long *out, int *status) {
+    __shared__ uint64_t bar[2];
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    const int warp = threadIdx.x / 32;
+    if (threadIdx.x % 32 == 0 && warp < 2) {
+        const long long t0 = clock64();
+        const bool ok = mbar_wait(&bar[warp], 0, &abort_flag);
+        out[2 + warp] = clock64() - t0;
+        out[warp] = ok ? 1 : 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && abort_flag) atomicExch(status, 5);
+}
+
 bool tmap2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_in,
             uint32_t box_out) {
     const uint64_t dims[2] = {inner, outer};
@@ -240,6 +269,12 @@ int blocks_mma_ts(const void *A, const void *B, float *D, int KK, int *d_status)
     const int smem = KK * 128 + 1024;
     cudaFuncSetAttribute(k_mma_ts, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     k_mma_ts<<<1, 128, smem>>>(static_cast<const __nv_bfloat16 *>(A), KK, mb, D, d_status);
+    return finish(d_status);
+}
+
+// out: 4 int64 (see k_wait_timeout).  Returns the status the kernel set.
+int blocks_wait_timeout(long long *out, int *d_status) {
+    k_wait_timeout<<<1, 64>>>(out, d_status);
     return finish(d_status);
 }
 

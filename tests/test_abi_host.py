@@ -185,6 +185,33 @@ def test_forward_from_state_rejects_bad_arguments(lib):
     assert ffs(q=0, flags=1) == E.KATA_ERR_INVALID_ARG
 
 
+def test_host_forward_rejects_bad_arguments(lib):
+    vp = ctypes.c_void_p
+    E = binding
+    need = lib.kata_chunked_forward_host_buffer_bytes(1, 8, 4096, 64, 64, 64, 1, 1)
+    assert need > 0
+    assert lib.kata_chunked_forward_host_buffer_bytes(1, 8, 4096, 48, 48, 64, 1, 1) == 0
+    # fewer heads per group, less staging
+    assert need < lib.kata_chunked_forward_host_buffer_bytes(1, 8, 4096, 64, 64, 64, 1, 4)
+    host = ctypes.create_string_buffer(64)  # host pointers are never read: every call fails first
+
+    def fh(q=True, out=True, so=None, zo=None, buf=FAKE, nbytes=None, H=8, dk=64):
+        a = vp(ctypes.addressof(host))
+        return lib.kata_chunked_forward_host(a if q else None, a, a, a if out else None, 1, H,
+                                             4096, dk, dk, 64, 1, vp(so) if so else None,
+                                             vp(zo) if zo else None, vp(buf) if buf else None,
+                                             need if nbytes is None else nbytes, 1, None)
+
+    assert fh(q=False) == E.KATA_ERR_INVALID_ARG
+    assert fh(out=False) == E.KATA_ERR_INVALID_ARG
+    assert fh(so=FAKE + 0x1000) == E.KATA_ERR_INVALID_ARG      # state_out without z_out
+    assert fh(dk=48) == E.KATA_ERR_UNSUPPORTED
+    assert fh(H=0) == E.KATA_ERR_INVALID_ARG
+    assert fh(buf=None) == E.KATA_ERR_WORKSPACE
+    assert fh(nbytes=need - 1) == E.KATA_ERR_WORKSPACE
+    assert fh(buf=FAKE + 16) == E.KATA_ERR_WORKSPACE             # not 256-byte aligned
+
+
 def test_decode_rejects_bad_arguments(lib):
     vp = ctypes.c_void_p
     E = binding

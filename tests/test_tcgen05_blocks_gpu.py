@@ -1,7 +1,10 @@
 """The sm_100a building blocks the tensor-core kernels rely on, checked on the
 GPU against CPU arithmetic: the 128-byte TMA swizzle, shared-memory
 descriptors (K-major and MN-major), the instruction descriptor, the layout of
-an A operand written to tensor memory, and the accumulator read-back."""
+an A operand written to tensor memory, and the accumulator read-back.  Also
+the bounded-wait failure path: a wait that can never complete gives up after
+the library's cycle budget, the kernel reports the time-out and returns, and
+the context stays usable."""
 import ctypes
 
 import numpy as np
@@ -23,6 +26,7 @@ def blocks():
     lib.blocks_tma_raw.argtypes = [vp, vp, i32, vp]
     lib.blocks_mma_ss.argtypes = [vp, vp, vp, i32, i32, vp]
     lib.blocks_mma_ts.argtypes = [vp, vp, vp, i32, vp]
+    lib.blocks_wait_timeout.argtypes = [vp, vp]
     return lib
 
 
@@ -80,3 +84,15 @@ def test_mma_a_from_tensor_memory(blocks, status, KK):
     assert blocks.blocks_mma_ts(_p(A), _p(B), _p(D), KK, _p(status)) == 0
     ref = A.float() @ B.float()
     torch.testing.assert_close(D, ref, rtol=1e-5, atol=1e-4)
+
+
+def test_bounded_wait_gives_up_and_the_context_stays_usable(blocks, status):
+    out = torch.full((4,), -1, dtype=torch.int64, device="cuda")
+    assert blocks.blocks_wait_timeout(_p(out), _p(status)) == 5  # the library's time-out code
+    ok0, ok1, c0, c1 = out.cpu().tolist()
+    assert ok0 == 0 and ok1 == 0            # neither wait claims its phase completed
+    assert max(c0, c1) >= 1 << 31           # the first to give up waited the whole budget
+    assert min(c0, c1) <= (1 << 31) + (1 << 28)  # the other left soon after the abort flag
+    # the context still runs work
+    x = torch.arange(1000, device="cuda", dtype=torch.float32)
+    assert float(x.sum().item()) == 499500.0
