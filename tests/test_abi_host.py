@@ -263,6 +263,26 @@ def test_packed_layout_calls_reject_bad_arguments(lib):
         assert conv(fn, d=Sp + 16) == E.KATA_ERR_INVALID_ARG         # destinations overlap
 
 
+def test_binding_rejects_host_tensors_and_bad_shapes(lib):
+    # checked in the binding before anything reaches the library
+    import torch
+
+    x = torch.zeros((1, 2, 8, 16), dtype=torch.bfloat16)
+    for call in (lambda: binding.kata_chunked_forward(x, x, x),
+                 lambda: binding.kata_quadratic_forward(x, x, x),
+                 lambda: binding.kata_chunked_state(x, x),
+                 lambda: binding.kata_decode_step(x[:, :, 0], x[:, :, 0], x[:, :, 0],
+                                                  torch.zeros((1, 2, 256, 16)),
+                                                  torch.zeros((1, 2, 16, 16)))):
+        with pytest.raises(binding.KataError) as e:
+            call()
+        assert e.value.status == binding.KATA_ERR_INVALID_ARG
+    # the host-buffer forward wants host tensors of matching shapes
+    with pytest.raises(binding.KataError):
+        binding.kata_chunked_forward_host(x, x, x, torch.zeros((1, 2, 8, 8), dtype=x.dtype))
+    assert binding.packed_rows(64) == 2080 and binding.packed_rows(16) == 136
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     saved = binding._lib
     try:
