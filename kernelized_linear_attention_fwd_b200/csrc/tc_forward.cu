@@ -243,7 +243,10 @@ constexpr uint32_t kTmS = 128;   // intra scores S[t][x]: 64 columns at 128 + 12
 constexpr uint32_t kTmP = 384;   // intra weights P[t][x] (bf16 pairs): 32 columns at 384 + 64 t + 32 x
 
 struct ReadBars {
-    uint64_t qfull[2], qempty[2], u, interdone, done, genin, ostaged;
+    // ostaged[b]: the output rows of the item in slot b are staged.  One per
+    // slot: a slot is refilled only after the store warp has released it, so
+    // neither barrier can complete twice ahead of the store warp's wait.
+    uint64_t qfull[2], qempty[2], u, interdone, done, genin, ostaged[2];
     uint64_t bfull[kRBRing], bempty[kRBRing], afull[kRRing], aempty[kRRing];
     uint64_t kvfull[2], kvempty[2];
     uint64_t sfull[kTiles][2], pfull[kTiles][2], pempty[kTiles][2];
@@ -812,7 +815,8 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         mbar_init(&bars.interdone, 2);
         mbar_init(&bars.done, 2);
         mbar_init(&bars.genin, 8);
-        mbar_init(&bars.ostaged, 8);
+        mbar_init(&bars.ostaged[0], 8);
+        mbar_init(&bars.ostaged[1], 8);
         for (int s = 0; s < kRBRing; ++s) {
             mbar_init(&bars.bfull[s], 1);
             mbar_init(&bars.bempty[s], 1);
@@ -1035,7 +1039,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             for (int x = sched.first; x < sched.end; x += sched.stride, ++j) {
                 const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg, has_init);
                 const int qb = j & 1;
-                if (!mbar_wait(&bars.ostaged, j & 1, abort)) break;
+                if (!mbar_wait(&bars.ostaged[qb], (j >> 1) & 1, abort)) break;
                 for (int t = 0; t < kTiles; ++t)
                     if (it.t0 + kQT * t < T)
                         tma_store_3d(&tm_o, sm + kSmItem + qb * kItemBytes + t * 16384, 0, it.t0 + kQT * t, it.bh);
@@ -1187,7 +1191,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.ostaged);
+                if (lane == 0) mbar_arrive(&bars.ostaged[qb]);
             }
         }
         tmem_st_wait();

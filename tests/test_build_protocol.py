@@ -1,0 +1,172 @@
+"""Barrier protocol of the persistent state builder (`tc_build`), on the CPU.
+
+A step-by-step model of every role of the kernel, with its ring sizes,
+barrier counts and phase arithmetic:
+- the TMA producer, which loads key/value tiles into a ring of 5;
+- the two MMA issuers, which take alternate 32-token stages of every tile
+  and commit the A slot, the tile and, per work item, `done`;
+- the 8 generation warps, which write the products of each stage into a ring
+  of 3 A slots in tensor memory and, after each item, drain the accumulators
+  to the staging buffer once the previous item's store has released it;
+- the store warp, which stores each staged item and releases the buffer.
+
+It runs over sequences of work items with ragged token-tile counts (a short
+last segment, single-tile items).  TMA loads and MMA commits complete at
+random later times (one issuer's commits in order) and the roles interleave
+at random, each at its own random speed.  Checked: no deadlock, and every wait observes exactly the phase
+it intends.  Planted mistakes (the drain not waiting for the staging buffer,
+an issuer waiting for the wrong A-slot phase) must be caught.
+"""
+import random
+
+import pytest
+
+from tests.test_readout_protocol import Bar, ProtocolError
+
+KERNEL = dict(kBTileRing=5, kBARing=3, kGenWarps=8)
+
+
+def simulate(items_ntt, seed, prm, planted=None):
+    R, A, n_gen = prm["kBTileRing"], prm["kBARing"], prm["kGenWarps"]
+    rng = random.Random(seed)
+    B = {}
+    for x in range(R):
+        B[f"tfull{x}"], B[f"tempty{x}"] = Bar(1), Bar(2)
+    for x in range(A):
+        B[f"afull{x}"], B[f"aempty{x}"] = Bar(32 * n_gen), Bar(1)
+    B.update(done=Bar(2), staged=Bar(32 * n_gen), sfree=Bar(1), drain0=Bar(1), drain1=Bar(1))
+    n_items = len(items_ntt)
+
+    def W(name, k):  # wait for phase k of `name` (k = -1: the fresh barrier's previous phase)
+        return ("wait", name, k)
+
+    def producer():
+        tt = 0
+        for n_tt in items_ntt:
+            for _ in range(n_tt):
+                yield W(f"tempty{tt % R}", tt // R - 1)
+                yield ("load", f"tfull{tt % R}", 2)  # keys^T and values
+                tt += 1
+
+    def issuer(me):
+        tt = 0
+        for n_tt in items_ntt:
+            for _ in range(n_tt):
+                G = 2 * tt + me
+                a = G % A
+                yield W(f"tfull{tt % R}", tt // R)
+                # planted: the wait one phase early (it would pass on the slot's previous fill)
+                yield W(f"afull{a}", G // A - 1 if planted == "issuer_phase" else G // A)
+                yield ("commit", f"aempty{a}")
+                yield ("commit", f"tempty{tt % R}")
+                tt += 1
+            yield ("commit", "done")
+        yield ("commit", f"drain{me}")
+        yield W(f"drain{me}", 0)
+
+    def gen(w):
+        tt = 0
+        for j, n_tt in enumerate(items_ntt):
+            yield W(f"tfull{tt % R}", tt // R)
+            for t in range(n_tt):
+                for half in range(2):
+                    G = 2 * tt + half
+                    a = G % A
+                    yield W(f"aempty{a}", G // A - 1)
+                    if half == 1 and t + 1 < n_tt:
+                        yield W(f"tfull{(tt + 1) % R}", (tt + 1) // R)
+                    yield ("arrive", f"afull{a}", 32)
+                tt += 1
+            yield W("done", j)
+            if j > 0 and planted != "drain_no_sfree":
+                yield W("sfree", j - 1)
+            yield ("write_stage", j)  # the drain: accumulators -> staging buffer
+            yield ("arrive", "staged", 32)
+
+    def storer():
+        for j in range(n_items):
+            yield W("staged", j)
+            yield ("read_stage", j)  # the store reads the staging buffer
+            yield ("arrive", "sfree", 1)
+
+    agents = {"prod": producer(), "iss0": issuer(0), "iss1": issuer(1), "store": storer()}
+    agents.update({f"gen{w}": gen(w) for w in range(n_gen)})
+    cur = dict.fromkeys(agents)
+    # each role runs at its own random speed, so that some runs starve one of
+    # them (a slow store warp, a slow issuer) and others race ahead
+    role_speed = {r: rng.choice((0.02, 0.2, 1.0)) for r in ("prod", "iss0", "iss1", "store", "gen")}
+    speed = {a: role_speed["gen" if a.startswith("gen") else a] for a in agents}
+    loads, commits = [], {"iss0": [], "iss1": []}
+    # the staging buffer: which item's rows it holds, and which item the store
+    # has finished reading; a drain may overwrite it only once the store of
+    # the previous item has read it
+    stage = {"item": -1, "read": -1}
+    while True:
+        runnable = [a for a, g in agents.items() if g is not None and
+                    (cur[a] is None or B[cur[a][1]].done(cur[a][2] & 1))]
+        pending = len(loads) + len(commits["iss0"]) + len(commits["iss1"])
+        if not runnable and not pending:
+            if all(g is None for g in agents.values()):
+                return
+            raise ProtocolError(f"deadlock: {[(a, cur[a]) for a in agents if agents[a] is not None]}")
+        # a role is ready this step with the probability of its speed; a slow
+        # role's turn passes to the copies and MMAs in flight or to faster roles
+        ready = [x for x in runnable if rng.random() < speed[x]]
+        if pending and (not ready or rng.random() < 0.4):
+            choice = rng.choice((["load"] if loads else []) + [a for a in commits if commits[a]])
+            if choice == "load":
+                bar = B[loads.pop(rng.randrange(len(loads)))]
+                bar.tx -= 1
+                bar.flip()
+            else:
+                B[commits[choice].pop(0)].arrive()
+            continue
+        a = rng.choice(ready or runnable)
+        if cur[a] is not None and B[cur[a][1]].phase != cur[a][2] + 1:
+            raise ProtocolError(f"{a} woke on the wrong phase of {cur[a][1]}")
+        try:
+            act = next(agents[a])
+        except StopIteration:
+            agents[a], cur[a] = None, None
+            continue
+        cur[a] = None
+        if act[0] == "wait":
+            if B[act[1]].phase not in (act[2], act[2] + 1):
+                raise ProtocolError(f"{a} waits on {act[1]} two phases behind")
+            cur[a] = act
+        elif act[0] == "write_stage":
+            if stage["read"] < act[1] - 1:
+                raise ProtocolError(f"drain of item {act[1]} overwrote item {act[1] - 1} before its store read it")
+            stage["item"] = max(stage["item"], act[1])
+        elif act[0] == "read_stage":
+            if stage["item"] != act[1]:
+                raise ProtocolError(f"store of item {act[1]} read the rows of item {stage['item']}")
+            stage["read"] = act[1]
+        elif act[0] == "arrive":
+            B[act[1]].arrive(act[2])
+        elif act[0] == "load":  # arrive.expect_tx, then the bytes land later
+            B[act[1]].tx += act[2]
+            B[act[1]].arrive()
+            loads.extend([act[1]] * act[2])
+        else:
+            commits[a].append(act[1])
+
+
+# token tiles per work item, as one CTA walks them: full 1024-token segments
+# (16 tiles of 64), a ragged last segment, single-tile segments, and runs
+# longer than the rings
+CASES = [[16, 16, 16], [16, 3, 16, 1], [1, 1, 1, 1, 1, 1], [2, 16, 5, 7, 16, 1, 4], [16], [4, 4]]
+
+
+def test_build_protocol_is_deadlock_free_and_phase_exact():
+    for seed in range(12):
+        for c, items in enumerate(CASES):
+            simulate(items, 100 * seed + c, KERNEL)
+
+
+@pytest.mark.parametrize("mistake", ["drain_no_sfree", "issuer_phase"])
+def test_model_catches_planted_mistakes(mistake):
+    with pytest.raises(ProtocolError):
+        for seed in range(40):
+            for c, items in enumerate(CASES):
+                simulate(items, 100 * seed + c, KERNEL, planted=mistake)

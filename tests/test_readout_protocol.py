@@ -9,11 +9,13 @@ heads, several items per CTA, the quadratic form's longest-first order, and
 first-segment items with an inter phase when the forward starts from a given
 state).  TMA loads and MMA commits complete
 asynchronously at random later times (one issuer's commits in order), and the
-roles interleave at random.  Checked: no deadlock, and every wait observes
+roles interleave at random, each at its own random speed.  Checked: no deadlock, and every wait observes
 exactly the phase it intends (a barrier never runs two phases past a waiter,
-which a parity wait could not tell apart).  A planted mistake -- the score
-buffer reused across work items without waiting for its last reader -- must be
-caught.
+which a parity wait could not tell apart).  Planted mistakes must be caught:
+the score buffer reused across work items without waiting for its last
+reader, and both item slots' outputs staged on one barrier (a real hazard of
+an earlier version of the kernel, found by this model once each role ran at
+its own speed).
 """
 import random
 
@@ -46,7 +48,7 @@ class Bar:
         return (self.phase & 1) != parity
 
 
-def simulate(T, L, BH, items, seed, prm, planted=False, init=False):
+def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=False):
     kQT, kTiles, kSB, kKB = prm['kQT'], prm['kTiles'], prm['kSB'], prm['kKB']
     kKVRing, kRStages, kRRing, kRBRing, kSlots = (prm['kKVRing'], prm['kRStages'], prm['kRRing'],
                                                   prm['kRBRing'], prm['kItemSlots'])
@@ -58,8 +60,13 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False):
         B[f'qfull{b}'], B[f'qempty{b}'] = Bar(1), Bar(3)
     for b in range(kKVRing):
         B[f'kvfull{b}'], B[f'kvempty{b}'] = Bar(1), Bar(2)
-    B.update(u=Bar(1), interdone=Bar(2), done=Bar(2), genin=Bar(kGen), ostaged=Bar(kGen),
-             drain0=Bar(1), drain1=Bar(1))
+    B.update(u=Bar(1), interdone=Bar(2), done=Bar(2), genin=Bar(kGen), drain0=Bar(1),
+             drain1=Bar(1))
+    for b in range(kSlots):  # output rows staged in item slot b
+        B[f'ostaged{b}'] = Bar(kGen)
+    # planted: one barrier for both slots (it may complete twice ahead of the store warp)
+    osb = (lambda j: 'ostaged0') if one_ostaged else (lambda j: f'ostaged{j % kSlots}')
+    osk = (lambda j: j) if one_ostaged else (lambda j: j // kSlots)
     for s in range(kRBRing):
         B[f'bfull{s}'], B[f'bempty{s}'] = Bar(1), Bar(1)
     for s in range(kRRing):
@@ -151,7 +158,7 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False):
 
     def storer():
         for j in range(len(items)):
-            yield W('ostaged', j)
+            yield W(osb(j), osk(j))
             yield ('arrive', f'qempty{j % kSlots}', 1)
 
     def gen(w):
@@ -174,11 +181,15 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False):
                 yield ('arrive', f'pfull{t}{n & 1}', 32)
             g_b += blocks(it, t)
             yield W('done', j)
-            yield ('arrive', 'ostaged', 1)
+            yield ('arrive', osb(j), 1)
 
     agents = {'prod': producer(), 'iss0': issuer(0), 'iss1': issuer(1), 'store': storer()}
     agents.update({f'gen{w}': gen(w) for w in range(kGen)})
     cur = dict.fromkeys(agents)
+    # each role runs at its own random speed (the squaring warps share one), so
+    # some runs starve a role and let the others race ahead of it
+    role_speed = {r: rng.choice((0.02, 0.2, 1.0)) for r in ('prod', 'iss0', 'iss1', 'store', 'gen')}
+    speed = {a: role_speed['gen' if a.startswith('gen') else a] for a in agents}
     loads, commits = [], {'iss0': [], 'iss1': []}
     while True:
         runnable = [a for a, g in agents.items() if g is not None and
@@ -188,7 +199,8 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False):
             if all(g is None for g in agents.values()):
                 return
             raise ProtocolError(f"deadlock: {[(a, cur[a]) for a in agents if agents[a] is not None]}")
-        if pending and (not runnable or rng.random() < 0.4):
+        ready = [x for x in runnable if rng.random() < speed[x]]
+        if pending and (not ready or rng.random() < 0.4):
             choice = rng.choice((['load'] if loads else []) + [a for a in commits if commits[a]])
             if choice == 'load':
                 bar = B[loads.pop(rng.randrange(len(loads)))]
@@ -197,7 +209,7 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False):
             else:
                 B[commits[choice].pop(0)].arrive()
             continue
-        a = rng.choice(runnable)
+        a = rng.choice(ready or runnable)
         if cur[a] is not None and B[cur[a][1]].phase != cur[a][2] + 1:
             raise ProtocolError(f"{a} woke on the wrong phase of {cur[a][1]}")
         try:
@@ -265,6 +277,21 @@ def test_initial_state_gives_every_item_an_inter_phase():
             n_ct = (T + cq - 1) // cq
             for c in range(g):
                 simulate(T, T, BH, quadratic_items(n_ct, BH, g, c), 13 * T + c, KERNEL, init=True)
+
+
+def test_model_catches_one_output_barrier_for_both_slots():
+    # the kernel once staged both slots' outputs on one barrier: with the store
+    # warp slow, the squaring warps complete it twice before the store warp's
+    # parity wait looks, which then never sees its phase
+    cq = KERNEL['kQT'] * KERNEL['kTiles']
+    with pytest.raises(ProtocolError):
+        for seed in range(40):
+            for T, BH, grid in QUADRATIC_CASES:
+                n_ct = (T + cq - 1) // cq
+                g = min(grid, n_ct * BH)
+                for c in range(g):
+                    simulate(T, T, BH, quadratic_items(n_ct, BH, g, c), 1000 * seed + 7 * T + c,
+                             KERNEL, one_ostaged=True)
 
 
 def test_quadratic_schedule_is_deadlock_free_and_phase_exact():
