@@ -26,9 +26,12 @@
  * kept in fp32; the output has the input's dtype.
  *
  * General contract of every entry point
- *   - All tensor pointers are DEVICE pointers, owned by the caller, 16-byte
- *     aligned, dense row-major with the layout stated per argument.  The
- *     library allocates nothing and keeps no state between calls.
+ *   - All tensor pointers are DEVICE pointers (except the host buffers of
+ *     kata_chunked_forward_host), owned by the caller, 16-byte aligned, dense
+ *     row-major with the layout stated per argument.  The library allocates
+ *     no memory and keeps no state between calls (kata_chunked_forward_noalloc
+ *     uses a static scratch array, kata_chunked_forward_host creates and
+ *     releases its own streams and events: both documented below).
  *   - Work is enqueued on `stream` (NULL = legacy default stream) and the call
  *     returns without synchronising.  Errors found on the host (bad sizes,
  *     null or misaligned pointers, short workspace) return before anything is
