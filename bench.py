@@ -713,7 +713,8 @@ def measure_other_configs(K, inputs, stream, flush, names=("lm340m_B4H16_T16384_
         res[name] = {"ms": ms, "tokens_per_s": w.B * w.T / (ms / 1e3),
                      "canonical_tflops": canon / (ms / 1e3) / 1e12,
                      "frac_of_measured_peak": canon / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
-                     "path": "tensor cores" if w.d == 64 else "fp32 CUDA cores"}
+                     "path": ("fp32 CUDA cores" if w.dtype != "bf16" else "tensor cores" if w.d == 64
+                              else f"tensor cores, heads zero-padded from d = {w.d} to 64")}
         del q, k, v, so, zo, out, ws
     return res
 

@@ -48,7 +48,8 @@ int *device_status_ptr() {
     return ptrs[dev];
 }
 
-kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype, Plan &p) {
+kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype, Plan &p,
+                      bool padded_ok) {
     if (B < 1 || H < 1 || T < 1 || dk < 1 || dv < 1) return KATA_ERR_INVALID_ARG;
     if (!valid_chunk(C)) return KATA_ERR_INVALID_ARG;
     if (dtype != KATA_F32 && dtype != KATA_BF16) return KATA_ERR_UNSUPPORTED;
@@ -77,14 +78,26 @@ kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dty
     p.ws_seg_state = 0;
     p.ws_total = align_up(seg_bytes);
     p.ws_extra = p.ws_total + align_up(total_bytes);
+    p.ws_aux = 0;
     p.ws_bytes = p.ws_extra;
+    if (dtype == KATA_BF16) {
+        // the padded tensor-core route: q, k, v and out padded to d = 64, then
+        // the d = 64 plan's workspace (its layout is recomputed at launch)
+        Plan p64;
+        if (make_plan(B, H, T, 64, 64, C, dtype, p64) != KATA_OK) return KATA_ERR_UNSUPPORTED;
+        const size_t pad = 4 * align_up((size_t)BH * T * 64 * 2);
+        p.ws_aux = pad;  // offset of the d = 64 workspace
+        const size_t padded_bytes = pad + p64.ws_bytes;
+        if (padded_bytes > p.ws_bytes) p.ws_bytes = padded_bytes;
+        if (padded_ok) p.path = Path::kPaddedTensorCore;
+    }
     return KATA_OK;
 }
 
 // The quadratic form is the chunked plan with one segment spanning the whole
 // sequence: no state is built, scanned or stored, so no workspace is used.
 kata_status make_quadratic_plan(int B, int H, int T, int dk, int dv, kata_dtype dtype, Plan &p) {
-    const kata_status s = make_plan(B, H, T, dk, dv, 256, dtype, p);
+    const kata_status s = make_plan(B, H, T, dk, dv, 256, dtype, p, false);
     if (s != KATA_OK) return s;
     p.L = T;
     p.n_seg = 1;
@@ -115,6 +128,10 @@ kata_status check_forward_io(const Plan &p, const void *q, const void *k, const 
 cudaError_t launch_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
                            float *state_out, float *z_out, const InitState &init, void *ws,
                            cudaStream_t st, bool reuse_seg = false) {
+    if (p.path == Path::kPaddedTensorCore)
+        return init.n == 0 && out != nullptr && !reuse_seg
+                   ? launch_padded_forward(p, q, k, v, out, state_out, z_out, ws, st)
+                   : cudaErrorInvalidValue;  // the padded route serves the plain forward only
     return p.path == Path::kTensorCore
                ? tc::launch_tc_forward(p, q, k, v, out, state_out, z_out, init, ws, st, reuse_seg)
                : launch_simt_forward(p, q, k, v, out, state_out, z_out, init, ws, st);
@@ -246,7 +263,7 @@ kata_status kata_chunked_state(const void *k, const void *v, int B, int H, int T
                                int C, kata_dtype dtype, float *state_out, float *z_out,
                                void *workspace, size_t workspace_bytes, kata_stream_t stream) {
     Plan p;
-    const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p);
+    const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p, false);
     if (ps != KATA_OK) return ps;
     if (!k || !v || !aligned16(k) || !aligned16(v)) return KATA_ERR_INVALID_ARG;
     const kata_status so = kata::check_state_out(p, state_out, z_out, nullptr, k, v, true);
@@ -268,7 +285,7 @@ kata_status kata_chunked_forward_from_state(const void *q, const void *k, const 
                                             unsigned flags, kata_stream_t stream) {
     Plan p;
     if (flags & ~KATA_REUSE_SEGMENT_STATES) return KATA_ERR_INVALID_ARG;
-    const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p);
+    const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p, false);
     if (ps != KATA_OK) return ps;
     const kata_status io = kata::check_forward_io(p, q, k, v, out);
     if (io != KATA_OK) return io;

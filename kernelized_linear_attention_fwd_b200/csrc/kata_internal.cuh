@@ -36,7 +36,9 @@ __host__ __device__ inline void packed_row_ij(int d, int r, int &i, int &j) {
 // ---------------------------------------------------------------------------
 // Forward plan: segment length, number of segments, workspace layout.
 // ---------------------------------------------------------------------------
-enum class Path : int { kSimt = 0, kTensorCore = 1 };
+// kPaddedTensorCore: bf16 heads of d = 16 or 32 zero-padded to 64 and run on
+// the tensor-core kernels (zeros add nothing to any product or sum).
+enum class Path : int { kSimt = 0, kTensorCore = 1, kPaddedTensorCore = 2 };
 
 struct Plan {
     int B, H, T, dk, dv, C;
@@ -54,8 +56,12 @@ struct Plan {
     size_t ws_bytes;
 };
 
-// Fills `p`; returns KATA_OK or the error the forward must return.
-kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype, Plan &p);
+// Fills `p`; returns KATA_OK or the error the forward must return.  padded_ok:
+// bf16 heads of d < 64 may take the padded tensor-core route (the plain
+// forward); otherwise they take the fp32 CUDA-core path.  The workspace size
+// covers both routes either way, so one size query serves every entry point.
+kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype, Plan &p,
+                      bool padded_ok = true);
 // The plan of the quadratic form: one segment of T tokens, no workspace.
 kata_status make_quadratic_plan(int B, int H, int T, int dk, int dv, kata_dtype dtype, Plan &p);
 
@@ -119,14 +125,21 @@ namespace tc {
 // reuse_seg: the workspace already holds every segment's state, written by a
 // state-only launch for the same keys, values and sizes; skip building them.
 void plan_tc_workspace(Plan &p);
+// d_out: head size of the exported state (< 64 when the heads were padded).
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v,
                               void *out, float *state_out, float *z_out, const InitState &init,
-                              void *ws, cudaStream_t st, bool reuse_seg = false);
+                              void *ws, cudaStream_t st, bool reuse_seg = false, int d_out = 64);
 // Streaming multiprocessors of the current device (cached).
 int num_sms();
 }  // namespace tc
 
 // Decode step on the dense (d^2 rows) or packed (d(d+1)/2 rows) state layout.
+// The plain forward of bf16 heads of d < 64, zero-padded to 64 in the
+// workspace and run on the tensor-core kernels.
+cudaError_t launch_padded_forward(const Plan &p, const void *q, const void *k, const void *v,
+                                  void *out, float *state_out, float *z_out, void *ws,
+                                  cudaStream_t st);
+
 cudaError_t launch_decode(int B, int H, int dk, int dv, kata_dtype dtype, const void *q,
                           const void *k, const void *v, void *out, float *state, float *z,
                           bool packed, cudaStream_t st);

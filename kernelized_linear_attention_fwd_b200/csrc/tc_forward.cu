@@ -15,7 +15,8 @@
 //   tc_read          per 256 queries: phi(Q) S_prev and q^T Z_prev q on tcgen05
 //                    (phi(Q) generated from registers into tensor memory), the
 //                    intra-segment squared-score term on tcgen05, the division
-//   tc_state_expand  fp32 total -> dense [64*64, 64] state and [64, 64] Z
+//   tc_state_expand  fp32 total -> dense [d*d, d] state and [d, d] Z (d <= 64:
+//                    heads zero-padded to 64 export their leading d x d part)
 #include <cuda_bf16.h>
 
 #include "kata_internal.cuh"
@@ -167,23 +168,23 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__restrict__ state_out,
-                float *__restrict__ z_out, long long BH) {
-    const long long per = (long long)kD * kD * kD + kD * kD;
+                float *__restrict__ z_out, long long BH, int d) {
+    const long long d3 = (long long)d * d * d, per = d3 + (long long)d * d;
     const long long idx = (long long)blockIdx.x * 256 + threadIdx.x;
     if (idx >= per * BH) return;
     const long long bh = idx / per;
     long long x = idx % per;
     const float *src = total + bh * stride_bh;
-    if (x < (long long)kD * kD * kD) {
-        const int row = (int)(x / kD), e = (int)(x % kD);
-        int i = row / kD, j = row % kD;
+    if (x < d3) {
+        const int row = (int)(x / d), e = (int)(x % d);
+        int i = row / d, j = row % d;
         if (i > j) { const int t = i; i = j; j = t; }
-        state_out[bh * kD * kD * kD + x] = src[(long long)row_index(i, j) * kD + e];
+        state_out[bh * d3 + x] = src[(long long)row_index(i, j) * kD + e];
     } else {
-        x -= (long long)kD * kD * kD;
-        int i = (int)(x / kD), j = (int)(x % kD);
+        x -= d3;
+        int i = (int)(x / d), j = (int)(x % d);
         if (i > j) { const int t = i; i = j; j = t; }
-        z_out[bh * kD * kD + x] = src[kZPacked0 + row_index(i, j)];
+        z_out[bh * d * d + x] = src[kZPacked0 + row_index(i, j)];
     }
 }
 
@@ -1252,7 +1253,7 @@ void plan_tc_workspace(Plan &p) {
 
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
                               float *state_out, float *z_out, const InitState &init, void *ws,
-                              cudaStream_t st, bool reuse_seg) {
+                              cudaStream_t st, bool reuse_seg, int d_out) {
     // no workspace (the quadratic plan): no state is built, scanned or read
     char *w = static_cast<char *>(ws);
     float *seg = w ? reinterpret_cast<float *>(w + p.ws_seg_state) : nullptr;
@@ -1327,9 +1328,11 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
     if (want_state) {
         const float *src = scan ? total : seg;
         const long long stride = scan ? kF32PerSeg : kF32PerSeg * p.n_seg;
-        const long long n = ((long long)kD * kD * kD + kD * kD) * BH;
+        if (d_out < 1 || d_out > kD) return cudaErrorInvalidValue;
+        const long long n = ((long long)d_out * d_out * d_out + (long long)d_out * d_out) * BH;
         ProfScope ps("tc_state_expand", st);
-        tc_state_expand<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, stride, state_out, z_out, BH);
+        tc_state_expand<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, stride, state_out, z_out, BH,
+                                                                     d_out);
     }
     return cudaGetLastError();
 }
