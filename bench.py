@@ -172,13 +172,24 @@ def load_traffic(kernel, workload):
 # ---------------------------------------------------------------------------
 
 
+def smi_device_id(props):
+    """nvidia-smi's name for the GPU behind torch device properties `props`:
+    its UUID ("GPU-..."), else its PCI bus id ("dddddddd:bb:dd.0")."""
+    u = str(getattr(props, "uuid", "") or "")
+    if u:
+        return u if u.startswith("GPU-") else "GPU-" + u
+    return "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index):
-        self.dev = device_index
+    def __init__(self, smi_id):
+        # smi_id: the GPU as nvidia-smi names it (UUID or PCI bus id); nvidia-smi
+        # ignores CUDA_VISIBLE_DEVICES, so torch's device index may name another GPU
+        self.dev = smi_id
         self.proc = None
         self.tmp = None
 
@@ -337,7 +348,7 @@ def run_ours(args, rank, world):
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    clocks = ClockSampler(dev)
+    clocks = ClockSampler(smi_device_id(torch.cuda.get_device_properties(dev)))
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()

@@ -28,10 +28,17 @@
  * General contract of every entry point
  *   - All tensor pointers are DEVICE pointers (except the host buffers of
  *     kata_chunked_forward_host), owned by the caller, 16-byte aligned, dense
- *     row-major with the layout stated per argument.  The library allocates
- *     no memory and keeps no state between calls (kata_chunked_forward_noalloc
- *     uses a static scratch array, kata_chunked_forward_host creates and
- *     releases its own streams and events: both documented below).
+ *     row-major with the layout stated per argument, in the memory of the
+ *     CURRENT device (or managed memory): the kernels run on the current
+ *     device, and a pointer to host memory or to another device's memory is
+ *     rejected with KATA_ERR_INVALID_ARG before anything is launched.  The
+ *     library allocates no device memory and keeps no state between calls
+ *     beyond per-device handles: the device addresses of its status word and
+ *     of the kata_chunked_forward_noalloc scratch (looked up on first use),
+ *     and the copy streams and events of kata_chunked_forward_host (created
+ *     on first use, reused after).  Those handles belong to the device's
+ *     context: do not use the library on a device after cudaDeviceReset() on
+ *     it within the same process.
  *   - Work is enqueued on `stream` (NULL = legacy default stream) and the call
  *     returns without synchronising.  Errors found on the host (bad sizes,
  *     null or misaligned pointers, short workspace) return before anything is
@@ -202,9 +209,10 @@ kata_status kata_chunked_forward_from_state(const void *q, const void *k, const 
  *
  * Work is ordered after what is already queued on `stream`, and `stream`
  * completes only after every copy of the call (out holds the result once
- * `stream` has been synchronised).  The call creates two streams and a few
- * events and releases them when their work is done.  Same results as
- * kata_chunked_forward on device copies of the inputs.
+ * `stream` has been synchronised).  The call's two copy streams and its
+ * events come from a per-device pool (created by the first call, reused by
+ * later ones; concurrent calls from several host threads each take their
+ * own).  Same results as kata_chunked_forward on device copies of the inputs.
  */
 size_t kata_chunked_forward_host_buffer_bytes(int B, int H, int T, int dk, int dv, int C,
                                               kata_dtype dtype, int heads_per_group);
@@ -234,7 +242,9 @@ kata_status kata_chunked_forward_host(const void *q, const void *k, const void *
  *     the tensors current before the call.
  *   - The first call on a device looks the array's device address up
  *     (cudaGetSymbolAddress) and caches it.  Make that first call before
- *     any stream capture on that device.
+ *     any stream capture on that device.  The cached address belongs to the
+ *     device's context: after cudaDeviceReset() on that device it is stale,
+ *     so do not call this entry point on it again in the same process.
  *   - All calls on a device share the one array, and the array keeps what the
  *     last call wrote.  Every scratch element a call reads was first written
  *     by that same call, so nothing needs clearing between calls.  Calls

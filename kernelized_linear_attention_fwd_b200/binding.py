@@ -120,23 +120,43 @@ def _dtype_code(t):
     raise KataError(KATA_ERR_UNSUPPORTED, f"dtype {t.dtype}")
 
 
-def _stream_handle(stream):
+def _stream_handle(stream, device=None):
+    """Handle of `stream`, or of the current stream of `device` (the device the
+    call's tensors live on) when None.  A given stream must belong to that
+    device: kernels run on the stream's device, and pointers of another
+    device's memory are not valid there."""
     import torch
 
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and stream.device != device:
+        raise KataError(KATA_ERR_INVALID_ARG,
+                        f"stream is on {stream.device}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on_device(device):
+    """Context that makes `device` current for the call: the library launches
+    on the current device and takes its per-device resources (status word,
+    static scratch) from it."""
+    import torch
+
+    return torch.cuda.device(device)
 
 
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _check(t, name, shape, dtype=None):
+def _check(t, name, shape, dtype=None, device=None):
+    """t (optional) is a contiguous CUDA tensor of `shape` and `dtype` on
+    `device` (the device of the call's first tensor)."""
     if t is None:
         return
     if not t.is_cuda:
         raise KataError(KATA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} is on {t.device}, want {device}")
     if not t.is_contiguous():
         raise KataError(KATA_ERR_INVALID_ARG, f"{name} must be contiguous")
     if tuple(t.shape) != tuple(shape):
@@ -162,34 +182,36 @@ def kata_chunked_forward(q, k, v, C=64, out=None, state_out=None, z_out=None, wo
 
     lib = load_library()
     B, H, T, dk = q.shape
+    dev = q.device
     dv = v.shape[-1]
-    _check(q, "q", (B, H, T, dk))
-    _check(k, "k", (B, H, T, dk), q.dtype)
-    _check(v, "v", (B, H, T, dv), q.dtype)
+    _check(q, "q", (B, H, T, dk), device=dev)
+    _check(k, "k", (B, H, T, dk), q.dtype, device=dev)
+    _check(v, "v", (B, H, T, dv), q.dtype, device=dev)
     code = _dtype_code(q)
     if out is None:
         out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
-    _check(out, "out", (B, H, T, dv), q.dtype)
-    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32)
-    _check(z_out, "z_out", (B, H, dk, dk), torch.float32)
-    need = lib.kata_chunked_forward_workspace_bytes(B, H, T, dk, dv, C, code)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.kata_chunked_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv, int(C),
-                                  code, _ptr(state_out), _ptr(z_out), _ptr(workspace), ws_bytes,
-                                  _stream_handle(stream))
+    _check(out, "out", (B, H, T, dv), q.dtype, device=dev)
+    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32, device=dev)
+    _check(z_out, "z_out", (B, H, dk, dk), torch.float32, device=dev)
+    workspace, ws_bytes = _workspace(lib, workspace, B, H, T, dk, dv, C, code, dev)
+    with _on_device(dev):
+        st = lib.kata_chunked_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv,
+                                      int(C), code, _ptr(state_out), _ptr(z_out),
+                                      _ptr(workspace), ws_bytes, _stream_handle(stream, dev))
     if st != KATA_OK:
         raise KataError(st, "kata_chunked_forward")
     return out
 
 
 def _workspace(lib, workspace, B, H, T, dk, dv, C, code, device):
+    """(workspace, bytes): the caller's (on `device`) or one allocated here."""
     import torch
 
     need = lib.kata_chunked_forward_workspace_bytes(B, H, T, dk, dv, C, code)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    if workspace is not None and (not workspace.is_cuda or workspace.device != device):
+        raise KataError(KATA_ERR_INVALID_ARG, f"workspace must be on {device}")
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     return workspace, nbytes
 
@@ -201,34 +223,39 @@ def kata_chunked_state(k, v, C=64, state_out=None, z_out=None, workspace=None, s
 
     lib = load_library()
     B, H, T, dk = k.shape
+    dev = k.device
     dv = v.shape[-1]
-    _check(k, "k", (B, H, T, dk))
-    _check(v, "v", (B, H, T, dv), k.dtype)
+    _check(k, "k", (B, H, T, dk), device=dev)
+    _check(v, "v", (B, H, T, dv), k.dtype, device=dev)
     code = _dtype_code(k)
     if state_out is None:
         state_out = torch.empty((B, H, dk * dk, dv), dtype=torch.float32, device=k.device)
     if z_out is None:
         z_out = torch.empty((B, H, dk, dk), dtype=torch.float32, device=k.device)
-    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32)
-    _check(z_out, "z_out", (B, H, dk, dk), torch.float32)
-    workspace, nbytes = _workspace(lib, workspace, B, H, T, dk, dv, C, code, k.device)
-    st = lib.kata_chunked_state(_ptr(k), _ptr(v), B, H, T, dk, dv, int(C), code, _ptr(state_out),
-                                _ptr(z_out), _ptr(workspace), nbytes, _stream_handle(stream))
+    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32, device=dev)
+    _check(z_out, "z_out", (B, H, dk, dk), torch.float32, device=dev)
+    workspace, nbytes = _workspace(lib, workspace, B, H, T, dk, dv, C, code, dev)
+    with _on_device(dev):
+        st = lib.kata_chunked_state(_ptr(k), _ptr(v), B, H, T, dk, dv, int(C), code,
+                                    _ptr(state_out), _ptr(z_out), _ptr(workspace), nbytes,
+                                    _stream_handle(stream, dev))
     if st != KATA_OK:
         raise KataError(st, "kata_chunked_state")
     return state_out, z_out
 
 
-def _stacked(t, name, inner, n_name):
+def _stacked(t, name, inner, n_name, device=None):
     """(n, stride in elements) of a stack of states: t is [n, *inner] whose
     blocks t[m] are each contiguous (any stride between blocks), or one state
-    [*inner] (n = 1)."""
+    [*inner] (n = 1), on `device`."""
     import torch
 
     if t is None:
         return 0, 0
     if not t.is_cuda or t.dtype != torch.float32:
         raise KataError(KATA_ERR_INVALID_ARG, f"{name} must be a CUDA float32 tensor")
+    if device is not None and t.device != device:
+        raise KataError(KATA_ERR_INVALID_ARG, f"{name} is on {t.device}, want {device}")
     if tuple(t.shape) == tuple(inner):
         t = t.unsqueeze(0)
     if t.dim() != len(inner) + 1 or tuple(t.shape[1:]) != tuple(inner):
@@ -256,28 +283,31 @@ def kata_chunked_forward_from_state(q, k, v, state_in, z_in, C=64, out=None, sta
 
     lib = load_library()
     B, H, T, dk = q.shape
+    dev = q.device
     dv = v.shape[-1]
-    _check(q, "q", (B, H, T, dk))
-    _check(k, "k", (B, H, T, dk), q.dtype)
-    _check(v, "v", (B, H, T, dv), q.dtype)
+    _check(q, "q", (B, H, T, dk), device=dev)
+    _check(k, "k", (B, H, T, dk), q.dtype, device=dev)
+    _check(v, "v", (B, H, T, dv), q.dtype, device=dev)
     code = _dtype_code(q)
-    n_s, s_stride = _stacked(state_in, "state_in", (B, H, dk * dk, dv), "n")
-    n_z, z_stride = _stacked(z_in, "z_in", (B, H, dk, dk), "n")
+    n_s, s_stride = _stacked(state_in, "state_in", (B, H, dk * dk, dv), "n", dev)
+    n_z, z_stride = _stacked(z_in, "z_in", (B, H, dk, dk), "n", dev)
     if n_s != n_z:
         raise KataError(KATA_ERR_INVALID_ARG, f"state_in holds {n_s} states, z_in {n_z}")
     if out is None:
         out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
-    _check(out, "out", (B, H, T, dv), q.dtype)
-    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32)
-    _check(z_out, "z_out", (B, H, dk, dk), torch.float32)
+    _check(out, "out", (B, H, T, dv), q.dtype, device=dev)
+    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32, device=dev)
+    _check(z_out, "z_out", (B, H, dk, dk), torch.float32, device=dev)
     if reuse_segment_states and workspace is None:
         raise KataError(KATA_ERR_WORKSPACE, "reusing segment states needs the state call's workspace")
-    workspace, nbytes = _workspace(lib, workspace, B, H, T, dk, dv, C, code, q.device)
-    st = lib.kata_chunked_forward_from_state(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv, int(C), code,
-        _ptr(state_in) if n_s else None, _ptr(z_in) if n_z else None, n_s, s_stride, z_stride,
-        _ptr(state_out), _ptr(z_out), _ptr(workspace), nbytes,
-        KATA_REUSE_SEGMENT_STATES if reuse_segment_states else 0, _stream_handle(stream))
+    workspace, nbytes = _workspace(lib, workspace, B, H, T, dk, dv, C, code, dev)
+    with _on_device(dev):
+        st = lib.kata_chunked_forward_from_state(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv, int(C), code,
+            _ptr(state_in) if n_s else None, _ptr(z_in) if n_z else None, n_s, s_stride, z_stride,
+            _ptr(state_out), _ptr(z_out), _ptr(workspace), nbytes,
+            KATA_REUSE_SEGMENT_STATES if reuse_segment_states else 0,
+            _stream_handle(stream, dev))
     if st != KATA_OK:
         raise KataError(st, "kata_chunked_forward_from_state")
     return out
@@ -316,17 +346,27 @@ def kata_chunked_forward_host(q, k, v, out, C=64, state_out=None, z_out=None,
     _check_host(v, "v", (B, H, T, dv), q.dtype)
     _check_host(out, "out", (B, H, T, dv), q.dtype)
     code = _dtype_code(q)
-    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32)
-    _check(z_out, "z_out", (B, H, dk, dk), torch.float32)
+    # the device that runs the call: the device buffer's, else the state's, else the current one
+    if device_buffer is not None:
+        dev = device_buffer.device
+    elif state_out is not None:
+        dev = state_out.device
+    else:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32, device=dev)
+    _check(z_out, "z_out", (B, H, dk, dk), torch.float32, device=dev)
     need = kata_chunked_forward_host_buffer_bytes(B, H, T, dk, dv, int(C), code,
                                                   int(heads_per_group))
     if device_buffer is None:
-        device_buffer = torch.empty(max(need, 256), dtype=torch.uint8, device="cuda")
+        device_buffer = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    if not device_buffer.is_cuda:
+        raise KataError(KATA_ERR_INVALID_ARG, "device_buffer must be a CUDA tensor")
     nbytes = device_buffer.numel() * device_buffer.element_size()
-    st = lib.kata_chunked_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv,
-                                       int(C), code, _ptr(state_out), _ptr(z_out),
-                                       _ptr(device_buffer), nbytes, int(heads_per_group),
-                                       _stream_handle(stream))
+    with _on_device(dev):
+        st = lib.kata_chunked_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk,
+                                           dv, int(C), code, _ptr(state_out), _ptr(z_out),
+                                           _ptr(device_buffer), nbytes, int(heads_per_group),
+                                           _stream_handle(stream, dev))
     if st != KATA_OK:
         raise KataError(st, "kata_chunked_forward_host")
     return out
@@ -347,19 +387,21 @@ def kata_chunked_forward_noalloc(q, k, v, C=64, out=None, state_out=None, z_out=
 
     lib = load_library()
     B, H, T, dk = q.shape
+    dev = q.device
     dv = v.shape[-1]
-    _check(q, "q", (B, H, T, dk))
-    _check(k, "k", (B, H, T, dk), q.dtype)
-    _check(v, "v", (B, H, T, dv), q.dtype)
+    _check(q, "q", (B, H, T, dk), device=dev)
+    _check(k, "k", (B, H, T, dk), q.dtype, device=dev)
+    _check(v, "v", (B, H, T, dv), q.dtype, device=dev)
     code = _dtype_code(q)
     if out is None:
         out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
-    _check(out, "out", (B, H, T, dv), q.dtype)
-    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32)
-    _check(z_out, "z_out", (B, H, dk, dk), torch.float32)
-    st = lib.kata_chunked_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv,
-                                          int(C), code, _ptr(state_out), _ptr(z_out),
-                                          _stream_handle(stream))
+    _check(out, "out", (B, H, T, dv), q.dtype, device=dev)
+    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32, device=dev)
+    _check(z_out, "z_out", (B, H, dk, dk), torch.float32, device=dev)
+    with _on_device(dev):
+        st = lib.kata_chunked_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T,
+                                              dk, dv, int(C), code, _ptr(state_out),
+                                              _ptr(z_out), _stream_handle(stream, dev))
     if st != KATA_OK:
         raise KataError(st, "kata_chunked_forward_noalloc")
     return out
@@ -372,16 +414,18 @@ def kata_quadratic_forward(q, k, v, out=None, stream=None):
 
     lib = load_library()
     B, H, T, dk = q.shape
+    dev = q.device
     dv = v.shape[-1]
-    _check(q, "q", (B, H, T, dk))
-    _check(k, "k", (B, H, T, dk), q.dtype)
-    _check(v, "v", (B, H, T, dv), q.dtype)
+    _check(q, "q", (B, H, T, dk), device=dev)
+    _check(k, "k", (B, H, T, dk), q.dtype, device=dev)
+    _check(v, "v", (B, H, T, dv), q.dtype, device=dev)
     code = _dtype_code(q)
     if out is None:
         out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
-    _check(out, "out", (B, H, T, dv), q.dtype)
-    st = lib.kata_quadratic_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv, code,
-                                    _stream_handle(stream))
+    _check(out, "out", (B, H, T, dv), q.dtype, device=dev)
+    with _on_device(dev):
+        st = lib.kata_quadratic_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv,
+                                        code, _stream_handle(stream, dev))
     if st != KATA_OK:
         raise KataError(st, "kata_quadratic_forward")
     return out
@@ -393,18 +437,20 @@ def kata_decode_step(q, k, v, state, z, out=None, stream=None):
 
     lib = load_library()
     B, H, dk = q.shape
+    dev = q.device
     dv = v.shape[-1]
-    _check(q, "q", (B, H, dk))
-    _check(k, "k", (B, H, dk), q.dtype)
-    _check(v, "v", (B, H, dv), q.dtype)
+    _check(q, "q", (B, H, dk), device=dev)
+    _check(k, "k", (B, H, dk), q.dtype, device=dev)
+    _check(v, "v", (B, H, dv), q.dtype, device=dev)
     code = _dtype_code(q)
     if out is None:
         out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
-    _check(out, "out", (B, H, dv), q.dtype)
-    _check(state, "state", (B, H, dk * dk, dv), torch.float32)
-    _check(z, "z", (B, H, dk, dk), torch.float32)
-    st = lib.kata_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state), _ptr(z), B, H,
-                              dk, dv, code, _stream_handle(stream))
+    _check(out, "out", (B, H, dv), q.dtype, device=dev)
+    _check(state, "state", (B, H, dk * dk, dv), torch.float32, device=dev)
+    _check(z, "z", (B, H, dk, dk), torch.float32, device=dev)
+    with _on_device(dev):
+        st = lib.kata_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state), _ptr(z),
+                                  B, H, dk, dv, code, _stream_handle(stream, dev))
     if st != KATA_OK:
         raise KataError(st, "kata_decode_step")
     return out
@@ -422,19 +468,22 @@ def kata_decode_step_packed(q, k, v, state_p, z_p, out=None, stream=None):
 
     lib = load_library()
     B, H, dk = q.shape
+    dev = q.device
     dv = v.shape[-1]
     R = packed_rows(dk)
-    _check(q, "q", (B, H, dk))
-    _check(k, "k", (B, H, dk), q.dtype)
-    _check(v, "v", (B, H, dv), q.dtype)
+    _check(q, "q", (B, H, dk), device=dev)
+    _check(k, "k", (B, H, dk), q.dtype, device=dev)
+    _check(v, "v", (B, H, dv), q.dtype, device=dev)
     code = _dtype_code(q)
     if out is None:
         out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
-    _check(out, "out", (B, H, dv), q.dtype)
-    _check(state_p, "state_p", (B, H, R, dv), torch.float32)
-    _check(z_p, "z_p", (B, H, R), torch.float32)
-    st = lib.kata_decode_step_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state_p),
-                                     _ptr(z_p), B, H, dk, dv, code, _stream_handle(stream))
+    _check(out, "out", (B, H, dv), q.dtype, device=dev)
+    _check(state_p, "state_p", (B, H, R, dv), torch.float32, device=dev)
+    _check(z_p, "z_p", (B, H, R), torch.float32, device=dev)
+    with _on_device(dev):
+        st = lib.kata_decode_step_packed(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state_p),
+                                         _ptr(z_p), B, H, dk, dv, code,
+                                         _stream_handle(stream, dev))
     if st != KATA_OK:
         raise KataError(st, "kata_decode_step_packed")
     return out
@@ -446,18 +495,20 @@ def kata_state_pack(state, z, state_p=None, z_p=None, stream=None):
 
     lib = load_library()
     B, H, dd, dv = state.shape
+    dev = state.device
     dk = z.shape[-1]
     R = packed_rows(dk)
-    _check(state, "state", (B, H, dk * dk, dv), torch.float32)
-    _check(z, "z", (B, H, dk, dk), torch.float32)
+    _check(state, "state", (B, H, dk * dk, dv), torch.float32, device=dev)
+    _check(z, "z", (B, H, dk, dk), torch.float32, device=dev)
     if state_p is None:
         state_p = torch.empty((B, H, R, dv), dtype=torch.float32, device=state.device)
     if z_p is None:
         z_p = torch.empty((B, H, R), dtype=torch.float32, device=state.device)
-    _check(state_p, "state_p", (B, H, R, dv), torch.float32)
-    _check(z_p, "z_p", (B, H, R), torch.float32)
-    st = lib.kata_state_pack(_ptr(state), _ptr(z), _ptr(state_p), _ptr(z_p), B, H, dk, dv,
-                             _stream_handle(stream))
+    _check(state_p, "state_p", (B, H, R, dv), torch.float32, device=dev)
+    _check(z_p, "z_p", (B, H, R), torch.float32, device=dev)
+    with _on_device(dev):
+        st = lib.kata_state_pack(_ptr(state), _ptr(z), _ptr(state_p), _ptr(z_p), B, H, dk, dv,
+                                 _stream_handle(stream, dev))
     if st != KATA_OK:
         raise KataError(st, "kata_state_pack")
     return state_p, z_p
@@ -469,23 +520,31 @@ def kata_state_unpack(state_p, z_p, state=None, z=None, stream=None):
 
     lib = load_library()
     B, H, R, dv = state_p.shape
+    dev = state_p.device
     dk = next(d for d in (16, 32, 64) if packed_rows(d) == R) if R in (136, 528, 2080) else 0
     if dk == 0:
         raise KataError(KATA_ERR_UNSUPPORTED, f"no supported head size has {R} packed rows")
-    _check(state_p, "state_p", (B, H, R, dv), torch.float32)
-    _check(z_p, "z_p", (B, H, R), torch.float32)
+    _check(state_p, "state_p", (B, H, R, dv), torch.float32, device=dev)
+    _check(z_p, "z_p", (B, H, R), torch.float32, device=dev)
     if state is None:
         state = torch.empty((B, H, dk * dk, dv), dtype=torch.float32, device=state_p.device)
     if z is None:
         z = torch.empty((B, H, dk, dk), dtype=torch.float32, device=state_p.device)
-    _check(state, "state", (B, H, dk * dk, dv), torch.float32)
-    _check(z, "z", (B, H, dk, dk), torch.float32)
-    st = lib.kata_state_unpack(_ptr(state_p), _ptr(z_p), _ptr(state), _ptr(z), B, H, dk, dv,
-                               _stream_handle(stream))
+    _check(state, "state", (B, H, dk * dk, dv), torch.float32, device=dev)
+    _check(z, "z", (B, H, dk, dk), torch.float32, device=dev)
+    with _on_device(dev):
+        st = lib.kata_state_unpack(_ptr(state_p), _ptr(z_p), _ptr(state), _ptr(z), B, H, dk, dv,
+                                   _stream_handle(stream, dev))
     if st != KATA_OK:
         raise KataError(st, "kata_state_unpack")
     return state, z
 
 
 def kata_get_device_status(stream=None) -> int:
-    return int(load_library().kata_get_device_status(_stream_handle(stream)))
+    """Synchronises `stream` (default: the current device's current stream) and
+    returns and clears the status word of the stream's device."""
+    import torch
+
+    dev = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
+    with _on_device(dev):
+        return int(load_library().kata_get_device_status(_stream_handle(stream, dev)))

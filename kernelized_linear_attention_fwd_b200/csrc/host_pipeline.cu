@@ -6,9 +6,17 @@
 // Each group runs through kata_chunked_forward itself (same kernels, same
 // checks).  Two device slots, each holding one group's q, k, v and out,
 // alternate between groups; events order the reuse of a slot after the copy
-// that last read it.  Streams and events are created per call and released
-// when their work completes.
+// that last read it.  The two copy streams and the events come from a
+// per-device pool: a call takes a set (creating one the first time), enqueues
+// its work and returns the set, so repeated calls create nothing, and calls
+// from several host threads each hold a set of their own while they enqueue.
+// Reusing a set is safe as soon as the call that held it has returned: a
+// stream wait captures an event's state when the wait is enqueued, so
+// recording the event again later changes no wait already queued.
 #include <stdint.h>
+
+#include <mutex>
+#include <vector>
 
 #include "kata_internal.cuh"
 
@@ -28,6 +36,56 @@ struct HostPlan {
 };
 
 constexpr int kSlots = 2;
+
+// Copy streams and events of one call.
+struct PipeSet {
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t e_start = nullptr, e_in[kSlots] = {}, e_comp[kSlots] = {}, e_out[kSlots] = {};
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_pool_mu;
+std::vector<PipeSet *> g_pool[kMaxDevices];
+
+PipeSet *create_set() {
+    PipeSet *ps = new PipeSet;
+    bool ok = cudaStreamCreateWithFlags(&ps->s_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&ps->s_out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&ps->e_start, cudaEventDisableTiming) == cudaSuccess;
+    for (int s = 0; s < kSlots && ok; ++s)
+        ok = cudaEventCreateWithFlags(&ps->e_in[s], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&ps->e_comp[s], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&ps->e_out[s], cudaEventDisableTiming) == cudaSuccess;
+    if (ok) return ps;
+    if (ps->s_in) cudaStreamDestroy(ps->s_in);
+    if (ps->s_out) cudaStreamDestroy(ps->s_out);
+    if (ps->e_start) cudaEventDestroy(ps->e_start);
+    for (int s = 0; s < kSlots; ++s) {
+        if (ps->e_in[s]) cudaEventDestroy(ps->e_in[s]);
+        if (ps->e_comp[s]) cudaEventDestroy(ps->e_comp[s]);
+        if (ps->e_out[s]) cudaEventDestroy(ps->e_out[s]);
+    }
+    delete ps;
+    return nullptr;
+}
+
+// A set of the current device, from the pool or new; nullptr on failure.
+PipeSet *acquire_set(int dev) {
+    {
+        std::lock_guard<std::mutex> lk(g_pool_mu);
+        if (!g_pool[dev].empty()) {
+            PipeSet *ps = g_pool[dev].back();
+            g_pool[dev].pop_back();
+            return ps;
+        }
+    }
+    return create_set();
+}
+
+void release_set(int dev, PipeSet *ps) {
+    std::lock_guard<std::mutex> lk(g_pool_mu);
+    g_pool[dev].push_back(ps);
+}
 
 kata_status host_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype,
                       int heads_per_group, HostPlan &hp) {
@@ -78,21 +136,26 @@ kata_status kata_chunked_forward_host(const void *q, const void *k, const void *
         (reinterpret_cast<uintptr_t>(device_buffer) & 255u) != 0)
         return KATA_ERR_WORKSPACE;
 
+    if (!kata::device_ptrs_ok({device_buffer, state_out, z_out})) return KATA_ERR_INVALID_ARG;
+    int device = -1;
+    if (cudaGetDevice(&device) != cudaSuccess) return KATA_ERR_CUDA;
+    if (device < 0 || device >= kata::kMaxDevices) return KATA_ERR_UNSUPPORTED;
+    kata::PipeSet *set = kata::acquire_set(device);
+    if (!set) return KATA_ERR_CUDA;
     cudaStream_t user = reinterpret_cast<cudaStream_t>(stream);
-    cudaStream_t s_in = nullptr, s_out = nullptr;
-    cudaEvent_t e_start = nullptr, e_in[kata::kSlots] = {}, e_comp[kata::kSlots] = {},
-                e_out[kata::kSlots] = {};
-    bool ok = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) == cudaSuccess &&
-              cudaEventCreateWithFlags(&e_start, cudaEventDisableTiming) == cudaSuccess;
+    cudaStream_t s_in = set->s_in, s_out = set->s_out;
+    cudaEvent_t e_start = set->e_start, *e_in = set->e_in, *e_comp = set->e_comp,
+                *e_out = set->e_out;
+    // the copies start after the work already queued on the caller's stream; a
+    // slot's first use waits on nothing of this call's, so its events are
+    // first recorded right after that start point
+    bool ok = cudaEventRecord(e_start, user) == cudaSuccess &&
+              cudaStreamWaitEvent(s_in, e_start, 0) == cudaSuccess &&
+              cudaStreamWaitEvent(s_out, e_start, 0) == cudaSuccess;
     for (int s = 0; s < kata::kSlots && ok; ++s)
-        ok = cudaEventCreateWithFlags(&e_in[s], cudaEventDisableTiming) == cudaSuccess &&
-             cudaEventCreateWithFlags(&e_comp[s], cudaEventDisableTiming) == cudaSuccess &&
-             cudaEventCreateWithFlags(&e_out[s], cudaEventDisableTiming) == cudaSuccess;
-    // the copies start after the work already queued on the caller's stream
-    ok = ok && cudaEventRecord(e_start, user) == cudaSuccess &&
-         cudaStreamWaitEvent(s_in, e_start, 0) == cudaSuccess &&
-         cudaStreamWaitEvent(s_out, e_start, 0) == cudaSuccess;
+        ok = cudaEventRecord(e_comp[s], user) == cudaSuccess &&
+             cudaEventRecord(e_out[s], s_out) == cudaSuccess &&
+             cudaEventRecord(e_in[s], s_in) == cudaSuccess;
 
     kata_status status = ok ? KATA_OK : KATA_ERR_CUDA;
     const char *qh = static_cast<const char *>(q), *kh = static_cast<const char *>(k),
@@ -139,17 +202,12 @@ kata_status kata_chunked_forward_host(const void *q, const void *k, const void *
     }
     // the caller's stream completes after every copy this call queued
     for (int s = 0; s < kata::kSlots; ++s) {
-        if (e_out[s]) cudaStreamWaitEvent(user, e_out[s], 0);
-        if (e_in[s]) cudaStreamWaitEvent(user, e_in[s], 0);
+        cudaEventRecord(e_out[s], s_out);
+        cudaEventRecord(e_in[s], s_in);
+        cudaStreamWaitEvent(user, e_out[s], 0);
+        cudaStreamWaitEvent(user, e_in[s], 0);
     }
-    if (s_in) cudaStreamDestroy(s_in);
-    if (s_out) cudaStreamDestroy(s_out);
-    if (e_start) cudaEventDestroy(e_start);
-    for (int s = 0; s < kata::kSlots; ++s) {
-        if (e_in[s]) cudaEventDestroy(e_in[s]);
-        if (e_comp[s]) cudaEventDestroy(e_comp[s]);
-        if (e_out[s]) cudaEventDestroy(e_out[s]);
-    }
+    kata::release_set(device, set);
     return status;
 }
 

@@ -2,6 +2,9 @@
 // Declarations and the contract of every entry point: include/kata.h.
 #include <stdint.h>
 
+#include <initializer_list>
+#include <mutex>
+
 #include "kata_internal.cuh"
 
 namespace kata {
@@ -37,15 +40,33 @@ int segment_length(int dk, int C) {
 }  // namespace
 
 int *device_status_ptr() {
+    static std::mutex mu;
     static int *ptrs[64] = {nullptr};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
     if (!ptrs[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
         ptrs[dev] = static_cast<int *>(p);
     }
     return ptrs[dev];
+}
+
+bool device_ptrs_ok(std::initializer_list<const void *> ptrs) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    for (const void *p : ptrs) {
+        if (p == nullptr) continue;
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+            cudaGetLastError();  // clear the error this query left, so it reaches no later call
+            return false;
+        }
+        if (a.type == cudaMemoryTypeManaged) continue;
+        if (a.type != cudaMemoryTypeDevice || a.device != dev) return false;
+    }
+    return true;
 }
 
 kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype, Plan &p,
@@ -182,6 +203,7 @@ kata_status decode_step(const void *q, const void *k, const void *v, void *out, 
     const size_t ns = BH * rows * dv * 4, nz = BH * rows * 4, no = BH * dv * es;
     if (overlaps(state, ns, z, nz) || overlaps(out, no, state, ns) || overlaps(out, no, z, nz))
         return KATA_ERR_INVALID_ARG;
+    if (!device_ptrs_ok({q, k, v, out, state, z})) return KATA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e = launch_decode(B, H, dk, dv, dtype, q, k, v, out, state, z, packed, st);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
@@ -204,6 +226,7 @@ kata_status state_convert(bool pack, const float *src_s, const float *src_z, flo
         if (overlaps(d, n, src_s, ss) || overlaps(d, n, src_z, sz)) return KATA_ERR_INVALID_ARG;
     }
     if (overlaps(dst_s, ds, dst_z, dz)) return KATA_ERR_INVALID_ARG;
+    if (!device_ptrs_ok({src_s, src_z, dst_s, dst_z})) return KATA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e = launch_state_convert(pack, B, H, dk, src_s, src_z, dst_s, dst_z, st);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
@@ -253,6 +276,8 @@ kata_status kata_chunked_forward(const void *q, const void *k, const void *v, vo
     if (so != KATA_OK) return so;
     const kata_status ws = kata::check_workspace(p, workspace, workspace_bytes);
     if (ws != KATA_OK) return ws;
+    if (!kata::device_ptrs_ok({q, k, v, out, state_out, z_out, p.ws_bytes ? workspace : nullptr}))
+        return KATA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e =
         kata::launch_forward(p, q, k, v, out, state_out, z_out, kata::InitState{}, workspace, st);
@@ -270,6 +295,8 @@ kata_status kata_chunked_state(const void *k, const void *v, int B, int H, int T
     if (so != KATA_OK) return so;
     const kata_status ws = kata::check_workspace(p, workspace, workspace_bytes);
     if (ws != KATA_OK) return ws;
+    if (!kata::device_ptrs_ok({k, v, state_out, z_out, p.ws_bytes ? workspace : nullptr}))
+        return KATA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e = kata::launch_forward(p, nullptr, k, v, nullptr, state_out, z_out,
                                                kata::InitState{}, workspace, st);
@@ -318,6 +345,9 @@ kata_status kata_chunked_forward_from_state(const void *q, const void *k, const 
     }
     const kata_status ws = kata::check_workspace(p, workspace, workspace_bytes);
     if (ws != KATA_OK) return ws;
+    if (!kata::device_ptrs_ok({q, k, v, out, state_out, z_out, init.s, init.z,
+                               p.ws_bytes ? workspace : nullptr}))
+        return KATA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e = kata::launch_forward(p, q, k, v, out, state_out, z_out, init, workspace,
                                                st, (flags & KATA_REUSE_SEGMENT_STATES) != 0);
@@ -333,6 +363,7 @@ kata_status kata_quadratic_forward(const void *q, const void *k, const void *v, 
     const kata_status io = kata::check_forward_io(p, q, k, v, out);
     if (io != KATA_OK) return io;
     if (p.BH * ((T + 255LL) / 256) >= 0x7fffffffLL) return KATA_ERR_UNSUPPORTED;
+    if (!kata::device_ptrs_ok({q, k, v, out})) return KATA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e =
         kata::launch_forward(p, q, k, v, out, nullptr, nullptr, kata::InitState{}, nullptr, st);

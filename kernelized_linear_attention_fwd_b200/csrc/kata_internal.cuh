@@ -6,6 +6,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <initializer_list>
+#include <mutex>
+
 #include "../../include/kata.h"
 
 namespace kata {
@@ -69,6 +72,12 @@ kata_status make_quadratic_plan(int B, int H, int T, int dk, int dv, kata_dtype 
 // fails (one per device; resolved on first use with that device current).
 int *device_status_ptr();
 
+// True when every non-null pointer is memory of the current device (or
+// managed memory).  Host memory and another device's memory are rejected, so
+// a call given them returns an error instead of launching kernels that would
+// fault.  Checked after every other host-side check.
+bool device_ptrs_ok(std::initializer_list<const void *> ptrs);
+
 // Kernel timing (include/kata_profile.h): no-ops unless profiling is enabled.
 int prof_begin(const char *name, cudaStream_t st);
 void prof_end(int ev, cudaStream_t st);
@@ -83,12 +92,16 @@ struct ProfScope {
 // Opt-in dynamic shared memory of a kernel, set once per device: the
 // attribute lasts for the life of the context, and setting it on every launch
 // costs host time that small launches cannot hide.
+// The per-device record is guarded, so host threads may make first calls at
+// the same time.
 template <auto Kernel>
 cudaError_t smem_opt_in_once(int bytes) {
+    static std::mutex mu;
     static int set_bytes[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(mu);
     if (dev >= 0 && dev < 64 && set_bytes[dev] == bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess && dev >= 0 && dev < 64) set_bytes[dev] = bytes;

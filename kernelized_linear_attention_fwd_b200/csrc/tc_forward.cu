@@ -19,6 +19,8 @@
 //                    heads zero-padded to 64 export their leading d x d part)
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "kata_internal.cuh"
 #include "sm100.cuh"
 #include "tc_layout.cuh"
@@ -1221,9 +1223,11 @@ bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const
 
 // Streaming multiprocessors of the current device (persistent grids).
 int num_sms() {
+    static std::mutex mu;
     static int cache[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lk(mu);
     if (!cache[dev]) {
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;

@@ -296,6 +296,50 @@ def test_binding_rejects_host_tensors_and_bad_shapes(lib):
     assert binding.packed_rows(64) == 2080 and binding.packed_rows(16) == 136
 
 
+class _FakeCudaTensor:
+    """Stands in for a CUDA tensor on a given device (no GPU needed): only the
+    attributes the binding's checks read."""
+
+    def __init__(self, shape, dtype, device):
+        import torch
+
+        self.shape = tuple(shape)
+        self.dtype = dtype
+        self.device = torch.device(device)
+        self.is_cuda = True
+
+    def is_contiguous(self):
+        return True
+
+
+def test_binding_rejects_tensors_on_another_device():
+    # every tensor of a call must live on the first tensor's device; the call
+    # then runs with that device current (the library launches on the current
+    # device and takes its status word and static scratch from it)
+    import torch
+
+    shape = (1, 2, 8, 16)
+    q = _FakeCudaTensor(shape, torch.bfloat16, "cuda:0")
+    binding._check(q, "q", shape, torch.bfloat16, device=torch.device("cuda:0"))
+    for name, dev in (("k", "cuda:1"), ("out", "cuda:3")):
+        t = _FakeCudaTensor(shape, torch.bfloat16, dev)
+        with pytest.raises(binding.KataError) as e:
+            binding._check(t, name, shape, torch.bfloat16, device=q.device)
+        assert e.value.status == binding.KATA_ERR_INVALID_ARG and name in str(e.value)
+    s = _FakeCudaTensor((3, 1, 2, 256, 16), torch.float32, "cuda:1")
+    with pytest.raises(binding.KataError):
+        binding._stacked(s, "state_in", (1, 2, 256, 16), "n", q.device)
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+KATA_NOALLOC_SCRATCH_BYTES\s+\(([^)]*)\)", text)
+    assert m, "KATA_NOALLOC_SCRATCH_BYTES not found in kata.h"
+    expr = m.group(1).replace("u", "")
+    assert re.fullmatch(r"[0-9 *+]+", expr), expr
+    assert eval(expr) == binding.KATA_NOALLOC_SCRATCH_BYTES
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     saved = binding._lib
     try:

@@ -47,7 +47,11 @@ def _noalloc_call(lib, q, k, v, out, C, so=None, zo=None):
     return st
 
 
-@pytest.mark.parametrize("dtype,d,T,H", [("bf16", 64, 3000, 2), ("f32", 32, 2100, 3)])
+# bf16 d = 64: the tensor-core route; bf16 d = 32 and 16: the padded route,
+# which puts the most in the array (four padded q/k/v/out slabs, then the
+# d = 64 workspace); fp32: the CUDA-core route.
+@pytest.mark.parametrize("dtype,d,T,H", [("bf16", 64, 3000, 2), ("bf16", 32, 2000, 2),
+                                         ("bf16", 16, 2000, 2), ("f32", 32, 2100, 3)])
 def test_noalloc_matches_workspace_forward_twice(lib, dtype, d, T, H):
     B = 1
     code = binding.KATA_BF16 if dtype == "bf16" else binding.KATA_F32
