@@ -119,6 +119,14 @@ def alg_flops_per_token_head(kind, d, dv, C):
     return {"build": build, "read": read, "forward": build + read}[kind]
 
 
+def segment_length(d, C):
+    """Tokens between the library's stored states (include/kata.h, argument C):
+    C itself for C >= 512, else a fixed length per head size."""
+    if C >= 512:
+        return C
+    return 1024 if d >= 64 else (512 if d >= 32 else 256)
+
+
 def kernel_roofline_units(name, w, C, BH, T, n_seg, E_floats):
     """(bound, algorithmic units per launch, unit) for a kernel of the forward."""
     d = dv = w.d
@@ -476,19 +484,24 @@ def run_ours(args, rank, world):
         others = measure_other_configs(K, inputs, stream, flush)
 
     # one rank's compute of the sequence-sharded forward, on this GPU
+    def kernel_times(fn, n):  # per-kernel device ms per call, from the library's events
+        lib.kata_profile_enable(1)
+        for _ in range(n):
+            flush()
+            fn()
+        torch.cuda.synchronize()
+        lib.kata_profile_enable(0)
+        return {name: round(t / n, 4) for name, (c, t) in profile_read().items()}
+
     seq_split = None
     if not args.no_extras and w.dtype == "bf16":
         fwd_ms = sum(t for n, (c, t) in prof.items() if "decode" not in n) / args.steps
-        def kernel_times(fn, n):  # per-kernel device ms per call, from the library's events
-            lib.kata_profile_enable(1)
-            for _ in range(n):
-                flush()
-                fn()
-            torch.cuda.synchronize()
-            lib.kata_profile_enable(0)
-            return {name: round(t / n, 4) for name, (c, t) in profile_read().items()}
-
         seq_split = measure_sequence_split(K, q, k, v, C, stream, flush, fwd_ms, kernel_times)
+
+    # chunk size x sequence length sweep of the long-context workload
+    sweep = None
+    if not args.no_extras and w.name == WORKLOAD:
+        sweep = measure_chunk_sweep(K, inputs, stream, flush, kernel_times)
 
     if rank != 0:
         return None
@@ -497,7 +510,7 @@ def run_ours(args, rank, world):
     peaks, peak_src = load_peaks()
     R = d * (d + 1) // 2
     E = R * (d + 1)
-    L = max(1024 if d >= 64 else (512 if d >= 32 else 256), C)
+    L = segment_length(d, C)
     n_seg = (T + L - 1) // L
     fwd_kernels = {n: v for n, v in prof.items() if "decode" not in n}
     dom = max(fwd_kernels, key=lambda n: fwd_kernels[n][1])
@@ -561,6 +574,7 @@ def run_ours(args, rank, world):
         "quadratic_form": quad,
         "sequence_split": seq_split,
         "other_workloads": others,
+        "chunk_sweep": sweep,
         "device_status": status,
         "forward_canonical": canon,
     }
@@ -732,6 +746,46 @@ def measure_other_configs(K, inputs, stream, flush, names=("lm340m_B4H16_T16384_
                      "path": ("fp32 CUDA cores" if w.dtype != "bf16" else "tensor cores" if w.d == 64
                               else f"tensor cores, heads zero-padded from d = {w.d} to 64")}
         del q, k, v, so, zo, out, ws
+    return res
+
+
+def measure_chunk_sweep(K, inputs, stream, flush, kernel_times, d=64,
+                        Ts=(8192, 32768, 131072), Cs=(64, 128, 256, 512, 1024, 2048), H=8):
+    """The chunked forward (with state export) of the long-context workload over
+    sequence lengths T and chunk sizes C.  C <= 256 runs one schedule (states
+    every 1024 tokens at d = 64), C >= 512 keeps a state every C tokens: the
+    sweep over C >= 512 is the sweep of the segment length L, which trades
+    state traffic and scan passes against intra-segment work.  Inputs drawn on
+    the device, L2 flushed before each launch.  frac: canonical flops of the
+    chunked form at that C against the measured peak."""
+    import torch
+
+    peaks, _ = load_peaks()
+    res = {}
+    for T in Ts:
+        q, k, v = inputs.make_qkv_device(1, H, T, d, d, seed=0)
+        so = torch.empty((1, H, d * d, d), dtype=torch.float32, device=q.device)
+        zo = torch.empty((1, H, d, d), dtype=torch.float32, device=q.device)
+        out = torch.empty_like(v)
+        for C in Cs:
+            ws = torch.empty(max(K.kata_chunked_forward_workspace_bytes(1, H, T, d, d, C, 1), 256),
+                             dtype=torch.uint8, device=q.device)
+
+            def fwd():
+                K.kata_chunked_forward(q, k, v, C=C, out=out, state_out=so, z_out=zo,
+                                       workspace=ws, stream=stream)
+
+            ms = time_launches(fwd, stream, flush, 5, warm=2)
+            canon = H * T * alg_flops_per_token_head("forward", d, d, C)
+            L = segment_length(d, C)
+            res[f"T{T}_C{C}"] = {
+                "T": T, "C": C, "segment_L": L, "n_seg": (T + L - 1) // L, "ms": ms,
+                "tokens_per_s": T / (ms / 1e3),
+                "canonical_tflops": canon / (ms / 1e3) / 1e12,
+                "frac_of_measured_peak": canon / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                "kernels_ms": kernel_times(fwd, 3)}
+            del ws
+        del q, k, v, so, zo, out
     return res
 
 

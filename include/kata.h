@@ -99,10 +99,20 @@ size_t kata_chunked_forward_workspace_bytes(int B, int H, int T, int dk, int dv,
  *   q, k   [B, H, T, dk]  dtype      queries, keys
  *   v      [B, H, T, dv]  dtype      values
  *   out    [B, H, T, dv]  dtype      y_t as defined above
- *   C      chunk size, one of 16, 32, 64, 128, 256.  The result does not
- *          depend on C (the form is exact); states are stored only at
- *          segment boundaries that are multiples of C, and everything inside
- *          a segment is computed in its causal quadratic form.
+ *   C      chunk size: 16, 32, 64, 128, 256, 512, 1024, 2048 or 4096.  The
+ *          result does not depend on C (the form is exact for every C).  C
+ *          sets where states are kept; between them the exact causal
+ *          quadratic form is used:
+ *            C <= 256: chunks are merged into segments of a fixed length per
+ *              head size, L = 1024 tokens for dk = 64 (512 for 32, 256 for
+ *              16), a multiple of C.  Every such C runs the same kernels on
+ *              the same schedule (the intra-segment term is computed in
+ *              64-key blocks with the diagonal block masked).
+ *            C >= 512: states are kept every C tokens (L = C), which trades
+ *              state traffic and scan depth (about 1/C) against intra-chunk
+ *              work (about C).
+ *          The scan over the ceil(T / L) segment states is the associative
+ *          scan across chunks.
  *   state_out  nullable, [B, H, dk*dk, dv] fp32: S_T = sum_{s<T} phi(k_s) v_s^T,
  *          row index i*dk + j (symmetric in i, j), ready for kata_decode_step.
  *   z_out  nullable, [B, H, dk, dk] fp32: Z_T = sum_{s<T} k_s k_s^T.

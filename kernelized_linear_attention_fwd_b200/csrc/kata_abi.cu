@@ -21,7 +21,8 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool valid_chunk(int C) {
-    return C == 16 || C == 32 || C == 64 || C == 128 || C == 256;
+    return C == 16 || C == 32 || C == 64 || C == 128 || C == 256 || C == 512 || C == 1024 ||
+           C == 2048 || C == 4096;
 }
 
 bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
@@ -31,10 +32,13 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 
 // Segment length: states are stored every L tokens.  Inside a segment the
 // exact causal quadratic form is used, so L trades state traffic (~1/L)
-// against quadratic work (~L); L is a multiple of C and of 128.
+// against quadratic work (~L).  Chunks of C <= 256 tokens are merged into
+// segments of a length fixed per head size (a multiple of C), so every such C
+// runs the same schedule; C >= 512 sets the segment itself (L = C).  L is a
+// multiple of 256, as the tensor-core readout's 256-query work items need.
 int segment_length(int dk, int C) {
-    const int target = dk >= 64 ? 1024 : (dk >= 32 ? 512 : 256);
-    return target > C ? target : C;
+    if (C >= 512) return C;
+    return dk >= 64 ? 1024 : (dk >= 32 ? 512 : 256);
 }
 
 }  // namespace

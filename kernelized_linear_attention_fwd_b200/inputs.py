@@ -7,6 +7,9 @@ benchmark) and the fp64 oracle consume exactly the bits it produces.
 Recipe (all workloads): q, k i.i.d. N(0, 1), each row divided by its L2 norm
 in float64 (the small bf16 workload first scales by 1/sqrt(d), which the
 normalisation undoes, kept for fidelity to its description); v i.i.d. N(0, 1).
+Two unnormalised recipes exercise the dynamic range of the public calls (the
+feature u u^T needs no normalisation): qk="raw" keeps the N(0, 1) rows as
+drawn, qk="spread" gives each unit row a norm 2^e with e uniform in [-6, 6].
 Values are rounded float64 -> float32 (round to nearest even) and, for bf16,
 float32 -> bf16 (round to nearest even on the bit pattern).
 
@@ -38,7 +41,7 @@ class Workload:
     d: int
     C: int
     dtype: str            # "f32" or "bf16"
-    qk: str = "unit"      # "unit" | "scaled_unit"
+    qk: str = "unit"      # "unit" | "scaled_unit" | "raw" | "spread"
     seed: int = 0
     decode_steps: int = 0  # > 0: recall-shaped decode workload
     n_pairs: int = 0
@@ -111,9 +114,15 @@ def _one_head(args):
     if qk == "scaled_unit":
         q = q / math.sqrt(dk)
         k = k / math.sqrt(dk)
-    if qk in ("unit", "scaled_unit"):
+    if qk in ("unit", "scaled_unit", "spread"):
         q = _unit_rows(q)
         k = _unit_rows(k)
+    if qk == "spread":
+        # row norms 2^e, e ~ U[-6, 6] (drawn after v, so q, k, v keep their draws)
+        q = q * np.exp2(g.uniform(-6.0, 6.0, size=(T, 1)))
+        k = k * np.exp2(g.uniform(-6.0, 6.0, size=(T, 1)))
+    elif qk not in ("unit", "scaled_unit", "raw"):
+        raise ValueError(f"unknown q/k recipe {qk!r}")
     return _store(q, dtype), _store(k, dtype), _store(v, dtype)
 
 

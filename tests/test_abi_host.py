@@ -73,6 +73,12 @@ def test_workspace_query(lib):
     c = W(2, 8, 131072, 64, 64, 64, 1)
     assert a > b > 0 and c >= 2 * a - 512
     assert W(1, 1, 256, 16, 16, 64, 0) > 0
+    # C <= 256 merges chunks into the same segments (same workspace); C >= 512
+    # keeps a state every C tokens (more states for smaller C)
+    assert W(1, 8, 131072, 64, 64, 16, 1) == W(1, 8, 131072, 64, 64, 256, 1) == a
+    assert W(1, 8, 131072, 64, 64, 1024, 1) == a
+    assert W(1, 8, 131072, 64, 64, 512, 1) > a > W(1, 8, 131072, 64, 64, 2048, 1) > 0
+    assert W(1, 8, 131072, 64, 64, 4096, 1) > 0 and W(1, 8, 131072, 64, 64, 8192, 1) == 0
 
 
 def test_workspace_covers_both_routes_for_small_bf16_heads(lib):
@@ -109,7 +115,8 @@ def test_forward_rejects_bad_arguments(lib):
     assert _fwd(lib, T=0) == E.KATA_ERR_INVALID_ARG
     assert _fwd(lib, T=-5) == E.KATA_ERR_INVALID_ARG
     assert _fwd(lib, C=48) == E.KATA_ERR_INVALID_ARG
-    assert _fwd(lib, C=512) == E.KATA_ERR_INVALID_ARG
+    assert _fwd(lib, C=8192) == E.KATA_ERR_INVALID_ARG
+    assert _fwd(lib, C=768) == E.KATA_ERR_INVALID_ARG
     assert _fwd(lib, dk=128, dv=128) == E.KATA_ERR_UNSUPPORTED
     assert _fwd(lib, dk=16, dv=32) == E.KATA_ERR_UNSUPPORTED
     assert _fwd(lib, dt=3) == E.KATA_ERR_UNSUPPORTED

@@ -17,7 +17,8 @@ import numpy as np
 import pytest
 
 from kernelized_linear_attention_fwd_b200 import inputs
-from tests.gpu_util import STATE_BOUND, TOL, from_device, row_err, sample_rows, to_device
+from tests.gpu_util import (TOL, assert_state_close, from_device, row_err, sample_rows,
+                            to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -47,11 +48,7 @@ def f32(a):
 
 
 def check_state(oracle_mod, Sg, Zg, k64, v64, dtype):
-    S, Z = oracle_mod.state(k64, v64)
-    Sabs, Zabs = oracle_mod.state(np.abs(k64), np.abs(v64))
-    u = STATE_BOUND[dtype]
-    assert np.all(np.abs(from_device(Sg) - S) <= u * Sabs + 1e-6)
-    assert np.all(np.abs(from_device(Zg) - Z) <= u * Zabs + 1e-6)
+    assert_state_close(oracle_mod, from_device(Sg), from_device(Zg), k64, v64, dtype)
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])

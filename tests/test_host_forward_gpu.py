@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 
 from kernelized_linear_attention_fwd_b200 import inputs
-from tests.gpu_util import STATE_BOUND, TOL, from_device, row_err, to_device
+from tests.gpu_util import TOL, assert_state_close, from_device, row_err, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -56,11 +56,7 @@ def test_host_forward(oracle_mod, dtype, d, B, H, T, G):
     yd = from_device(K.kata_chunked_forward(to_device(q, dtype), to_device(k, dtype),
                                             to_device(v, dtype), C=64))
     assert row_err(y, yd) <= (1e-6 if dtype == "f32" else 2.0 ** -7)
-    S, Z = oracle_mod.state(k64, v64)
-    Sabs, Zabs = oracle_mod.state(np.abs(k64), np.abs(v64))
-    u = STATE_BOUND[dtype]
-    assert np.all(np.abs(from_device(so) - S) <= u * Sabs + 1e-6)
-    assert np.all(np.abs(from_device(zo) - Z) <= u * Zabs + 1e-6)
+    assert_state_close(oracle_mod, from_device(so), from_device(zo), k64, v64, dtype)
 
 
 def test_host_forward_orders_after_the_stream():

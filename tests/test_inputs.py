@@ -43,3 +43,26 @@ def test_named_workloads():
     pos, pick = inputs.recall_decode_plan(plan_w)
     assert pos.shape == (4096,) and len(np.unique(pos)) == 4096 and pos.max() < 32768
     assert pick.shape == (1024, 64, 16) and pick.max() < 4096
+
+
+def test_unnormalised_recipes():
+    # raw: the N(0, 1) rows as drawn (norms near sqrt(d)); spread: unit
+    # directions with norms 2^e, e uniform in [-6, 6]; v is the same draw in
+    # every recipe, and the directions of spread rows are those of unit rows
+    qr, kr, vr = inputs.make_qkv(1, 2, 4000, 64, 64, "f32", seed=3, qk="raw")
+    qs, ks, vs = inputs.make_qkv(1, 2, 4000, 64, 64, "f32", seed=3, qk="spread")
+    qu, ku, vu = inputs.make_qkv(1, 2, 4000, 64, 64, "f32", seed=3, qk="unit")
+    assert np.array_equal(vr, vu) and np.array_equal(vs, vu)
+    nr = np.linalg.norm(kr.astype(np.float64), axis=-1)
+    assert abs(nr.mean() - 8.0) < 0.2
+    ns = np.log2(np.linalg.norm(ks.astype(np.float64), axis=-1))
+    assert ns.min() >= -6.001 and ns.max() <= 6.001 and ns.max() - ns.min() > 11.5
+    assert abs(ns.mean()) < 0.3
+    cos = (ks.astype(np.float64) * ku).sum(-1) / np.linalg.norm(ks.astype(np.float64), axis=-1)
+    assert np.allclose(cos, 1.0, atol=1e-5)
+    try:
+        inputs.make_qkv(1, 1, 4, 8, 8, "f32", qk="bogus")
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("unknown recipe accepted")

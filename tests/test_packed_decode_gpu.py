@@ -16,7 +16,7 @@ import numpy as np
 import pytest
 
 from kernelized_linear_attention_fwd_b200 import inputs
-from tests.gpu_util import STATE_BOUND, TOL, from_device, row_err, to_device
+from tests.gpu_util import TOL, assert_state_close, from_device, row_err, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -80,11 +80,7 @@ def test_packed_decode_steps(oracle_mod, dtype, d):
     yref = oracle_mod.forward(q64, k64, v64)[:, :, T:]
     assert row_err(np.stack(ys, axis=2), yref) <= TOL[dtype]
     S2, Z2 = K.kata_state_unpack(Sp, Zp)
-    Sref, Zref = oracle_mod.state(k64, v64)
-    Sabs, Zabs = oracle_mod.state(np.abs(k64), np.abs(v64))
-    u = STATE_BOUND[dtype]
-    assert np.all(np.abs(from_device(S2) - Sref) <= u * Sabs + 1e-6)
-    assert np.all(np.abs(from_device(Z2) - Zref) <= u * Zabs + 1e-6)
+    assert_state_close(oracle_mod, from_device(S2), from_device(Z2), k64, v64, dtype)
 
 
 @pytest.mark.parametrize("BH", [1, 8, 37, 148, 1024])
