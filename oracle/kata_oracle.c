@@ -367,3 +367,194 @@ void kata_oracle_decode_step(const double *q, const double *k, const double *v, 
         readout(q + bh * dk, Sh, Zh, dk, dv, y + bh * dv, den ? den + bh : NULL);
     }
 }
+
+/* ------------------------------------------------------------------ */
+/* KATA-Mg: several rank-one PSD factors per head.                      */
+/* ------------------------------------------------------------------ */
+
+/* gist.science summary, Technical summary 2.3 ("Variantes"): KATA-Mg uses
+ * several PSD factors to trade state size against packing efficiency.  The
+ * pages name the variant without its formula; the reading taken (listed with
+ * the other readings in the design notes): the feature cone is a product of
+ * g rank-one PSD cones (2.1: the admissible geometries are the irreducible
+ * factors of the Koecher-Vinberg classification, of which a symmetric cone is
+ * a product), factor m with its own projection dimension p = dk / g (2.2)
+ * acting on coordinates [m p, (m + 1) p) of q and k.  The inner product on a
+ * product of cones is the sum of the factors' inner products, so
+ *
+ *     w_ts = sum_m (q_t^(m) . k_s^(m))^2 ,   y_t = sum_{s<=t} w_ts v_s / sum_{s<=t} w_ts
+ *
+ * with y_t = 0 when the sum is 0 (as for one factor).  The state is the g
+ * blocks S^(m)[(i,j), e] = sum_s k_si k_sj v_se with i, j both in block m, and
+ * Z^(m) likewise; g = 1 is the single factor above.  dk must be a multiple
+ * of g. */
+
+/* The Mg weight of query row qt and key row ks. */
+static double mg_weight(const double *qt, const double *ks, int dk, int g) {
+    const int p = dk / g;
+    double w = 0.0;
+    for (int m = 0; m < g; ++m) {
+        double dot = 0.0;
+        for (int i = m * p; i < (m + 1) * p; ++i) dot += qt[i] * ks[i];
+        w += dot * dot;
+    }
+    return w;
+}
+
+typedef struct {
+    const double *q, *k, *v;
+    double *y, *den;
+    long T;
+    int dk, dv, g;
+    const long *bh_idx, *t_idx; /* NULL: every row, item = bh*T + t */
+} mg_rows_ctx;
+
+static void mg_rows_item(void *c, long item) {
+    mg_rows_ctx *x = (mg_rows_ctx *)c;
+    long bh, t;
+    if (x->bh_idx) {
+        bh = x->bh_idx[item];
+        t = x->t_idx[item];
+    } else {
+        bh = item / x->T;
+        t = item % x->T;
+    }
+    const int dk = x->dk, dv = x->dv;
+    const double *qt = x->q + (bh * x->T + t) * dk;
+    double *y = x->y + item * dv;
+    double den = 0.0;
+    for (int e = 0; e < dv; ++e) y[e] = 0.0;
+    for (long s = 0; s <= t; ++s) {
+        const double *vs = x->v + (bh * x->T + s) * dv;
+        double w = mg_weight(qt, x->k + (bh * x->T + s) * dk, dk, x->g);
+        den += w;
+        for (int e = 0; e < dv; ++e) y[e] += w * vs[e];
+    }
+    for (int e = 0; e < dv; ++e) y[e] = (den == 0.0) ? 0.0 : y[e] / den;
+    if (x->den) x->den[item] = den;
+}
+
+/* Every row of every head; returns 1 (nothing computed) if g does not divide dk. */
+int kata_oracle_forward_mg(const double *q, const double *k, const double *v, double *y,
+                           double *den, long BH, long T, int dk, int dv, int g, int nthreads) {
+    if (g < 1 || dk % g != 0) return 1;
+    mg_rows_ctx c = {q, k, v, y, den, T, dk, dv, g, NULL, NULL};
+    run_items(mg_rows_item, &c, BH * T, nthreads);
+    return 0;
+}
+
+/* Selected rows (bh_idx[r], t_idx[r]); y: [nrows][dv]; den: [nrows]. */
+int kata_oracle_forward_mg_rows(const double *q, const double *k, const double *v, long T,
+                                int dk, int dv, int g, const long *bh_idx, const long *t_idx,
+                                long nrows, double *y, double *den, int nthreads) {
+    if (g < 1 || dk % g != 0) return 1;
+    mg_rows_ctx c = {q, k, v, y, den, T, dk, dv, g, bh_idx, t_idx};
+    run_items(mg_rows_item, &c, nrows, nthreads);
+    return 0;
+}
+
+/* The Mg state after the first n tokens, in the dense layout of the single
+ * factor: S[(i,j), e] = sum_{s<n} k_si k_sj v_se and Z[i, j] = sum_{s<n} k_si k_sj
+ * when i and j lie in the same block of p coordinates, and 0 otherwise (the
+ * g blocks of the product cone's state, side by side). */
+typedef struct {
+    const double *k, *v;
+    double *S, *Z;
+    long T, n;
+    int dk, dv, g;
+} mg_state_ctx;
+
+static void mg_state_item(void *c, long bh) {
+    mg_state_ctx *x = (mg_state_ctx *)c;
+    const int dk = x->dk, dv = x->dv, p = dk / x->g;
+    double *S = x->S + bh * (long)dk * dk * dv;
+    double *Z = x->Z + bh * (long)dk * dk;
+    memset(S, 0, sizeof(double) * (size_t)dk * dk * dv);
+    memset(Z, 0, sizeof(double) * (size_t)dk * dk);
+    for (long s = 0; s < x->n; ++s) {
+        const double *ks = x->k + (bh * x->T + s) * dk;
+        const double *vs = x->v + (bh * x->T + s) * dv;
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dk; ++j) {
+                if (i / p != j / p) continue;
+                double f = ks[i] * ks[j];
+                Z[i * dk + j] += f;
+                double *row = S + ((long)i * dk + j) * dv;
+                for (int e = 0; e < dv; ++e) row[e] += f * vs[e];
+            }
+    }
+}
+
+int kata_oracle_state_mg(const double *k, const double *v, long BH, long T, long n, int dk,
+                         int dv, int g, double *S, double *Z, int nthreads) {
+    if (g < 1 || dk % g != 0) return 1;
+    mg_state_ctx c = {k, v, S, Z, T, n, dk, dv, g};
+    run_items(mg_state_item, &c, BH, nthreads);
+    return 0;
+}
+
+/* Recurrent Mg form: per token, the block state update then the readout
+ * phi(q)^T S / (q^T Z q) over the blocks (zeros elsewhere add nothing); a
+ * second route to the Mg outputs. */
+typedef struct {
+    const double *q, *k, *v;
+    double *y;
+    long T;
+    int dk, dv, g;
+} mg_rec_ctx;
+
+static void mg_rec_item(void *c, long bh) {
+    mg_rec_ctx *x = (mg_rec_ctx *)c;
+    const int dk = x->dk, dv = x->dv, p = dk / x->g;
+    double *S = (double *)calloc((size_t)dk * dk * dv, sizeof(double));
+    double *Z = (double *)calloc((size_t)dk * dk, sizeof(double));
+    for (long t = 0; t < x->T; ++t) {
+        const double *kt = x->k + (bh * x->T + t) * dk;
+        const double *vt = x->v + (bh * x->T + t) * dv;
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dk; ++j) {
+                if (i / p != j / p) continue;
+                double f = kt[i] * kt[j];
+                Z[i * dk + j] += f;
+                double *row = S + ((long)i * dk + j) * dv;
+                for (int e = 0; e < dv; ++e) row[e] += f * vt[e];
+            }
+        readout(x->q + (bh * x->T + t) * dk, S, Z, dk, dv, x->y + (bh * x->T + t) * dv, NULL);
+    }
+    free(S);
+    free(Z);
+}
+
+int kata_oracle_forward_mg_recurrent(const double *q, const double *k, const double *v,
+                                     double *y, long BH, long T, int dk, int dv, int g,
+                                     int nthreads) {
+    if (g < 1 || dk % g != 0) return 1;
+    mg_rec_ctx c = {q, k, v, y, T, dk, dv, g};
+    run_items(mg_rec_item, &c, BH, nthreads);
+    return 0;
+}
+
+/* One Mg decode step: the block state update for token (k, v), then the
+ * readout with query q, current token included.  S, Z hold Mg states (zeros
+ * outside the blocks) and stay so. */
+int kata_oracle_decode_step_mg(const double *q, const double *k, const double *v, double *S,
+                               double *Z, double *y, double *den, long BH, int dk, int dv,
+                               int g) {
+    if (g < 1 || dk % g != 0) return 1;
+    const int p = dk / g;
+    for (long bh = 0; bh < BH; ++bh) {
+        double *Sh = S + bh * (long)dk * dk * dv;
+        double *Zh = Z + bh * (long)dk * dk;
+        const double *kh = k + bh * dk, *vh = v + bh * dv;
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dk; ++j) {
+                if (i / p != j / p) continue;
+                double f = kh[i] * kh[j];
+                Zh[i * dk + j] += f;
+                double *row = Sh + ((long)i * dk + j) * dv;
+                for (int e = 0; e < dv; ++e) row[e] += f * vh[e];
+            }
+        readout(q + bh * dk, Sh, Zh, dk, dv, y + bh * dv, den ? den + bh : NULL);
+    }
+    return 0;
+}
