@@ -110,12 +110,14 @@ def job_throughput(world, tokens_per_rank, ms_max):
 # ---------------------------------------------------------------------------
 
 
-def alg_flops_per_token_head(kind, d, dv, C):
+def alg_flops_per_token_head(kind, d, dv, C, g=1):
     """Canonical flops of the method's chunked-state form, per token and head:
     state build 2 d^2 dv + normaliser build 2 d^2; readout 2 d^2 dv + normaliser
-    readout 2 d^2 + causal intra-chunk term (C + 1)(d + dv)."""
-    build = 2 * d * d * dv + 2 * d * d
-    read = 2 * d * d * dv + 2 * d * d + (C + 1) * (d + dv)
+    readout 2 d^2 + causal intra-chunk term (C + 1)(d + dv).  With g factors
+    (KATA-Mg) the state has d^2 / g rows instead of d^2."""
+    rows = d * d // g
+    build = 2 * rows * dv + 2 * rows
+    read = 2 * rows * dv + 2 * rows + (C + 1) * (d + dv)
     return {"build": build, "read": read, "forward": build + read}[kind]
 
 
@@ -498,6 +500,14 @@ def run_ours(args, rank, world):
         fwd_ms = sum(t for n, (c, t) in prof.items() if "decode" not in n) / args.steps
         seq_split = measure_sequence_split(K, q, k, v, C, stream, flush, fwd_ms, kernel_times)
 
+    # KATA-Mg with two factors on the same inputs
+    mg = None
+    if not args.no_extras and w.dtype == "bf16" and d == 64:
+        m1_ms = sum(t for n, (c, t) in prof.items() if "decode" not in n) / args.steps
+        mg = measure_mg(K, q, k, v, C, stream, flush, kernel_times, m1_ms)
+        if K.kata_get_device_status() != 0:
+            raise RuntimeError("device status set by the two-factor forward")
+
     # chunk size x sequence length sweep of the long-context workload
     sweep = None
     if not args.no_extras and w.name == WORKLOAD:
@@ -575,6 +585,7 @@ def run_ours(args, rank, world):
         "sequence_split": seq_split,
         "other_workloads": others,
         "chunk_sweep": sweep,
+        "mg_two_factors": mg,
         "device_status": status,
         "forward_canonical": canon,
     }
@@ -746,6 +757,36 @@ def measure_other_configs(K, inputs, stream, flush, names=("lm340m_B4H16_T16384_
                      "path": ("fp32 CUDA cores" if w.dtype != "bf16" else "tensor cores" if w.d == 64
                               else f"tensor cores, heads zero-padded from d = {w.d} to 64")}
         del q, k, v, so, zo, out, ws
+    return res
+
+
+def measure_mg(K, q, k, v, C, stream, flush, kernel_times, m1_ms, g=2):
+    """The KATA-Mg forward (g factors, state exported) on the step's own
+    inputs, beside the single-factor forward: ms, tokens/s, canonical flops of
+    the g-factor form against the measured peak, per-kernel times."""
+    import torch
+
+    peaks, _ = load_peaks()
+    B, H, T, d = q.shape
+    so = torch.empty((B, H, d * d, d), dtype=torch.float32, device=q.device)
+    zo = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    out = torch.empty_like(v)
+    ws = torch.empty(max(K.kata_mg_chunked_forward_workspace_bytes(B, H, T, d, d, C, g, 1), 256),
+                     dtype=torch.uint8, device=q.device)
+
+    def fwd():
+        K.kata_mg_chunked_forward(q, k, v, g=g, C=C, out=out, state_out=so, z_out=zo,
+                                  workspace=ws, stream=stream)
+
+    ms = time_launches(fwd, stream, flush, 5, warm=2)
+    canon = B * H * T * alg_flops_per_token_head("forward", d, d, C, g)
+    res = {"g": g, "ms": ms, "tokens_per_s": B * T / (ms / 1e3),
+           "canonical_flop_per_token_head": alg_flops_per_token_head("forward", d, d, C, g),
+           "canonical_tflops": canon / (ms / 1e3) / 1e12,
+           "frac_of_measured_peak": canon / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+           "speedup_vs_one_factor_forward": m1_ms / ms,
+           "kernels_ms": kernel_times(fwd, 3)}
+    del so, zo, out, ws
     return res
 
 

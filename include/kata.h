@@ -269,6 +269,42 @@ kata_status kata_chunked_forward_noalloc(const void *q, const void *k, const voi
                                          kata_stream_t stream);
 
 /*
+ * KATA-Mg: g rank-one PSD factors per head (gist.science summary 2.3,
+ * "Variantes": several PSD factors, trading state size against packing
+ * efficiency).  The pages print no formula; the reading implemented (2.1: the
+ * admissible cones are products of Koecher-Vinberg factors; 2.2: a projection
+ * dimension p per factor) is the product of g rank-one PSD cones, factor m
+ * acting on the coordinates [m p, (m+1) p) of q and k, p = dk / g:
+ *
+ *     w_ts = sum_m (q_t^(m) . k_s^(m))^2,
+ *     y_t  = sum_{s<=t} w_ts v_s / sum_{s<=t} w_ts                 (y_t = 0 if 0)
+ *
+ * The state is the g blocks of p*p x dv (dk^2 / g rows in all): 2 factors
+ * halve the state of one.  g = 1 is kata_chunked_forward itself.
+ *
+ *   kata_mg_chunked_forward: as kata_chunked_forward (same arguments plus g,
+ *       same workspace rules with its own size query).  g in {1, 2}: bf16
+ *       heads of dk = 64 with g = 2 run the tensor-core path on a layout of the
+ *       1056 pairs inside the factors; other head sizes and fp32 run fp32
+ *       CUDA-core arithmetic.  Other g: KATA_ERR_UNSUPPORTED.
+ *       state_out / z_out: the dense layouts of kata_chunked_forward, holding
+ *       zeros at every pair (i, j) whose coordinates lie in different factors.
+ *   kata_mg_decode_step: kata_decode_step for g factors on that dense layout:
+ *       S[(i,j)] += k_i k_j v and Z[i,j] += k_i k_j only for i, j in one
+ *       factor (the other rows stay zero and are neither read nor written),
+ *       then y = phi(q)^T S / (q^T Z q).  g in {1, 2}.
+ */
+size_t kata_mg_chunked_forward_workspace_bytes(int B, int H, int T, int dk, int dv, int C, int g,
+                                               kata_dtype dtype);
+kata_status kata_mg_chunked_forward(const void *q, const void *k, const void *v, void *out, int B,
+                                    int H, int T, int dk, int dv, int C, int g, kata_dtype dtype,
+                                    float *state_out, float *z_out, void *workspace,
+                                    size_t workspace_bytes, kata_stream_t stream);
+kata_status kata_mg_decode_step(const void *q, const void *k, const void *v, void *out,
+                                float *state, float *z, int B, int H, int dk, int dv, int g,
+                                kata_dtype dtype, kata_stream_t stream);
+
+/*
  * Causal KATA forward in its quadratic form: the flash-attention-style
  * operating point (gist.science summary 2.3, "two operating points", the
  * O(T^2) forward that never forms the state; arXiv abstract,

@@ -16,6 +16,9 @@ from .binding import (  # noqa: F401
     kata_decode_step,
     kata_decode_step_packed,
     kata_get_device_status,
+    kata_mg_chunked_forward,
+    kata_mg_chunked_forward_workspace_bytes,
+    kata_mg_decode_step,
     kata_quadratic_forward,
     kata_state_pack,
     kata_state_unpack,

@@ -36,6 +36,9 @@ EXPORTS = (
     "kata_chunked_forward_host_buffer_bytes",
     "kata_chunked_forward_host",
     "kata_quadratic_forward",
+    "kata_mg_chunked_forward_workspace_bytes",
+    "kata_mg_chunked_forward",
+    "kata_mg_decode_step",
     "kata_decode_step",
     "kata_decode_step_packed",
     "kata_state_pack",
@@ -87,6 +90,13 @@ def load_library(path: str = LIB_PATH):
     lib.kata_chunked_forward_noalloc.restype = i32
     lib.kata_chunked_forward_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                  i32, fp, fp, vp]
+    lib.kata_mg_chunked_forward_workspace_bytes.restype = sz
+    lib.kata_mg_chunked_forward_workspace_bytes.argtypes = [i32] * 8
+    lib.kata_mg_chunked_forward.restype = i32
+    lib.kata_mg_chunked_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                            i32, fp, fp, vp, sz, vp]
+    lib.kata_mg_decode_step.restype = i32
+    lib.kata_mg_decode_step.argtypes = [vp, vp, vp, vp, fp, fp, i32, i32, i32, i32, i32, i32, vp]
     lib.kata_quadratic_forward.restype = i32
     lib.kata_quadratic_forward.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
     lib.kata_decode_step.restype = i32
@@ -404,6 +414,71 @@ def kata_chunked_forward_noalloc(q, k, v, C=64, out=None, state_out=None, z_out=
                                               _ptr(z_out), _stream_handle(stream, dev))
     if st != KATA_OK:
         raise KataError(st, "kata_chunked_forward_noalloc")
+    return out
+
+
+def kata_mg_chunked_forward_workspace_bytes(B, H, T, dk, dv, C, g, dtype_code) -> int:
+    return int(load_library().kata_mg_chunked_forward_workspace_bytes(B, H, T, dk, dv, C, g,
+                                                                      dtype_code))
+
+
+def kata_mg_chunked_forward(q, k, v, g=2, C=64, out=None, state_out=None, z_out=None,
+                            workspace=None, stream=None):
+    """KATA-Mg forward: g rank-one PSD factors on consecutive blocks of dk / g
+    coordinates, weight sum_m (q^(m).k^(m))^2.  Arguments as
+    kata_chunked_forward; the exported state holds zeros across factors."""
+    import torch
+
+    lib = load_library()
+    B, H, T, dk = q.shape
+    dev = q.device
+    dv = v.shape[-1]
+    _check(q, "q", (B, H, T, dk), device=dev)
+    _check(k, "k", (B, H, T, dk), q.dtype, device=dev)
+    _check(v, "v", (B, H, T, dv), q.dtype, device=dev)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", (B, H, T, dv), q.dtype, device=dev)
+    _check(state_out, "state_out", (B, H, dk * dk, dv), torch.float32, device=dev)
+    _check(z_out, "z_out", (B, H, dk, dk), torch.float32, device=dev)
+    need = lib.kata_mg_chunked_forward_workspace_bytes(B, H, T, dk, dv, int(C), int(g), code)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is not None and (not workspace.is_cuda or workspace.device != dev):
+        raise KataError(KATA_ERR_INVALID_ARG, f"workspace must be on {dev}")
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with _on_device(dev):
+        st = lib.kata_mg_chunked_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, T, dk, dv,
+                                         int(C), int(g), code, _ptr(state_out), _ptr(z_out),
+                                         _ptr(workspace), nbytes, _stream_handle(stream, dev))
+    if st != KATA_OK:
+        raise KataError(st, "kata_mg_chunked_forward")
+    return out
+
+
+def kata_mg_decode_step(q, k, v, state, z, g=2, out=None, stream=None):
+    """One KATA-Mg decode step, in place on the dense (state, z) of g factors."""
+    import torch
+
+    lib = load_library()
+    B, H, dk = q.shape
+    dev = q.device
+    dv = v.shape[-1]
+    _check(q, "q", (B, H, dk), device=dev)
+    _check(k, "k", (B, H, dk), q.dtype, device=dev)
+    _check(v, "v", (B, H, dv), q.dtype, device=dev)
+    code = _dtype_code(q)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _check(out, "out", (B, H, dv), q.dtype, device=dev)
+    _check(state, "state", (B, H, dk * dk, dv), torch.float32, device=dev)
+    _check(z, "z", (B, H, dk, dk), torch.float32, device=dev)
+    with _on_device(dev):
+        st = lib.kata_mg_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(state), _ptr(z),
+                                     B, H, dk, dv, int(g), code, _stream_handle(stream, dev))
+    if st != KATA_OK:
+        raise KataError(st, "kata_mg_decode_step")
     return out
 
 

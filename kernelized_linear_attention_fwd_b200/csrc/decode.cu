@@ -19,6 +19,11 @@
 // off the diagonal and 1 on it at readout), which holds the same information
 // in half the bytes, so the step moves half the data.  Pack and unpack
 // kernels convert between them.
+//
+// KATA-Mg with G factors (gist.science summary 2.3, "Variantes"), on the dense
+// layout: only rows (i, j) with i and j in one factor of dk / G coordinates
+// carry state; the others hold zeros and are neither read nor written, so
+// the step streams 1 / G of the bytes.  G = 1 is the single factor.
 #include <cooperative_groups.h>
 
 #include "kata_internal.cuh"
@@ -64,10 +69,12 @@ __device__ __forceinline__ void packed_ij(int r, int &i, int &j) {
 template <int P, bool PACKED>
 constexpr int min_ctas_per_sm() { return !PACKED && P == 1 ? 4 : 3; }
 
-template <int DK, int DV, int P, bool PACKED, typename TIn>
+template <int DK, int DV, int P, bool PACKED, typename TIn, int G = 1>
 __global__ void __launch_bounds__(kThreads, min_ctas_per_sm<P, PACKED>())
 decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
                    TIn *__restrict__ out, float *__restrict__ S, float *__restrict__ Z) {
+    static_assert(G == 1 || !PACKED, "factors only on the dense layout");
+    constexpr int FW = DK / G;  // coordinates per factor
     constexpr int ROWS = state_rows<DK, PACKED>();
     constexpr int V4 = DV / 4;               // float4 slots per state row
     constexpr int RPI = kThreads / V4;       // rows covered per pass
@@ -107,8 +114,12 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
     for (int row0 = row_base + rg; row0 < row_end; row0 += RPI * UNR) {
         float4 s[UNR];
 #pragma unroll
-        for (int u = 0; u < UNR; ++u)
-            if (row0 + u * RPI < row_end) s[u] = Sh[(long long)(row0 + u * RPI) * V4 + c4];
+        for (int u = 0; u < UNR; ++u) {
+            const int row = row0 + u * RPI;
+            // rows across factors (G > 1) hold zeros and stay so
+            const bool held = row < row_end && (G == 1 || (row / DK) / FW == (row % DK) / FW);
+            s[u] = held ? Sh[(long long)row * V4 + c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
             const int row = row0 + u * RPI;
@@ -122,7 +133,8 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
                 i = row / DK;
                 j = row % DK;
             }
-            const float f = sk[i] * sk[j];
+            // a row across factors stays zero: no update, so no readout share
+            const float f = (G == 1 || i / FW == j / FW) ? sk[i] * sk[j] : 0.f;
             const float w = (PACKED && i != j ? 2.f : 1.f) * (sq[i] * sq[j]);
             s[u].x = fmaf(f, vv.x, s[u].x);
             s[u].y = fmaf(f, vv.y, s[u].y);
@@ -134,8 +146,11 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
             a3 = fmaf(w, s[u].w, a3);
         }
 #pragma unroll
-        for (int u = 0; u < UNR; ++u)
-            if (row0 + u * RPI < row_end) Sh[(long long)(row0 + u * RPI) * V4 + c4] = s[u];
+        for (int u = 0; u < UNR; ++u) {
+            const int row = row0 + u * RPI;
+            if (row < row_end && (G == 1 || (row / DK) / FW == (row % DK) / FW))
+                Sh[(long long)row * V4 + c4] = s[u];
+        }
     }
 
     // normaliser: Z += k k^T, den = q^T Z q (this CTA's slice of the d^2 entries)
@@ -150,6 +165,7 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
         } else {
             i = x / DK;
             j = x % DK;
+            if (G > 1 && i / FW != j / FW) continue;
         }
         const float z = Zh[x] + sk[i] * sk[j];
         Zh[x] = z;
@@ -192,10 +208,10 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
     }
 }
 
-template <int DK, int DV, int P, bool PACKED, typename TIn>
+template <int DK, int DV, int P, bool PACKED, typename TIn, int G>
 cudaError_t launch_parts(int BH, const void *q, const void *k, const void *v, void *out, float *S,
                          float *Z, cudaStream_t st) {
-    auto kern = decode_step_kernel<DK, DV, P, PACKED, TIn>;
+    auto kern = decode_step_kernel<DK, DV, P, PACKED, TIn, G>;
     const TIn *qq = static_cast<const TIn *>(q), *kk = static_cast<const TIn *>(k),
               *vv = static_cast<const TIn *>(v);
     TIn *oo = static_cast<TIn *>(out);
@@ -219,7 +235,7 @@ cudaError_t launch_parts(int BH, const void *q, const void *k, const void *v, vo
     }
 }
 
-template <int DK, int DV, bool PACKED, typename TIn>
+template <int DK, int DV, bool PACKED, typename TIn, int G = 1>
 cudaError_t run(int BH, const void *q, const void *k, const void *v, void *out, float *S,
                 float *Z, cudaStream_t st) {
     // split heads over clusters while a CTA per head would leave SMs idle
@@ -227,22 +243,22 @@ cudaError_t run(int BH, const void *q, const void *k, const void *v, void *out, 
     int parts = 1;
     const int sms = tc::num_sms();
     while (parts < MP && (long long)BH * parts < sms) parts *= 2;
-    ProfScope ps(PACKED ? "decode_step_packed" : "decode_step", st);
+    ProfScope ps(PACKED ? "decode_step_packed" : G == 1 ? "decode_step" : "decode_step_mg", st);
     switch (parts) {
-        case 1: return launch_parts<DK, DV, 1, PACKED, TIn>(BH, q, k, v, out, S, Z, st);
-        case 2: return launch_parts<DK, DV, (MP >= 2 ? 2 : 1), PACKED, TIn>(BH, q, k, v, out, S, Z, st);
-        case 4: return launch_parts<DK, DV, (MP >= 4 ? 4 : 1), PACKED, TIn>(BH, q, k, v, out, S, Z, st);
-        default: return launch_parts<DK, DV, (MP >= 8 ? 8 : 1), PACKED, TIn>(BH, q, k, v, out, S, Z, st);
+        case 1: return launch_parts<DK, DV, 1, PACKED, TIn, G>(BH, q, k, v, out, S, Z, st);
+        case 2: return launch_parts<DK, DV, (MP >= 2 ? 2 : 1), PACKED, TIn, G>(BH, q, k, v, out, S, Z, st);
+        case 4: return launch_parts<DK, DV, (MP >= 4 ? 4 : 1), PACKED, TIn, G>(BH, q, k, v, out, S, Z, st);
+        default: return launch_parts<DK, DV, (MP >= 8 ? 8 : 1), PACKED, TIn, G>(BH, q, k, v, out, S, Z, st);
     }
 }
 
-template <bool PACKED, typename TIn>
+template <bool PACKED, typename TIn, int G = 1>
 cudaError_t dispatch(int BH, int dk, const void *q, const void *k, const void *v, void *out,
                      float *S, float *Z, cudaStream_t st) {
     switch (dk) {
-        case 16: return run<16, 16, PACKED, TIn>(BH, q, k, v, out, S, Z, st);
-        case 32: return run<32, 32, PACKED, TIn>(BH, q, k, v, out, S, Z, st);
-        case 64: return run<64, 64, PACKED, TIn>(BH, q, k, v, out, S, Z, st);
+        case 16: return run<16, 16, PACKED, TIn, G>(BH, q, k, v, out, S, Z, st);
+        case 32: return run<32, 32, PACKED, TIn, G>(BH, q, k, v, out, S, Z, st);
+        case 64: return run<64, 64, PACKED, TIn, G>(BH, q, k, v, out, S, Z, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -324,6 +340,16 @@ cudaError_t launch_decode(int B, int H, int dk, int dv, kata_dtype dtype, const 
                    : dispatch<true, float>(BH, dk, q, k, v, out, state, z, st);
     return dtype == KATA_BF16 ? dispatch<false, __nv_bfloat16>(BH, dk, q, k, v, out, state, z, st)
                               : dispatch<false, float>(BH, dk, q, k, v, out, state, z, st);
+}
+
+cudaError_t launch_decode_mg(int B, int H, int dk, int g, kata_dtype dtype, const void *q,
+                             const void *k, const void *v, void *out, float *state, float *z,
+                             cudaStream_t st) {
+    const int BH = B * H;
+    if (g == 1) return launch_decode(B, H, dk, dk, dtype, q, k, v, out, state, z, false, st);
+    if (g != 2) return cudaErrorInvalidValue;
+    return dtype == KATA_BF16 ? dispatch<false, __nv_bfloat16, 2>(BH, dk, q, k, v, out, state, z, st)
+                              : dispatch<false, float, 2>(BH, dk, q, k, v, out, state, z, st);
 }
 
 cudaError_t launch_state_convert(bool pack, int B, int H, int dk, const float *src_s,

@@ -119,6 +119,32 @@ kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dty
     return KATA_OK;
 }
 
+// KATA-Mg with g factors: g = 1 is the plain plan.  g = 2: bf16 heads of
+// d = 64 take the tensor-core path (its two-factor layout); every other head
+// size and dtype takes the fp32 CUDA-core path (the padded route would put
+// the factor boundary in the wrong place).  Other g: unsupported.
+kata_status make_plan_mg(int B, int H, int T, int dk, int dv, int C, int g, kata_dtype dtype,
+                         Plan &p) {
+    if (g == 1) return make_plan(B, H, T, dk, dv, C, dtype, p);
+    if (g < 1) return KATA_ERR_INVALID_ARG;
+    const kata_status s = make_plan(B, H, T, dk, dv, C, dtype, p, false);
+    if (s != KATA_OK) return s;
+    if (g != 2 || dk % g != 0) return KATA_ERR_UNSUPPORTED;
+    p.g = g;
+    p.R = packed_rows_g(dk, g);
+    if (p.path == Path::kTensorCore) {
+        tc::plan_tc_workspace(p);
+        return KATA_OK;
+    }
+    const size_t E = (size_t)p.R * (dv + 1);
+    p.ws_seg_state = 0;
+    p.ws_total = align_up((size_t)p.BH * p.n_seg * E * sizeof(float));
+    p.ws_extra = p.ws_total + align_up((size_t)p.BH * E * sizeof(float));
+    p.ws_aux = 0;
+    p.ws_bytes = p.ws_extra;
+    return KATA_OK;
+}
+
 // The quadratic form is the chunked plan with one segment spanning the whole
 // sequence: no state is built, scanned or stored, so no workspace is used.
 kata_status make_quadratic_plan(int B, int H, int T, int dk, int dv, kata_dtype dtype, Plan &p) {
@@ -189,11 +215,12 @@ kata_status check_state_out(const Plan &p, const float *state_out, const float *
     return KATA_OK;
 }
 
-// The decode step on either state layout.
+// The decode step on either state layout; g factors (KATA-Mg) on the dense one.
 kata_status decode_step(const void *q, const void *k, const void *v, void *out, float *state,
                         float *z, int B, int H, int dk, int dv, kata_dtype dtype, bool packed,
-                        kata_stream_t stream) {
-    if (B < 1 || H < 1 || dk < 1 || dv < 1) return KATA_ERR_INVALID_ARG;
+                        kata_stream_t stream, int g = 1) {
+    if (B < 1 || H < 1 || dk < 1 || dv < 1 || g < 1) return KATA_ERR_INVALID_ARG;
+    if (g > 2 || (packed && g != 1)) return KATA_ERR_UNSUPPORTED;
     if (dtype != KATA_F32 && dtype != KATA_BF16) return KATA_ERR_UNSUPPORTED;
     if (dk != dv || (dk != 16 && dk != 32 && dk != 64)) return KATA_ERR_UNSUPPORTED;
     if ((long long)B * H > 0x7fffffffLL / 8) return KATA_ERR_UNSUPPORTED;
@@ -209,7 +236,8 @@ kata_status decode_step(const void *q, const void *k, const void *v, void *out, 
         return KATA_ERR_INVALID_ARG;
     if (!device_ptrs_ok({q, k, v, out, state, z})) return KATA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const cudaError_t e = launch_decode(B, H, dk, dv, dtype, q, k, v, out, state, z, packed, st);
+    const cudaError_t e = g == 1 ? launch_decode(B, H, dk, dv, dtype, q, k, v, out, state, z, packed, st)
+                                 : launch_decode_mg(B, H, dk, g, dtype, q, k, v, out, state, z, st);
     return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
 }
 
@@ -273,6 +301,34 @@ kata_status kata_chunked_forward(const void *q, const void *k, const void *v, vo
                                  size_t workspace_bytes, kata_stream_t stream) {
     Plan p;
     const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p);
+    if (ps != KATA_OK) return ps;
+    const kata_status io = kata::check_forward_io(p, q, k, v, out);
+    if (io != KATA_OK) return io;
+    const kata_status so = kata::check_state_out(p, state_out, z_out, q, k, v, false);
+    if (so != KATA_OK) return so;
+    const kata_status ws = kata::check_workspace(p, workspace, workspace_bytes);
+    if (ws != KATA_OK) return ws;
+    if (!kata::device_ptrs_ok({q, k, v, out, state_out, z_out, p.ws_bytes ? workspace : nullptr}))
+        return KATA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e =
+        kata::launch_forward(p, q, k, v, out, state_out, z_out, kata::InitState{}, workspace, st);
+    return e == cudaSuccess ? KATA_OK : KATA_ERR_CUDA;
+}
+
+size_t kata_mg_chunked_forward_workspace_bytes(int B, int H, int T, int dk, int dv, int C, int g,
+                                               kata_dtype dtype) {
+    Plan p;
+    if (kata::make_plan_mg(B, H, T, dk, dv, C, g, dtype, p) != KATA_OK) return 0;
+    return p.ws_bytes;
+}
+
+kata_status kata_mg_chunked_forward(const void *q, const void *k, const void *v, void *out, int B,
+                                    int H, int T, int dk, int dv, int C, int g, kata_dtype dtype,
+                                    float *state_out, float *z_out, void *workspace,
+                                    size_t workspace_bytes, kata_stream_t stream) {
+    Plan p;
+    const kata_status ps = kata::make_plan_mg(B, H, T, dk, dv, C, g, dtype, p);
     if (ps != KATA_OK) return ps;
     const kata_status io = kata::check_forward_io(p, q, k, v, out);
     if (io != KATA_OK) return io;
@@ -378,6 +434,12 @@ kata_status kata_decode_step(const void *q, const void *k, const void *v, void *
                              float *state, float *z, int B, int H, int dk, int dv,
                              kata_dtype dtype, kata_stream_t stream) {
     return kata::decode_step(q, k, v, out, state, z, B, H, dk, dv, dtype, false, stream);
+}
+
+kata_status kata_mg_decode_step(const void *q, const void *k, const void *v, void *out,
+                                float *state, float *z, int B, int H, int dk, int dv, int g,
+                                kata_dtype dtype, kata_stream_t stream) {
+    return kata::decode_step(q, k, v, out, state, z, B, H, dk, dv, dtype, false, stream, g);
 }
 
 kata_status kata_decode_step_packed(const void *q, const void *k, const void *v, void *out,

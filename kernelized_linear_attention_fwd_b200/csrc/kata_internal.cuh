@@ -36,6 +36,26 @@ __host__ __device__ inline void packed_row_ij(int d, int r, int &i, int &j) {
     j = a + r;
 }
 
+// KATA-Mg with G factors of P = DK / G coordinates each: only pairs (i, j)
+// inside one factor carry state.  The packed rows are the G factors' own
+// packed rows one after the other: row r = f * Rp + r', Rp = P (P + 1) / 2,
+// is the pair (f P + i', f P + j') of the factor's row r' = (i', j').  G = 1
+// is the layout above.
+__host__ __device__ constexpr int packed_rows_g(int d, int G) { return G * packed_rows(d / G); }
+
+__host__ __device__ inline void packed_row_ij_g(int d, int G, int r, int &i, int &j) {
+    const int P = d / G, Rp = packed_rows(P), f = r / Rp;
+    packed_row_ij(P, r - f * Rp, i, j);
+    i += f * P;
+    j += f * P;
+}
+
+// Packed row of the pair (i, j), i <= j, both in one factor.
+__host__ __device__ inline int packed_row_index_g(int d, int G, int i, int j) {
+    const int P = d / G, f = i / P;
+    return f * packed_rows(P) + packed_row_start(P, i - f * P) + (j - i);
+}
+
 // ---------------------------------------------------------------------------
 // Forward plan: segment length, number of segments, workspace layout.
 // ---------------------------------------------------------------------------
@@ -50,6 +70,7 @@ struct Plan {
     int L;      // segment length (tokens), a multiple of C and of 128; T in the quadratic plan
     int n_seg;  // ceil(T / L)
     int R;      // packed feature rows
+    int g = 1;  // rank-one PSD factors per head (KATA-Mg; 1 = the single factor)
     Path path;
     // workspace (bytes from the base, all 256-byte aligned)
     size_t ws_seg_state;  // fp32 per-segment states, exclusive prefix after the scan
@@ -156,6 +177,11 @@ cudaError_t launch_padded_forward(const Plan &p, const void *q, const void *k, c
 cudaError_t launch_decode(int B, int H, int dk, int dv, kata_dtype dtype, const void *q,
                           const void *k, const void *v, void *out, float *state, float *z,
                           bool packed, cudaStream_t st);
+// The decode step of KATA-Mg with g factors on the dense layout (g = 1: the
+// dense step above).
+cudaError_t launch_decode_mg(int B, int H, int dk, int g, kata_dtype dtype, const void *q,
+                             const void *k, const void *v, void *out, float *state, float *z,
+                             cudaStream_t st);
 // Dense <-> packed state conversion (pack: dense -> packed).
 cudaError_t launch_state_convert(bool pack, int B, int H, int dk, const float *src_s,
                                  const float *src_z, float *dst_s, float *dst_z, cudaStream_t st);

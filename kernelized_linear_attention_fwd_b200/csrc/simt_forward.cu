@@ -14,7 +14,10 @@
 //                       tile's own segment, then the division (summary 2.1)
 //   4. state_expand     packed total -> dense [dk*dk, dv] state and [dk, dk] Z
 //
-// All arithmetic is fp32.
+// All arithmetic is fp32.  G factors (KATA-Mg, gist.science summary 2.3
+// "Variantes"): each factor is its own block of dk / G coordinates, only pairs
+// inside a factor carry state, and the intra weight is the sum over factors of
+// the squared block inner products.  G = 1 is the single-factor form.
 #include "kata_internal.cuh"
 
 namespace kata {
@@ -27,11 +30,11 @@ constexpr int kRowB = 32;   // state rows per inter step in seg_read
 // 1. Per-segment state increments.
 // grid.x = row-block + nrb * (segment + n_build * bh); block 256 = 32 rows x 8 e-groups
 // ---------------------------------------------------------------------------
-template <int DK, int DV, typename TIn>
+template <int DK, int DV, int G, typename TIn>
 __global__ void __launch_bounds__(256)
 seg_state_build(const TIn *__restrict__ k, const TIn *__restrict__ v, float *__restrict__ seg_state,
                 int T, int L, int n_seg, int n_build) {
-    constexpr int R = packed_rows(DK);
+    constexpr int R = packed_rows_g(DK, G);
     constexpr long long E = (long long)R * (DV + 1);
     constexpr int EG = DV / 8;
     constexpr int NRB = (R + 31) / 32;
@@ -48,7 +51,7 @@ seg_state_build(const TIn *__restrict__ k, const TIn *__restrict__ v, float *__r
     const int r = rb * 32 + lr;
     const bool live = r < R;
     int i = 0, j = 0;
-    if (live) packed_row_ij(DK, r, i, j);
+    if (live) packed_row_ij_g(DK, G, r, i, j);
 
     float acc[EG];
 #pragma unroll
@@ -97,7 +100,7 @@ seg_state_build(const TIn *__restrict__ k, const TIn *__restrict__ v, float *__r
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 seg_scan(float *__restrict__ seg_state, float *__restrict__ total, long long E, int n_seg,
-         int n_valid, int dk, int dv, const float *__restrict__ init_s,
+         int n_valid, int dk, int dv, int g, const float *__restrict__ init_s,
          const float *__restrict__ init_z, int n_in, long long s_stride, long long z_stride) {
     __shared__ float tile[32][33];
     const int lane = threadIdx.x, w = threadIdx.y;
@@ -114,7 +117,7 @@ seg_scan(float *__restrict__ seg_state, float *__restrict__ total, long long E, 
         if (e >= E) continue;
         const bool z_part = e >= R * dv;
         int i, j;
-        packed_row_ij(dk, (int)(z_part ? e - R * dv : e / dv), i, j);
+        packed_row_ij_g(dk, g, (int)(z_part ? e - R * dv : e / dv), i, j);
         for (int n = 0; n < n_in; ++n)
             carry[cc] += z_part ? init_z[n * z_stride + (bh * dk + i) * dk + j]
                                 : init_s[n * s_stride + ((bh * dk + i) * dk + j) * dv + e % dv];
@@ -177,12 +180,12 @@ struct ReadSmem {
     static constexpr size_t kBytes = kFloats * sizeof(float) + packed_rows(DK) * sizeof(unsigned short);
 };
 
-template <int DK, int DV, typename TIn>
+template <int DK, int DV, int G, typename TIn>
 __global__ void __launch_bounds__(256)
 seg_read(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
          TIn *__restrict__ out, const float *__restrict__ seg_state, int T, int L, int n_seg,
          bool has_init) {
-    constexpr int R = packed_rows(DK);
+    constexpr int R = packed_rows_g(DK, G);
     constexpr long long E = (long long)R * (DV + 1);
     constexpr int TE = DV / 16;
     using SM = ReadSmem<DK, DV>;
@@ -218,7 +221,7 @@ seg_read(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__rest
     }
     for (int r = tid; r < R; r += 256) {
         int i, j;
-        packed_row_ij(DK, r, i, j);
+        packed_row_ij_g(DK, G, r, i, j);
         sij[r] = (unsigned short)(i | (j << 8));
     }
     float num[4][TE], den[4];
@@ -284,10 +287,15 @@ seg_read(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__rest
         __syncthreads();
         for (int x = tid; x < kTok * kTok; x += 256) {
             const int qq = x / kTok, s = x % kTok;
-            float dot = 0.f;
+            float w = 0.f;
 #pragma unroll
-            for (int c = 0; c < DK; ++c) dot = fmaf(sq[qq * (DK + 1) + c], sk[s * (DK + 1) + c], dot);
-            float w = dot * dot;
+            for (int f = 0; f < G; ++f) {  // one squared inner product per factor
+                float dot = 0.f;
+#pragma unroll
+                for (int c = f * (DK / G); c < (f + 1) * (DK / G); ++c)
+                    dot = fmaf(sq[qq * (DK + 1) + c], sk[s * (DK + 1) + c], dot);
+                w = fmaf(dot, dot, w);
+            }
             if (k0 + s > t0 + qq || k0 + s >= kend) w = 0.f;
             sp[qq * (kTok + 1) + s] = w;
         }
@@ -323,11 +331,11 @@ seg_read(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__rest
 // ---------------------------------------------------------------------------
 // 4. Packed total -> dense state [dk*dk, dv] and Z [dk, dk].
 // ---------------------------------------------------------------------------
-template <int DK, int DV>
+template <int DK, int DV, int G>
 __global__ void __launch_bounds__(256)
 state_expand(const float *__restrict__ total, long long stride_bh, float *__restrict__ state_out,
              float *__restrict__ z_out, long long BH) {
-    constexpr int R = packed_rows(DK);
+    constexpr int R = packed_rows_g(DK, G), P = DK / G;
     const long long per = (long long)DK * DK * DV + DK * DK;
     const long long idx = (long long)blockIdx.x * 256 + threadIdx.x;
     if (idx >= per * BH) return;
@@ -338,21 +346,22 @@ state_expand(const float *__restrict__ total, long long stride_bh, float *__rest
         const int row = (int)(x / DV), e = (int)(x % DV);
         int i = row / DK, j = row % DK;
         if (i > j) { const int t = i; i = j; j = t; }
-        const int r = packed_row_start(DK, i) + (j - i);
-        state_out[bh * DK * DK * DV + x] = src[(long long)r * DV + e];
+        // pairs across factors carry no state
+        state_out[bh * DK * DK * DV + x] =
+            i / P == j / P ? src[(long long)packed_row_index_g(DK, G, i, j) * DV + e] : 0.f;
     } else {
         x -= (long long)DK * DK * DV;
         int i = (int)(x / DK), j = (int)(x % DK);
         if (i > j) { const int t = i; i = j; j = t; }
-        const int r = packed_row_start(DK, i) + (j - i);
-        z_out[bh * DK * DK + x] = src[(long long)R * DV + r];
+        z_out[bh * DK * DK + x] =
+            i / P == j / P ? src[(long long)R * DV + packed_row_index_g(DK, G, i, j)] : 0.f;
     }
 }
 
-template <int DK, int DV, typename TIn>
+template <int DK, int DV, int G, typename TIn>
 cudaError_t run(const Plan &p, const TIn *q, const TIn *k, const TIn *v, TIn *out,
                 float *state_out, float *z_out, const InitState &init, void *ws, cudaStream_t st) {
-    constexpr int R = packed_rows(DK);
+    constexpr int R = packed_rows_g(DK, G);
     constexpr long long E = (long long)R * (DV + 1);
     const long long BH = p.BH;
     // no workspace (the quadratic plan): no state is built, scanned or read
@@ -370,32 +379,32 @@ cudaError_t run(const Plan &p, const TIn *q, const TIn *k, const TIn *v, TIn *ou
     if (n_build > 0) {
         const long long grid = (long long)((R + 31) / 32) * n_build * BH;
         ProfScope ps("simt_seg_state_build", st);
-        seg_state_build<DK, DV, TIn><<<(unsigned)grid, 256, 0, st>>>(k, v, seg, p.T, p.L, p.n_seg,
-                                                                     n_build);
+        seg_state_build<DK, DV, G, TIn><<<(unsigned)grid, 256, 0, st>>>(k, v, seg, p.T, p.L,
+                                                                        p.n_seg, n_build);
     }
     if (scan) {
         const long long grid = ((E + 31) / 32) * BH;
         ProfScope ps("seg_scan", st);
         seg_scan<<<(unsigned)grid, dim3(32, 8), 0, st>>>(seg, want_state ? total : nullptr, E,
-                                                         p.n_seg, n_build, DK, DV, init.s, init.z,
+                                                         p.n_seg, n_build, DK, DV, G, init.s, init.z,
                                                          init.n, init.s_stride, init.z_stride);
     }
     if (readout) {
         using SM = ReadSmem<DK, DV>;
-        cudaError_t e = smem_opt_in_once<seg_read<DK, DV, TIn>>((int)SM::kBytes);
+        cudaError_t e = smem_opt_in_once<seg_read<DK, DV, G, TIn>>((int)SM::kBytes);
         if (e != cudaSuccess) return e;
         const long long grid = (long long)((p.T + kTok - 1) / kTok) * BH;
         ProfScope ps("simt_seg_read", st);
-        seg_read<DK, DV, TIn><<<(unsigned)grid, 256, SM::kBytes, st>>>(q, k, v, out, seg, p.T,
-                                                                        p.L, p.n_seg, has_init);
+        seg_read<DK, DV, G, TIn><<<(unsigned)grid, 256, SM::kBytes, st>>>(q, k, v, out, seg, p.T,
+                                                                           p.L, p.n_seg, has_init);
     }
     if (want_state) {
         const float *src = scan ? total : seg;
         const long long stride = scan ? E : E * p.n_seg;
         const long long n = ((long long)DK * DK * DV + DK * DK) * BH;
         ProfScope ps("state_expand", st);
-        state_expand<DK, DV><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, stride, state_out,
-                                                                          z_out, BH);
+        state_expand<DK, DV, G><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, stride, state_out,
+                                                                             z_out, BH);
     }
     return cudaGetLastError();
 }
@@ -407,10 +416,14 @@ cudaError_t dispatch(const Plan &p, const void *q, const void *k, const void *v,
     const TIn *K = static_cast<const TIn *>(k);
     const TIn *V = static_cast<const TIn *>(v);
     TIn *O = static_cast<TIn *>(out);
-    switch (p.dk) {
-        case 16: return run<16, 16, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
-        case 32: return run<32, 32, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
-        case 64: return run<64, 64, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
+    const int key = p.dk * 4 + p.g;
+    switch (key) {
+        case 16 * 4 + 1: return run<16, 16, 1, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
+        case 32 * 4 + 1: return run<32, 32, 1, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
+        case 64 * 4 + 1: return run<64, 64, 1, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
+        case 16 * 4 + 2: return run<16, 16, 2, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
+        case 32 * 4 + 2: return run<32, 32, 2, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
+        case 64 * 4 + 2: return run<64, 64, 2, TIn>(p, Q, K, V, O, so, zo, init, ws, st);
         default: return cudaErrorInvalidValue;
     }
 }

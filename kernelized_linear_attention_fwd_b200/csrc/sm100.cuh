@@ -321,6 +321,12 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+// a * b + c on both halves, one rounding.
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
 __device__ __forceinline__ float f32x2_lo(uint64_t a) { return __uint_as_float(static_cast<uint32_t>(a)); }
 __device__ __forceinline__ float f32x2_hi(uint64_t a) { return __uint_as_float(static_cast<uint32_t>(a >> 32)); }
 // Both halves rounded to bf16 (round to nearest even), low half first.

@@ -32,7 +32,8 @@ namespace {
 
 using namespace kata::sm100;
 
-constexpr long long kBf16PerSeg = (long long)kBf16Rows * kD;  // 147,456 bf16
+// bf16 prefix elements per (head, segment): the state rows, then Z hi and lo
+KATA_HD constexpr long long bf16_per_seg(int G) { return (long long)bf16_rows(G) * kD; }
 
 // ---------------------------------------------------------------------------
 // Exclusive prefix over segments (the associative scan across chunk states)
@@ -48,7 +49,9 @@ constexpr long long kBf16PerSeg = (long long)kBf16Rows * kD;  // 147,456 bf16
 // (fp32) or 8-byte (bf16) vector per lane.  RUN is the smallest of 2, 4, 8,
 // 16 whose pass covers every segment (at most 16): with few segments a short
 // run keeps the registers, and so the blocks resident per SM, that the
-// latency of these short blocks needs.
+// latency of these short blocks needs.  G factors (KATA-Mg): the layout with
+// G factors; the dense Z prefix then also gets zeros at the pairs across
+// factors, which the readout's q^T Z q must not see.
 // grid.x = element-block + n_eb * bh; block 256.
 // ---------------------------------------------------------------------------
 constexpr int kScanWarps = 8;
@@ -57,48 +60,106 @@ __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
     return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
 
-template <int RUN>
+// One thread's 4 consecutive elements of a (head, segment) state: where they
+// sit (state rows or packed normaliser rows, and the pairs of the latter).
+template <int G>
+struct ScanLane {
+    long long e0;
+    bool z_part;
+    int zr;
+    int zi[4], zj[4];
+    __device__ __forceinline__ ScanLane(long long e) : e0(e) {
+        z_part = e0 >= z_packed0(G);
+        zr = z_part ? (int)(e0 - z_packed0(G)) : 0;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const PairIJ pij = row_ij_g(G, zr + x);
+            zi[x] = pij.i;
+            zj[x] = pij.j;
+        }
+    }
+
+    // The initial state of these 4 packed elements: the sum of n_in dense states.
+    __device__ __forceinline__ float4 init(long long bh, const float *init_s, const float *init_z,
+                                           int n_in, long long s_stride, long long z_stride) const {
+        float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int n = 0; n < n_in; ++n) {
+            if (!z_part) {
+                const PairIJ pij = row_ij_g(G, (int)(e0 / kD));
+                if (pij.i <= pij.j)
+                    carry = f4add(carry, *reinterpret_cast<const float4 *>(
+                                             init_s + n * s_stride +
+                                             ((bh * kD + pij.i) * kD + pij.j) * kD + e0 % kD));
+            } else {
+                const float *zn = init_z + n * z_stride + bh * kD * kD;
+                float zv[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) zv[x] = zi[x] <= zj[x] ? zn[zi[x] * kD + zj[x]] : 0.f;
+                carry = f4add(carry, make_float4(zv[0], zv[1], zv[2], zv[3]));
+            }
+        }
+        return carry;
+    }
+
+    // Writes the prefix p of these elements into one segment's bf16 prefix dst.
+    __device__ __forceinline__ void write(__nv_bfloat16 *dst, float4 p, int lane) const {
+        if (!z_part) {
+            uint2 o;
+            o.x = pack_bf16x2(p.x, p.y);
+            o.y = pack_bf16x2(p.z, p.w);
+            *reinterpret_cast<uint2 *>(dst + e0) = o;
+            return;
+        }
+        // dense Z[i][j] and Z[j][i] as hi + lo bf16
+        const float pv[4] = {p.x, p.y, p.z, p.w};
+        __nv_bfloat16 *zh = dst + (long long)zhi_row0(G) * kD;
+        __nv_bfloat16 *zl = dst + (long long)zlo_row0(G) * kD;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            if (zi[x] > zj[x]) continue;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(pv[x]);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(pv[x] - __bfloat162float(hi));
+            zh[zi[x] * kD + zj[x]] = hi;
+            zl[zi[x] * kD + zj[x]] = lo;
+            zh[zj[x] * kD + zi[x]] = hi;
+            zl[zj[x] * kD + zi[x]] = lo;
+        }
+        if constexpr (G == 2) {
+            // zeros at the 32 x 32 pairs across the two factors (both halves of the
+            // symmetric Z), spread over the 32 lanes of the packed-z blocks
+            constexpr int kCross = 32 * 32, kThr = 32 * (state_rows(G) / 128);
+            const int zt = (zr / 128) * 32 + lane;
+            const __nv_bfloat16 z0 = __float2bfloat16_rn(0.f);
+#pragma unroll
+            for (int x = 0; x < (kCross + kThr - 1) / kThr; ++x) {
+                const int pi = zt + kThr * x;
+                if (pi >= kCross) break;
+                const int ci = pi / 32, cj = 32 + pi % 32;
+                zh[ci * kD + cj] = z0;
+                zl[ci * kD + cj] = z0;
+                zh[cj * kD + ci] = z0;
+                zl[cj * kD + ci] = z0;
+            }
+        }
+    }
+};
+
+template <int G, int RUN>
 __global__ void __launch_bounds__(256, RUN == 2 ? 5 : RUN == 4 ? 4 : 2)  // blocks per SM without spills
 tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ prefix,
             float *__restrict__ total, int n_seg, int n_valid, const float *__restrict__ init_s,
             const float *__restrict__ init_z, int n_in, long long s_stride, long long z_stride) {
     __shared__ float4 part[2][kScanWarps][32];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    constexpr long long E = kF32PerSeg;
+    constexpr long long E = f32_per_seg(G);
     constexpr long long n_eb = E / 128;
-    constexpr long long n_zb = kStateRows / 128;  // packed-z blocks (scattered writes): run them first
+    constexpr long long n_zb = state_rows(G) / 128;  // packed-z blocks (scattered writes): run them first
     const long long eb = (blockIdx.x % n_eb + (n_eb - n_zb)) % n_eb;
     const long long bh = blockIdx.x / n_eb;
-    const long long e0 = eb * 128 + 4 * lane;
-    const float *base = seg_state + bh * (long long)n_seg * E + e0;
-    __nv_bfloat16 *pbase = prefix ? prefix + bh * (long long)n_seg * kBf16PerSeg : nullptr;
-    // packed z: the thread's 4 rows and their pairs (i, j); padding rows have i > j
-    const bool z_part = e0 >= kZPacked0;
-    const int zr = z_part ? (int)(e0 - kZPacked0) : 0;
-    int zi[4], zj[4];
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-        const PairIJ pij = row_ij(zr + x);
-        zi[x] = pij.i;
-        zj[x] = pij.j;
-    }
-    // the initial state of these 4 packed elements: dense rows i * 64 + j
-    float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int n = 0; n < n_in; ++n) {
-        if (!z_part) {
-            const PairIJ pij = row_ij((int)(e0 / kD));
-            if (pij.i <= pij.j)
-                carry = f4add(carry, *reinterpret_cast<const float4 *>(
-                                         init_s + n * s_stride +
-                                         ((bh * kD + pij.i) * kD + pij.j) * kD + e0 % kD));
-        } else {
-            const float *zn = init_z + n * z_stride + bh * kD * kD;
-            float zv[4];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) zv[x] = zi[x] <= zj[x] ? zn[zi[x] * kD + zj[x]] : 0.f;
-            carry = f4add(carry, make_float4(zv[0], zv[1], zv[2], zv[3]));
-        }
-    }
+    const ScanLane<G> sl(eb * 128 + 4 * lane);
+    const float *base = seg_state + bh * (long long)n_seg * E + sl.e0;
+    __nv_bfloat16 *pbase = prefix ? prefix + bh * (long long)n_seg * bf16_per_seg(G) : nullptr;
+    float4 carry = sl.init(bh, init_s, init_z, n_in, s_stride, z_stride);
     const int g_first = n_in > 0 ? 0 : 1;  // without one, segment 0 has an empty prefix
 
     for (int g0 = 0; g0 < n_seg; g0 += kScanWarps * RUN) {
@@ -137,56 +198,77 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
         for (int i = 0; i < RUN; ++i) {
             const int g = gw + i;
             if (prefix == nullptr || g < g_first || g >= n_seg) continue;
-            const float4 p = f4add(v[i], off);
-            __nv_bfloat16 *dst = pbase + (long long)g * kBf16PerSeg;
-            if (!z_part) {
-                uint2 o;
-                o.x = pack_bf16x2(p.x, p.y);
-                o.y = pack_bf16x2(p.z, p.w);
-                *reinterpret_cast<uint2 *>(dst + e0) = o;
-            } else {
-                // dense Z[i][j] and Z[j][i] as hi + lo bf16
-                const float pv[4] = {p.x, p.y, p.z, p.w};
-                __nv_bfloat16 *zh = dst + (long long)kZHiRow0 * kD, *zl = dst + (long long)kZLoRow0 * kD;
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    if (zi[x] > zj[x]) continue;
-                    const __nv_bfloat16 hi = __float2bfloat16_rn(pv[x]);
-                    const __nv_bfloat16 lo = __float2bfloat16_rn(pv[x] - __bfloat162float(hi));
-                    zh[zi[x] * kD + zj[x]] = hi;
-                    zl[zi[x] * kD + zj[x]] = lo;
-                    zh[zj[x] * kD + zi[x]] = hi;
-                    zl[zj[x] * kD + zi[x]] = lo;
-                }
-            }
+            sl.write(pbase + (long long)g * bf16_per_seg(G), f4add(v[i], off), lane);
         }
     }
     if (total != nullptr && w == 0)
-        *reinterpret_cast<float4 *>(total + bh * E + e0) = carry;
+        *reinterpret_cast<float4 *>(total + bh * E + sl.e0) = carry;
+}
+
+// The same scan for short sequences (at most RUN <= 16 segments): one warp
+// per element block holds every segment in registers and scans them
+// sequentially, eight element blocks per CTA, with no cross-warp exchange and
+// no barrier.  A sequence of a few segments (a short prompt, one rank's block
+// of a sequence split over GPUs) otherwise runs thousands of blocks that each
+// move a few kilobytes between three barriers.
+// grid.x = ceil(n_eb * BH / 8); block 256.
+template <int G, int RUN>
+__global__ void __launch_bounds__(256, RUN <= 4 ? 4 : 2)
+tc_seg_scan_short(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ prefix,
+                  float *__restrict__ total, int n_seg, int n_valid, long long BH,
+                  const float *__restrict__ init_s, const float *__restrict__ init_z, int n_in,
+                  long long s_stride, long long z_stride) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    constexpr long long E = f32_per_seg(G);
+    constexpr long long n_eb = E / 128;
+    const long long gidx = (long long)blockIdx.x * kScanWarps + w;  // warp-uniform
+    if (gidx >= n_eb * BH) return;
+    const long long bh = gidx / n_eb, eb = gidx % n_eb;
+    const ScanLane<G> sl(eb * 128 + 4 * lane);
+    const float *base = seg_state + bh * (long long)n_seg * E + sl.e0;
+    __nv_bfloat16 *pbase = prefix ? prefix + bh * (long long)n_seg * bf16_per_seg(G) : nullptr;
+    float4 v[RUN];
+#pragma unroll
+    for (int i = 0; i < RUN; ++i)
+        v[i] = i < n_valid ? *reinterpret_cast<const float4 *>(base + (long long)i * E)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 run = sl.init(bh, init_s, init_z, n_in, s_stride, z_stride);
+    const int g_first = n_in > 0 ? 0 : 1;
+#pragma unroll
+    for (int i = 0; i < RUN; ++i) {
+        if (prefix != nullptr && i >= g_first && i < n_seg)
+            sl.write(pbase + (long long)i * bf16_per_seg(G), run, lane);
+        run = f4add(run, v[i]);
+    }
+    if (total != nullptr) *reinterpret_cast<float4 *>(total + bh * E + sl.e0) = run;
 }
 
 // ---------------------------------------------------------------------------
-// fp32 total (packed rows) -> dense state [64*64][64] and Z [64][64].
+// fp32 total (packed rows) -> dense state [D*D][D] and Z [D][D].  D < 64: the
+// heads were zero-padded to 64, and the leading D x D part is exported.  G
+// factors (KATA-Mg): pairs across factors are not in the layout and export 0.
+// D is a template parameter so the index arithmetic divides by constants.
 // ---------------------------------------------------------------------------
+template <int G, int D>
 __global__ void __launch_bounds__(256)
 tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__restrict__ state_out,
-                float *__restrict__ z_out, long long BH, int d) {
-    const long long d3 = (long long)d * d * d, per = d3 + (long long)d * d;
+                float *__restrict__ z_out, long long BH) {
+    constexpr long long d3 = (long long)D * D * D, per = d3 + (long long)D * D;
     const long long idx = (long long)blockIdx.x * 256 + threadIdx.x;
     if (idx >= per * BH) return;
     const long long bh = idx / per;
     long long x = idx % per;
     const float *src = total + bh * stride_bh;
     if (x < d3) {
-        const int row = (int)(x / d), e = (int)(x % d);
-        int i = row / d, j = row % d;
+        const int row = (int)(x / D), e = (int)(x % D);
+        int i = row / D, j = row % D;
         if (i > j) { const int t = i; i = j; j = t; }
-        state_out[bh * d3 + x] = src[(long long)row_index(i, j) * kD + e];
+        state_out[bh * d3 + x] = same_factor(G, i, j) ? src[(long long)row_index_g(G, i, j) * kD + e] : 0.f;
     } else {
         x -= d3;
-        int i = (int)(x / d), j = (int)(x % d);
+        int i = (int)(x / D), j = (int)(x % D);
         if (i > j) { const int t = i; i = j; j = t; }
-        z_out[bh * d * d + x] = src[kZPacked0 + row_index(i, j)];
+        z_out[bh * D * D + x] = same_factor(G, i, j) ? src[z_packed0(G) + row_index_g(G, i, j)] : 0.f;
     }
 }
 
@@ -220,7 +302,8 @@ constexpr int kCtaQ = kQT * kTiles;      // 256 queries per item
 constexpr int kKB = 128;                 // key/value block loaded by TMA
 constexpr int kSB = 64;                  // score block (MMA N of Q K^T)
 constexpr int kRKs = 8;                  // 16-row K-steps per inter stage (128 state rows)
-constexpr int kRStages = kStateRows / (16 * kRKs);  // 17
+// inter stages (128 state rows each): 17 for one factor, 9 for two
+KATA_HD constexpr int read_stages(int G) { return state_rows(G) / (16 * kRKs); }
 constexpr int kRRing = 3;                // inter A ring depth (tensor memory)
 constexpr int kRBRing = 4;               // inter B ring depth (state-prefix tiles, shared memory)
 constexpr int kRStageBytes = kRKs * 16 * 128;   // bf16 state-prefix rows per stage
@@ -242,8 +325,16 @@ constexpr int kSmAlloc = kSmBytes + 1024;
 constexpr uint32_t kTmO = 0;     // O[t]: 64 columns at 64 t
 constexpr uint32_t kTmA = 128;   // inter A slot s: 128 columns at 128 + 128 s (tile t at + 64 t)
 constexpr uint32_t kTmU = 384;   // U[t] = Q Z (before slot 2 is first written): 64 columns at 384 + 64 t
-constexpr uint32_t kTmS = 128;   // intra scores S[t][x]: 64 columns at 128 + 128 t + 64 x
+constexpr uint32_t kTmS = 128;   // intra scores of tile t: 128 columns at 128 + 128 t (see score_depth)
 constexpr uint32_t kTmP = 384;   // intra weights P[t][x] (bf16 pairs): 32 columns at 384 + 64 t + 32 x
+
+// Score buffers per tile in the intra phase.  One factor: two buffers of 64
+// columns (the scores of key block n + 1 are formed while block n is squared).
+// Two factors (KATA-Mg): one buffer of 128 columns holding both factors'
+// scores of a 64-key block side by side; the other tile's buffer gives the
+// overlap.  Either way a tile's score columns are 128 + 128 t .. + 127.
+template <int G>
+__host__ __device__ constexpr int score_depth() { return G == 1 ? 2 : 1; }
 
 struct ReadBars {
     // ostaged[b]: the output rows of the item in slot b are staged.  One per
@@ -328,9 +419,9 @@ __host__ __device__ constexpr int pair_weight(PairIJ p) { return p.i < p.j ? 2 :
 // 1 for i = j, 0 for padding rows.  The layout makes the word q_i (q_j,
 // q_j+1) or (q_i, q_i+1) q_j, one bf16x2 product; a common factor 2 is put on
 // the duplicated operand (exact), other weights multiply the product (exact).
-template <int R>
+template <int G, int R>
 __device__ __forceinline__ uint32_t gen_word(const uint32_t (&q2)[32]) {
-    constexpr PairIJ a = row_ij(R), b = row_ij(R + 1);
+    constexpr PairIJ a = row_ij_g(G, R), b = row_ij_g(G, R + 1);
     constexpr int c0 = pair_weight(a), c1 = pair_weight(b);
     static_assert((a.i == b.i && b.j == a.j + 1 && a.j % 2 == 0) ||
                       (a.j == b.j && b.i == a.i + 1 && a.i % 2 == 0),
@@ -350,25 +441,25 @@ __device__ __forceinline__ uint32_t gen_word(const uint32_t (&q2)[32]) {
 }
 
 // The 8 words of K-step K (state rows 16 K .. 16 K + 15).
-template <int K>
+template <int G, int K>
 __device__ __forceinline__ void gen_kstep(const uint32_t (&q2)[32], uint32_t *out) {
-    out[0] = gen_word<16 * K + 0>(q2);
-    out[1] = gen_word<16 * K + 2>(q2);
-    out[2] = gen_word<16 * K + 4>(q2);
-    out[3] = gen_word<16 * K + 6>(q2);
-    out[4] = gen_word<16 * K + 8>(q2);
-    out[5] = gen_word<16 * K + 10>(q2);
-    out[6] = gen_word<16 * K + 12>(q2);
-    out[7] = gen_word<16 * K + 14>(q2);
+    out[0] = gen_word<G, 16 * K + 0>(q2);
+    out[1] = gen_word<G, 16 * K + 2>(q2);
+    out[2] = gen_word<G, 16 * K + 4>(q2);
+    out[3] = gen_word<G, 16 * K + 6>(q2);
+    out[4] = gen_word<G, 16 * K + 8>(q2);
+    out[5] = gen_word<G, 16 * K + 10>(q2);
+    out[6] = gen_word<G, 16 * K + 12>(q2);
+    out[7] = gen_word<G, 16 * K + 14>(q2);
 }
 
 // First half (K-steps 0-3) of inter stage ST.
-template <int ST>
+template <int G, int ST>
 __device__ __forceinline__ void gen_stage_lo(const uint32_t (&q2)[32], uint32_t (&x)[32]) {
-    gen_kstep<kRKs * ST + 0>(q2, x);
-    gen_kstep<kRKs * ST + 1>(q2, x + 8);
-    gen_kstep<kRKs * ST + 2>(q2, x + 16);
-    gen_kstep<kRKs * ST + 3>(q2, x + 24);
+    gen_kstep<G, kRKs * ST + 0>(q2, x);
+    gen_kstep<G, kRKs * ST + 1>(q2, x + 8);
+    gen_kstep<G, kRKs * ST + 2>(q2, x + 16);
+    gen_kstep<G, kRKs * ST + 3>(q2, x + 24);
 }
 
 // Generates the inter stages of one item into the A ring, software-pipelined:
@@ -376,44 +467,41 @@ __device__ __forceinline__ void gen_stage_lo(const uint32_t (&q2)[32], uint32_t 
 // while the tensor-memory stores of stage ST are in flight, the first half of
 // stage ST + 1 is generated.  `g0` is the number of stages generated before
 // this item (ring slot and phase).
-template <int ST>
-struct GenLoop {
-    __device__ __forceinline__ static bool run(const uint32_t (&q2)[32], ReadBars &bars,
-                                               uint32_t ta_tile, int g0, volatile int *abort,
-                                               const uint32_t (&x)[32]) {
-        const int G = g0 + ST;
-        const int s = G % kRRing;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[s], ((G / kRRing) & 1) ^ 1, abort)))
-            return false;
-        tc_fence_after();
-        tmem_st32(ta_tile + 128 * s, x);
-        {
-            uint32_t y[16];
-            gen_kstep<kRKs * ST + 4>(q2, y);
-            gen_kstep<kRKs * ST + 5>(q2, y + 8);
-            tmem_st16(ta_tile + 128 * s + 32, y);
-        }
-        {
-            uint32_t y[16];
-            gen_kstep<kRKs * ST + 6>(q2, y);
-            gen_kstep<kRKs * ST + 7>(q2, y + 8);
-            tmem_st16(ta_tile + 128 * s + 48, y);
-        }
+template <int G, int ST>
+__device__ __forceinline__ bool gen_loop(const uint32_t (&q2)[32], ReadBars &bars, uint32_t ta_tile,
+                                         int g0, volatile int *abort, const uint32_t (&x)[32]) {
+    const int n = g0 + ST;
+    const int s = n % kRRing;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[s], ((n / kRRing) & 1) ^ 1, abort)))
+        return false;
+    tc_fence_after();
+    tmem_st32(ta_tile + 128 * s, x);
+    {
+        uint32_t y[16];
+        gen_kstep<G, kRKs * ST + 4>(q2, y);
+        gen_kstep<G, kRKs * ST + 5>(q2, y + 8);
+        tmem_st16(ta_tile + 128 * s + 32, y);
+    }
+    {
+        uint32_t y[16];
+        gen_kstep<G, kRKs * ST + 6>(q2, y);
+        gen_kstep<G, kRKs * ST + 7>(q2, y + 8);
+        tmem_st16(ta_tile + 128 * s + 48, y);
+    }
+    if constexpr (ST + 1 < read_stages(G)) {
         uint32_t xn[32];
-        if constexpr (ST + 1 < kRStages) gen_stage_lo<ST + 1>(q2, xn);
+        gen_stage_lo<G, ST + 1>(q2, xn);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars.afull[s]);
-        return GenLoop<ST + 1>::run(q2, bars, ta_tile, g0, abort, xn);
-    }
-};
-template <>
-struct GenLoop<kRStages> {
-    __device__ __forceinline__ static bool run(const uint32_t (&)[32], ReadBars &, uint32_t, int,
-                                               volatile int *, const uint32_t (&)[32]) {
+        return gen_loop<G, ST + 1>(q2, bars, ta_tile, g0, abort, xn);
+    } else {
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars.afull[s]);
         return true;
     }
-};
+}
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     const uint32_t s = smem_u32(p);
@@ -584,16 +672,18 @@ __device__ __forceinline__ bool build_item_gen(BuildBars &bars, const uint8_t *s
     return true;
 }
 
+template <int G>
 __device__ __forceinline__ void build_item_geom(int item, int n_build, int T, int L, int &c, int &g, int &bh,
                                                 int &s0, int &n_tt) {
-    c = item % kBuildItems;
-    const int rest = item / kBuildItems;
+    c = item % build_items(G);
+    const int rest = item / build_items(G);
     g = rest % n_build;
     bh = rest / n_build;
     s0 = g * L;
     n_tt = (min(L, T - s0) + kBTok - 1) / kBTok;
 }
 
+template <int G>
 __global__ void __launch_bounds__(kBuildThreads, 1)
 tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_v,
          const __grid_constant__ CUtensorMap tm_st, float *__restrict__ seg_state, int T, int L,
@@ -648,7 +738,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 int c, g, bh, s0, n_tt;
-                build_item_geom(item, n_build, T, L, c, g, bh, s0, n_tt);
+                build_item_geom<G>(item, n_build, T, L, c, g, bh, s0, n_tt);
                 for (int t = 0; t < n_tt; ++t, ++tt) {
                     const int b = tt % kBTileRing;
                     ok = mbar_wait(&bars.tempty[b], ((tt / kBTileRing) & 1) ^ 1, abort);
@@ -672,13 +762,13 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 int c, g, bh, s0, n_tt;
-                build_item_geom(item, n_build, T, L, c, g, bh, s0, n_tt);
-                const int nt = build_item_tiles(c);
+                build_item_geom<G>(item, n_build, T, L, c, g, bh, s0, n_tt);
+                const int nt = build_item_tiles(G, c);
                 for (int t = 0; t < n_tt && ok; ++t, ++tt) {
-                    const int G = 2 * tt + me;  // global stage: this issuer takes one half of each tile
-                    const int b = tt % kBTileRing, a = G % kBARing;
+                    const int gs = 2 * tt + me;  // global stage: this issuer takes one half of each tile
+                    const int b = tt % kBTileRing, a = gs % kBARing;
                     ok = mbar_wait(&bars.tfull[b], (tt / kBTileRing) & 1, abort) &&
-                         mbar_wait(&bars.afull[a], (G / kBARing) & 1, abort);
+                         mbar_wait(&bars.afull[a], (gs / kBARing) & 1, abort);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t vaddr = sbase + b * kBTileBytes + 8192 + 4096 * me;
@@ -707,12 +797,12 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             int j = 0;
             for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
                 int c, g, bh, s0, n_tt;
-                build_item_geom(item, n_build, T, L, c, g, bh, s0, n_tt);
+                build_item_geom<G>(item, n_build, T, L, c, g, bh, s0, n_tt);
                 if (!mbar_wait(&bars.staged, j & 1, abort)) break;
-                for (int m = 0; m < build_item_tiles(c); ++m)
+                for (int m = 0; m < build_item_tiles(G, c); ++m)
                     for (int h = 0; h < 2; ++h)
                         tma_store_3d(&tm_st, sm + kBStage + (2 * m + h) * kBStageBox, 32 * h,
-                                     128 * build_item_tile(c, m), bh * n_seg + g);
+                                     128 * build_item_tile(G, c, m), bh * n_seg + g);
                 bulk_commit_group();
                 bulk_wait_read_all();
                 mbar_arrive(&bars.sfree);
@@ -741,12 +831,12 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
             int c, g, bh, s0, n_tt;
-            build_item_geom(item, n_build, T, L, c, g, bh, s0, n_tt);
-            const int nt = build_item_tiles(c);
+            build_item_geom<G>(item, n_build, T, L, c, g, bh, s0, n_tt);
+            const int nt = build_item_tiles(G, c);
             int im[kBTiles], jcol = 0;
 #pragma unroll
             for (int m = 0; m < kBTiles; ++m) {
-                const PairIJ pij = row_ij(128 * build_item_tile(c, m < nt ? m : 0) + row);
+                const PairIJ pij = row_ij_g(G, 128 * build_item_tile(G, c, m < nt ? m : 0) + row);
                 im[m] = pij.i;
                 jcol = pij.j;  // the same for every tile of the item
             }
@@ -761,7 +851,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             // chunk c of row r at chunk c ^ (r % 8): conflict-free), its packed z
             // (column 64) straight to global memory.
             tc_fence_after();
-            float *zbase = seg_state + ((long long)bh * n_seg + g) * kF32PerSeg + kZPacked0;
+            float *zbase = seg_state + ((long long)bh * n_seg + g) * f32_per_seg(G) + z_packed0(G);
             for (int m = 2 * wg; m < 2 * wg + 2 && m < nt; ++m) {
                 uint32_t o[32];
 #pragma unroll
@@ -776,7 +866,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
                 }
                 tmem_ld8(tm + kBN * m + 64 + lane_base, o);
                 tmem_ld_wait();
-                zbase[128 * build_item_tile(c, m) + row] = __uint_as_float(o[0]);
+                zbase[128 * build_item_tile(G, c, m) + row] = __uint_as_float(o[0]);
             }
             fence_proxy_async_smem();
             mbar_arrive(&bars.staged);
@@ -791,6 +881,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
     if (tid == 0 && abort_flag) set_timeout_status(status);
 }
 
+template <int G>
 __global__ void __launch_bounds__(kReadThreads, 1)
 tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
@@ -804,6 +895,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
     uint8_t *sm = align1024(smem_raw);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const ReadSched sched = read_sched(n_items, n_ct, n_seg);
+    constexpr int kSDepth = score_depth<G>();
 
     if (tid == 0) {
         abort_flag = 0;
@@ -868,10 +960,10 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     if (it.inter)
                         for (int zz = 0; zz < 4; ++zz)  // Z hi rows 2560..2623, Z lo rows 2624..2687
                             tma_load_3d(slot + kTiles * 16384 + zz * 4096, &tm_s, &bars.qfull[qb], 0,
-                                        kZHiRow0 + 32 * zz, it.sidx);
+                                        zhi_row0(G) + 32 * zz, it.sidx);
                     ++n_q;
                 }
-                for (int st = 0; it.inter && st < kRStages && ok; ++st) {
+                for (int st = 0; it.inter && st < read_stages(G) && ok; ++st) {
                     const int s = n_bs % kRBRing;
                     ok = mbar_wait(&bars.bempty[s], ((n_bs / kRBRing) & 1) ^ 1, abort);
                     if (!ok) break;
@@ -939,11 +1031,11 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                         }
                         mma_commit(&bars.u);
                     }
-                    for (int st = me; st < kRStages && ok; st += 2) {
-                        const int G = n_inter * kRStages + st;
-                        const int s = G % kRRing, sb = G % kRBRing;
-                        ok = mbar_wait(&bars.bfull[sb], (G / kRBRing) & 1, abort) &&
-                             mbar_wait(&bars.afull[s], (G / kRRing) & 1, abort);
+                    for (int st = me; st < read_stages(G) && ok; st += 2) {
+                        const int ns = n_inter * read_stages(G) + st;
+                        const int s = ns % kRRing, sb = ns % kRBRing;
+                        ok = mbar_wait(&bars.bfull[sb], (ns / kRBRing) & 1, abort) &&
+                             mbar_wait(&bars.afull[s], (ns / kRRing) & 1, abort);
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t ta = tm + kTmA + 128 * s;
@@ -969,30 +1061,40 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                 const int gb[kTiles] = {g_b0, g_b1};
                 const int nbm = max(nb[0], nb[1]);
                 for (int b = 0; b < nbm && ok; ++b) {
-                    const int G = g_kv + b / 2;
-                    if ((b & 1) == 0) ok = mbar_wait(&bars.kvfull[G & 1], (G >> 1) & 1, abort);
+                    const int kvb = g_kv + b / 2;
+                    if ((b & 1) == 0) ok = mbar_wait(&bars.kvfull[kvb & 1], (kvb >> 1) & 1, abort);
                     if (me == 0) {
-                        // scores Q K^T into S[t][n % 2] (n = the tile's running block count),
-                        // once the squaring warps have read block n - 2 from that buffer,
-                        // which may belong to the previous item
+                        // scores Q K^T into score buffer n % kSDepth of tile t (n = the
+                        // tile's running block count), once the squaring warps have read
+                        // block n - kSDepth from that buffer, which may belong to the
+                        // previous item
 #pragma unroll
                         for (int t = 0; t < kTiles; ++t)
-                            if (ok && gb[t] + b >= 2 && b < nb[t]) {
-                                const int n = gb[t] + b - 2;
+                            if (ok && gb[t] + b >= kSDepth && b < nb[t]) {
+                                const int n = gb[t] + b - kSDepth;
                                 ok = mbar_wait(&bars.pfull[t][n & 1], (n >> 1) & 1, abort);
                             }
                         if (!ok) break;
                         tc_fence_after();
-                        const uint64_t dk = desc_add(dK, 16384 * (G & 1) + 8192 * (b & 1));
+                        const uint64_t dk = desc_add(dK, 16384 * (kvb & 1) + 8192 * (b & 1));
 #pragma unroll
                         for (int t = 0; t < kTiles; ++t) {
                             if (b >= nb[t]) continue;
-                            const int n = gb[t] + b, x = n & 1;
+                            const int n = gb[t] + b, x = n % kSDepth;
                             const uint64_t dQt = desc_sw128(slot + t * 16384, 16, 1024);
+                            if constexpr (G == 1) {
 #pragma unroll
-                            for (int ks = 0; ks < 4; ++ks)
-                                mma_ss(tm + kTmS + 128 * t + 64 * x, desc_add(dQt, 32 * ks), desc_add(dk, 32 * ks),
-                                       id_qk, ks > 0);
+                                for (int ks = 0; ks < 4; ++ks)
+                                    mma_ss(tm + kTmS + 128 * t + 64 * x, desc_add(dQt, 32 * ks),
+                                           desc_add(dk, 32 * ks), id_qk, ks > 0);
+                            } else {
+                                // one score per factor: coordinates 0-31 (K-steps 0, 1) into
+                                // columns 0-63 of the tile's buffer, 32-63 (K-steps 2, 3) into 64-127
+#pragma unroll
+                                for (int ks = 0; ks < 4; ++ks)
+                                    mma_ss(tm + kTmS + 128 * t + 64 * (ks / 2), desc_add(dQt, 32 * ks),
+                                           desc_add(dk, 32 * ks), id_qk, (ks & 1) != 0);
+                            }
                             mma_commit(&bars.sfull[t][x]);
                         }
                     } else {
@@ -1005,7 +1107,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                             }
                         if (!ok) break;
                         tc_fence_after();
-                        const uint64_t dv = desc_add(dV, 16384 * (G & 1) + 8192 * (b & 1));
+                        const uint64_t dv = desc_add(dV, 16384 * (kvb & 1) + 8192 * (b & 1));
 #pragma unroll
                         for (int t = 0; t < kTiles; ++t) {
                             if (b >= nb[t]) continue;
@@ -1018,7 +1120,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                         }
                     }
                     // this issuer is done with K/V block b / 2
-                    if ((b & 1) || b == nbm - 1) mma_commit(&bars.kvempty[G & 1]);
+                    if ((b & 1) || b == nbm - 1) mma_commit(&bars.kvempty[kvb & 1]);
                 }
                 if (!ok) break;
                 g_kv += it.n_kv;
@@ -1109,43 +1211,69 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     }
                 }
                 uint32_t x0[32];
-                gen_stage_lo<0>(q2, x0);
-                ok = GenLoop<0>::run(q2, bars, tA, n_inter * kRStages, abort, x0);
+                gen_stage_lo<G, 0>(q2, x0);
+                ok = gen_loop<G, 0>(q2, bars, tA, n_inter * read_stages(G), abort, x0);
                 if (!ok) break;
                 ++n_inter;
             }
             float l = 0.f;
             const int n_b = read_tile_blocks(it, t, T);
             for (int b = 0; b < n_b && ok; ++b) {
-                const int n = g_b + b, x = n & 1;
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfull[t][x], (n >> 1) & 1, abort));
+                const int n = g_b + b, x = n & 1, xs = n % kSDepth;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfull[t][xs], (n / kSDepth) & 1, abort));
                 if (!ok) break;
                 tc_fence_after();
-                uint32_t r[64], p[32];
-                tmem_ld32(tS + 64 * x, r);
-                tmem_ld32(tS + 64 * x + 32, r + 32);
-                tmem_ld_wait();
+                uint32_t p[32];
                 const int kbs = it.seg0 + kSB * b;
-                // weights w = s^2 (packed fp32 pairs), four partial row sums
+                // every key of the block precedes every query of the tile
+                const bool full = kbs + kSB - 1 <= tq0;
+                const int lim = tq - kbs;  // otherwise keys kbs + c with c <= lim are visible
+                // weights w (packed fp32 pairs), four partial row sums
                 uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-                if (kbs + kSB - 1 <= tq0) {  // every key of the block precedes every query of the tile
+                if constexpr (G == 1) {
+                    // w = s^2
+                    uint32_t r[64];
+                    tmem_ld32(tS + 64 * xs, r);
+                    tmem_ld32(tS + 64 * xs + 32, r + 32);
+                    tmem_ld_wait();
+                    if (full) {
 #pragma unroll
-                    for (int y = 0; y < 32; ++y) {
-                        const uint64_t s2 = f32x2_pack(r[2 * y], r[2 * y + 1]);
-                        const uint64_t w2 = f32x2_mul(s2, s2);
-                        acc[y & 3] = f32x2_add(acc[y & 3], w2);
-                        p[y] = f32x2_to_bf16x2(w2);
+                        for (int y = 0; y < 32; ++y) {
+                            const uint64_t s2 = f32x2_pack(r[2 * y], r[2 * y + 1]);
+                            const uint64_t w2 = f32x2_mul(s2, s2);
+                            acc[y & 3] = f32x2_add(acc[y & 3], w2);
+                            p[y] = f32x2_to_bf16x2(w2);
+                        }
+                    } else {
+#pragma unroll
+                        for (int y = 0; y < 32; ++y) {
+                            const uint32_t m0 = 2 * y <= lim ? r[2 * y] : 0u;
+                            const uint32_t m1 = 2 * y + 1 <= lim ? r[2 * y + 1] : 0u;
+                            const uint64_t s2 = f32x2_pack(m0, m1);
+                            const uint64_t w2 = f32x2_mul(s2, s2);
+                            acc[y & 3] = f32x2_add(acc[y & 3], w2);
+                            p[y] = f32x2_to_bf16x2(w2);
+                        }
                     }
                 } else {
-                    const int lim = tq - kbs;  // keys kbs + c with c <= lim are visible
+                    // w = a^2 + b^2, a and b the two factors' scores (columns 0-63 and
+                    // 64-127 of the tile's buffer), 32 keys at a time
 #pragma unroll
-                    for (int y = 0; y < 32; ++y) {
-                        const uint32_t m0 = 2 * y <= lim ? r[2 * y] : 0u;
-                        const uint32_t m1 = 2 * y + 1 <= lim ? r[2 * y + 1] : 0u;
-                        const uint64_t s2 = f32x2_pack(m0, m1);
-                        const uint64_t w2 = f32x2_mul(s2, s2);
-                        acc[y & 3] = f32x2_add(acc[y & 3], w2);
-                        p[y] = f32x2_to_bf16x2(w2);
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t ra[32], rb[32];
+                        tmem_ld32(tS + 32 * h, ra);
+                        tmem_ld32(tS + 64 + 32 * h, rb);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int y = 0; y < 16; ++y) {
+                            const int c = 32 * h + 2 * y;
+                            const bool v0 = full || c <= lim, v1 = full || c + 1 <= lim;
+                            const uint64_t a2 = f32x2_pack(v0 ? ra[2 * y] : 0u, v1 ? ra[2 * y + 1] : 0u);
+                            const uint64_t b2 = f32x2_pack(v0 ? rb[2 * y] : 0u, v1 ? rb[2 * y + 1] : 0u);
+                            const uint64_t w2 = f32x2_fma(b2, b2, f32x2_mul(a2, a2));
+                            acc[y & 3] = f32x2_add(acc[y & 3], w2);
+                            p[16 * h + y] = f32x2_to_bf16x2(w2);
+                        }
                     }
                 }
                 {
@@ -1206,58 +1334,41 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
     if (tid == 0 && abort_flag) set_timeout_status(status);
 }
 
+template <int G>
 bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const void *prefix, void *out,
                CUtensorMap *mq, CUtensorMap *mk, CUtensorMap *mv, CUtensorMap *ms, CUtensorMap *mo) {
     const uint64_t dqkv[3] = {(uint64_t)kD, (uint64_t)p.T, (uint64_t)p.BH};
     const uint64_t sqkv[2] = {(uint64_t)kD * 2, (uint64_t)p.T * kD * 2};
     const uint32_t bqkv[3] = {64, 128, 1};
-    const uint64_t ds[3] = {(uint64_t)kD, (uint64_t)kBf16Rows, (uint64_t)(p.BH * p.n_seg)};
-    const uint64_t ss[2] = {(uint64_t)kD * 2, (uint64_t)kBf16Rows * kD * 2};
+    const uint64_t ds[3] = {(uint64_t)kD, (uint64_t)bf16_rows(G), (uint64_t)(p.BH * p.n_seg)};
+    const uint64_t ss[2] = {(uint64_t)kD * 2, (uint64_t)bf16_rows(G) * kD * 2};
     const uint32_t bs[3] = {64, 32, 1};
     return make_tmap_bf16(mq, q, 3, dqkv, sqkv, bqkv) && make_tmap_bf16(mk, k, 3, dqkv, sqkv, bqkv) &&
            make_tmap_bf16(mv, v, 3, dqkv, sqkv, bqkv) &&
            make_tmap_bf16(ms, prefix ? prefix : q, 3, ds, ss, bs) && make_tmap_bf16(mo, out, 3, dqkv, sqkv, bqkv);
 }
 
-}  // namespace
-
-// Streaming multiprocessors of the current device (persistent grids).
-int num_sms() {
-    static std::mutex mu;
-    static int cache[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    std::lock_guard<std::mutex> lk(mu);
-    if (!cache[dev]) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cache[dev] = n;
+template <int G>
+cudaError_t launch_expand(const float *src, long long stride, float *state_out, float *z_out, long long BH,
+                          int d_out, cudaStream_t st) {
+    const long long n = ((long long)d_out * d_out * d_out + (long long)d_out * d_out) * BH;
+    const unsigned grid = (unsigned)((n + 255) / 256);
+    ProfScope ps(G == 1 ? "tc_state_expand" : "tc_state_expand_m2", st);
+    if (G == 2 && d_out != kD) return cudaErrorInvalidValue;
+    switch (d_out) {
+        case 16: tc_state_expand<G, 16><<<grid, 256, 0, st>>>(src, stride, state_out, z_out, BH); break;
+        case 32: tc_state_expand<G, 32><<<grid, 256, 0, st>>>(src, stride, state_out, z_out, BH); break;
+        case 64: tc_state_expand<G, 64><<<grid, 256, 0, st>>>(src, stride, state_out, z_out, BH); break;
+        default: return cudaErrorInvalidValue;
     }
-    return cache[dev];
+    return cudaSuccess;
 }
 
-// Workspace of the tensor-core path (bytes; 256-aligned parts):
-//   fp32 segment states  BH * n_seg * 2176 * 65 * 4   (state rows, then packed z)
-//   fp32 total           BH * 2176 * 65 * 4
-//   bf16 prefixes        BH * n_seg * 2304 * 64 * 2
-//   transposed keys      BH * 64 * T_pad * 2      (T_pad = T rounded up to 64)
-void plan_tc_workspace(Plan &p) {
-    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t seg = (size_t)p.BH * p.n_seg * kF32PerSeg * 4;
-    const size_t tot = (size_t)p.BH * kF32PerSeg * 4;
-    const size_t pre = (size_t)p.BH * p.n_seg * kBf16PerSeg * 2;
-    const size_t T_pad = (size_t)(p.T + 63) / 64 * 64;
-    const size_t kt = (size_t)p.BH * kD * T_pad * 2;
-    p.ws_seg_state = 0;
-    p.ws_total = up(seg);
-    p.ws_extra = p.ws_total + up(tot);
-    p.ws_aux = p.ws_extra + up(pre);
-    p.ws_bytes = p.ws_aux + up(kt);
-}
-
-cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
-                              float *state_out, float *z_out, const InitState &init, void *ws,
-                              cudaStream_t st, bool reuse_seg, int d_out) {
+// The forward with G factors (1: KATA-M1; 2: KATA-Mg with two factors).
+template <int G>
+cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, const void *v, void *out,
+                                float *state_out, float *z_out, const InitState &init, void *ws,
+                                cudaStream_t st, bool reuse_seg, int d_out) {
     // no workspace (the quadratic plan): no state is built, scanned or read
     char *w = static_cast<char *>(ws);
     float *seg = w ? reinterpret_cast<float *>(w + p.ws_seg_state) : nullptr;
@@ -1291,54 +1402,109 @@ cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const
         const uint64_t dqkv[3] = {(uint64_t)kD, (uint64_t)p.T, (uint64_t)BH};
         const uint64_t sqkv[2] = {(uint64_t)kD * 2, (uint64_t)p.T * kD * 2};
         const uint32_t b64[3] = {64, 64, 1};
-        const uint64_t dst[3] = {(uint64_t)kD, (uint64_t)kStateRows, (uint64_t)(BH * p.n_seg)};
-        const uint64_t sst[2] = {(uint64_t)kD * 4, (uint64_t)kF32PerSeg * 4};
+        const uint64_t dst[3] = {(uint64_t)kD, (uint64_t)state_rows(G), (uint64_t)(BH * p.n_seg)};
+        const uint64_t sst[2] = {(uint64_t)kD * 4, (uint64_t)f32_per_seg(G) * 4};
         const uint32_t bst[3] = {32, 128, 1};
         if (!make_tmap_bf16(&mkt, kt, 3, dkt, skt, bkt) || !make_tmap_bf16(&mvb, v, 3, dqkv, sqkv, b64) ||
             !make_tmap(&mst, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, seg, 3, dst, sst, bst))
             return cudaErrorInvalidValue;
-        cudaError_t e = smem_opt_in_once<tc_build>(kBSmAlloc);
+        cudaError_t e = smem_opt_in_once<tc_build<G>>(kBSmAlloc);
         if (e != cudaSuccess) return e;
-        const long long n_items = (long long)kBuildItems * n_build * BH;
+        const long long n_items = (long long)build_items(G) * n_build * BH;
         const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
-        ProfScope ps("tc_build", st);
-        tc_build<<<(unsigned)grid, kBuildThreads, kBSmAlloc, st>>>(mkt, mvb, mst, seg, p.T, p.L, p.n_seg,
-                                                                    n_build, (int)n_items, status);
+        ProfScope ps(G == 1 ? "tc_build" : "tc_build_m2", st);
+        tc_build<G><<<(unsigned)grid, kBuildThreads, kBSmAlloc, st>>>(mkt, mvb, mst, seg, p.T, p.L, p.n_seg,
+                                                                       n_build, (int)n_items, status);
     }
     if (scan) {
-        ProfScope ps("tc_seg_scan", st);
-        const long long grid = (kF32PerSeg / 128) * BH;
-        auto kern = p.n_seg <= 2 * kScanWarps ? tc_seg_scan<2>
-                    : p.n_seg <= 4 * kScanWarps ? tc_seg_scan<4>
-                    : p.n_seg <= 8 * kScanWarps ? tc_seg_scan<8>
-                                                : tc_seg_scan<16>;
-        kern<<<(unsigned)grid, 256, 0, st>>>(seg, readout ? prefix : nullptr,
-                                             want_state ? total : nullptr, p.n_seg, n_valid, init.s,
-                                             init.z, init.n, init.s_stride, init.z_stride);
+        ProfScope ps(G == 1 ? "tc_seg_scan" : "tc_seg_scan_m2", st);
+        __nv_bfloat16 *pre = readout ? prefix : nullptr;
+        float *tot = want_state ? total : nullptr;
+        if (p.n_seg <= 16) {
+            // few segments: one warp per element block (no cross-warp scan)
+            const long long grid = ((f32_per_seg(G) / 128) * BH + kScanWarps - 1) / kScanWarps;
+            auto kern = p.n_seg <= 4 ? tc_seg_scan_short<G, 4>
+                        : p.n_seg <= 8 ? tc_seg_scan_short<G, 8> : tc_seg_scan_short<G, 16>;
+            kern<<<(unsigned)grid, 256, 0, st>>>(seg, pre, tot, p.n_seg, n_valid, BH, init.s, init.z,
+                                                 init.n, init.s_stride, init.z_stride);
+        } else {
+            const long long grid = (f32_per_seg(G) / 128) * BH;
+            auto kern = p.n_seg <= 4 * kScanWarps ? tc_seg_scan<G, 4>
+                        : p.n_seg <= 8 * kScanWarps ? tc_seg_scan<G, 8>
+                                                    : tc_seg_scan<G, 16>;
+            kern<<<(unsigned)grid, 256, 0, st>>>(seg, pre, tot, p.n_seg, n_valid, init.s, init.z,
+                                                 init.n, init.s_stride, init.z_stride);
+        }
     }
     if (readout) {
         CUtensorMap mq, mk, mv, ms, mo;
-        if (!make_maps(p, q, k, v, prefix, out, &mq, &mk, &mv, &ms, &mo)) return cudaErrorInvalidValue;
-        cudaError_t e = smem_opt_in_once<tc_read>(kSmAlloc);
+        if (!make_maps<G>(p, q, k, v, prefix, out, &mq, &mk, &mv, &ms, &mo)) return cudaErrorInvalidValue;
+        cudaError_t e = smem_opt_in_once<tc_read<G>>(kSmAlloc);
         if (e != cudaSuccess) return e;
         const int n_ct = (p.T + kCtaQ - 1) / kCtaQ;
         const long long n_items = (long long)n_ct * BH;
         if (n_items >= 0x7fffffffLL - 4096) return cudaErrorInvalidValue;
         const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
-        ProfScope ps("tc_read", st);
-        tc_read<<<(unsigned)grid, kReadThreads, kSmAlloc, st>>>(
+        ProfScope ps(G == 1 ? "tc_read" : "tc_read_m2", st);
+        tc_read<G><<<(unsigned)grid, kReadThreads, kSmAlloc, st>>>(
             mq, mk, mv, ms, mo, p.T, p.L, p.n_seg, n_ct, (int)n_items, has_init, status);
     }
     if (want_state) {
         const float *src = scan ? total : seg;
-        const long long stride = scan ? kF32PerSeg : kF32PerSeg * p.n_seg;
+        const long long stride = scan ? f32_per_seg(G) : f32_per_seg(G) * p.n_seg;
         if (d_out < 1 || d_out > kD) return cudaErrorInvalidValue;
-        const long long n = ((long long)d_out * d_out * d_out + (long long)d_out * d_out) * BH;
-        ProfScope ps("tc_state_expand", st);
-        tc_state_expand<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(src, stride, state_out, z_out, BH,
-                                                                     d_out);
+        const cudaError_t e = launch_expand<G>(src, stride, state_out, z_out, BH, d_out, st);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
+}
+
+}  // namespace
+
+// Streaming multiprocessors of the current device (persistent grids).
+int num_sms() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// Workspace of the tensor-core path (bytes; 256-aligned parts), R = 2176 state
+// rows for one factor, 1152 for two (tc_layout.cuh):
+//   fp32 segment states  BH * n_seg * R * 65 * 4   (state rows, then packed z)
+//   fp32 total           BH * R * 65 * 4
+//   bf16 prefixes        BH * n_seg * (R + 128) * 64 * 2
+//   transposed keys      BH * 64 * T_pad * 2      (T_pad = T rounded up to 64)
+void plan_tc_workspace(Plan &p) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const int G = p.g;
+    const size_t seg = (size_t)p.BH * p.n_seg * f32_per_seg(G) * 4;
+    const size_t tot = (size_t)p.BH * f32_per_seg(G) * 4;
+    const size_t pre = (size_t)p.BH * p.n_seg * bf16_per_seg(G) * 2;
+    const size_t T_pad = (size_t)(p.T + 63) / 64 * 64;
+    const size_t kt = (size_t)p.BH * kD * T_pad * 2;
+    p.ws_seg_state = 0;
+    p.ws_total = up(seg);
+    p.ws_extra = p.ws_total + up(tot);
+    p.ws_aux = p.ws_extra + up(pre);
+    p.ws_bytes = p.ws_aux + up(kt);
+}
+
+cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
+                              float *state_out, float *z_out, const InitState &init, void *ws,
+                              cudaStream_t st, bool reuse_seg, int d_out) {
+    switch (p.g) {
+        case 1: return launch_tc_forward_g<1>(p, q, k, v, out, state_out, z_out, init, ws, st, reuse_seg, d_out);
+        case 2: return launch_tc_forward_g<2>(p, q, k, v, out, state_out, z_out, init, ws, st, reuse_seg, d_out);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace tc

@@ -101,5 +101,58 @@ KATA_HD constexpr int row_index(int i, int j) {
     return first ? 128 * (12 + m) + g : 128 * 16 + 4 * g + m;
 }
 
+// ---------------------------------------------------------------------------
+// KATA-Mg with g = 2 factors (coordinates 0-31 and 32-63, each its own
+// rank-one PSD factor): the state holds only the pairs (i, j), i <= j, inside
+// one factor, 2 x 32 * 33 / 2 = 1056 rows, in 9 tiles (1152 rows):
+//   tiles 0-3   the off-diagonal 16 x 16 blocks of the two factors, (0-15,
+//               16-31) and (32-47, 48-63), as half-strips: tile m, lane
+//               16 s + jj holds i = 4 s + m, j = 16 + jj for s < 4 and
+//               i = 32 + 4 (s - 4) + m, j = 48 + jj for s >= 4;
+//   tiles 4-8   the four diagonal 16 x 16 triangles, laid out as tiles 12-16
+//               of the single-factor layout.
+// The same properties hold: builder item 0 (tiles 0-3) and item 1 (tiles
+// 4-7) keep one j per lane across their 4 tiles, item 2 is tile 8, and every
+// 32-bit word of phi(q) is one bf16x2 product.
+// ---------------------------------------------------------------------------
+KATA_HD constexpr int state_tiles(int G) { return G == 1 ? kStateTiles : 9; }
+KATA_HD constexpr int state_rows(int G) { return 128 * state_tiles(G); }
+KATA_HD constexpr long long z_packed0(int G) { return (long long)state_rows(G) * kD; }
+KATA_HD constexpr long long f32_per_seg(int G) { return z_packed0(G) + state_rows(G); }
+KATA_HD constexpr int bf16_rows(int G) { return state_rows(G) + 2 * kD; }
+KATA_HD constexpr int zhi_row0(int G) { return state_rows(G); }
+KATA_HD constexpr int zlo_row0(int G) { return state_rows(G) + kD; }
+KATA_HD constexpr int build_items(int G) { return G == 1 ? kBuildItems : 3; }
+KATA_HD constexpr int build_item_tiles(int G, int c) { return c < build_items(G) - 1 ? 4 : 1; }
+KATA_HD constexpr int build_item_tile(int G, int c, int m) {
+    return c < build_items(G) - 1 ? 4 * c + m : state_tiles(G) - 1;
+}
+// Tiles of the g = 2 layout taken over from the single-factor layout.
+constexpr int kM2TileShift = 8;
+
+// (i, j) of state row r of the layout with G factors.
+KATA_HD constexpr PairIJ row_ij_g(int G, int r) {
+    if (G == 1) return row_ij(r);
+    const int tile = r / 128, lane = r % 128;
+    if (tile < 4) {
+        const int s = lane / 16, jj = lane % 16;
+        return s < 4 ? PairIJ{4 * s + tile, 16 + jj} : PairIJ{32 + 4 * (s - 4) + tile, 48 + jj};
+    }
+    return row_ij(r + 128 * kM2TileShift);
+}
+
+// Both coordinates in the same factor of G (a pair the layout holds).
+KATA_HD constexpr bool same_factor(int G, int i, int j) { return i / (kD / G) == j / (kD / G); }
+
+// State row of the pair (i, j), i <= j, same_factor(G, i, j), in the layout with G factors.
+KATA_HD constexpr int row_index_g(int G, int i, int j) {
+    if (G == 1) return row_index(i, j);
+    if (i / 16 < j / 16) {
+        const int f = i / 32, ii = i - 32 * f;
+        return 128 * (ii % 4) + 16 * (ii / 4 + 4 * f) + j % 16;
+    }
+    return row_index(i, j) - 128 * kM2TileShift;
+}
+
 }  // namespace tc
 }  // namespace kata

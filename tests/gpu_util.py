@@ -37,29 +37,39 @@ STATE_SIGMAS = 6.0
 U_BF16 = 2.0 ** -8
 
 
-def state_bounds(oracle_mod, k64, v64, dtype):
+def _state_fn(oracle_mod, g):
+    """The oracle's state of one factor (g = 1) or of KATA-Mg with g factors."""
+    if g == 1:
+        return oracle_mod.state
+    return lambda k, v: oracle_mod.state_mg(k, v, g)
+
+
+def state_bounds(oracle_mod, k64, v64, dtype, g=1):
     """Per-entry bounds (S, Z) of an exported state against the fp64 oracle's:
     the expected-error bound above for bf16, 2^-16 R1 for fp32."""
-    S1, Z1 = oracle_mod.state(np.abs(k64), np.abs(v64))
+    state = _state_fn(oracle_mod, g)
+    S1, Z1 = state(np.abs(k64), np.abs(v64))
     if dtype != "bf16":
         u = STATE_BOUND[dtype]
         return u * S1 + 1e-6, u * Z1 + 1e-6
-    S2, Z2 = oracle_mod.state(k64 * k64, v64 * v64)
+    S2, Z2 = state(k64 * k64, v64 * v64)
     c = STATE_SIGMAS * U_BF16 / np.sqrt(3.0)
     return (c * np.sqrt(S2) + 2.0 ** -16 * S1 + 1e-6,
             c * np.sqrt(Z2) + 2.0 ** -16 * Z1 + 1e-6)
 
 
-def assert_state_close(oracle_mod, Sg, Zg, k64, v64, dtype):
+def assert_state_close(oracle_mod, Sg, Zg, k64, v64, dtype, g=1):
     """Exported state (numpy S [..., d*d, dv], Z [..., d, d]) against the fp64
-    oracle's state of the same tokens: state_bounds, and the worst-case
-    STATE_BOUND as an outer check.  Returns the largest error / bound."""
-    S, Z = oracle_mod.state(k64, v64)
-    bS, bZ = state_bounds(oracle_mod, k64, v64, dtype)
+    oracle's state of the same tokens (g > 1: of KATA-Mg with g factors, zeros
+    across factors): state_bounds, and the worst-case STATE_BOUND as an outer
+    check.  Returns the largest error / bound."""
+    state = _state_fn(oracle_mod, g)
+    S, Z = state(k64, v64)
+    bS, bZ = state_bounds(oracle_mod, k64, v64, dtype, g)
     eS, eZ = np.abs(Sg - S), np.abs(Zg - Z)
     assert np.all(eS <= bS), f"state entry off by {np.max(eS / bS):.2f} x its bound"
     assert np.all(eZ <= bZ), f"Z entry off by {np.max(eZ / bZ):.2f} x its bound"
-    Sabs, Zabs = oracle_mod.state(np.abs(k64), np.abs(v64))
+    Sabs, Zabs = state(np.abs(k64), np.abs(v64))
     u = STATE_BOUND[dtype]
     assert np.all(eS <= u * Sabs + 1e-6) and np.all(eZ <= u * Zabs + 1e-6)
     return float(max(np.max(eS / bS), np.max(eZ / bZ)))

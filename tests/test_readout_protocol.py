@@ -15,14 +15,19 @@ which a parity wait could not tell apart).  Planted mistakes must be caught:
 the score buffer reused across work items without waiting for its last
 reader, and both item slots' outputs staged on one barrier (a real hazard of
 an earlier version of the kernel, found by this model once each role ran at
-its own speed).
+its own speed).  The same model runs the KATA-Mg two-factor configuration
+(9 inter stages, one score buffer per tile).
 """
 import random
 
 import pytest
 
 KERNEL = dict(kQT=128, kTiles=2, kSB=64, kKB=128, kKVRing=2, kRStages=17, kRRing=3, kRBRing=4,
-              kItemSlots=2)
+              kItemSlots=2, kSDepth=2)
+# KATA-Mg with two factors: 9 inter stages, and one score buffer per tile
+# (both factors' scores side by side), so a tile's next scores wait for the
+# squaring warps to read the previous block
+KERNEL_M2 = dict(KERNEL, kRStages=9, kSDepth=1)
 
 
 class ProtocolError(AssertionError):
@@ -52,7 +57,7 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
     kQT, kTiles, kSB, kKB = prm['kQT'], prm['kTiles'], prm['kSB'], prm['kKB']
     kKVRing, kRStages, kRRing, kRBRing, kSlots = (prm['kKVRing'], prm['kRStages'], prm['kRRing'],
                                                   prm['kRBRing'], prm['kItemSlots'])
-    kCtaQ, kHalves, kGen = kQT * kTiles, kKB // kSB, 4 * kTiles
+    kCtaQ, kHalves, kGen, D = kQT * kTiles, kKB // kSB, 4 * kTiles, prm['kSDepth']
     rng = random.Random(seed)
     n_ct = (T + kCtaQ - 1) // kCtaQ
     B = {}
@@ -73,7 +78,9 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
         B[f'afull{s}'], B[f'aempty{s}'] = Bar(kGen * 32), Bar(1)
     for t in range(kTiles):
         for x in range(2):
-            B[f'sfull{t}{x}'], B[f'pfull{t}{x}'], B[f'pempty{t}{x}'] = Bar(1), Bar(128), Bar(1)
+            B[f'pfull{t}{x}'], B[f'pempty{t}{x}'] = Bar(128), Bar(1)
+        for x in range(D):
+            B[f'sfull{t}{x}'] = Bar(1)
 
     def item(i):
         t0 = (i % n_ct) * kCtaQ
@@ -136,15 +143,15 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
                     yield W(f'kvfull{G % kKVRing}', G // kKVRing)
                 for t in range(kTiles):
                     if b < nb[t]:
-                        reuse = (b >= 2) if planted else (gb[t] + b >= 2)
+                        reuse = (b >= D) if planted else (gb[t] + b >= D)
                         if me == 0 and reuse:
-                            yield W(f'pfull{t}{(gb[t] + b - 2) & 1}', (gb[t] + b - 2) >> 1)
+                            yield W(f'pfull{t}{(gb[t] + b - D) & 1}', (gb[t] + b - D) >> 1)
                         if me == 1:
                             yield W(f'pfull{t}{(gb[t] + b) & 1}', (gb[t] + b) >> 1)
                 for t in range(kTiles):
                     if b < nb[t]:
                         n = gb[t] + b
-                        yield ('commit', f'sfull{t}{n & 1}' if me == 0 else f'pempty{t}{n & 1}')
+                        yield ('commit', f'sfull{t}{n % D}' if me == 0 else f'pempty{t}{n & 1}')
                 if h == kHalves - 1 or b == nbm - 1:
                     yield ('commit', f'kvempty{G % kKVRing}')
             g_kv += it['n_kv']
@@ -176,7 +183,7 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
                 n_inter += 1
             for b in range(blocks(it, t)):
                 n = g_b + b
-                yield W(f'sfull{t}{n & 1}', n >> 1)
+                yield W(f'sfull{t}{n % D}', n // D)
                 yield W(f'pempty{t}{n & 1}', (n >> 1) - 1)
                 yield ('arrive', f'pfull{t}{n & 1}', 32)
             g_b += blocks(it, t)
@@ -310,3 +317,19 @@ def test_quadratic_schedule_is_deadlock_free_and_phase_exact():
 def test_model_catches_a_score_buffer_reused_across_items():
     with pytest.raises(ProtocolError):
         run_cases(KERNEL, seeds=range(4), planted=True)
+
+
+def test_two_factor_readout_protocol():
+    run_cases(KERNEL_M2, seeds=range(2))
+    cq = KERNEL_M2['kQT'] * KERNEL_M2['kTiles']
+    for T, L, BH, grid in CASES[:4]:
+        n_items = (T + cq - 1) // cq * BH
+        g = min(grid, n_items)
+        for c in range(g):
+            simulate(T, L, BH, list(range(c * n_items // g, (c + 1) * n_items // g)), 17 * T + c,
+                     KERNEL_M2, init=True)
+
+
+def test_model_catches_a_two_factor_score_buffer_reused_across_items():
+    with pytest.raises(ProtocolError):
+        run_cases(KERNEL_M2, seeds=range(4), planted=True)
