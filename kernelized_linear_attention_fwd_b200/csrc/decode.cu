@@ -66,11 +66,11 @@ __device__ __forceinline__ void packed_ij(int r, int &i, int &j) {
 
 // CTAs per SM the register budget must allow (loads in flight per SM): 4 fit
 // the dense single-CTA kernel without spills, 3 the others.
-template <int P, bool PACKED>
-constexpr int min_ctas_per_sm() { return !PACKED && P == 1 ? 4 : 3; }
+template <int P, bool PACKED, int G = 1>
+constexpr int min_ctas_per_sm() { return !PACKED && P == 1 && G == 1 ? 4 : 3; }
 
 template <int DK, int DV, int P, bool PACKED, typename TIn, int G = 1>
-__global__ void __launch_bounds__(kThreads, min_ctas_per_sm<P, PACKED>())
+__global__ void __launch_bounds__(kThreads, min_ctas_per_sm<P, PACKED, G>())
 decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
                    TIn *__restrict__ out, float *__restrict__ S, float *__restrict__ Z) {
     static_assert(G == 1 || !PACKED, "factors only on the dense layout");
@@ -113,12 +113,18 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
 
     for (int row0 = row_base + rg; row0 < row_end; row0 += RPI * UNR) {
         float4 s[UNR];
+        if constexpr (G == 1) {
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const int row = row0 + u * RPI;
-            // rows across factors (G > 1) hold zeros and stay so
-            const bool held = row < row_end && (G == 1 || (row / DK) / FW == (row % DK) / FW);
-            s[u] = held ? Sh[(long long)row * V4 + c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int u = 0; u < UNR; ++u)
+                if (row0 + u * RPI < row_end) s[u] = Sh[(long long)(row0 + u * RPI) * V4 + c4];
+        } else {
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int row = row0 + u * RPI;
+                // rows across factors hold zeros and stay so: not read
+                const bool held = row < row_end && (row / DK) / FW == (row % DK) / FW;
+                s[u] = held ? Sh[(long long)row * V4 + c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
         }
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
@@ -134,7 +140,8 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
                 j = row % DK;
             }
             // a row across factors stays zero: no update, so no readout share
-            const float f = (G == 1 || i / FW == j / FW) ? sk[i] * sk[j] : 0.f;
+            float f = sk[i] * sk[j];
+            if constexpr (G > 1) f = i / FW == j / FW ? f : 0.f;
             const float w = (PACKED && i != j ? 2.f : 1.f) * (sq[i] * sq[j]);
             s[u].x = fmaf(f, vv.x, s[u].x);
             s[u].y = fmaf(f, vv.y, s[u].y);
@@ -145,11 +152,17 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
             a2 = fmaf(w, s[u].z, a2);
             a3 = fmaf(w, s[u].w, a3);
         }
+        if constexpr (G == 1) {
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const int row = row0 + u * RPI;
-            if (row < row_end && (G == 1 || (row / DK) / FW == (row % DK) / FW))
-                Sh[(long long)row * V4 + c4] = s[u];
+            for (int u = 0; u < UNR; ++u)
+                if (row0 + u * RPI < row_end) Sh[(long long)(row0 + u * RPI) * V4 + c4] = s[u];
+        } else {
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int row = row0 + u * RPI;
+                if (row < row_end && (row / DK) / FW == (row % DK) / FW)
+                    Sh[(long long)row * V4 + c4] = s[u];
+            }
         }
     }
 

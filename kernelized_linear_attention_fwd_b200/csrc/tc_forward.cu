@@ -125,20 +125,18 @@ struct ScanLane {
             zl[zj[x] * kD + zi[x]] = lo;
         }
         if constexpr (G == 2) {
-            // zeros at the 32 x 32 pairs across the two factors (both halves of the
-            // symmetric Z), spread over the 32 lanes of the packed-z blocks
-            constexpr int kCross = 32 * 32, kThr = 32 * (state_rows(G) / 128);
+            // zeros at the pairs across the two factors: in each of Z hi and Z lo,
+            // rows 0-31 columns 32-63 and rows 32-63 columns 0-31, as 16-byte runs
+            // of 8 zeros (512 stores), spread over the lanes of the packed-z blocks
+            constexpr int kStores = 2 * 64 * 4, kThr = 32 * (state_rows(G) / 128);
             const int zt = (zr / 128) * 32 + lane;
-            const __nv_bfloat16 z0 = __float2bfloat16_rn(0.f);
 #pragma unroll
-            for (int x = 0; x < (kCross + kThr - 1) / kThr; ++x) {
-                const int pi = zt + kThr * x;
-                if (pi >= kCross) break;
-                const int ci = pi / 32, cj = 32 + pi % 32;
-                zh[ci * kD + cj] = z0;
-                zl[ci * kD + cj] = z0;
-                zh[cj * kD + ci] = z0;
-                zl[cj * kD + ci] = z0;
+            for (int x = 0; x < (kStores + kThr - 1) / kThr; ++x) {
+                const int si = zt + kThr * x;
+                if (si >= kStores) break;
+                const int row = (si % 256) / 4, col = (row < 32 ? 32 : 0) + 8 * (si % 4);
+                __nv_bfloat16 *dz = (si < 256 ? zh : zl) + row * kD + col;
+                *reinterpret_cast<uint4 *>(dz) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
     }
@@ -343,7 +341,10 @@ struct ReadBars {
     uint64_t qfull[2], qempty[2], u, interdone, done, genin, ostaged[2];
     uint64_t bfull[kRBRing], bempty[kRBRing], afull[kRRing], aempty[kRRing];
     uint64_t kvfull[2], kvempty[2];
-    uint64_t sfull[kTiles][2], pfull[kTiles][2], pempty[kTiles][2];
+    // sfull: scores in a tile's score buffer; sload: the squaring warps have read
+    // them (the buffer may take the next scores); pfull / pempty: the weights
+    // in the tile's weight buffer are stored / consumed by the P-V MMAs
+    uint64_t sfull[kTiles][2], sload[kTiles][2], pfull[kTiles][2], pempty[kTiles][2];
     uint64_t drain[2];
 };
 
@@ -923,6 +924,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         for (int t = 0; t < kTiles; ++t)
             for (int x = 0; x < 2; ++x) {
                 mbar_init(&bars.sfull[t][x], 1);
+                mbar_init(&bars.sload[t][x], 4 * 32);
                 mbar_init(&bars.pfull[t][x], 4 * 32);
                 mbar_init(&bars.pempty[t][x], 1);
             }
@@ -1065,14 +1067,14 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     if ((b & 1) == 0) ok = mbar_wait(&bars.kvfull[kvb & 1], (kvb >> 1) & 1, abort);
                     if (me == 0) {
                         // scores Q K^T into score buffer n % kSDepth of tile t (n = the
-                        // tile's running block count), once the squaring warps have read
-                        // block n - kSDepth from that buffer, which may belong to the
-                        // previous item
+                        // tile's running block count), as soon as the squaring warps have
+                        // loaded block n - kSDepth from that buffer (which may belong to
+                        // the previous item) into registers
 #pragma unroll
                         for (int t = 0; t < kTiles; ++t)
                             if (ok && gb[t] + b >= kSDepth && b < nb[t]) {
                                 const int n = gb[t] + b - kSDepth;
-                                ok = mbar_wait(&bars.pfull[t][n & 1], (n >> 1) & 1, abort);
+                                ok = mbar_wait(&bars.sload[t][n % kSDepth], (n / kSDepth) & 1, abort);
                             }
                         if (!ok) break;
                         tc_fence_after();
@@ -1236,6 +1238,8 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     tmem_ld32(tS + 64 * xs, r);
                     tmem_ld32(tS + 64 * xs + 32, r + 32);
                     tmem_ld_wait();
+                    tc_fence_before();
+                    mbar_arrive(&bars.sload[t][xs]);  // the buffer may take the next scores
                     if (full) {
 #pragma unroll
                         for (int y = 0; y < 32; ++y) {
@@ -1275,6 +1279,8 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                             p[16 * h + y] = f32x2_to_bf16x2(w2);
                         }
                     }
+                    tc_fence_before();
+                    mbar_arrive(&bars.sload[t][xs]);  // the buffer may take the next scores
                 }
                 {
                     const uint64_t a01 = f32x2_add(acc[0], acc[1]), a23 = f32x2_add(acc[2], acc[3]);

@@ -1,8 +1,9 @@
 """Barrier protocol of the persistent tensor-core readout (`tc_read`), on the CPU.
 
 A step-by-step model of every role of the kernel -- TMA producer, the two MMA
-issuers (alternate inter stages; scores Q K^T by issuer 0, weights times values
-by issuer 1), the output-store warp and the squaring warps -- with the same
+issuers (alternate inter stages; scores Q K^T by issuer 0, reusing a score
+buffer once the squaring warps have loaded it; weights times values by issuer
+1), the output-store warp and the squaring warps -- with the same
 ring sizes, barrier counts and phase arithmetic as the kernel, run over
 sequences of work items (ragged tails, empty second tiles, single-segment
 heads, several items per CTA, the quadratic form's longest-first order, and
@@ -80,7 +81,7 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
         for x in range(2):
             B[f'pfull{t}{x}'], B[f'pempty{t}{x}'] = Bar(128), Bar(1)
         for x in range(D):
-            B[f'sfull{t}{x}'] = Bar(1)
+            B[f'sfull{t}{x}'], B[f'sload{t}{x}'] = Bar(1), Bar(128)
 
     def item(i):
         t0 = (i % n_ct) * kCtaQ
@@ -144,8 +145,8 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
                 for t in range(kTiles):
                     if b < nb[t]:
                         reuse = (b >= D) if planted else (gb[t] + b >= D)
-                        if me == 0 and reuse:
-                            yield W(f'pfull{t}{(gb[t] + b - D) & 1}', (gb[t] + b - D) >> 1)
+                        if me == 0 and reuse:  # the squaring warps have loaded block n - D
+                            yield W(f'sload{t}{(gb[t] + b - D) % D}', (gb[t] + b - D) // D)
                         if me == 1:
                             yield W(f'pfull{t}{(gb[t] + b) & 1}', (gb[t] + b) >> 1)
                 for t in range(kTiles):
@@ -184,6 +185,7 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
             for b in range(blocks(it, t)):
                 n = g_b + b
                 yield W(f'sfull{t}{n % D}', n // D)
+                yield ('arrive', f'sload{t}{n % D}', 32)
                 yield W(f'pempty{t}{n & 1}', (n >> 1) - 1)
                 yield ('arrive', f'pfull{t}{n & 1}', 32)
             g_b += blocks(it, t)

@@ -31,7 +31,8 @@ def rounded_product_state(k64, v64):
     return S, Z
 
 
-@pytest.mark.parametrize("d,T,qk", [(16, 300, "unit"), (64, 2500, "unit"), (32, 1500, "spread")])
+@pytest.mark.parametrize("d,T,qk", [(16, 300, "unit"), (64, 2500, "unit"), (32, 1500, "spread"),
+                                    (16, 32768, "unit")])
 def test_rounded_state_passes_and_a_one_percent_tile_fails(oracle_mod, d, T, qk):
     _, k, v = inputs.make_qkv(1, 2, T, d, d, "bf16", seed=d, qk=qk)
     k64, v64 = inputs.widen(k, "bf16")[0], inputs.widen(v, "bf16")[0]
@@ -53,3 +54,39 @@ def test_rounded_state_passes_and_a_one_percent_tile_fails(oracle_mod, d, T, qk)
     badz = Zr.copy()
     badz[:, 3] *= 1.01
     assert np.any(np.abs(badz - Z) > bZ)
+
+
+def test_rounding_bias_of_bf16_products_is_covered():
+    """bf16(p) / p - 1 is not zero-mean: the low bits of products of 8-bit
+    significands are not uniform, squares most of all.  The bias grows like
+    T on sums of positive terms (the diagonal of Z), which a zero-mean model
+    would miss; BIAS_BF16 must cover it with room."""
+    from tests.gpu_util import BIAS_BF16
+
+    g = np.random.default_rng(0)
+    k = inputs.widen(inputs.f32_to_bf16_bits((g.standard_normal(2_000_000) / 8).astype(np.float32)),
+                     "bf16")
+    k2 = inputs.widen(inputs.f32_to_bf16_bits((g.standard_normal(2_000_000) / 8).astype(np.float32)),
+                      "bf16")
+    for p in (k * k, k * k2):
+        pr = inputs.widen(inputs.f32_to_bf16_bits(p.astype(np.float32)), "bf16")
+        mean = float(np.mean((pr - p) / p))
+        assert abs(mean) <= BIAS_BF16 / 2
+    sq_mean = float(np.mean((inputs.widen(inputs.f32_to_bf16_bits((k * k).astype(np.float32)),
+                                          "bf16") - k * k) / (k * k)))
+    assert sq_mean > 2.0 ** -14  # the squares' bias is real, and positive
+    # on Z's diagonal over 32768 unit keys the bias dominates the zero-mean part
+    _, kk, vv = inputs.make_qkv(1, 1, 32768, 16, 16, "bf16", seed=5)
+    k64, v64 = inputs.widen(kk, "bf16")[0], inputs.widen(vv, "bf16")[0]
+    _, Z = oracle_mod_state(k64, v64)
+    _, Zr = rounded_product_state(k64, v64)
+    diag = np.arange(16)
+    err = (Zr - Z)[:, diag, diag]
+    assert np.all(err > 0)  # every diagonal entry is pushed up
+    assert np.all(np.abs(err) <= BIAS_BF16 * np.abs(Z[:, diag, diag]))
+
+
+def oracle_mod_state(k64, v64):
+    from oracle import oracle
+
+    return oracle.state(k64, v64)
