@@ -297,7 +297,8 @@ tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__r
 constexpr int kQT = 128;                 // query tile (MMA M)
 constexpr int kTiles = 2;                // query tiles per item
 constexpr int kCtaQ = kQT * kTiles;      // 256 queries per item
-constexpr int kKB = 128;                 // key/value block loaded by TMA
+constexpr int kKB = 64;                  // key/value block loaded by TMA (one score block)
+constexpr int kKVRing = 4;               // key/value blocks in flight (shared memory)
 constexpr int kSB = 64;                  // score block (MMA N of Q K^T)
 constexpr int kRKs = 8;                  // 16-row K-steps per inter stage (128 state rows)
 // inter stages (128 state rows each): 17 for one factor, 9 for two
@@ -314,9 +315,10 @@ constexpr int kReadThreads = 384;
 constexpr int kItemBytes = kTiles * 16384 + 16384;  // Q tiles [128 x 64] x 2, Z hi / lo [64 x 64]
 constexpr int kSmItem = 0;                       // 2 item slots (double buffer)
 constexpr int kSmS = kSmItem + 2 * kItemBytes;   // ring of [128 x 64] state-prefix tiles
-constexpr int kSmK = kSmS + kRBRing * kRStageBytes;  // 2 x [128 x 64] keys
-constexpr int kSmV = kSmK + 2 * 16384;           // 2 x [128 x 64] values
-constexpr int kSmBytes = kSmV + 2 * 16384;
+constexpr int kKVBytes = kKB * kD * 2;          // one [64 x 64] bf16 key or value block
+constexpr int kSmK = kSmS + kRBRing * kRStageBytes;  // kKVRing x [64 x 64] keys
+constexpr int kSmV = kSmK + kKVRing * kKVBytes;  // kKVRing x [64 x 64] values
+constexpr int kSmBytes = kSmV + kKVRing * kKVBytes;
 constexpr int kSmAlloc = kSmBytes + 1024;
 
 // tensor memory columns (512 allocated)
@@ -340,7 +342,7 @@ struct ReadBars {
     // neither barrier can complete twice ahead of the store warp's wait.
     uint64_t qfull[2], qempty[2], u, interdone, done, genin, ostaged[2];
     uint64_t bfull[kRBRing], bempty[kRBRing], afull[kRRing], aempty[kRRing];
-    uint64_t kvfull[2], kvempty[2];
+    uint64_t kvfull[kKVRing], kvempty[kKVRing];
     // sfull: scores in a tile's score buffer; sload: the squaring warps have read
     // them (the buffer may take the next scores); pfull / pempty: the weights
     // in the tile's weight buffer are stored / consumed by the P-V MMAs
@@ -597,12 +599,13 @@ struct BuildBars {
     uint64_t drain[2];
 };
 
-// Products k_i k_j of one 16-token step (this warpgroup's half of a 32-token
-// stage) for the thread's NT rows: p[8 m + w] holds tokens 2 w, 2 w + 1.
+// Products k_i k_j of one 16-token step (16-byte chunks 4 half + 2 sub and
+// 4 half + 2 sub + 1 of the 64-token key tile) for the thread's NT rows:
+// p[8 m + w] holds tokens 2 w, 2 w + 1 of row m.
 template <int NT>
-__device__ __forceinline__ void build_products(const uint8_t *kt, int half, int wg, int jcol,
-                                               const int (&im)[kBTiles], uint32_t (&p)[8 * NT]) {
-    const int c0 = 4 * half + 2 * wg, c1 = c0 + 1;  // 16-byte chunks of this warpgroup's 16 tokens
+__device__ __forceinline__ void build_products(const uint8_t *kt, int half, int sub, int jcol,
+                                               const int (&im)[kBTiles], uint32_t *p) {
+    const int c0 = 4 * half + 2 * sub, c1 = c0 + 1;
     uint32_t own[8];
     {
         const uint8_t *r = kt + jcol * 128;
@@ -624,52 +627,86 @@ __device__ __forceinline__ void build_products(const uint8_t *kt, int half, int 
     }
 }
 
-template <int NT>
-__device__ __forceinline__ void build_store(uint32_t taddr, const uint32_t (&p)[8 * NT]) {
-    if constexpr (NT == 4) tmem_st32(taddr, p);
-    else tmem_st8(taddr, p);
+// Stages of a work item: two 32-token stages per 64-token tile for an item
+// of 4 accumulator tiles (8 MMAs per stage); one "wide" 128-token stage per
+// two tiles for an item of a single accumulator tile, so that its stages hold
+// 8 MMAs too instead of 2 (a stage costs about the same whatever it holds).
+__device__ __forceinline__ int build_item_stages(int nt, int n_tt) {
+    return nt == 1 ? (n_tt + 1) / 2 : 2 * n_tt;
 }
 
-// Generation side of one item: 2 stages per 64-token tile.  `tt` is the
-// CTA's running tile counter (ring slot and phase), advanced past the item.
-template <int NT>
+// Generation side of an item of 4 tiles: 2 stages per 64-token tile.  `tt`
+// and `ns` are the CTA's running tile and stage counters (ring slots and
+// phases), advanced past the item.
 __device__ __forceinline__ bool build_item_gen(BuildBars &bars, const uint8_t *sm, uint32_t ta, int wg,
-                                               int jcol, const int (&im)[kBTiles], int &tt, int n_tt,
-                                               volatile int *abort) {
-    uint32_t pa[8 * NT], pb[8 * NT];
+                                               int jcol, const int (&im)[kBTiles], int &tt, int &ns,
+                                               int n_tt, volatile int *abort) {
+    uint32_t pa[8 * kBTiles], pb[8 * kBTiles];
     {
         const int b = tt % kBTileRing;
         if (!__all_sync(0xffffffffu, mbar_wait(&bars.tfull[b], (tt / kBTileRing) & 1, abort))) return false;
-        build_products<NT>(sm + b * kBTileBytes, 0, wg, jcol, im, pa);
+        build_products<kBTiles>(sm + b * kBTileBytes, 0, wg, jcol, im, pa);
     }
     for (int t = 0; t < n_tt; ++t, ++tt) {
         const int b = tt % kBTileRing;
-        int G = 2 * tt, a = G % kBARing;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((G / kBARing) & 1) ^ 1, abort)))
+        int gs = ns + 2 * t, a = gs % kBARing;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((gs / kBARing) & 1) ^ 1, abort)))
             return false;
         tc_fence_after();
-        build_store<NT>(ta + 64 * a, pa);
-        build_products<NT>(sm + b * kBTileBytes, 1, wg, jcol, im, pb);
+        tmem_st32(ta + 64 * a, pa);
+        build_products<kBTiles>(sm + b * kBTileBytes, 1, wg, jcol, im, pb);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars.afull[a]);
 
-        G = 2 * tt + 1;
-        a = G % kBARing;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((G / kBARing) & 1) ^ 1, abort)))
+        gs = ns + 2 * t + 1;
+        a = gs % kBARing;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((gs / kBARing) & 1) ^ 1, abort)))
             return false;
         tc_fence_after();
-        build_store<NT>(ta + 64 * a, pb);
+        tmem_st32(ta + 64 * a, pb);
         if (t + 1 < n_tt) {
             const int bn = (tt + 1) % kBTileRing;
             if (!__all_sync(0xffffffffu, mbar_wait(&bars.tfull[bn], ((tt + 1) / kBTileRing) & 1, abort)))
                 return false;
-            build_products<NT>(sm + bn * kBTileBytes, 0, wg, jcol, im, pa);
+            build_products<kBTiles>(sm + bn * kBTileBytes, 0, wg, jcol, im, pa);
         }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars.afull[a]);
     }
+    ns += 2 * n_tt;
+    return true;
+}
+
+// Generation side of an item of a single tile: wide stages of two 64-token
+// tiles, warpgroup wg taking tile 2 s + wg of stage s (all four of its
+// 16-token steps, A-slot columns 32 wg .. 32 wg + 31).  A warpgroup without a
+// tile in the last stage (odd tile count) only arrives.
+__device__ __forceinline__ bool build_item_gen_wide(BuildBars &bars, const uint8_t *sm, uint32_t ta,
+                                                    int wg, int jcol, const int (&im)[kBTiles], int &tt,
+                                                    int &ns, int n_tt, volatile int *abort) {
+    const int n_st = build_item_stages(1, n_tt);
+    for (int s = 0; s < n_st; ++s) {
+        const int gs = ns + s, a = gs % kBARing, t = 2 * s + wg;
+        uint32_t p[32];
+        if (t < n_tt) {
+            const int tg = tt + t, b = tg % kBTileRing;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bars.tfull[b], (tg / kBTileRing) & 1, abort)))
+                return false;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) build_products<1>(sm + b * kBTileBytes, q >> 1, q & 1, jcol, im, p + 8 * q);
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((gs / kBARing) & 1) ^ 1, abort)))
+            return false;
+        tc_fence_after();
+        if (t < n_tt) tmem_st32(ta + 64 * a, p);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars.afull[a]);
+    }
+    tt += n_tt;
+    ns += n_st;
     return true;
 }
 
@@ -759,37 +796,77 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             const int me = warp - kBIssuer0;
             const uint32_t idesc = idesc_bf16(128, kBN, 0, 1);
             const uint32_t sbase = smem_u32(sm);
-            int tt = 0;  // global tile counter
-            bool ok = true;
-            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+            int tt = 0, ns = 0, j = 0;  // global tile and stage counters, item count
+            bool ok = true, issued = false;
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
                 int c, g, bh, s0, n_tt;
                 build_item_geom<G>(item, n_build, T, L, c, g, bh, s0, n_tt);
                 const int nt = build_item_tiles(G, c);
-                for (int t = 0; t < n_tt && ok; ++t, ++tt) {
-                    const int gs = 2 * tt + me;  // global stage: this issuer takes one half of each tile
-                    const int b = tt % kBTileRing, a = gs % kBARing;
-                    ok = mbar_wait(&bars.tfull[b], (tt / kBTileRing) & 1, abort) &&
-                         mbar_wait(&bars.afull[a], (gs / kBARing) & 1, abort);
+                const bool wide = nt == 1;
+                const int n_st = build_item_stages(nt, n_tt);
+                int mine = 0;
+                // the issuers take alternate stages of the CTA's running stage count
+                for (int st = (ns + me) & 1; st < n_st && ok; st += 2) {
+                    const int gs = ns + st, a = gs % kBARing;
+                    const int t0 = wide ? 2 * st : st / 2;                      // first tile of the stage
+                    const int ntl = wide ? (n_tt - t0 < 2 ? n_tt - t0 : 2) : 1;  // its tiles
+                    for (int x = 0; x < ntl && ok; ++x) {
+                        const int tg = tt + t0 + x;
+                        ok = mbar_wait(&bars.tfull[tg % kBTileRing], (tg / kBTileRing) & 1, abort);
+                    }
+                    ok = ok && mbar_wait(&bars.afull[a], (gs / kBARing) & 1, abort);
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t vaddr = sbase + b * kBTileBytes + 8192 + 4096 * me;
-                    const uint32_t oaddr = sbase + kBOnes + 4096 * me;
-                    const uint64_t dv = desc_sw128(vaddr, oaddr - vaddr, 1024);
                     const uint32_t ta = tm + kBTmA + 64 * a;
+                    if (wide) {
+                        // 16-token steps kk of the stage's tiles into the one accumulator
+                        for (int kk = 0; kk < 4 * ntl; ++kk) {
+                            const int b = (tt + t0 + kk / 4) % kBTileRing;
+                            const uint32_t vaddr = sbase + b * kBTileBytes + 8192;
+                            const uint64_t dv = desc_sw128(vaddr, sbase + kBOnes - vaddr, 1024);
+                            mma_ts(tm, ta + 8 * kk, desc_add(dv, 2048 * (kk % 4)), idesc, 1);
+                        }
+                    } else {
+                        const int h = st & 1;  // the 32-token half of tile t0
+                        const int b = (tt + t0) % kBTileRing;
+                        const uint32_t vaddr = sbase + b * kBTileBytes + 8192 + 4096 * h;
+                        const uint32_t oaddr = sbase + kBOnes + 4096 * h;
+                        const uint64_t dv = desc_sw128(vaddr, oaddr - vaddr, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < 2; ++kk)
+                        for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
-                        for (int m = 0; m < kBTiles; ++m)
-                            if (m < nt)
+                            for (int m = 0; m < kBTiles; ++m)
                                 mma_ts(tm + kBN * m, ta + 32 * kk + 8 * m, desc_add(dv, 2048 * kk), idesc, 1);
+                    }
+                    issued = true;
+                    ++mine;
                     mma_commit(&bars.aempty[a]);
-                    mma_commit(&bars.tempty[b]);
+                    // a tile takes two arrivals: its two 32-token halves
+                    for (int x = 0; x < ntl; ++x) {
+                        const int b = (tt + t0 + x) % kBTileRing;
+                        mma_commit(&bars.tempty[b]);
+                        if (wide) mma_commit(&bars.tempty[b]);
+                    }
                 }
-                if (ok) mma_commit(&bars.done);  // this item's accumulation complete (with the other issuer)
+                if (!ok) break;
+                if (mine) {
+                    mma_commit(&bars.done);  // this item's accumulation complete (with the other issuer)
+                } else {
+                    // no stage in this item: arrive directly, once this issuer's commit for
+                    // the previous item has landed (earlier, it would complete that item's
+                    // phase while its MMAs still run)
+                    if (j > 0 && !mbar_wait(&bars.done, (j - 1) & 1, abort)) break;
+                    mbar_arrive(&bars.done);
+                }
+                tt += n_tt;
+                ns += n_st;
             }
             // no MMA of this CTA may still read or write tensor memory when it is freed
-            mma_commit(&bars.drain[me]);
-            mbar_wait_issued(&bars.drain[me], 0);
+            // (a commit is made only after an MMA of this thread)
+            if (issued) {
+                mma_commit(&bars.drain[me]);
+                mbar_wait_issued(&bars.drain[me], 0);
+            }
         }
     } else if (warp == kBStoreWarp) {
         // ------------------------------------------------------------ write-back of drained tiles
@@ -828,7 +905,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             }
         };
         zero_acc();
-        int tt = 0, j = 0;
+        int tt = 0, ns = 0, j = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
             int c, g, bh, s0, n_tt;
@@ -842,8 +919,8 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
                 jcol = pij.j;  // the same for every tile of the item
             }
             const uint32_t ta = tm + kBTmA + 32 * wg + lane_base;
-            ok = nt == kBTiles ? build_item_gen<kBTiles>(bars, sm, ta, wg, jcol, im, tt, n_tt, abort)
-                               : build_item_gen<1>(bars, sm, ta, wg, jcol, im, tt, n_tt, abort);
+            ok = nt == kBTiles ? build_item_gen(bars, sm, ta, wg, jcol, im, tt, ns, n_tt, abort)
+                               : build_item_gen_wide(bars, sm, ta, wg, jcol, im, tt, ns, n_tt, abort);
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.done, j & 1, abort));
             if (ok && j > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfree, (j - 1) & 1, abort));
             if (!ok) break;
@@ -854,20 +931,22 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             tc_fence_after();
             float *zbase = seg_state + ((long long)bh * n_seg + g) * f32_per_seg(G) + z_packed0(G);
             for (int m = 2 * wg; m < 2 * wg + 2 && m < nt; ++m) {
-                uint32_t o[32];
+                // the tile's 64 values and its normaliser column in one round trip
+                uint32_t o[64], oz[8];
+                tmem_ld32(tm + kBN * m + lane_base, o);
+                tmem_ld32(tm + kBN * m + 32 + lane_base, o + 32);
+                tmem_ld8(tm + kBN * m + 64 + lane_base, oz);
+                tmem_ld_wait();
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    tmem_ld32(tm + kBN * m + 32 * h + lane_base, o);
-                    tmem_ld_wait();
                     uint8_t *box = sm + kBStage + (2 * m + h) * kBStageBox + row * 128;
 #pragma unroll
                     for (int x = 0; x < 8; ++x)
                         *reinterpret_cast<uint4 *>(box + ((x ^ (row & 7)) * 16)) =
-                            make_uint4(o[4 * x], o[4 * x + 1], o[4 * x + 2], o[4 * x + 3]);
+                            make_uint4(o[32 * h + 4 * x], o[32 * h + 4 * x + 1], o[32 * h + 4 * x + 2],
+                                       o[32 * h + 4 * x + 3]);
                 }
-                tmem_ld8(tm + kBN * m + 64 + lane_base, o);
-                tmem_ld_wait();
-                zbase[128 * build_item_tile(G, c, m) + row] = __uint_as_float(o[0]);
+                zbase[128 * build_item_tile(G, c, m) + row] = __uint_as_float(oz[0]);
             }
             fence_proxy_async_smem();
             mbar_arrive(&bars.staged);
@@ -903,9 +982,11 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars.qfull[b], 1);
             mbar_init(&bars.qempty[b], 3);  // both issuers' commits + the output store's read
-            mbar_init(&bars.kvfull[b], 1);
-            mbar_init(&bars.kvempty[b], 2);
             mbar_init(&bars.drain[b], 1);
+        }
+        for (int b = 0; b < kKVRing; ++b) {
+            mbar_init(&bars.kvfull[b], 1);
+            mbar_init(&bars.kvempty[b], 2);  // both issuers' commits
         }
         mbar_init(&bars.u, 1);
         mbar_init(&bars.interdone, 2);
@@ -976,12 +1057,12 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     ++n_bs;
                 }
                 for (int kb = 0; kb < it.n_kv && ok; ++kb) {
-                    const int s = n_kv & 1;
-                    ok = mbar_wait(&bars.kvempty[s], ((n_kv >> 1) & 1) ^ 1, abort);
+                    const int s = n_kv % kKVRing;
+                    ok = mbar_wait(&bars.kvempty[s], ((n_kv / kKVRing) & 1) ^ 1, abort);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(&bars.kvfull[s], 32768);
-                    tma_load_3d(sm + kSmK + s * 16384, &tm_k, &bars.kvfull[s], 0, it.seg0 + kb * kKB, it.bh);
-                    tma_load_3d(sm + kSmV + s * 16384, &tm_v, &bars.kvfull[s], 0, it.seg0 + kb * kKB, it.bh);
+                    mbar_arrive_expect_tx(&bars.kvfull[s], 2 * kKVBytes);
+                    tma_load_3d(sm + kSmK + s * kKVBytes, &tm_k, &bars.kvfull[s], 0, it.seg0 + kb * kKB, it.bh);
+                    tma_load_3d(sm + kSmV + s * kKVBytes, &tm_v, &bars.kvfull[s], 0, it.seg0 + kb * kKB, it.bh);
                     ++n_kv;
                 }
             }
@@ -990,8 +1071,8 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                 mbar_wait_issued(&bars.qfull[x & 1], (x >> 1) & 1);
             for (int x = (n_bs > kRBRing ? n_bs - kRBRing : 0); x < n_bs; ++x)
                 mbar_wait_issued(&bars.bfull[x % kRBRing], (x / kRBRing) & 1);
-            for (int x = (n_kv > 2 ? n_kv - 2 : 0); x < n_kv; ++x)
-                mbar_wait_issued(&bars.kvfull[x & 1], (x >> 1) & 1);
+            for (int x = (n_kv > kKVRing ? n_kv - kKVRing : 0); x < n_kv; ++x)
+                mbar_wait_issued(&bars.kvfull[x % kKVRing], (x / kKVRing) & 1);
         }
     } else if (warp == kIssuer0 || warp == kIssuer0 + 1) {
         // ------------------------------------------------------------ MMA issuers
@@ -1058,13 +1139,14 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     tc_fence_after();
                     ++n_inter;
                 }
-                // intra phase over 64-key blocks b (block b uses K/V block b / 2, half b % 2)
+                // intra phase over 64-key blocks b (block b uses key/value block b)
                 const int nb[kTiles] = {read_tile_blocks(it, 0, T), read_tile_blocks(it, 1, T)};
                 const int gb[kTiles] = {g_b0, g_b1};
                 const int nbm = max(nb[0], nb[1]);
                 for (int b = 0; b < nbm && ok; ++b) {
-                    const int kvb = g_kv + b / 2;
-                    if ((b & 1) == 0) ok = mbar_wait(&bars.kvfull[kvb & 1], (kvb >> 1) & 1, abort);
+                    // score block b uses key/value block b of the item
+                    const int kvb = g_kv + b, kvs = kvb % kKVRing;
+                    ok = mbar_wait(&bars.kvfull[kvs], (kvb / kKVRing) & 1, abort);
                     if (me == 0) {
                         // scores Q K^T into score buffer n % kSDepth of tile t (n = the
                         // tile's running block count), as soon as the squaring warps have
@@ -1078,7 +1160,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                             }
                         if (!ok) break;
                         tc_fence_after();
-                        const uint64_t dk = desc_add(dK, 16384 * (kvb & 1) + 8192 * (b & 1));
+                        const uint64_t dk = desc_add(dK, kKVBytes * kvs);
 #pragma unroll
                         for (int t = 0; t < kTiles; ++t) {
                             if (b >= nb[t]) continue;
@@ -1109,7 +1191,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                             }
                         if (!ok) break;
                         tc_fence_after();
-                        const uint64_t dv = desc_add(dV, 16384 * (kvb & 1) + 8192 * (b & 1));
+                        const uint64_t dv = desc_add(dV, kKVBytes * kvs);
 #pragma unroll
                         for (int t = 0; t < kTiles; ++t) {
                             if (b >= nb[t]) continue;
@@ -1121,8 +1203,8 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                             mma_commit(&bars.pempty[t][x]);
                         }
                     }
-                    // this issuer is done with K/V block b / 2
-                    if ((b & 1) || b == nbm - 1) mma_commit(&bars.kvempty[kvb & 1]);
+                    // this issuer is done with key/value block b
+                    mma_commit(&bars.kvempty[kvs]);
                 }
                 if (!ok) break;
                 g_kv += it.n_kv;
@@ -1349,8 +1431,9 @@ bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const
     const uint64_t ds[3] = {(uint64_t)kD, (uint64_t)bf16_rows(G), (uint64_t)(p.BH * p.n_seg)};
     const uint64_t ss[2] = {(uint64_t)kD * 2, (uint64_t)bf16_rows(G) * kD * 2};
     const uint32_t bs[3] = {64, 32, 1};
-    return make_tmap_bf16(mq, q, 3, dqkv, sqkv, bqkv) && make_tmap_bf16(mk, k, 3, dqkv, sqkv, bqkv) &&
-           make_tmap_bf16(mv, v, 3, dqkv, sqkv, bqkv) &&
+    const uint32_t bkv[3] = {64, kKB, 1};
+    return make_tmap_bf16(mq, q, 3, dqkv, sqkv, bqkv) && make_tmap_bf16(mk, k, 3, dqkv, sqkv, bkv) &&
+           make_tmap_bf16(mv, v, 3, dqkv, sqkv, bkv) &&
            make_tmap_bf16(ms, prefix ? prefix : q, 3, ds, ss, bs) && make_tmap_bf16(mo, out, 3, dqkv, sqkv, bqkv);
 }
 

@@ -23,7 +23,7 @@ import random
 
 import pytest
 
-KERNEL = dict(kQT=128, kTiles=2, kSB=64, kKB=128, kKVRing=2, kRStages=17, kRRing=3, kRBRing=4,
+KERNEL = dict(kQT=128, kTiles=2, kSB=64, kKB=64, kKVRing=4, kRStages=17, kRRing=3, kRBRing=4,
               kItemSlots=2, kSDepth=2)
 # KATA-Mg with two factors: 9 inter stages, and one score buffer per tile
 # (both factors' scores side by side), so a tile's next scores wait for the
