@@ -599,13 +599,12 @@ struct BuildBars {
     uint64_t drain[2];
 };
 
-// Products k_i k_j of one 16-token step (16-byte chunks 4 half + 2 sub and
-// 4 half + 2 sub + 1 of the 64-token key tile) for the thread's NT rows:
-// p[8 m + w] holds tokens 2 w, 2 w + 1 of row m.
+// Products k_i k_j of one 16-token step (this warpgroup's half of a 32-token
+// stage) for the thread's NT rows: p[8 m + w] holds tokens 2 w, 2 w + 1.
 template <int NT>
-__device__ __forceinline__ void build_products(const uint8_t *kt, int half, int sub, int jcol,
-                                               const int (&im)[kBTiles], uint32_t *p) {
-    const int c0 = 4 * half + 2 * sub, c1 = c0 + 1;
+__device__ __forceinline__ void build_products(const uint8_t *kt, int half, int wg, int jcol,
+                                               const int (&im)[kBTiles], uint32_t (&p)[8 * NT]) {
+    const int c0 = 4 * half + 2 * wg, c1 = c0 + 1;  // 16-byte chunks of this warpgroup's 16 tokens
     uint32_t own[8];
     {
         const uint8_t *r = kt + jcol * 128;
@@ -627,86 +626,52 @@ __device__ __forceinline__ void build_products(const uint8_t *kt, int half, int 
     }
 }
 
-// Stages of a work item: two 32-token stages per 64-token tile for an item
-// of 4 accumulator tiles (8 MMAs per stage); one "wide" 128-token stage per
-// two tiles for an item of a single accumulator tile, so that its stages hold
-// 8 MMAs too instead of 2 (a stage costs about the same whatever it holds).
-__device__ __forceinline__ int build_item_stages(int nt, int n_tt) {
-    return nt == 1 ? (n_tt + 1) / 2 : 2 * n_tt;
+template <int NT>
+__device__ __forceinline__ void build_store(uint32_t taddr, const uint32_t (&p)[8 * NT]) {
+    if constexpr (NT == 4) tmem_st32(taddr, p);
+    else tmem_st8(taddr, p);
 }
 
-// Generation side of an item of 4 tiles: 2 stages per 64-token tile.  `tt`
-// and `ns` are the CTA's running tile and stage counters (ring slots and
-// phases), advanced past the item.
+// Generation side of one item: 2 stages per 64-token tile.  `tt` is the
+// CTA's running tile counter (ring slot and phase), advanced past the item.
+template <int NT>
 __device__ __forceinline__ bool build_item_gen(BuildBars &bars, const uint8_t *sm, uint32_t ta, int wg,
-                                               int jcol, const int (&im)[kBTiles], int &tt, int &ns,
-                                               int n_tt, volatile int *abort) {
-    uint32_t pa[8 * kBTiles], pb[8 * kBTiles];
+                                               int jcol, const int (&im)[kBTiles], int &tt, int n_tt,
+                                               volatile int *abort) {
+    uint32_t pa[8 * NT], pb[8 * NT];
     {
         const int b = tt % kBTileRing;
         if (!__all_sync(0xffffffffu, mbar_wait(&bars.tfull[b], (tt / kBTileRing) & 1, abort))) return false;
-        build_products<kBTiles>(sm + b * kBTileBytes, 0, wg, jcol, im, pa);
+        build_products<NT>(sm + b * kBTileBytes, 0, wg, jcol, im, pa);
     }
     for (int t = 0; t < n_tt; ++t, ++tt) {
         const int b = tt % kBTileRing;
-        int gs = ns + 2 * t, a = gs % kBARing;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((gs / kBARing) & 1) ^ 1, abort)))
+        int G = 2 * tt, a = G % kBARing;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((G / kBARing) & 1) ^ 1, abort)))
             return false;
         tc_fence_after();
-        tmem_st32(ta + 64 * a, pa);
-        build_products<kBTiles>(sm + b * kBTileBytes, 1, wg, jcol, im, pb);
+        build_store<NT>(ta + 64 * a, pa);
+        build_products<NT>(sm + b * kBTileBytes, 1, wg, jcol, im, pb);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars.afull[a]);
 
-        gs = ns + 2 * t + 1;
-        a = gs % kBARing;
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((gs / kBARing) & 1) ^ 1, abort)))
+        G = 2 * tt + 1;
+        a = G % kBARing;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((G / kBARing) & 1) ^ 1, abort)))
             return false;
         tc_fence_after();
-        tmem_st32(ta + 64 * a, pb);
+        build_store<NT>(ta + 64 * a, pb);
         if (t + 1 < n_tt) {
             const int bn = (tt + 1) % kBTileRing;
             if (!__all_sync(0xffffffffu, mbar_wait(&bars.tfull[bn], ((tt + 1) / kBTileRing) & 1, abort)))
                 return false;
-            build_products<kBTiles>(sm + bn * kBTileBytes, 0, wg, jcol, im, pa);
+            build_products<NT>(sm + bn * kBTileBytes, 0, wg, jcol, im, pa);
         }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars.afull[a]);
     }
-    ns += 2 * n_tt;
-    return true;
-}
-
-// Generation side of an item of a single tile: wide stages of two 64-token
-// tiles, warpgroup wg taking tile 2 s + wg of stage s (all four of its
-// 16-token steps, A-slot columns 32 wg .. 32 wg + 31).  A warpgroup without a
-// tile in the last stage (odd tile count) only arrives.
-__device__ __forceinline__ bool build_item_gen_wide(BuildBars &bars, const uint8_t *sm, uint32_t ta,
-                                                    int wg, int jcol, const int (&im)[kBTiles], int &tt,
-                                                    int &ns, int n_tt, volatile int *abort) {
-    const int n_st = build_item_stages(1, n_tt);
-    for (int s = 0; s < n_st; ++s) {
-        const int gs = ns + s, a = gs % kBARing, t = 2 * s + wg;
-        uint32_t p[32];
-        if (t < n_tt) {
-            const int tg = tt + t, b = tg % kBTileRing;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bars.tfull[b], (tg / kBTileRing) & 1, abort)))
-                return false;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) build_products<1>(sm + b * kBTileBytes, q >> 1, q & 1, jcol, im, p + 8 * q);
-        }
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.aempty[a], ((gs / kBARing) & 1) ^ 1, abort)))
-            return false;
-        tc_fence_after();
-        if (t < n_tt) tmem_st32(ta + 64 * a, p);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&bars.afull[a]);
-    }
-    tt += n_tt;
-    ns += n_st;
     return true;
 }
 
@@ -796,77 +761,37 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             const int me = warp - kBIssuer0;
             const uint32_t idesc = idesc_bf16(128, kBN, 0, 1);
             const uint32_t sbase = smem_u32(sm);
-            int tt = 0, ns = 0, j = 0;  // global tile and stage counters, item count
-            bool ok = true, issued = false;
-            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
+            int tt = 0;  // global tile counter
+            bool ok = true;
+            for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 int c, g, bh, s0, n_tt;
                 build_item_geom<G>(item, n_build, T, L, c, g, bh, s0, n_tt);
                 const int nt = build_item_tiles(G, c);
-                const bool wide = nt == 1;
-                const int n_st = build_item_stages(nt, n_tt);
-                int mine = 0;
-                // the issuers take alternate stages of the CTA's running stage count
-                for (int st = (ns + me) & 1; st < n_st && ok; st += 2) {
-                    const int gs = ns + st, a = gs % kBARing;
-                    const int t0 = wide ? 2 * st : st / 2;                      // first tile of the stage
-                    const int ntl = wide ? (n_tt - t0 < 2 ? n_tt - t0 : 2) : 1;  // its tiles
-                    for (int x = 0; x < ntl && ok; ++x) {
-                        const int tg = tt + t0 + x;
-                        ok = mbar_wait(&bars.tfull[tg % kBTileRing], (tg / kBTileRing) & 1, abort);
-                    }
-                    ok = ok && mbar_wait(&bars.afull[a], (gs / kBARing) & 1, abort);
+                for (int t = 0; t < n_tt && ok; ++t, ++tt) {
+                    const int gs = 2 * tt + me;  // global stage: this issuer takes one half of each tile
+                    const int b = tt % kBTileRing, a = gs % kBARing;
+                    ok = mbar_wait(&bars.tfull[b], (tt / kBTileRing) & 1, abort) &&
+                         mbar_wait(&bars.afull[a], (gs / kBARing) & 1, abort);
                     if (!ok) break;
                     tc_fence_after();
+                    const uint32_t vaddr = sbase + b * kBTileBytes + 8192 + 4096 * me;
+                    const uint32_t oaddr = sbase + kBOnes + 4096 * me;
+                    const uint64_t dv = desc_sw128(vaddr, oaddr - vaddr, 1024);
                     const uint32_t ta = tm + kBTmA + 64 * a;
-                    if (wide) {
-                        // 16-token steps kk of the stage's tiles into the one accumulator
-                        for (int kk = 0; kk < 4 * ntl; ++kk) {
-                            const int b = (tt + t0 + kk / 4) % kBTileRing;
-                            const uint32_t vaddr = sbase + b * kBTileBytes + 8192;
-                            const uint64_t dv = desc_sw128(vaddr, sbase + kBOnes - vaddr, 1024);
-                            mma_ts(tm, ta + 8 * kk, desc_add(dv, 2048 * (kk % 4)), idesc, 1);
-                        }
-                    } else {
-                        const int h = st & 1;  // the 32-token half of tile t0
-                        const int b = (tt + t0) % kBTileRing;
-                        const uint32_t vaddr = sbase + b * kBTileBytes + 8192 + 4096 * h;
-                        const uint32_t oaddr = sbase + kBOnes + 4096 * h;
-                        const uint64_t dv = desc_sw128(vaddr, oaddr - vaddr, 1024);
 #pragma unroll
-                        for (int kk = 0; kk < 2; ++kk)
+                    for (int kk = 0; kk < 2; ++kk)
 #pragma unroll
-                            for (int m = 0; m < kBTiles; ++m)
+                        for (int m = 0; m < kBTiles; ++m)
+                            if (m < nt)
                                 mma_ts(tm + kBN * m, ta + 32 * kk + 8 * m, desc_add(dv, 2048 * kk), idesc, 1);
-                    }
-                    issued = true;
-                    ++mine;
                     mma_commit(&bars.aempty[a]);
-                    // a tile takes two arrivals: its two 32-token halves
-                    for (int x = 0; x < ntl; ++x) {
-                        const int b = (tt + t0 + x) % kBTileRing;
-                        mma_commit(&bars.tempty[b]);
-                        if (wide) mma_commit(&bars.tempty[b]);
-                    }
+                    mma_commit(&bars.tempty[b]);
                 }
-                if (!ok) break;
-                if (mine) {
-                    mma_commit(&bars.done);  // this item's accumulation complete (with the other issuer)
-                } else {
-                    // no stage in this item: arrive directly, once this issuer's commit for
-                    // the previous item has landed (earlier, it would complete that item's
-                    // phase while its MMAs still run)
-                    if (j > 0 && !mbar_wait(&bars.done, (j - 1) & 1, abort)) break;
-                    mbar_arrive(&bars.done);
-                }
-                tt += n_tt;
-                ns += n_st;
+                if (ok) mma_commit(&bars.done);  // this item's accumulation complete (with the other issuer)
             }
             // no MMA of this CTA may still read or write tensor memory when it is freed
-            // (a commit is made only after an MMA of this thread)
-            if (issued) {
-                mma_commit(&bars.drain[me]);
-                mbar_wait_issued(&bars.drain[me], 0);
-            }
+            mma_commit(&bars.drain[me]);
+            mbar_wait_issued(&bars.drain[me], 0);
         }
     } else if (warp == kBStoreWarp) {
         // ------------------------------------------------------------ write-back of drained tiles
@@ -905,7 +830,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             }
         };
         zero_acc();
-        int tt = 0, ns = 0, j = 0;
+        int tt = 0, j = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
             int c, g, bh, s0, n_tt;
@@ -919,8 +844,8 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
                 jcol = pij.j;  // the same for every tile of the item
             }
             const uint32_t ta = tm + kBTmA + 32 * wg + lane_base;
-            ok = nt == kBTiles ? build_item_gen(bars, sm, ta, wg, jcol, im, tt, ns, n_tt, abort)
-                               : build_item_gen_wide(bars, sm, ta, wg, jcol, im, tt, ns, n_tt, abort);
+            ok = nt == kBTiles ? build_item_gen<kBTiles>(bars, sm, ta, wg, jcol, im, tt, n_tt, abort)
+                               : build_item_gen<1>(bars, sm, ta, wg, jcol, im, tt, n_tt, abort);
             if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars.done, j & 1, abort));
             if (ok && j > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfree, (j - 1) & 1, abort));
             if (!ok) break;
@@ -931,22 +856,20 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
             tc_fence_after();
             float *zbase = seg_state + ((long long)bh * n_seg + g) * f32_per_seg(G) + z_packed0(G);
             for (int m = 2 * wg; m < 2 * wg + 2 && m < nt; ++m) {
-                // the tile's 64 values and its normaliser column in one round trip
-                uint32_t o[64], oz[8];
-                tmem_ld32(tm + kBN * m + lane_base, o);
-                tmem_ld32(tm + kBN * m + 32 + lane_base, o + 32);
-                tmem_ld8(tm + kBN * m + 64 + lane_base, oz);
-                tmem_ld_wait();
+                uint32_t o[32];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
+                    tmem_ld32(tm + kBN * m + 32 * h + lane_base, o);
+                    tmem_ld_wait();
                     uint8_t *box = sm + kBStage + (2 * m + h) * kBStageBox + row * 128;
 #pragma unroll
                     for (int x = 0; x < 8; ++x)
                         *reinterpret_cast<uint4 *>(box + ((x ^ (row & 7)) * 16)) =
-                            make_uint4(o[32 * h + 4 * x], o[32 * h + 4 * x + 1], o[32 * h + 4 * x + 2],
-                                       o[32 * h + 4 * x + 3]);
+                            make_uint4(o[4 * x], o[4 * x + 1], o[4 * x + 2], o[4 * x + 3]);
                 }
-                zbase[128 * build_item_tile(G, c, m) + row] = __uint_as_float(oz[0]);
+                tmem_ld8(tm + kBN * m + 64 + lane_base, o);
+                tmem_ld_wait();
+                zbase[128 * build_item_tile(G, c, m) + row] = __uint_as_float(o[0]);
             }
             fence_proxy_async_smem();
             mbar_arrive(&bars.staged);
