@@ -76,7 +76,7 @@ struct Plan {
     size_t ws_seg_state;  // fp32 per-segment states, exclusive prefix after the scan
     size_t ws_total;      // fp32 total state (packed), when needed
     size_t ws_extra;      // path-specific
-    size_t ws_aux;        // path-specific (tensor-core path: transposed keys)
+    size_t ws_aux;        // path-specific (padded route: the d = 64 workspace)
     size_t ws_bytes;
 };
 

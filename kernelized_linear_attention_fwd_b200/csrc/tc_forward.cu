@@ -7,9 +7,9 @@
 // stored every L tokens (a segment); inside a segment the causal quadratic
 // form is used, which equals the chunk-by-chunk propagation exactly.
 //
-//   k_transpose      keys transposed per head (tokens contiguous)
 //   tc_build         per segment on tcgen05: dS = sum phi(k) v^T on the
 //                    half-strip rows (tc_layout.cuh) and dZ = sum k k^T, fp32
+//                    (the key tiles are transposed in shared memory on the way)
 //   tc_seg_scan      exclusive prefix over segments (associative scan) into a
 //                    bf16 copy for the readout, plus the fp32 total
 //   tc_read          per 256 queries: phi(Q) S_prev and q^T Z_prev q on tcgen05
@@ -519,58 +519,24 @@ __device__ __forceinline__ void set_timeout_status(int *status) {
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
 // ---------------------------------------------------------------------------
-// Keys transposed per head: kt[bh][d][t] (tokens contiguous), zero-padded to
-// T_pad (a multiple of 64), so the state builder can read, for a feature
-// index, 16 consecutive tokens as one 32-byte run.
-// grid.x = token-tile (T_pad / 64) + n_tt * bh; block 256.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
-k_transpose(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ kt, int T, int T_pad) {
-    // [token][feature] tile in 32-bit words, even tokens in rows 0..31 and odd
-    // tokens in rows 32..63; rows of 33 words keep both the row-wise writes
-    // and the column-wise reads free of bank conflicts.
-    __shared__ uint32_t tile[64][33];
-    const int n_tt = T_pad / 64;
-    const long long bh = blockIdx.x / n_tt;
-    const int t0 = (blockIdx.x % n_tt) * 64;
-    const uint32_t *src = reinterpret_cast<const uint32_t *>(k);
-    uint32_t in[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {  // 64 tokens x 32 words
-        const int x = threadIdx.x + 256 * r, s = x / 32, w = x % 32, t = t0 + s;
-        in[r] = t < T ? src[((bh * T + t) * kD) / 2 + w] : 0u;
-    }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int x = threadIdx.x + 256 * r, s = x / 32;
-        tile[(s & 1) * 32 + s / 2][x % 32] = in[r];
-    }
-    __syncthreads();
-    uint32_t *dst = reinterpret_cast<uint32_t *>(kt);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {  // 64 features x 32 token pairs
-        const int x = threadIdx.x + 256 * r, d = x / 32, s2 = x % 32;
-        const uint32_t a = tile[s2][d / 2], b2 = tile[32 + s2][d / 2];
-        const uint32_t w = (d & 1) ? ((a >> 16) | (b2 & 0xFFFF0000u)) : ((a & 0xFFFFu) | (b2 << 16));
-        dst[((bh * kD + d) * T_pad + t0) / 2 + s2] = w;
-    }
-}
-
-// ---------------------------------------------------------------------------
 // State builder on tcgen05 (persistent: one CTA per SM loops over work items).
 //
 // Work item = (head, segment, c), c = 0..4; item c accumulates its state
 // tiles (4 tiles for c < 4, the single tile 16 for c = 4; rows as laid out in
 // tc_layout.cuh) over the segment's tokens:  D[m] += A[m] . [V | 1]  with
 // A[m][(i, j)][token] = k_i k_j generated from the transposed keys into tensor
-// memory by the thread owning the row's lane, and the MN-major B operand
+// memory by the thread owning the row's lane (from the key tile transposed in
+// shared memory), and the MN-major B operand
 // [V | 1] = the value tile (64 columns) followed by a constant block whose
 // first column is one, so column 64 of D accumulates the packed normaliser
 // z = sum k_i k_j (N = 80; an N = 64 MMA costs the same issue time).
 // Roles: warps 0-3 / 4-7 generate the first / second 16-token step of every
 // 32-token stage (software-pipelined: the next stage's products are formed
 // while this stage's tensor-memory stores are in flight) and drain the
-// accumulators into swizzled shared memory; warp 8 is the TMA producer;
+// accumulators into swizzled shared memory; warp 8 loads the key and value
+// tiles by TMA and warp 12 transposes each key tile in place once it has
+// landed (d x tokens, so a thread reads 16 consecutive tokens of one feature
+// as one 32-byte run);
 // warps 9 and 10 issue the MMAs of alternate stages; warp 11 writes the
 // drained tiles back with TMA stores, so the next item's MMAs start as soon as
 // the accumulators are read.  Barrier phases run on across items.
@@ -580,7 +546,7 @@ constexpr int kBTiles = 4;                // accumulator tiles (the most an item
 constexpr int kBN = 80;                   // MMA N: 64 values, the ones column, 15 zero columns
 constexpr int kBTok = 64;                 // tokens per TMA tile (2 stages)
 constexpr int kBTileRing = 5;
-constexpr int kBTileBytes = 2 * 8192;     // K^T tile, V tile
+constexpr int kBTileBytes = 2 * 8192;     // key tile (transposed in place), value tile
 constexpr int kBOnes = kBTileRing * kBTileBytes;   // ones block [64 x 64] bf16, swizzled
 constexpr int kBStage = kBOnes + 8192;             // staging: tile m, half h at + (2 m + h) * 16 KB
 constexpr int kBStageBox = 16384;                  // [128 rows x 32 fp32], 128-byte swizzle
@@ -589,15 +555,61 @@ constexpr int kBARing = 3;                // A stages in tensor memory
 constexpr int kBTmaWarp = 8;
 constexpr int kBIssuer0 = 9;
 constexpr int kBStoreWarp = 11;
-constexpr int kBuildThreads = 384;
+constexpr int kBTransWarp = 12;
+constexpr int kBuildThreads = 416;
 constexpr uint32_t kBTmA = kBTiles * kBN; // 320: A slot s at 320 + 64 s, step kk at + 32 kk
 
 struct BuildBars {
-    uint64_t tfull[kBTileRing], tempty[kBTileRing];
+    // kraw: a tile's keys and values landed (the issuers need only the values);
+    // tfull: its keys transposed (the generation warps read them); tempty: the
+    // slot may be refilled
+    uint64_t kraw[kBTileRing], tfull[kBTileRing], tempty[kBTileRing];
     uint64_t afull[kBARing], aempty[kBARing];
     uint64_t done, staged, sfree;
     uint64_t drain[2];
 };
+
+// In-place transpose of one [64 tokens x 64 features] bf16 key tile in the
+// 128-byte swizzle (16-byte chunk c of row r at chunk c ^ (r % 8)) into
+// [64 features x 64 tokens] in the same swizzle, by one warp.  The tile is a
+// grid of 8 x 8 blocks of 8 x 8 elements; block (R, C) (tokens 8R.., features
+// 8C..) becomes block (C, R) transposed.  Lane l + 8 q takes the blocks
+// (l, (l + q) % 8) and (l, (l + q + 4) % 8): in every 8-lane phase of a
+// 16-byte access the lanes touch 8 distinct chunk columns, on the loads
+// (C ^ u) and on the stores (R ^ u), so neither conflicts.  Every lane reads
+// both its blocks before any lane writes.
+__device__ __forceinline__ void transpose_key_tile(uint8_t *tile, int lane) {
+    const int R = lane & 7, q = lane >> 3;
+    uint32_t a[2][8][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int C = (R + q + 4 * h) & 7;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint4 x = *reinterpret_cast<const uint4 *>(tile + (8 * R + u) * 128 + ((C ^ u) * 16));
+            a[h][u][0] = x.x;
+            a[h][u][1] = x.y;
+            a[h][u][2] = x.z;
+            a[h][u][3] = x.w;
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int C = (R + q + 4 * h) & 7;
+        // row v (feature 8C + v) of the transposed block: tokens 2w, 2w + 1 in word w
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const uint32_t sel = (v & 1) ? 0x7632u : 0x5410u;
+            uint4 y;
+            y.x = __byte_perm(a[h][0][v >> 1], a[h][1][v >> 1], sel);
+            y.y = __byte_perm(a[h][2][v >> 1], a[h][3][v >> 1], sel);
+            y.z = __byte_perm(a[h][4][v >> 1], a[h][5][v >> 1], sel);
+            y.w = __byte_perm(a[h][6][v >> 1], a[h][7][v >> 1], sel);
+            *reinterpret_cast<uint4 *>(tile + (8 * C + v) * 128 + ((R ^ v) * 16)) = y;
+        }
+    }
+}
 
 // Products k_i k_j of one 16-token step (this warpgroup's half of a 32-token
 // stage) for the thread's NT rows: p[8 m + w] holds tokens 2 w, 2 w + 1.
@@ -688,7 +700,7 @@ __device__ __forceinline__ void build_item_geom(int item, int n_build, int T, in
 
 template <int G>
 __global__ void __launch_bounds__(kBuildThreads, 1)
-tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUtensorMap tm_v,
+tc_build(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
          const __grid_constant__ CUtensorMap tm_st, float *__restrict__ seg_state, int T, int L,
          int n_seg, int n_build, int n_items, int *status) {
     extern __shared__ uint8_t smem_raw[];
@@ -702,7 +714,8 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
     if (tid == 0) {
         abort_flag = 0;
         for (int x = 0; x < kBTileRing; ++x) {
-            mbar_init(&bars.tfull[x], 1);
+            mbar_init(&bars.kraw[x], 1);
+            mbar_init(&bars.tfull[x], 32);  // every lane of the transposing warp
             mbar_init(&bars.tempty[x], 2);
         }
         for (int x = 0; x < kBARing; ++x) {
@@ -734,10 +747,12 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
 
     if (warp == kBTmaWarp) {
         // ------------------------------------------------------------ producer
+        // the key tile (row-major: zero rows past T) and the value tile of each
+        // 64-token tile, on a CTA-wide tile counter across items
         if (lane == 0) {
-            tma_prefetch_desc(&tm_kt);
+            tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            int tt = 0;  // global tile counter
+            int tt = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
                 int c, g, bh, s0, n_tt;
@@ -747,13 +762,30 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
                     ok = mbar_wait(&bars.tempty[b], ((tt / kBTileRing) & 1) ^ 1, abort);
                     if (!ok) break;
                     uint8_t *st = sm + b * kBTileBytes;
-                    mbar_arrive_expect_tx(&bars.tfull[b], kBTileBytes);
-                    tma_load_3d(st, &tm_kt, &bars.tfull[b], s0 + kBTok * t, 0, bh);
-                    tma_load_3d(st + 8192, &tm_v, &bars.tfull[b], 0, s0 + kBTok * t, bh);
+                    mbar_arrive_expect_tx(&bars.kraw[b], kBTileBytes);
+                    tma_load_3d(st, &tm_k, &bars.kraw[b], 0, s0 + kBTok * t, bh);
+                    tma_load_3d(st + 8192, &tm_v, &bars.kraw[b], 0, s0 + kBTok * t, bh);
                 }
             }
+            // every load issued must have landed before the CTA exits
             for (int t = (tt > kBTileRing ? tt - kBTileRing : 0); t < tt; ++t)
-                mbar_wait_issued(&bars.tfull[t % kBTileRing], (t / kBTileRing) & 1);
+                mbar_wait_issued(&bars.kraw[t % kBTileRing], (t / kBTileRing) & 1);
+        }
+    } else if (warp == kBTransWarp) {
+        // ------------------------------------------------------------ key transposer
+        // each key tile, once landed, transposed in place for the generation warps
+        int tt = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+            int c, g, bh, s0, n_tt;
+            build_item_geom<G>(item, n_build, T, L, c, g, bh, s0, n_tt);
+            for (int t = 0; t < n_tt; ++t, ++tt) {
+                const int b = tt % kBTileRing;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars.kraw[b], (tt / kBTileRing) & 1, abort));
+                if (!ok) break;
+                transpose_key_tile(sm + b * kBTileBytes, lane);
+                mbar_arrive(&bars.tfull[b]);
+            }
         }
     } else if (warp == kBIssuer0 || warp == kBIssuer0 + 1) {
         // ------------------------------------------------------------ MMA issuers
@@ -770,7 +802,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_kt, const __grid_constant__ CUte
                 for (int t = 0; t < n_tt && ok; ++t, ++tt) {
                     const int gs = 2 * tt + me;  // global stage: this issuer takes one half of each tile
                     const int b = tt % kBTileRing, a = gs % kBARing;
-                    ok = mbar_wait(&bars.tfull[b], (tt / kBTileRing) & 1, abort) &&
+                    ok = mbar_wait(&bars.kraw[b], (tt / kBTileRing) & 1, abort) &&
                          mbar_wait(&bars.afull[a], (gs / kBARing) & 1, abort);
                     if (!ok) break;
                     tc_fence_after();
@@ -1386,7 +1418,6 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
     float *seg = w ? reinterpret_cast<float *>(w + p.ws_seg_state) : nullptr;
     float *total = w ? reinterpret_cast<float *>(w + p.ws_total) : nullptr;
     __nv_bfloat16 *prefix = w ? reinterpret_cast<__nv_bfloat16 *>(w + p.ws_extra) : nullptr;
-    __nv_bfloat16 *kt = w ? reinterpret_cast<__nv_bfloat16 *>(w + p.ws_aux) : nullptr;
     const bool readout = out != nullptr;
     const bool want_state = state_out != nullptr;
     const bool has_init = init.n > 0;
@@ -1396,28 +1427,19 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
     const int n_valid = reuse_seg ? p.n_seg : n_build;
     const bool scan = p.n_seg > 1 || has_init;
     const long long BH = p.BH;
-    const int T_pad = (p.T + 63) / 64 * 64;
     int *status = device_status_ptr();
     if (!status) return cudaErrorUnknown;
     if ((has_init || n_build > 0 || want_state || reuse_seg) && !w) return cudaErrorInvalidValue;
 
     if (n_build > 0) {
-        {
-            ProfScope ps("tc_k_transpose", st);
-            k_transpose<<<(unsigned)((T_pad / 64) * BH), 256, 0, st>>>(
-                static_cast<const __nv_bfloat16 *>(k), kt, p.T, T_pad);
-        }
-        CUtensorMap mkt, mvb, mst;
-        const uint64_t dkt[3] = {(uint64_t)T_pad, (uint64_t)kD, (uint64_t)BH};
-        const uint64_t skt[2] = {(uint64_t)T_pad * 2, (uint64_t)kD * T_pad * 2};
-        const uint32_t bkt[3] = {64, 64, 1};
+        CUtensorMap mkb, mvb, mst;
         const uint64_t dqkv[3] = {(uint64_t)kD, (uint64_t)p.T, (uint64_t)BH};
         const uint64_t sqkv[2] = {(uint64_t)kD * 2, (uint64_t)p.T * kD * 2};
         const uint32_t b64[3] = {64, 64, 1};
         const uint64_t dst[3] = {(uint64_t)kD, (uint64_t)state_rows(G), (uint64_t)(BH * p.n_seg)};
         const uint64_t sst[2] = {(uint64_t)kD * 4, (uint64_t)f32_per_seg(G) * 4};
         const uint32_t bst[3] = {32, 128, 1};
-        if (!make_tmap_bf16(&mkt, kt, 3, dkt, skt, bkt) || !make_tmap_bf16(&mvb, v, 3, dqkv, sqkv, b64) ||
+        if (!make_tmap_bf16(&mkb, k, 3, dqkv, sqkv, b64) || !make_tmap_bf16(&mvb, v, 3, dqkv, sqkv, b64) ||
             !make_tmap(&mst, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, seg, 3, dst, sst, bst))
             return cudaErrorInvalidValue;
         cudaError_t e = smem_opt_in_once<tc_build<G>>(kBSmAlloc);
@@ -1425,7 +1447,7 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
         const long long n_items = (long long)build_items(G) * n_build * BH;
         const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
         ProfScope ps(G == 1 ? "tc_build" : "tc_build_m2", st);
-        tc_build<G><<<(unsigned)grid, kBuildThreads, kBSmAlloc, st>>>(mkt, mvb, mst, seg, p.T, p.L, p.n_seg,
+        tc_build<G><<<(unsigned)grid, kBuildThreads, kBSmAlloc, st>>>(mkb, mvb, mst, seg, p.T, p.L, p.n_seg,
                                                                        n_build, (int)n_items, status);
     }
     if (scan) {
@@ -1493,20 +1515,17 @@ int num_sms() {
 //   fp32 segment states  BH * n_seg * R * 65 * 4   (state rows, then packed z)
 //   fp32 total           BH * R * 65 * 4
 //   bf16 prefixes        BH * n_seg * (R + 128) * 64 * 2
-//   transposed keys      BH * 64 * T_pad * 2      (T_pad = T rounded up to 64)
 void plan_tc_workspace(Plan &p) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     const int G = p.g;
     const size_t seg = (size_t)p.BH * p.n_seg * f32_per_seg(G) * 4;
     const size_t tot = (size_t)p.BH * f32_per_seg(G) * 4;
     const size_t pre = (size_t)p.BH * p.n_seg * bf16_per_seg(G) * 2;
-    const size_t T_pad = (size_t)(p.T + 63) / 64 * 64;
-    const size_t kt = (size_t)p.BH * kD * T_pad * 2;
     p.ws_seg_state = 0;
     p.ws_total = up(seg);
     p.ws_extra = p.ws_total + up(tot);
-    p.ws_aux = p.ws_extra + up(pre);
-    p.ws_bytes = p.ws_aux + up(kt);
+    p.ws_aux = 0;
+    p.ws_bytes = p.ws_extra + up(pre);
 }
 
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,

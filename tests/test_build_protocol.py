@@ -3,6 +3,8 @@
 A step-by-step model of every role of the kernel, with its ring sizes,
 barrier counts and phase arithmetic:
 - the TMA producer, which loads key/value tiles into a ring of 5;
+- the transposing warp, which transposes each key tile in place once it has
+  landed and hands it to the generation warps;
 - the two MMA issuers, which take alternate 32-token stages of every tile
   and commit the A slot, the tile and, per work item, `done`;
 - the 8 generation warps, which write the products of each stage into a ring
@@ -15,9 +17,12 @@ last segment, single-tile items).  TMA loads and MMA commits complete at
 random later times (one issuer's commits in order) and the roles interleave
 at random, each at its own random speed.  Checked: no deadlock, every wait
 observes exactly the phase it intends, no drain starts while an MMA of its
-item runs, and no issuer commits before it has issued an MMA (a commit with
-nothing of its own to track is not relied on).  Planted mistakes (the drain not waiting for the staging buffer,
-an issuer waiting for the wrong A-slot phase) must be caught.
+item runs, no issuer commits before it has issued an MMA (a commit with
+nothing of its own to track is not relied on), no key tile is transposed
+before it has landed, and no slot is refilled or rewritten while a generation
+warp still reads its keys.  Planted mistakes (the drain not waiting for the
+staging buffer, an issuer waiting for the wrong A-slot phase, a load not
+waiting for its slot, a transpose not waiting for its keys) must be caught.
 """
 import random
 
@@ -33,7 +38,7 @@ def simulate(items_ntt, seed, prm, planted=None):
     rng = random.Random(seed)
     B = {}
     for x in range(R):
-        B[f"tfull{x}"], B[f"tempty{x}"] = Bar(1), Bar(2)
+        B[f"kraw{x}"], B[f"tfull{x}"], B[f"tempty{x}"] = Bar(1), Bar(32), Bar(2)
     for x in range(A):
         B[f"afull{x}"], B[f"aempty{x}"] = Bar(32 * n_gen), Bar(1)
     B.update(done=Bar(2), staged=Bar(32 * n_gen), sfree=Bar(1), drain0=Bar(1), drain1=Bar(1))
@@ -45,13 +50,22 @@ def simulate(items_ntt, seed, prm, planted=None):
     def W(name, k):  # wait for phase k of `name` (k = -1: the fresh barrier's previous phase)
         return ("wait", name, k)
 
-    def producer():
-        tt = 0
-        for n_tt in items_ntt:
-            for _ in range(n_tt):
+    total = sum(items_ntt)
+    readers = {}  # key tile -> generation warps reading it
+    transposed = set()
+
+    def loader():
+        for tt in range(total):
+            if planted != "load_no_tempty":
                 yield W(f"tempty{tt % R}", tt // R - 1)
-                yield ("load", f"tfull{tt % R}", 2)  # keys^T and values
-                tt += 1
+            yield ("load", tt)  # keys and values, landing on kraw
+
+    def transposer():
+        for tt in range(total):
+            if planted != "transpose_early":
+                yield W(f"kraw{tt % R}", tt // R)
+            yield ("transpose", tt)
+            yield ("arrive", f"tfull{tt % R}", 32)
 
     def issuer(me):
         tt = 0
@@ -59,7 +73,7 @@ def simulate(items_ntt, seed, prm, planted=None):
             for _ in range(n_tt):
                 G = 2 * tt + me
                 a = G % A
-                yield W(f"tfull{tt % R}", tt // R)
+                yield W(f"kraw{tt % R}", tt // R)  # the values
                 # planted: the wait one phase early (it would pass on the slot's previous fill)
                 yield W(f"afull{a}", G // A - 1 if planted == "issuer_phase" else G // A)
                 yield ("mma", me, j)
@@ -74,6 +88,7 @@ def simulate(items_ntt, seed, prm, planted=None):
         tt = 0
         for j, n_tt in enumerate(items_ntt):
             yield W(f"tfull{tt % R}", tt // R)
+            yield ("read_keys", tt)
             for t in range(n_tt):
                 for half in range(2):
                     G = 2 * tt + half
@@ -81,6 +96,9 @@ def simulate(items_ntt, seed, prm, planted=None):
                     yield W(f"aempty{a}", G // A - 1)
                     if half == 1 and t + 1 < n_tt:
                         yield W(f"tfull{(tt + 1) % R}", (tt + 1) // R)
+                        yield ("read_keys", tt + 1)
+                    if half == 0:  # both halves' products of the tile are formed
+                        yield ("keys_read", tt)
                     yield ("arrive", f"afull{a}", 32)
                 tt += 1
             yield W("done", j)
@@ -95,12 +113,13 @@ def simulate(items_ntt, seed, prm, planted=None):
             yield ("read_stage", j)  # the store reads the staging buffer
             yield ("arrive", "sfree", 1)
 
-    agents = {"prod": producer(), "iss0": issuer(0), "iss1": issuer(1), "store": storer()}
+    agents = {"load": loader(), "trans": transposer(), "iss0": issuer(0), "iss1": issuer(1),
+              "store": storer()}
     agents.update({f"gen{w}": gen(w) for w in range(n_gen)})
     cur = dict.fromkeys(agents)
     # each role runs at its own random speed, so that some runs starve one of
     # them (a slow store warp, a slow issuer) and others race ahead
-    role_speed = {r: rng.choice((0.02, 0.2, 1.0)) for r in ("prod", "iss0", "iss1", "store", "gen")}
+    role_speed = {r: rng.choice((0.02, 0.2, 1.0)) for r in ("load", "trans", "iss0", "iss1", "store", "gen")}
     speed = {a: role_speed["gen" if a.startswith("gen") else a] for a in agents}
     loads, commits = [], {"iss0": [], "iss1": []}
     # the staging buffer: which item's rows it holds, and which item the store
@@ -160,10 +179,27 @@ def simulate(items_ntt, seed, prm, planted=None):
             stage["read"] = act[1]
         elif act[0] == "arrive":
             B[act[1]].arrive(act[2])
-        elif act[0] == "load":  # arrive.expect_tx, then the bytes land later
-            B[act[1]].tx += act[2]
-            B[act[1]].arrive()
-            loads.extend([act[1]] * act[2])
+        elif act[0] == "load":  # arrive.expect_tx, then the keys and values land later
+            tt = act[1]
+            if readers.get(tt - R, 0):
+                raise ProtocolError(f"tile {tt} loaded over tile {tt - R} while its keys are read")
+            bar = f"kraw{tt % R}"
+            B[bar].tx += 2
+            B[bar].arrive()
+            loads.extend([bar] * 2)
+        elif act[0] == "transpose":
+            tt = act[1]
+            if B[f"kraw{tt % R}"].phase <= tt // R or B[f"kraw{tt % R}"].tx:
+                raise ProtocolError(f"tile {tt} transposed before its keys landed")
+            if readers.get(tt - R, 0):
+                raise ProtocolError(f"tile {tt} transposed over tile {tt - R} while its keys are read")
+            transposed.add(tt)
+        elif act[0] == "read_keys":
+            if act[1] not in transposed:
+                raise ProtocolError(f"{a} reads the keys of tile {act[1]} before they are transposed")
+            readers[act[1]] = readers.get(act[1], 0) + 1
+        elif act[0] == "keys_read":
+            readers[act[1]] -= 1
         else:
             if not issued[int(a[-1])]:
                 raise ProtocolError(f"{a} commits {act[1]} before issuing any MMA")
@@ -182,7 +218,7 @@ def test_build_protocol_is_deadlock_free_and_phase_exact():
             simulate(items, 100 * seed + c, KERNEL)
 
 
-@pytest.mark.parametrize("mistake", ["drain_no_sfree", "issuer_phase"])
+@pytest.mark.parametrize("mistake", ["drain_no_sfree", "issuer_phase", "load_no_tempty", "transpose_early"])
 def test_model_catches_planted_mistakes(mistake):
     with pytest.raises(ProtocolError):
         for seed in range(40):
