@@ -278,15 +278,16 @@ tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__r
 // Work item = 256 queries (two 128-query tiles) of one segment.  Roles:
 //   warps 0-3 / 4-7  phi(Q) generation, then squared-score masking and the
 //                    epilogue, for tile 0 / tile 1 (thread = query row)
-//   warp 8           TMA producer (Q and the Z prefix into a double-buffered
-//                    item slot, state-prefix stages, K/V blocks)
+//   warp 8           TMA producer (Q into a double-buffered item slot; the
+//                    Z prefix and the state-prefix stages through the prefix
+//                    ring; key and value blocks through rings of their own)
 //   warps 9, 10      MMA issuers.  In the inter phase they take alternate
 //                    stages (so one issuer's wait overlaps the other's queued
-//                    MMAs).  In the intra phase warp 9 issues the scores
-//                    Q K^T of both tiles and warp 10 the weights times
-//                    values P V, so the scores of key block b + 1 run while
-//                    block b is squared, and neither issuer waits right
-//                    behind its own just-committed MMAs.
+//                    MMAs).  In the intra phase, which runs in steps (key
+//                    block, tile) over three score buffers, warp 9 issues
+//                    the scores Q K^T and warp 10 the weights times values
+//                    P V, so the scores of later steps run while earlier
+//                    steps are squared.
 //   warp 11          writes the finished output tiles (staged by the
 //                    epilogue in the item's Q slot) back with TMA stores.
 // Every barrier phase runs on across items.  Accumulators are zeroed by
@@ -297,9 +298,12 @@ tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__r
 constexpr int kQT = 128;                 // query tile (MMA M)
 constexpr int kTiles = 2;                // query tiles per item
 constexpr int kCtaQ = kQT * kTiles;      // 256 queries per item
-constexpr int kKB = 64;                  // key/value block loaded by TMA (one score block)
-constexpr int kKVRing = 4;               // key/value blocks in flight (shared memory)
-constexpr int kSB = 64;                  // score block (MMA N of Q K^T)
+// Keys per intra step (one key/value block, one score buffer): 128 for one
+// factor (scores Q K^T with N = 128), 64 for two (both factors' scores side
+// by side, N = 64 each).
+KATA_HD constexpr int step_keys(int G) { return G == 1 ? 128 : 64; }
+constexpr int kKVMax = 6;                // key (or value) ring slots, the most either form uses
+constexpr int kSBufs = 3;                // score buffers, shared round-robin by the two tiles
 constexpr int kRKs = 8;                  // 16-row K-steps per inter stage (128 state rows)
 // inter stages (128 state rows each): 17 for one factor, 9 for two
 KATA_HD constexpr int read_stages(int G) { return state_rows(G) / (16 * kRKs); }
@@ -312,29 +316,33 @@ constexpr int kStoreWarp = 11;
 constexpr int kReadThreads = 384;
 
 // shared memory (from a 1024-byte aligned base)
-constexpr int kItemBytes = kTiles * 16384 + 16384;  // Q tiles [128 x 64] x 2, Z hi / lo [64 x 64]
+constexpr int kItemBytes = kTiles * 16384;  // Q tiles [128 x 64] x 2
 constexpr int kSmItem = 0;                       // 2 item slots (double buffer)
-constexpr int kSmS = kSmItem + 2 * kItemBytes;   // ring of [128 x 64] state-prefix tiles
-constexpr int kKVBytes = kKB * kD * 2;          // one [64 x 64] bf16 key or value block
-constexpr int kSmK = kSmS + kRBRing * kRStageBytes;  // kKVRing x [64 x 64] keys
-constexpr int kSmV = kSmK + kKVRing * kKVBytes;  // kKVRing x [64 x 64] values
-constexpr int kSmBytes = kSmV + kKVRing * kKVBytes;
+// ring of [128 x 64] state-prefix tiles; an item with a prefix takes 1 +
+// read_stages(G) entries: its Z hi / lo ([64 x 64] each), then the stages
+constexpr int kSmS = kSmItem + 2 * kItemBytes;
+KATA_HD constexpr int kv_bytes(int G) { return step_keys(G) * kD * 2; }  // one key or value block
+constexpr int kKVRingBytes = 49152;              // keys (or values) of the whole ring
+// key (and value) blocks in flight: 3 of 128 keys, or 6 of 64
+KATA_HD constexpr int kv_ring(int G) { return kKVRingBytes / kv_bytes(G); }
+constexpr int kSmK = kSmS + kRBRing * kRStageBytes;  // ring of [step_keys x 64] key blocks
+constexpr int kSmV = kSmK + kKVRingBytes;         // ring of [step_keys x 64] value blocks
+constexpr int kSmBytes = kSmV + kKVRingBytes;
 constexpr int kSmAlloc = kSmBytes + 1024;
 
 // tensor memory columns (512 allocated)
 constexpr uint32_t kTmO = 0;     // O[t]: 64 columns at 64 t
 constexpr uint32_t kTmA = 128;   // inter A slot s: 128 columns at 128 + 128 s (tile t at + 64 t)
 constexpr uint32_t kTmU = 384;   // U[t] = Q Z (before slot 2 is first written): 64 columns at 384 + 64 t
-constexpr uint32_t kTmS = 128;   // intra scores of tile t: 128 columns at 128 + 128 t (see score_depth)
-constexpr uint32_t kTmP = 384;   // intra weights P[t][x] (bf16 pairs): 32 columns at 384 + 64 t + 32 x
-
-// Score buffers per tile in the intra phase.  One factor: two buffers of 64
-// columns (the scores of key block n + 1 are formed while block n is squared).
-// Two factors (KATA-Mg): one buffer of 128 columns holding both factors'
-// scores of a 64-key block side by side; the other tile's buffer gives the
-// overlap.  Either way a tile's score columns are 128 + 128 t .. + 127.
-template <int G>
-__host__ __device__ constexpr int score_depth() { return G == 1 ? 2 : 1; }
+// Intra score buffer x: 128 columns at 128 + 128 x (the inter phase's columns,
+// free once its MMAs are done).  The intra phase runs in steps (key block b,
+// tile t), b-major, on a CTA-wide step count n; step n uses buffer n % 3.
+// One factor: the 128 scores of the step, then its weights (bf16 pairs, 64
+// columns) written over the first half once the squaring warps have read it.
+// Two factors: the two factors' 64 scores side by side, the weights (32
+// columns) over the first quarter.  The weights times values MMAs read them
+// there; the buffer takes new scores once those MMAs are done.
+constexpr uint32_t kTmBuf = 128;
 
 struct ReadBars {
     // ostaged[b]: the output rows of the item in slot b are staged.  One per
@@ -342,11 +350,16 @@ struct ReadBars {
     // neither barrier can complete twice ahead of the store warp's wait.
     uint64_t qfull[2], qempty[2], u, interdone, done, genin, ostaged[2];
     uint64_t bfull[kRBRing], bempty[kRBRing], afull[kRRing], aempty[kRRing];
-    uint64_t kvfull[kKVRing], kvempty[kKVRing];
-    // sfull: scores in a tile's score buffer; sload: the squaring warps have read
-    // them (the buffer may take the next scores); pfull / pempty: the weights
-    // in the tile's weight buffer are stored / consumed by the P-V MMAs
-    uint64_t sfull[kTiles][2], sload[kTiles][2], pfull[kTiles][2], pempty[kTiles][2];
+    // key and value rings apart; the keys of a block free well before its
+    // values.  No commit releases a slot (a commit costs its issuer ~100 cycles
+    // and commits arrive ~200 apart): kempty is a plain arrival by the squaring
+    // warps that saw the block's last scores land, vempty one by issuer 0 when
+    // it has seen the block's last products done (before reusing that buffer).
+    uint64_t kfull[kKVMax], kempty[kKVMax], vfull[kKVMax], vempty[kKVMax];
+    // per score buffer: sfull, the step's scores formed; pfull, its weights
+    // stored over them; bfree, its weights times values done (the buffer may
+    // take the scores of step n + 3)
+    uint64_t sfull[kSBufs], pfull[kSBufs], bfree[kSBufs];
     uint64_t drain[2];
 };
 
@@ -357,6 +370,9 @@ struct ReadItem {
 };
 
 // has_init: the forward starts from a given state, so segment 0 has a prefix too.
+// n_kv: key/value blocks (step_keys(G) keys) from the segment start to the
+// item's last query.
+template <int G>
 __device__ __forceinline__ ReadItem read_item(int i, int n_ct, int T, int L, int n_seg, bool has_init) {
     ReadItem it;
     it.bh = i / n_ct;
@@ -366,7 +382,7 @@ __device__ __forceinline__ ReadItem read_item(int i, int n_ct, int T, int L, int
     it.sidx = it.bh * n_seg + g;
     it.inter = g > 0 || has_init;
     const int tend = min(it.t0 + kCtaQ, T);
-    it.n_kv = (tend - it.seg0 + kKB - 1) / kKB;
+    it.n_kv = (tend - it.seg0 + step_keys(G) - 1) / step_keys(G);
     return it;
 }
 
@@ -400,12 +416,20 @@ __device__ __forceinline__ ReadSched read_sched(int n_items, int n_ct, int n_seg
     return s;
 }
 
-// 64-key score blocks of tile t: keys seg0 .. min(end of tile, T) - 1; none
-// when the tile starts at or after T.
+// Key blocks of tile t: keys seg0 .. min(end of tile, T) - 1; none when the
+// tile starts at or after T.  Tile 0 never has more blocks than tile 1 unless
+// tile 1 has none.
+template <int G>
 __device__ __forceinline__ int read_tile_blocks(const ReadItem &it, int t, int T) {
     const int q0 = it.t0 + kQT * t;
     if (q0 >= T) return 0;
-    return (min(q0 + kQT, T) - it.seg0 + kSB - 1) / kSB;
+    return (min(q0 + kQT, T) - it.seg0 + step_keys(G) - 1) / step_keys(G);
+}
+
+// Steps of an item before its step (key block b, tile t): the steps run
+// b-major over the tiles that have a block b.
+__device__ __forceinline__ int step_before(int b, int t, int nb0, int nb1) {
+    return min(b, nb0) + min(b, nb1) + (t == 1 && b < nb0 ? 1 : 0);
 }
 
 // q_x duplicated into both halves of a bf16 pair.
@@ -930,7 +954,6 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
     uint8_t *sm = align1024(smem_raw);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const ReadSched sched = read_sched(n_items, n_ct, n_seg);
-    constexpr int kSDepth = score_depth<G>();
 
     if (tid == 0) {
         abort_flag = 0;
@@ -939,9 +962,11 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             mbar_init(&bars.qempty[b], 3);  // both issuers' commits + the output store's read
             mbar_init(&bars.drain[b], 1);
         }
-        for (int b = 0; b < kKVRing; ++b) {
-            mbar_init(&bars.kvfull[b], 1);
-            mbar_init(&bars.kvempty[b], 2);  // both issuers' commits
+        for (int b = 0; b < kKVMax; ++b) {
+            mbar_init(&bars.kfull[b], 1);
+            mbar_init(&bars.kempty[b], 1);
+            mbar_init(&bars.vfull[b], 1);
+            mbar_init(&bars.vempty[b], 1);
         }
         mbar_init(&bars.u, 1);
         mbar_init(&bars.interdone, 2);
@@ -957,13 +982,11 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             mbar_init(&bars.afull[s], 8 * 32);
             mbar_init(&bars.aempty[s], 1);
         }
-        for (int t = 0; t < kTiles; ++t)
-            for (int x = 0; x < 2; ++x) {
-                mbar_init(&bars.sfull[t][x], 1);
-                mbar_init(&bars.sload[t][x], 4 * 32);
-                mbar_init(&bars.pfull[t][x], 4 * 32);
-                mbar_init(&bars.pempty[t][x], 1);
-            }
+        for (int x = 0; x < kSBufs; ++x) {
+            mbar_init(&bars.sfull[x], 1);
+            mbar_init(&bars.pfull[x], 4);  // one arrival per squaring warp of the step's tile
+            mbar_init(&bars.bfree[x], 1);
+        }
         fence_mbarrier_init();
     }
     if (warp == kIssuer0) {
@@ -983,42 +1006,50 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_s);
-            int n_q = 0, n_bs = 0, n_kv = 0;  // loads issued into each ring
+            int n_q = 0, n_bs = 0, n_kv = 0, n_v = 0;  // loads issued into each ring (n_kv: keys)
             bool ok = true;
             for (int x = sched.first; x < sched.end && ok; x += sched.stride) {
-                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg, has_init);
+                const ReadItem it = read_item<G>(sched.item(x), n_ct, T, L, n_seg, has_init);
                 {
                     const int qb = n_q & 1;
                     uint8_t *slot = sm + kSmItem + qb * kItemBytes;
                     ok = mbar_wait(&bars.qempty[qb], ((n_q >> 1) & 1) ^ 1, abort);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(&bars.qfull[qb], kTiles * 16384 + (it.inter ? 16384 : 0));
+                    mbar_arrive_expect_tx(&bars.qfull[qb], kTiles * 16384);
                     for (int t = 0; t < kTiles; ++t)
                         tma_load_3d(slot + t * 16384, &tm_q, &bars.qfull[qb], 0, it.t0 + t * kQT, it.bh);
-                    if (it.inter)
-                        for (int zz = 0; zz < 4; ++zz)  // Z hi rows 2560..2623, Z lo rows 2624..2687
-                            tma_load_3d(slot + kTiles * 16384 + zz * 4096, &tm_s, &bars.qfull[qb], 0,
-                                        zhi_row0(G) + 32 * zz, it.sidx);
                     ++n_q;
                 }
-                for (int st = 0; it.inter && st < read_stages(G) && ok; ++st) {
+                // entry -1: Z hi / lo (the 128 prefix rows from zhi_row0); then the stages
+                for (int st = -1; it.inter && st < read_stages(G) && ok; ++st) {
                     const int s = n_bs % kRBRing;
                     ok = mbar_wait(&bars.bempty[s], ((n_bs / kRBRing) & 1) ^ 1, abort);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&bars.bfull[s], kRStageBytes);
+                    const int row0 = st < 0 ? zhi_row0(G) : 16 * kRKs * st;
                     for (int bx = 0; bx < kRStageBytes / 4096; ++bx)
                         tma_load_3d(sm + kSmS + s * kRStageBytes + 4096 * bx, &tm_s, &bars.bfull[s], 0,
-                                    16 * kRKs * st + 32 * bx, it.sidx);
+                                    row0 + 32 * bx, it.sidx);
                     ++n_bs;
                 }
                 for (int kb = 0; kb < it.n_kv && ok; ++kb) {
-                    const int s = n_kv % kKVRing;
-                    ok = mbar_wait(&bars.kvempty[s], ((n_kv / kKVRing) & 1) ^ 1, abort);
+                    const int s = n_kv % kv_ring(G);
+                    const uint32_t par = ((n_kv / kv_ring(G)) & 1) ^ 1;
+                    ok = mbar_wait(&bars.kempty[s], par, abort);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(&bars.kvfull[s], 2 * kKVBytes);
-                    tma_load_3d(sm + kSmK + s * kKVBytes, &tm_k, &bars.kvfull[s], 0, it.seg0 + kb * kKB, it.bh);
-                    tma_load_3d(sm + kSmV + s * kKVBytes, &tm_v, &bars.kvfull[s], 0, it.seg0 + kb * kKB, it.bh);
+                    mbar_arrive_expect_tx(&bars.kfull[s], kv_bytes(G));
+                    tma_load_3d(sm + kSmK + s * kv_bytes(G), &tm_k, &bars.kfull[s], 0,
+                                it.seg0 + kb * step_keys(G), it.bh);
+                    ok = mbar_wait(&bars.vempty[s], par, abort);
+                    if (!ok) {
+                        ++n_kv;  // its keys are in flight: waited for below
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars.vfull[s], kv_bytes(G));
+                    tma_load_3d(sm + kSmV + s * kv_bytes(G), &tm_v, &bars.vfull[s], 0,
+                                it.seg0 + kb * step_keys(G), it.bh);
                     ++n_kv;
+                    ++n_v;
                 }
             }
             // every load issued must have landed before the CTA exits
@@ -1026,22 +1057,28 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                 mbar_wait_issued(&bars.qfull[x & 1], (x >> 1) & 1);
             for (int x = (n_bs > kRBRing ? n_bs - kRBRing : 0); x < n_bs; ++x)
                 mbar_wait_issued(&bars.bfull[x % kRBRing], (x / kRBRing) & 1);
-            for (int x = (n_kv > kKVRing ? n_kv - kKVRing : 0); x < n_kv; ++x)
-                mbar_wait_issued(&bars.kvfull[x % kKVRing], (x / kKVRing) & 1);
+            for (int x = (n_kv > kv_ring(G) ? n_kv - kv_ring(G) : 0); x < n_kv; ++x)
+                mbar_wait_issued(&bars.kfull[x % kv_ring(G)], (x / kv_ring(G)) & 1);
+            for (int x = (n_v > kv_ring(G) ? n_v - kv_ring(G) : 0); x < n_v; ++x)
+                mbar_wait_issued(&bars.vfull[x % kv_ring(G)], (x / kv_ring(G)) & 1);
         }
     } else if (warp == kIssuer0 || warp == kIssuer0 + 1) {
         // ------------------------------------------------------------ MMA issuers
         if (lane == 0) {
             const int me = warp - kIssuer0;
             const uint32_t id_n64 = idesc_bf16(kQT, 64, 0, 1);  // B MN-major, N = 64
-            const uint32_t id_qk = idesc_bf16(kQT, kSB, 0, 0);  // B = keys, K-major
+            // scores: B = keys, K-major; N = 128 keys (one factor) or 64 per factor
+            const uint32_t id_qk = idesc_bf16(kQT, G == 1 ? 128 : 64, 0, 0);
             const uint64_t dS = desc_sw128(smem_u32(sm + kSmS), 8192, 1024);
             const uint64_t dK = desc_sw128(smem_u32(sm + kSmK), 16, 1024);
             const uint64_t dV = desc_sw128(smem_u32(sm + kSmV), 8192, 1024);
-            int n_inter = 0, g_kv = 0, g_b0 = 0, g_b1 = 0, j = 0;
+            int n_inter = 0, g_kv = 0, ns = 0, j = 0;  // ns: the CTA's intra step count
+            // issuer 0, per score buffer (4 bits each): the key/value slot + 1 whose
+            // values the buffer's current step finishes reading, or 0
+            uint32_t vrel = 0;
             bool ok = true;
             for (int x = sched.first; x < sched.end && ok; x += sched.stride, ++j) {
-                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg, has_init);
+                const ReadItem it = read_item<G>(sched.item(x), n_ct, T, L, n_seg, has_init);
                 const int qb = j & 1;
                 const uint32_t slot = smem_u32(sm + kSmItem + qb * kItemBytes);
                 ok = mbar_wait(&bars.qfull[qb], (j >> 1) & 1, abort);
@@ -1055,7 +1092,12 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                             if (!ok) break;
                             tc_fence_after();
                         }
-                        const uint64_t dZ = desc_sw128(slot + kTiles * 16384, 8192, 1024);
+                        // Z hi / lo: the item's first state-prefix ring entry
+                        const int ze = n_inter * (read_stages(G) + 1), zs = ze % kRBRing;
+                        ok = mbar_wait(&bars.bfull[zs], (ze / kRBRing) & 1, abort);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint64_t dZ = desc_add(dS, kRStageBytes * zs);
                         for (int u = 0; u < kTiles; ++u) {
                             const uint64_t dq = desc_sw128(slot + u * 16384, 16, 1024);
 #pragma unroll
@@ -1068,12 +1110,16 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                                        desc_add(dZ, 8192 + 2048 * ks), id_n64, 1);
                         }
                         mma_commit(&bars.u);
+                        mma_commit(&bars.bempty[zs]);
                     }
                     for (int st = me; st < read_stages(G) && ok; st += 2) {
-                        const int ns = n_inter * read_stages(G) + st;
-                        const int s = ns % kRRing, sb = ns % kRBRing;
-                        ok = mbar_wait(&bars.bfull[sb], (ns / kRBRing) & 1, abort) &&
-                             mbar_wait(&bars.afull[s], (ns / kRRing) & 1, abort);
+                        // gs: the CTA's inter stage count (A ring); be: its prefix ring entry
+                        const int gs = n_inter * read_stages(G) + st, be = n_inter * (read_stages(G) + 1) + 1 + st;
+                        const int s = gs % kRRing, sb = be % kRBRing;
+                        // the A stage first: the generation warps start after U, so the
+                        // ring entry before this one (perhaps Z, the other issuer's) is done
+                        ok = mbar_wait(&bars.afull[s], (gs / kRRing) & 1, abort) &&
+                             mbar_wait(&bars.bfull[sb], (be / kRBRing) & 1, abort);
                         if (!ok) break;
                         tc_fence_after();
                         const uint32_t ta = tm + kTmA + 128 * s;
@@ -1094,77 +1140,66 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     tc_fence_after();
                     ++n_inter;
                 }
-                // intra phase over 64-key blocks b (block b uses key/value block b)
-                const int nb[kTiles] = {read_tile_blocks(it, 0, T), read_tile_blocks(it, 1, T)};
-                const int gb[kTiles] = {g_b0, g_b1};
+                // Intra phase, step by step (key block b, tile t; b-major).  Issuer 0
+                // forms the scores of step n in buffer n % 3 once the weights times
+                // values of step n - 3 have freed it; issuer 1 multiplies the step's
+                // weights, stored over its scores, by the values.  Each issuer
+                // releases key/value block b after its last step of the block.
+                const int nb[kTiles] = {read_tile_blocks<G>(it, 0, T), read_tile_blocks<G>(it, 1, T)};
                 const int nbm = max(nb[0], nb[1]);
                 for (int b = 0; b < nbm && ok; ++b) {
-                    // score block b uses key/value block b of the item
-                    const int kvb = g_kv + b, kvs = kvb % kKVRing;
-                    ok = mbar_wait(&bars.kvfull[kvs], (kvb / kKVRing) & 1, abort);
-                    if (me == 0) {
-                        // scores Q K^T into score buffer n % kSDepth of tile t (n = the
-                        // tile's running block count), as soon as the squaring warps have
-                        // loaded block n - kSDepth from that buffer (which may belong to
-                        // the previous item) into registers
-#pragma unroll
-                        for (int t = 0; t < kTiles; ++t)
-                            if (ok && gb[t] + b >= kSDepth && b < nb[t]) {
-                                const int n = gb[t] + b - kSDepth;
-                                ok = mbar_wait(&bars.sload[t][n % kSDepth], (n / kSDepth) & 1, abort);
+                    const int kvb = g_kv + b, kvs = kvb % kv_ring(G);
+                    // issuer 0 reads the block's keys; issuer 1 its values, which the
+                    // squaring warps have seen land before they hand over the weights
+                    if (me == 0) ok = mbar_wait(&bars.kfull[kvs], (kvb / kv_ring(G)) & 1, abort);
+                    for (int t = 0; t < kTiles && ok; ++t) {
+                        if (b >= nb[t]) continue;
+                        const int x = ns % kSBufs;
+                        const uint32_t buf = tm + kTmBuf + 128 * x;
+                        if (me == 0) {
+                            if (ns >= kSBufs) {
+                                ok = mbar_wait(&bars.bfree[x], ((ns - kSBufs) / kSBufs) & 1, abort);
+                                if (!ok) break;
+                                // step ns - 3 was the last of its block: that block's values are read
+                                const uint32_t code = (vrel >> (4 * x)) & 15u;
+                                if (code) mbar_arrive(&bars.vempty[code - 1]);
                             }
-                        if (!ok) break;
-                        tc_fence_after();
-                        const uint64_t dk = desc_add(dK, kKVBytes * kvs);
-#pragma unroll
-                        for (int t = 0; t < kTiles; ++t) {
-                            if (b >= nb[t]) continue;
-                            const int n = gb[t] + b, x = n % kSDepth;
+                            // this step's block slot + 1 if it is the block's last step
+                            // (tile 1's, or tile 0's when tile 1 has no block b), else 0
+                            const bool last = t == 1 || b >= nb[1];
+                            vrel = (vrel & ~(15u << (4 * x))) | ((last ? kvs + 1u : 0u) << (4 * x));
+                            tc_fence_after();
+                            const uint64_t dk = desc_add(dK, kv_bytes(G) * kvs);
                             const uint64_t dQt = desc_sw128(slot + t * 16384, 16, 1024);
                             if constexpr (G == 1) {
 #pragma unroll
                                 for (int ks = 0; ks < 4; ++ks)
-                                    mma_ss(tm + kTmS + 128 * t + 64 * x, desc_add(dQt, 32 * ks),
-                                           desc_add(dk, 32 * ks), id_qk, ks > 0);
+                                    mma_ss(buf, desc_add(dQt, 32 * ks), desc_add(dk, 32 * ks), id_qk, ks > 0);
                             } else {
                                 // one score per factor: coordinates 0-31 (K-steps 0, 1) into
-                                // columns 0-63 of the tile's buffer, 32-63 (K-steps 2, 3) into 64-127
+                                // columns 0-63 of the buffer, 32-63 (K-steps 2, 3) into 64-127
 #pragma unroll
                                 for (int ks = 0; ks < 4; ++ks)
-                                    mma_ss(tm + kTmS + 128 * t + 64 * (ks / 2), desc_add(dQt, 32 * ks),
-                                           desc_add(dk, 32 * ks), id_qk, (ks & 1) != 0);
+                                    mma_ss(buf + 64 * (ks / 2), desc_add(dQt, 32 * ks), desc_add(dk, 32 * ks),
+                                           id_qk, (ks & 1) != 0);
                             }
-                            mma_commit(&bars.sfull[t][x]);
+                            mma_commit(&bars.sfull[x]);
+                        } else {
+                            ok = mbar_wait(&bars.pfull[x], (ns / kSBufs) & 1, abort);
+                            if (!ok) break;
+                            tc_fence_after();
+                            const uint64_t dv = desc_add(dV, kv_bytes(G) * kvs);
+#pragma unroll
+                            for (int ks = 0; ks < step_keys(G) / 16; ++ks)
+                                mma_ts(tm + kTmO + 64 * t, buf + 8 * ks, desc_add(dv, 2048 * ks), id_n64, 1);
+                            mma_commit(&bars.bfree[x]);
                         }
-                    } else {
-                        // weights P (from tensor memory) times values into O[t]
-#pragma unroll
-                        for (int t = 0; t < kTiles; ++t)
-                            if (ok && b < nb[t]) {
-                                const int n = gb[t] + b;
-                                ok = mbar_wait(&bars.pfull[t][n & 1], (n >> 1) & 1, abort);
-                            }
-                        if (!ok) break;
-                        tc_fence_after();
-                        const uint64_t dv = desc_add(dV, kKVBytes * kvs);
-#pragma unroll
-                        for (int t = 0; t < kTiles; ++t) {
-                            if (b >= nb[t]) continue;
-                            const int n = gb[t] + b, x = n & 1;
-#pragma unroll
-                            for (int ks = 0; ks < kSB / 16; ++ks)
-                                mma_ts(tm + kTmO + 64 * t, tm + kTmP + 64 * t + 32 * x + 8 * ks,
-                                       desc_add(dv, 2048 * ks), id_n64, 1);
-                            mma_commit(&bars.pempty[t][x]);
-                        }
+                        ++ns;
                     }
-                    // this issuer is done with key/value block b
-                    mma_commit(&bars.kvempty[kvs]);
+                    if (!ok) break;
                 }
                 if (!ok) break;
                 g_kv += it.n_kv;
-                g_b0 += nb[0];
-                g_b1 += nb[1];
                 // every generation warp has entered this item, so `done` cannot run a phase ahead of it
                 ok = mbar_wait(&bars.genin, j & 1, abort);
                 if (!ok) break;
@@ -1181,7 +1216,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             tma_prefetch_desc(&tm_o);
             int j = 0;
             for (int x = sched.first; x < sched.end; x += sched.stride, ++j) {
-                const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg, has_init);
+                const ReadItem it = read_item<G>(sched.item(x), n_ct, T, L, n_seg, has_init);
                 const int qb = j & 1;
                 if (!mbar_wait(&bars.ostaged[qb], (j >> 1) & 1, abort)) break;
                 for (int t = 0; t < kTiles; ++t)
@@ -1199,8 +1234,6 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         const int row = 32 * qd + lane;
         const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
         const uint32_t tO = tm + kTmO + 64 * t + lane_base;
-        const uint32_t tS = tm + kTmS + 128 * t + lane_base;
-        const uint32_t tP = tm + kTmP + 64 * t + lane_base;
         const uint32_t tU = tm + kTmU + 64 * t + lane_base;
         const uint32_t tA = tm + kTmA + 64 * t + lane_base;
         uint32_t zero[32];
@@ -1210,10 +1243,10 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         tmem_st32(tO, zero);
         tmem_st32(tO + 32, zero);
         tmem_st_wait();
-        int n_inter = 0, g_b = 0, j = 0;
+        int n_inter = 0, ns = 0, g_kv = 0, j = 0;  // ns: the CTA's intra step count
         bool ok = true;
         for (int x = sched.first; x < sched.end && ok; x += sched.stride, ++j) {
-            const ReadItem it = read_item(sched.item(x), n_ct, T, L, n_seg, has_init);
+            const ReadItem it = read_item<G>(sched.item(x), n_ct, T, L, n_seg, has_init);
             const int qb = j & 1;
             if (lane == 0) mbar_arrive(&bars.genin);
             ok = __all_sync(0xffffffffu, mbar_wait(&bars.qfull[qb], (j >> 1) & 1, abort));
@@ -1256,54 +1289,63 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                 ++n_inter;
             }
             float l = 0.f;
-            const int n_b = read_tile_blocks(it, t, T);
+            const int nb0 = read_tile_blocks<G>(it, 0, T), nb1 = read_tile_blocks<G>(it, 1, T);
+            const int n_b = t == 0 ? nb0 : nb1;
             for (int b = 0; b < n_b && ok; ++b) {
-                const int n = g_b + b, x = n & 1, xs = n % kSDepth;
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfull[t][xs], (n / kSDepth) & 1, abort));
+                const int n = ns + step_before(b, t, nb0, nb1), x = n % kSBufs;
+                const uint32_t tB = tm + kTmBuf + 128 * x + lane_base;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars.sfull[x], (n / kSBufs) & 1, abort));
                 if (!ok) break;
+                // the block's last scores have landed: its keys are read
+                if (qd == 0 && lane == 0 && (t == 1 || b >= nb1))
+                    mbar_arrive(&bars.kempty[(g_kv + b) % kv_ring(G)]);
                 tc_fence_after();
-                uint32_t p[32];
-                const int kbs = it.seg0 + kSB * b;
+                const int kbs = it.seg0 + step_keys(G) * b;
                 // every key of the block precedes every query of the tile
-                const bool full = kbs + kSB - 1 <= tq0;
+                const bool full = kbs + step_keys(G) - 1 <= tq0;
                 const int lim = tq - kbs;  // otherwise keys kbs + c with c <= lim are visible
                 // weights w (packed fp32 pairs), four partial row sums
                 uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
                 if constexpr (G == 1) {
-                    // w = s^2
-                    uint32_t r[64];
-                    tmem_ld32(tS + 64 * xs, r);
-                    tmem_ld32(tS + 64 * xs + 32, r + 32);
-                    tmem_ld_wait();
-                    tc_fence_before();
-                    mbar_arrive(&bars.sload[t][xs]);  // the buffer may take the next scores
-                    if (full) {
+                    // w = s^2, 64 keys at a time; each half's weights (bf16 pairs, 32
+                    // columns) go over the scores of keys 0-63, already read
 #pragma unroll
-                        for (int y = 0; y < 32; ++y) {
-                            const uint64_t s2 = f32x2_pack(r[2 * y], r[2 * y + 1]);
-                            const uint64_t w2 = f32x2_mul(s2, s2);
-                            acc[y & 3] = f32x2_add(acc[y & 3], w2);
-                            p[y] = f32x2_to_bf16x2(w2);
-                        }
-                    } else {
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t r[64], p[32];
+                        tmem_ld32(tB + 64 * h, r);
+                        tmem_ld32(tB + 64 * h + 32, r + 32);
+                        tmem_ld_wait();
+                        if (full) {
 #pragma unroll
-                        for (int y = 0; y < 32; ++y) {
-                            const uint32_t m0 = 2 * y <= lim ? r[2 * y] : 0u;
-                            const uint32_t m1 = 2 * y + 1 <= lim ? r[2 * y + 1] : 0u;
-                            const uint64_t s2 = f32x2_pack(m0, m1);
-                            const uint64_t w2 = f32x2_mul(s2, s2);
-                            acc[y & 3] = f32x2_add(acc[y & 3], w2);
-                            p[y] = f32x2_to_bf16x2(w2);
+                            for (int y = 0; y < 32; ++y) {
+                                const uint64_t s2 = f32x2_pack(r[2 * y], r[2 * y + 1]);
+                                const uint64_t w2 = f32x2_mul(s2, s2);
+                                acc[y & 3] = f32x2_add(acc[y & 3], w2);
+                                p[y] = f32x2_to_bf16x2(w2);
+                            }
+                        } else {
+#pragma unroll
+                            for (int y = 0; y < 32; ++y) {
+                                const int c = 64 * h + 2 * y;
+                                const uint32_t m0 = c <= lim ? r[2 * y] : 0u;
+                                const uint32_t m1 = c + 1 <= lim ? r[2 * y + 1] : 0u;
+                                const uint64_t s2 = f32x2_pack(m0, m1);
+                                const uint64_t w2 = f32x2_mul(s2, s2);
+                                acc[y & 3] = f32x2_add(acc[y & 3], w2);
+                                p[y] = f32x2_to_bf16x2(w2);
+                            }
                         }
+                        tmem_st32(tB + 32 * h, p);
                     }
                 } else {
                     // w = a^2 + b^2, a and b the two factors' scores (columns 0-63 and
-                    // 64-127 of the tile's buffer), 32 keys at a time
+                    // 64-127), 32 keys at a time; each half's weights (16 columns) go
+                    // over factor-a scores already read
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        uint32_t ra[32], rb[32];
-                        tmem_ld32(tS + 32 * h, ra);
-                        tmem_ld32(tS + 64 + 32 * h, rb);
+                        uint32_t ra[32], rb[32], p[16];
+                        tmem_ld32(tB + 32 * h, ra);
+                        tmem_ld32(tB + 64 + 32 * h, rb);
                         tmem_ld_wait();
 #pragma unroll
                         for (int y = 0; y < 16; ++y) {
@@ -1313,28 +1355,31 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                             const uint64_t b2 = f32x2_pack(v0 ? rb[2 * y] : 0u, v1 ? rb[2 * y + 1] : 0u);
                             const uint64_t w2 = f32x2_fma(b2, b2, f32x2_mul(a2, a2));
                             acc[y & 3] = f32x2_add(acc[y & 3], w2);
-                            p[16 * h + y] = f32x2_to_bf16x2(w2);
+                            p[y] = f32x2_to_bf16x2(w2);
                         }
+                        tmem_st16(tB + 16 * h, p);
                     }
-                    tc_fence_before();
-                    mbar_arrive(&bars.sload[t][xs]);  // the buffer may take the next scores
                 }
                 {
                     const uint64_t a01 = f32x2_add(acc[0], acc[1]), a23 = f32x2_add(acc[2], acc[3]);
                     const uint64_t a = f32x2_add(a01, a23);
                     l += f32x2_lo(a) + f32x2_hi(a);
                 }
-                // the weights of block n - 2 (same buffer) must have been consumed
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars.pempty[t][x], ((n >> 1) & 1) ^ 1, abort));
-                if (!ok) break;
-                tc_fence_after();
-                tmem_st32(tP + 32 * x, p);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&bars.pfull[t][x]);
+                __syncwarp();
+                if (lane == 0) {
+                    // the block's values have landed (issuer 1, which reads them, learns
+                    // it from pfull: a wait of its own would stall behind its MMAs)
+                    const int kvb = g_kv + b;
+                    ok = mbar_wait(&bars.vfull[kvb % kv_ring(G)], (kvb / kv_ring(G)) & 1, abort);
+                    if (ok) mbar_arrive(&bars.pfull[x]);  // the step's weights are in place
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
             }
             if (!ok) break;
-            g_b += n_b;
+            ns += nb0 + nb1;
+            g_kv += it.n_kv;
             ok = __all_sync(0xffffffffu, mbar_wait(&bars.done, j & 1, abort));
             if (!ok) break;
             tc_fence_after();
@@ -1386,7 +1431,7 @@ bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const
     const uint64_t ds[3] = {(uint64_t)kD, (uint64_t)bf16_rows(G), (uint64_t)(p.BH * p.n_seg)};
     const uint64_t ss[2] = {(uint64_t)kD * 2, (uint64_t)bf16_rows(G) * kD * 2};
     const uint32_t bs[3] = {64, 32, 1};
-    const uint32_t bkv[3] = {64, kKB, 1};
+    const uint32_t bkv[3] = {64, (uint32_t)step_keys(G), 1};
     return make_tmap_bf16(mq, q, 3, dqkv, sqkv, bqkv) && make_tmap_bf16(mk, k, 3, dqkv, sqkv, bkv) &&
            make_tmap_bf16(mv, v, 3, dqkv, sqkv, bkv) &&
            make_tmap_bf16(ms, prefix ? prefix : q, 3, ds, ss, bs) && make_tmap_bf16(mo, out, 3, dqkv, sqkv, bqkv);

@@ -1,34 +1,39 @@
 """Barrier protocol of the persistent tensor-core readout (`tc_read`), on the CPU.
 
 A step-by-step model of every role of the kernel -- TMA producer, the two MMA
-issuers (alternate inter stages; scores Q K^T by issuer 0, reusing a score
-buffer once the squaring warps have loaded it; weights times values by issuer
-1), the output-store warp and the squaring warps -- with the same
-ring sizes, barrier counts and phase arithmetic as the kernel, run over
-sequences of work items (ragged tails, empty second tiles, single-segment
-heads, several items per CTA, the quadratic form's longest-first order, and
-first-segment items with an inter phase when the forward starts from a given
-state).  TMA loads and MMA commits complete
-asynchronously at random later times (one issuer's commits in order), and the
-roles interleave at random, each at its own random speed.  Checked: no deadlock, and every wait observes
-exactly the phase it intends (a barrier never runs two phases past a waiter,
-which a parity wait could not tell apart).  Planted mistakes must be caught:
-the score buffer reused across work items without waiting for its last
-reader, and both item slots' outputs staged on one barrier (a real hazard of
-an earlier version of the kernel, found by this model once each role ran at
-its own speed).  The same model runs the KATA-Mg two-factor configuration
-(9 inter stages, one score buffer per tile).
+issuers (alternate inter stages; in the intra phase, steps (key block b, tile
+t) b-major on three score buffers shared round-robin by the tiles: issuer 0
+forms a step's scores once the buffer's previous step has finished its
+weights times values, issuer 1 multiplies the step's weights, written over its
+scores, by the values), the output-store warp and the squaring warps -- with
+the same ring sizes, barrier counts and phase arithmetic as the kernel, run
+over sequences of work items (ragged tails, empty second tiles,
+single-segment heads, several items per CTA, the quadratic form's
+longest-first order, and first-segment items with an inter phase when the
+forward starts from a given state).  TMA loads and MMA commits complete
+asynchronously at random later times (one issuer's commits in order), and
+the roles interleave at random, each at its own random speed.  Checked: no
+deadlock, every wait observes exactly the phase it intends (a barrier never
+runs two phases past a waiter, which a parity wait could not tell apart:
+each tile waits on only some phases of a buffer's barrier), and no step's
+scores are issued into a buffer whose previous step's products are still
+running, and no key or value block is loaded over one whose scores or
+products are still running.  Planted mistakes must be caught: a score buffer taking new scores
+without waiting for its previous step's products, and both item slots'
+outputs staged on one barrier (a real hazard of an earlier version of the
+kernel, found by this model once each role ran at its own speed).  The same
+model runs the KATA-Mg two-factor configuration (9 inter stages, 64-key
+steps, rings of 6 key and 6 value blocks).
 """
 import random
 
 import pytest
 
-KERNEL = dict(kQT=128, kTiles=2, kSB=64, kKB=64, kKVRing=4, kRStages=17, kRRing=3, kRBRing=4,
-              kItemSlots=2, kSDepth=2)
-# KATA-Mg with two factors: 9 inter stages, and one score buffer per tile
-# (both factors' scores side by side), so a tile's next scores wait for the
-# squaring warps to read the previous block
-KERNEL_M2 = dict(KERNEL, kRStages=9, kSDepth=1)
+KERNEL = dict(kQT=128, kTiles=2, kKB=128, kKVRing=3, kRStages=17, kRRing=3, kRBRing=4,
+              kItemSlots=2, kSBufs=3)
+# KATA-Mg with two factors: 9 inter stages, and 64-key steps (both factors'
+# scores side by side in a buffer) in a ring of 4 key/value blocks
+KERNEL_M2 = dict(KERNEL, kRStages=9, kKB=64, kKVRing=6)
 
 
 class ProtocolError(AssertionError):
@@ -55,17 +60,18 @@ class Bar:
 
 
 def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=False):
-    kQT, kTiles, kSB, kKB = prm['kQT'], prm['kTiles'], prm['kSB'], prm['kKB']
+    kQT, kTiles, kKB, kS = prm['kQT'], prm['kTiles'], prm['kKB'], prm['kSBufs']
     kKVRing, kRStages, kRRing, kRBRing, kSlots = (prm['kKVRing'], prm['kRStages'], prm['kRRing'],
                                                   prm['kRBRing'], prm['kItemSlots'])
-    kCtaQ, kHalves, kGen, D = kQT * kTiles, kKB // kSB, 4 * kTiles, prm['kSDepth']
+    kCtaQ, kGen = kQT * kTiles, 4 * kTiles
     rng = random.Random(seed)
     n_ct = (T + kCtaQ - 1) // kCtaQ
     B = {}
     for b in range(kSlots):
         B[f'qfull{b}'], B[f'qempty{b}'] = Bar(1), Bar(3)
     for b in range(kKVRing):
-        B[f'kvfull{b}'], B[f'kvempty{b}'] = Bar(1), Bar(2)
+        for r in 'kv':  # key and value rings apart; released by plain arrivals
+            B[f'{r}full{b}'], B[f'{r}empty{b}'] = Bar(1), Bar(1)
     B.update(u=Bar(1), interdone=Bar(2), done=Bar(2), genin=Bar(kGen), drain0=Bar(1),
              drain1=Bar(1))
     for b in range(kSlots):  # output rows staged in item slot b
@@ -77,11 +83,11 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
         B[f'bfull{s}'], B[f'bempty{s}'] = Bar(1), Bar(1)
     for s in range(kRRing):
         B[f'afull{s}'], B[f'aempty{s}'] = Bar(kGen * 32), Bar(1)
-    for t in range(kTiles):
-        for x in range(2):
-            B[f'pfull{t}{x}'], B[f'pempty{t}{x}'] = Bar(128), Bar(1)
-        for x in range(D):
-            B[f'sfull{t}{x}'], B[f'sload{t}{x}'] = Bar(1), Bar(128)
+    for x in range(kS):  # score buffers, shared round-robin by the tiles' steps
+        B[f'sfull{x}'], B[f'pfull{x}'], B[f'bfree{x}'] = Bar(1), Bar(4), Bar(1)
+    pv_done = set()  # steps whose weights times values have completed
+    qk_done = set()  # steps whose scores have completed
+    block_steps = {}  # key/value block -> its steps
 
     def item(i):
         t0 = (i % n_ct) * kCtaQ
@@ -91,7 +97,10 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
 
     def blocks(it, t):
         q0 = it['t0'] + kQT * t
-        return 0 if q0 >= T else (min(q0 + kQT, T) - it['seg0'] + kSB - 1) // kSB
+        return 0 if q0 >= T else (min(q0 + kQT, T) - it['seg0'] + kKB - 1) // kKB
+
+    def before(b, t, nb):  # steps of the item before step (b, t), b-major
+        return min(b, nb[0]) + min(b, nb[1]) + (1 if t == 1 and b < nb[0] else 0)
 
     def W(name, k):  # wait for phase k (k = -1: the fresh barrier's "previous" phase)
         return ('wait', name, k)
@@ -102,22 +111,24 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
             it = item(i)
             qb = n_q % kSlots
             yield W(f'qempty{qb}', n_q // kSlots - 1)
-            yield ('load', f'qfull{qb}', kTiles + it['inter'])
+            yield ('load', f'qfull{qb}', kTiles)
             n_q += 1
-            for _ in range(kRStages if it['inter'] else 0):
+            for _ in range(1 + kRStages if it['inter'] else 0):  # Z hi / lo, then the stages
                 s = n_bs % kRBRing
                 yield W(f'bempty{s}', n_bs // kRBRing - 1)
                 yield ('load', f'bfull{s}', 1)
                 n_bs += 1
             for _ in range(it['n_kv']):
                 s = n_kv % kKVRing
-                yield W(f'kvempty{s}', n_kv // kKVRing - 1)
-                yield ('load', f'kvfull{s}', 2)
+                yield W(f'kempty{s}', n_kv // kKVRing - 1)
+                yield ('load', f'kfull{s}', 1, n_kv)
+                yield W(f'vempty{s}', n_kv // kKVRing - 1)
+                yield ('load', f'vfull{s}', 1, n_kv)
                 n_kv += 1
 
     def issuer(me):
-        n_inter = g_kv = 0
-        g_b = [0] * kTiles
+        n_inter = g_kv = ns = 0
+        vrel = [None] * kS  # per buffer: the slot whose values its step finishes reading
         for j, i in enumerate(items):
             it = item(i)
             qb = j % kSlots
@@ -126,38 +137,44 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
                 if me == 0:
                     if j > 0:
                         yield W('done', j - 1)
+                    ze = n_inter * (kRStages + 1)  # Z hi / lo: the item's first prefix entry
+                    yield W(f'bfull{ze % kRBRing}', ze // kRBRing)
                     yield ('commit', 'u')
+                    yield ('commit', f'bempty{ze % kRBRing}')
                 for st in range(me, kRStages, 2):
-                    G = n_inter * kRStages + st
-                    yield W(f'bfull{G % kRBRing}', G // kRBRing)
+                    G, E = n_inter * kRStages + st, n_inter * (kRStages + 1) + 1 + st
                     yield W(f'afull{G % kRRing}', G // kRRing)
-                    yield ('commit', f'bempty{G % kRBRing}')
+                    yield W(f'bfull{E % kRBRing}', E // kRBRing)
+                    yield ('commit', f'bempty{E % kRBRing}')
                     yield ('commit', f'aempty{G % kRRing}')
                 yield ('commit', 'interdone')
                 yield W('interdone', n_inter)
                 n_inter += 1
             nb = [blocks(it, t) for t in range(kTiles)]
-            gb, nbm = list(g_b), max(nb)
-            for b in range(nbm):
-                G, h = g_kv + b // kHalves, b % kHalves
-                if h == 0:
-                    yield W(f'kvfull{G % kKVRing}', G // kKVRing)
+            for b in range(max(nb)):
+                G = g_kv + b
+                if me == 0:  # issuer 1 learns of the values from the squaring warps
+                    yield W(f'kfull{G % kKVRing}', G // kKVRing)
                 for t in range(kTiles):
-                    if b < nb[t]:
-                        reuse = (b >= D) if planted else (gb[t] + b >= D)
-                        if me == 0 and reuse:  # the squaring warps have loaded block n - D
-                            yield W(f'sload{t}{(gb[t] + b - D) % D}', (gb[t] + b - D) // D)
-                        if me == 1:
-                            yield W(f'pfull{t}{(gb[t] + b) & 1}', (gb[t] + b) >> 1)
-                for t in range(kTiles):
-                    if b < nb[t]:
-                        n = gb[t] + b
-                        yield ('commit', f'sfull{t}{n % D}' if me == 0 else f'pempty{t}{n & 1}')
-                if h == kHalves - 1 or b == nbm - 1:
-                    yield ('commit', f'kvempty{G % kKVRing}')
+                    if b >= nb[t]:
+                        continue
+                    n, x = ns + before(b, t, nb), (ns + before(b, t, nb)) % kS
+                    if me == 0:
+                        # the buffer's previous step must have finished its products
+                        # (planted: not waited for)
+                        if n >= kS and not planted:
+                            yield W(f'bfree{x}', (n - kS) // kS)
+                            if vrel[x] is not None:  # step n - 3 ended its block: values read
+                                yield ('arrive', f'vempty{vrel[x]}', 1)
+                        vrel[x] = G % kKVRing if (t == 1 or b >= nb[1]) else None
+                        yield ('qk', n, G)
+                        yield ('commit', (f'sfull{x}', ('qk', n)))
+                    else:
+                        yield W(f'pfull{x}', n // kS)
+                        yield ('mma',)
+                        yield ('commit', (f'bfree{x}', ('pv', n)))
             g_kv += it['n_kv']
-            for t in range(kTiles):
-                g_b[t] += nb[t]
+            ns += nb[0] + nb[1]
             yield W('genin', j)
             yield ('commit', 'done')
             yield ('commit', f'qempty{qb}')
@@ -170,7 +187,7 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
             yield ('arrive', f'qempty{j % kSlots}', 1)
 
     def gen(w):
-        t, n_inter, g_b = w // 4, 0, 0
+        t, n_inter, ns, g_kv = w // 4, 0, 0, 0
         for j, i in enumerate(items):
             it = item(i)
             yield ('arrive', 'genin', 1)
@@ -182,13 +199,18 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
                     yield W(f'aempty{G % kRRing}', G // kRRing - 1)
                     yield ('arrive', f'afull{G % kRRing}', 32)
                 n_inter += 1
-            for b in range(blocks(it, t)):
-                n = g_b + b
-                yield W(f'sfull{t}{n % D}', n // D)
-                yield ('arrive', f'sload{t}{n % D}', 32)
-                yield W(f'pempty{t}{n & 1}', (n >> 1) - 1)
-                yield ('arrive', f'pfull{t}{n & 1}', 32)
-            g_b += blocks(it, t)
+            nb = [blocks(it, 0), blocks(it, 1)]
+            for b in range(nb[t]):
+                n = ns + before(b, t, nb)
+                yield W(f'sfull{n % kS}', n // kS)
+                G = g_kv + b
+                if w % 4 == 0 and (t == 1 or b >= nb[1]):  # the block's last scores: keys read
+                    yield ('arrive', f'kempty{G % kKVRing}', 1)
+                # the block's values landed, then the weights are handed over
+                yield W(f'vfull{G % kKVRing}', G // kKVRing)
+                yield ('arrive', f'pfull{n % kS}', 1)  # weights stored over the scores
+            ns += nb[0] + nb[1]
+            g_kv += it['n_kv']
             yield W('done', j)
             yield ('arrive', osb(j), 1)
 
@@ -216,7 +238,11 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
                 bar.tx -= 1
                 bar.flip()
             else:
-                B[commits[choice].pop(0)].arrive()
+                c = commits[choice].pop(0)
+                if isinstance(c, tuple):  # the scores or products of a step are complete
+                    c, (kind, step) = c
+                    (qk_done if kind == 'qk' else pv_done).add(step)
+                B[c].arrive()
             continue
         a = rng.choice(ready or runnable)
         if cur[a] is not None and B[cur[a][1]].phase != cur[a][2] + 1:
@@ -234,9 +260,23 @@ def simulate(T, L, BH, items, seed, prm, planted=False, init=False, one_ostaged=
         elif act[0] == 'arrive':
             B[act[1]].arrive(act[2])
         elif act[0] == 'load':  # arrive.expect_tx, then the bytes land later
+            if len(act) > 3 and act[3] >= kKVRing:  # a key or value block into a used slot
+                old = block_steps.get(act[3] - kKVRing, [])
+                done_set = qk_done if act[1].startswith('k') else pv_done
+                if len(old) < len(set(old)) or any(n not in done_set for n in old) or not old:
+                    raise ProtocolError(f"block {act[3]} loaded over block {act[3] - kKVRing} "
+                                        f"while MMAs still read its {'keys' if act[1][0] == 'k' else 'values'}")
             B[act[1]].tx += act[2]
             B[act[1]].arrive()
             loads.extend([act[1]] * act[2])
+        elif act[0] == 'qk':
+            n = act[1]
+            block_steps.setdefault(act[2], []).append(n)
+            if n >= kS and n - kS not in pv_done:
+                raise ProtocolError(f"scores of step {n} issued over step {n - kS}'s weights "
+                                    "before its products finished")
+        elif act[0] == 'mma':
+            pass
         else:
             commits[a].append(act[1])
 
@@ -316,7 +356,7 @@ def test_quadratic_schedule_is_deadlock_free_and_phase_exact():
         assert sorted(walked) == list(range(n_ct * BH))  # every item exactly once
 
 
-def test_model_catches_a_score_buffer_reused_across_items():
+def test_model_catches_a_score_buffer_reused_before_its_products():
     with pytest.raises(ProtocolError):
         run_cases(KERNEL, seeds=range(4), planted=True)
 
@@ -332,6 +372,6 @@ def test_two_factor_readout_protocol():
                      KERNEL_M2, init=True)
 
 
-def test_model_catches_a_two_factor_score_buffer_reused_across_items():
+def test_model_catches_a_two_factor_score_buffer_reused_before_its_products():
     with pytest.raises(ProtocolError):
         run_cases(KERNEL_M2, seeds=range(4), planted=True)
