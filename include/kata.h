@@ -122,9 +122,10 @@ size_t kata_chunked_forward_workspace_bytes(int B, int H, int T, int dk, int dv,
  *          that is 0).  Its contents on entry do not matter.
  *
  * dtype KATA_BF16 runs the tensor-core (tcgen05) path: d = 64 directly,
- * d = 16 and 32 with the heads zero-padded to 64 inside the workspace (exact:
- * zeros add nothing to any product or sum).  KATA_F32 runs fp32 CUDA-core
- * arithmetic end to end.
+ * d = 16 and 32 read as 64 by the kernels' tensor maps, which fill the
+ * columns past d with zeros (exact: zeros add nothing to any product or sum;
+ * the output store writes only the first d columns).  KATA_F32 runs fp32
+ * CUDA-core arithmetic end to end.
  */
 kata_status kata_chunked_forward(const void *q, const void *k, const void *v, void *out, int B,
                                  int H, int T, int dk, int dv, int C, kata_dtype dtype,

@@ -74,7 +74,7 @@ bool device_ptrs_ok(std::initializer_list<const void *> ptrs) {
 }
 
 kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype, Plan &p,
-                      bool padded_ok) {
+                      bool small_tc) {
     if (B < 1 || H < 1 || T < 1 || dk < 1 || dv < 1) return KATA_ERR_INVALID_ARG;
     if (!valid_chunk(C)) return KATA_ERR_INVALID_ARG;
     if (dtype != KATA_F32 && dtype != KATA_BF16) return KATA_ERR_UNSUPPORTED;
@@ -89,14 +89,18 @@ kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dty
     p.C = C;
     p.dtype = dtype;
     p.BH = BH;
-    p.R = packed_rows(dk);
-    p.L = segment_length(dk, C);
-    p.n_seg = (T + p.L - 1) / p.L;
-    p.path = (dtype == KATA_BF16 && dk == 64) ? Path::kTensorCore : Path::kSimt;
+    p.path = (dtype == KATA_BF16 && (dk == 64 || small_tc)) ? Path::kTensorCore : Path::kSimt;
     if (p.path == Path::kTensorCore) {
+        // the tensor-core kernels compute every head as d = 64
+        p.R = packed_rows(64);
+        p.L = segment_length(64, C);
+        p.n_seg = (T + p.L - 1) / p.L;
         tc::plan_tc_workspace(p);
         return KATA_OK;
     }
+    p.R = packed_rows(dk);
+    p.L = segment_length(dk, C);
+    p.n_seg = (T + p.L - 1) / p.L;
     const size_t E = (size_t)p.R * (dv + 1);
     const size_t seg_bytes = (size_t)BH * p.n_seg * E * sizeof(float);
     const size_t total_bytes = (size_t)BH * E * sizeof(float);  // also for one segment + initial state
@@ -105,24 +109,13 @@ kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dty
     p.ws_extra = p.ws_total + align_up(total_bytes);
     p.ws_aux = 0;
     p.ws_bytes = p.ws_extra;
-    if (dtype == KATA_BF16) {
-        // the padded tensor-core route: q, k, v and out padded to d = 64, then
-        // the d = 64 plan's workspace (its layout is recomputed at launch)
-        Plan p64;
-        if (make_plan(B, H, T, 64, 64, C, dtype, p64) != KATA_OK) return KATA_ERR_UNSUPPORTED;
-        const size_t pad = 4 * align_up((size_t)BH * T * 64 * 2);
-        p.ws_aux = pad;  // offset of the d = 64 workspace
-        const size_t padded_bytes = pad + p64.ws_bytes;
-        if (padded_bytes > p.ws_bytes) p.ws_bytes = padded_bytes;
-        if (padded_ok) p.path = Path::kPaddedTensorCore;
-    }
     return KATA_OK;
 }
 
 // KATA-Mg with g factors: g = 1 is the plain plan.  g = 2: bf16 heads of
 // d = 64 take the tensor-core path (its two-factor layout); every other head
-// size and dtype takes the fp32 CUDA-core path (the padded route would put
-// the factor boundary in the wrong place).  Other g: unsupported.
+// size and dtype takes the fp32 CUDA-core path (the tensor-core kernels'
+// d = 64 view of a smaller head would put the factor boundary at 32, not d/2).  Other g: unsupported.
 kata_status make_plan_mg(int B, int H, int T, int dk, int dv, int C, int g, kata_dtype dtype,
                          Plan &p) {
     if (g == 1) return make_plan(B, H, T, dk, dv, C, dtype, p);
@@ -148,7 +141,7 @@ kata_status make_plan_mg(int B, int H, int T, int dk, int dv, int C, int g, kata
 // The quadratic form is the chunked plan with one segment spanning the whole
 // sequence: no state is built, scanned or stored, so no workspace is used.
 kata_status make_quadratic_plan(int B, int H, int T, int dk, int dv, kata_dtype dtype, Plan &p) {
-    const kata_status s = make_plan(B, H, T, dk, dv, 256, dtype, p, false);
+    const kata_status s = make_plan(B, H, T, dk, dv, 256, dtype, p);
     if (s != KATA_OK) return s;
     p.L = T;
     p.n_seg = 1;
@@ -179,10 +172,6 @@ kata_status check_forward_io(const Plan &p, const void *q, const void *k, const 
 cudaError_t launch_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
                            float *state_out, float *z_out, const InitState &init, void *ws,
                            cudaStream_t st, bool reuse_seg = false) {
-    if (p.path == Path::kPaddedTensorCore)
-        return init.n == 0 && out != nullptr && !reuse_seg
-                   ? launch_padded_forward(p, q, k, v, out, state_out, z_out, ws, st)
-                   : cudaErrorInvalidValue;  // the padded route serves the plain forward only
     return p.path == Path::kTensorCore
                ? tc::launch_tc_forward(p, q, k, v, out, state_out, z_out, init, ws, st, reuse_seg)
                : launch_simt_forward(p, q, k, v, out, state_out, z_out, init, ws, st);
@@ -348,7 +337,7 @@ kata_status kata_chunked_state(const void *k, const void *v, int B, int H, int T
                                int C, kata_dtype dtype, float *state_out, float *z_out,
                                void *workspace, size_t workspace_bytes, kata_stream_t stream) {
     Plan p;
-    const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p, false);
+    const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p);
     if (ps != KATA_OK) return ps;
     if (!k || !v || !aligned16(k) || !aligned16(v)) return KATA_ERR_INVALID_ARG;
     const kata_status so = kata::check_state_out(p, state_out, z_out, nullptr, k, v, true);
@@ -372,7 +361,7 @@ kata_status kata_chunked_forward_from_state(const void *q, const void *k, const 
                                             unsigned flags, kata_stream_t stream) {
     Plan p;
     if (flags & ~KATA_REUSE_SEGMENT_STATES) return KATA_ERR_INVALID_ARG;
-    const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p, false);
+    const kata_status ps = kata::make_plan(B, H, T, dk, dv, C, dtype, p);
     if (ps != KATA_OK) return ps;
     const kata_status io = kata::check_forward_io(p, q, k, v, out);
     if (io != KATA_OK) return io;
@@ -398,6 +387,7 @@ kata_status kata_chunked_forward_from_state(const void *q, const void *k, const 
              overlaps(z_out, nz, state_in, span_s) || overlaps(z_out, nz, z_in, span_z)))
             return KATA_ERR_INVALID_ARG;
         init.s = state_in;
+        init.d = dk;
         init.z = z_in;
         init.n = n_in;
         init.s_stride = (long long)s_stride;

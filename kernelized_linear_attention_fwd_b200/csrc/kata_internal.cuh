@@ -59,9 +59,10 @@ __host__ __device__ inline int packed_row_index_g(int d, int G, int i, int j) {
 // ---------------------------------------------------------------------------
 // Forward plan: segment length, number of segments, workspace layout.
 // ---------------------------------------------------------------------------
-// kPaddedTensorCore: bf16 heads of d = 16 or 32 zero-padded to 64 and run on
-// the tensor-core kernels (zeros add nothing to any product or sum).
-enum class Path : int { kSimt = 0, kTensorCore = 1, kPaddedTensorCore = 2 };
+// kTensorCore: bf16 heads of d = 64, and of d = 16 or 32 read as 64 by the
+// tensor maps (TMA fills the columns past d with zeros, which add nothing to
+// any product or sum; the output store writes only the first d columns).
+enum class Path : int { kSimt = 0, kTensorCore = 1 };
 
 struct Plan {
     int B, H, T, dk, dv, C;
@@ -69,23 +70,23 @@ struct Plan {
     long long BH;
     int L;      // segment length (tokens), a multiple of C and of 128; T in the quadratic plan
     int n_seg;  // ceil(T / L)
-    int R;      // packed feature rows
+    int R;      // packed feature rows (of d = 64 on the tensor-core path)
     int g = 1;  // rank-one PSD factors per head (KATA-Mg; 1 = the single factor)
     Path path;
     // workspace (bytes from the base, all 256-byte aligned)
     size_t ws_seg_state;  // fp32 per-segment states, exclusive prefix after the scan
     size_t ws_total;      // fp32 total state (packed), when needed
     size_t ws_extra;      // path-specific
-    size_t ws_aux;        // path-specific (padded route: the d = 64 workspace)
+    size_t ws_aux;        // path-specific (unused)
     size_t ws_bytes;
 };
 
-// Fills `p`; returns KATA_OK or the error the forward must return.  padded_ok:
-// bf16 heads of d < 64 may take the padded tensor-core route (the plain
-// forward); otherwise they take the fp32 CUDA-core path.  The workspace size
-// covers both routes either way, so one size query serves every entry point.
+// Fills `p`; returns KATA_OK or the error the forward must return.  small_tc:
+// bf16 heads of d < 64 run the tensor-core kernels (read as 64 by the tensor
+// maps); without it (KATA-Mg, whose factors split the head at d / 2) they
+// take the fp32 CUDA-core path.
 kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dtype, Plan &p,
-                      bool padded_ok = true);
+                      bool small_tc = true);
 // The plan of the quadratic form: one segment of T tokens, no workspace.
 kata_status make_quadratic_plan(int B, int H, int T, int dk, int dv, kata_dtype dtype, Plan &p);
 
@@ -139,14 +140,16 @@ __device__ __forceinline__ void store_out(__nv_bfloat16 *p, long long i, float x
     p[i] = __float2bfloat16_rn(x);
 }
 
-// Initial state of a forward: the sum of n dense states, S [B, H, dk*dk, dv]
-// and Z [B, H, dk, dk] fp32; input m starts s_stride (z_stride) floats after
-// input m - 1.  n = 0: the forward starts from the empty state.
+// Initial state of a forward: the sum of n dense states, S [B, H, d*d, d]
+// and Z [B, H, d, d] fp32 (d = the plan's dk); input m starts s_stride
+// (z_stride) floats after input m - 1.  n = 0: the forward starts from the
+// empty state.
 struct InitState {
     const float *s = nullptr;
     const float *z = nullptr;
     int n = 0;
     long long s_stride = 0, z_stride = 0;
+    int d = 64;
 };
 
 // Launchers (return cudaSuccess or the launch error).  out == nullptr skips
@@ -155,25 +158,19 @@ cudaError_t launch_simt_forward(const Plan &p, const void *q, const void *k, con
                                 void *out, float *state_out, float *z_out, const InitState &init,
                                 void *ws, cudaStream_t st);
 namespace tc {
-// Tensor-core path (bf16, d = dv = 64): workspace layout and launcher.
+// Tensor-core path (bf16, d = dv in {16, 32, 64}, computed as 64): workspace
+// layout and launcher.
 // reuse_seg: the workspace already holds every segment's state, written by a
 // state-only launch for the same keys, values and sizes; skip building them.
 void plan_tc_workspace(Plan &p);
-// d_out: head size of the exported state (< 64 when the heads were padded).
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v,
                               void *out, float *state_out, float *z_out, const InitState &init,
-                              void *ws, cudaStream_t st, bool reuse_seg = false, int d_out = 64);
+                              void *ws, cudaStream_t st, bool reuse_seg = false);
 // Streaming multiprocessors of the current device (cached).
 int num_sms();
 }  // namespace tc
 
 // Decode step on the dense (d^2 rows) or packed (d(d+1)/2 rows) state layout.
-// The plain forward of bf16 heads of d < 64, zero-padded to 64 in the
-// workspace and run on the tensor-core kernels.
-cudaError_t launch_padded_forward(const Plan &p, const void *q, const void *k, const void *v,
-                                  void *out, float *state_out, float *z_out, void *ws,
-                                  cudaStream_t st);
-
 cudaError_t launch_decode(int B, int H, int dk, int dv, kata_dtype dtype, const void *q,
                           const void *k, const void *v, void *out, float *state, float *z,
                           bool packed, cudaStream_t st);

@@ -16,7 +16,7 @@
 //                    (phi(Q) generated from registers into tensor memory), the
 //                    intra-segment squared-score term on tcgen05, the division
 //   tc_state_expand  fp32 total -> dense [d*d, d] state and [d, d] Z (d <= 64:
-//                    heads zero-padded to 64 export their leading d x d part)
+//                    heads of d < 64, computed as 64, export their leading d x d part)
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -79,22 +79,26 @@ struct ScanLane {
         }
     }
 
-    // The initial state of these 4 packed elements: the sum of n_in dense states.
+    // The initial state of these 4 packed elements: the sum of n_in dense states
+    // of head size d (<= 64: the coordinates past d are zero).
     __device__ __forceinline__ float4 init(long long bh, const float *init_s, const float *init_z,
-                                           int n_in, long long s_stride, long long z_stride) const {
+                                           int n_in, long long s_stride, long long z_stride,
+                                           int d) const {
         float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int n = 0; n < n_in; ++n) {
             if (!z_part) {
                 const PairIJ pij = row_ij_g(G, (int)(e0 / kD));
-                if (pij.i <= pij.j)
+                const int e = (int)(e0 % kD);  // 4 consecutive values, all below d or none
+                if (pij.i <= pij.j && pij.j < d && e < d)
                     carry = f4add(carry, *reinterpret_cast<const float4 *>(
                                              init_s + n * s_stride +
-                                             ((bh * kD + pij.i) * kD + pij.j) * kD + e0 % kD));
+                                             ((bh * d + pij.i) * d + pij.j) * d + e));
             } else {
-                const float *zn = init_z + n * z_stride + bh * kD * kD;
+                const float *zn = init_z + n * z_stride + bh * d * d;
                 float zv[4];
 #pragma unroll
-                for (int x = 0; x < 4; ++x) zv[x] = zi[x] <= zj[x] ? zn[zi[x] * kD + zj[x]] : 0.f;
+                for (int x = 0; x < 4; ++x)
+                    zv[x] = zi[x] <= zj[x] && zj[x] < d ? zn[zi[x] * d + zj[x]] : 0.f;
                 carry = f4add(carry, make_float4(zv[0], zv[1], zv[2], zv[3]));
             }
         }
@@ -146,7 +150,8 @@ template <int G, int RUN>
 __global__ void __launch_bounds__(256, RUN == 2 ? 5 : RUN == 4 ? 4 : 2)  // blocks per SM without spills
 tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ prefix,
             float *__restrict__ total, int n_seg, int n_valid, const float *__restrict__ init_s,
-            const float *__restrict__ init_z, int n_in, long long s_stride, long long z_stride) {
+            const float *__restrict__ init_z, int n_in, long long s_stride, long long z_stride,
+            int d_in) {
     __shared__ float4 part[2][kScanWarps][32];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     constexpr long long E = f32_per_seg(G);
@@ -157,7 +162,7 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
     const ScanLane<G> sl(eb * 128 + 4 * lane);
     const float *base = seg_state + bh * (long long)n_seg * E + sl.e0;
     __nv_bfloat16 *pbase = prefix ? prefix + bh * (long long)n_seg * bf16_per_seg(G) : nullptr;
-    float4 carry = sl.init(bh, init_s, init_z, n_in, s_stride, z_stride);
+    float4 carry = sl.init(bh, init_s, init_z, n_in, s_stride, z_stride, d_in);
     const int g_first = n_in > 0 ? 0 : 1;  // without one, segment 0 has an empty prefix
 
     for (int g0 = 0; g0 < n_seg; g0 += kScanWarps * RUN) {
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(256, RUN <= 4 ? 4 : 2)
 tc_seg_scan_short(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ prefix,
                   float *__restrict__ total, int n_seg, int n_valid, long long BH,
                   const float *__restrict__ init_s, const float *__restrict__ init_z, int n_in,
-                  long long s_stride, long long z_stride) {
+                  long long s_stride, long long z_stride, int d_in) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     constexpr long long E = f32_per_seg(G);
     constexpr long long n_eb = E / 128;
@@ -230,7 +235,7 @@ tc_seg_scan_short(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict
     for (int i = 0; i < RUN; ++i)
         v[i] = i < n_valid ? *reinterpret_cast<const float4 *>(base + (long long)i * E)
                            : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 run = sl.init(bh, init_s, init_z, n_in, s_stride, z_stride);
+    float4 run = sl.init(bh, init_s, init_z, n_in, s_stride, z_stride, d_in);
     const int g_first = n_in > 0 ? 0 : 1;
 #pragma unroll
     for (int i = 0; i < RUN; ++i) {
@@ -243,7 +248,8 @@ tc_seg_scan_short(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict
 
 // ---------------------------------------------------------------------------
 // fp32 total (packed rows) -> dense state [D*D][D] and Z [D][D].  D < 64: the
-// heads were zero-padded to 64, and the leading D x D part is exported.  G
+// heads were computed as 64 (columns past D zero), and the leading D x D part
+// is exported.  G
 // factors (KATA-Mg): pairs across factors are not in the layout and export 0.
 // D is a template parameter so the index arithmetic divides by constants.
 // ---------------------------------------------------------------------------
@@ -1425,8 +1431,10 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
 template <int G>
 bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const void *prefix, void *out,
                CUtensorMap *mq, CUtensorMap *mk, CUtensorMap *mv, CUtensorMap *ms, CUtensorMap *mo) {
-    const uint64_t dqkv[3] = {(uint64_t)kD, (uint64_t)p.T, (uint64_t)p.BH};
-    const uint64_t sqkv[2] = {(uint64_t)kD * 2, (uint64_t)p.T * kD * 2};
+    // inner extent d (the boxes stay 64 wide: columns past d read as zeros, and
+    // the output store writes only the first d)
+    const uint64_t dqkv[3] = {(uint64_t)p.dk, (uint64_t)p.T, (uint64_t)p.BH};
+    const uint64_t sqkv[2] = {(uint64_t)p.dk * 2, (uint64_t)p.T * p.dk * 2};
     const uint32_t bqkv[3] = {64, 128, 1};
     const uint64_t ds[3] = {(uint64_t)kD, (uint64_t)bf16_rows(G), (uint64_t)(p.BH * p.n_seg)};
     const uint64_t ss[2] = {(uint64_t)kD * 2, (uint64_t)bf16_rows(G) * kD * 2};
@@ -1457,7 +1465,10 @@ cudaError_t launch_expand(const float *src, long long stride, float *state_out, 
 template <int G>
 cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, const void *v, void *out,
                                 float *state_out, float *z_out, const InitState &init, void *ws,
-                                cudaStream_t st, bool reuse_seg, int d_out) {
+                                cudaStream_t st, bool reuse_seg) {
+    // heads of d < 64 are read as 64 by every tensor map (TMA zero-fills the
+    // columns past d) and exported at their own size
+    const int d_out = p.dk;
     // no workspace (the quadratic plan): no state is built, scanned or read
     char *w = static_cast<char *>(ws);
     float *seg = w ? reinterpret_cast<float *>(w + p.ws_seg_state) : nullptr;
@@ -1478,8 +1489,8 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
 
     if (n_build > 0) {
         CUtensorMap mkb, mvb, mst;
-        const uint64_t dqkv[3] = {(uint64_t)kD, (uint64_t)p.T, (uint64_t)BH};
-        const uint64_t sqkv[2] = {(uint64_t)kD * 2, (uint64_t)p.T * kD * 2};
+        const uint64_t dqkv[3] = {(uint64_t)p.dk, (uint64_t)p.T, (uint64_t)BH};
+        const uint64_t sqkv[2] = {(uint64_t)p.dk * 2, (uint64_t)p.T * p.dk * 2};
         const uint32_t b64[3] = {64, 64, 1};
         const uint64_t dst[3] = {(uint64_t)kD, (uint64_t)state_rows(G), (uint64_t)(BH * p.n_seg)};
         const uint64_t sst[2] = {(uint64_t)kD * 4, (uint64_t)f32_per_seg(G) * 4};
@@ -1505,14 +1516,14 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
             auto kern = p.n_seg <= 4 ? tc_seg_scan_short<G, 4>
                         : p.n_seg <= 8 ? tc_seg_scan_short<G, 8> : tc_seg_scan_short<G, 16>;
             kern<<<(unsigned)grid, 256, 0, st>>>(seg, pre, tot, p.n_seg, n_valid, BH, init.s, init.z,
-                                                 init.n, init.s_stride, init.z_stride);
+                                                 init.n, init.s_stride, init.z_stride, init.d);
         } else {
             const long long grid = (f32_per_seg(G) / 128) * BH;
             auto kern = p.n_seg <= 4 * kScanWarps ? tc_seg_scan<G, 4>
                         : p.n_seg <= 8 * kScanWarps ? tc_seg_scan<G, 8>
                                                     : tc_seg_scan<G, 16>;
             kern<<<(unsigned)grid, 256, 0, st>>>(seg, pre, tot, p.n_seg, n_valid, init.s, init.z,
-                                                 init.n, init.s_stride, init.z_stride);
+                                                 init.n, init.s_stride, init.z_stride, init.d);
         }
     }
     if (readout) {
@@ -1575,10 +1586,10 @@ void plan_tc_workspace(Plan &p) {
 
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
                               float *state_out, float *z_out, const InitState &init, void *ws,
-                              cudaStream_t st, bool reuse_seg, int d_out) {
+                              cudaStream_t st, bool reuse_seg) {
     switch (p.g) {
-        case 1: return launch_tc_forward_g<1>(p, q, k, v, out, state_out, z_out, init, ws, st, reuse_seg, d_out);
-        case 2: return launch_tc_forward_g<2>(p, q, k, v, out, state_out, z_out, init, ws, st, reuse_seg, d_out);
+        case 1: return launch_tc_forward_g<1>(p, q, k, v, out, state_out, z_out, init, ws, st, reuse_seg);
+        case 2: return launch_tc_forward_g<2>(p, q, k, v, out, state_out, z_out, init, ws, st, reuse_seg);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -81,17 +81,15 @@ def test_workspace_query(lib):
     assert W(1, 8, 131072, 64, 64, 4096, 1) > 0 and W(1, 8, 131072, 64, 64, 8192, 1) == 0
 
 
-def test_workspace_covers_both_routes_for_small_bf16_heads(lib):
-    # bf16 heads of d < 64: the chunked forward pads them to 64 on the tensor
-    # cores (four padded q/k/v/out slabs, then the d = 64 workspace), the
-    # state-only and from-state calls keep the fp32 CUDA-core layout (the same
-    # as for fp32 inputs); one size query must cover both
+def test_small_bf16_heads_take_the_d64_tensor_core_workspace(lib):
+    # bf16 heads of d < 64 run the tensor-core kernels, which read them as
+    # d = 64 (the tensor maps zero-fill the columns past d): the same workspace
+    # as d = 64, with no padded copies; fp32 keeps its CUDA-core layout
     W = lib.kata_chunked_forward_workspace_bytes
-    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
     for B, H, T, d in [(2, 4, 4096, 32), (1, 3, 1000, 16), (1, 1, 1, 32), (4, 2, 2049, 16)]:
-        padded = 4 * up(B * H * T * 64 * 2) + W(B, H, T, 64, 64, 64, 1)
-        cuda_core = W(B, H, T, d, d, 64, 0)
-        assert W(B, H, T, d, d, 64, 1) == max(padded, cuda_core)
+        for C in (64, 512):
+            assert W(B, H, T, d, d, C, 1) == W(B, H, T, 64, 64, C, 1)
+        assert W(B, H, T, d, d, 64, 0) < W(B, H, T, 64, 64, 64, 0)
 
 
 FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced: every call below fails first
