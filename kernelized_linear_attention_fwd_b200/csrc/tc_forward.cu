@@ -253,26 +253,38 @@ tc_seg_scan_short(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict
 // factors (KATA-Mg): pairs across factors are not in the layout and export 0.
 // D is a template parameter so the index arithmetic divides by constants.
 // ---------------------------------------------------------------------------
+// A thread writes 4 consecutive outputs (one 16-byte store: the outputs are
+// 16-byte aligned, and D, the packed row length and the per-head strides are
+// multiples of 4).
 template <int G, int D>
 __global__ void __launch_bounds__(256)
 tc_state_expand(const float *__restrict__ total, long long stride_bh, float *__restrict__ state_out,
                 float *__restrict__ z_out, long long BH) {
-    constexpr long long d3 = (long long)D * D * D, per = d3 + (long long)D * D;
+    constexpr int d3 = D * D * D, per4 = (d3 + D * D) / 4;
     const long long idx = (long long)blockIdx.x * 256 + threadIdx.x;
-    if (idx >= per * BH) return;
-    const long long bh = idx / per;
-    long long x = idx % per;
+    if (idx >= (long long)per4 * BH) return;
+    const long long bh = idx / per4;
+    const int x = 4 * (int)(idx % per4);
     const float *src = total + bh * stride_bh;
     if (x < d3) {
-        const int row = (int)(x / D), e = (int)(x % D);
+        // values e .. e + 3 of dense row (i, j): the packed row of the pair
+        const int row = x / D, e = x % D;
         int i = row / D, j = row % D;
         if (i > j) { const int t = i; i = j; j = t; }
-        state_out[bh * d3 + x] = same_factor(G, i, j) ? src[(long long)row_index_g(G, i, j) * kD + e] : 0.f;
+        const float4 v = same_factor(G, i, j)
+                             ? *reinterpret_cast<const float4 *>(src + (long long)row_index_g(G, i, j) * kD + e)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(state_out + bh * d3 + x) = v;
     } else {
-        x -= d3;
-        int i = (int)(x / D), j = (int)(x % D);
-        if (i > j) { const int t = i; i = j; j = t; }
-        z_out[bh * D * D + x] = same_factor(G, i, j) ? src[z_packed0(G) + row_index_g(G, i, j)] : 0.f;
+        // Z[i][j0 .. j0 + 3]
+        const int xz = x - d3, i = xz / D, j0 = xz % D;
+        float z[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int a = min(i, j0 + u), b = max(i, j0 + u);
+            z[u] = same_factor(G, a, b) ? src[z_packed0(G) + row_index_g(G, a, b)] : 0.f;
+        }
+        *reinterpret_cast<float4 *>(z_out + bh * (D * D) + xz) = make_float4(z[0], z[1], z[2], z[3]);
     }
 }
 
@@ -1448,7 +1460,7 @@ bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const
 template <int G>
 cudaError_t launch_expand(const float *src, long long stride, float *state_out, float *z_out, long long BH,
                           int d_out, cudaStream_t st) {
-    const long long n = ((long long)d_out * d_out * d_out + (long long)d_out * d_out) * BH;
+    const long long n = ((long long)d_out * d_out * d_out + (long long)d_out * d_out) / 4 * BH;
     const unsigned grid = (unsigned)((n + 255) / 256);
     ProfScope ps(G == 1 ? "tc_state_expand" : "tc_state_expand_m2", st);
     if (G == 2 && d_out != kD) return cudaErrorInvalidValue;
