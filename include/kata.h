@@ -103,11 +103,12 @@ size_t kata_chunked_forward_workspace_bytes(int B, int H, int T, int dk, int dv,
  *          result does not depend on C (the form is exact for every C).  C
  *          sets where states are kept; between them the exact causal
  *          quadratic form is used:
- *            C <= 256: chunks are merged into segments of a fixed length per
- *              head size, L = 1024 tokens for dk = 64 (512 for 32, 256 for
- *              16), a multiple of C.  Every such C runs the same kernels on
- *              the same schedule (the intra-segment term is computed in
- *              64-key blocks with the diagonal block masked).
+ *            C <= 256: chunks are merged into segments of a fixed length,
+ *              a multiple of C: L = 1024 tokens for bf16 (the tensor cores,
+ *              every head size) and for fp32 dk = 64, 512 for fp32 dk = 32,
+ *              256 for fp32 dk = 16.  Every such C runs the same kernels on
+ *              the same schedule (on the tensor cores the intra-segment term
+ *              is computed in 128-key steps with the diagonal block masked).
  *            C >= 512: states are kept every C tokens (L = C), which trades
  *              state traffic and scan depth (about 1/C) against intra-chunk
  *              work (about C).

@@ -32,11 +32,14 @@ def _lib():
     assert K.kata_get_device_status() == 0
 
 
-def seg_len(d, C):
+def seg_len(d, C, dtype="bf16"):
     """Tokens between stored states: C itself for C >= 512, else a fixed
-    length per head size (include/kata.h, argument C)."""
+    length: 1024 on the tensor cores (bf16, every head size), per head size on
+    the fp32 path (include/kata.h, argument C)."""
     if C >= 512:
         return C
+    if dtype == "bf16":
+        return 1024
     return 1024 if d >= 64 else (512 if d >= 32 else 256)
 
 
@@ -82,7 +85,7 @@ def test_small_bf16_full(oracle_mod):
 def _sampled_check(oracle_mod, q, k, v, dtype, Cs, n_uniform=512):
     B, H, T, d = q.shape
     q64, k64, v64 = (inputs.widen(x, dtype).reshape(B * H, T, -1) for x in (q, k, v))
-    rows = sample_rows(T, min(Cs), min(seg_len(d, C) for C in Cs), n_uniform=n_uniform)
+    rows = sample_rows(T, min(Cs), min(seg_len(d, C, dtype) for C in Cs), n_uniform=n_uniform)
     bh = np.repeat(np.arange(B * H), len(rows))
     tt = np.tile(rows, B * H)
     yref = oracle_mod.forward_rows(q64, k64, v64, bh, tt)
