@@ -387,7 +387,6 @@ kata_status kata_chunked_forward_from_state(const void *q, const void *k, const 
              overlaps(z_out, nz, state_in, span_s) || overlaps(z_out, nz, z_in, span_z)))
             return KATA_ERR_INVALID_ARG;
         init.s = state_in;
-        init.d = dk;
         init.z = z_in;
         init.n = n_in;
         init.s_stride = (long long)s_stride;

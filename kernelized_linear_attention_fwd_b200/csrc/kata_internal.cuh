@@ -149,7 +149,6 @@ struct InitState {
     const float *z = nullptr;
     int n = 0;
     long long s_stride = 0, z_stride = 0;
-    int d = 64;
 };
 
 // Launchers (return cudaSuccess or the launch error).  out == nullptr skips

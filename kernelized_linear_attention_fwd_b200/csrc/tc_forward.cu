@@ -11,12 +11,13 @@
 //                    half-strip rows (tc_layout.cuh) and dZ = sum k k^T, fp32
 //                    (the key tiles are transposed in shared memory on the way)
 //   tc_seg_scan      exclusive prefix over segments (associative scan) into a
-//                    bf16 copy for the readout, plus the fp32 total
+//                    bf16 copy for the readout, and the total: written as the
+//                    dense exported state (one factor) or kept packed in fp32
 //   tc_read          per 256 queries: phi(Q) S_prev and q^T Z_prev q on tcgen05
 //                    (phi(Q) generated from registers into tensor memory), the
 //                    intra-segment squared-score term on tcgen05, the division
-//   tc_state_expand  fp32 total -> dense [d*d, d] state and [d, d] Z (d <= 64:
-//                    heads of d < 64, computed as 64, export their leading d x d part)
+//   tc_state_expand  two factors: fp32 packed total -> dense [d*d, d] state and
+//                    [d, d] Z, zeros at the pairs across factors
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -37,10 +38,13 @@ KATA_HD constexpr long long bf16_per_seg(int G) { return (long long)bf16_rows(G)
 
 // ---------------------------------------------------------------------------
 // Exclusive prefix over segments (the associative scan across chunk states)
-// -> bf16 copy for the readout (Z split into hi and lo parts), and the fp32
-// total.  An initial state (the sum of n_in dense states) seeds the running
-// sum, so every prefix and the total include it and segment 0 gets a prefix
-// too; prefix == nullptr computes the total only.
+// -> bf16 copy for the readout (Z split into hi and lo parts), and the total:
+// the fp32 packed total (total != nullptr) and/or the dense exported state
+// (state_out != nullptr: S [d*d][d] and Z [d][d] of head size d <= 64,
+// written straight from the scan's registers; one factor only).  An initial
+// state (the sum of n_in dense states of head size d) seeds the running sum,
+// so every prefix and the total include it and segment 0 gets a prefix too;
+// prefix == nullptr computes the total only.
 // Reduce-then-scan per block of 128 consecutive elements of one head
 // (32 lanes x float4): warp w takes a run of RUN consecutive segments,
 // holds them in registers and forms their running sums; the 8 run totals are
@@ -52,7 +56,7 @@ KATA_HD constexpr long long bf16_per_seg(int G) { return (long long)bf16_rows(G)
 // latency of these short blocks needs.  G factors (KATA-Mg): the layout with
 // G factors; the dense Z prefix then also gets zeros at the pairs across
 // factors, which the readout's q^T Z q must not see.
-// grid.x = element-block + n_eb * bh; block 256.
+// grid.x = n_eb * BH (the packed-z blocks of all heads first); block 256.
 // ---------------------------------------------------------------------------
 constexpr int kScanWarps = 8;
 
@@ -80,29 +84,77 @@ struct ScanLane {
     }
 
     // The initial state of these 4 packed elements: the sum of n_in dense states
-    // of head size d (<= 64: the coordinates past d are zero).
+    // of head size d (<= 64: the coordinates past d are zero), added in order
+    // n = 0, 1, ...; the loads of U states are in flight at a time.
+    template <int U>
     __device__ __forceinline__ float4 init(long long bh, const float *init_s, const float *init_z,
                                            int n_in, long long s_stride, long long z_stride,
                                            int d) const {
         float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int n = 0; n < n_in; ++n) {
-            if (!z_part) {
-                const PairIJ pij = row_ij_g(G, (int)(e0 / kD));
-                const int e = (int)(e0 % kD);  // 4 consecutive values, all below d or none
-                if (pij.i <= pij.j && pij.j < d && e < d)
-                    carry = f4add(carry, *reinterpret_cast<const float4 *>(
-                                             init_s + n * s_stride +
-                                             ((bh * d + pij.i) * d + pij.j) * d + e));
-            } else {
-                const float *zn = init_z + n * z_stride + bh * d * d;
-                float zv[4];
+        if (n_in <= 0) return carry;
+        if (!z_part) {
+            const PairIJ pij = row_ij_g(G, (int)(e0 / kD));
+            const int e = (int)(e0 % kD);  // 4 consecutive values, all below d or none
+            if (pij.i > pij.j || pij.j >= d || e >= d) return carry;
+            const float *src = init_s + ((bh * d + pij.i) * d + pij.j) * d + e;
+            int n = 0;
+            for (; n + U <= n_in; n += U) {
+                float4 a[U];
 #pragma unroll
-                for (int x = 0; x < 4; ++x)
-                    zv[x] = zi[x] <= zj[x] && zj[x] < d ? zn[zi[x] * d + zj[x]] : 0.f;
-                carry = f4add(carry, make_float4(zv[0], zv[1], zv[2], zv[3]));
+                for (int u = 0; u < U; ++u) a[u] = *reinterpret_cast<const float4 *>(src + (n + u) * s_stride);
+#pragma unroll
+                for (int u = 0; u < U; ++u) carry = f4add(carry, a[u]);
             }
+            for (; n < n_in; ++n) carry = f4add(carry, *reinterpret_cast<const float4 *>(src + n * s_stride));
+            return carry;
+        }
+        // packed normaliser entries: Z[i][j] of each of the 4 pairs
+        int off[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) off[x] = zi[x] <= zj[x] && zj[x] < d ? zi[x] * d + zj[x] : -1;
+        const float *zb = init_z + bh * d * d;
+        int n = 0;
+        for (; n + U <= n_in; n += U) {
+            float a[U][4];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int x = 0; x < 4; ++x) a[u][x] = off[x] >= 0 ? zb[(n + u) * z_stride + off[x]] : 0.f;
+#pragma unroll
+            for (int u = 0; u < U; ++u) carry = f4add(carry, make_float4(a[u][0], a[u][1], a[u][2], a[u][3]));
+        }
+        for (; n < n_in; ++n) {
+            float a[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) a[x] = off[x] >= 0 ? zb[n * z_stride + off[x]] : 0.f;
+            carry = f4add(carry, make_float4(a[0], a[1], a[2], a[3]));
         }
         return carry;
+    }
+
+    // Writes the total t of these elements into the dense exported state of
+    // head bh, head size d (<= 64): S [d*d][d] at state_out and Z [d][d] at
+    // z_out, both (i, j) and (j, i).  One factor only: there every dense entry
+    // is a pair of the layout, so the scan lanes cover the whole export.
+    __device__ __forceinline__ void write_dense(float *state_out, float *z_out, long long bh, float4 t,
+                                                int d) const {
+        if (!z_part) {
+            const PairIJ pij = row_ij_g(G, (int)(e0 / kD));
+            const int e = (int)(e0 % kD);
+            if (pij.i > pij.j || pij.j >= d || e >= d) return;
+            float *s = state_out + bh * d * d * d;
+            *reinterpret_cast<float4 *>(s + ((long long)pij.i * d + pij.j) * d + e) = t;
+            if (pij.i != pij.j) *reinterpret_cast<float4 *>(s + ((long long)pij.j * d + pij.i) * d + e) = t;
+            return;
+        }
+        const float tv[4] = {t.x, t.y, t.z, t.w};
+        float *z = z_out + bh * d * d;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            if (zi[x] > zj[x] || zj[x] >= d) continue;
+            z[zi[x] * d + zj[x]] = tv[x];
+            z[zj[x] * d + zi[x]] = tv[x];
+        }
     }
 
     // Writes the prefix p of these elements into one segment's bf16 prefix dst.
@@ -151,18 +203,22 @@ __global__ void __launch_bounds__(256, RUN == 2 ? 5 : RUN == 4 ? 4 : 2)  // bloc
 tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ prefix,
             float *__restrict__ total, int n_seg, int n_valid, const float *__restrict__ init_s,
             const float *__restrict__ init_z, int n_in, long long s_stride, long long z_stride,
-            int d_in) {
+            int d, float *__restrict__ state_out, float *__restrict__ z_out) {
     __shared__ float4 part[2][kScanWarps][32];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     constexpr long long E = f32_per_seg(G);
     constexpr long long n_eb = E / 128;
-    constexpr long long n_zb = state_rows(G) / 128;  // packed-z blocks (scattered writes): run them first
-    const long long eb = (blockIdx.x % n_eb + (n_eb - n_zb)) % n_eb;
-    const long long bh = blockIdx.x / n_eb;
+    // The packed-z blocks of every head (their dense Z prefix goes out in
+    // scattered 2-byte stores) take the first CTAs, so they start in the first
+    // wave; the state blocks follow, head-major.
+    constexpr long long n_zb = state_rows(G) / 128, n_sb = n_eb - n_zb;
+    const long long NZ = n_zb * (gridDim.x / n_eb), x = blockIdx.x;
+    const long long bh = x < NZ ? x / n_zb : (x - NZ) / n_sb;
+    const long long eb = x < NZ ? n_sb + x % n_zb : (x - NZ) % n_sb;
     const ScanLane<G> sl(eb * 128 + 4 * lane);
     const float *base = seg_state + bh * (long long)n_seg * E + sl.e0;
     __nv_bfloat16 *pbase = prefix ? prefix + bh * (long long)n_seg * bf16_per_seg(G) : nullptr;
-    float4 carry = sl.init(bh, init_s, init_z, n_in, s_stride, z_stride, d_in);
+    float4 carry = sl.template init<RUN <= 4 ? 2 : 4>(bh, init_s, init_z, n_in, s_stride, z_stride, d);
     const int g_first = n_in > 0 ? 0 : 1;  // without one, segment 0 has an empty prefix
 
     for (int g0 = 0; g0 < n_seg; g0 += kScanWarps * RUN) {
@@ -204,8 +260,10 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
             sl.write(pbase + (long long)g * bf16_per_seg(G), f4add(v[i], off), lane);
         }
     }
-    if (total != nullptr && w == 0)
-        *reinterpret_cast<float4 *>(total + bh * E + sl.e0) = carry;
+    if (w == 0) {
+        if (total != nullptr) *reinterpret_cast<float4 *>(total + bh * E + sl.e0) = carry;
+        if (state_out != nullptr) sl.write_dense(state_out, z_out, bh, carry, d);
+    }
 }
 
 // The same scan for short sequences (at most RUN <= 16 segments): one warp
@@ -214,19 +272,35 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
 // no barrier.  A sequence of a few segments (a short prompt, one rank's block
 // of a sequence split over GPUs) otherwise runs thousands of blocks that each
 // move a few kilobytes between three barriers.
-// grid.x = ceil(n_eb * BH / 8); block 256.
+// grid.x = ceil(n_eb * BH / 8) (at least n_zb * BH); block 256.
 template <int G, int RUN>
-__global__ void __launch_bounds__(256, RUN <= 4 ? 4 : 2)
+__global__ void __launch_bounds__(256, RUN > 8 ? 2 : RUN > 4 || G == 2 ? 3 : 4)  // blocks per SM without spills
 tc_seg_scan_short(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ prefix,
                   float *__restrict__ total, int n_seg, int n_valid, long long BH,
                   const float *__restrict__ init_s, const float *__restrict__ init_z, int n_in,
-                  long long s_stride, long long z_stride, int d_in) {
+                  long long s_stride, long long z_stride, int d, float *__restrict__ state_out,
+                  float *__restrict__ z_out) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     constexpr long long E = f32_per_seg(G);
     constexpr long long n_eb = E / 128;
-    const long long gidx = (long long)blockIdx.x * kScanWarps + w;  // warp-uniform
+    // The warp's element block.  The packed-z blocks, whose dense Z prefix
+    // goes out in scattered 2-byte stores, take warp 0 of the first n_zb * BH
+    // CTAs, one per CTA, so that no SM serialises several of them; the state
+    // blocks fill the other warps in order (head-major).
+    constexpr long long n_zb = state_rows(G) / 128, n_sb = n_eb - n_zb;
+    const long long NZ = n_zb * BH, blk = blockIdx.x;
+    const long long gidx = blk * kScanWarps + w;  // warp-uniform
     if (gidx >= n_eb * BH) return;
-    const long long bh = gidx / n_eb, eb = gidx % n_eb;
+    long long bh, eb;
+    if (w == 0 && blk < NZ) {
+        bh = blk / n_zb;
+        eb = n_sb + blk % n_zb;
+    } else {
+        const long long zb_before = blk + (w > 0 ? 1 : 0) < NZ ? blk + (w > 0 ? 1 : 0) : NZ;
+        const long long s = gidx - zb_before;
+        bh = s / n_sb;
+        eb = s % n_sb;
+    }
     const ScanLane<G> sl(eb * 128 + 4 * lane);
     const float *base = seg_state + bh * (long long)n_seg * E + sl.e0;
     __nv_bfloat16 *pbase = prefix ? prefix + bh * (long long)n_seg * bf16_per_seg(G) : nullptr;
@@ -235,7 +309,7 @@ tc_seg_scan_short(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict
     for (int i = 0; i < RUN; ++i)
         v[i] = i < n_valid ? *reinterpret_cast<const float4 *>(base + (long long)i * E)
                            : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 run = sl.init(bh, init_s, init_z, n_in, s_stride, z_stride, d_in);
+    float4 run = sl.template init<RUN <= 4 ? 1 : RUN <= 8 ? 2 : 4>(bh, init_s, init_z, n_in, s_stride, z_stride, d);
     const int g_first = n_in > 0 ? 0 : 1;
 #pragma unroll
     for (int i = 0; i < RUN; ++i) {
@@ -244,14 +318,16 @@ tc_seg_scan_short(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict
         run = f4add(run, v[i]);
     }
     if (total != nullptr) *reinterpret_cast<float4 *>(total + bh * E + sl.e0) = run;
+    if (state_out != nullptr) sl.write_dense(state_out, z_out, bh, run, d);
 }
 
 // ---------------------------------------------------------------------------
-// fp32 total (packed rows) -> dense state [D*D][D] and Z [D][D].  D < 64: the
-// heads were computed as 64 (columns past D zero), and the leading D x D part
-// is exported.  G
-// factors (KATA-Mg): pairs across factors are not in the layout and export 0.
-// D is a template parameter so the index arithmetic divides by constants.
+// fp32 total (packed rows) -> dense state [D*D][D] and Z [D][D], for G = 2
+// factors (KATA-Mg, D = 64), whose pairs across factors are not in the layout
+// and export 0 (one factor exports straight from the scan, every dense entry
+// being a pair of its layout).  D < 64 would export the leading D x D part of
+// heads computed as 64.  D is a template parameter so the index arithmetic
+// divides by constants.
 // ---------------------------------------------------------------------------
 // A thread writes 4 consecutive outputs (one 16-byte store: the outputs are
 // 16-byte aligned, and D, the packed row length and the per-head strides are
@@ -1457,19 +1533,14 @@ bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const
            make_tmap_bf16(ms, prefix ? prefix : q, 3, ds, ss, bs) && make_tmap_bf16(mo, out, 3, dqkv, sqkv, bqkv);
 }
 
-template <int G>
-cudaError_t launch_expand(const float *src, long long stride, float *state_out, float *z_out, long long BH,
-                          int d_out, cudaStream_t st) {
-    const long long n = ((long long)d_out * d_out * d_out + (long long)d_out * d_out) / 4 * BH;
+// The dense export of two factors (d = 64).
+cudaError_t launch_expand_m2(const float *src, long long stride, float *state_out, float *z_out, long long BH,
+                             int d_out, cudaStream_t st) {
+    if (d_out != kD) return cudaErrorInvalidValue;
+    const long long n = ((long long)kD * kD * kD + (long long)kD * kD) / 4 * BH;
     const unsigned grid = (unsigned)((n + 255) / 256);
-    ProfScope ps(G == 1 ? "tc_state_expand" : "tc_state_expand_m2", st);
-    if (G == 2 && d_out != kD) return cudaErrorInvalidValue;
-    switch (d_out) {
-        case 16: tc_state_expand<G, 16><<<grid, 256, 0, st>>>(src, stride, state_out, z_out, BH); break;
-        case 32: tc_state_expand<G, 32><<<grid, 256, 0, st>>>(src, stride, state_out, z_out, BH); break;
-        case 64: tc_state_expand<G, 64><<<grid, 256, 0, st>>>(src, stride, state_out, z_out, BH); break;
-        default: return cudaErrorInvalidValue;
-    }
+    ProfScope ps("tc_state_expand_m2", st);
+    tc_state_expand<2, kD><<<grid, 256, 0, st>>>(src, stride, state_out, z_out, BH);
     return cudaSuccess;
 }
 
@@ -1493,11 +1564,15 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
     // every segment's increment is in the workspace already
     const int n_build = reuse_seg ? 0 : want_state ? p.n_seg : p.n_seg - 1;
     const int n_valid = reuse_seg ? p.n_seg : n_build;
-    const bool scan = p.n_seg > 1 || has_init;
+    // one factor: the scan writes the exported state, so it runs whenever a
+    // state is wanted (with one segment and no initial state it only copies)
+    const bool dense_from_scan = G == 1 && want_state;
+    const bool scan = p.n_seg > 1 || has_init || dense_from_scan;
     const long long BH = p.BH;
     int *status = device_status_ptr();
     if (!status) return cudaErrorUnknown;
     if ((has_init || n_build > 0 || want_state || reuse_seg) && !w) return cudaErrorInvalidValue;
+    if (want_state && (d_out < 1 || d_out > kD)) return cudaErrorInvalidValue;
 
     if (n_build > 0) {
         CUtensorMap mkb, mvb, mst;
@@ -1521,21 +1596,25 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
     if (scan) {
         ProfScope ps(G == 1 ? "tc_seg_scan" : "tc_seg_scan_m2", st);
         __nv_bfloat16 *pre = readout ? prefix : nullptr;
-        float *tot = want_state ? total : nullptr;
+        float *tot = want_state && !dense_from_scan ? total : nullptr;
+        float *s_out = dense_from_scan ? state_out : nullptr;
+        float *z_dense = dense_from_scan ? z_out : nullptr;
         if (p.n_seg <= 16) {
             // few segments: one warp per element block (no cross-warp scan)
             const long long grid = ((f32_per_seg(G) / 128) * BH + kScanWarps - 1) / kScanWarps;
             auto kern = p.n_seg <= 4 ? tc_seg_scan_short<G, 4>
                         : p.n_seg <= 8 ? tc_seg_scan_short<G, 8> : tc_seg_scan_short<G, 16>;
             kern<<<(unsigned)grid, 256, 0, st>>>(seg, pre, tot, p.n_seg, n_valid, BH, init.s, init.z,
-                                                 init.n, init.s_stride, init.z_stride, init.d);
+                                                 init.n, init.s_stride, init.z_stride, d_out, s_out,
+                                                 z_dense);
         } else {
             const long long grid = (f32_per_seg(G) / 128) * BH;
             auto kern = p.n_seg <= 4 * kScanWarps ? tc_seg_scan<G, 4>
                         : p.n_seg <= 8 * kScanWarps ? tc_seg_scan<G, 8>
                                                     : tc_seg_scan<G, 16>;
             kern<<<(unsigned)grid, 256, 0, st>>>(seg, pre, tot, p.n_seg, n_valid, init.s, init.z,
-                                                 init.n, init.s_stride, init.z_stride, init.d);
+                                                 init.n, init.s_stride, init.z_stride, d_out, s_out,
+                                                 z_dense);
         }
     }
     if (readout) {
@@ -1551,11 +1630,10 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
         tc_read<G><<<(unsigned)grid, kReadThreads, kSmAlloc, st>>>(
             mq, mk, mv, ms, mo, p.T, p.L, p.n_seg, n_ct, (int)n_items, has_init, status);
     }
-    if (want_state) {
+    if (want_state && !dense_from_scan) {
         const float *src = scan ? total : seg;
         const long long stride = scan ? f32_per_seg(G) : f32_per_seg(G) * p.n_seg;
-        if (d_out < 1 || d_out > kD) return cudaErrorInvalidValue;
-        const cudaError_t e = launch_expand<G>(src, stride, state_out, z_out, BH, d_out, st);
+        const cudaError_t e = launch_expand_m2(src, stride, state_out, z_out, BH, d_out, st);
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();

@@ -61,8 +61,8 @@ def test_state_only(oracle_mod, dtype, d, T):
     check_state(oracle_mod, S, Z, k64, v64, dtype)
     # the state the forward exports, within the same bound (not bitwise: on the
     # tensor-core path two MMA issuers add into one accumulator in issue order)
-    so = torch.empty_like(S)
-    zo = torch.empty_like(Z)
+    so = torch.full_like(S, float("nan"))  # an entry left unwritten fails the check
+    zo = torch.full_like(Z, float("nan"))
     K.kata_chunked_forward(dev(q, dtype), dev(k, dtype), dev(v, dtype), C=64, state_out=so,
                            z_out=zo)
     torch.cuda.synchronize()
@@ -76,8 +76,8 @@ def test_forward_from_one_state(oracle_mod, dtype, d, Th, Tb):
     q, k, v = inputs.make_qkv(1, 3, Th + Tb, d, d, dtype, seed=Th + 3 * Tb + d)
     q64, k64, v64 = (inputs.widen(x, dtype) for x in (q, k, v))
     S0, Z0 = oracle_mod.state(k64[:, :, :Th], v64[:, :, :Th])
-    so = torch.empty((1, 3, d * d, d), dtype=torch.float32, device="cuda")
-    zo = torch.empty((1, 3, d, d), dtype=torch.float32, device="cuda")
+    so = torch.full((1, 3, d * d, d), float("nan"), dtype=torch.float32, device="cuda")
+    zo = torch.full((1, 3, d, d), float("nan"), dtype=torch.float32, device="cuda")
     blk = [dev(x[:, :, Th:], dtype) for x in (q, k, v)]
     out = K.kata_chunked_forward_from_state(*blk, f32(S0), f32(Z0), C=64, state_out=so, z_out=zo)
     torch.cuda.synchronize()

@@ -48,8 +48,9 @@ def run_forward(q, k, v, dtype, C, want_state=False):
     B, H, T, dk = q.shape
     so = zo = None
     if want_state:
-        so = torch.empty((B, H, dk * dk, dk), dtype=torch.float32, device="cuda")
-        zo = torch.empty((B, H, dk, dk), dtype=torch.float32, device="cuda")
+        # NaN-filled, so an entry the export does not write fails the comparison
+        so = torch.full((B, H, dk * dk, dk), float("nan"), dtype=torch.float32, device="cuda")
+        zo = torch.full((B, H, dk, dk), float("nan"), dtype=torch.float32, device="cuda")
     out = K.kata_chunked_forward(qd, kd, vd, C=C, state_out=so, z_out=zo)
     torch.cuda.synchronize()
     return out, so, zo
