@@ -755,7 +755,7 @@ def measure_other_configs(K, inputs, stream, flush, names=("lm340m_B4H16_T16384_
                      "canonical_tflops": canon / (ms / 1e3) / 1e12,
                      "frac_of_measured_peak": canon / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
                      "path": ("fp32 CUDA cores" if w.dtype != "bf16" else "tensor cores" if w.d == 64
-                              else f"tensor cores, heads of d = {w.d} read as 64 (zero-filled by TMA)")}
+                              else f"tensor cores, heads of d = {w.d} read as 64 (zero-filled by TMA), two-factor layout")}
         del q, k, v, so, zo, out, ws
     return res
 

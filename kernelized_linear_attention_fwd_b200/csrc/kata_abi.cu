@@ -91,8 +91,10 @@ kata_status make_plan(int B, int H, int T, int dk, int dv, int C, kata_dtype dty
     p.BH = BH;
     p.path = (dtype == KATA_BF16 && (dk == 64 || small_tc)) ? Path::kTensorCore : Path::kSimt;
     if (p.path == Path::kTensorCore) {
-        // the tensor-core kernels compute every head as d = 64
-        p.R = packed_rows(64);
+        // the tensor-core kernels compute every head as d = 64; a head of d <= 32
+        // as a two-factor head whose second factor (coordinates 32-63) is zero
+        p.tc_g = dk <= 32 ? 2 : 1;
+        p.R = packed_rows_g(64, p.tc_g);
         p.L = segment_length(64, C);
         p.n_seg = (T + p.L - 1) / p.L;
         tc::plan_tc_workspace(p);
@@ -126,6 +128,7 @@ kata_status make_plan_mg(int B, int H, int T, int dk, int dv, int C, int g, kata
     p.g = g;
     p.R = packed_rows_g(dk, g);
     if (p.path == Path::kTensorCore) {
+        p.tc_g = g;
         tc::plan_tc_workspace(p);
         return KATA_OK;
     }
@@ -143,6 +146,7 @@ kata_status make_plan_mg(int B, int H, int T, int dk, int dv, int C, int g, kata
 kata_status make_quadratic_plan(int B, int H, int T, int dk, int dv, kata_dtype dtype, Plan &p) {
     const kata_status s = make_plan(B, H, T, dk, dv, 256, dtype, p);
     if (s != KATA_OK) return s;
+    p.tc_g = 1;  // no state: the one-factor readout, whose intra steps are 128 keys
     p.L = T;
     p.n_seg = 1;
     p.ws_seg_state = p.ws_total = p.ws_extra = p.ws_aux = p.ws_bytes = 0;

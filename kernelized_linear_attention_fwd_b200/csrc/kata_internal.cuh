@@ -61,7 +61,8 @@ __host__ __device__ inline int packed_row_index_g(int d, int G, int i, int j) {
 // ---------------------------------------------------------------------------
 // kTensorCore: bf16 heads of d = 64, and of d = 16 or 32 read as 64 by the
 // tensor maps (TMA fills the columns past d with zeros, which add nothing to
-// any product or sum; the output store writes only the first d columns).
+// any product or sum; the output store writes only the first d columns) and
+// run on the two-factor layout (Plan::tc_g).
 enum class Path : int { kSimt = 0, kTensorCore = 1 };
 
 struct Plan {
@@ -72,6 +73,11 @@ struct Plan {
     int n_seg;  // ceil(T / L)
     int R;      // packed feature rows (of d = 64 on the tensor-core path)
     int g = 1;  // rank-one PSD factors per head (KATA-Mg; 1 = the single factor)
+    // Factors of the tensor-core layout the kernels run: g, except that a
+    // single-factor head of d <= 32 runs the two-factor layout (its
+    // coordinates 32-63, read as zeros, form a second factor that contributes
+    // nothing), which holds its state in 1152 rows instead of 2176.
+    int tc_g = 1;
     Path path;
     // workspace (bytes from the base, all 256-byte aligned)
     size_t ws_seg_state;  // fp32 per-segment states, exclusive prefix after the scan

@@ -1552,7 +1552,8 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
                                 float *state_out, float *z_out, const InitState &init, void *ws,
                                 cudaStream_t st, bool reuse_seg) {
     // heads of d < 64 are read as 64 by every tensor map (TMA zero-fills the
-    // columns past d) and exported at their own size
+    // columns past d; with G = 2 the second factor is then zero) and exported
+    // at their own size
     const int d_out = p.dk;
     // no workspace (the quadratic plan): no state is built, scanned or read
     char *w = static_cast<char *>(ws);
@@ -1566,9 +1567,11 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
     // every segment's increment is in the workspace already
     const int n_build = reuse_seg ? 0 : want_state ? p.n_seg : p.n_seg - 1;
     const int n_valid = reuse_seg ? p.n_seg : n_build;
-    // one factor: the scan writes the exported state, so it runs whenever a
-    // state is wanted (with one segment and no initial state it only copies)
-    const bool dense_from_scan = G == 1 && want_state;
+    // the scan writes the exported state when every dense entry is a pair of
+    // the layout (one factor, or heads of d <= 32 on the two-factor layout),
+    // so it runs whenever a state is wanted (with one segment and no initial
+    // state it only copies)
+    const bool dense_from_scan = want_state && (G == 1 || d_out <= kD / 2);
     const bool scan = p.n_seg > 1 || has_init || dense_from_scan;
     const long long BH = p.BH;
     int *status = device_status_ptr();
@@ -1665,7 +1668,7 @@ int num_sms() {
 //   bf16 prefixes        BH * n_seg * (R + 128) * 64 * 2
 void plan_tc_workspace(Plan &p) {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    const int G = p.g;
+    const int G = p.tc_g;
     const size_t seg = (size_t)p.BH * p.n_seg * f32_per_seg(G) * 4;
     const size_t tot = (size_t)p.BH * f32_per_seg(G) * 4;
     const size_t pre = (size_t)p.BH * p.n_seg * bf16_per_seg(G) * 2;
@@ -1679,7 +1682,7 @@ void plan_tc_workspace(Plan &p) {
 cudaError_t launch_tc_forward(const Plan &p, const void *q, const void *k, const void *v, void *out,
                               float *state_out, float *z_out, const InitState &init, void *ws,
                               cudaStream_t st, bool reuse_seg) {
-    switch (p.g) {
+    switch (p.tc_g) {
         case 1: return launch_tc_forward_g<1>(p, q, k, v, out, state_out, z_out, init, ws, st, reuse_seg);
         case 2: return launch_tc_forward_g<2>(p, q, k, v, out, state_out, z_out, init, ws, st, reuse_seg);
         default: return cudaErrorInvalidValue;

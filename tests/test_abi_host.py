@@ -81,14 +81,18 @@ def test_workspace_query(lib):
     assert W(1, 8, 131072, 64, 64, 4096, 1) > 0 and W(1, 8, 131072, 64, 64, 8192, 1) == 0
 
 
-def test_small_bf16_heads_take_the_d64_tensor_core_workspace(lib):
-    # bf16 heads of d < 64 run the tensor-core kernels, which read them as
-    # d = 64 (the tensor maps zero-fill the columns past d): the same workspace
-    # as d = 64, with no padded copies; fp32 keeps its CUDA-core layout
+def test_small_bf16_heads_take_the_two_factor_tensor_core_workspace(lib):
+    # bf16 heads of d <= 32 run the tensor-core kernels, which read them as
+    # d = 64 (the tensor maps zero-fill the columns past d) on the two-factor
+    # layout (coordinates 32-63 are a second factor that contributes nothing):
+    # the workspace of a two-factor d = 64 head, smaller than the one-factor
+    # one, with no padded copies; fp32 keeps its CUDA-core layout
     W = lib.kata_chunked_forward_workspace_bytes
+    Wmg = lib.kata_mg_chunked_forward_workspace_bytes
     for B, H, T, d in [(2, 4, 4096, 32), (1, 3, 1000, 16), (1, 1, 1, 32), (4, 2, 2049, 16)]:
         for C in (64, 512):
-            assert W(B, H, T, d, d, C, 1) == W(B, H, T, 64, 64, C, 1)
+            assert W(B, H, T, d, d, C, 1) == Wmg(B, H, T, 64, 64, C, 2, 1)
+            assert W(B, H, T, d, d, C, 1) < W(B, H, T, 64, 64, C, 1)
         assert W(B, H, T, d, d, 64, 0) < W(B, H, T, 64, 64, 64, 0)
 
 
