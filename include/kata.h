@@ -129,7 +129,8 @@ size_t kata_chunked_forward_workspace_bytes(int B, int H, int T, int dk, int dv,
  * run the kernels' two-factor state layout (the same as kata_mg_chunked_forward
  * with g = 2 at d = 64): coordinates 32-63 are zero, so (q.k)^2 = (q_a.k_a)^2
  * + (q_b.k_b)^2 with the second term 0, and the state needs 1152 packed rows
- * instead of 2176.  KATA_F32 runs fp32 CUDA-core arithmetic end to end.
+ * instead of 2176; the intra-segment scores are formed whole.  KATA_F32 runs
+ * fp32 CUDA-core arithmetic end to end.
  */
 kata_status kata_chunked_forward(const void *q, const void *k, const void *v, void *out, int B,
                                  int H, int T, int dk, int dv, int C, kata_dtype dtype,

@@ -1036,7 +1036,11 @@ tc_build(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
     if (tid == 0 && abort_flag) set_timeout_status(status);
 }
 
-template <int G>
+// G: factors of the state layout (inter phase); GI: factors of the
+// intra-segment weight (1: (q.k)^2 in 128-key steps; 2: the sum over the two
+// factors in 64-key steps).  A single-factor head of d <= 32 runs G = 2,
+// GI = 1: its state on the two-factor layout, its scores whole.
+template <int G, int GI>
 __global__ void __launch_bounds__(kReadThreads, 1)
 tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
@@ -1105,7 +1109,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             int n_q = 0, n_bs = 0, n_kv = 0, n_v = 0;  // loads issued into each ring (n_kv: keys)
             bool ok = true;
             for (int x = sched.first; x < sched.end && ok; x += sched.stride) {
-                const ReadItem it = read_item<G>(sched.item(x), n_ct, T, L, n_seg, has_init);
+                const ReadItem it = read_item<GI>(sched.item(x), n_ct, T, L, n_seg, has_init);
                 {
                     const int qb = n_q & 1;
                     uint8_t *slot = sm + kSmItem + qb * kItemBytes;
@@ -1129,21 +1133,21 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     ++n_bs;
                 }
                 for (int kb = 0; kb < it.n_kv && ok; ++kb) {
-                    const int s = n_kv % kv_ring(G);
-                    const uint32_t par = ((n_kv / kv_ring(G)) & 1) ^ 1;
+                    const int s = n_kv % kv_ring(GI);
+                    const uint32_t par = ((n_kv / kv_ring(GI)) & 1) ^ 1;
                     ok = mbar_wait(&bars.kempty[s], par, abort);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(&bars.kfull[s], kv_bytes(G));
-                    tma_load_3d(sm + kSmK + s * kv_bytes(G), &tm_k, &bars.kfull[s], 0,
-                                it.seg0 + kb * step_keys(G), it.bh);
+                    mbar_arrive_expect_tx(&bars.kfull[s], kv_bytes(GI));
+                    tma_load_3d(sm + kSmK + s * kv_bytes(GI), &tm_k, &bars.kfull[s], 0,
+                                it.seg0 + kb * step_keys(GI), it.bh);
                     ok = mbar_wait(&bars.vempty[s], par, abort);
                     if (!ok) {
                         ++n_kv;  // its keys are in flight: waited for below
                         break;
                     }
-                    mbar_arrive_expect_tx(&bars.vfull[s], kv_bytes(G));
-                    tma_load_3d(sm + kSmV + s * kv_bytes(G), &tm_v, &bars.vfull[s], 0,
-                                it.seg0 + kb * step_keys(G), it.bh);
+                    mbar_arrive_expect_tx(&bars.vfull[s], kv_bytes(GI));
+                    tma_load_3d(sm + kSmV + s * kv_bytes(GI), &tm_v, &bars.vfull[s], 0,
+                                it.seg0 + kb * step_keys(GI), it.bh);
                     ++n_kv;
                     ++n_v;
                 }
@@ -1153,10 +1157,10 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                 mbar_wait_issued(&bars.qfull[x & 1], (x >> 1) & 1);
             for (int x = (n_bs > kRBRing ? n_bs - kRBRing : 0); x < n_bs; ++x)
                 mbar_wait_issued(&bars.bfull[x % kRBRing], (x / kRBRing) & 1);
-            for (int x = (n_kv > kv_ring(G) ? n_kv - kv_ring(G) : 0); x < n_kv; ++x)
-                mbar_wait_issued(&bars.kfull[x % kv_ring(G)], (x / kv_ring(G)) & 1);
-            for (int x = (n_v > kv_ring(G) ? n_v - kv_ring(G) : 0); x < n_v; ++x)
-                mbar_wait_issued(&bars.vfull[x % kv_ring(G)], (x / kv_ring(G)) & 1);
+            for (int x = (n_kv > kv_ring(GI) ? n_kv - kv_ring(GI) : 0); x < n_kv; ++x)
+                mbar_wait_issued(&bars.kfull[x % kv_ring(GI)], (x / kv_ring(GI)) & 1);
+            for (int x = (n_v > kv_ring(GI) ? n_v - kv_ring(GI) : 0); x < n_v; ++x)
+                mbar_wait_issued(&bars.vfull[x % kv_ring(GI)], (x / kv_ring(GI)) & 1);
         }
     } else if (warp == kIssuer0 || warp == kIssuer0 + 1) {
         // ------------------------------------------------------------ MMA issuers
@@ -1164,7 +1168,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             const int me = warp - kIssuer0;
             const uint32_t id_n64 = idesc_bf16(kQT, 64, 0, 1);  // B MN-major, N = 64
             // scores: B = keys, K-major; N = 128 keys (one factor) or 64 per factor
-            const uint32_t id_qk = idesc_bf16(kQT, G == 1 ? 128 : 64, 0, 0);
+            const uint32_t id_qk = idesc_bf16(kQT, GI == 1 ? 128 : 64, 0, 0);
             const uint64_t dS = desc_sw128(smem_u32(sm + kSmS), 8192, 1024);
             const uint64_t dK = desc_sw128(smem_u32(sm + kSmK), 16, 1024);
             const uint64_t dV = desc_sw128(smem_u32(sm + kSmV), 8192, 1024);
@@ -1174,7 +1178,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             uint32_t vrel = 0;
             bool ok = true;
             for (int x = sched.first; x < sched.end && ok; x += sched.stride, ++j) {
-                const ReadItem it = read_item<G>(sched.item(x), n_ct, T, L, n_seg, has_init);
+                const ReadItem it = read_item<GI>(sched.item(x), n_ct, T, L, n_seg, has_init);
                 const int qb = j & 1;
                 const uint32_t slot = smem_u32(sm + kSmItem + qb * kItemBytes);
                 ok = mbar_wait(&bars.qfull[qb], (j >> 1) & 1, abort);
@@ -1241,13 +1245,13 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                 // values of step n - 3 have freed it; issuer 1 multiplies the step's
                 // weights, stored over its scores, by the values.  Each issuer
                 // releases key/value block b after its last step of the block.
-                const int nb[kTiles] = {read_tile_blocks<G>(it, 0, T), read_tile_blocks<G>(it, 1, T)};
+                const int nb[kTiles] = {read_tile_blocks<GI>(it, 0, T), read_tile_blocks<GI>(it, 1, T)};
                 const int nbm = max(nb[0], nb[1]);
                 for (int b = 0; b < nbm && ok; ++b) {
-                    const int kvb = g_kv + b, kvs = kvb % kv_ring(G);
+                    const int kvb = g_kv + b, kvs = kvb % kv_ring(GI);
                     // issuer 0 reads the block's keys; issuer 1 its values, which the
                     // squaring warps have seen land before they hand over the weights
-                    if (me == 0) ok = mbar_wait(&bars.kfull[kvs], (kvb / kv_ring(G)) & 1, abort);
+                    if (me == 0) ok = mbar_wait(&bars.kfull[kvs], (kvb / kv_ring(GI)) & 1, abort);
                     for (int t = 0; t < kTiles && ok; ++t) {
                         if (b >= nb[t]) continue;
                         const int x = ns % kSBufs;
@@ -1265,9 +1269,9 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                             const bool last = t == 1 || b >= nb[1];
                             vrel = (vrel & ~(15u << (4 * x))) | ((last ? kvs + 1u : 0u) << (4 * x));
                             tc_fence_after();
-                            const uint64_t dk = desc_add(dK, kv_bytes(G) * kvs);
+                            const uint64_t dk = desc_add(dK, kv_bytes(GI) * kvs);
                             const uint64_t dQt = desc_sw128(slot + t * 16384, 16, 1024);
-                            if constexpr (G == 1) {
+                            if constexpr (GI == 1) {
 #pragma unroll
                                 for (int ks = 0; ks < 4; ++ks)
                                     mma_ss(buf, desc_add(dQt, 32 * ks), desc_add(dk, 32 * ks), id_qk, ks > 0);
@@ -1284,9 +1288,9 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                             ok = mbar_wait(&bars.pfull[x], (ns / kSBufs) & 1, abort);
                             if (!ok) break;
                             tc_fence_after();
-                            const uint64_t dv = desc_add(dV, kv_bytes(G) * kvs);
+                            const uint64_t dv = desc_add(dV, kv_bytes(GI) * kvs);
 #pragma unroll
-                            for (int ks = 0; ks < step_keys(G) / 16; ++ks)
+                            for (int ks = 0; ks < step_keys(GI) / 16; ++ks)
                                 mma_ts(tm + kTmO + 64 * t, buf + 8 * ks, desc_add(dv, 2048 * ks), id_n64, 1);
                             mma_commit(&bars.bfree[x]);
                         }
@@ -1312,7 +1316,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             tma_prefetch_desc(&tm_o);
             int j = 0;
             for (int x = sched.first; x < sched.end; x += sched.stride, ++j) {
-                const ReadItem it = read_item<G>(sched.item(x), n_ct, T, L, n_seg, has_init);
+                const ReadItem it = read_item<GI>(sched.item(x), n_ct, T, L, n_seg, has_init);
                 const int qb = j & 1;
                 if (!mbar_wait(&bars.ostaged[qb], (j >> 1) & 1, abort)) break;
                 for (int t = 0; t < kTiles; ++t)
@@ -1342,7 +1346,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
         int n_inter = 0, ns = 0, g_kv = 0, j = 0;  // ns: the CTA's intra step count
         bool ok = true;
         for (int x = sched.first; x < sched.end && ok; x += sched.stride, ++j) {
-            const ReadItem it = read_item<G>(sched.item(x), n_ct, T, L, n_seg, has_init);
+            const ReadItem it = read_item<GI>(sched.item(x), n_ct, T, L, n_seg, has_init);
             const int qb = j & 1;
             if (lane == 0) mbar_arrive(&bars.genin);
             ok = __all_sync(0xffffffffu, mbar_wait(&bars.qfull[qb], (j >> 1) & 1, abort));
@@ -1385,7 +1389,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                 ++n_inter;
             }
             float l = 0.f;
-            const int nb0 = read_tile_blocks<G>(it, 0, T), nb1 = read_tile_blocks<G>(it, 1, T);
+            const int nb0 = read_tile_blocks<GI>(it, 0, T), nb1 = read_tile_blocks<GI>(it, 1, T);
             const int n_b = t == 0 ? nb0 : nb1;
             for (int b = 0; b < n_b && ok; ++b) {
                 const int n = ns + step_before(b, t, nb0, nb1), x = n % kSBufs;
@@ -1394,15 +1398,15 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                 if (!ok) break;
                 // the block's last scores have landed: its keys are read
                 if (qd == 0 && lane == 0 && (t == 1 || b >= nb1))
-                    mbar_arrive(&bars.kempty[(g_kv + b) % kv_ring(G)]);
+                    mbar_arrive(&bars.kempty[(g_kv + b) % kv_ring(GI)]);
                 tc_fence_after();
-                const int kbs = it.seg0 + step_keys(G) * b;
+                const int kbs = it.seg0 + step_keys(GI) * b;
                 // every key of the block precedes every query of the tile
-                const bool full = kbs + step_keys(G) - 1 <= tq0;
+                const bool full = kbs + step_keys(GI) - 1 <= tq0;
                 const int lim = tq - kbs;  // otherwise keys kbs + c with c <= lim are visible
                 // weights w (packed fp32 pairs), four partial row sums
                 uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-                if constexpr (G == 1) {
+                if constexpr (GI == 1) {
                     // w = s^2, 64 keys at a time; each half's weights (bf16 pairs, 32
                     // columns) go over the scores of keys 0-63, already read
 #pragma unroll
@@ -1468,7 +1472,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     // the block's values have landed (issuer 1, which reads them, learns
                     // it from pfull: a wait of its own would stall behind its MMAs)
                     const int kvb = g_kv + b;
-                    ok = mbar_wait(&bars.vfull[kvb % kv_ring(G)], (kvb / kv_ring(G)) & 1, abort);
+                    ok = mbar_wait(&bars.vfull[kvb % kv_ring(GI)], (kvb / kv_ring(GI)) & 1, abort);
                     if (ok) mbar_arrive(&bars.pfull[x]);  // the step's weights are in place
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -1518,7 +1522,7 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
     if (tid == 0 && abort_flag) set_timeout_status(status);
 }
 
-template <int G>
+template <int G, int GI>
 bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const void *prefix, void *out,
                CUtensorMap *mq, CUtensorMap *mk, CUtensorMap *mv, CUtensorMap *ms, CUtensorMap *mo) {
     // inner extent d (the boxes stay 64 wide: columns past d read as zeros, and
@@ -1529,7 +1533,7 @@ bool make_maps(const Plan &p, const void *q, const void *k, const void *v, const
     const uint64_t ds[3] = {(uint64_t)kD, (uint64_t)bf16_rows(G), (uint64_t)(p.BH * p.n_seg)};
     const uint64_t ss[2] = {(uint64_t)kD * 2, (uint64_t)bf16_rows(G) * kD * 2};
     const uint32_t bs[3] = {64, 32, 1};
-    const uint32_t bkv[3] = {64, (uint32_t)step_keys(G), 1};
+    const uint32_t bkv[3] = {64, (uint32_t)step_keys(GI), 1};
     return make_tmap_bf16(mq, q, 3, dqkv, sqkv, bqkv) && make_tmap_bf16(mk, k, 3, dqkv, sqkv, bkv) &&
            make_tmap_bf16(mv, v, 3, dqkv, sqkv, bkv) &&
            make_tmap_bf16(ms, prefix ? prefix : q, 3, ds, ss, bs) && make_tmap_bf16(mo, out, 3, dqkv, sqkv, bqkv);
@@ -1543,6 +1547,24 @@ cudaError_t launch_expand_m2(const float *src, long long stride, float *state_ou
     const unsigned grid = (unsigned)((n + 255) / 256);
     ProfScope ps("tc_state_expand_m2", st);
     tc_state_expand<2, kD><<<grid, 256, 0, st>>>(src, stride, state_out, z_out, BH);
+    return cudaSuccess;
+}
+
+// The readout of a forward on the G-factor layout with GI-factor weights.
+template <int G, int GI>
+cudaError_t launch_read(const Plan &p, const void *q, const void *k, const void *v, const void *prefix,
+                        void *out, bool has_init, int *status, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, ms, mo;
+    if (!make_maps<G, GI>(p, q, k, v, prefix, out, &mq, &mk, &mv, &ms, &mo)) return cudaErrorInvalidValue;
+    cudaError_t e = smem_opt_in_once<tc_read<G, GI>>(kSmAlloc);
+    if (e != cudaSuccess) return e;
+    const int n_ct = (p.T + kCtaQ - 1) / kCtaQ;
+    const long long n_items = (long long)n_ct * p.BH;
+    if (n_items >= 0x7fffffffLL - 4096) return cudaErrorInvalidValue;
+    const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
+    ProfScope ps(GI == 1 ? "tc_read" : "tc_read_m2", st);
+    tc_read<G, GI><<<(unsigned)grid, kReadThreads, kSmAlloc, st>>>(mq, mk, mv, ms, mo, p.T, p.L, p.n_seg,
+                                                                   n_ct, (int)n_items, has_init, status);
     return cudaSuccess;
 }
 
@@ -1623,17 +1645,11 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
         }
     }
     if (readout) {
-        CUtensorMap mq, mk, mv, ms, mo;
-        if (!make_maps<G>(p, q, k, v, prefix, out, &mq, &mk, &mv, &ms, &mo)) return cudaErrorInvalidValue;
-        cudaError_t e = smem_opt_in_once<tc_read<G>>(kSmAlloc);
+        // a single-factor head on the two-factor layout (d <= 32): whole scores
+        const cudaError_t e = G == 2 && p.g == 1
+                                  ? launch_read<G, 1>(p, q, k, v, prefix, out, has_init, status, st)
+                                  : launch_read<G, G>(p, q, k, v, prefix, out, has_init, status, st);
         if (e != cudaSuccess) return e;
-        const int n_ct = (p.T + kCtaQ - 1) / kCtaQ;
-        const long long n_items = (long long)n_ct * BH;
-        if (n_items >= 0x7fffffffLL - 4096) return cudaErrorInvalidValue;
-        const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
-        ProfScope ps(G == 1 ? "tc_read" : "tc_read_m2", st);
-        tc_read<G><<<(unsigned)grid, kReadThreads, kSmAlloc, st>>>(
-            mq, mk, mv, ms, mo, p.T, p.L, p.n_seg, n_ct, (int)n_items, has_init, status);
     }
     if (want_state && !dense_from_scan) {
         const float *src = scan ? total : seg;

@@ -23,7 +23,8 @@ without waiting for its previous step's products, and both item slots'
 outputs staged on one barrier (a real hazard of an earlier version of the
 kernel, found by this model once each role ran at its own speed).  The same
 model runs the KATA-Mg two-factor configuration (9 inter stages, 64-key
-steps, rings of 6 key and 6 value blocks).
+steps, rings of 6 key and 6 value blocks) and the configuration of
+single-factor heads of d <= 32 (9 inter stages, 128-key steps).
 """
 import random
 
@@ -34,6 +35,9 @@ KERNEL = dict(kQT=128, kTiles=2, kKB=128, kKVRing=3, kRStages=17, kRRing=3, kRBR
 # KATA-Mg with two factors: 9 inter stages, and 64-key steps (both factors'
 # scores side by side in a buffer) in a ring of 4 key/value blocks
 KERNEL_M2 = dict(KERNEL, kRStages=9, kKB=64, kKVRing=6)
+# A single-factor head of d <= 32 on the two-factor layout: 9 inter stages,
+# the single factor's 128-key steps
+KERNEL_SMALL = dict(KERNEL, kRStages=9)
 
 
 class ProtocolError(AssertionError):
@@ -375,3 +379,16 @@ def test_two_factor_readout_protocol():
 def test_model_catches_a_two_factor_score_buffer_reused_before_its_products():
     with pytest.raises(ProtocolError):
         run_cases(KERNEL_M2, seeds=range(4), planted=True)
+
+
+def test_small_head_readout_protocol():
+    # single-factor heads of d <= 32: the two-factor layout's 9 inter stages
+    # with the single factor's 128-key intra steps
+    run_cases(KERNEL_SMALL, seeds=range(2))
+    cq = KERNEL_SMALL['kQT'] * KERNEL_SMALL['kTiles']
+    for T, L, BH, grid in CASES[:4]:
+        n_items = (T + cq - 1) // cq * BH
+        g = min(grid, n_items)
+        for c in range(g):
+            simulate(T, L, BH, list(range(c * n_items // g, (c + 1) * n_items // g)), 19 * T + c,
+                     KERNEL_SMALL, init=True)
