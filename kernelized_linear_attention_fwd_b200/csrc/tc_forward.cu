@@ -1045,7 +1045,7 @@ __global__ void __launch_bounds__(kReadThreads, 1)
 tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_s,
         const __grid_constant__ CUtensorMap tm_o, int T, int L, int n_seg, int n_ct, int n_items,
-        bool has_init, int *status) {
+        bool has_init, int qk_ks, int *status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ ReadBars bars;
     __shared__ uint32_t tmem_base;
@@ -1272,9 +1272,12 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                             const uint64_t dk = desc_add(dK, kv_bytes(GI) * kvs);
                             const uint64_t dQt = desc_sw128(slot + t * 16384, 16, 1024);
                             if constexpr (GI == 1) {
+                                // K-steps of the head's own coordinates only (qk_ks = d / 16:
+                                // the columns past d are zeros)
 #pragma unroll
                                 for (int ks = 0; ks < 4; ++ks)
-                                    mma_ss(buf, desc_add(dQt, 32 * ks), desc_add(dk, 32 * ks), id_qk, ks > 0);
+                                    if (ks < qk_ks)
+                                        mma_ss(buf, desc_add(dQt, 32 * ks), desc_add(dk, 32 * ks), id_qk, ks > 0);
                             } else {
                                 // one score per factor: coordinates 0-31 (K-steps 0, 1) into
                                 // columns 0-63 of the buffer, 32-63 (K-steps 2, 3) into 64-127
@@ -1562,9 +1565,11 @@ cudaError_t launch_read(const Plan &p, const void *q, const void *k, const void 
     const long long n_items = (long long)n_ct * p.BH;
     if (n_items >= 0x7fffffffLL - 4096) return cudaErrorInvalidValue;
     const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
+    // score K-steps: one per 16 coordinates of the head (two factors: all four)
+    const int qk_ks = GI == 1 ? (p.dk + 15) / 16 : 4;
     ProfScope ps(GI == 1 ? "tc_read" : "tc_read_m2", st);
     tc_read<G, GI><<<(unsigned)grid, kReadThreads, kSmAlloc, st>>>(mq, mk, mv, ms, mo, p.T, p.L, p.n_seg,
-                                                                   n_ct, (int)n_items, has_init, status);
+                                                                   n_ct, (int)n_items, has_init, qk_ks, status);
     return cudaSuccess;
 }
 

@@ -28,7 +28,8 @@ import kernelized_linear_attention_fwd_b200 as K  # noqa: E402
 from kernelized_linear_attention_fwd_b200.csrc import build as kbuild  # noqa: E402
 
 RECIPES = ("raw", "spread")
-# (dtype, d): the tensor-core path at d = 64 and below (heads read as 64), the CUDA-core path
+# (dtype, d): the tensor-core path at d = 64 and below (heads read as 64; d = 32 on the
+# two-factor state layout), the CUDA-core path
 PATHS = (("bf16", 64), ("bf16", 32), ("f32", 64), ("f32", 16))
 
 

@@ -48,7 +48,8 @@ def _noalloc_call(lib, q, k, v, out, C, so=None, zo=None):
 
 
 # bf16 d = 64, 32 and 16: the tensor-core route (heads below 64 read as 64
-# by the tensor maps); fp32: the CUDA-core route.
+# by the tensor maps, on the two-factor state layout); fp32: the CUDA-core
+# route.
 @pytest.mark.parametrize("dtype,d,T,H", [("bf16", 64, 3000, 2), ("bf16", 32, 2000, 2),
                                          ("bf16", 16, 2000, 2), ("f32", 32, 2100, 3)])
 def test_noalloc_matches_workspace_forward_twice(lib, dtype, d, T, H):
