@@ -32,8 +32,13 @@ namespace kata {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kUnroll = 4;
 constexpr int kMaxParts = 8;  // portable cluster size
+// State rows a thread has in flight: 4, or 8 when a single-factor head is
+// split over a full cluster (few heads, one or two CTAs per SM: the step is
+// then bound by the latency of each CTA's passes, not by the bytes in flight
+// per SM).
+template <int P, int G>
+constexpr int unroll_of() { return P == kMaxParts && G == 1 ? 8 : 4; }
 
 // Rows of the d^2-row state that one pass of the block covers.
 template <int DV>
@@ -65,9 +70,12 @@ __device__ __forceinline__ void packed_ij(int r, int &i, int &j) {
 }
 
 // CTAs per SM the register budget must allow (loads in flight per SM): 4 fit
-// the dense single-CTA kernel without spills, 3 the others.
+// the dense single-CTA kernel without spills, 3 the others, 2 the full-cluster
+// split with its deeper unroll.
 template <int P, bool PACKED, int G = 1>
-constexpr int min_ctas_per_sm() { return !PACKED && P == 1 && G == 1 ? 4 : 3; }
+constexpr int min_ctas_per_sm() {
+    return unroll_of<P, G>() == 8 ? 2 : !PACKED && P == 1 && G == 1 ? 4 : 3;
+}
 
 template <int DK, int DV, int P, bool PACKED, typename TIn, int G = 1>
 __global__ void __launch_bounds__(kThreads, min_ctas_per_sm<P, PACKED, G>())
@@ -78,7 +86,7 @@ decode_step_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const T
     constexpr int ROWS = state_rows<DK, PACKED>();
     constexpr int V4 = DV / 4;               // float4 slots per state row
     constexpr int RPI = kThreads / V4;       // rows covered per pass
-    constexpr int UNR = (ROWS / P / RPI) < kUnroll ? (ROWS / P / RPI) : kUnroll;
+    constexpr int UNR = (ROWS / P / RPI) < unroll_of<P, G>() ? (ROWS / P / RPI) : unroll_of<P, G>();
     static_assert(UNR >= 1, "every CTA covers at least one pass");
     __shared__ float sq[DK], sk[DK], sv[DV];
     __shared__ float red[RPI][DV + 1];
