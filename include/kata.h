@@ -196,6 +196,15 @@ kata_status kata_chunked_state(const void *k, const void *v, int B, int H, int T
  *              The result is the same either way; a workspace that does not
  *              hold those states gives wrong outputs, never a fault.  Other
  *              bits: KATA_ERR_INVALID_ARG.
+ *
+ * Accuracy (bf16): the term phi(q_t)^T S_0 is formed from bf16 products
+ * q_i q_j and a bf16 copy of the state, so its rounding error scales with
+ * sum_s (sum_i |q_t,i k_s,i|)^2 |v_s| over the history's tokens s, not with
+ * the term itself (the products' signs cancel).  After a long history the
+ * positive weights dominate; after a history of only a few tokens, a row
+ * whose small total weight comes mostly from history keys nearly orthogonal
+ * to its query can miss the bf16 tolerance of the plain forward.  fp32
+ * inputs have the same structure at fp32 rounding.
  */
 #define KATA_REUSE_SEGMENT_STATES 1u
 

@@ -1,4 +1,5 @@
-// KATA causal forward, tensor-core path (bf16 q, k, v, d = dv = 64, sm_100a).
+// KATA causal forward, tensor-core path (bf16 q, k, v, d = dv = 64, sm_100a;
+// heads of d = 16 and 32 read as 64, on the two-factor layout).
 //
 // Exact chunked-state form (gist.science summary of "Kernelized Linear
 // Attention: Breaking the Capacity Wall with Symmetric Cones", Technical
@@ -12,12 +13,13 @@
 //                    (the key tiles are transposed in shared memory on the way)
 //   tc_seg_scan      exclusive prefix over segments (associative scan) into a
 //                    bf16 copy for the readout, and the total: written as the
-//                    dense exported state (one factor) or kept packed in fp32
+//                    dense exported state (one factor, and heads of d <= 32)
+//                    or kept packed in fp32 (two factors of d = 64)
 //   tc_read          per 256 queries: phi(Q) S_prev and q^T Z_prev q on tcgen05
 //                    (phi(Q) generated from registers into tensor memory), the
 //                    intra-segment squared-score term on tcgen05, the division
-//   tc_state_expand  two factors: fp32 packed total -> dense [d*d, d] state and
-//                    [d, d] Z, zeros at the pairs across factors
+//   tc_state_expand  two factors of d = 64: fp32 packed total -> dense [d*d, d]
+//                    state and [d, d] Z, zeros at the pairs across factors
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -326,10 +328,11 @@ tc_seg_scan_short(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict
 // ---------------------------------------------------------------------------
 // fp32 total (packed rows) -> dense state [D*D][D] and Z [D][D], for G = 2
 // factors (KATA-Mg, D = 64), whose pairs across factors are not in the layout
-// and export 0 (one factor exports straight from the scan, every dense entry
-// being a pair of its layout).  D < 64 would export the leading D x D part of
-// heads computed as 64.  D is a template parameter so the index arithmetic
-// divides by constants.
+// and export 0 (one factor, and heads of d <= 32 on the two-factor layout,
+// export straight from the scan, every dense entry being a pair of the
+// layout).  D < 64 would export the leading D x D part of heads computed as
+// 64.  D is a template parameter so the index arithmetic divides by
+// constants.
 // ---------------------------------------------------------------------------
 // A thread writes 4 consecutive outputs (one 16-byte store: the outputs are
 // 16-byte aligned, and D, the packed row length and the per-head strides are
