@@ -119,6 +119,16 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// Programmatic dependent launch.  griddep_wait: wait until the grids this one
+// depends on have completed and their memory is visible (a no-op for a grid
+// launched without the programmatic attribute).  griddep_launch_dependents:
+// let the dependent grid start launching once every CTA of this one has
+// executed it (its CTAs still wait in griddep_wait for this grid to finish).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Tiled TMA store from shared memory (bulk-group completion).  Elements
 // outside the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, const void *smem_src, int c0, int c1,

@@ -208,6 +208,11 @@ tc_seg_scan(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict__ pre
             float *__restrict__ total, int n_seg, int n_valid, const float *__restrict__ init_s,
             const float *__restrict__ init_z, int n_in, long long s_stride, long long z_stride,
             int d, float *__restrict__ state_out, float *__restrict__ z_out) {
+    // launched after the builder, perhaps as its programmatic dependent: the
+    // readout may start launching now; the segment states are read after the
+    // builder has finished
+    griddep_launch_dependents();
+    griddep_wait();
     __shared__ float4 part[2][kScanWarps][32];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     constexpr long long E = f32_per_seg(G);
@@ -284,6 +289,8 @@ tc_seg_scan_short(const float *__restrict__ seg_state, __nv_bfloat16 *__restrict
                   const float *__restrict__ init_s, const float *__restrict__ init_z, int n_in,
                   long long s_stride, long long z_stride, int d, float *__restrict__ state_out,
                   float *__restrict__ z_out) {
+    griddep_launch_dependents();  // as tc_seg_scan
+    griddep_wait();
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     constexpr long long E = f32_per_seg(G);
     constexpr long long n_eb = E / 128;
@@ -867,6 +874,7 @@ tc_build(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUten
     tc_fence_after();
     const uint32_t tm = tmem_base;
     volatile int *abort = &abort_flag;
+    griddep_launch_dependents();  // the scan may start launching (it waits for this grid to finish)
 
     if (warp == kBTmaWarp) {
         // ------------------------------------------------------------ producer
@@ -1101,6 +1109,9 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
     tc_fence_after();
     const uint32_t tm = tmem_base;
     volatile int *abort = &abort_flag;
+    // perhaps launched as the scan's programmatic dependent: the prefixes are
+    // read only once the scan has finished
+    griddep_wait();
 
     if (warp == kTmaWarp) {
         // ------------------------------------------------------------ producer
@@ -1556,10 +1567,30 @@ cudaError_t launch_expand_m2(const float *src, long long stride, float *state_ou
     return cudaSuccess;
 }
 
+// Launches `kern` on `st`, as the programmatic dependent of the stream's
+// previous kernel when `pdl`: its CTAs may then start (and run their
+// prologue) while that kernel finishes, and wait in griddep_wait before they
+// read what it wrote.
+template <typename... Exp, typename... Act>
+cudaError_t launch_k(bool pdl, void (*kern)(Exp...), unsigned grid, unsigned block, size_t smem,
+                     cudaStream_t st, Act &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Act &&>(args)...);
+}
+
 // The readout of a forward on the G-factor layout with GI-factor weights.
 template <int G, int GI>
 cudaError_t launch_read(const Plan &p, const void *q, const void *k, const void *v, const void *prefix,
-                        void *out, bool has_init, int *status, cudaStream_t st) {
+                        void *out, bool has_init, int *status, cudaStream_t st, bool pdl) {
     CUtensorMap mq, mk, mv, ms, mo;
     if (!make_maps<G, GI>(p, q, k, v, prefix, out, &mq, &mk, &mv, &ms, &mo)) return cudaErrorInvalidValue;
     cudaError_t e = smem_opt_in_once<tc_read<G, GI>>(kSmAlloc);
@@ -1571,9 +1602,8 @@ cudaError_t launch_read(const Plan &p, const void *q, const void *k, const void 
     // score K-steps: one per 16 coordinates of the head (two factors: all four)
     const int qk_ks = GI == 1 ? (p.dk + 15) / 16 : 4;
     ProfScope ps(GI == 1 ? "tc_read" : "tc_read_m2", st);
-    tc_read<G, GI><<<(unsigned)grid, kReadThreads, kSmAlloc, st>>>(mq, mk, mv, ms, mo, p.T, p.L, p.n_seg,
-                                                                   n_ct, (int)n_items, has_init, qk_ks, status);
-    return cudaSuccess;
+    return launch_k(pdl, tc_read<G, GI>, (unsigned)grid, kReadThreads, kSmAlloc, st, mq, mk, mv, ms, mo, p.T,
+                    p.L, p.n_seg, n_ct, (int)n_items, has_init, qk_ks, status);
 }
 
 // The forward with G factors (1: KATA-M1; 2: KATA-Mg with two factors).
@@ -1608,6 +1638,13 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
     if (!status) return cudaErrorUnknown;
     if ((has_init || n_build > 0 || want_state || reuse_seg) && !w) return cudaErrorInvalidValue;
     if (want_state && (d_out < 1 || d_out > kD)) return cudaErrorInvalidValue;
+    // Small problems (the builder's and the readout's work items at most one
+    // per SM) chain their kernels as programmatic dependents, so that a
+    // kernel's launch and prologue overlap its predecessor's tail; larger ones
+    // launch plainly (early dependents would take SMs from the previous
+    // kernel's last waves).
+    const long long read_items = (long long)((p.T + kCtaQ - 1) / kCtaQ) * BH;
+    const bool small = (long long)build_items(G) * n_build * BH <= num_sms() && read_items <= num_sms();
 
     if (n_build > 0) {
         CUtensorMap mkb, mvb, mst;
@@ -1639,24 +1676,27 @@ cudaError_t launch_tc_forward_g(const Plan &p, const void *q, const void *k, con
             const long long grid = ((f32_per_seg(G) / 128) * BH + kScanWarps - 1) / kScanWarps;
             auto kern = p.n_seg <= 4 ? tc_seg_scan_short<G, 4>
                         : p.n_seg <= 8 ? tc_seg_scan_short<G, 8> : tc_seg_scan_short<G, 16>;
-            kern<<<(unsigned)grid, 256, 0, st>>>(seg, pre, tot, p.n_seg, n_valid, BH, init.s, init.z,
-                                                 init.n, init.s_stride, init.z_stride, d_out, s_out,
-                                                 z_dense);
+            const cudaError_t e = launch_k(small && n_build > 0, kern, (unsigned)grid, 256u, 0, st, seg, pre,
+                                           tot, p.n_seg, n_valid, BH, init.s, init.z, init.n, init.s_stride,
+                                           init.z_stride, d_out, s_out, z_dense);
+            if (e != cudaSuccess) return e;
         } else {
             const long long grid = (f32_per_seg(G) / 128) * BH;
             auto kern = p.n_seg <= 4 * kScanWarps ? tc_seg_scan<G, 4>
                         : p.n_seg <= 8 * kScanWarps ? tc_seg_scan<G, 8>
                                                     : tc_seg_scan<G, 16>;
-            kern<<<(unsigned)grid, 256, 0, st>>>(seg, pre, tot, p.n_seg, n_valid, init.s, init.z,
-                                                 init.n, init.s_stride, init.z_stride, d_out, s_out,
-                                                 z_dense);
+            const cudaError_t e = launch_k(small && n_build > 0, kern, (unsigned)grid, 256u, 0, st, seg, pre,
+                                           tot, p.n_seg, n_valid, init.s, init.z, init.n, init.s_stride,
+                                           init.z_stride, d_out, s_out, z_dense);
+            if (e != cudaSuccess) return e;
         }
     }
     if (readout) {
         // a single-factor head on the two-factor layout (d <= 32): whole scores
+        const bool pdl = small && scan;  // the dependent of this call's scan
         const cudaError_t e = G == 2 && p.g == 1
-                                  ? launch_read<G, 1>(p, q, k, v, prefix, out, has_init, status, st)
-                                  : launch_read<G, G>(p, q, k, v, prefix, out, has_init, status, st);
+                                  ? launch_read<G, 1>(p, q, k, v, prefix, out, has_init, status, st, pdl)
+                                  : launch_read<G, G>(p, q, k, v, prefix, out, has_init, status, st, pdl);
         if (e != cudaSuccess) return e;
     }
     if (want_state && !dense_from_scan) {
