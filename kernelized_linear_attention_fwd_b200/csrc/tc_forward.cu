@@ -1109,9 +1109,6 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
     tc_fence_after();
     const uint32_t tm = tmem_base;
     volatile int *abort = &abort_flag;
-    // perhaps launched as the scan's programmatic dependent: the prefixes are
-    // read only once the scan has finished
-    griddep_wait();
 
     if (warp == kTmaWarp) {
         // ------------------------------------------------------------ producer
@@ -1121,9 +1118,19 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_s);
             int n_q = 0, n_bs = 0, n_kv = 0, n_v = 0;  // loads issued into each ring (n_kv: keys)
-            bool ok = true;
+            bool ok = true, scanned = false;
             for (int x = sched.first; x < sched.end && ok; x += sched.stride) {
                 const ReadItem it = read_item<GI>(sched.item(x), n_ct, T, L, n_seg, has_init);
+                // Launched as the scan's programmatic dependent (small problems),
+                // this kernel may run while the scan does: the prefixes (the one
+                // input the scan writes) are loaded only after griddepcontrol.wait,
+                // while queries, keys and values, and the items without an inter
+                // phase, go ahead.  Other threads read no global memory before
+                // this thread's loads land.
+                if (it.inter && !scanned) {
+                    griddep_wait();
+                    scanned = true;
+                }
                 {
                     const int qb = n_q & 1;
                     uint8_t *slot = sm + kSmItem + qb * kItemBytes;
@@ -1166,6 +1173,9 @@ tc_read(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtens
                     ++n_v;
                 }
             }
+            // no CTA finishes before the scan (a CTA whose items have no inter
+            // phase waits here)
+            if (!scanned) griddep_wait();
             // every load issued must have landed before the CTA exits
             for (int x = (n_q > 2 ? n_q - 2 : 0); x < n_q; ++x)
                 mbar_wait_issued(&bars.qfull[x & 1], (x >> 1) & 1);
