@@ -50,6 +50,14 @@
  *     KATA_ERR_UNSUPPORTED.  T >= 1 (any value; the ragged tail is exact).
  *   - Calls on different streams may run concurrently if their buffers are
  *     disjoint.
+ *   - A call's kernels run after the work queued on `stream` before it and
+ *     end before the work queued after it starts.  On small problems (each
+ *     kernel at most one work item per SM) the chunked forwards start their
+ *     scan and readout as programmatic dependents of the call's previous
+ *     kernel (CUDA programmatic dependent launch): they may begin while it
+ *     finishes, but read nothing it writes until it has finished, and the
+ *     call's last kernel ends after all of them.  Captured into a CUDA graph,
+ *     those launches become programmatic edges.
  */
 #ifndef KATA_H_
 #define KATA_H_
