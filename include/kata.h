@@ -52,8 +52,9 @@
  *     disjoint.
  *   - A call's kernels run after the work queued on `stream` before it and
  *     end before the work queued after it starts.  On small problems (each
- *     kernel at most one work item per SM) the chunked forwards start their
- *     scan and readout as programmatic dependents of the call's previous
+ *     kernel at most one work item per SM) the chunked calls (the forwards,
+ *     the state-only call) start their scan, and the forwards their readout,
+ *     as programmatic dependents of the call's previous
  *     kernel (CUDA programmatic dependent launch): they may begin while it
  *     finishes, but read nothing it writes until it has finished, and the
  *     call's last kernel ends after all of them.  Captured into a CUDA graph,
